@@ -1,0 +1,284 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+None of these retypes the oracle's own formula: each compares it with a closed
+form, an invariant, a different algorithm (Sinkhorn-Knopp scaling on an explicit
+kernel matrix, Cuturi 2013, listed among the FS2 page's references), or a
+numerical derivative. A plausible slip in ``oracle.c`` -- a dropped log-weight
+term, a sign, a swapped operand, an off-by-one in the schedule -- fails one of them.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from streaming_sinkhorn_b200 import workloads
+
+
+def dense_cost(x, y):
+    x = np.asarray(x, np.float64)
+    y = np.asarray(y, np.float64)
+    return ((x[:, None, :] - y[None, :, :]) ** 2).sum(-1)
+
+
+def scaling_sinkhorn(x, y, a, b, eps, n_iters, g0=None):
+    """Sinkhorn-Knopp on the explicit Gibbs kernel K = exp(-C/eps).
+
+    u = a / (K v), v = b / (K^T u), v0 = b exp(g0/eps). Returns the potentials in the
+    log-domain convention: f = -eps log(K v), g = -eps log(K^T u).
+    """
+    C = dense_cost(x, y)
+    K = np.exp(-C / eps)
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    v = b.copy() if g0 is None else b * np.exp(np.asarray(g0, np.float64) / eps)
+    for _ in range(n_iters):
+        Kv = K @ v
+        u = a / Kv
+        Ktu = K.T @ u
+        v = b / Ktu
+    return -eps * np.log(Kv), -eps * np.log(Ktu)
+
+
+def dense_plan(x, y, a, b, eps, f, g):
+    C = dense_cost(x, y)
+    return (np.asarray(a, np.float64)[:, None] * np.asarray(b, np.float64)[None, :]
+            * np.exp((np.asarray(f)[:, None] + np.asarray(g)[None, :] - C) / eps))
+
+
+def small(n, m, d, seed, eps=0.5, zero_frac=0.0, mass=1.0):
+    w = workloads.random_small(n, m, d, seed, eps=eps, zero_frac=zero_frac, mass=mass)
+    a = w.a.astype(np.float64)
+    b = w.b.astype(np.float64)
+    b *= a.sum() / b.sum()  # balance the masses exactly in float64
+    return w.x.astype(np.float64), w.y.astype(np.float64), a, b, w.eps
+
+
+# --- N = M = 1 -----------------------------------------------------------------------
+
+@pytest.mark.parametrize("w", [1.0, 0.25, 3.0])
+def test_single_pair_closed_form(w):
+    """One point each, weights w: after one iteration f = C - eps log w, g = 0,
+    so f + g = C - eps log w (= C for unit weights) and further iterations keep it."""
+    x = np.array([[0.3, -1.2, 2.0]])
+    y = np.array([[1.1, 0.4, -0.5]])
+    C = float(((x - y) ** 2).sum())
+    eps = 0.7
+    a = np.array([w])
+    b = np.array([w])
+    for iters in (1, 2, 5):
+        f, g = oracle.potentials(x, y, a, b, eps, iters)
+        assert f[0] == pytest.approx(C - eps * np.log(w), rel=1e-14, abs=1e-14)
+        assert g[0] == pytest.approx(0.0, abs=1e-13)
+        assert f[0] + g[0] == pytest.approx(C - eps * np.log(w), rel=1e-14, abs=1e-14)
+
+
+# --- brute-force scaling Sinkhorn ---------------------------------------------------------
+
+@pytest.mark.parametrize("n,m,d,seed,zero_frac", [(7, 5, 2, 0, 0.0), (31, 40, 3, 1, 0.2),
+                                                  (64, 33, 5, 2, 0.1), (1, 9, 2, 3, 0.0)])
+@pytest.mark.parametrize("iters", [1, 2, 7])
+def test_matches_scaling_sinkhorn(n, m, d, seed, zero_frac, iters):
+    x, y, a, b, _ = small(n, m, d, seed, zero_frac=zero_frac)
+    C = dense_cost(x, y)
+    eps = float(C.max()) / 30.0  # keeps C/eps < 700 so exp(-C/eps) is finite
+    f, g = oracle.potentials(x, y, a, b, eps, iters)
+    fs, gs = scaling_sinkhorn(x, y, a, b, eps, iters)
+    np.testing.assert_allclose(f, fs, rtol=1e-11, atol=1e-12 * C.max())
+    np.testing.assert_allclose(g, gs, rtol=1e-11, atol=1e-12 * C.max())
+
+
+def test_matches_scaling_with_warm_start():
+    x, y, a, b, _ = small(20, 13, 3, 5)
+    eps = float(dense_cost(x, y).max()) / 20.0
+    g0 = np.random.default_rng(9).standard_normal(13) * 0.3
+    f, g = oracle.potentials(x, y, a, b, eps, 4, g_init=g0)
+    fs, gs = scaling_sinkhorn(x, y, a, b, eps, 4, g0=g0)
+    np.testing.assert_allclose(f, fs, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(g, gs, rtol=1e-11, atol=1e-12)
+
+
+def test_row_subset_equals_full_update():
+    x, y, a, b, eps = small(50, 37, 3, 6)
+    g = np.random.default_rng(1).standard_normal(37)
+    full = oracle.lse_update(x, y, b, g, eps)
+    rows = np.array([49, 0, 17, 17, 3])
+    np.testing.assert_array_equal(oracle.lse_update(x, y, b, g, eps, rows=rows), full[rows])
+
+
+# --- gauge invariance ---------------------------------------------------------------------
+
+@pytest.mark.parametrize("c", [0.37, -2.5])
+def test_gauge_shift(c):
+    """Starting from g0 - c gives (f + c, g - c) at every iterate and the same cost."""
+    x, y, a, b, eps = small(25, 18, 2, 7)
+    f0, g0 = oracle.potentials(x, y, a, b, eps, 3)
+    f1, g1 = oracle.potentials(x, y, a, b, eps, 3, g_init=np.full(18, -c))
+    np.testing.assert_allclose(f1, f0 + c, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(g1, g0 - c, rtol=0, atol=1e-12)
+    assert oracle.cost(x, y, a, b, eps, f1, g1) == pytest.approx(
+        oracle.cost(x, y, a, b, eps, f0, g0), rel=1e-12, abs=1e-12)
+
+
+# --- marginals ----------------------------------------------------------------------------
+
+def test_marginals_after_each_update():
+    """Right after an f-update P 1 = a; right after a g-update P^T 1 = b (to rounding)."""
+    x, y, a, b, eps = small(30, 22, 3, 8, zero_frac=0.2)
+    f, g = oracle.potentials(x, y, a, b, eps, 2)
+    r = oracle.plan_row_sums(x, y, a, b, eps, f, g)
+    c = oracle.plan_col_sums(x, y, a, b, eps, f, g)
+    np.testing.assert_allclose(c, b, rtol=1e-12, atol=1e-15)
+    assert np.abs(r - a).max() > 1e-6  # not converged after 2 iterations
+    f2 = oracle.lse_update(x, y, b, g, eps)  # fresh f-update
+    np.testing.assert_allclose(oracle.plan_row_sums(x, y, a, b, eps, f2, g), a, rtol=1e-12,
+                               atol=1e-15)
+
+
+def test_marginals_at_convergence():
+    x, y, a, b, _ = small(16, 12, 2, 9)
+    eps = 1.0
+    f, g = oracle.potentials(x, y, a, b, eps, 400)
+    res = oracle.marginal_residual(x, y, a, b, eps, f, g)
+    assert res[1] < 1e-13 and res[3] < 1e-13
+    assert res[0] < 1e-12 and res[2] < 1e-12
+
+
+def test_residual_matches_dense_plan():
+    x, y, a, b, eps = small(19, 27, 3, 10, zero_frac=0.15)
+    f, g = oracle.potentials(x, y, a, b, eps, 3)
+    f = f + 0.01 * np.sin(np.arange(19))  # arbitrary (f, g), not an iterate
+    P = dense_plan(x, y, a, b, eps, f, g)
+    np.testing.assert_allclose(oracle.plan_row_sums(x, y, a, b, eps, f, g), P.sum(1), rtol=1e-13)
+    np.testing.assert_allclose(oracle.plan_col_sums(x, y, a, b, eps, f, g), P.sum(0), rtol=1e-13)
+    res = oracle.marginal_residual(x, y, a, b, eps, f, g)
+    dr, dc = np.abs(P.sum(1) - a), np.abs(P.sum(0) - b)
+    np.testing.assert_allclose(res, [dr.sum(), dr.max(), dc.sum(), dc.max()], rtol=1e-12)
+
+
+# --- cost -----------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mass", [1.0, 2.5, 0.3])
+def test_cost_dual_objective(mass):
+    """The explicit double sum equals the dense-plan dual objective, and right after a
+    g-update (P^T 1 = b) it reduces to <f,a> + <g,b> - eps*m*(1 - m)."""
+    x, y, a, b, eps = small(21, 14, 2, 11, mass=mass)
+    f, g = oracle.potentials(x, y, a, b, eps, 3)
+    P = dense_plan(x, y, a, b, eps, f, g)
+    dense = f @ a + g @ b - eps * (P.sum() - a.sum() * b.sum())
+    got = oracle.cost(x, y, a, b, eps, f, g)
+    assert got == pytest.approx(dense, rel=1e-12, abs=1e-14)
+    m = b.sum()
+    assert got == pytest.approx(f @ a + g @ b - eps * m * (1.0 - m), rel=1e-10, abs=1e-12)
+
+
+def test_large_eps_product_limit():
+    """eps -> infinity: P -> a (x) b, so the cost tends to <C, a (x) b> (closed form in
+    O(N + M)) with an error that shrinks like 1/eps, and the gradient tends to
+    2 a_i (x_i - sum_j b_j y_j)."""
+    x, y, a, b, _ = small(17, 23, 3, 12)
+    a /= a.sum()  # unit mass exactly, so the -eps*m*(1-m) term vanishes
+    b /= b.sum()
+    C = dense_cost(x, y)
+    closed = (a @ (x ** 2).sum(1)) + (b @ (y ** 2).sum(1)) - 2.0 * (a @ x) @ (b @ y)
+    assert closed == pytest.approx(a @ C @ b, rel=1e-12)
+    errs = []
+    for scale in (1e3, 1e4):
+        eps = scale * C.max()
+        f, g = oracle.potentials(x, y, a, b, eps, 5)
+        errs.append(abs(oracle.cost(x, y, a, b, eps, f, g) - closed))
+        gr = oracle.grad_x(x, y, a, b, eps, g)
+        lim = 2.0 * a[:, None] * (x - (b @ y)[None, :])
+        np.testing.assert_allclose(gr, lim, rtol=0, atol=50.0 / scale * np.abs(lim).max())
+    assert errs[0] < 1e-2 * C.max()
+    assert errs[1] < errs[0] / 5.0  # O(1/eps)
+
+
+# --- gradient -------------------------------------------------------------------------------
+
+def test_grad_matches_dense_plan():
+    x, y, a, b, eps = small(23, 31, 3, 13, zero_frac=0.1)
+    f, g = oracle.potentials(x, y, a, b, eps, 4)
+    C = dense_cost(x, y)
+    ft = -eps * np.log(np.exp(-C / eps) @ (b * np.exp(g / eps)))
+    P = dense_plan(x, y, a, b, eps, ft, g)
+    ref = 2.0 * (a[:, None] * x - P @ y)
+    got = oracle.grad_x(x, y, a, b, eps, g)
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-13)
+    rows = np.array([5, 0, 22])
+    np.testing.assert_array_equal(oracle.grad_x(x, y, a, b, eps, g, rows=rows), got[rows])
+
+
+def test_grad_central_finite_difference():
+    """At convergence the envelope gradient is the derivative of the solved cost.
+
+    float64, 6 random directions per point, central differences; each perturbed cost
+    is re-solved to convergence (SinkSLOT README, "dropped-term finite difference").
+    """
+    x, y, a, b, _ = small(10, 9, 2, 14)
+    eps = 0.8
+    iters = 600
+
+    def solved_cost(xx):
+        f, g = oracle.potentials(xx, y, a, b, eps, iters)
+        return oracle.cost(xx, y, a, b, eps, f, g), f, g
+
+    _, f, g = solved_cost(x)
+    assert oracle.marginal_residual(x, y, a, b, eps, f, g)[1] < 1e-14
+    grad = oracle.grad_x(x, y, a, b, eps, g)
+    rng = np.random.default_rng(0)
+    h = 1e-5
+    worst = 0.0
+    for i in range(x.shape[0]):
+        for _ in range(6):
+            v = rng.standard_normal(x.shape[1])
+            v /= np.linalg.norm(v)
+            xp = x.copy()
+            xm = x.copy()
+            xp[i] += h * v
+            xm[i] -= h * v
+            fd = (solved_cost(xp)[0] - solved_cost(xm)[0]) / (2 * h)
+            worst = max(worst, abs(fd - grad[i] @ v))
+    assert worst < 1e-8 * max(1.0, np.abs(grad).max() * 100)
+
+
+def test_grad_fd_gap_shrinks_with_residual():
+    """Before convergence the envelope gradient misses a term that vanishes with the
+    marginal residual (SinkSLOT README, "gradient term split")."""
+    x, y, a, b, _ = small(8, 8, 2, 15)
+    eps = 0.5
+    v = np.zeros_like(x)
+    v[3] = [0.6, 0.8]
+    h = 1e-5
+    gaps = []
+    for iters in (16, 64, 128):
+        def c(xx):
+            f, g = oracle.potentials(xx, y, a, b, eps, iters)
+            return oracle.cost(xx, y, a, b, eps, f, g)
+        _, g = oracle.potentials(x, y, a, b, eps, iters)
+        fd = (c(x + h * v) - c(x - h * v)) / (2 * h)
+        gaps.append(abs(fd - (oracle.grad_x(x, y, a, b, eps, g) * v).sum()))
+    assert gaps[2] < gaps[1] < gaps[0]
+    assert gaps[2] < 1e-9
+
+
+# --- errors ---------------------------------------------------------------------------------
+
+def test_mass_mismatch_raises():
+    x, y, a, b, eps = small(5, 6, 2, 16)
+    with pytest.raises(oracle.OracleError) as e:
+        oracle.potentials(x, y, a, b * 1.001, eps, 2)
+    assert e.value.code == -2
+    oracle.potentials(x, y, a, b * (1 + 1e-7), eps, 2)  # inside the 1e-5 relative band
+
+
+def test_zero_mass_and_negative_weight_raise():
+    x, y, a, b, eps = small(5, 6, 2, 17)
+    with pytest.raises(oracle.OracleError):
+        oracle.potentials(x, y, np.zeros(5), np.zeros(6), eps, 1)
+    bad = a.copy()
+    bad[1] = -0.1
+    with pytest.raises(oracle.OracleError):
+        oracle.potentials(x, y, bad, b, eps, 1)
+    with pytest.raises(oracle.OracleError):
+        oracle.potentials(x, y, a, b, 0.0, 1)
+    with pytest.raises(oracle.OracleError):
+        oracle.potentials(x, y, a, b, eps, 0)
