@@ -1,0 +1,411 @@
+"""Throughput of the streaming log-domain Sinkhorn hot path on B200.
+
+One step = one full pass of the hot path over one synthetic problem: fs_potentials
+(the fixed-count alternating iterations), fs_grad_x, fs_marginal_residual and fs_cost,
+each called through the C ABI exactly as a user calls it. The metric is pair
+evaluations per second, N*M*iters / step time (each iteration runs two N*M passes).
+
+Default workload: the clustered unit-cube problem, N = M = 2^20, d = 3, 1000 Gaussians
+(std 0.01), eps = (N^(-1/3))^2 = 2^(-40/3), 20 iterations (the FlashSinkhorn 2 scale
+rule "blur = mean interparticle distance"), float32.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c5] [--impl reference]
+
+Under torchrun (N > 1) each rank solves its own independently seeded instance of the
+same workload (replicas; weak scaling); value = all ranks' pair evaluations / the
+slowest rank's time. `--impl reference` times the float64 CPU oracle on a bounded sample
+of the same workload on this host's cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "pair-evals/s (N·M·iters/s) log-domain Sinkhorn; % of ex2/FMA roofline"
+UNIT = "pair-evals/s"
+CONFIG_INDEX = {"c1": 0, "c2": 1, "c3": 2, "c4": 3, "c5": 4}
+# MUFU ex2 throughput per SM per clock on sm_100 (16 results/clk/SM, CUDA throughput table).
+EX2_PER_CLK_PER_SM = 16
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="c5", choices=sorted(CONFIG_INDEX))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU seconds of the oracle sample")
+    return ap.parse_args()
+
+
+def workload(cfg: str, rank: int):
+    from streaming_sinkhorn_b200 import workloads
+    import dataclasses
+    w = workloads.config(CONFIG_INDEX[cfg])
+    if rank:
+        # an independently seeded replica of the same recipe
+        base = {0: workloads.gaussian_shifted, 1: workloads.gaussian_pair}
+        idx = CONFIG_INDEX[cfg]
+        if idx == 4:
+            w = dataclasses.replace(workloads.clustered_cube(n=w.n, seed=w.seed + 1000 * rank,
+                                                             eps=w.eps, n_iters=w.n_iters),
+                                    name=w.name)
+        elif idx in base:
+            w = dataclasses.replace(base[idx](n=w.n, d=w.d, seed=w.seed + 1000 * rank, eps=w.eps,
+                                              n_iters=w.n_iters), name=w.name)
+    return w
+
+
+# ---------------------------------------------------------------- clocks ----------
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"fs_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------- roofline ---------
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "streaming_sinkhorn_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(cfg: str):
+    """Per-launch DRAM bytes of the LSE pass from a committed ncu summary, if it was
+    measured on the current kernel sources (profiles/lse_pass_traffic.txt)."""
+    path = os.path.join(ROOT, "profiles", "lse_pass_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    rec = {}
+    for line in open(path):
+        if "=" in line and not line.lstrip().startswith("#"):
+            k, v = line.split("=", 1)
+            rec[k.strip()] = v.strip()
+    if rec.get("kernel_source_digest") != kernel_source_digest() or rec.get("config") != cfg:
+        return None
+    try:
+        return float(rec["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        try:
+            return json.load(open(path))
+        except ValueError:
+            return {}
+    return {}
+
+
+# ---------------------------------------------------------------- oracle sample ----
+
+def oracle_sample(w, target_s: float):
+    """Times the float64 oracle's f-update over a sample of rows against all M columns.
+
+    Returns (pair-evals/s in the metric's unit, threads, description). One iteration is
+    two N*M passes, so pairs/s of one pass / 2 is N*M*iters/s.
+    """
+    import oracle
+    oracle.build()
+    g0 = np.zeros(w.m, dtype=np.float64)
+    rng = np.random.default_rng(0)
+    rows = rng.choice(w.n, size=min(w.n, 4), replace=False)
+    t0 = time.perf_counter()
+    oracle.lse_update(w.x, w.y, w.b, g0, w.eps, rows=rows)
+    per_row = (time.perf_counter() - t0) / len(rows)
+    k = int(max(1, min(w.n, target_s / max(per_row, 1e-9))))
+    rows = rng.choice(w.n, size=k, replace=False)
+    t0 = time.perf_counter()
+    oracle.lse_update(w.x, w.y, w.b, g0, w.eps, rows=rows)
+    dt = time.perf_counter() - t0
+    pairs = float(k) * w.m
+    value = pairs / dt / 2.0
+    desc = (f"float64 oracle f-update (two-pass LSE, direct-difference cost) over {k} sampled "
+            f"rows x all {w.m} columns of {w.name} ({pairs:.3e} pair evaluations, {dt:.1f} s); "
+            f"scaled to N*M*iters/s as pair-evals/s / 2")
+    return value, oracle.threads(), desc, dt
+
+
+# ---------------------------------------------------------------- native arm -------
+
+def run_native(args, rank, world, local_rank):
+    import torch
+    import streaming_sinkhorn_b200 as fs
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    w = workload(args.config, rank)
+    dev = torch.device("cuda", local_rank)
+    x = torch.from_numpy(w.x).to(dev)
+    y = torch.from_numpy(w.y).to(dev)
+    a = torch.from_numpy(w.a).to(dev)
+    b = torch.from_numpy(w.b).to(dev)
+    f = torch.empty(w.n, dtype=torch.float32, device=dev)
+    g = torch.empty(w.m, dtype=torch.float32, device=dev)
+    gx = torch.empty((w.n, w.d), dtype=torch.float32, device=dev)
+    ws = torch.empty(fs.workspace_bytes(w.n, w.m, w.d, dev), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fs.potentials(x, y, a, b, eps=w.eps, n_iters=w.n_iters, out=(f, g), workspace=ws)
+        fs.grad_x(x, y, g, a, b, eps=w.eps, out=gx, workspace=ws)
+        res = fs.marginal_residual(x, y, f, g, a, b, eps=w.eps, workspace=ws)
+        c = fs.cost(x, y, f, g, a, b, eps=w.eps, workspace=ws)
+        return res, c
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    fs.timing_enable(True)
+    fs.timing_reset()
+    launches0 = fs.launch_count()
+    barrier()
+    total_ms = 0.0
+    for _ in range(args.steps):
+        flush.zero_()  # L2 flush between timed steps, outside the step's events
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        res, c = step()
+        e1.record(stream)
+        e1.synchronize()
+        total_ms += e0.elapsed_time(e1)
+    barrier()
+    launches = fs.launch_count() - launches0
+    timing = fs.timing_get()
+    fs.timing_enable(False)
+    clk = clocks.stop()
+    ms_per_step = total_ms / args.steps
+    if dist is not None:
+        t = torch.tensor([ms_per_step], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_per_step = float(t.item())
+    pairs_per_step = float(w.n) * w.m * w.n_iters
+    value = pairs_per_step * world / (ms_per_step / 1e3)
+
+    # roofline of the dominant kernel: the potential-update pass
+    lse = timing["lse_pass"]
+    per_launch_ms = lse["total_ms"] / max(lse["launches"], 1)
+    per_launch_pairs = lse["pairs"] / max(lse["launches"], 1)
+    achieved = per_launch_pairs / (per_launch_ms / 1e3)  # ex2 / s
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    max_mhz = clk.get("sm_max_mhz") or measured_peaks().get("sm_max_mhz") or 1965.0
+    peak = sms * EX2_PER_CLK_PER_SM * max_mhz * 1e6
+    roofline = {"bound": "alu", "achieved": achieved / 1e12, "peak": peak / 1e12,
+                "unit": "Tex2/s", "frac": achieved / peak,
+                "traffic": recorded_traffic(args.config),
+                "kernel": "lse_pass_kernel (potential update)",
+                "peak_basis": f"{sms} SMs x {EX2_PER_CLK_PER_SM} ex2/clk x {max_mhz:.0f} MHz",
+                "frac_at_observed_clock": (achieved / (sms * EX2_PER_CLK_PER_SM * clk["sm_mhz"] * 1e6)
+                                           if clk.get("sm_mhz") else None),
+                "launches_timed": lse["launches"], "ms_per_launch": per_launch_ms}
+
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "n": w.n, "m": w.m, "d": w.d, "eps": w.eps,
+                   "iters": w.n_iters, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "step": "fs_potentials + fs_grad_x + fs_marginal_residual + fs_cost",
+                   "l2": "flushed between timed steps (256 MiB write); inputs 25 MB"},
+        "gpu_launches": int(launches),
+        "roofline": roofline,
+        "clocks": clk,
+        "kernel_timing": timing,
+        "check": {"residual": [float(v) for v in res.cpu().numpy()], "cost": float(c.item())},
+    }
+
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(args, w, dev, world, dist)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, desc, _ = oracle_sample(w, args.cpu_seconds)
+        result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                  "sample": desc}
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def run_e2e(args, w, dev, world, dist):
+    """Same metric through fs_solve_host: host inputs copied in and results copied out
+    inside every timed step."""
+    import torch
+    import streaming_sinkhorn_b200 as fs
+    pin = lambda v: torch.from_numpy(v).pin_memory()  # noqa: E731
+    xh, yh, ah, bh = pin(w.x), pin(w.y), pin(w.a), pin(w.b)
+    out = {"f": torch.empty(w.n, dtype=torch.float32).pin_memory(),
+           "g": torch.empty(w.m, dtype=torch.float32).pin_memory(),
+           "grad_x": torch.empty((w.n, w.d), dtype=torch.float32).pin_memory(),
+           "cost": torch.empty(1, dtype=torch.float64).pin_memory(),
+           "residual": torch.empty(4, dtype=torch.float64).pin_memory()}
+    import ctypes
+    from streaming_sinkhorn_b200 import _lib
+    p = _lib.fs_problem(xh.data_ptr(), yh.data_ptr(), ah.data_ptr(), bh.data_ptr(), w.n, w.m, w.d,
+                        w.eps)
+    nbytes = int(_lib.load().fs_solve_host_workspace_bytes(ctypes.byref(p)))
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    steps = args.e2e_steps if args.e2e_steps is not None else args.steps
+    fs.solve_host(xh, yh, ah, bh, eps=w.eps, n_iters=w.n_iters, device=dev, workspace=ws, out=out)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fs.solve_host(xh, yh, ah, bh, eps=w.eps, n_iters=w.n_iters, device=dev, workspace=ws, out=out)
+    e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = (w.n * w.d + w.m * w.d + w.n + w.m) * 4
+    d2h = (w.n + w.m + w.n * w.d) * 4 + 5 * 8
+    return {"value": float(w.n) * w.m * w.n_iters * world / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "steps": steps, "api": "fs_solve_host (pinned host buffers)"}
+
+
+# ---------------------------------------------------------------- reference arm ----
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = workload(args.config, 0)
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, min(per_step, 3.0))
+    vals, secs = [], 0.0
+    desc, cores = "", 1
+    for _ in range(args.steps):
+        v, cores, desc, dt = oracle_sample(w, per_step)
+        vals.append(v)
+        secs += dt
+    value = float(np.mean(vals))
+    pairs_per_step = float(w.n) * w.m * w.n_iters
+    ms_per_step = pairs_per_step / value * 1e3
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "n": w.n, "m": w.m, "d": w.d, "eps": w.eps,
+                   "iters": w.n_iters, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc + "; each step one such sample"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and "WORLD_SIZE" in os.environ:
+        world = int(os.environ["WORLD_SIZE"])
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1 and "RANK" not in os.environ:
+        raise SystemExit("--gpus N > 1 must be launched with torchrun (one process per GPU)")
+    from streaming_sinkhorn_b200 import build
+    if not os.path.exists(build.LIB):
+        build.build()
+    run_native(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+/*
+ * fs.h -- C ABI of the streaming log-domain Sinkhorn library (libfs.so, sm_100a).
+ *
+ * Entropic optimal transport between two weighted point clouds under the squared
+ * Euclidean ground cost C_ij = |x_i - y_j|^2 (SinkSLOT README, "Tensor Contract").
+ * The N x M cost or kernel matrix is never stored: every pass recomputes the cost
+ * tile by tile on chip and reduces it with an online log-sum-exp (FlashSinkhorn
+ * summary, Methodology sections 1-2: attention-form reformulation, online LSE,
+ * fusion, row-stationary traversal).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Array arguments are DEVICE pointers to contiguous float32 data, row-major for
+ *    the (n, d) and (m, d) clouds, unless an entry point says otherwise. The caller
+ *    owns every buffer; the library never allocates device memory. Scratch space is
+ *    passed in as `ws` (ws_bytes >= fs_workspace_bytes(problem), 256-byte aligned);
+ *    its contents need not be initialised and are not preserved between calls.
+ *  - Every call is ordered on `stream` (NULL = the legacy default stream) and is
+ *    blocking: it returns after its work has finished, having read back the input
+ *    validation and the kernels' error word. Outputs are complete on return.
+ *  - Weights a, b are used exactly as given, not normalised; NULL means uniform 1/n
+ *    (resp. 1/m). They must be finite and >= 0, zero entries are legal, and their
+ *    sums (accumulated in float64) must agree to 1e-5 relative and be positive
+ *    (SinkSLOT README, "Tensor Contract": sums must match, zero entries legal).
+ *  - n != m is allowed; 1 <= d <= FS_MAX_D; eps must be finite and > 0.
+ *  - Potentials are in cost units (f, g), not divided by eps.
+ *  - Errors are returned as fs_status; on error the outputs are unspecified and no
+ *    GPU state is left behind (the call has drained its own work on `stream`).
+ *
+ * Thread safety: calls may run concurrently from several host threads on different
+ * streams and workspaces. Kernel timing (fs_timing_*) is process-wide.
+ */
+#ifndef FS_H_
+#define FS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FS_API __attribute__((visibility("default")))
+#else
+#define FS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL selects the legacy default stream. */
+typedef struct CUstream_st* fs_stream_t;
+
+#define FS_MAX_D 64
+
+/* One OT problem. Pointer fields are device pointers (host pointers for fs_solve_host). */
+typedef struct {
+  const float* x; /* (n, d) source points */
+  const float* y; /* (m, d) target points */
+  const float* a; /* (n,) source weights, or NULL for uniform 1/n */
+  const float* b; /* (m,) target weights, or NULL for uniform 1/m */
+  int64_t n;      /* number of source points, >= 1 */
+  int64_t m;      /* number of target points, >= 1 */
+  int32_t d;      /* dimension, 1..FS_MAX_D */
+  float eps;      /* entropic regularisation, finite and > 0, in cost units */
+} fs_problem;
+
+typedef enum {
+  FS_OK = 0,
+  FS_ERR_NULL = 1,             /* a required pointer is NULL */
+  FS_ERR_SHAPE = 2,            /* n < 1, m < 1, d < 1, or sizes overflow */
+  FS_ERR_EPS = 3,              /* eps not finite or <= 0 */
+  FS_ERR_ITERS = 4,            /* n_iters < 1 */
+  FS_ERR_NEGATIVE_WEIGHT = 5,  /* a weight is negative or not finite */
+  FS_ERR_NONFINITE_INPUT = 6,  /* a coordinate (or a given potential) is not finite */
+  FS_ERR_MASS_MISMATCH = 7,    /* |sum a - sum b| > 1e-5 * max(sum a, sum b) */
+  FS_ERR_ZERO_MASS = 8,        /* sum a == 0 (so every weight is zero) */
+  FS_ERR_UNSUPPORTED_D = 9,    /* d > FS_MAX_D */
+  FS_ERR_WORKSPACE = 10,       /* ws NULL, misaligned or smaller than required */
+  FS_ERR_TIMEOUT = 11,         /* a kernel's bounded wait expired; outputs invalid */
+  FS_ERR_CUDA = 12,            /* a CUDA runtime call failed (see fs_last_cuda_error) */
+  FS_ERR_ALIGNMENT = 13        /* a device pointer is not 4-byte aligned */
+} fs_status;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+FS_API const char* fs_status_string(fs_status s);
+
+/* Text of the last CUDA error seen by this host thread inside the library, or "". */
+FS_API const char* fs_last_cuda_error(void);
+
+/*
+ * Bytes of scratch space every entry point below needs for `p` (pointer fields of
+ * `p` are not read). Returns 0 when the shape (n, m, d) is invalid. The size depends
+ * on the current device's SM count, so query it with the device current that the
+ * calls will use.
+ */
+FS_API size_t fs_workspace_bytes(const fs_problem* p);
+
+/*
+ * Fixed-count alternating Sinkhorn (SinkSLOT README, API Reference: variant
+ * "alternating", stop_mode "fixed"; FlashSinkhorn summary, section 1 for the update):
+ *   g <- g_init (or 0 when g_init is NULL)
+ *   repeat n_iters times:
+ *     f_i <- -eps * LSE_j[(g_j - C_ij)/eps + log b_j]       (one fused streaming pass)
+ *     g_j <- -eps * LSE_i[(f_i - C_ij)/eps + log a_i]       (one fused streaming pass)
+ * Outputs: f (n floats) and g (m floats), the iterate after the last g-update.
+ * g_init (m floats, device) may alias g.
+ */
+FS_API fs_status fs_potentials(const fs_problem* p, int32_t n_iters, const float* g_init, float* f,
+                        float* g, void* ws, size_t ws_bytes, fs_stream_t stream);
+
+/*
+ * Dual objective at (f, g):
+ *   D(f, g) = <f, a> + <g, b> - eps * (sum_ij P_ij - m_a * m_b),
+ *   P_ij = a_i b_j exp((f_i + g_j - C_ij)/eps),  m_a = sum a, m_b = sum b.
+ * sum_ij P_ij is evaluated exactly by one streaming column pass, so any (f, g) is
+ * accepted; right after fs_potentials (P^T 1 = b) it equals
+ * <f,a> + <g,b> - eps*m*(1 - m). Writes one double to `out` (device).
+ */
+FS_API fs_status fs_cost(const fs_problem* p, const float* f, const float* g, double* out, void* ws,
+                  size_t ws_bytes, fs_stream_t stream);
+
+/*
+ * Envelope gradient of the cost with respect to x (FlashSinkhorn summary, section 3:
+ * transport-matrix application without materialising P):
+ *   ft = F(g) (a fresh f-update, fused into the same pass), Pt_ij = a_i b_j
+ *   exp((ft_i + g_j - C_ij)/eps), so sum_j Pt_ij = a_i and
+ *   grad_x[i, :] = 2 * (a_i x_i - sum_j Pt_ij y_j) = 2 a_i (x_i - T_i),
+ * T_i the barycentric projection of x_i. Only g is needed. Writes (n, d) floats.
+ */
+FS_API fs_status fs_grad_x(const fs_problem* p, const float* g, float* grad_x, void* ws,
+                    size_t ws_bytes, fs_stream_t stream);
+
+/*
+ * Marginal residuals of the plan of (f, g) (SinkSLOT README, stop_mode "marginal";
+ * FlashSinkhorn 2 abstract, "marginal residual"):
+ *   r_i = sum_j P_ij = a_i exp((f_i - F(g)_i)/eps)   (one streaming row pass)
+ *   c_j = sum_i P_ij = b_j exp((g_j - G(f)_j)/eps)   (one streaming column pass)
+ * Writes 4 doubles to `out` (device): [sum|r - a|, max|r - a|, sum|c - b|, max|c - b|].
+ * row_marg (n floats) and col_marg (m floats), when not NULL, receive r and c.
+ */
+FS_API fs_status fs_marginal_residual(const fs_problem* p, const float* f, const float* g, double* out,
+                               float* row_marg, float* col_marg, void* ws, size_t ws_bytes,
+                               fs_stream_t stream);
+
+/*
+ * One call for callers whose data live in HOST memory: copies x, y, a, b (and nothing
+ * else) to the device, runs fs_potentials, fs_grad_x, fs_marginal_residual and
+ * fs_cost, and copies f, g, grad_x, the cost and the four residual norms back.
+ * Pointer fields of `p` and every array argument are HOST pointers (page-locked
+ * memory makes the copies asynchronous; pageable memory works but is slower);
+ * grad_x, cost and residual may be NULL to skip those steps. `ws` is device scratch
+ * of at least fs_solve_host_workspace_bytes(p) bytes.
+ */
+FS_API size_t fs_solve_host_workspace_bytes(const fs_problem* p);
+FS_API fs_status fs_solve_host(const fs_problem* p, int32_t n_iters, float* f, float* g, float* grad_x,
+                        double* cost, double* residual, void* ws, size_t ws_bytes,
+                        fs_stream_t stream);
+
+/*
+ * Kernel timing, off by default. When on, every launch of the streaming passes is
+ * bracketed by CUDA events recorded on the stream it runs on, and each entry point
+ * adds the measured durations before returning. Process-wide; not for concurrent use.
+ */
+typedef struct {
+  int64_t launches; /* launches measured since the last reset */
+  double total_ms;  /* their summed device durations */
+  double pairs;     /* (row, column) pairs they evaluated, i.e. exponentials */
+} fs_timing_entry;
+
+typedef struct {
+  fs_timing_entry lse_pass;  /* potential-update passes (f and g half-iterations) */
+  fs_timing_entry grad_pass; /* gradient passes */
+  fs_timing_entry marg_pass; /* marginal / plan-mass passes (residual and cost) */
+  fs_timing_entry combine;   /* split-column merge kernels */
+} fs_timing;
+
+FS_API void fs_timing_enable(int on);
+FS_API void fs_timing_reset(void);
+FS_API void fs_timing_get(fs_timing* out);
+
+/* Number of CUDA kernels this library has launched in this process (all entry points,
+ * all devices), counted at each launch site. */
+FS_API int64_t fs_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FS_H_ */

@@ -1,0 +1,775 @@
+// fs_api.cu -- the C ABI (include/fs.h): argument checks, input validation on the device,
+// workspace carving, launch planning and stream ordering of the streaming passes.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/fs.h"
+#include "fs_kernels.cuh"
+
+namespace fs {
+namespace {
+
+thread_local char g_cuda_err[256] = "";
+std::atomic<int64_t> g_launches{0};
+
+struct CudaFail {};
+
+inline void ck(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) {
+    snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", what, cudaGetErrorString(e));
+    throw CudaFail{};
+  }
+}
+#define CK(call) ck((call), #call)
+
+// ---------------- kernel timing ----------------
+std::mutex g_timing_mu;
+bool g_timing_on = false;
+fs_timing g_timing = {};
+
+enum TimedKind { kTLse = 0, kTGrad = 1, kTMarg = 2, kTCombine = 3 };
+
+struct TimedLaunch {
+  cudaEvent_t start, stop;
+  int kind;
+  double pairs;
+};
+
+class Timer {
+ public:
+  explicit Timer(cudaStream_t s) : stream_(s) {
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    on_ = g_timing_on;
+  }
+  ~Timer() {
+    for (auto& t : rec_) {
+      cudaEventDestroy(t.start);
+      cudaEventDestroy(t.stop);
+    }
+  }
+  int begin() {
+    if (!on_) return -1;
+    TimedLaunch t{};
+    CK(cudaEventCreate(&t.start));
+    CK(cudaEventCreate(&t.stop));
+    CK(cudaEventRecord(t.start, stream_));
+    rec_.push_back(t);
+    return static_cast<int>(rec_.size()) - 1;
+  }
+  void end(int idx, int kind, double pairs) {
+    if (idx < 0) return;
+    rec_[idx].kind = kind;
+    rec_[idx].pairs = pairs;
+    CK(cudaEventRecord(rec_[idx].stop, stream_));
+  }
+  // Call after the stream has been synchronised.
+  void collect() {
+    if (!on_) return;
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    for (auto& t : rec_) {
+      float ms = 0.f;
+      CK(cudaEventElapsedTime(&ms, t.start, t.stop));
+      fs_timing_entry* e = t.kind == kTLse    ? &g_timing.lse_pass
+                           : t.kind == kTGrad ? &g_timing.grad_pass
+                           : t.kind == kTMarg ? &g_timing.marg_pass
+                                              : &g_timing.combine;
+      e->launches += 1;
+      e->total_ms += ms;
+      e->pairs += t.pairs;
+    }
+  }
+
+ private:
+  cudaStream_t stream_;
+  bool on_ = false;
+  std::vector<TimedLaunch> rec_;
+};
+
+// ---------------- shapes, plans and the workspace ----------------
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+int padded_dim(int d) {
+  if (d <= 4) return d;
+  if (d <= 8) return 8;
+  if (d <= 16) return 16;
+  if (d <= 32) return 32;
+  return 64;
+}
+
+int64_t pairs_pad(int64_t count) { return round_up(ceil_div(count, 2), kPairPad); }
+
+// Launch variants of the streaming pass: (rows per thread, threads per CTA).
+struct Variant {
+  int R, NT;
+};
+// LSE passes for D <= 16, from most to least rows per CTA.
+constexpr Variant kLseVariants[3] = {{4, 256}, {2, 128}, {1, 128}};
+// Gradient passes for D <= 16.
+constexpr Variant kGradVariants[2] = {{2, 256}, {1, 128}};
+// Everything for D > 16.
+constexpr Variant kWideVariant = {1, 128};
+
+struct Plan {
+  int variant;  // index into the variant table of this pass type
+  int R, NT;
+  int64_t row_blocks, rows_pad;
+  int tile_pairs;
+  int n_splits;
+  int64_t pairs_per_split;
+};
+
+int num_sms_current() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaGetLastError();
+  return sms > 0 ? sms : 148;
+}
+
+Plan make_plan(int64_t n_rows, int64_t key_pairs, int D, bool grad, int sms) {
+  const int64_t target = static_cast<int64_t>(sms) * 8;  // >= ~4 waves of 2 CTAs per SM
+  const int max_tile = D > 16 ? 32 : 128;
+  const Variant* vars;
+  int nv;
+  if (D > 16) {
+    vars = &kWideVariant;
+    nv = 1;
+  } else if (grad) {
+    vars = kGradVariants;
+    nv = 2;
+  } else {
+    vars = kLseVariants;
+    nv = 3;
+  }
+  Plan p{};
+  // Most rows per CTA whose (row blocks x tiles) still fills the machine; else the smallest.
+  int chosen = nv - 1;
+  for (int v = 0; v < nv; ++v) {
+    const int64_t rb = ceil_div(n_rows, static_cast<int64_t>(vars[v].R) * vars[v].NT);
+    if (rb * (key_pairs / max_tile) >= target) {
+      chosen = v;
+      break;
+    }
+  }
+  p.variant = chosen;
+  p.R = vars[chosen].R;
+  p.NT = vars[chosen].NT;
+  const int64_t rpc = static_cast<int64_t>(p.R) * p.NT;
+  p.row_blocks = ceil_div(n_rows, rpc);
+  p.rows_pad = p.row_blocks * rpc;
+  int tile = max_tile;
+  while (tile > 16 && p.row_blocks * (key_pairs / tile) < target) tile /= 2;
+  p.tile_pairs = tile;
+  const int64_t tiles = key_pairs / tile;
+  int64_t splits = std::min<int64_t>(tiles, std::max<int64_t>(1, ceil_div(target, p.row_blocks)));
+  splits = std::min<int64_t>(splits, 65535);
+  const int64_t per = ceil_div(tiles, splits);
+  p.n_splits = static_cast<int>(ceil_div(tiles, per));
+  p.pairs_per_split = per * tile;
+  return p;
+}
+
+int64_t partial_floats(const Plan& p, int D, bool grad) {
+  if (p.n_splits <= 1) return 0;
+  return static_cast<int64_t>(p.n_splits) * p.rows_pad * (2 + (grad ? D : 0));
+}
+
+constexpr size_t kAlign = 256;
+constexpr int kScalarDoubles = 256;  // 2 KiB of float64 scalars
+
+// Offsets (in doubles) inside the scalar block.
+constexpr int kSumX = 0;      // [64]
+constexpr int kSumY = 64;     // [64]
+constexpr int kSumA = 128;
+constexpr int kSumB = 129;
+constexpr int kAccRow = 130;  // [3]
+constexpr int kAccCol = 133;  // [3]
+constexpr int kDotFA = 136;
+constexpr int kDotGB = 137;
+constexpr int kFlags = 140;   // unsigned, in the bytes of this double
+constexpr int kErr = 141;     // unsigned
+
+struct Layout {
+  int D;       // padded dimension
+  int KP;      // floats per key pair
+  int64_t px;  // key pairs of x (padded)
+  int64_t py;
+  size_t off_scalars, off_kx, off_ky, off_lwx, off_lwy, off_part, total;
+  int64_t part_floats;
+};
+
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+Layout make_layout(int64_t n, int64_t m, int d, int sms) {
+  Layout L{};
+  L.D = padded_dim(d);
+  L.KP = key_pair_floats(L.D);
+  L.px = pairs_pad(n);
+  L.py = pairs_pad(m);
+  int64_t pf = 0;
+  for (int grad = 0; grad < 2; ++grad) {
+    pf = std::max(pf, partial_floats(make_plan(n, L.py, L.D, grad, sms), L.D, grad));
+    pf = std::max(pf, partial_floats(make_plan(m, L.px, L.D, grad, sms), L.D, grad));
+  }
+  L.part_floats = pf;
+  size_t o = 0;
+  L.off_scalars = o;
+  o = align_up(o + kScalarDoubles * sizeof(double));
+  L.off_kx = o;
+  o = align_up(o + static_cast<size_t>(L.px) * L.KP * sizeof(float));
+  L.off_ky = o;
+  o = align_up(o + static_cast<size_t>(L.py) * L.KP * sizeof(float));
+  L.off_lwx = o;
+  o = align_up(o + static_cast<size_t>(2 * L.px) * sizeof(float));
+  L.off_lwy = o;
+  o = align_up(o + static_cast<size_t>(2 * L.py) * sizeof(float));
+  L.off_part = o;
+  o = align_up(o + static_cast<size_t>(pf) * sizeof(float));
+  L.total = o;
+  return L;
+}
+
+bool shape_ok(const fs_problem* p) {
+  return p && p->n >= 1 && p->m >= 1 && p->d >= 1 && p->n <= (int64_t(1) << 40) &&
+         p->m <= (int64_t(1) << 40);
+}
+
+inline bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; }
+
+// ---------------- kernel dispatch ----------------
+
+template <int D, int R, int NT, bool GRAD>
+void launch_pass_t(const PassParams& P, const Plan& pl, cudaStream_t st) {
+  constexpr int G = (D > 16) ? 4 : 8;
+  constexpr int MINB = (D > 16) ? 1 : (NT == 256 ? 2 : 4);
+  auto kern = lse_pass_kernel<D, R, NT, G, GRAD, MINB>;
+  const size_t smem = static_cast<size_t>(kStages) * pl.tile_pairs * key_pair_floats(D) * 4;
+  static bool attr_set = false;  // per instantiation; idempotent, so a race is harmless
+  if (!attr_set) {
+    CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            static_cast<int>(kStages * 128 * key_pair_floats(D) * 4)));
+    attr_set = true;
+  }
+  dim3 grid(static_cast<unsigned>(pl.row_blocks), static_cast<unsigned>(pl.n_splits));
+  kern<<<grid, NT, smem, st>>>(P);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
+template <int D>
+void launch_pass_d(const PassParams& P, const Plan& pl, bool grad, cudaStream_t st) {
+  if constexpr (D > 16) {
+    if (grad)
+      launch_pass_t<D, 1, 128, true>(P, pl, st);
+    else
+      launch_pass_t<D, 1, 128, false>(P, pl, st);
+  } else {
+    if (grad) {
+      if (pl.variant == 0)
+        launch_pass_t<D, 2, 256, true>(P, pl, st);
+      else
+        launch_pass_t<D, 1, 128, true>(P, pl, st);
+    } else {
+      if (pl.variant == 0)
+        launch_pass_t<D, 4, 256, false>(P, pl, st);
+      else if (pl.variant == 1)
+        launch_pass_t<D, 2, 128, false>(P, pl, st);
+      else
+        launch_pass_t<D, 1, 128, false>(P, pl, st);
+    }
+  }
+}
+
+template <int D>
+void launch_combine_d(const PassParams& P, bool grad, cudaStream_t st) {
+  const unsigned blocks = static_cast<unsigned>(ceil_div(P.n_rows, 256));
+  if (grad)
+    combine_kernel<D, true><<<blocks, 256, 0, st>>>(P);
+  else
+    combine_kernel<D, false><<<blocks, 256, 0, st>>>(P);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
+#define FS_DISPATCH_D(D, FN, ...)                 \
+  switch (D) {                                    \
+    case 1: FN<1>(__VA_ARGS__); break;            \
+    case 2: FN<2>(__VA_ARGS__); break;            \
+    case 3: FN<3>(__VA_ARGS__); break;            \
+    case 4: FN<4>(__VA_ARGS__); break;            \
+    case 8: FN<8>(__VA_ARGS__); break;            \
+    case 16: FN<16>(__VA_ARGS__); break;          \
+    case 32: FN<32>(__VA_ARGS__); break;          \
+    default: FN<64>(__VA_ARGS__); break;          \
+  }
+
+template <int D>
+void launch_pack_d(const float* pts, int64_t count, int d, const Center& c, const float* w,
+                   float wu, float* keys, float* lw, int64_t pp, cudaStream_t st) {
+  const unsigned blocks = static_cast<unsigned>(ceil_div(2 * pp, 256));
+  pack_kernel<D><<<blocks, 256, 0, st>>>(pts, count, d, c, w, wu, keys, lw, pp);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
+template <int D>
+void launch_bias_d(float* keys, int64_t count, const float* pot, const float* lw, double kappa,
+                   cudaStream_t st) {
+  const unsigned blocks = static_cast<unsigned>(ceil_div(count, 256));
+  key_bias_kernel<D><<<blocks, 256, 0, st>>>(keys, count, pot, lw, kappa);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
+// ---------------- one call's context ----------------
+
+struct Ctx {
+  const fs_problem* p;
+  cudaStream_t st;
+  Layout L;
+  int sms;
+  unsigned char* ws;
+  double* scal;
+  float* kx;
+  float* ky;
+  float* lwx;
+  float* lwy;
+  float* part;
+  double ma, mb;  // weight sums
+  double kappa;
+  Timer* timer;
+};
+
+fs_status check_common(const fs_problem* p, void* ws, size_t ws_bytes, size_t* need_out,
+                       int sms) {
+  if (!p) return FS_ERR_NULL;
+  if (!shape_ok(p)) return FS_ERR_SHAPE;
+  if (p->d > FS_MAX_D) return FS_ERR_UNSUPPORTED_D;
+  if (!(std::isfinite(p->eps) && p->eps > 0.0f)) return FS_ERR_EPS;
+  if (!p->x || !p->y) return FS_ERR_NULL;
+  if (!aligned4(p->x) || !aligned4(p->y) || !aligned4(p->a) || !aligned4(p->b))
+    return FS_ERR_ALIGNMENT;
+  const Layout L = make_layout(p->n, p->m, p->d, sms);
+  *need_out = L.total;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || ws_bytes < L.total)
+    return FS_ERR_WORKSPACE;
+  return FS_OK;
+}
+
+void carve(Ctx& c, void* ws) {
+  c.ws = static_cast<unsigned char*>(ws);
+  c.scal = reinterpret_cast<double*>(c.ws + c.L.off_scalars);
+  c.kx = reinterpret_cast<float*>(c.ws + c.L.off_kx);
+  c.ky = reinterpret_cast<float*>(c.ws + c.L.off_ky);
+  c.lwx = reinterpret_cast<float*>(c.ws + c.L.off_lwx);
+  c.lwy = reinterpret_cast<float*>(c.ws + c.L.off_lwy);
+  c.part = reinterpret_cast<float*>(c.ws + c.L.off_part);
+}
+
+unsigned* flags_ptr(double* scal) { return reinterpret_cast<unsigned*>(scal + kFlags); }
+unsigned* err_ptr(double* scal) { return reinterpret_cast<unsigned*>(scal + kErr); }
+
+unsigned reduce_blocks(int64_t count, int sms) {
+  return static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(ceil_div(count, 256), sms * 4)));
+}
+
+// Validates inputs on the device (one stream sync), packs both clouds and their log-weights.
+// `pots` lists potentials to check for finiteness (device pointers with their lengths).
+fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& pots) {
+  const fs_problem* p = c.p;
+  CK(cudaMemsetAsync(c.scal, 0, kScalarDoubles * sizeof(double), c.st));
+  dim3 gx(reduce_blocks(p->n, c.sms), p->d), gy(reduce_blocks(p->m, c.sms), p->d);
+  reduce_coords_kernel<<<gx, 256, 0, c.st>>>(p->x, p->n, p->d, c.scal + kSumX, flags_ptr(c.scal));
+  CK(cudaGetLastError());
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  reduce_coords_kernel<<<gy, 256, 0, c.st>>>(p->y, p->m, p->d, c.scal + kSumY, flags_ptr(c.scal));
+  CK(cudaGetLastError());
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (p->a) {
+    reduce_weights_kernel<<<reduce_blocks(p->n, c.sms), 256, 0, c.st>>>(p->a, p->n, c.scal + kSumA,
+                                                                       flags_ptr(c.scal));
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  if (p->b) {
+    reduce_weights_kernel<<<reduce_blocks(p->m, c.sms), 256, 0, c.st>>>(p->b, p->m, c.scal + kSumB,
+                                                                       flags_ptr(c.scal));
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  for (auto& pv : pots) {
+    check_finite_kernel<<<reduce_blocks(pv.second, c.sms), 256, 0, c.st>>>(pv.first, pv.second,
+                                                                          flags_ptr(c.scal));
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  double host[kFlags + 2];
+  CK(cudaMemcpyAsync(host, c.scal, sizeof(host), cudaMemcpyDeviceToHost, c.st));
+  CK(cudaStreamSynchronize(c.st));
+  unsigned flags;
+  memcpy(&flags, &host[kFlags], sizeof(unsigned));
+  if (flags & 2u) return FS_ERR_NEGATIVE_WEIGHT;
+  if (flags & (1u | 4u)) return FS_ERR_NONFINITE_INPUT;
+  c.ma = p->a ? host[kSumA] : static_cast<double>(static_cast<float>(1.0 / p->n)) * p->n;
+  c.mb = p->b ? host[kSumB] : static_cast<double>(static_cast<float>(1.0 / p->m)) * p->m;
+  if (!(c.ma > 0.0) || !(c.mb > 0.0)) return FS_ERR_ZERO_MASS;
+  if (std::fabs(c.ma - c.mb) > 1e-5 * std::max(c.ma, c.mb)) return FS_ERR_MASS_MISMATCH;
+
+  Center ctr{};
+  for (int k = 0; k < p->d; ++k)
+    ctr.c[k] = (host[kSumX + k] + host[kSumY + k]) / static_cast<double>(p->n + p->m);
+  const float wu_x = static_cast<float>(1.0 / p->n), wu_y = static_cast<float>(1.0 / p->m);
+  FS_DISPATCH_D(c.L.D, launch_pack_d, p->x, p->n, p->d, ctr, p->a, wu_x, c.kx, c.lwx, c.L.px, c.st);
+  FS_DISPATCH_D(c.L.D, launch_pack_d, p->y, p->m, p->d, ctr, p->b, wu_y, c.ky, c.lwy, c.L.py, c.st);
+  return FS_OK;
+}
+
+// Sets the key bias of one cloud from a potential (NULL = zero potential).
+void set_bias(Ctx& c, bool cloud_x, const float* pot) {
+  if (cloud_x)
+    FS_DISPATCH_D(c.L.D, launch_bias_d, c.kx, c.p->n, pot, c.lwx, c.kappa, c.st)
+  else
+    FS_DISPATCH_D(c.L.D, launch_bias_d, c.ky, c.p->m, pot, c.lwy, c.kappa, c.st)
+}
+
+// One streaming pass with rows from cloud x (rows_x) or y, keys from the other cloud.
+void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out, float* marg_out,
+              float* grad_out, double* acc) {
+  const fs_problem* p = c.p;
+  const bool grad = kind == kGrad;
+  const int64_t n_rows = rows_x ? p->n : p->m;
+  const int64_t key_pairs = rows_x ? c.L.py : c.L.px;
+  const Plan pl = make_plan(n_rows, key_pairs, c.L.D, grad, c.sms);
+  PassParams P{};
+  P.keys = rows_x ? c.ky : c.kx;
+  P.qkeys = rows_x ? c.kx : c.ky;
+  P.n_rows = n_rows;
+  P.key_pairs = key_pairs;
+  P.pairs_per_split = pl.pairs_per_split;
+  P.tile_pairs = pl.tile_pairs;
+  P.n_splits = pl.n_splits;
+  P.rows_pad = pl.rows_pad;
+  P.kind = kind;
+  P.d_real = p->d;
+  P.kappa = c.kappa;
+  P.two_kappa = static_cast<float>(2.0 * c.kappa);
+  P.eps_ln2 = 1.0 / c.kappa;
+  P.lw = rows_x ? c.lwx : c.lwy;
+  P.w = rows_x ? p->a : p->b;
+  P.w_uniform = static_cast<float>(1.0 / n_rows);
+  P.pot_in = pot_in;
+  P.pot_out = pot_out;
+  P.marg_out = marg_out;
+  P.grad_out = grad_out;
+  P.acc = acc;
+  P.part_m = c.part;
+  P.part_l = c.part + static_cast<int64_t>(pl.n_splits) * pl.rows_pad;
+  P.part_a = c.part + 2 * static_cast<int64_t>(pl.n_splits) * pl.rows_pad;
+  P.err = err_ptr(c.scal);
+  const double pairs = static_cast<double>(n_rows) * static_cast<double>(rows_x ? p->m : p->n);
+  const int tk = grad ? kTGrad : (kind == kMarg ? kTMarg : kTLse);
+  int ti = c.timer->begin();
+  FS_DISPATCH_D(c.L.D, launch_pass_d, P, pl, grad, c.st);
+  c.timer->end(ti, tk, pairs);
+  if (pl.n_splits > 1) {
+    ti = c.timer->begin();
+    FS_DISPATCH_D(c.L.D, launch_combine_d, P, grad, c.st);
+    c.timer->end(ti, kTCombine, 0.0);
+  }
+}
+
+// Drains the stream and reads the kernels' error word.
+fs_status finish(Ctx& c) {
+  unsigned err = 0;
+  CK(cudaMemcpyAsync(&err, err_ptr(c.scal), sizeof(unsigned), cudaMemcpyDeviceToHost, c.st));
+  CK(cudaStreamSynchronize(c.st));
+  c.timer->collect();
+  return err ? FS_ERR_TIMEOUT : FS_OK;
+}
+
+template <typename F>
+fs_status guarded(cudaStream_t st, F&& body) {
+  try {
+    return body();
+  } catch (const CudaFail&) {
+    cudaStreamSynchronize(st);
+    cudaGetLastError();
+    return FS_ERR_CUDA;
+  }
+}
+
+fs_status begin(Ctx& c, const fs_problem* p, void* ws, size_t ws_bytes, fs_stream_t stream) {
+  c.sms = num_sms_current();
+  size_t need = 0;
+  const fs_status s = check_common(p, ws, ws_bytes, &need, c.sms);
+  if (s != FS_OK) return s;
+  c.p = p;
+  c.st = reinterpret_cast<cudaStream_t>(stream);
+  c.L = make_layout(p->n, p->m, p->d, c.sms);
+  c.kappa = 1.4426950408889634 / static_cast<double>(p->eps);
+  carve(c, ws);
+  return FS_OK;
+}
+
+}  // namespace
+
+// ---------------- entry points ----------------
+
+fs_status potentials_impl(const fs_problem* p, int32_t n_iters, const float* g_init, float* f,
+                          float* g, void* ws, size_t ws_bytes, fs_stream_t stream) {
+  Ctx c{};
+  fs_status s = begin(c, p, ws, ws_bytes, stream);
+  if (s != FS_OK) return s;
+  if (!f || !g) return FS_ERR_NULL;
+  if (!aligned4(f) || !aligned4(g) || !aligned4(g_init)) return FS_ERR_ALIGNMENT;
+  if (n_iters < 1) return FS_ERR_ITERS;
+  Timer timer(c.st);
+  c.timer = &timer;
+  return guarded(c.st, [&]() -> fs_status {
+    std::vector<std::pair<const float*, int64_t>> pots;
+    if (g_init) pots.push_back({g_init, p->m});
+    fs_status r = prepare(c, pots);
+    if (r != FS_OK) return r;
+    set_bias(c, false, g_init);
+    for (int32_t it = 0; it < n_iters; ++it) {
+      run_pass(c, true, kPot, nullptr, f, nullptr, nullptr, nullptr);   // f <- F(g)
+      run_pass(c, false, kPot, nullptr, g, nullptr, nullptr, nullptr);  // g <- G(f)
+    }
+    return finish(c);
+  });
+}
+
+}  // namespace fs
+
+extern "C" {
+
+const char* fs_status_string(fs_status s) {
+  switch (s) {
+    case FS_OK: return "FS_OK";
+    case FS_ERR_NULL: return "FS_ERR_NULL: a required pointer is NULL";
+    case FS_ERR_SHAPE: return "FS_ERR_SHAPE: n, m and d must be >= 1";
+    case FS_ERR_EPS: return "FS_ERR_EPS: eps must be finite and > 0";
+    case FS_ERR_ITERS: return "FS_ERR_ITERS: n_iters must be >= 1";
+    case FS_ERR_NEGATIVE_WEIGHT: return "FS_ERR_NEGATIVE_WEIGHT: weights must be finite and >= 0";
+    case FS_ERR_NONFINITE_INPUT: return "FS_ERR_NONFINITE_INPUT: a coordinate or potential is not finite";
+    case FS_ERR_MASS_MISMATCH: return "FS_ERR_MASS_MISMATCH: sum(a) and sum(b) differ by more than 1e-5 relative";
+    case FS_ERR_ZERO_MASS: return "FS_ERR_ZERO_MASS: the total mass is zero";
+    case FS_ERR_UNSUPPORTED_D: return "FS_ERR_UNSUPPORTED_D: d exceeds FS_MAX_D";
+    case FS_ERR_WORKSPACE: return "FS_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case FS_ERR_TIMEOUT: return "FS_ERR_TIMEOUT: a kernel's bounded wait expired";
+    case FS_ERR_CUDA: return "FS_ERR_CUDA: a CUDA runtime call failed";
+    case FS_ERR_ALIGNMENT: return "FS_ERR_ALIGNMENT: device pointers must be 4-byte aligned";
+  }
+  return "unknown fs_status";
+}
+
+const char* fs_last_cuda_error(void) { return fs::g_cuda_err; }
+
+size_t fs_workspace_bytes(const fs_problem* p) {
+  if (!fs::shape_ok(p) || p->d > FS_MAX_D) return 0;
+  return fs::make_layout(p->n, p->m, p->d, fs::num_sms_current()).total;
+}
+
+fs_status fs_potentials(const fs_problem* p, int32_t n_iters, const float* g_init, float* f,
+                        float* g, void* ws, size_t ws_bytes, fs_stream_t stream) {
+  return fs::potentials_impl(p, n_iters, g_init, f, g, ws, ws_bytes, stream);
+}
+
+fs_status fs_grad_x(const fs_problem* p, const float* g, float* grad_x, void* ws, size_t ws_bytes,
+                    fs_stream_t stream) {
+  using namespace fs;
+  Ctx c{};
+  fs_status s = begin(c, p, ws, ws_bytes, stream);
+  if (s != FS_OK) return s;
+  if (!g || !grad_x) return FS_ERR_NULL;
+  if (!aligned4(g) || !aligned4(grad_x)) return FS_ERR_ALIGNMENT;
+  Timer timer(c.st);
+  c.timer = &timer;
+  return guarded(c.st, [&]() -> fs_status {
+    fs_status r = prepare(c, {{g, p->m}});
+    if (r != FS_OK) return r;
+    set_bias(c, false, g);
+    run_pass(c, true, kGrad, nullptr, nullptr, nullptr, grad_x, nullptr);
+    return finish(c);
+  });
+}
+
+fs_status fs_marginal_residual(const fs_problem* p, const float* f, const float* g, double* out,
+                               float* row_marg, float* col_marg, void* ws, size_t ws_bytes,
+                               fs_stream_t stream) {
+  using namespace fs;
+  Ctx c{};
+  fs_status s = begin(c, p, ws, ws_bytes, stream);
+  if (s != FS_OK) return s;
+  if (!f || !g || !out) return FS_ERR_NULL;
+  if (!aligned4(f) || !aligned4(g) || !aligned4(row_marg) || !aligned4(col_marg) ||
+      (reinterpret_cast<uintptr_t>(out) & 7u))
+    return FS_ERR_ALIGNMENT;
+  Timer timer(c.st);
+  c.timer = &timer;
+  return guarded(c.st, [&]() -> fs_status {
+    fs_status r = prepare(c, {{f, p->n}, {g, p->m}});
+    if (r != FS_OK) return r;
+    set_bias(c, false, g);  // keys y carry g: row pass gives F(g)
+    set_bias(c, true, f);   // keys x carry f: column pass gives G(f)
+    run_pass(c, true, kMarg, f, nullptr, row_marg, nullptr, c.scal + kAccRow);
+    run_pass(c, false, kMarg, g, nullptr, col_marg, nullptr, c.scal + kAccCol);
+    residual_finish_kernel<<<1, 32, 0, c.st>>>(c.scal + kAccRow, c.scal + kAccCol, out);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return finish(c);
+  });
+}
+
+fs_status fs_cost(const fs_problem* p, const float* f, const float* g, double* out, void* ws,
+                  size_t ws_bytes, fs_stream_t stream) {
+  using namespace fs;
+  Ctx c{};
+  fs_status s = begin(c, p, ws, ws_bytes, stream);
+  if (s != FS_OK) return s;
+  if (!f || !g || !out) return FS_ERR_NULL;
+  if (!aligned4(f) || !aligned4(g) || (reinterpret_cast<uintptr_t>(out) & 7u))
+    return FS_ERR_ALIGNMENT;
+  Timer timer(c.st);
+  c.timer = &timer;
+  return guarded(c.st, [&]() -> fs_status {
+    fs_status r = prepare(c, {{f, p->n}, {g, p->m}});
+    if (r != FS_OK) return r;
+    set_bias(c, true, f);  // keys x carry f: column pass gives c_j = sum_i P_ij
+    run_pass(c, false, kMarg, g, nullptr, nullptr, nullptr, c.scal + kAccCol);
+    dot_kernel<<<reduce_blocks(p->n, c.sms), 256, 0, c.st>>>(f, p->a, static_cast<float>(1.0 / p->n),
+                                                            p->n, c.scal + kDotFA);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    dot_kernel<<<reduce_blocks(p->m, c.sms), 256, 0, c.st>>>(g, p->b, static_cast<float>(1.0 / p->m),
+                                                            p->m, c.scal + kDotGB);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    cost_finish_kernel<<<1, 32, 0, c.st>>>(c.scal + kDotFA, c.scal + kDotGB, c.scal + kAccCol + 2,
+                                           static_cast<double>(p->eps), c.ma * c.mb, out);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return finish(c);
+  });
+}
+
+size_t fs_solve_host_workspace_bytes(const fs_problem* p) {
+  using namespace fs;
+  if (!shape_ok(p) || p->d > FS_MAX_D) return 0;
+  const size_t n = static_cast<size_t>(p->n), m = static_cast<size_t>(p->m),
+               d = static_cast<size_t>(p->d);
+  size_t o = fs_workspace_bytes(p);
+  o = align_up(o + n * d * 4);      // x
+  o = align_up(o + m * d * 4);      // y
+  o = align_up(o + n * 4);          // a
+  o = align_up(o + m * 4);          // b
+  o = align_up(o + n * 4);          // f
+  o = align_up(o + m * 4);          // g
+  o = align_up(o + n * d * 4);      // grad
+  o = align_up(o + 8 * sizeof(double));  // cost + residual
+  return o;
+}
+
+fs_status fs_solve_host(const fs_problem* hp, int32_t n_iters, float* f, float* g, float* grad_x,
+                        double* cost, double* residual, void* ws, size_t ws_bytes,
+                        fs_stream_t stream) {
+  using namespace fs;
+  if (!hp) return FS_ERR_NULL;
+  if (!shape_ok(hp)) return FS_ERR_SHAPE;
+  if (hp->d > FS_MAX_D) return FS_ERR_UNSUPPORTED_D;
+  if (!hp->x || !hp->y || !f || !g) return FS_ERR_NULL;
+  if (n_iters < 1) return FS_ERR_ITERS;
+  const size_t need = fs_solve_host_workspace_bytes(hp);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || ws_bytes < need)
+    return FS_ERR_WORKSPACE;
+  const size_t n = static_cast<size_t>(hp->n), m = static_cast<size_t>(hp->m),
+               d = static_cast<size_t>(hp->d);
+  const size_t inner = fs_workspace_bytes(hp);
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  size_t o = inner;
+  float* dx = reinterpret_cast<float*>(base + o);
+  o = align_up(o + n * d * 4);
+  float* dy = reinterpret_cast<float*>(base + o);
+  o = align_up(o + m * d * 4);
+  float* da = reinterpret_cast<float*>(base + o);
+  o = align_up(o + n * 4);
+  float* db = reinterpret_cast<float*>(base + o);
+  o = align_up(o + m * 4);
+  float* df = reinterpret_cast<float*>(base + o);
+  o = align_up(o + n * 4);
+  float* dg = reinterpret_cast<float*>(base + o);
+  o = align_up(o + m * 4);
+  float* dgrad = reinterpret_cast<float*>(base + o);
+  o = align_up(o + n * d * 4);
+  double* dsc = reinterpret_cast<double*>(base + o);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  try {
+    CK(cudaMemcpyAsync(dx, hp->x, n * d * 4, cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(dy, hp->y, m * d * 4, cudaMemcpyHostToDevice, st));
+    if (hp->a) CK(cudaMemcpyAsync(da, hp->a, n * 4, cudaMemcpyHostToDevice, st));
+    if (hp->b) CK(cudaMemcpyAsync(db, hp->b, m * 4, cudaMemcpyHostToDevice, st));
+  } catch (const CudaFail&) {
+    cudaStreamSynchronize(st);
+    cudaGetLastError();
+    return FS_ERR_CUDA;
+  }
+  fs_problem dp = *hp;
+  dp.x = dx;
+  dp.y = dy;
+  dp.a = hp->a ? da : nullptr;
+  dp.b = hp->b ? db : nullptr;
+  fs_status s = fs_potentials(&dp, n_iters, nullptr, df, dg, ws, inner, stream);
+  if (s != FS_OK) return s;
+  if (grad_x) {
+    s = fs_grad_x(&dp, dg, dgrad, ws, inner, stream);
+    if (s != FS_OK) return s;
+  }
+  if (residual) {
+    s = fs_marginal_residual(&dp, df, dg, dsc + 1, nullptr, nullptr, ws, inner, stream);
+    if (s != FS_OK) return s;
+  }
+  if (cost) {
+    s = fs_cost(&dp, df, dg, dsc, ws, inner, stream);
+    if (s != FS_OK) return s;
+  }
+  try {
+    CK(cudaMemcpyAsync(f, df, n * 4, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(g, dg, m * 4, cudaMemcpyDeviceToHost, st));
+    if (grad_x) CK(cudaMemcpyAsync(grad_x, dgrad, n * d * 4, cudaMemcpyDeviceToHost, st));
+    if (residual) CK(cudaMemcpyAsync(residual, dsc + 1, 4 * sizeof(double), cudaMemcpyDeviceToHost, st));
+    if (cost) CK(cudaMemcpyAsync(cost, dsc, sizeof(double), cudaMemcpyDeviceToHost, st));
+    CK(cudaStreamSynchronize(st));
+  } catch (const CudaFail&) {
+    cudaStreamSynchronize(st);
+    cudaGetLastError();
+    return FS_ERR_CUDA;
+  }
+  return FS_OK;
+}
+
+int64_t fs_launch_count(void) { return fs::g_launches.load(std::memory_order_relaxed); }
+
+void fs_timing_enable(int on) {
+  std::lock_guard<std::mutex> lk(fs::g_timing_mu);
+  fs::g_timing_on = on != 0;
+}
+
+void fs_timing_reset(void) {
+  std::lock_guard<std::mutex> lk(fs::g_timing_mu);
+  fs::g_timing = fs_timing{};
+}
+
+void fs_timing_get(fs_timing* out) {
+  if (!out) return;
+  std::lock_guard<std::mutex> lk(fs::g_timing_mu);
+  *out = fs::g_timing;
+}
+
+}  // extern "C"

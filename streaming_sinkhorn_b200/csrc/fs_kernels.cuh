@@ -1,0 +1,527 @@
+// fs_kernels.cuh -- CUDA kernels of the streaming log-domain Sinkhorn passes (sm_100a).
+//
+// One pass evaluates, for every query row i, the base-2 log-sum-exp over all key
+// columns j of the biased dot-product score
+//     s_ij = (2 kappa x_i) . y_j + h_j,      kappa = log2(e) / eps,
+//     h_j  = kappa (g_j - |y_j|^2) + log2 b_j,
+// which is the FlashSinkhorn attention-form of the log-domain update (FlashSinkhorn
+// summary, Methodology section 1: the cost |x|^2 + |y|^2 - 2 x.y splits into a dot
+// product plus per-column and per-row biases). Then
+//     F(g)_i = |x_i|^2 - LSE2_j(s_ij) / kappa.
+// The same pass with the roles of the clouds swapped is the g-update.
+//
+// Layout in HBM. Each cloud is stored once as "packed keys": point pairs (2p, 2p+1)
+// share KP floats laid out as [c0 c0' c1 c1' ... c_{D-1} c_{D-1}' h h' pad], i.e. every
+// coordinate (and the bias h) of the two points sits side by side so that one 64-bit
+// register holds the same component of two columns, ready for the packed fp32x2 FMA.
+// Coordinates are centred on the common mean of both clouds (the cost is translation
+// invariant); the pair count is padded to a multiple of 128 with zero coordinates and
+// h = kLogZero, which contribute nothing.
+//
+// A CTA owns NT*R query rows (R rows per thread, kept in registers) and streams one
+// contiguous range of key pairs through shared memory with TMA bulk copies
+// (kStages-deep ring, mbarrier completion). Each thread runs an online max/sum over its
+// rows: per group of G key pairs the row max is taken first; the running sum is
+// rescaled only when that max exceeds the running offset by more than kLazyThr (terms
+// then stay below 2^kLazyThr), so the per-pair work is d packed FMAs, one packed add,
+// one MUFU ex2 per column and a packed accumulate. When the key range is split over
+// several CTAs, each writes its (max, sum[, weighted coordinates]) partial and a combine
+// kernel merges them with a second-level LSE.
+#pragma once
+
+#include <cfloat>
+#include <cmath>
+#include "fs_device.cuh"
+
+namespace fs {
+
+// Floats per packed key pair for padded dimension D: 2(D+1) rounded up to 4.
+__host__ __device__ constexpr int key_pair_floats(int D) { return ((2 * (D + 1) + 3) / 4) * 4; }
+
+constexpr int kStages = 3;
+constexpr float kLazyThr = 8.0f;
+constexpr int kPairPad = 128;  // key pairs are padded to a multiple of this
+
+enum PassKind : int { kPot = 0, kMarg = 1, kGrad = 2 };
+
+struct PassParams {
+  const float* keys;        // streamed cloud, packed
+  float* qkeys;             // query cloud, packed (coordinates read; h written by kPot)
+  int64_t n_rows;           // real number of query rows
+  int64_t key_pairs;        // padded key pair count
+  int64_t pairs_per_split;  // key pairs per split (multiple of tile_pairs)
+  int32_t tile_pairs;       // key pairs per shared-memory stage
+  int32_t n_splits;         // gridDim.y
+  int64_t rows_pad;         // row stride of the partial arrays
+  int32_t kind;             // PassKind
+  int32_t d_real;           // true dimension (<= D)
+  float two_kappa;          // 2 log2(e) / eps
+  double kappa;             // log2(e) / eps
+  double eps_ln2;           // eps ln 2 = 1 / kappa
+  const float* lw;          // log2 weights of the query cloud (kLogZero for zeros)
+  const float* w;           // linear weights of the query cloud, or NULL
+  float w_uniform;          // weight used when w == NULL
+  const float* pot_in;      // kMarg: given potential of the query cloud
+  float* pot_out;           // kPot: new potential of the query cloud
+  float* marg_out;          // kMarg: plan marginal per row, or NULL
+  float* grad_out;          // kGrad: (n_rows, d_real)
+  double* acc;              // kMarg: [sum |r - w|, max |r - w|, sum r]
+  float* part_m;            // partial maxima   [split][rows_pad]
+  float* part_l;            // partial sums     [split][rows_pad]
+  float* part_a;            // partial weighted coordinates [split][D][rows_pad]
+  unsigned* err;            // error word
+};
+
+// Offset of coordinate slot k (k == D is the bias h) of point i in packed keys.
+template <int D>
+__device__ __forceinline__ int64_t key_slot(int64_t i, int k) {
+  return (i >> 1) * key_pair_floats(D) + 2 * k + (i & 1);
+}
+
+// ---- per-row completion, shared by the direct epilogue and the combine kernel -----------
+
+template <int D>
+__device__ __forceinline__ double row_sqnorm(const float* qkeys, int64_t i) {
+  double s = 0.0;
+#pragma unroll
+  for (int k = 0; k < D; ++k) {
+    const double c = qkeys[key_slot<D>(i, k)];
+    s += c * c;
+  }
+  return s;
+}
+
+// kPot: write the new potential and the key bias this row carries into the next pass.
+//   pot_i = |x_i|^2 - LSE2_i / kappa,   h_i = log2 w_i - LSE2_i  (= kappa (pot_i - |x_i|^2) + log2 w_i)
+template <int D>
+__device__ __forceinline__ void finish_pot(const PassParams& P, int64_t i, double lse2) {
+  const double xn = row_sqnorm<D>(P.qkeys, i);
+  P.pot_out[i] = static_cast<float>(xn - lse2 * P.eps_ln2);
+  P.qkeys[key_slot<D>(i, D)] = static_cast<float>(static_cast<double>(P.lw[i]) - lse2);
+}
+
+// kMarg: plan marginal r_i = w_i 2^(kappa (pot_i - |x_i|^2) + LSE2_i) = w_i exp((pot_i - F_i)/eps).
+template <int D>
+__device__ __forceinline__ void finish_marg(const PassParams& P, int64_t i, double lse2,
+                                            double& dev, double& mass) {
+  const double w = P.w ? static_cast<double>(P.w[i]) : static_cast<double>(P.w_uniform);
+  double r = 0.0;
+  if (w > 0.0) {
+    const double xn = row_sqnorm<D>(P.qkeys, i);
+    r = w * exp2(P.kappa * (static_cast<double>(P.pot_in[i]) - xn) + lse2);
+  }
+  if (P.marg_out) P.marg_out[i] = static_cast<float>(r);
+  dev = fabs(r - w);
+  mass = r;
+}
+
+// kGrad: grad_i = 2 w_i (x_i - T_i), T_i = sum_j p_ij y_j / sum_j p_ij (centred coordinates).
+template <int D>
+__device__ __forceinline__ void finish_grad(const PassParams& P, int64_t i, const float* acc,
+                                            float l) {
+  const float w = P.w ? P.w[i] : P.w_uniform;
+  const float inv = 1.0f / l;
+  for (int k = 0; k < P.d_real; ++k) {
+    const float c = P.qkeys[key_slot<D>(i, k)];
+    P.grad_out[i * P.d_real + k] = 2.0f * w * (c - acc[k] * inv);
+  }
+}
+
+// Block-wide sum/max of the marginal deviations, then one atomic per block.
+__device__ __forceinline__ void block_reduce_marg(double dev_sum, double dev_max, double mass,
+                                                  double* acc) {
+  __shared__ double sh[3][32];
+  dev_sum = warp_sum(dev_sum);
+  dev_max = warp_max(dev_max);
+  mass = warp_sum(mass);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (lane == 0) {
+    sh[0][wid] = dev_sum;
+    sh[1][wid] = dev_max;
+    sh[2][wid] = mass;
+  }
+  __syncthreads();
+  if (wid == 0) {
+    const int nw = (blockDim.x + 31) >> 5;
+    double s = lane < nw ? sh[0][lane] : 0.0;
+    double mx = lane < nw ? sh[1][lane] : 0.0;
+    double ms = lane < nw ? sh[2][lane] : 0.0;
+    s = warp_sum(s);
+    mx = warp_max(mx);
+    ms = warp_sum(ms);
+    if (lane == 0) {
+      atomicAdd(&acc[0], s);
+      atomic_max_nonneg(&acc[1], mx);
+      atomicAdd(&acc[2], ms);
+    }
+  }
+}
+
+// ---- the fused streaming pass -------------------------------------------------------------
+
+template <int D, int R, int NT, int G, bool GRAD, int MINB>
+__global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) {
+  constexpr int KP = key_pair_floats(D);
+  constexpr int NV = KP / 4;
+  constexpr int NA = GRAD ? D : 1;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  __shared__ uint64_t bars[kStages];
+
+  float* stages = reinterpret_cast<float*>(smem_raw);
+  const int tid = threadIdx.x;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (NT * R);
+  const int split = blockIdx.y;
+  const int64_t p_begin = static_cast<int64_t>(split) * P.pairs_per_split;
+  int64_t p_end = p_begin + P.pairs_per_split;
+  if (p_end > P.key_pairs) p_end = P.key_pairs;
+  const int n_tiles = static_cast<int>((p_end - p_begin) / P.tile_pairs);
+  const uint32_t stage_floats = static_cast<uint32_t>(P.tile_pairs) * KP;
+  const uint32_t stage_bytes = stage_floats * 4u;
+  const float* key_src = P.keys + p_begin * KP;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int s = 0; s < kStages && s < n_tiles; ++s) {
+      mbar_expect_tx(&bars[s], stage_bytes);
+      bulk_g2s(stages + s * stage_floats, key_src + static_cast<int64_t>(s) * stage_floats,
+               stage_bytes, &bars[s]);
+    }
+  }
+
+  // Query rows: 2 kappa x_i, duplicated into both lanes of a packed register.
+  u64 Q[R][D];
+  float m[R];
+  u64 L[R];
+  u64 A[R][NA];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int64_t i = row0 + r * NT + tid;
+#pragma unroll
+    for (int k = 0; k < D; ++k) {
+      const float c = (i < P.n_rows) ? P.qkeys[key_slot<D>(i, k)] : 0.0f;
+      const float q = P.two_kappa * c;
+      Q[r][k] = pk(q, q);
+    }
+    m[r] = -INFINITY;
+    L[r] = pk(0.0f, 0.0f);
+#pragma unroll
+    for (int k = 0; k < NA; ++k) A[r][k] = pk(0.0f, 0.0f);
+  }
+
+  int t = 0;
+  bool aborted = false;
+  for (; t < n_tiles; ++t) {
+    const int st = t % kStages;
+    const uint32_t parity = static_cast<uint32_t>(t / kStages) & 1u;
+    const bool ok = mbar_wait_bounded(&bars[st], parity);
+    if (__syncthreads_or(!ok)) {
+      aborted = true;
+      break;
+    }
+    const float* tile = stages + st * stage_floats;
+    for (int pg = 0; pg < P.tile_pairs; pg += G) {
+      u64 s[R][G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const ulonglong2* pv = reinterpret_cast<const ulonglong2*>(tile + (pg + g) * KP);
+        u64 comp[2 * NV];
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          const ulonglong2 q = pv[v];
+          comp[2 * v] = q.x;
+          comp[2 * v + 1] = q.y;
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          u64 acc = comp[D];
+#pragma unroll
+          for (int k = 0; k < D; ++k) acc = fma2(Q[r][k], comp[k], acc);
+          s[r][g] = acc;
+        }
+      }
+      // Row max over the group; lazy rescale of the running sums.
+      u64 negm[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        float a0, a1;
+        upk(s[r][0], a0, a1);
+        float mx = fmaxf(a0, a1);
+#pragma unroll
+        for (int g = 1; g < G; ++g) {
+          upk(s[r][g], a0, a1);
+          mx = max3(mx, a0, a1);
+        }
+        if (mx > m[r] + kLazyThr) {
+          const float sc = ex2(m[r] - mx);
+          const u64 sc2 = pk(sc, sc);
+          L[r] = mul2(L[r], sc2);
+          if (GRAD) {
+#pragma unroll
+            for (int k = 0; k < NA; ++k) A[r][k] = mul2(A[r][k], sc2);
+          }
+          m[r] = mx;
+        }
+        negm[r] = pk(-m[r], -m[r]);
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        u64 comp[2 * NV];
+        if (GRAD) {
+          const ulonglong2* pv = reinterpret_cast<const ulonglong2*>(tile + (pg + g) * KP);
+#pragma unroll
+          for (int v = 0; v < NV; ++v) {
+            const ulonglong2 q = pv[v];
+            comp[2 * v] = q.x;
+            comp[2 * v + 1] = q.y;
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          float t0, t1;
+          upk(add2(s[r][g], negm[r]), t0, t1);
+          const u64 e = pk(ex2(t0), ex2(t1));
+          L[r] = add2(L[r], e);
+          if (GRAD) {
+#pragma unroll
+            for (int k = 0; k < NA; ++k) A[r][k] = fma2(e, comp[k], A[r][k]);
+          }
+        }
+      }
+    }
+    __syncthreads();
+    if (tid == 0 && t + kStages < n_tiles) {
+      fence_proxy_async_smem();
+      mbar_expect_tx(&bars[st], stage_bytes);
+      bulk_g2s(stages + st * stage_floats,
+               key_src + static_cast<int64_t>(t + kStages) * stage_floats, stage_bytes,
+               &bars[st]);
+    }
+  }
+
+  if (aborted) {
+    // Record the timeout, let this CTA's own copies still in flight land (bounded), leave.
+    if (tid == 0) {
+      atomicOr(P.err, kErrTimeout);
+      for (int u = t; u < n_tiles && u < t + kStages; ++u)
+        (void)mbar_wait_bounded(&bars[u % kStages], static_cast<uint32_t>(u / kStages) & 1u);
+    }
+    return;
+  }
+
+  if (P.n_splits == 1) {
+    double dev_sum = 0.0, dev_max = 0.0, mass = 0.0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t i = row0 + r * NT + tid;
+      if (i >= P.n_rows) continue;
+      float l0, l1;
+      upk(L[r], l0, l1);
+      const float l = l0 + l1;
+      if (GRAD) {
+        float a[NA];
+#pragma unroll
+        for (int k = 0; k < NA; ++k) {
+          float a0, a1;
+          upk(A[r][k], a0, a1);
+          a[k] = a0 + a1;
+        }
+        finish_grad<D>(P, i, a, l);
+      } else {
+        const double lse2 = static_cast<double>(m[r]) + log2(static_cast<double>(l));
+        if (P.kind == kPot) {
+          finish_pot<D>(P, i, lse2);
+        } else {
+          double dv, ms;
+          finish_marg<D>(P, i, lse2, dv, ms);
+          dev_sum += dv;
+          dev_max = fmax(dev_max, dv);
+          mass += ms;
+        }
+      }
+    }
+    if (!GRAD && P.kind == kMarg) block_reduce_marg(dev_sum, dev_max, mass, P.acc);
+  } else {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t i = row0 + r * NT + tid;
+      if (i >= P.n_rows) continue;
+      float l0, l1;
+      upk(L[r], l0, l1);
+      const int64_t o = static_cast<int64_t>(split) * P.rows_pad + i;
+      P.part_m[o] = m[r];
+      P.part_l[o] = l0 + l1;
+      if (GRAD) {
+#pragma unroll
+        for (int k = 0; k < NA; ++k) {
+          float a0, a1;
+          upk(A[r][k], a0, a1);
+          P.part_a[(static_cast<int64_t>(split) * D + k) * P.rows_pad + i] = a0 + a1;
+        }
+      }
+    }
+  }
+}
+
+// Second-level LSE over the split partials of each row, then the row completion.
+template <int D, bool GRAD>
+__global__ void __launch_bounds__(256) combine_kernel(const PassParams P) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  double dev = 0.0, mass = 0.0;
+  if (i < P.n_rows) {
+    float mx = -INFINITY;
+    for (int s = 0; s < P.n_splits; ++s) mx = fmaxf(mx, P.part_m[s * P.rows_pad + i]);
+    double l = 0.0;
+    float a[GRAD ? D : 1];
+    if (GRAD) {
+      for (int k = 0; k < D; ++k) a[k] = 0.0f;
+    }
+    for (int s = 0; s < P.n_splits; ++s) {
+      const int64_t o = s * P.rows_pad + i;
+      const float w = ex2(P.part_m[o] - mx);
+      l += static_cast<double>(P.part_l[o]) * w;
+      if (GRAD) {
+        for (int k = 0; k < D; ++k) a[k] += P.part_a[(static_cast<int64_t>(s) * D + k) * P.rows_pad + i] * w;
+      }
+    }
+    if (GRAD) {
+      finish_grad<D>(P, i, a, static_cast<float>(l));
+    } else {
+      const double lse2 = static_cast<double>(mx) + log2(l);
+      if (P.kind == kPot) {
+        finish_pot<D>(P, i, lse2);
+      } else {
+        finish_marg<D>(P, i, lse2, dev, mass);
+      }
+    }
+  }
+  if (!GRAD && P.kind == kMarg) block_reduce_marg(dev, dev, mass, P.acc);
+}
+
+// ---- preparation kernels --------------------------------------------------------------
+
+struct Center {
+  double c[64];
+};
+
+// Coordinate sums (float64) per dimension, and a flag for non-finite coordinates.
+__global__ void __launch_bounds__(256) reduce_coords_kernel(const float* pts, int64_t count,
+                                                            int32_t d, double* sums,
+                                                            unsigned* flags) {
+  const int k = blockIdx.y;
+  double s = 0.0;
+  int bad = 0;
+  for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < count;
+       j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float v = pts[j * d + k];
+    bad |= !isfinite(v);
+    s += v;
+  }
+  s = warp_sum(s);
+  bad = warp_or(bad);
+  if ((threadIdx.x & 31) == 0) {
+    atomicAdd(&sums[k], s);
+    if (bad) atomicOr(flags, 1u);
+  }
+}
+
+// Weight sum (float64); flags bit 2 for a negative or non-finite weight.
+__global__ void __launch_bounds__(256) reduce_weights_kernel(const float* w, int64_t count,
+                                                             double* sum, unsigned* flags) {
+  double s = 0.0;
+  int bad = 0;
+  for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < count;
+       j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float v = w[j];
+    bad |= !(v >= 0.0f) || isinf(v);
+    s += v;
+  }
+  s = warp_sum(s);
+  bad = warp_or(bad);
+  if ((threadIdx.x & 31) == 0) {
+    atomicAdd(sum, s);
+    if (bad) atomicOr(flags, 2u);
+  }
+}
+
+// Flags bit 4 for a non-finite entry of a given potential.
+__global__ void __launch_bounds__(256) check_finite_kernel(const float* v, int64_t count,
+                                                           unsigned* flags) {
+  int bad = 0;
+  for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < count;
+       j += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    bad |= !isfinite(v[j]);
+  bad = warp_or(bad);
+  if ((threadIdx.x & 31) == 0 && bad) atomicOr(flags, 4u);
+}
+
+// Packed keys (centred coordinates, bias slot left to key_bias_kernel) and log2 weights
+// for all padded points of one cloud.
+template <int D>
+__global__ void __launch_bounds__(256) pack_kernel(const float* pts, int64_t count, int32_t d_real,
+                                                   const Center ctr, const float* w,
+                                                   float w_uniform, float* keys, float* lw,
+                                                   int64_t pairs_pad) {
+  constexpr int KP = key_pair_floats(D);
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j >= 2 * pairs_pad) return;
+  const int64_t base = (j >> 1) * KP + (j & 1);
+  if (j < count) {
+#pragma unroll
+    for (int k = 0; k < D; ++k)
+      keys[base + 2 * k] =
+          k < d_real ? static_cast<float>(static_cast<double>(pts[j * d_real + k]) - ctr.c[k]) : 0.0f;
+    const float wj = w ? w[j] : w_uniform;
+    lw[j] = wj > 0.0f ? static_cast<float>(log2(static_cast<double>(wj))) : kLogZero;
+  } else {
+#pragma unroll
+    for (int k = 0; k < D; ++k) keys[base + 2 * k] = 0.0f;
+    keys[base + 2 * D] = kLogZero;
+    lw[j] = kLogZero;
+  }
+  // zero the padding floats after the bias slot
+#pragma unroll
+  for (int k = 2 * D + 2; k < KP; k += 2) keys[base + k] = 0.0f;
+}
+
+// Key bias of every real point: h_j = kappa (pot_j - |c_j|^2) + log2 w_j (pot = 0 if NULL).
+template <int D>
+__global__ void __launch_bounds__(256) key_bias_kernel(float* keys, int64_t count, const float* pot,
+                                                       const float* lw, double kappa) {
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j >= count) return;
+  const double cn = row_sqnorm<D>(keys, j);
+  const double p = pot ? static_cast<double>(pot[j]) : 0.0;
+  keys[key_slot<D>(j, D)] = static_cast<float>(kappa * (p - cn) + static_cast<double>(lw[j]));
+}
+
+// <v, w> in float64 (w NULL = uniform weight wu).
+__global__ void __launch_bounds__(256) dot_kernel(const float* v, const float* w, float wu,
+                                                  int64_t count, double* out) {
+  double s = 0.0;
+  for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < count;
+       j += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    s += static_cast<double>(v[j]) * static_cast<double>(w ? w[j] : wu);
+  s = warp_sum(s);
+  if ((threadIdx.x & 31) == 0) atomicAdd(out, s);
+}
+
+// cost = <f,a> + <g,b> - eps * (plan mass - m_a m_b)
+__global__ void cost_finish_kernel(const double* fa, const double* gb, const double* mass,
+                                   double eps, double mamb, double* out) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) out[0] = fa[0] + gb[0] - eps * (mass[0] - mamb);
+}
+
+__global__ void residual_finish_kernel(const double* row_acc, const double* col_acc, double* out) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) {
+    out[0] = row_acc[0];
+    out[1] = row_acc[1];
+    out[2] = col_acc[0];
+    out[3] = col_acc[1];
+  }
+}
+
+}  // namespace fs
