@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="c5", choices=sorted(CONFIG_INDEX))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--n", type=int, default=None,
+                    help="clustered workload only: use n = m points (eps by the same spacing rule)")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -55,9 +57,14 @@ def parse():
     return ap.parse_args()
 
 
-def workload(cfg: str, rank: int):
+def workload(cfg: str, rank: int, n_override=None):
     from streaming_sinkhorn_b200 import workloads
     import dataclasses
+    if n_override is not None:
+        if cfg != "c5":
+            raise SystemExit("--n applies to the clustered workload (c5) only")
+        w = workloads.clustered_cube(n=n_override, seed=4 + 1000 * rank, n_iters=20)
+        return dataclasses.replace(w, name=f"clustered_cube_n{n_override}")
     w = workloads.config(CONFIG_INDEX[cfg])
     if rank:
         # an independently seeded replica of the same recipe
@@ -209,7 +216,7 @@ def run_native(args, rank, world, local_rank):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local_rank))
-    w = workload(args.config, rank)
+    w = workload(args.config, rank, args.n)
     dev = torch.device("cuda", local_rank)
     x = torch.from_numpy(w.x).to(dev)
     y = torch.from_numpy(w.y).to(dev)
@@ -361,7 +368,7 @@ def run_e2e(args, w, dev, world, dist):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    w = workload(args.config, 0)
+    w = workload(args.config, 0, args.n)
     per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample(w, min(per_step, 3.0))

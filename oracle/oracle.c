@@ -41,6 +41,9 @@
 #include <omp.h>
 #endif
 
+/* Below this many pair terms a call runs on one thread: a parallel region costs more. */
+#define ORC_PARALLEL_MIN_WORK 2000000LL
+
 #define ORC_OK 0
 #define ORC_ERR_ARG (-1)
 #define ORC_ERR_MASS (-2)
@@ -85,7 +88,7 @@ int oracle_lse_update(const double* P, int64_t np, const double* Q, int64_t nq, 
   if (!P || !Q || !wq || !pot_q || !out || np < 1 || nq < 1 || d < 1 || !(eps > 0.0))
     return ORC_ERR_ARG;
   int bad = 0;
-#pragma omp parallel
+#pragma omp parallel if (n_rows * nq * d > ORC_PARALLEL_MIN_WORK)
   {
     double* z = (double*)malloc(sizeof(double) * (size_t)nq);
     if (!z) {
@@ -166,7 +169,7 @@ int oracle_plan_row_sums(const double* x, int64_t n, const double* y, int64_t m,
                          const double* g, const int64_t* rows, int64_t n_rows, double* out) {
   if (!x || !y || !a || !b || !f || !g || !out || n < 1 || m < 1 || d < 1 || !(eps > 0.0))
     return ORC_ERR_ARG;
-#pragma omp parallel for schedule(dynamic, 16)
+#pragma omp parallel for schedule(dynamic, 16) if (n_rows * m * d > ORC_PARALLEL_MIN_WORK)
   for (int64_t k = 0; k < n_rows; ++k) {
     int64_t i = rows ? rows[k] : k;
     double s = 0.0;
@@ -224,7 +227,7 @@ int oracle_grad_x(const double* x, int64_t n, const double* y, int64_t m, int32_
     return rc;
   }
   int bad = 0;
-#pragma omp parallel
+#pragma omp parallel if (n_rows * m * d > ORC_PARALLEL_MIN_WORK)
   {
     double* acc = (double*)malloc(sizeof(double) * (size_t)d);
     if (!acc) {

@@ -3,6 +3,10 @@ import sys
 
 import pytest
 
+# The oracle's OpenMP threads sleep instead of spinning while idle, so many small oracle
+# calls stay fast when the host's cores are busy.
+os.environ.setdefault("OMP_WAIT_POLICY", "PASSIVE")
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
