@@ -112,7 +112,7 @@ struct Variant {
 // LSE passes for D <= 16, from most to least rows per CTA.
 constexpr Variant kLseVariants[3] = {{4, 256}, {2, 128}, {1, 128}};
 // Gradient passes for D <= 16.
-constexpr Variant kGradVariants[2] = {{2, 256}, {1, 128}};
+constexpr Variant kGradVariants[2] = {{2, 128}, {1, 128}};
 // Everything for D > 16.
 constexpr Variant kWideVariant = {1, 128};
 
@@ -185,8 +185,6 @@ constexpr size_t kAlign = 256;
 constexpr int kScalarDoubles = 256;  // 2 KiB of float64 scalars
 
 // Offsets (in doubles) inside the scalar block.
-constexpr int kSumX = 0;      // [64]
-constexpr int kSumY = 64;     // [64]
 constexpr int kSumA = 128;
 constexpr int kSumB = 129;
 constexpr int kAccRow = 130;  // [3]
@@ -248,7 +246,7 @@ inline bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr)
 template <int D, int R, int NT, bool GRAD>
 void launch_pass_t(const PassParams& P, const Plan& pl, cudaStream_t st) {
   constexpr int G = (D > 16) ? 4 : 8;
-  constexpr int MINB = (D > 16) ? 1 : (NT == 256 ? 2 : 4);
+  constexpr int MINB = (D > 16) ? 1 : (GRAD ? 3 : (NT == 256 ? 2 : 4));
   auto kern = lse_pass_kernel<D, R, NT, G, GRAD, MINB>;
   const size_t smem = static_cast<size_t>(kStages) * pl.tile_pairs * key_pair_floats(D) * 4;
   static bool attr_set = false;  // per instantiation; idempotent, so a race is harmless
@@ -273,7 +271,7 @@ void launch_pass_d(const PassParams& P, const Plan& pl, bool grad, cudaStream_t 
   } else {
     if (grad) {
       if (pl.variant == 0)
-        launch_pass_t<D, 2, 256, true>(P, pl, st);
+        launch_pass_t<D, 2, 128, true>(P, pl, st);
       else
         launch_pass_t<D, 1, 128, true>(P, pl, st);
     } else {
@@ -311,10 +309,10 @@ void launch_combine_d(const PassParams& P, bool grad, cudaStream_t st) {
   }
 
 template <int D>
-void launch_pack_d(const float* pts, int64_t count, int d, const Center& c, const float* w,
-                   float wu, float* keys, float* lw, int64_t pp, cudaStream_t st) {
+void launch_pack_d(const float* pts, int64_t count, int d, const float* w, float wu, float* keys,
+                   float* lw, int64_t pp, cudaStream_t st) {
   const unsigned blocks = static_cast<unsigned>(ceil_div(2 * pp, 256));
-  pack_kernel<D><<<blocks, 256, 0, st>>>(pts, count, d, c, w, wu, keys, lw, pp);
+  pack_kernel<D><<<blocks, 256, 0, st>>>(pts, count, d, w, wu, keys, lw, pp);
   CK(cudaGetLastError());
   g_launches.fetch_add(1, std::memory_order_relaxed);
 }
@@ -385,11 +383,12 @@ unsigned reduce_blocks(int64_t count, int sms) {
 fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& pots) {
   const fs_problem* p = c.p;
   CK(cudaMemsetAsync(c.scal, 0, kScalarDoubles * sizeof(double), c.st));
-  dim3 gx(reduce_blocks(p->n, c.sms), p->d), gy(reduce_blocks(p->m, c.sms), p->d);
-  reduce_coords_kernel<<<gx, 256, 0, c.st>>>(p->x, p->n, p->d, c.scal + kSumX, flags_ptr(c.scal));
+  check_coords_kernel<<<reduce_blocks(p->n * p->d, c.sms), 256, 0, c.st>>>(p->x, p->n * p->d,
+                                                                           flags_ptr(c.scal));
   CK(cudaGetLastError());
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  reduce_coords_kernel<<<gy, 256, 0, c.st>>>(p->y, p->m, p->d, c.scal + kSumY, flags_ptr(c.scal));
+  check_coords_kernel<<<reduce_blocks(p->m * p->d, c.sms), 256, 0, c.st>>>(p->y, p->m * p->d,
+                                                                           flags_ptr(c.scal));
   CK(cudaGetLastError());
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (p->a) {
@@ -422,12 +421,9 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
   if (!(c.ma > 0.0) || !(c.mb > 0.0)) return FS_ERR_ZERO_MASS;
   if (std::fabs(c.ma - c.mb) > 1e-5 * std::max(c.ma, c.mb)) return FS_ERR_MASS_MISMATCH;
 
-  Center ctr{};
-  for (int k = 0; k < p->d; ++k)
-    ctr.c[k] = (host[kSumX + k] + host[kSumY + k]) / static_cast<double>(p->n + p->m);
   const float wu_x = static_cast<float>(1.0 / p->n), wu_y = static_cast<float>(1.0 / p->m);
-  FS_DISPATCH_D(c.L.D, launch_pack_d, p->x, p->n, p->d, ctr, p->a, wu_x, c.kx, c.lwx, c.L.px, c.st);
-  FS_DISPATCH_D(c.L.D, launch_pack_d, p->y, p->m, p->d, ctr, p->b, wu_y, c.ky, c.lwy, c.L.py, c.st);
+  FS_DISPATCH_D(c.L.D, launch_pack_d, p->x, p->n, p->d, p->a, wu_x, c.kx, c.lwx, c.L.px, c.st);
+  FS_DISPATCH_D(c.L.D, launch_pack_d, p->y, p->m, p->d, p->b, wu_y, c.ky, c.lwy, c.L.py, c.st);
   return FS_OK;
 }
 
@@ -459,7 +455,8 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
   P.kind = kind;
   P.d_real = p->d;
   P.kappa = c.kappa;
-  P.two_kappa = static_cast<float>(2.0 * c.kappa);
+  P.kappa_f = static_cast<float>(c.kappa);
+  P.inv_kappa_f = static_cast<float>(1.0 / c.kappa);
   P.eps_ln2 = 1.0 / c.kappa;
   P.lw = rows_x ? c.lwx : c.lwy;
   P.w = rows_x ? p->a : p->b;

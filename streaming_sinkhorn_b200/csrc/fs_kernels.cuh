@@ -1,32 +1,34 @@
 // fs_kernels.cuh -- CUDA kernels of the streaming log-domain Sinkhorn passes (sm_100a).
 //
 // One pass evaluates, for every query row i, the base-2 log-sum-exp over all key
-// columns j of the biased dot-product score
-//     s_ij = (2 kappa x_i) . y_j + h_j,      kappa = log2(e) / eps,
-//     h_j  = kappa (g_j - |y_j|^2) + log2 b_j,
-// which is the FlashSinkhorn attention-form of the log-domain update (FlashSinkhorn
-// summary, Methodology section 1: the cost |x|^2 + |y|^2 - 2 x.y splits into a dot
-// product plus per-column and per-row biases). Then
-//     F(g)_i = |x_i|^2 - LSE2_j(s_ij) / kappa.
-// The same pass with the roles of the clouds swapped is the g-update.
+// columns j of
+//     z_ij = H_j - kappa |x_i - y_j|^2,   kappa = log2(e) / eps,   H_j = kappa g_j + log2 b_j,
+// so that the f-update of the log-domain iteration (FlashSinkhorn summary, Methodology
+// section 1) is F(g)_i = -LSE2_j(z_ij) / kappa. The same pass with the roles of the clouds
+// swapped is the g-update. The squared distance is taken as a direct difference of the
+// float32 input coordinates: its rounding error is relative to the local distances and
+// potentials, where the expanded |x|^2 + |y|^2 - 2 x.y form loses precision in proportion to
+// the squared distance from the origin (which over a few hundred slowly mixing iterations
+// moves outlying potentials by more than 1e-4).
 //
 // Layout in HBM. Each cloud is stored once as "packed keys": point pairs (2p, 2p+1)
-// share KP floats laid out as [c0 c0' c1 c1' ... c_{D-1} c_{D-1}' h h' pad], i.e. every
-// coordinate (and the bias h) of the two points sits side by side so that one 64-bit
-// register holds the same component of two columns, ready for the packed fp32x2 FMA.
-// Coordinates are centred on the common mean of both clouds (the cost is translation
-// invariant); the pair count is padded to a multiple of 128 with zero coordinates and
-// h = kLogZero, which contribute nothing.
+// share KP floats laid out as [c0 c0' c1 c1' ... c_{D-1} c_{D-1}' H H' pad], i.e. every
+// coordinate (and the bias H) of the two points sits side by side so that one 64-bit
+// register holds the same component of two columns, ready for the packed fp32x2 ops.
+// The pair count is padded to a multiple of 128 with zero coordinates and H = kLogZero,
+// which contribute nothing.
 //
 // A CTA owns NT*R query rows (R rows per thread, kept in registers) and streams one
 // contiguous range of key pairs through shared memory with TMA bulk copies
 // (kStages-deep ring, mbarrier completion). Each thread runs an online max/sum over its
-// rows: per group of G key pairs the row max is taken first; the running sum is
-// rescaled only when that max exceeds the running offset by more than kLazyThr (terms
-// then stay below 2^kLazyThr), so the per-pair work is d packed FMAs, one packed add,
-// one MUFU ex2 per column and a packed accumulate. When the key range is split over
-// several CTAs, each writes its (max, sum[, weighted coordinates]) partial and a combine
-// kernel merges them with a second-level LSE.
+// rows. The running offset m_i is folded into the distance accumulator,
+//     t_ij = H_j - kappa (m_i / kappa + sum_k (x_ik - y_jk)^2) = z_ij - m_i,
+// so a column pair costs d packed subtracts, d + 1 packed FMAs, two MUFU ex2 and one packed
+// accumulate. Per group of G key pairs the row max of t is taken first and the running sum
+// is rescaled only when it exceeds the offset by more than kLazyThr (terms then stay below
+// 2^kLazyThr). When the key range is split over several CTAs, each writes its
+// (max, sum[, weighted differences]) partial and a combine kernel merges them with a
+// second-level LSE.
 #pragma once
 
 #include <cfloat>
@@ -41,12 +43,15 @@ __host__ __device__ constexpr int key_pair_floats(int D) { return ((2 * (D + 1) 
 constexpr int kStages = 3;
 constexpr float kLazyThr = 8.0f;
 constexpr int kPairPad = 128;  // key pairs are padded to a multiple of this
+// A group whose largest exponent is below this holds only zero-weight or padding
+// columns; it never sets the running offset.
+constexpr float kEmptyCut = -1.0e29f;
 
 enum PassKind : int { kPot = 0, kMarg = 1, kGrad = 2 };
 
 struct PassParams {
   const float* keys;        // streamed cloud, packed
-  float* qkeys;             // query cloud, packed (coordinates read; h written by kPot)
+  float* qkeys;             // query cloud, packed (coordinates read; H written by kPot)
   int64_t n_rows;           // real number of query rows
   int64_t key_pairs;        // padded key pair count
   int64_t pairs_per_split;  // key pairs per split (multiple of tile_pairs)
@@ -55,7 +60,8 @@ struct PassParams {
   int64_t rows_pad;         // row stride of the partial arrays
   int32_t kind;             // PassKind
   int32_t d_real;           // true dimension (<= D)
-  float two_kappa;          // 2 log2(e) / eps
+  float kappa_f;            // log2(e) / eps
+  float inv_kappa_f;        // eps ln 2
   double kappa;             // log2(e) / eps
   double eps_ln2;           // eps ln 2 = 1 / kappa
   const float* lw;          // log2 weights of the query cloud (kLogZero for zeros)
@@ -66,13 +72,13 @@ struct PassParams {
   float* marg_out;          // kMarg: plan marginal per row, or NULL
   float* grad_out;          // kGrad: (n_rows, d_real)
   double* acc;              // kMarg: [sum |r - w|, max |r - w|, sum r]
-  float* part_m;            // partial maxima   [split][rows_pad]
-  float* part_l;            // partial sums     [split][rows_pad]
-  float* part_a;            // partial weighted coordinates [split][D][rows_pad]
+  float* part_m;            // partial offsets [split][rows_pad]
+  float* part_l;            // partial sums    [split][rows_pad]
+  float* part_a;            // partial weighted differences [split][D][rows_pad]
   unsigned* err;            // error word
 };
 
-// Offset of coordinate slot k (k == D is the bias h) of point i in packed keys.
+// Offset of coordinate slot k (k == D is the bias H) of point i in packed keys.
 template <int D>
 __device__ __forceinline__ int64_t key_slot(int64_t i, int k) {
   return (i >> 1) * key_pair_floats(D) + 2 * k + (i & 1);
@@ -80,51 +86,31 @@ __device__ __forceinline__ int64_t key_slot(int64_t i, int k) {
 
 // ---- per-row completion, shared by the direct epilogue and the combine kernel -----------
 
-template <int D>
-__device__ __forceinline__ double row_sqnorm(const float* qkeys, int64_t i) {
-  double s = 0.0;
-#pragma unroll
-  for (int k = 0; k < D; ++k) {
-    const double c = qkeys[key_slot<D>(i, k)];
-    s += c * c;
-  }
-  return s;
-}
-
-// kPot: write the new potential and the key bias this row carries into the next pass.
-//   pot_i = |x_i|^2 - LSE2_i / kappa,   h_i = log2 w_i - LSE2_i  (= kappa (pot_i - |x_i|^2) + log2 w_i)
+// kPot: the new potential and the bias this row carries as a key into the next pass:
+//   pot_i = -LSE2_i / kappa,   H_i = kappa pot_i + log2 w_i = log2 w_i - LSE2_i.
 template <int D>
 __device__ __forceinline__ void finish_pot(const PassParams& P, int64_t i, double lse2) {
-  const double xn = row_sqnorm<D>(P.qkeys, i);
-  P.pot_out[i] = static_cast<float>(xn - lse2 * P.eps_ln2);
+  P.pot_out[i] = static_cast<float>(-lse2 * P.eps_ln2);
   P.qkeys[key_slot<D>(i, D)] = static_cast<float>(static_cast<double>(P.lw[i]) - lse2);
 }
 
-// kMarg: plan marginal r_i = w_i 2^(kappa (pot_i - |x_i|^2) + LSE2_i) = w_i exp((pot_i - F_i)/eps).
-template <int D>
+// kMarg: plan marginal r_i = w_i 2^(kappa pot_i + LSE2_i) = w_i exp((pot_i - F_i)/eps).
 __device__ __forceinline__ void finish_marg(const PassParams& P, int64_t i, double lse2,
                                             double& dev, double& mass) {
   const double w = P.w ? static_cast<double>(P.w[i]) : static_cast<double>(P.w_uniform);
   double r = 0.0;
-  if (w > 0.0) {
-    const double xn = row_sqnorm<D>(P.qkeys, i);
-    r = w * exp2(P.kappa * (static_cast<double>(P.pot_in[i]) - xn) + lse2);
-  }
+  if (w > 0.0) r = w * exp2(P.kappa * static_cast<double>(P.pot_in[i]) + lse2);
   if (P.marg_out) P.marg_out[i] = static_cast<float>(r);
   dev = fabs(r - w);
   mass = r;
 }
 
-// kGrad: grad_i = 2 w_i (x_i - T_i), T_i = sum_j p_ij y_j / sum_j p_ij (centred coordinates).
-template <int D>
-__device__ __forceinline__ void finish_grad(const PassParams& P, int64_t i, const float* acc,
+// kGrad: grad_i = 2 w_i (x_i - T_i) = 2 w_i sum_j p_ij (x_i - y_j) / sum_j p_ij.
+__device__ __forceinline__ void finish_grad(const PassParams& P, int64_t i, const float* dsum,
                                             float l) {
   const float w = P.w ? P.w[i] : P.w_uniform;
-  const float inv = 1.0f / l;
-  for (int k = 0; k < P.d_real; ++k) {
-    const float c = P.qkeys[key_slot<D>(i, k)];
-    P.grad_out[i * P.d_real + k] = 2.0f * w * (c - acc[k] * inv);
-  }
+  const float s = 2.0f * w / l;
+  for (int k = 0; k < P.d_real; ++k) P.grad_out[i * P.d_real + k] = s * dsum[k];
 }
 
 // Block-wide sum/max of the marginal deviations, then one atomic per block.
@@ -159,10 +145,22 @@ __device__ __forceinline__ void block_reduce_marg(double dev_sum, double dev_max
 
 // ---- the fused streaming pass -------------------------------------------------------------
 
+// Loads the packed components of key pair p of a shared-memory tile.
+template <int D>
+__device__ __forceinline__ void load_pair(const float* tile, int p, u64 (&comp)[key_pair_floats(D) / 2]) {
+  constexpr int NV = key_pair_floats(D) / 4;
+  const ulonglong2* pv = reinterpret_cast<const ulonglong2*>(tile + p * key_pair_floats(D));
+#pragma unroll
+  for (int v = 0; v < NV; ++v) {
+    const ulonglong2 q = pv[v];
+    comp[2 * v] = q.x;
+    comp[2 * v + 1] = q.y;
+  }
+}
+
 template <int D, int R, int NT, int G, bool GRAD, int MINB>
 __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) {
   constexpr int KP = key_pair_floats(D);
-  constexpr int NV = KP / 4;
   constexpr int NA = GRAD ? D : 1;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ uint64_t bars[kStages];
@@ -192,21 +190,26 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     }
   }
 
-  // Query rows: 2 kappa x_i, duplicated into both lanes of a packed register.
-  u64 Q[R][D];
-  float m[R];
-  u64 L[R];
+  // Row state: coordinates duplicated into both lanes of a packed register; the running
+  // offset m (log2 units), `base` (m, or 0 while no column has set it) and mk = base/kappa
+  // folded into the distance accumulator; the running sums L (two lanes: even and odd
+  // columns) and, for the gradient, the weighted differences A = sum p (x - y).
+  u64 X[R][D];
+  float m[R], base[R];
+  u64 mk[R], L[R];
   u64 A[R][NA];
+  const u64 nkappa = pk(-P.kappa_f, -P.kappa_f);
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     const int64_t i = row0 + r * NT + tid;
 #pragma unroll
     for (int k = 0; k < D; ++k) {
       const float c = (i < P.n_rows) ? P.qkeys[key_slot<D>(i, k)] : 0.0f;
-      const float q = P.two_kappa * c;
-      Q[r][k] = pk(q, q);
+      X[r][k] = pk(c, c);
     }
     m[r] = -INFINITY;
+    base[r] = 0.0f;
+    mk[r] = pk(0.0f, 0.0f);
     L[r] = pk(0.0f, 0.0f);
 #pragma unroll
     for (int k = 0; k < NA; ++k) A[r][k] = pk(0.0f, 0.0f);
@@ -224,70 +227,64 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     }
     const float* tile = stages + st * stage_floats;
     for (int pg = 0; pg < P.tile_pairs; pg += G) {
-      u64 s[R][G];
+      u64 tv[R][G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const ulonglong2* pv = reinterpret_cast<const ulonglong2*>(tile + (pg + g) * KP);
-        u64 comp[2 * NV];
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-          const ulonglong2 q = pv[v];
-          comp[2 * v] = q.x;
-          comp[2 * v + 1] = q.y;
-        }
+        u64 comp[KP / 2];
+        load_pair<D>(tile, pg + g, comp);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          u64 acc = comp[D];
+          u64 acc = mk[r];
 #pragma unroll
-          for (int k = 0; k < D; ++k) acc = fma2(Q[r][k], comp[k], acc);
-          s[r][g] = acc;
+          for (int k = 0; k < D; ++k) {
+            const u64 dk = sub2(X[r][k], comp[k]);
+            acc = fma2(dk, dk, acc);
+          }
+          tv[r][g] = fma2(nkappa, acc, comp[D]);  // H - kappa (m/kappa + |x - y|^2)
         }
       }
-      // Row max over the group; lazy rescale of the running sums.
-      u64 negm[R];
+      // Group max; lazy rescale of the running sums (always on a row's first real group).
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         float a0, a1;
-        upk(s[r][0], a0, a1);
+        upk(tv[r][0], a0, a1);
         float mx = fmaxf(a0, a1);
 #pragma unroll
         for (int g = 1; g < G; ++g) {
-          upk(s[r][g], a0, a1);
+          upk(tv[r][g], a0, a1);
           mx = max3(mx, a0, a1);
         }
-        if (mx > m[r] + kLazyThr) {
-          const float sc = ex2(m[r] - mx);
+        const float mx_abs = mx + base[r];
+        if (mx_abs > m[r] + kLazyThr && mx > kEmptyCut) {
+          const float sc = ex2(m[r] - mx_abs);
           const u64 sc2 = pk(sc, sc);
           L[r] = mul2(L[r], sc2);
           if (GRAD) {
 #pragma unroll
             for (int k = 0; k < NA; ++k) A[r][k] = mul2(A[r][k], sc2);
           }
-          m[r] = mx;
+          const u64 sh = pk(-mx, -mx);
+#pragma unroll
+          for (int g = 0; g < G; ++g) tv[r][g] = add2(tv[r][g], sh);
+          m[r] = mx_abs;
+          base[r] = mx_abs;
+          const float q = mx_abs * P.inv_kappa_f;
+          mk[r] = pk(q, q);
         }
-        negm[r] = pk(-m[r], -m[r]);
       }
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        u64 comp[2 * NV];
-        if (GRAD) {
-          const ulonglong2* pv = reinterpret_cast<const ulonglong2*>(tile + (pg + g) * KP);
-#pragma unroll
-          for (int v = 0; v < NV; ++v) {
-            const ulonglong2 q = pv[v];
-            comp[2 * v] = q.x;
-            comp[2 * v + 1] = q.y;
-          }
-        }
+        u64 comp[KP / 2];
+        if (GRAD) load_pair<D>(tile, pg + g, comp);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           float t0, t1;
-          upk(add2(s[r][g], negm[r]), t0, t1);
+          upk(tv[r][g], t0, t1);
           const u64 e = pk(ex2(t0), ex2(t1));
           L[r] = add2(L[r], e);
           if (GRAD) {
 #pragma unroll
-            for (int k = 0; k < NA; ++k) A[r][k] = fma2(e, comp[k], A[r][k]);
+            for (int k = 0; k < NA; ++k) A[r][k] = fma2(e, sub2(X[r][k], comp[k]), A[r][k]);
           }
         }
       }
@@ -329,14 +326,14 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
           upk(A[r][k], a0, a1);
           a[k] = a0 + a1;
         }
-        finish_grad<D>(P, i, a, l);
+        finish_grad(P, i, a, l);
       } else {
         const double lse2 = static_cast<double>(m[r]) + log2(static_cast<double>(l));
         if (P.kind == kPot) {
           finish_pot<D>(P, i, lse2);
         } else {
           double dv, ms;
-          finish_marg<D>(P, i, lse2, dv, ms);
+          finish_marg(P, i, lse2, dv, ms);
           dev_sum += dv;
           dev_max = fmax(dev_max, dv);
           mass += ms;
@@ -366,7 +363,8 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
   }
 }
 
-// Second-level LSE over the split partials of each row, then the row completion.
+// Second-level LSE over the split partials of each row, then the row completion. A split
+// whose columns were all zero-weight or padding left m = -inf and sum 0 and drops out.
 template <int D, bool GRAD>
 __global__ void __launch_bounds__(256) combine_kernel(const PassParams P) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -381,20 +379,22 @@ __global__ void __launch_bounds__(256) combine_kernel(const PassParams P) {
     }
     for (int s = 0; s < P.n_splits; ++s) {
       const int64_t o = s * P.rows_pad + i;
-      const float w = ex2(P.part_m[o] - mx);
+      const float pm = P.part_m[o];
+      if (pm == -INFINITY) continue;
+      const float w = ex2(pm - mx);
       l += static_cast<double>(P.part_l[o]) * w;
       if (GRAD) {
         for (int k = 0; k < D; ++k) a[k] += P.part_a[(static_cast<int64_t>(s) * D + k) * P.rows_pad + i] * w;
       }
     }
     if (GRAD) {
-      finish_grad<D>(P, i, a, static_cast<float>(l));
+      finish_grad(P, i, a, static_cast<float>(l));
     } else {
       const double lse2 = static_cast<double>(mx) + log2(l);
       if (P.kind == kPot) {
         finish_pot<D>(P, i, lse2);
       } else {
-        finish_marg<D>(P, i, lse2, dev, mass);
+        finish_marg(P, i, lse2, dev, mass);
       }
     }
   }
@@ -403,29 +403,15 @@ __global__ void __launch_bounds__(256) combine_kernel(const PassParams P) {
 
 // ---- preparation kernels --------------------------------------------------------------
 
-struct Center {
-  double c[64];
-};
-
-// Coordinate sums (float64) per dimension, and a flag for non-finite coordinates.
-__global__ void __launch_bounds__(256) reduce_coords_kernel(const float* pts, int64_t count,
-                                                            int32_t d, double* sums,
-                                                            unsigned* flags) {
-  const int k = blockIdx.y;
-  double s = 0.0;
+// Flags bit 1 for a non-finite coordinate.
+__global__ void __launch_bounds__(256) check_coords_kernel(const float* pts, int64_t count,
+                                                           unsigned* flags) {
   int bad = 0;
   for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < count;
-       j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float v = pts[j * d + k];
-    bad |= !isfinite(v);
-    s += v;
-  }
-  s = warp_sum(s);
+       j += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    bad |= !isfinite(pts[j]);
   bad = warp_or(bad);
-  if ((threadIdx.x & 31) == 0) {
-    atomicAdd(&sums[k], s);
-    if (bad) atomicOr(flags, 1u);
-  }
+  if ((threadIdx.x & 31) == 0 && bad) atomicOr(flags, 1u);
 }
 
 // Weight sum (float64); flags bit 2 for a negative or non-finite weight.
@@ -458,22 +444,19 @@ __global__ void __launch_bounds__(256) check_finite_kernel(const float* v, int64
   if ((threadIdx.x & 31) == 0 && bad) atomicOr(flags, 4u);
 }
 
-// Packed keys (centred coordinates, bias slot left to key_bias_kernel) and log2 weights
-// for all padded points of one cloud.
+// Packed keys (input coordinates, bias slot left to key_bias_kernel) and log2 weights for
+// all padded points of one cloud.
 template <int D>
 __global__ void __launch_bounds__(256) pack_kernel(const float* pts, int64_t count, int32_t d_real,
-                                                   const Center ctr, const float* w,
-                                                   float w_uniform, float* keys, float* lw,
-                                                   int64_t pairs_pad) {
+                                                   const float* w, float w_uniform, float* keys,
+                                                   float* lw, int64_t pairs_pad) {
   constexpr int KP = key_pair_floats(D);
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (j >= 2 * pairs_pad) return;
   const int64_t base = (j >> 1) * KP + (j & 1);
   if (j < count) {
 #pragma unroll
-    for (int k = 0; k < D; ++k)
-      keys[base + 2 * k] =
-          k < d_real ? static_cast<float>(static_cast<double>(pts[j * d_real + k]) - ctr.c[k]) : 0.0f;
+    for (int k = 0; k < D; ++k) keys[base + 2 * k] = k < d_real ? pts[j * d_real + k] : 0.0f;
     const float wj = w ? w[j] : w_uniform;
     lw[j] = wj > 0.0f ? static_cast<float>(log2(static_cast<double>(wj))) : kLogZero;
   } else {
@@ -487,15 +470,14 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* pts, int64_t cou
   for (int k = 2 * D + 2; k < KP; k += 2) keys[base + k] = 0.0f;
 }
 
-// Key bias of every real point: h_j = kappa (pot_j - |c_j|^2) + log2 w_j (pot = 0 if NULL).
+// Key bias of every real point: H_j = kappa pot_j + log2 w_j (pot = 0 if NULL).
 template <int D>
 __global__ void __launch_bounds__(256) key_bias_kernel(float* keys, int64_t count, const float* pot,
                                                        const float* lw, double kappa) {
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (j >= count) return;
-  const double cn = row_sqnorm<D>(keys, j);
   const double p = pot ? static_cast<double>(pot[j]) : 0.0;
-  keys[key_slot<D>(j, D)] = static_cast<float>(kappa * (p - cn) + static_cast<double>(lw[j]));
+  keys[key_slot<D>(j, D)] = static_cast<float>(kappa * p + static_cast<double>(lw[j]));
 }
 
 // <v, w> in float64 (w NULL = uniform weight wu).

@@ -74,11 +74,13 @@ def c5_run():
 
 
 def test_c5_full_run_matches_warm_restart(c5_run):
-    """20 iterations in one call equal 19 iterations plus one warm-started iteration."""
+    """20 iterations in one call equal 19 iterations plus one warm-started iteration, up to
+    the float32 rounding of g between the two calls (a restart rebuilds the key bias from
+    the rounded g instead of carrying it from the previous pass)."""
     w, (x, y, a, b), f, g, _ = c5_run
     f20, g20 = fs.potentials(x, y, a, b, eps=w.eps, n_iters=w.n_iters)
-    np.testing.assert_array_equal(f20.cpu().numpy(), f)
-    np.testing.assert_array_equal(g20.cpu().numpy(), g)
+    assert_potential_close(f20.cpu().numpy(), f, "f", rel=1e-6)
+    assert_potential_close(g20.cpu().numpy(), g, "g", rel=1e-6)
 
 
 def test_c5_sampled_updates(c5_run):
