@@ -142,6 +142,35 @@ FS_API fs_status fs_marginal_residual(const fs_problem* p, const float* f, const
                                fs_stream_t stream);
 
 /*
+ * fs_potentials for callers that cannot allocate device memory. The pages have no
+ * counterpart to this entry point; it exists for the library's users.
+ *
+ * Some callers may not call cudaMalloc or cudaFree at all: a host application whose
+ * device memory is owned entirely by its own pool allocator, or a latency-critical loop
+ * that must not hit the implicit device synchronisation those calls can cause. They pass
+ * only their inputs and outputs (same meaning, layout and ownership as fs_potentials);
+ * the scratch space comes from a fixed array of FS_NOALLOC_SCRATCH_BYTES bytes in device
+ * global memory that the library declares statically. Every device that loads the
+ * library holds that array until the process exits.
+ *
+ *  - Problems whose fs_workspace_bytes() exceeds FS_NOALLOC_SCRATCH_BYTES are rejected
+ *    with FS_ERR_WORKSPACE before any device work. At d = 3 every problem with
+ *    n, m <= 80000 fits; larger d needs more scratch per point.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call before any
+ *    stream capture on the device.
+ *  - No call allocates or frees device memory (no cudaMalloc, cudaFree or allocating
+ *    library routine).
+ *  - All calls on a device share the one array and it keeps what the last call wrote:
+ *    calls that overlap on the GPU (two streams or host threads at once) race and give
+ *    wrong results. Serialise them.
+ * Other errors are those of fs_potentials.
+ */
+#define FS_NOALLOC_SCRATCH_BYTES (16u << 20)
+FS_API fs_status fs_potentials_noalloc(const fs_problem* p, int32_t n_iters, const float* g_init,
+                                       float* f, float* g, fs_stream_t stream);
+
+/*
  * One call for callers whose data live in HOST memory: copies x, y, a, b (and nothing
  * else) to the device, runs fs_potentials, fs_grad_x, fs_marginal_residual and
  * fs_cost, and copies f, g, grad_x, the cost and the four residual norms back.

@@ -25,6 +25,7 @@ EXPORTS = (
     "fs_status_string", "fs_last_cuda_error", "fs_workspace_bytes", "fs_potentials", "fs_cost",
     "fs_grad_x", "fs_marginal_residual", "fs_solve_host_workspace_bytes", "fs_solve_host",
     "fs_timing_enable", "fs_timing_reset", "fs_timing_get", "fs_launch_count",
+    "fs_potentials_noalloc",
 )
 
 
@@ -81,6 +82,8 @@ def load():
     lib.fs_timing_reset.restype = None
     lib.fs_timing_get.argtypes = [ctypes.POINTER(fs_timing)]
     lib.fs_timing_get.restype = None
+    lib.fs_potentials_noalloc.argtypes = [P, i32, vp, vp, vp, vp]
+    lib.fs_potentials_noalloc.restype = ctypes.c_int
     lib.fs_launch_count.argtypes = []
     lib.fs_launch_count.restype = ctypes.c_int64
     _lib = lib
