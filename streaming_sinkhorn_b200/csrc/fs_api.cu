@@ -105,15 +105,17 @@ int padded_dim(int d) {
 
 int64_t pairs_pad(int64_t count) { return round_up(ceil_div(count, 2), kPairPad); }
 
-// Launch variants of the streaming pass: (rows per thread, threads per CTA).
+// Launch variants of the streaming pass. Index 0 has the most rows per CTA; the planner
+// falls back to index 1 only for problems too small to fill the GPU otherwise.
+//   D <= 16, potential/marginal passes: (R, NT, G, min CTAs/SM) = (2, 128, 8, 6), (1, 128, 8, 8)
+//   D <= 16, gradient passes:                                   (2, 128, 8, 3), (1, 128, 8, 4)
+//   D > 16, every pass:                                          (1, 128, 4, 1)
+// (2 rows per thread at 6 CTAs/SM measured fastest among 1-8 rows x 128-512 threads.)
 struct Variant {
   int R, NT;
 };
-// LSE passes for D <= 16, from most to least rows per CTA.
-constexpr Variant kLseVariants[3] = {{4, 256}, {2, 128}, {1, 128}};
-// Gradient passes for D <= 16.
+constexpr Variant kLseVariants[2] = {{2, 128}, {1, 128}};
 constexpr Variant kGradVariants[2] = {{2, 128}, {1, 128}};
-// Everything for D > 16.
 constexpr Variant kWideVariant = {1, 128};
 
 struct Plan {
@@ -133,8 +135,14 @@ int num_sms_current() {
   return sms > 0 ? sms : 148;
 }
 
+size_t pass_smem_bytes(int D, int tile_pairs) {
+  return static_cast<size_t>(kStages) * tile_pairs * key_pair_floats(D) * 4;
+}
+
+int occupancy_for(int D, bool grad, int variant, size_t smem);  // defined after the kernels
+
 Plan make_plan(int64_t n_rows, int64_t key_pairs, int D, bool grad, int sms) {
-  const int64_t target = static_cast<int64_t>(sms) * 8;  // >= ~4 waves of 2 CTAs per SM
+  const int64_t fill = static_cast<int64_t>(sms) * 4;
   const int max_tile = D > 16 ? 32 : 128;
   const Variant* vars;
   int nv;
@@ -146,14 +154,14 @@ Plan make_plan(int64_t n_rows, int64_t key_pairs, int D, bool grad, int sms) {
     nv = 2;
   } else {
     vars = kLseVariants;
-    nv = 3;
+    nv = 2;
   }
   Plan p{};
   // Most rows per CTA whose (row blocks x tiles) still fills the machine; else the smallest.
   int chosen = nv - 1;
   for (int v = 0; v < nv; ++v) {
     const int64_t rb = ceil_div(n_rows, static_cast<int64_t>(vars[v].R) * vars[v].NT);
-    if (rb * (key_pairs / max_tile) >= target) {
+    if (rb * (key_pairs / max_tile) >= fill) {
       chosen = v;
       break;
     }
@@ -165,12 +173,28 @@ Plan make_plan(int64_t n_rows, int64_t key_pairs, int D, bool grad, int sms) {
   p.row_blocks = ceil_div(n_rows, rpc);
   p.rows_pad = p.row_blocks * rpc;
   int tile = max_tile;
-  while (tile > 16 && p.row_blocks * (key_pairs / tile) < target) tile /= 2;
+  while (tile > 16 && p.row_blocks * (key_pairs / tile) < fill) tile /= 2;
   p.tile_pairs = tile;
   const int64_t tiles = key_pairs / tile;
-  int64_t splits = std::min<int64_t>(tiles, std::max<int64_t>(1, ceil_div(target, p.row_blocks)));
-  splits = std::min<int64_t>(splits, 65535);
-  const int64_t per = ceil_div(tiles, splits);
+  // Column splits: the grid is row_blocks x splits equal units over `slots` resident CTAs.
+  // Take the fewest splits whose last wave is at least 97 % full (or the best within 4096).
+  const int64_t slots =
+      static_cast<int64_t>(sms) * occupancy_for(D, grad, chosen, pass_smem_bytes(D, tile));
+  int64_t best_s = 1;
+  double best_eff = -1.0;
+  const int64_t s_max = std::min<int64_t>(std::min<int64_t>(tiles, 4096), 65535);
+  for (int64_t sp = 1; sp <= s_max; ++sp) {
+    const int64_t per = ceil_div(tiles, sp);
+    const int64_t s_real = ceil_div(tiles, per);
+    const double waves = static_cast<double>(p.row_blocks * s_real) / static_cast<double>(slots);
+    const double eff = waves / std::ceil(waves);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best_s = s_real;
+    }
+    if (waves >= 1.0 && eff >= 0.97) break;
+  }
+  const int64_t per = ceil_div(tiles, best_s);
   p.n_splits = static_cast<int>(ceil_div(tiles, per));
   p.pairs_per_split = per * tile;
   return p;
@@ -243,46 +267,81 @@ inline bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr)
 
 // ---------------- kernel dispatch ----------------
 
-template <int D, int R, int NT, bool GRAD>
-void launch_pass_t(const PassParams& P, const Plan& pl, cudaStream_t st) {
-  constexpr int G = (D > 16) ? 4 : 8;
-  constexpr int MINB = (D > 16) ? 1 : (GRAD ? 3 : (NT == 256 ? 2 : 4));
-  auto kern = lse_pass_kernel<D, R, NT, G, GRAD, MINB>;
-  const size_t smem = static_cast<size_t>(kStages) * pl.tile_pairs * key_pair_floats(D) * 4;
-  static bool attr_set = false;  // per instantiation; idempotent, so a race is harmless
-  if (!attr_set) {
-    CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                            static_cast<int>(kStages * 128 * key_pair_floats(D) * 4)));
-    attr_set = true;
+template <int D, int R, int NT, bool GRAD, int G, int MINB>
+struct PassKernel {
+  static constexpr auto fn = lse_pass_kernel<D, R, NT, G, GRAD, MINB>;
+  static void set_smem_attr() {
+    static bool done = false;  // idempotent, so a race between threads is harmless
+    if (!done) {
+      CK(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(pass_smem_bytes(D, 128))));
+      done = true;
+    }
   }
-  dim3 grid(static_cast<unsigned>(pl.row_blocks), static_cast<unsigned>(pl.n_splits));
-  kern<<<grid, NT, smem, st>>>(P);
-  CK(cudaGetLastError());
-  g_launches.fetch_add(1, std::memory_order_relaxed);
+  static void launch(const PassParams& P, const Plan& pl, cudaStream_t st) {
+    set_smem_attr();
+    dim3 grid(static_cast<unsigned>(pl.row_blocks), static_cast<unsigned>(pl.n_splits));
+    fn<<<grid, NT, pass_smem_bytes(D, pl.tile_pairs), st>>>(P);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  static int occupancy(size_t smem) {
+    int n = 0;
+    set_smem_attr();
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, NT, smem) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = MINB;
+    }
+    return n;
+  }
+};
+
+// The kernel of (D, pass type, variant): calls op.template run<Kernel>().
+template <int D, typename Op>
+void with_pass_kernel(bool grad, int variant, Op&& op) {
+  if constexpr (D > 16) {
+    if (grad)
+      op.template run<PassKernel<D, 1, 128, true, 4, 1>>();
+    else
+      op.template run<PassKernel<D, 1, 128, false, 4, 1>>();
+  } else {
+    if (grad) {
+      if (variant == 0)
+        op.template run<PassKernel<D, 2, 128, true, 8, 3>>();
+      else
+        op.template run<PassKernel<D, 1, 128, true, 8, 4>>();
+    } else {
+      if (variant == 0)
+        op.template run<PassKernel<D, 2, 128, false, 8, 6>>();
+      else
+        op.template run<PassKernel<D, 1, 128, false, 8, 8>>();
+    }
+  }
 }
+
+struct LaunchOp {
+  const PassParams& P;
+  const Plan& pl;
+  cudaStream_t st;
+  template <typename K>
+  void run() { K::launch(P, pl, st); }
+};
+
+struct OccupancyOp {
+  size_t smem;
+  int result = 1;
+  template <typename K>
+  void run() { result = K::occupancy(smem); }
+};
 
 template <int D>
 void launch_pass_d(const PassParams& P, const Plan& pl, bool grad, cudaStream_t st) {
-  if constexpr (D > 16) {
-    if (grad)
-      launch_pass_t<D, 1, 128, true>(P, pl, st);
-    else
-      launch_pass_t<D, 1, 128, false>(P, pl, st);
-  } else {
-    if (grad) {
-      if (pl.variant == 0)
-        launch_pass_t<D, 2, 128, true>(P, pl, st);
-      else
-        launch_pass_t<D, 1, 128, true>(P, pl, st);
-    } else {
-      if (pl.variant == 0)
-        launch_pass_t<D, 4, 256, false>(P, pl, st);
-      else if (pl.variant == 1)
-        launch_pass_t<D, 2, 128, false>(P, pl, st);
-      else
-        launch_pass_t<D, 1, 128, false>(P, pl, st);
-    }
-  }
+  with_pass_kernel<D>(grad, pl.variant, LaunchOp{P, pl, st});
+}
+
+template <int D>
+void occupancy_d(bool grad, int variant, OccupancyOp* op) {
+  with_pass_kernel<D>(grad, variant, *op);
 }
 
 template <int D>
@@ -307,6 +366,17 @@ void launch_combine_d(const PassParams& P, bool grad, cudaStream_t st) {
     case 32: FN<32>(__VA_ARGS__); break;          \
     default: FN<64>(__VA_ARGS__); break;          \
   }
+
+int occupancy_for(int D, bool grad, int variant, size_t smem) {
+  OccupancyOp op{smem};
+  try {
+    FS_DISPATCH_D(D, occupancy_d, grad, variant, &op);
+  } catch (const CudaFail&) {
+    cudaGetLastError();
+    op.result = 1;
+  }
+  return op.result;
+}
 
 template <int D>
 void launch_pack_d(const float* pts, int64_t count, int d, const float* w, float wu, float* keys,

@@ -215,6 +215,8 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     for (int k = 0; k < NA; ++k) A[r][k] = pk(0.0f, 0.0f);
   }
 
+  // One CTA barrier per tile: after it every thread has finished the previous tile, so its
+  // stage can be refilled, and a timed-out wait anywhere in the CTA is visible to all.
   int t = 0;
   bool aborted = false;
   for (; t < n_tiles; ++t) {
@@ -224,6 +226,14 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     if (__syncthreads_or(!ok)) {
       aborted = true;
       break;
+    }
+    if (tid == 0 && t >= 1 && t - 1 + kStages < n_tiles) {
+      const int ps = (t - 1) % kStages;
+      fence_proxy_async_smem();
+      mbar_expect_tx(&bars[ps], stage_bytes);
+      bulk_g2s(stages + ps * stage_floats,
+               key_src + static_cast<int64_t>(t - 1 + kStages) * stage_floats, stage_bytes,
+               &bars[ps]);
     }
     const float* tile = stages + st * stage_floats;
     for (int pg = 0; pg < P.tile_pairs; pg += G) {
@@ -289,21 +299,15 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
         }
       }
     }
-    __syncthreads();
-    if (tid == 0 && t + kStages < n_tiles) {
-      fence_proxy_async_smem();
-      mbar_expect_tx(&bars[st], stage_bytes);
-      bulk_g2s(stages + st * stage_floats,
-               key_src + static_cast<int64_t>(t + kStages) * stage_floats, stage_bytes,
-               &bars[st]);
-    }
   }
 
   if (aborted) {
     // Record the timeout, let this CTA's own copies still in flight land (bounded), leave.
+    // Tiles t .. t + kStages - 2 were issued (tile t + kStages - 1 is issued only after the
+    // barrier of tile t, which was not passed).
     if (tid == 0) {
       atomicOr(P.err, kErrTimeout);
-      for (int u = t; u < n_tiles && u < t + kStages; ++u)
+      for (int u = t; u < n_tiles && u < t + kStages - 1; ++u)
         (void)mbar_wait_bounded(&bars[u % kStages], static_cast<uint32_t>(u / kStages) & 1u);
     }
     return;
