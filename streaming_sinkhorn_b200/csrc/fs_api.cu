@@ -9,7 +9,7 @@
 #include <vector>
 
 #include "../../include/fs.h"
-#include "fs_kernels.cuh"
+#include "fs_tc.cuh"
 
 namespace fs {
 namespace {
@@ -205,10 +205,49 @@ int64_t partial_floats(const Plan& p, int D, bool grad) {
   return static_cast<int64_t>(p.n_splits) * p.rows_pad * (2 + (grad ? D : 0));
 }
 
+// Points wider than 16 coordinates take the tensor-core pass for potential and marginal
+// passes (the gradient pass stays on the FMA path); its padded width is 32, 48 or 64.
+int tc_dim(int d) { return d <= 16 ? 0 : (d <= 32 ? 32 : (d <= 48 ? 48 : 64)); }
+int64_t tc_pad(int64_t count) { return round_up(count, kTcRows); }
+
+struct TcPlan {
+  int64_t row_blocks, rows_pad, key_tiles, tiles_per_split;
+  int n_splits;
+};
+
+int occupancy_tc(int Dtc);  // defined with the launchers
+
+TcPlan make_tc_plan(int64_t n_rows, int64_t n_keys, int Dtc, int sms) {
+  TcPlan p{};
+  p.row_blocks = ceil_div(n_rows, kTcRows);
+  p.rows_pad = p.row_blocks * kTcRows;
+  p.key_tiles = tc_pad(n_keys) / kTcCols;
+  const int64_t slots = static_cast<int64_t>(sms) * occupancy_tc(Dtc);
+  int64_t best_s = 1;
+  double best_eff = -1.0;
+  const int64_t s_max = std::min<int64_t>(p.key_tiles, 4096);
+  for (int64_t sp = 1; sp <= s_max; ++sp) {
+    const int64_t per = ceil_div(p.key_tiles, sp);
+    const int64_t s_real = ceil_div(p.key_tiles, per);
+    const double waves = static_cast<double>(p.row_blocks * s_real) / static_cast<double>(slots);
+    const double eff = waves / std::ceil(waves);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best_s = s_real;
+    }
+    if (waves >= 1.0 && eff >= 0.97) break;
+  }
+  p.tiles_per_split = ceil_div(p.key_tiles, best_s);
+  p.n_splits = static_cast<int>(ceil_div(p.key_tiles, p.tiles_per_split));
+  return p;
+}
+
 constexpr size_t kAlign = 256;
 constexpr int kScalarDoubles = 256;  // 2 KiB of float64 scalars
 
 // Offsets (in doubles) inside the scalar block.
+constexpr int kSumX = 0;      // [64] coordinate sums of x (tensor-core path)
+constexpr int kSumY = 64;     // [64] coordinate sums of y
 constexpr int kSumA = 128;
 constexpr int kSumB = 129;
 constexpr int kAccRow = 130;  // [3]
@@ -217,13 +256,17 @@ constexpr int kDotFA = 136;
 constexpr int kDotGB = 137;
 constexpr int kFlags = 140;   // unsigned, in the bytes of this double
 constexpr int kErr = 141;     // unsigned
+constexpr int kMaxAbs = 142;  // unsigned: float bits of the largest |coordinate| of x and y
 
 struct Layout {
-  int D;       // padded dimension
+  int D;       // padded dimension of the FMA path
   int KP;      // floats per key pair
   int64_t px;  // key pairs of x (padded)
   int64_t py;
+  int Dtc;     // padded dimension of the tensor-core path, 0 if unused
+  int64_t tx, ty;  // points of x and y padded to whole 128-point tiles (tensor-core path)
   size_t off_scalars, off_kx, off_ky, off_lwx, off_lwy, off_part, total;
+  size_t off_rimg_x, off_kimg_x, off_rimg_y, off_kimg_y, off_nrm_x, off_nrm_y, off_hy_x, off_hy_y;
   int64_t part_floats;
 };
 
@@ -240,6 +283,13 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms) {
     pf = std::max(pf, partial_floats(make_plan(n, L.py, L.D, grad, sms), L.D, grad));
     pf = std::max(pf, partial_floats(make_plan(m, L.px, L.D, grad, sms), L.D, grad));
   }
+  L.Dtc = tc_dim(d);
+  L.tx = tc_pad(n);
+  L.ty = tc_pad(m);
+  if (L.Dtc) {
+    for (const TcPlan& tp : {make_tc_plan(n, m, L.Dtc, sms), make_tc_plan(m, n, L.Dtc, sms)})
+      if (tp.n_splits > 1) pf = std::max<int64_t>(pf, 2 * tp.n_splits * tp.rows_pad);
+  }
   L.part_floats = pf;
   size_t o = 0;
   L.off_scalars = o;
@@ -254,6 +304,25 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms) {
   o = align_up(o + static_cast<size_t>(2 * L.py) * sizeof(float));
   L.off_part = o;
   o = align_up(o + static_cast<size_t>(pf) * sizeof(float));
+  if (L.Dtc) {
+    const size_t kbytes = static_cast<size_t>(3 * L.Dtc) * 2;  // fp16 per point per image
+    L.off_rimg_x = o;
+    o = align_up(o + static_cast<size_t>(L.tx) * kbytes);
+    L.off_kimg_x = o;
+    o = align_up(o + static_cast<size_t>(L.tx) * kbytes);
+    L.off_rimg_y = o;
+    o = align_up(o + static_cast<size_t>(L.ty) * kbytes);
+    L.off_kimg_y = o;
+    o = align_up(o + static_cast<size_t>(L.ty) * kbytes);
+    L.off_nrm_x = o;
+    o = align_up(o + static_cast<size_t>(L.tx) * sizeof(float));
+    L.off_nrm_y = o;
+    o = align_up(o + static_cast<size_t>(L.ty) * sizeof(float));
+    L.off_hy_x = o;
+    o = align_up(o + static_cast<size_t>(L.tx) * sizeof(float));
+    L.off_hy_y = o;
+    o = align_up(o + static_cast<size_t>(L.ty) * sizeof(float));
+  }
   L.total = o;
   return L;
 }
@@ -367,6 +436,68 @@ void launch_combine_d(const PassParams& P, bool grad, cudaStream_t st) {
     default: FN<64>(__VA_ARGS__); break;          \
   }
 
+template <int Dtc>
+struct TcKernel {
+  static constexpr auto fn = lse_pass_tc_kernel<Dtc>;
+  static void set_smem_attr() {
+    static bool done = false;  // idempotent, so a race between threads is harmless
+    if (!done) {
+      CK(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(TcShape<Dtc>::SMEM)));
+      done = true;
+    }
+  }
+  static void launch(const PassParams& P, const TcParams& T, const TcPlan& pl, cudaStream_t st) {
+    set_smem_attr();
+    dim3 grid(static_cast<unsigned>(pl.row_blocks), static_cast<unsigned>(pl.n_splits));
+    fn<<<grid, kTcThreads, TcShape<Dtc>::SMEM, st>>>(P, T);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  static int occupancy() {
+    int n = 0;
+    try {
+      set_smem_attr();
+    } catch (const CudaFail&) {
+      cudaGetLastError();
+      return 1;
+    }
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kTcThreads, TcShape<Dtc>::SMEM) !=
+            cudaSuccess ||
+        n < 1) {
+      cudaGetLastError();
+      n = 1;
+    }
+    return n;
+  }
+};
+
+int occupancy_tc(int Dtc) {
+  switch (Dtc) {
+    case 32: return TcKernel<32>::occupancy();
+    case 48: return TcKernel<48>::occupancy();
+    default: return TcKernel<64>::occupancy();
+  }
+}
+
+void launch_tc(int Dtc, const PassParams& P, const TcParams& T, const TcPlan& pl, cudaStream_t st) {
+  switch (Dtc) {
+    case 32: TcKernel<32>::launch(P, T, pl, st); break;
+    case 48: TcKernel<48>::launch(P, T, pl, st); break;
+    default: TcKernel<64>::launch(P, T, pl, st); break;
+  }
+}
+
+template <int Dtc>
+void launch_images(const float* pts, int64_t count, int d, const TcCenter& ctr, float scale,
+                   unsigned char* rimg, unsigned char* kimg, float* nrm, int64_t pad,
+                   cudaStream_t st) {
+  build_images_kernel<Dtc><<<static_cast<unsigned>(ceil_div(pad, 256)), 256, 0, st>>>(
+      pts, count, d, ctr, scale, rimg, kimg, nrm, pad);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
 int occupancy_for(int D, bool grad, int variant, size_t smem) {
   OccupancyOp op{smem};
   try {
@@ -413,6 +544,10 @@ struct Ctx {
   double ma, mb;  // weight sums
   double kappa;
   Timer* timer;
+  bool use_tc;    // potential and marginal passes on the tensor cores
+  unsigned char *rimg_x, *kimg_x, *rimg_y, *kimg_y;
+  float *nrm_x, *nrm_y, *hy_x, *hy_y;
+  float c2;       // 2 kappa / s^2
 };
 
 fs_status check_common(const fs_problem* p, void* ws, size_t ws_bytes, size_t* need_out,
@@ -439,6 +574,16 @@ void carve(Ctx& c, void* ws) {
   c.lwx = reinterpret_cast<float*>(c.ws + c.L.off_lwx);
   c.lwy = reinterpret_cast<float*>(c.ws + c.L.off_lwy);
   c.part = reinterpret_cast<float*>(c.ws + c.L.off_part);
+  if (c.L.Dtc) {
+    c.rimg_x = c.ws + c.L.off_rimg_x;
+    c.kimg_x = c.ws + c.L.off_kimg_x;
+    c.rimg_y = c.ws + c.L.off_rimg_y;
+    c.kimg_y = c.ws + c.L.off_kimg_y;
+    c.nrm_x = reinterpret_cast<float*>(c.ws + c.L.off_nrm_x);
+    c.nrm_y = reinterpret_cast<float*>(c.ws + c.L.off_nrm_y);
+    c.hy_x = reinterpret_cast<float*>(c.ws + c.L.off_hy_x);
+    c.hy_y = reinterpret_cast<float*>(c.ws + c.L.off_hy_y);
+  }
 }
 
 unsigned* flags_ptr(double* scal) { return reinterpret_cast<unsigned*>(scal + kFlags); }
@@ -450,9 +595,21 @@ unsigned reduce_blocks(int64_t count, int sms) {
 
 // Validates inputs on the device (one stream sync), packs both clouds and their log-weights.
 // `pots` lists potentials to check for finiteness (device pointers with their lengths).
-fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& pots) {
+fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& pots,
+                  bool need_tc) {
   const fs_problem* p = c.p;
+  c.use_tc = need_tc && c.L.Dtc > 0;
   CK(cudaMemsetAsync(c.scal, 0, kScalarDoubles * sizeof(double), c.st));
+  if (c.use_tc) {
+    unsigned* mx = reinterpret_cast<unsigned*>(c.scal + kMaxAbs);
+    dim3 gx(reduce_blocks(p->n, c.sms), p->d), gy(reduce_blocks(p->m, c.sms), p->d);
+    coord_stats_kernel<<<gx, 256, 0, c.st>>>(p->x, p->n, p->d, c.scal + kSumX, mx);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    coord_stats_kernel<<<gy, 256, 0, c.st>>>(p->y, p->m, p->d, c.scal + kSumY, mx);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
   check_coords_kernel<<<reduce_blocks(p->n * p->d, c.sms), 256, 0, c.st>>>(p->x, p->n * p->d,
                                                                            flags_ptr(c.scal));
   CK(cudaGetLastError());
@@ -479,7 +636,7 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
     CK(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
-  double host[kFlags + 2];
+  double host[kMaxAbs + 1];
   CK(cudaMemcpyAsync(host, c.scal, sizeof(host), cudaMemcpyDeviceToHost, c.st));
   CK(cudaStreamSynchronize(c.st));
   unsigned flags;
@@ -494,11 +651,65 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
   const float wu_x = static_cast<float>(1.0 / p->n), wu_y = static_cast<float>(1.0 / p->m);
   FS_DISPATCH_D(c.L.D, launch_pack_d, p->x, p->n, p->d, p->a, wu_x, c.kx, c.lwx, c.L.px, c.st);
   FS_DISPATCH_D(c.L.D, launch_pack_d, p->y, p->m, p->d, p->b, wu_y, c.ky, c.lwy, c.L.py, c.st);
+  if (c.use_tc) {
+    // Centre on the common mean (the cost is translation invariant) and scale by a power of
+    // two that puts the largest centred coordinate near 2^14, well inside fp16 range.
+    TcCenter ctr{};
+    double cmax = 0.0;
+    for (int k = 0; k < p->d; ++k) {
+      ctr.c[k] = (host[kSumX + k] + host[kSumY + k]) / static_cast<double>(p->n + p->m);
+      cmax = std::max(cmax, std::fabs(ctr.c[k]));
+    }
+    unsigned bits;
+    memcpy(&bits, &host[kMaxAbs], sizeof(unsigned));
+    float fmaxabs;
+    memcpy(&fmaxabs, &bits, sizeof(float));
+    const double bound = static_cast<double>(fmaxabs) + cmax;
+    const double scale = bound > 0.0 ? std::exp2(std::floor(std::log2(16384.0 / bound))) : 1.0;
+    c.c2 = static_cast<float>(2.0 * c.kappa / (scale * scale));
+    switch (c.L.Dtc) {
+      case 32:
+        launch_images<32>(p->x, p->n, p->d, ctr, static_cast<float>(scale), c.rimg_x, c.kimg_x, c.nrm_x, c.L.tx, c.st);
+        launch_images<32>(p->y, p->m, p->d, ctr, static_cast<float>(scale), c.rimg_y, c.kimg_y, c.nrm_y, c.L.ty, c.st);
+        break;
+      case 48:
+        launch_images<48>(p->x, p->n, p->d, ctr, static_cast<float>(scale), c.rimg_x, c.kimg_x, c.nrm_x, c.L.tx, c.st);
+        launch_images<48>(p->y, p->m, p->d, ctr, static_cast<float>(scale), c.rimg_y, c.kimg_y, c.nrm_y, c.L.ty, c.st);
+        break;
+      default:
+        launch_images<64>(p->x, p->n, p->d, ctr, static_cast<float>(scale), c.rimg_x, c.kimg_x, c.nrm_x, c.L.tx, c.st);
+        launch_images<64>(p->y, p->m, p->d, ctr, static_cast<float>(scale), c.rimg_y, c.kimg_y, c.nrm_y, c.L.ty, c.st);
+        break;
+    }
+  }
   return FS_OK;
 }
 
-// Sets the key bias of one cloud from a potential (NULL = zero potential).
+// Sets the key bias of one cloud from a potential (NULL = zero potential), in the form the
+// next pass reads: the packed-key slot (FMA path) or the hy array (tensor-core path).
+void set_bias(Ctx& c, bool cloud_x, const float* pot);
+
+// prepare() followed by a zero-potential bias on both clouds in the tensor-core layout, so
+// the padding columns of both hy arrays hold log2(0) before any pass reads them.
+fs_status prepare_all(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& pots,
+                      bool need_tc) {
+  const fs_status r = prepare(c, pots, need_tc);
+  if (r != FS_OK || !c.use_tc) return r;
+  set_bias(c, true, nullptr);
+  set_bias(c, false, nullptr);
+  return FS_OK;
+}
+
 void set_bias(Ctx& c, bool cloud_x, const float* pot) {
+  if (c.use_tc) {
+    const int64_t count = cloud_x ? c.p->n : c.p->m, pad = cloud_x ? c.L.tx : c.L.ty;
+    tc_key_bias_kernel<<<static_cast<unsigned>(ceil_div(pad, 256)), 256, 0, c.st>>>(
+        cloud_x ? c.hy_x : c.hy_y, count, pad, pot, cloud_x ? c.lwx : c.lwy,
+        cloud_x ? c.nrm_x : c.nrm_y, c.kappa);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return;
+  }
   if (cloud_x)
     FS_DISPATCH_D(c.L.D, launch_bias_d, c.kx, c.p->n, pot, c.lwx, c.kappa, c.st)
   else
@@ -506,8 +717,58 @@ void set_bias(Ctx& c, bool cloud_x, const float* pot) {
 }
 
 // One streaming pass with rows from cloud x (rows_x) or y, keys from the other cloud.
+void run_pass_tc(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out,
+                 float* marg_out, double* acc) {
+  const fs_problem* p = c.p;
+  const int64_t n_rows = rows_x ? p->n : p->m, n_keys = rows_x ? p->m : p->n;
+  const TcPlan pl = make_tc_plan(n_rows, n_keys, c.L.Dtc, c.sms);
+  PassParams P{};
+  P.n_rows = n_rows;
+  P.n_splits = pl.n_splits;
+  P.rows_pad = pl.rows_pad;
+  P.kind = kind;
+  P.d_real = p->d;
+  P.kappa = c.kappa;
+  P.kappa_f = static_cast<float>(c.kappa);
+  P.inv_kappa_f = static_cast<float>(1.0 / c.kappa);
+  P.eps_ln2 = 1.0 / c.kappa;
+  P.lw = rows_x ? c.lwx : c.lwy;
+  P.w = rows_x ? p->a : p->b;
+  P.w_uniform = static_cast<float>(1.0 / n_rows);
+  P.pot_in = pot_in;
+  P.pot_out = pot_out;
+  P.marg_out = marg_out;
+  P.acc = acc;
+  P.part_m = c.part;
+  P.part_l = c.part + static_cast<int64_t>(pl.n_splits) * pl.rows_pad;
+  P.err = err_ptr(c.scal);
+  P.hy_out = rows_x ? c.hy_x : c.hy_y;
+  P.nrm = rows_x ? c.nrm_x : c.nrm_y;
+  TcParams T{};
+  T.row_img = rows_x ? c.rimg_x : c.rimg_y;
+  T.key_img = rows_x ? c.kimg_y : c.kimg_x;
+  T.key_hy = rows_x ? c.hy_y : c.hy_x;
+  T.row_nrm = rows_x ? c.nrm_x : c.nrm_y;
+  T.key_tiles = pl.key_tiles;
+  T.tiles_per_split = pl.tiles_per_split;
+  T.c2 = c.c2;
+  const double pairs = static_cast<double>(n_rows) * static_cast<double>(n_keys);
+  int ti = c.timer->begin();
+  launch_tc(c.L.Dtc, P, T, pl, c.st);
+  c.timer->end(ti, kind == kMarg ? kTMarg : kTLse, pairs);
+  if (pl.n_splits > 1) {
+    ti = c.timer->begin();
+    FS_DISPATCH_D(c.L.D, launch_combine_d, P, false, c.st);
+    c.timer->end(ti, kTCombine, 0.0);
+  }
+}
+
 void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out, float* marg_out,
               float* grad_out, double* acc) {
+  if (c.use_tc && kind != kGrad) {
+    run_pass_tc(c, rows_x, kind, pot_in, pot_out, marg_out, acc);
+    return;
+  }
   const fs_problem* p = c.p;
   const bool grad = kind == kGrad;
   const int64_t n_rows = rows_x ? p->n : p->m;
@@ -602,7 +863,7 @@ fs_status potentials_impl(const fs_problem* p, int32_t n_iters, const float* g_i
   return guarded(c.st, [&]() -> fs_status {
     std::vector<std::pair<const float*, int64_t>> pots;
     if (g_init) pots.push_back({g_init, p->m});
-    fs_status r = prepare(c, pots);
+    fs_status r = prepare_all(c, pots, true);
     if (r != FS_OK) return r;
     set_bias(c, false, g_init);
     for (int32_t it = 0; it < n_iters; ++it) {
@@ -660,7 +921,7 @@ fs_status fs_grad_x(const fs_problem* p, const float* g, float* grad_x, void* ws
   Timer timer(c.st);
   c.timer = &timer;
   return guarded(c.st, [&]() -> fs_status {
-    fs_status r = prepare(c, {{g, p->m}});
+    fs_status r = prepare_all(c, {{g, p->m}}, false);
     if (r != FS_OK) return r;
     set_bias(c, false, g);
     run_pass(c, true, kGrad, nullptr, nullptr, nullptr, grad_x, nullptr);
@@ -682,7 +943,7 @@ fs_status fs_marginal_residual(const fs_problem* p, const float* f, const float*
   Timer timer(c.st);
   c.timer = &timer;
   return guarded(c.st, [&]() -> fs_status {
-    fs_status r = prepare(c, {{f, p->n}, {g, p->m}});
+    fs_status r = prepare_all(c, {{f, p->n}, {g, p->m}}, true);
     if (r != FS_OK) return r;
     set_bias(c, false, g);  // keys y carry g: row pass gives F(g)
     set_bias(c, true, f);   // keys x carry f: column pass gives G(f)
@@ -707,7 +968,7 @@ fs_status fs_cost(const fs_problem* p, const float* f, const float* g, double* o
   Timer timer(c.st);
   c.timer = &timer;
   return guarded(c.st, [&]() -> fs_status {
-    fs_status r = prepare(c, {{f, p->n}, {g, p->m}});
+    fs_status r = prepare_all(c, {{f, p->n}, {g, p->m}}, true);
     if (r != FS_OK) return r;
     set_bias(c, true, f);  // keys x carry f: column pass gives c_j = sum_i P_ij
     run_pass(c, false, kMarg, g, nullptr, nullptr, nullptr, c.scal + kAccCol);

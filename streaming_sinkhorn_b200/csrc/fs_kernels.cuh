@@ -76,6 +76,10 @@ struct PassParams {
   float* part_l;            // partial sums    [split][rows_pad]
   float* part_a;            // partial weighted differences [split][D][rows_pad]
   unsigned* err;            // error word
+  // tensor-core passes: the next pass's key bias hy_i = H_i - kappa |x_i|^2 of the query
+  // cloud (written instead of the packed-key slot) and its centred squared norms
+  float* hy_out;
+  const float* nrm;
 };
 
 // Offset of coordinate slot k (k == D is the bias H) of point i in packed keys.
@@ -91,7 +95,11 @@ __device__ __forceinline__ int64_t key_slot(int64_t i, int k) {
 template <int D>
 __device__ __forceinline__ void finish_pot(const PassParams& P, int64_t i, double lse2) {
   P.pot_out[i] = static_cast<float>(-lse2 * P.eps_ln2);
-  P.qkeys[key_slot<D>(i, D)] = static_cast<float>(static_cast<double>(P.lw[i]) - lse2);
+  const double h = static_cast<double>(P.lw[i]) - lse2;
+  if (P.hy_out)
+    P.hy_out[i] = static_cast<float>(h - P.kappa * static_cast<double>(P.nrm[i]));
+  else
+    P.qkeys[key_slot<D>(i, D)] = static_cast<float>(h);
 }
 
 // kMarg: plan marginal r_i = w_i 2^(kappa pot_i + LSE2_i) = w_i exp((pot_i - F_i)/eps).
