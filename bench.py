@@ -186,7 +186,9 @@ def oracle_sample(w, target_s: float):
     oracle.build()
     g0 = np.zeros(w.m, dtype=np.float64)
     rng = np.random.default_rng(0)
-    rows = rng.choice(w.n, size=min(w.n, 4), replace=False)
+    # calibrate on enough rows to keep every oracle thread busy
+    k0 = min(w.n, max(64, 8 * oracle.threads()))
+    rows = rng.choice(w.n, size=k0, replace=False)
     t0 = time.perf_counter()
     oracle.lse_update(w.x, w.y, w.b, g0, w.eps, rows=rows)
     per_row = (time.perf_counter() - t0) / len(rows)

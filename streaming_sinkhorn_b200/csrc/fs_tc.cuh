@@ -18,11 +18,13 @@
 // (stride-byte offset). A tile is therefore one contiguous block that a single TMA bulk copy
 // moves into shared memory.
 //
-// Kernel: one CTA per 128-row block and column split, 256 threads. Thread 0 streams key
-// tiles (B image + hy) through a 3-stage ring with bulk copies and issues the MMAs for tile
-// t into one of two TMEM accumulators while the 8 warps run the online max/sum on tile
-// t - 1 (warp w reads TMEM lanes 32 (w % 4) .. +31, columns of half w / 4). One CTA barrier
-// per tile separates the readers of an accumulator buffer and a stage from their refill.
+// Kernel: one CTA per 128-row block and column split, 10 warps with fixed roles. Warp 8
+// streams key tiles (B image + hy) through a 3-stage ring with TMA bulk copies; warp 9
+// issues the MMAs of tile t into one of two TMEM accumulators; warps 0-7 run the online
+// max/sum (warp w reads TMEM lanes 32 (w % 4) .. +31, the columns of half w / 4 of each
+// tile). Roles hand off through mbarriers only: a tile's stage is free once its MMAs have
+// completed (tcgen05.commit) and the 8 epilogue warps have read its biases; an accumulator
+// is free once the 8 epilogue warps have loaded it. No CTA barrier runs per tile.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -33,7 +35,8 @@ namespace fs {
 constexpr int kTcRows = 128;     // rows per CTA (MMA M)
 constexpr int kTcCols = 128;     // key columns per tile (MMA N)
 constexpr int kTcStages = 3;
-constexpr int kTcThreads = 256;  // 8 warps: 4 TMEM lane quarters x 2 column halves
+constexpr int kTcEpiWarps = 8;  // epilogue warps: 4 TMEM lane quarters x 2 column halves
+constexpr int kTcThreads = (kTcEpiWarps + 2) * 32;  // + a producer warp and an MMA warp
 constexpr uint32_t kTcTmemCols = 256;  // two accumulators of kTcCols fp32 columns
 
 template <int D>
@@ -94,6 +97,22 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
       : "memory");
 }
 
+// 32 consecutive fp32 columns of this thread's TMEM lane; the caller waits (tcgen05.wait::ld).
+__device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
 // 32 consecutive fp32 columns of this thread's TMEM lane.
 __device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
@@ -121,34 +140,62 @@ struct TcParams {
   float c2;                      // 2 kappa / s^2: scale of the MMA result
 };
 
+// Waits for phase `parity` of `bar`, giving up after kWaitLimitNs or as soon as another
+// role of the CTA has raised `abort`.
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassParams P,
                                                                    const TcParams T) {
   using S = TcShape<D>;
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ uint64_t full_bar[kTcStages];
-  __shared__ uint64_t mma_bar[2];
+  __shared__ uint64_t full_bar[kTcStages];   // tile landed (producer's expect_tx)
+  __shared__ uint64_t free_bar[kTcStages];   // stage reusable: MMA commit + 8 epilogue warps
+  __shared__ uint64_t mma_bar[2];            // accumulator ready (MMA commit)
+  __shared__ uint64_t acc_free_bar[2];       // accumulator read by the 8 epilogue warps
   __shared__ uint64_t a_bar;
   __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
   __shared__ float2 merge[kTcRows];
 
   unsigned char* sA = smem;
   unsigned char* sStage = smem + S::TILE_BYTES;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int quarter = warp & 3, half = warp >> 2;
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kTcRows;
   const int split = blockIdx.y;
   const int64_t t_begin = static_cast<int64_t>(split) * T.tiles_per_split;
   int64_t t_end = t_begin + T.tiles_per_split;
   if (t_end > T.key_tiles) t_end = T.key_tiles;
   const int n_tiles = static_cast<int>(t_end - t_begin);
+  volatile int* abort = &abort_sh;
 
   if (tid == 0) {
-    for (int s = 0; s < kTcStages; ++s) mbar_init(&full_bar[s], 1);
-    mbar_init(&mma_bar[0], 1);
-    mbar_init(&mma_bar[1], 1);
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&free_bar[s], kTcEpiWarps + 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&mma_bar[b], 1);
+      mbar_init(&acc_free_bar[b], kTcEpiWarps);
+    }
     mbar_init(&a_bar, 1);
+    abort_sh = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -162,136 +209,137 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  // Thread 0's record of the asynchronous work it started, for a bounded drain on timeout.
-  int tiles_issued = 0, full_waited = 0, mma_committed = 0, mma_waited = 0;
-  auto issue_tile = [&](int t) {  // thread 0 only
-    ++tiles_issued;
-    const int st = t % kTcStages;
-    unsigned char* dst = sStage + st * S::STAGE_BYTES;
-    const int64_t kt = t_begin + t;
-    mbar_expect_tx(&full_bar[st], S::TILE_BYTES + S::HY_BYTES);
-    bulk_g2s(dst, T.key_img + kt * S::TILE_BYTES, S::TILE_BYTES, &full_bar[st]);
-    bulk_g2s(dst + S::TILE_BYTES, T.key_hy + kt * kTcCols, S::HY_BYTES, &full_bar[st]);
-  };
-  if (tid == 0) {
-    mbar_expect_tx(&a_bar, S::TILE_BYTES);
-    bulk_g2s(sA, T.row_img + (row0 >> 7) * S::TILE_BYTES, S::TILE_BYTES, &a_bar);
-    for (int t = 0; t < kTcStages && t < n_tiles; ++t) issue_tile(t);
-  }
-
-  // Row state of this thread: one row, the columns of its half of every tile.
+  float m = -INFINITY;  // epilogue row state (origin-free running offset) ...
+  u64 L = pk(0.0f, 0.0f);
+  const int quarter = warp & 3, half = (warp >> 2) & 1;
   const int r = quarter * 32 + lane;
   const int64_t i = row0 + r;
-  const float knrm = (i < P.n_rows) ? P.kappa_f * T.row_nrm[i] : 0.0f;
-  float m = -INFINITY, base = 0.0f, mo = knrm;
-  u64 L = pk(0.0f, 0.0f);
-  const u64 c2 = pk(T.c2, T.c2);
-  const uint32_t idesc = tc_instr_desc(kTcRows, kTcCols);
 
-  bool fail = false;
-  if (tid == 0) fail = !mbar_wait_bounded(&a_bar, 0);
-  int t = 0;
-  bool aborted = false;
-  for (; t <= n_tiles; ++t) {
-    // MMA for tile t into accumulator t & 1.
-    if (t < n_tiles && tid == 0 && !fail) {
-      const int st = t % kTcStages;
-      if (!mbar_wait_bounded(&full_bar[st], static_cast<uint32_t>(t / kTcStages) & 1u)) {
-        fail = true;
-      } else {
-        ++full_waited;
+  if (warp == kTcEpiWarps) {
+    // ---- producer: the row block once, then key tiles through the stage ring ----------
+    if (lane == 0) {
+      int issued = 0, waited_free = 0;
+      mbar_expect_tx(&a_bar, S::TILE_BYTES);
+      bulk_g2s(sA, T.row_img + (row0 >> 7) * S::TILE_BYTES, S::TILE_BYTES, &a_bar);
+      for (int t = 0; t < n_tiles; ++t) {
+        const int st = t % kTcStages;
+        if (t >= kTcStages) {
+          if (!tc_wait(&free_bar[st], static_cast<uint32_t>((t - kTcStages) / kTcStages) & 1u, abort))
+            break;
+          ++waited_free;
+        }
+        unsigned char* dst = sStage + st * S::STAGE_BYTES;
+        const int64_t kt = t_begin + t;
+        fence_proxy_async_smem();
+        mbar_expect_tx(&full_bar[st], S::TILE_BYTES + S::HY_BYTES);
+        bulk_g2s(dst, T.key_img + kt * S::TILE_BYTES, S::TILE_BYTES, &full_bar[st]);
+        bulk_g2s(dst + S::TILE_BYTES, T.key_hy + kt * kTcCols, S::HY_BYTES, &full_bar[st]);
+        ++issued;
+      }
+      (void)waited_free;
+      // Copies never waited for by the MMA role: let them land before the CTA exits.
+      if (*abort) {
+        (void)mbar_wait_bounded(&a_bar, 0);
+        for (int t = (issued > kTcStages ? issued - kTcStages : 0); t < issued; ++t)
+          (void)mbar_wait_bounded(&full_bar[t % kTcStages], static_cast<uint32_t>(t / kTcStages) & 1u);
+      }
+    }
+  } else if (warp == kTcEpiWarps + 1) {
+    // ---- MMA issuer: tile t into accumulator t & 1 --------------------------------------
+    if (lane == 0) {
+      const uint32_t idesc = tc_instr_desc(kTcRows, kTcCols);
+      int committed = 0;
+      bool ok = tc_wait(&a_bar, 0, abort);
+      for (int t = 0; ok && t < n_tiles; ++t) {
+        const int st = t % kTcStages, b = t & 1;
+        if (!tc_wait(&full_bar[st], static_cast<uint32_t>(t / kTcStages) & 1u, abort)) break;
+        if (t >= 2 && !tc_wait(&acc_free_bar[b], static_cast<uint32_t>((t - 2) >> 1) & 1u, abort))
+          break;
         tc_fence_after();
         const uint32_t a0 = smem_u32(sA);
         const uint32_t b0 = smem_u32(sStage + st * S::STAGE_BYTES);
-        const uint32_t d = tmem + static_cast<uint32_t>(t & 1) * kTcCols;
+        const uint32_t d = tmem + static_cast<uint32_t>(b) * kTcCols;
 #pragma unroll
         for (int s = 0; s < S::KSTEPS; ++s) {
           tc_mma_f16(d, tc_smem_desc(a0 + s * 2 * S::LBO, S::LBO, S::SBO),
                      tc_smem_desc(b0 + s * 2 * S::LBO, S::LBO, S::SBO), idesc, s > 0 ? 1u : 0u);
         }
-        tc_commit(&mma_bar[t & 1]);
-        ++mma_committed;
+        tc_commit(&mma_bar[b]);
+        tc_commit(&free_bar[st]);
+        ++committed;
       }
+      // On abort, let the MMAs already issued finish before TMEM is released.
+      if (*abort && committed > 0)
+        (void)mbar_wait_bounded(&mma_bar[(committed - 1) & 1],
+                                static_cast<uint32_t>((committed - 1) >> 1) & 1u);
     }
-    // Online LSE over tile t - 1 (the TMEM loads below are warp-collective).
-    __syncwarp();
-    if (t >= 1) {
-      const int u = t - 1;
-      if (!mbar_wait_bounded(&mma_bar[u & 1], static_cast<uint32_t>(u >> 1) & 1u))
-        fail = true;
-      else
-        ++mma_waited;
-      if (!fail) {
-        tc_fence_after();
-        const float* hy = reinterpret_cast<const float*>(sStage + (u % kTcStages) * S::STAGE_BYTES +
-                                                         S::TILE_BYTES);
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          const int col0 = half * 64 + c * 32;
-          float v[32];
-          tc_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
-                      static_cast<uint32_t>(u & 1) * kTcCols + col0,
-                  v);
-          const u64* hv = reinterpret_cast<const u64*>(hy + col0);
-          const u64 nmo = pk(-mo, -mo);
-          u64 tv[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) tv[j] = add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), hv[j]), nmo);
-          float a0, a1;
-          upk(tv[0], a0, a1);
-          float mx = fmaxf(a0, a1);
-#pragma unroll
-          for (int j = 1; j < 16; ++j) {
-            upk(tv[j], a0, a1);
-            mx = max3(mx, a0, a1);
-          }
-          const float mx_abs = mx + base;
-          if (mx_abs > m + kLazyThr && mx > kEmptyCut) {
-            const float sc = ex2(m - mx_abs);
-            L = mul2(L, pk(sc, sc));
-            const u64 sh = pk(-mx, -mx);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) tv[j] = add2(tv[j], sh);
-            m = mx_abs;
-            base = mx_abs;
-            mo = knrm + m;
-          }
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float t0, t1;
-            upk(tv[j], t0, t1);
-            L = add2(L, pk(ex2(t0), ex2(t1)));
-          }
-        }
-      }
+  } else {
+    // ---- epilogue warps: online max/sum of one row over half of every tile ------------
+    const float knrm = (i < P.n_rows) ? P.kappa_f * T.row_nrm[i] : 0.0f;
+    float base = 0.0f, mo = knrm;
+    const u64 c2 = pk(T.c2, T.c2);
+    for (int u = 0; u < n_tiles; ++u) {
+      const int b = u & 1, st = u % kTcStages;
+      if (!tc_wait(&mma_bar[b], static_cast<uint32_t>(u >> 1) & 1u, abort)) break;
+      tc_fence_after();
+      const float* hy = reinterpret_cast<const float*>(sStage + st * S::STAGE_BYTES + S::TILE_BYTES);
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(b) * kTcCols + half * 64;
+      float v[64];
+      tc_ld32_nowait(tbase, v);
+      tc_ld32_nowait(tbase + 32, v + 32);
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_free_bar[b]);
+      const u64* hv = reinterpret_cast<const u64*>(hy + half * 64);
+      u64 tv[32];
+      const u64 nmo = pk(-mo, -mo);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) tv[j] = add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), hv[j]), nmo);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&free_bar[st]);
+      float a0, a1;
+      upk(tv[0], a0, a1);
+      float mx = fmaxf(a0, a1);
+#pragma unroll
+      for (int j = 1; j < 32; ++j) {
+        upk(tv[j], a0, a1);
+        mx = max3(mx, a0, a1);
+      }
+      const float mx_abs = mx + base;
+      if (mx_abs > m + kLazyThr && mx > kEmptyCut) {
+        const float sc = ex2(m - mx_abs);
+        L = mul2(L, pk(sc, sc));
+        const u64 sh = pk(-mx, -mx);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) tv[j] = add2(tv[j], sh);
+        m = mx_abs;
+        base = mx_abs;
+        mo = knrm + m;
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float t0, t1;
+        upk(tv[j], t0, t1);
+        L = add2(L, pk(ex2(t0), ex2(t1)));
+      }
     }
-    if (__syncthreads_or(fail)) {
-      aborted = true;
-      break;
-    }
-    // Stage (t - 1) % 3 is free: its MMA is complete and its hy has been read.
-    if (tid == 0 && t >= 1 && t - 1 + kTcStages < n_tiles) issue_tile(t - 1 + kTcStages);
   }
 
-  if (aborted) {
-    // Record the timeout; let this CTA's own copies and MMAs in flight finish (bounded).
-    // At most one phase of each barrier is outstanding, so the parities are unambiguous.
-    if (tid == 0) {
-      atomicOr(P.err, kErrTimeout);
-      for (int u = full_waited; u < tiles_issued; ++u)
-        (void)mbar_wait_bounded(&full_bar[u % kTcStages], static_cast<uint32_t>(u / kTcStages) & 1u);
-      for (int u = mma_waited; u < mma_committed; ++u)
-        (void)mbar_wait_bounded(&mma_bar[u & 1], static_cast<uint32_t>(u >> 1) & 1u);
-    }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (abort_sh) {
+    if (tid == 0) atomicOr(P.err, kErrTimeout);
   } else {
     // Merge the two column halves of each row, then finish the row.
     float l0, l1;
     upk(L, l0, l1);
-    if (half == 1) merge[r] = make_float2(m, l0 + l1);
+    if (warp < kTcEpiWarps && half == 1) merge[r] = make_float2(m, l0 + l1);
     __syncthreads();
     double dev = 0.0, mass = 0.0;
-    if (half == 0 && i < P.n_rows) {
+    if (warp < kTcEpiWarps && half == 0 && i < P.n_rows) {
       const float2 o = merge[r];
       const float mm = fmaxf(m, o.x);
       float l = 0.0f;
