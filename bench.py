@@ -279,7 +279,10 @@ def run_native(args, rank, world, local_rank):
     # roofline of the dominant kernel: the potential-update pass
     lse = timing["lse_pass"]
     per_launch_ms = lse["total_ms"] / max(lse["launches"], 1)
-    per_launch_pairs = lse["pairs"] / max(lse["launches"], 1)
+    # exponentials actually issued (after block screening; padding included); the tensor-core
+    # path does not screen and reports none, so its nominal pair count stands
+    executed = lse["evaluated"] if lse["evaluated"] > 0 else lse["pairs"]
+    per_launch_pairs = executed / max(lse["launches"], 1)
     achieved = per_launch_pairs / (per_launch_ms / 1e3)  # ex2 / s
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     max_mhz = clk.get("sm_max_mhz") or measured_peaks().get("sm_max_mhz") or 1965.0
@@ -291,7 +294,10 @@ def run_native(args, rank, world, local_rank):
                 "peak_basis": f"{sms} SMs x {EX2_PER_CLK_PER_SM} ex2/clk x {max_mhz:.0f} MHz",
                 "frac_at_observed_clock": (achieved / (sms * EX2_PER_CLK_PER_SM * clk["sm_mhz"] * 1e6)
                                            if clk.get("sm_mhz") else None),
-                "launches_timed": lse["launches"], "ms_per_launch": per_launch_ms}
+                "launches_timed": lse["launches"], "ms_per_launch": per_launch_ms,
+                "executed_ex2_per_launch": per_launch_pairs,
+                "nominal_pairs_per_launch": lse["pairs"] / max(lse["launches"], 1),
+                "screened_fraction": (1.0 - executed / lse["pairs"]) if lse["pairs"] else 0.0}
 
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -192,7 +192,9 @@ FS_API fs_status fs_solve_host(const fs_problem* p, int32_t n_iters, float* f, f
 typedef struct {
   int64_t launches; /* launches measured since the last reset */
   double total_ms;  /* their summed device durations */
-  double pairs;     /* (row, column) pairs they evaluated, i.e. exponentials */
+  double pairs;     /* (row, column) pairs the problem defines for them: N * M per pass */
+  double evaluated; /* pairs actually evaluated (exponentials issued, padding included)
+                       after block screening; filled for the potential passes */
 } fs_timing_entry;
 
 typedef struct {

@@ -251,5 +251,6 @@ def timing_get() -> dict:
     _lib.load().fs_timing_get(ctypes.byref(t))
     return {name: {"launches": int(getattr(t, name).launches),
                    "total_ms": float(getattr(t, name).total_ms),
-                   "pairs": float(getattr(t, name).pairs)}
+                   "pairs": float(getattr(t, name).pairs),
+                   "evaluated": float(getattr(t, name).evaluated)}
             for name in ("lse_pass", "grad_pass", "marg_pass", "combine")}

@@ -37,7 +37,7 @@ class fs_problem(ctypes.Structure):
 
 class fs_timing_entry(ctypes.Structure):
     _fields_ = [("launches", ctypes.c_int64), ("total_ms", ctypes.c_double),
-                ("pairs", ctypes.c_double)]
+                ("pairs", ctypes.c_double), ("evaluated", ctypes.c_double)]
 
 
 class fs_timing(ctypes.Structure):

@@ -67,10 +67,12 @@ class Timer {
     rec_[idx].pairs = pairs;
     CK(cudaEventRecord(rec_[idx].stop, stream_));
   }
-  // Call after the stream has been synchronised.
-  void collect() {
+  // Call after the stream has been synchronised; `evaluated` = pairs the potential passes
+  // of this call evaluated after screening.
+  void collect(double evaluated) {
     if (!on_) return;
     std::lock_guard<std::mutex> lk(g_timing_mu);
+    g_timing.lse_pass.evaluated += evaluated;
     for (auto& t : rec_) {
       float ms = 0.f;
       CK(cudaEventElapsedTime(&ms, t.start, t.stop));
@@ -177,15 +179,18 @@ Plan make_plan(int64_t n_rows, int64_t key_pairs, int D, bool grad, int sms) {
   p.tile_pairs = tile;
   const int64_t tiles = key_pairs / tile;
   // Column splits: the grid is row_blocks x splits equal units over `slots` resident CTAs.
-  // Take the fewest splits whose last wave is at least 97 % full (or the best within 4096).
+  // Take the fewest splits whose last wave is at least 97 % full, else the best one within
+  // max(4 waves, 3 splits per row block) units (which bounds the partial buffers).
   const int64_t slots =
       static_cast<int64_t>(sms) * occupancy_for(D, grad, chosen, pass_smem_bytes(D, tile));
+  const int64_t max_units = std::max<int64_t>(4 * slots, 3 * p.row_blocks);
   int64_t best_s = 1;
   double best_eff = -1.0;
   const int64_t s_max = std::min<int64_t>(std::min<int64_t>(tiles, 4096), 65535);
   for (int64_t sp = 1; sp <= s_max; ++sp) {
     const int64_t per = ceil_div(tiles, sp);
     const int64_t s_real = ceil_div(tiles, per);
+    if (sp > 1 && p.row_blocks * s_real > max_units) break;
     const double waves = static_cast<double>(p.row_blocks * s_real) / static_cast<double>(slots);
     const double eff = waves / std::ceil(waves);
     if (eff > best_eff + 1e-9) {
@@ -223,12 +228,14 @@ TcPlan make_tc_plan(int64_t n_rows, int64_t n_keys, int Dtc, int sms) {
   p.rows_pad = p.row_blocks * kTcRows;
   p.key_tiles = tc_pad(n_keys) / kTcCols;
   const int64_t slots = static_cast<int64_t>(sms) * occupancy_tc(Dtc);
+  const int64_t max_units = std::max<int64_t>(4 * slots, 3 * p.row_blocks);
   int64_t best_s = 1;
   double best_eff = -1.0;
   const int64_t s_max = std::min<int64_t>(p.key_tiles, 4096);
   for (int64_t sp = 1; sp <= s_max; ++sp) {
     const int64_t per = ceil_div(p.key_tiles, sp);
     const int64_t s_real = ceil_div(p.key_tiles, per);
+    if (sp > 1 && p.row_blocks * s_real > max_units) break;
     const double waves = static_cast<double>(p.row_blocks * s_real) / static_cast<double>(slots);
     const double eff = waves / std::ceil(waves);
     if (eff > best_eff + 1e-9) {
@@ -257,6 +264,9 @@ constexpr int kDotGB = 137;
 constexpr int kFlags = 140;   // unsigned, in the bytes of this double
 constexpr int kErr = 141;     // unsigned
 constexpr int kMaxAbs = 142;  // unsigned: float bits of the largest |coordinate| of x and y
+constexpr int kBox = 144;     // ints: ordered lo[3], hi[3] of the first three coordinates
+constexpr int kDmin = 147;    // ints: ordered smallest key-bias change of x, of y
+constexpr int kEval = 148;    // uint64: pairs evaluated by screened potential passes
 
 struct Layout {
   int D;       // padded dimension of the FMA path
@@ -267,6 +277,12 @@ struct Layout {
   int64_t tx, ty;  // points of x and y padded to whole 128-point tiles (tensor-core path)
   size_t off_scalars, off_kx, off_ky, off_lwx, off_lwy, off_part, total;
   size_t off_rimg_x, off_kimg_x, off_rimg_y, off_kimg_y, off_nrm_x, off_nrm_y, off_hy_x, off_hy_y;
+  // spatial order and screening (FMA path): permutations, sort keys, per-tile boxes and bias
+  // maxima, and the LSE2 of every row in its last pass
+  bool sorted;
+  int64_t sort_n;  // keys of the bitonic sort (power of two, >= kSortSmem)
+  size_t off_perm_x, off_perm_y, off_sortkeys, off_box_x, off_box_y, off_hmax_x, off_hmax_y,
+      off_lse_x, off_lse_y;
   int64_t part_floats;
 };
 
@@ -322,6 +338,31 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms) {
     o = align_up(o + static_cast<size_t>(L.tx) * sizeof(float));
     L.off_hy_y = o;
     o = align_up(o + static_cast<size_t>(L.ty) * sizeof(float));
+  }
+  L.sorted = L.Dtc == 0;
+  if (L.sorted) {
+    int64_t sn = kSortSmem;
+    while (sn < std::max(n, m)) sn <<= 1;
+    L.sort_n = sn;
+    const int64_t tiles_x = L.px / kPairPad, tiles_y = L.py / kPairPad;
+    L.off_perm_x = o;
+    o = align_up(o + static_cast<size_t>(n) * sizeof(int));
+    L.off_perm_y = o;
+    o = align_up(o + static_cast<size_t>(m) * sizeof(int));
+    L.off_sortkeys = o;
+    o = align_up(o + static_cast<size_t>(sn) * sizeof(uint64_t));
+    L.off_box_x = o;
+    o = align_up(o + static_cast<size_t>(tiles_x) * 2 * L.D * sizeof(float));
+    L.off_box_y = o;
+    o = align_up(o + static_cast<size_t>(tiles_y) * 2 * L.D * sizeof(float));
+    L.off_hmax_x = o;
+    o = align_up(o + static_cast<size_t>(tiles_x) * sizeof(float));
+    L.off_hmax_y = o;
+    o = align_up(o + static_cast<size_t>(tiles_y) * sizeof(float));
+    L.off_lse_x = o;
+    o = align_up(o + static_cast<size_t>(n) * sizeof(float));
+    L.off_lse_y = o;
+    o = align_up(o + static_cast<size_t>(m) * sizeof(float));
   }
   L.total = o;
   return L;
@@ -510,19 +551,63 @@ int occupancy_for(int D, bool grad, int variant, size_t smem) {
 }
 
 template <int D>
-void launch_pack_d(const float* pts, int64_t count, int d, const float* w, float wu, float* keys,
-                   float* lw, int64_t pp, cudaStream_t st) {
+void launch_pack_d(const float* pts, int64_t count, int d, const float* w, float wu,
+                   const int* perm, float* keys, float* lw, int64_t pp, cudaStream_t st) {
   const unsigned blocks = static_cast<unsigned>(ceil_div(2 * pp, 256));
-  pack_kernel<D><<<blocks, 256, 0, st>>>(pts, count, d, w, wu, keys, lw, pp);
+  pack_kernel<D><<<blocks, 256, 0, st>>>(pts, count, d, w, wu, perm, keys, lw, pp);
   CK(cudaGetLastError());
   g_launches.fetch_add(1, std::memory_order_relaxed);
 }
 
 template <int D>
-void launch_bias_d(float* keys, int64_t count, const float* pot, const float* lw, double kappa,
-                   cudaStream_t st) {
+void launch_bias_d(float* keys, int64_t count, const float* pot, const int* perm, const float* lw,
+                   double kappa, cudaStream_t st) {
   const unsigned blocks = static_cast<unsigned>(ceil_div(count, 256));
-  key_bias_kernel<D><<<blocks, 256, 0, st>>>(keys, count, pot, lw, kappa);
+  key_bias_kernel<D><<<blocks, 256, 0, st>>>(keys, count, pot, perm, lw, kappa);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
+template <int D>
+void launch_tile_box_d(const float* keys, int64_t count, int64_t tiles, float* box,
+                       cudaStream_t st) {
+  tile_box_kernel<D><<<static_cast<unsigned>(tiles), 256, 0, st>>>(keys, count, box);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
+template <int D>
+void launch_tile_hmax_d(const float* keys, int64_t count, int64_t tiles, float* hmax,
+                        cudaStream_t st) {
+  tile_hmax_kernel<D><<<static_cast<unsigned>(tiles), 256, 0, st>>>(keys, count, hmax);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
+// Morton order of one cloud: keys (code << 32 | index), bitonic sort, permutation.
+void sort_cloud(const float* pts, int64_t count, int d, const MortonFrame& F, uint64_t* keys,
+                int64_t sort_n, int* perm, cudaStream_t st) {
+  morton_keys_kernel<<<static_cast<unsigned>(ceil_div(sort_n, 256)), 256, 0, st>>>(
+      pts, count, d, F, keys, sort_n);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  const unsigned sblocks = static_cast<unsigned>(sort_n / kSortSmem);
+  bitonic_smem_kernel<<<sblocks, kSortBlock, 0, st>>>(keys, 0);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  for (int64_t k = 2 * kSortSmem; k <= sort_n; k <<= 1) {
+    for (int64_t j = k / 2; j >= kSortSmem; j >>= 1) {
+      bitonic_global_kernel<<<static_cast<unsigned>(ceil_div(sort_n / 2, 256)), 256, 0, st>>>(
+          keys, sort_n, k, j);
+      CK(cudaGetLastError());
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+    }
+    bitonic_smem_kernel<<<sblocks, kSortBlock, 0, st>>>(keys, k);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  perm_from_keys_kernel<<<static_cast<unsigned>(ceil_div(count, 256)), 256, 0, st>>>(keys, count,
+                                                                                      perm);
   CK(cudaGetLastError());
   g_launches.fetch_add(1, std::memory_order_relaxed);
 }
@@ -548,6 +633,9 @@ struct Ctx {
   unsigned char *rimg_x, *kimg_x, *rimg_y, *kimg_y;
   float *nrm_x, *nrm_y, *hy_x, *hy_y;
   float c2;       // 2 kappa / s^2
+  int *perm_x, *perm_y;         // sorted slot -> original index (NULL when unsorted)
+  uint64_t* sortkeys;
+  float *box_x, *box_y, *hmax_x, *hmax_y, *lse_x, *lse_y;
 };
 
 fs_status check_common(const fs_problem* p, void* ws, size_t ws_bytes, size_t* need_out,
@@ -584,6 +672,17 @@ void carve(Ctx& c, void* ws) {
     c.hy_x = reinterpret_cast<float*>(c.ws + c.L.off_hy_x);
     c.hy_y = reinterpret_cast<float*>(c.ws + c.L.off_hy_y);
   }
+  if (c.L.sorted) {
+    c.perm_x = reinterpret_cast<int*>(c.ws + c.L.off_perm_x);
+    c.perm_y = reinterpret_cast<int*>(c.ws + c.L.off_perm_y);
+    c.sortkeys = reinterpret_cast<uint64_t*>(c.ws + c.L.off_sortkeys);
+    c.box_x = reinterpret_cast<float*>(c.ws + c.L.off_box_x);
+    c.box_y = reinterpret_cast<float*>(c.ws + c.L.off_box_y);
+    c.hmax_x = reinterpret_cast<float*>(c.ws + c.L.off_hmax_x);
+    c.hmax_y = reinterpret_cast<float*>(c.ws + c.L.off_hmax_y);
+    c.lse_x = reinterpret_cast<float*>(c.ws + c.L.off_lse_x);
+    c.lse_y = reinterpret_cast<float*>(c.ws + c.L.off_lse_y);
+  }
 }
 
 unsigned* flags_ptr(double* scal) { return reinterpret_cast<unsigned*>(scal + kFlags); }
@@ -600,6 +699,20 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
   const fs_problem* p = c.p;
   c.use_tc = need_tc && c.L.Dtc > 0;
   CK(cudaMemsetAsync(c.scal, 0, kScalarDoubles * sizeof(double), c.st));
+  const int sdims = std::min(p->d, kSortDims);
+  if (c.L.sorted) {
+    // bounding box of both clouds: lo starts at +3.4e38, hi at -3.4e38 (as ordered ints)
+    int* box = reinterpret_cast<int*>(c.scal + kBox);
+    CK(cudaMemsetAsync(box, 0x7F, kSortDims * sizeof(int), c.st));
+    CK(cudaMemsetAsync(box + kSortDims, 0x80, kSortDims * sizeof(int), c.st));
+    dim3 gx(reduce_blocks(p->n, c.sms), sdims), gy(reduce_blocks(p->m, c.sms), sdims);
+    bbox_kernel<<<gx, 256, 0, c.st>>>(p->x, p->n, p->d, box, box + kSortDims);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    bbox_kernel<<<gy, 256, 0, c.st>>>(p->y, p->m, p->d, box, box + kSortDims);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
   if (c.use_tc) {
     unsigned* mx = reinterpret_cast<unsigned*>(c.scal + kMaxAbs);
     dim3 gx(reduce_blocks(p->n, c.sms), p->d), gy(reduce_blocks(p->m, c.sms), p->d);
@@ -636,7 +749,7 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
     CK(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
-  double host[kMaxAbs + 1];
+  double host[kBox + 3];  // through the bounding box (6 ints at kBox)
   CK(cudaMemcpyAsync(host, c.scal, sizeof(host), cudaMemcpyDeviceToHost, c.st));
   CK(cudaStreamSynchronize(c.st));
   unsigned flags;
@@ -648,9 +761,31 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
   if (!(c.ma > 0.0) || !(c.mb > 0.0)) return FS_ERR_ZERO_MASS;
   if (std::fabs(c.ma - c.mb) > 1e-5 * std::max(c.ma, c.mb)) return FS_ERR_MASS_MISMATCH;
 
+  if (c.L.sorted) {
+    // Morton order on the first three coordinates over the common bounding box.
+    int boxi[2 * kSortDims];
+    memcpy(boxi, &host[kBox], sizeof(boxi));
+    MortonFrame F{};
+    F.dims = sdims;
+    F.bits = sdims == 3 ? 10 : (sdims == 2 ? 16 : 30);
+    for (int k = 0; k < sdims; ++k) {
+      const float lo = ord_float(boxi[k]), hi = ord_float(boxi[kSortDims + k]);
+      F.lo[k] = lo;
+      F.scale[k] = hi > lo ? static_cast<float>(((1u << F.bits) - 1u) / (static_cast<double>(hi) - lo))
+                           : 0.0f;
+    }
+    sort_cloud(p->x, p->n, p->d, F, c.sortkeys, c.L.sort_n, c.perm_x, c.st);
+    sort_cloud(p->y, p->m, p->d, F, c.sortkeys, c.L.sort_n, c.perm_y, c.st);
+  }
   const float wu_x = static_cast<float>(1.0 / p->n), wu_y = static_cast<float>(1.0 / p->m);
-  FS_DISPATCH_D(c.L.D, launch_pack_d, p->x, p->n, p->d, p->a, wu_x, c.kx, c.lwx, c.L.px, c.st);
-  FS_DISPATCH_D(c.L.D, launch_pack_d, p->y, p->m, p->d, p->b, wu_y, c.ky, c.lwy, c.L.py, c.st);
+  FS_DISPATCH_D(c.L.D, launch_pack_d, p->x, p->n, p->d, p->a, wu_x, c.perm_x, c.kx, c.lwx, c.L.px,
+                c.st);
+  FS_DISPATCH_D(c.L.D, launch_pack_d, p->y, p->m, p->d, p->b, wu_y, c.perm_y, c.ky, c.lwy, c.L.py,
+                c.st);
+  if (c.L.sorted) {
+    FS_DISPATCH_D(c.L.D, launch_tile_box_d, c.kx, p->n, c.L.px / kPairPad, c.box_x, c.st);
+    FS_DISPATCH_D(c.L.D, launch_tile_box_d, c.ky, p->m, c.L.py / kPairPad, c.box_y, c.st);
+  }
   if (c.use_tc) {
     // Centre on the common mean (the cost is translation invariant) and scale by a power of
     // two that puts the largest centred coordinate near 2^14, well inside fp16 range.
@@ -711,9 +846,9 @@ void set_bias(Ctx& c, bool cloud_x, const float* pot) {
     return;
   }
   if (cloud_x)
-    FS_DISPATCH_D(c.L.D, launch_bias_d, c.kx, c.p->n, pot, c.lwx, c.kappa, c.st)
+    FS_DISPATCH_D(c.L.D, launch_bias_d, c.kx, c.p->n, pot, c.perm_x, c.lwx, c.kappa, c.st)
   else
-    FS_DISPATCH_D(c.L.D, launch_bias_d, c.ky, c.p->m, pot, c.lwy, c.kappa, c.st)
+    FS_DISPATCH_D(c.L.D, launch_bias_d, c.ky, c.p->m, pot, c.perm_y, c.lwy, c.kappa, c.st)
 }
 
 // One streaming pass with rows from cloud x (rows_x) or y, keys from the other cloud.
@@ -764,7 +899,7 @@ void run_pass_tc(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_
 }
 
 void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out, float* marg_out,
-              float* grad_out, double* acc) {
+              float* grad_out, double* acc, bool screen = false) {
   if (c.use_tc && kind != kGrad) {
     run_pass_tc(c, rows_x, kind, pot_in, pot_out, marg_out, acc);
     return;
@@ -801,6 +936,25 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
   P.part_l = c.part + static_cast<int64_t>(pl.n_splits) * pl.rows_pad;
   P.part_a = c.part + 2 * static_cast<int64_t>(pl.n_splits) * pl.rows_pad;
   P.err = err_ptr(c.scal);
+  int* dmin_slots = reinterpret_cast<int*>(c.scal + kDmin);
+  if (c.L.sorted) {
+    P.perm = rows_x ? c.perm_x : c.perm_y;
+    if (kind == kPot) {
+      // this pass writes the query cloud's biases: record their change and its LSE2
+      P.lse_out = rows_x ? c.lse_x : c.lse_y;
+      P.dmin_out = dmin_slots + (rows_x ? 0 : 1);
+      P.evaluated = reinterpret_cast<unsigned long long*>(c.scal + kEval);
+      CK(cudaMemsetAsync(P.dmin_out, 0x7F, sizeof(int), c.st));
+      if (screen) {
+        P.screen = 1;
+        P.key_box = rows_x ? c.box_y : c.box_x;
+        P.key_hmax = rows_x ? c.hmax_y : c.hmax_x;
+        P.key_dmin = dmin_slots + (rows_x ? 1 : 0);
+        P.lse_prev = rows_x ? c.lse_x : c.lse_y;
+        P.log2_keys = static_cast<float>(std::log2(static_cast<double>(rows_x ? p->m : p->n)));
+      }
+    }
+  }
   const double pairs = static_cast<double>(n_rows) * static_cast<double>(rows_x ? p->m : p->n);
   const int tk = grad ? kTGrad : (kind == kMarg ? kTMarg : kTLse);
   int ti = c.timer->begin();
@@ -811,14 +965,23 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
     FS_DISPATCH_D(c.L.D, launch_combine_d, P, grad, c.st);
     c.timer->end(ti, kTCombine, 0.0);
   }
+  if (c.L.sorted && kind == kPot) {
+    // largest bias per tile of the cloud just updated: the next pass screens against it
+    FS_DISPATCH_D(c.L.D, launch_tile_hmax_d, rows_x ? c.kx : c.ky, n_rows,
+                  (rows_x ? c.L.px : c.L.py) / kPairPad, rows_x ? c.hmax_x : c.hmax_y, c.st);
+  }
 }
 
 // Drains the stream and reads the kernels' error word.
 fs_status finish(Ctx& c) {
-  unsigned err = 0;
-  CK(cudaMemcpyAsync(&err, err_ptr(c.scal), sizeof(unsigned), cudaMemcpyDeviceToHost, c.st));
+  double tail[kEval - kErr + 1];
+  CK(cudaMemcpyAsync(tail, c.scal + kErr, sizeof(tail), cudaMemcpyDeviceToHost, c.st));
   CK(cudaStreamSynchronize(c.st));
-  c.timer->collect();
+  unsigned err;
+  unsigned long long evaluated;
+  memcpy(&err, &tail[0], sizeof(unsigned));
+  memcpy(&evaluated, &tail[kEval - kErr], sizeof(evaluated));
+  c.timer->collect(static_cast<double>(evaluated));
   return err ? FS_ERR_TIMEOUT : FS_OK;
 }
 
@@ -866,9 +1029,11 @@ fs_status potentials_impl(const fs_problem* p, int32_t n_iters, const float* g_i
     fs_status r = prepare_all(c, pots, true);
     if (r != FS_OK) return r;
     set_bias(c, false, g_init);
+    // From the second iteration on every row has a previous LSE2 and the keys a recorded
+    // bias change, so the passes can screen key tiles.
     for (int32_t it = 0; it < n_iters; ++it) {
-      run_pass(c, true, kPot, nullptr, f, nullptr, nullptr, nullptr);   // f <- F(g)
-      run_pass(c, false, kPot, nullptr, g, nullptr, nullptr, nullptr);  // g <- G(f)
+      run_pass(c, true, kPot, nullptr, f, nullptr, nullptr, nullptr, it > 0);   // f <- F(g)
+      run_pass(c, false, kPot, nullptr, g, nullptr, nullptr, nullptr, it > 0);  // g <- G(f)
     }
     return finish(c);
   });

@@ -34,6 +34,7 @@
 #include <cfloat>
 #include <cmath>
 #include "fs_device.cuh"
+#include "fs_sort.cuh"
 
 namespace fs {
 
@@ -80,7 +81,23 @@ struct PassParams {
   // cloud (written instead of the packed-key slot) and its centred squared norms
   float* hy_out;
   const float* nrm;
+  // spatially sorted clouds: sorted row -> original index of the query cloud (NULL: identity)
+  const int* perm;
+  // block screening (potential passes after the first two)
+  int32_t screen;           // 1: skip key tiles whose every term is provably negligible
+  const float* key_box;     // [tile][2D]: bounding box of each 256-point key tile
+  const float* key_hmax;    // [tile]: largest key bias H of each key tile
+  const int* key_dmin;      // ordered int: smallest change of the key biases since the last pass
+  const float* lse_prev;    // LSE2 of every query row in its previous pass (sorted order)
+  float log2_keys;          // log2(number of keys)
+  float* lse_out;           // kPot: LSE2 of every query row (sorted order)
+  int* dmin_out;            // kPot: ordered int, smallest change of the H this pass writes
+  unsigned long long* evaluated;  // pairs evaluated after screening
 };
+
+constexpr int kScreenTile = 256;      // points per screening tile (= kPairPad pairs)
+constexpr int kScreenMaxTiles = 4096; // tiles one CTA can screen (list in shared memory)
+constexpr float kSkipMargin = 150.0f; // skipped terms are below 2^-150 of the row's largest
 
 // Offset of coordinate slot k (k == D is the bias H) of point i in packed keys.
 template <int D>
@@ -92,23 +109,32 @@ __device__ __forceinline__ int64_t key_slot(int64_t i, int k) {
 
 // kPot: the new potential and the bias this row carries as a key into the next pass:
 //   pot_i = -LSE2_i / kappa,   H_i = kappa pot_i + log2 w_i = log2 w_i - LSE2_i.
+// Returns the change of the row's key bias (new - previous), for the screening bound.
 template <int D>
-__device__ __forceinline__ void finish_pot(const PassParams& P, int64_t i, double lse2) {
-  P.pot_out[i] = static_cast<float>(-lse2 * P.eps_ln2);
+__device__ __forceinline__ float finish_pot(const PassParams& P, int64_t i, double lse2) {
+  const int64_t oi = P.perm ? P.perm[i] : i;
+  P.pot_out[oi] = static_cast<float>(-lse2 * P.eps_ln2);
+  if (P.lse_out) P.lse_out[i] = static_cast<float>(lse2);
   const double h = static_cast<double>(P.lw[i]) - lse2;
-  if (P.hy_out)
+  if (P.hy_out) {
     P.hy_out[i] = static_cast<float>(h - P.kappa * static_cast<double>(P.nrm[i]));
-  else
-    P.qkeys[key_slot<D>(i, D)] = static_cast<float>(h);
+    return 0.0f;
+  }
+  const int64_t slot = key_slot<D>(i, D);
+  const float hn = static_cast<float>(h);
+  const float delta = hn - P.qkeys[slot];
+  P.qkeys[slot] = hn;
+  return delta;
 }
 
 // kMarg: plan marginal r_i = w_i 2^(kappa pot_i + LSE2_i) = w_i exp((pot_i - F_i)/eps).
 __device__ __forceinline__ void finish_marg(const PassParams& P, int64_t i, double lse2,
                                             double& dev, double& mass) {
-  const double w = P.w ? static_cast<double>(P.w[i]) : static_cast<double>(P.w_uniform);
+  const int64_t oi = P.perm ? P.perm[i] : i;
+  const double w = P.w ? static_cast<double>(P.w[oi]) : static_cast<double>(P.w_uniform);
   double r = 0.0;
-  if (w > 0.0) r = w * exp2(P.kappa * static_cast<double>(P.pot_in[i]) + lse2);
-  if (P.marg_out) P.marg_out[i] = static_cast<float>(r);
+  if (w > 0.0) r = w * exp2(P.kappa * static_cast<double>(P.pot_in[oi]) + lse2);
+  if (P.marg_out) P.marg_out[oi] = static_cast<float>(r);
   dev = fabs(r - w);
   mass = r;
 }
@@ -116,9 +142,17 @@ __device__ __forceinline__ void finish_marg(const PassParams& P, int64_t i, doub
 // kGrad: grad_i = 2 w_i (x_i - T_i) = 2 w_i sum_j p_ij (x_i - y_j) / sum_j p_ij.
 __device__ __forceinline__ void finish_grad(const PassParams& P, int64_t i, const float* dsum,
                                             float l) {
-  const float w = P.w ? P.w[i] : P.w_uniform;
+  const int64_t oi = P.perm ? P.perm[i] : i;
+  const float w = P.w ? P.w[oi] : P.w_uniform;
   const float s = 2.0f * w / l;
-  for (int k = 0; k < P.d_real; ++k) P.grad_out[i * P.d_real + k] = s * dsum[k];
+  for (int k = 0; k < P.d_real; ++k) P.grad_out[oi * P.d_real + k] = s * dsum[k];
+}
+
+// Warp-wide minimum of the bias changes, one atomic per warp (NaN never wins fminf).
+__device__ __forceinline__ void reduce_dmin(float v, int* out) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((threadIdx.x & 31) == 0 && out) atomicMin(out, float_ord(v));
 }
 
 // Block-wide sum/max of the marginal deviations, then one atomic per block.
@@ -189,14 +223,6 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
   }
-  __syncthreads();
-  if (tid == 0) {
-    for (int s = 0; s < kStages && s < n_tiles; ++s) {
-      mbar_expect_tx(&bars[s], stage_bytes);
-      bulk_g2s(stages + s * stage_floats, key_src + static_cast<int64_t>(s) * stage_floats,
-               stage_bytes, &bars[s]);
-    }
-  }
 
   // Row state: coordinates duplicated into both lanes of a packed register; the running
   // offset m (log2 units), `base` (m, or 0 while no column has set it) and mk = base/kappa
@@ -223,11 +249,129 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     for (int k = 0; k < NA; ++k) A[r][k] = pk(0.0f, 0.0f);
   }
 
+  // Block screening. A lower bound on each row's largest exponent this pass is its previous
+  // LSE2 plus the smallest change of the key biases since, minus log2(#keys) (the largest
+  // term is at least the sum over the count). A key tile is skipped when its largest bias
+  // minus kappa times the squared distance between the CTA's row box and the tile's box lies
+  // more than kSkipMargin below the smallest of those bounds: each skipped term is then below
+  // 2^-kSkipMargin of its row's largest term. The kept tiles form a list in shared memory.
+  __shared__ unsigned short tlist[kScreenMaxTiles];
+  __shared__ unsigned smask[kScreenMaxTiles / 32];
+  __shared__ int s_box[2 * D];
+  __shared__ int s_mlb, s_count;
+  int n_work = n_tiles;
+  const bool screening = P.screen && P.tile_pairs == kScreenTile / 2 && n_tiles <= kScreenMaxTiles;
+  if (screening) {
+    const int nwords = (n_tiles + 31) / 32;
+    for (int w = tid; w < nwords; w += NT) smask[w] = 0u;
+    if (tid < D) {
+      s_box[tid] = 0x7FFFFFFF;
+      s_box[D + tid] = static_cast<int>(0x80000000u);
+    }
+    if (tid == 0) s_mlb = 0x7FFFFFFF;
+    __syncthreads();
+    const float dmin = ord_float(*P.key_dmin);
+    float lo[D], hi[D], mlb = INFINITY;
+#pragma unroll
+    for (int k = 0; k < D; ++k) {
+      lo[k] = INFINITY;
+      hi[k] = -INFINITY;
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t i = row0 + r * NT + tid;
+      if (i < P.n_rows) {
+#pragma unroll
+        for (int k = 0; k < D; ++k) {
+          float c0, c1;
+          upk(X[r][k], c0, c1);
+          lo[k] = fminf(lo[k], c0);
+          hi[k] = fmaxf(hi[k], c0);
+        }
+        mlb = fminf(mlb, P.lse_prev[i] + dmin - P.log2_keys);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mlb = fminf(mlb, __shfl_xor_sync(0xffffffffu, mlb, o));
+#pragma unroll
+      for (int k = 0; k < D; ++k) {
+        lo[k] = fminf(lo[k], __shfl_xor_sync(0xffffffffu, lo[k], o));
+        hi[k] = fmaxf(hi[k], __shfl_xor_sync(0xffffffffu, hi[k], o));
+      }
+    }
+    if ((tid & 31) == 0) {
+      atomicMin(&s_mlb, float_ord(mlb));
+#pragma unroll
+      for (int k = 0; k < D; ++k) {
+        atomicMin(&s_box[k], float_ord(lo[k]));
+        atomicMax(&s_box[D + k], float_ord(hi[k]));
+      }
+    }
+    __syncthreads();
+    const float mlb_min = ord_float(s_mlb);
+    const int64_t T0 = p_begin / (kScreenTile / 2);
+    for (int tt = tid; tt < n_tiles; tt += NT) {
+      const float* bx = P.key_box + (T0 + tt) * 2 * D;
+      float d2 = 0.0f;
+#pragma unroll
+      for (int k = 0; k < D; ++k) {
+        const float gap = fmaxf(fmaxf(bx[k] - ord_float(s_box[D + k]), ord_float(s_box[k]) - bx[D + k]), 0.0f);
+        d2 = fmaf(gap, gap, d2);
+      }
+      const float ub = P.key_hmax[T0 + tt] - P.kappa_f * d2;
+      if (ub >= mlb_min - kSkipMargin) atomicOr(&smask[tt >> 5], 1u << (tt & 31));
+    }
+    __syncthreads();
+    if (tid < 32) {
+      int running = 0;
+      for (int w0 = 0; w0 < nwords; w0 += 32) {
+        const int w = w0 + tid;
+        unsigned word = w < nwords ? smask[w] : 0u;
+        const int cnt = __popc(word);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (tid >= o) incl += v;
+        }
+        int pos = running + incl - cnt;
+        while (word) {
+          const int b = __ffs(word) - 1;
+          tlist[pos++] = static_cast<unsigned short>(w * 32 + b);
+          word &= word - 1u;
+        }
+        running += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (tid == 0) {
+        s_count = running;
+        if (P.evaluated)
+          atomicAdd(P.evaluated, static_cast<unsigned long long>(running) * kScreenTile * (R * NT));
+      }
+    }
+    __syncthreads();
+    n_work = s_count;
+  } else {
+    __syncthreads();
+    if (tid == 0 && P.evaluated)
+      atomicAdd(P.evaluated, static_cast<unsigned long long>(n_tiles) * P.tile_pairs * 2 * (R * NT));
+  }
+  auto tile_src = [&](int e) -> const float* {
+    const int tt = screening ? static_cast<int>(tlist[e]) : e;
+    return key_src + static_cast<int64_t>(tt) * stage_floats;
+  };
+  if (tid == 0) {
+    for (int s = 0; s < kStages && s < n_work; ++s) {
+      mbar_expect_tx(&bars[s], stage_bytes);
+      bulk_g2s(stages + s * stage_floats, tile_src(s), stage_bytes, &bars[s]);
+    }
+  }
+
   // One CTA barrier per tile: after it every thread has finished the previous tile, so its
   // stage can be refilled, and a timed-out wait anywhere in the CTA is visible to all.
   int t = 0;
   bool aborted = false;
-  for (; t < n_tiles; ++t) {
+  for (; t < n_work; ++t) {
     const int st = t % kStages;
     const uint32_t parity = static_cast<uint32_t>(t / kStages) & 1u;
     const bool ok = mbar_wait_bounded(&bars[st], parity);
@@ -235,13 +379,11 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       aborted = true;
       break;
     }
-    if (tid == 0 && t >= 1 && t - 1 + kStages < n_tiles) {
+    if (tid == 0 && t >= 1 && t - 1 + kStages < n_work) {
       const int ps = (t - 1) % kStages;
       fence_proxy_async_smem();
       mbar_expect_tx(&bars[ps], stage_bytes);
-      bulk_g2s(stages + ps * stage_floats,
-               key_src + static_cast<int64_t>(t - 1 + kStages) * stage_floats, stage_bytes,
-               &bars[ps]);
+      bulk_g2s(stages + ps * stage_floats, tile_src(t - 1 + kStages), stage_bytes, &bars[ps]);
     }
     const float* tile = stages + st * stage_floats;
     for (int pg = 0; pg < P.tile_pairs; pg += G) {
@@ -315,7 +457,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     // barrier of tile t, which was not passed).
     if (tid == 0) {
       atomicOr(P.err, kErrTimeout);
-      for (int u = t; u < n_tiles && u < t + kStages - 1; ++u)
+      for (int u = t; u < n_work && u < t + kStages - 1; ++u)
         (void)mbar_wait_bounded(&bars[u % kStages], static_cast<uint32_t>(u / kStages) & 1u);
     }
     return;
@@ -323,6 +465,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
 
   if (P.n_splits == 1) {
     double dev_sum = 0.0, dev_max = 0.0, mass = 0.0;
+    float dmin = INFINITY;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int64_t i = row0 + r * NT + tid;
@@ -342,7 +485,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       } else {
         const double lse2 = static_cast<double>(m[r]) + log2(static_cast<double>(l));
         if (P.kind == kPot) {
-          finish_pot<D>(P, i, lse2);
+          dmin = fminf(dmin, finish_pot<D>(P, i, lse2));
         } else {
           double dv, ms;
           finish_marg(P, i, lse2, dv, ms);
@@ -353,6 +496,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       }
     }
     if (!GRAD && P.kind == kMarg) block_reduce_marg(dev_sum, dev_max, mass, P.acc);
+    if (!GRAD && P.kind == kPot) reduce_dmin(dmin, P.dmin_out);
   } else {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -381,6 +525,7 @@ template <int D, bool GRAD>
 __global__ void __launch_bounds__(256) combine_kernel(const PassParams P) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   double dev = 0.0, mass = 0.0;
+  float dmin = INFINITY;
   if (i < P.n_rows) {
     float mx = -INFINITY;
     for (int s = 0; s < P.n_splits; ++s) mx = fmaxf(mx, P.part_m[s * P.rows_pad + i]);
@@ -404,13 +549,14 @@ __global__ void __launch_bounds__(256) combine_kernel(const PassParams P) {
     } else {
       const double lse2 = static_cast<double>(mx) + log2(l);
       if (P.kind == kPot) {
-        finish_pot<D>(P, i, lse2);
+        dmin = finish_pot<D>(P, i, lse2);
       } else {
         finish_marg(P, i, lse2, dev, mass);
       }
     }
   }
   if (!GRAD && P.kind == kMarg) block_reduce_marg(dev, dev, mass, P.acc);
+  if (!GRAD && P.kind == kPot) reduce_dmin(dmin, P.dmin_out);
 }
 
 // ---- preparation kernels --------------------------------------------------------------
@@ -460,16 +606,18 @@ __global__ void __launch_bounds__(256) check_finite_kernel(const float* v, int64
 // all padded points of one cloud.
 template <int D>
 __global__ void __launch_bounds__(256) pack_kernel(const float* pts, int64_t count, int32_t d_real,
-                                                   const float* w, float w_uniform, float* keys,
-                                                   float* lw, int64_t pairs_pad) {
+                                                   const float* w, float w_uniform,
+                                                   const int* perm, float* keys, float* lw,
+                                                   int64_t pairs_pad) {
   constexpr int KP = key_pair_floats(D);
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (j >= 2 * pairs_pad) return;
   const int64_t base = (j >> 1) * KP + (j & 1);
   if (j < count) {
+    const int64_t src = perm ? perm[j] : j;  // slot j holds point perm[j]
 #pragma unroll
-    for (int k = 0; k < D; ++k) keys[base + 2 * k] = k < d_real ? pts[j * d_real + k] : 0.0f;
-    const float wj = w ? w[j] : w_uniform;
+    for (int k = 0; k < D; ++k) keys[base + 2 * k] = k < d_real ? pts[src * d_real + k] : 0.0f;
+    const float wj = w ? w[src] : w_uniform;
     lw[j] = wj > 0.0f ? static_cast<float>(log2(static_cast<double>(wj))) : kLogZero;
   } else {
 #pragma unroll
@@ -485,10 +633,11 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* pts, int64_t cou
 // Key bias of every real point: H_j = kappa pot_j + log2 w_j (pot = 0 if NULL).
 template <int D>
 __global__ void __launch_bounds__(256) key_bias_kernel(float* keys, int64_t count, const float* pot,
-                                                       const float* lw, double kappa) {
+                                                       const int* perm, const float* lw,
+                                                       double kappa) {
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (j >= count) return;
-  const double p = pot ? static_cast<double>(pot[j]) : 0.0;
+  const double p = pot ? static_cast<double>(pot[perm ? perm[j] : j]) : 0.0;
   keys[key_slot<D>(j, D)] = static_cast<float>(kappa * p + static_cast<double>(lw[j]));
 }
 
