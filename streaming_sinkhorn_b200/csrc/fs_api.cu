@@ -67,12 +67,14 @@ class Timer {
     rec_[idx].pairs = pairs;
     CK(cudaEventRecord(rec_[idx].stop, stream_));
   }
-  // Call after the stream has been synchronised; `evaluated` = pairs the potential passes
-  // of this call evaluated after screening.
-  void collect(double evaluated) {
+  // Call after the stream has been synchronised; `evaluated[k]` = pairs the sorted passes
+  // of timed kind k evaluated in this call after screening.
+  void collect(const unsigned long long* evaluated) {
     if (!on_) return;
     std::lock_guard<std::mutex> lk(g_timing_mu);
-    g_timing.lse_pass.evaluated += evaluated;
+    g_timing.lse_pass.evaluated += static_cast<double>(evaluated[kTLse]);
+    g_timing.grad_pass.evaluated += static_cast<double>(evaluated[kTGrad]);
+    g_timing.marg_pass.evaluated += static_cast<double>(evaluated[kTMarg]);
     for (auto& t : rec_) {
       float ms = 0.f;
       CK(cudaEventElapsedTime(&ms, t.start, t.stop));
@@ -266,7 +268,7 @@ constexpr int kErr = 141;     // unsigned
 constexpr int kMaxAbs = 142;  // unsigned: float bits of the largest |coordinate| of x and y
 constexpr int kBox = 144;     // ints: ordered lo[3], hi[3] of the first three coordinates
 constexpr int kDmin = 147;    // ints: ordered smallest key-bias change of x, of y
-constexpr int kEval = 148;    // uint64: pairs evaluated by screened potential passes
+constexpr int kEval = 148;    // uint64[3]: pairs evaluated by sorted passes, by TimedKind
 
 struct Layout {
   int D;       // padded dimension of the FMA path
@@ -849,6 +851,11 @@ void set_bias(Ctx& c, bool cloud_x, const float* pot) {
     FS_DISPATCH_D(c.L.D, launch_bias_d, c.kx, c.p->n, pot, c.perm_x, c.lwx, c.kappa, c.st)
   else
     FS_DISPATCH_D(c.L.D, launch_bias_d, c.ky, c.p->m, pot, c.perm_y, c.lwy, c.kappa, c.st)
+  if (c.L.sorted) {
+    // largest bias per tile, for the screening of the passes that take this cloud as keys
+    FS_DISPATCH_D(c.L.D, launch_tile_hmax_d, cloud_x ? c.kx : c.ky, cloud_x ? c.p->n : c.p->m,
+                  (cloud_x ? c.L.px : c.L.py) / kPairPad, cloud_x ? c.hmax_x : c.hmax_y, c.st);
+  }
 }
 
 // One streaming pass with rows from cloud x (rows_x) or y, keys from the other cloud.
@@ -898,8 +905,10 @@ void run_pass_tc(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_
   }
 }
 
+// Sorted FMA passes screen key tiles (see the kernel); `history` adds the bound from the
+// rows' previous LSE2 and the keys' bias change, which exists from a solve's second iteration.
 void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out, float* marg_out,
-              float* grad_out, double* acc, bool screen = false) {
+              float* grad_out, double* acc, bool history = false) {
   if (c.use_tc && kind != kGrad) {
     run_pass_tc(c, rows_x, kind, pot_in, pot_out, marg_out, acc);
     return;
@@ -937,18 +946,19 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
   P.part_a = c.part + 2 * static_cast<int64_t>(pl.n_splits) * pl.rows_pad;
   P.err = err_ptr(c.scal);
   int* dmin_slots = reinterpret_cast<int*>(c.scal + kDmin);
+  const int tk = grad ? kTGrad : (kind == kMarg ? kTMarg : kTLse);
   if (c.L.sorted) {
     P.perm = rows_x ? c.perm_x : c.perm_y;
+    P.screen = 1;
+    P.key_box = rows_x ? c.box_y : c.box_x;
+    P.key_hmax = rows_x ? c.hmax_y : c.hmax_x;
+    P.evaluated = reinterpret_cast<unsigned long long*>(c.scal + kEval + tk);
     if (kind == kPot) {
       // this pass writes the query cloud's biases: record their change and its LSE2
       P.lse_out = rows_x ? c.lse_x : c.lse_y;
       P.dmin_out = dmin_slots + (rows_x ? 0 : 1);
-      P.evaluated = reinterpret_cast<unsigned long long*>(c.scal + kEval);
       CK(cudaMemsetAsync(P.dmin_out, 0x7F, sizeof(int), c.st));
-      if (screen) {
-        P.screen = 1;
-        P.key_box = rows_x ? c.box_y : c.box_x;
-        P.key_hmax = rows_x ? c.hmax_y : c.hmax_x;
+      if (history) {
         P.key_dmin = dmin_slots + (rows_x ? 1 : 0);
         P.lse_prev = rows_x ? c.lse_x : c.lse_y;
         P.log2_keys = static_cast<float>(std::log2(static_cast<double>(rows_x ? p->m : p->n)));
@@ -956,7 +966,6 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
     }
   }
   const double pairs = static_cast<double>(n_rows) * static_cast<double>(rows_x ? p->m : p->n);
-  const int tk = grad ? kTGrad : (kind == kMarg ? kTMarg : kTLse);
   int ti = c.timer->begin();
   FS_DISPATCH_D(c.L.D, launch_pass_d, P, pl, grad, c.st);
   c.timer->end(ti, tk, pairs);
@@ -974,14 +983,14 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
 
 // Drains the stream and reads the kernels' error word.
 fs_status finish(Ctx& c) {
-  double tail[kEval - kErr + 1];
+  double tail[kEval + 3 - kErr];
   CK(cudaMemcpyAsync(tail, c.scal + kErr, sizeof(tail), cudaMemcpyDeviceToHost, c.st));
   CK(cudaStreamSynchronize(c.st));
   unsigned err;
-  unsigned long long evaluated;
+  unsigned long long evaluated[3];
   memcpy(&err, &tail[0], sizeof(unsigned));
-  memcpy(&evaluated, &tail[kEval - kErr], sizeof(evaluated));
-  c.timer->collect(static_cast<double>(evaluated));
+  memcpy(evaluated, &tail[kEval - kErr], sizeof(evaluated));
+  c.timer->collect(evaluated);
   return err ? FS_ERR_TIMEOUT : FS_OK;
 }
 

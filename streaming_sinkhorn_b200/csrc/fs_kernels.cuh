@@ -249,29 +249,48 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     for (int k = 0; k < NA; ++k) A[r][k] = pk(0.0f, 0.0f);
   }
 
-  // Block screening. A lower bound on each row's largest exponent this pass is its previous
-  // LSE2 plus the smallest change of the key biases since, minus log2(#keys) (the largest
-  // term is at least the sum over the count). A key tile is skipped when its largest bias
-  // minus kappa times the squared distance between the CTA's row box and the tile's box lies
-  // more than kSkipMargin below the smallest of those bounds: each skipped term is then below
-  // 2^-kSkipMargin of its row's largest term. The kept tiles form a list in shared memory.
+  // Block screening (sorted clouds). Every pass first processes an anchor tile: the key
+  // tile whose exponents have the largest upper bound (its largest bias minus kappa times
+  // the squared distance between the CTA's row box and the tile's box). The running offset
+  // it leaves is a value some term of the row reaches, hence a lower bound on the row's
+  // largest exponent; a potential pass with history also has the bound "previous LSE2 plus
+  // the smallest change of the key biases, minus log2(#keys)" (the largest term is at least
+  // the sum over the count). Every other tile whose upper bound lies more than kSkipMargin
+  // below the smallest of those bounds over the CTA's rows is skipped: each omitted term is
+  // under 2^-kSkipMargin of its row's largest. The kept tiles form a list in shared memory.
   __shared__ unsigned short tlist[kScreenMaxTiles];
   __shared__ unsigned smask[kScreenMaxTiles / 32];
   __shared__ int s_box[2 * D];
   __shared__ int s_mlb, s_count;
+  __shared__ unsigned long long s_best;
+  const bool screening = P.screen && P.tile_pairs == kScreenTile / 2 && n_tiles > 1 &&
+                         n_tiles <= kScreenMaxTiles;
+  const bool history = screening && P.lse_prev && P.key_dmin;
+  const int64_t T0 = p_begin / (kScreenTile / 2);
   int n_work = n_tiles;
-  const bool screening = P.screen && P.tile_pairs == kScreenTile / 2 && n_tiles <= kScreenMaxTiles;
+  // Upper bound of the exponents of key tile tt for any row of this CTA.
+  auto tile_ub = [&](int tt) -> float {
+    const float* bx = P.key_box + (T0 + tt) * 2 * D;
+    float d2 = 0.0f;
+#pragma unroll
+    for (int k = 0; k < D; ++k) {
+      const float gap =
+          fmaxf(fmaxf(bx[k] - ord_float(s_box[D + k]), ord_float(s_box[k]) - bx[D + k]), 0.0f);
+      d2 = fmaf(gap, gap, d2);
+    }
+    return P.key_hmax[T0 + tt] - P.kappa_f * d2;
+  };
   if (screening) {
-    const int nwords = (n_tiles + 31) / 32;
-    for (int w = tid; w < nwords; w += NT) smask[w] = 0u;
     if (tid < D) {
       s_box[tid] = 0x7FFFFFFF;
       s_box[D + tid] = static_cast<int>(0x80000000u);
     }
-    if (tid == 0) s_mlb = 0x7FFFFFFF;
+    if (tid == 0) {
+      s_mlb = 0x7FFFFFFF;
+      s_best = 0ull;
+    }
     __syncthreads();
-    const float dmin = ord_float(*P.key_dmin);
-    float lo[D], hi[D], mlb = INFINITY;
+    float lo[D], hi[D];
 #pragma unroll
     for (int k = 0; k < D; ++k) {
       lo[k] = INFINITY;
@@ -288,12 +307,10 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
           lo[k] = fminf(lo[k], c0);
           hi[k] = fmaxf(hi[k], c0);
         }
-        mlb = fminf(mlb, P.lse_prev[i] + dmin - P.log2_keys);
       }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      mlb = fminf(mlb, __shfl_xor_sync(0xffffffffu, mlb, o));
 #pragma unroll
       for (int k = 0; k < D; ++k) {
         lo[k] = fminf(lo[k], __shfl_xor_sync(0xffffffffu, lo[k], o));
@@ -301,7 +318,6 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       }
     }
     if ((tid & 31) == 0) {
-      atomicMin(&s_mlb, float_ord(mlb));
 #pragma unroll
       for (int k = 0; k < D; ++k) {
         atomicMin(&s_box[k], float_ord(lo[k]));
@@ -309,48 +325,24 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       }
     }
     __syncthreads();
-    const float mlb_min = ord_float(s_mlb);
-    const int64_t T0 = p_begin / (kScreenTile / 2);
+    // anchor: largest upper bound, ties to the lower tile (key = ordered ub, then ~index)
+    unsigned long long best = 0ull;
     for (int tt = tid; tt < n_tiles; tt += NT) {
-      const float* bx = P.key_box + (T0 + tt) * 2 * D;
-      float d2 = 0.0f;
-#pragma unroll
-      for (int k = 0; k < D; ++k) {
-        const float gap = fmaxf(fmaxf(bx[k] - ord_float(s_box[D + k]), ord_float(s_box[k]) - bx[D + k]), 0.0f);
-        d2 = fmaf(gap, gap, d2);
-      }
-      const float ub = P.key_hmax[T0 + tt] - P.kappa_f * d2;
-      if (ub >= mlb_min - kSkipMargin) atomicOr(&smask[tt >> 5], 1u << (tt & 31));
+      const unsigned ub = static_cast<unsigned>(float_ord(tile_ub(tt))) ^ 0x80000000u;
+      const unsigned long long key =
+          (static_cast<unsigned long long>(ub) << 32) | static_cast<unsigned>(0xFFFF - tt);
+      best = best > key ? best : key;
     }
-    __syncthreads();
-    if (tid < 32) {
-      int running = 0;
-      for (int w0 = 0; w0 < nwords; w0 += 32) {
-        const int w = w0 + tid;
-        unsigned word = w < nwords ? smask[w] : 0u;
-        const int cnt = __popc(word);
-        int incl = cnt;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (tid >= o) incl += v;
-        }
-        int pos = running + incl - cnt;
-        while (word) {
-          const int b = __ffs(word) - 1;
-          tlist[pos++] = static_cast<unsigned short>(w * 32 + b);
-          word &= word - 1u;
-        }
-        running += __shfl_sync(0xffffffffu, incl, 31);
-      }
-      if (tid == 0) {
-        s_count = running;
-        if (P.evaluated)
-          atomicAdd(P.evaluated, static_cast<unsigned long long>(running) * kScreenTile * (R * NT));
-      }
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+      best = best > other ? best : other;
     }
+    if ((tid & 31) == 0) atomicMax(&s_best, best);
     __syncthreads();
-    n_work = s_count;
+    if (tid == 0) tlist[0] = static_cast<unsigned short>(0xFFFF - (s_best & 0xFFFFull));
+    __syncthreads();
+    n_work = 1;  // the anchor; the kept tiles are appended once it is processed
   } else {
     __syncthreads();
     if (tid == 0 && P.evaluated)
@@ -360,32 +352,9 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     const int tt = screening ? static_cast<int>(tlist[e]) : e;
     return key_src + static_cast<int64_t>(tt) * stage_floats;
   };
-  if (tid == 0) {
-    for (int s = 0; s < kStages && s < n_work; ++s) {
-      mbar_expect_tx(&bars[s], stage_bytes);
-      bulk_g2s(stages + s * stage_floats, tile_src(s), stage_bytes, &bars[s]);
-    }
-  }
 
-  // One CTA barrier per tile: after it every thread has finished the previous tile, so its
-  // stage can be refilled, and a timed-out wait anywhere in the CTA is visible to all.
-  int t = 0;
-  bool aborted = false;
-  for (; t < n_work; ++t) {
-    const int st = t % kStages;
-    const uint32_t parity = static_cast<uint32_t>(t / kStages) & 1u;
-    const bool ok = mbar_wait_bounded(&bars[st], parity);
-    if (__syncthreads_or(!ok)) {
-      aborted = true;
-      break;
-    }
-    if (tid == 0 && t >= 1 && t - 1 + kStages < n_work) {
-      const int ps = (t - 1) % kStages;
-      fence_proxy_async_smem();
-      mbar_expect_tx(&bars[ps], stage_bytes);
-      bulk_g2s(stages + ps * stage_floats, tile_src(t - 1 + kStages), stage_bytes, &bars[ps]);
-    }
-    const float* tile = stages + st * stage_floats;
+  // Online max/sum of this thread's rows over one key tile in shared memory.
+  auto process_tile = [&](const float* tile) {
     for (int pg = 0; pg < P.tile_pairs; pg += G) {
       u64 tv[R][G];
 #pragma unroll
@@ -449,6 +418,98 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
         }
       }
     }
+  };
+
+  // After the anchor: the lower bounds, the screen of the other tiles, the list, and the
+  // first copies of the kept tiles.
+  auto screen_rest = [&]() {
+    const int anchor = tlist[0];
+    const float dmin = history ? ord_float(*P.key_dmin) : 0.0f;
+    float mlb = INFINITY;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t i = row0 + r * NT + tid;
+      if (i < P.n_rows) {
+        float b = m[r];
+        if (history) b = fmaxf(b, P.lse_prev[i] + dmin - P.log2_keys);
+        mlb = fminf(mlb, b);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mlb = fminf(mlb, __shfl_xor_sync(0xffffffffu, mlb, o));
+    const int nwords = (n_tiles + 31) / 32;
+    for (int w = tid; w < nwords; w += NT) smask[w] = 0u;
+    if ((tid & 31) == 0) atomicMin(&s_mlb, float_ord(mlb));
+    __syncthreads();
+    const float mlb_min = ord_float(s_mlb);
+    for (int tt = tid; tt < n_tiles; tt += NT) {
+      if (tt != anchor && tile_ub(tt) >= mlb_min - kSkipMargin)
+        atomicOr(&smask[tt >> 5], 1u << (tt & 31));
+    }
+    __syncthreads();
+    if (tid < 32) {
+      int running = 1;  // slot 0 holds the anchor
+      for (int w0 = 0; w0 < nwords; w0 += 32) {
+        const int w = w0 + tid;
+        unsigned word = w < nwords ? smask[w] : 0u;
+        const int cnt = __popc(word);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (tid >= o) incl += v;
+        }
+        int pos = running + incl - cnt;
+        while (word) {
+          const int bit = __ffs(word) - 1;
+          tlist[pos++] = static_cast<unsigned short>(w * 32 + bit);
+          word &= word - 1u;
+        }
+        running += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (tid == 0) {
+        s_count = running;
+        if (P.evaluated)
+          atomicAdd(P.evaluated, static_cast<unsigned long long>(running) * kScreenTile * (R * NT));
+      }
+    }
+    __syncthreads();
+    n_work = s_count;
+    if (tid == 0) {
+      for (int e = 1; e < kStages && e < n_work; ++e) {
+        mbar_expect_tx(&bars[e], stage_bytes);
+        bulk_g2s(stages + e * stage_floats, tile_src(e), stage_bytes, &bars[e]);
+      }
+    }
+  };
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages && s < n_work; ++s) {
+      mbar_expect_tx(&bars[s], stage_bytes);
+      bulk_g2s(stages + s * stage_floats, tile_src(s), stage_bytes, &bars[s]);
+    }
+  }
+
+  // One CTA barrier per tile: after it every thread has finished the previous tile, so its
+  // stage can be refilled, and a timed-out wait anywhere in the CTA is visible to all.
+  int t = 0;
+  bool aborted = false;
+  for (; t < n_work; ++t) {
+    const int st = t % kStages;
+    const uint32_t parity = static_cast<uint32_t>(t / kStages) & 1u;
+    const bool ok = mbar_wait_bounded(&bars[st], parity);
+    if (__syncthreads_or(!ok)) {
+      aborted = true;
+      break;
+    }
+    if (tid == 0 && t >= 1 && t - 1 + kStages < n_work) {
+      const int ps = (t - 1) % kStages;
+      fence_proxy_async_smem();
+      mbar_expect_tx(&bars[ps], stage_bytes);
+      bulk_g2s(stages + ps * stage_floats, tile_src(t - 1 + kStages), stage_bytes, &bars[ps]);
+    }
+    process_tile(stages + st * stage_floats);
+    if (screening && t == 0) screen_rest();
   }
 
   if (aborted) {
