@@ -194,14 +194,15 @@ typedef struct {
   double total_ms;  /* their summed device durations */
   double pairs;     /* (row, column) pairs the problem defines for them: N * M per pass */
   double evaluated; /* pairs actually evaluated (exponentials issued, padding included)
-                       after block screening; filled for the potential passes */
+                       after block screening; filled for passes on sorted clouds (d <= 16) */
 } fs_timing_entry;
 
 typedef struct {
   fs_timing_entry lse_pass;  /* potential-update passes (f and g half-iterations) */
   fs_timing_entry grad_pass; /* gradient passes */
   fs_timing_entry marg_pass; /* marginal / plan-mass passes (residual and cost) */
-  fs_timing_entry combine;   /* split-column merge kernels */
+  fs_timing_entry combine;   /* second-level merges of split or unit partials */
+  fs_timing_entry screen;    /* block screening and unit planning on sorted clouds */
 } fs_timing;
 
 FS_API void fs_timing_enable(int on);

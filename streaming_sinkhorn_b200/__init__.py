@@ -253,4 +253,4 @@ def timing_get() -> dict:
                    "total_ms": float(getattr(t, name).total_ms),
                    "pairs": float(getattr(t, name).pairs),
                    "evaluated": float(getattr(t, name).evaluated)}
-            for name in ("lse_pass", "grad_pass", "marg_pass", "combine")}
+            for name in ("lse_pass", "grad_pass", "marg_pass", "combine", "screen")}

@@ -42,7 +42,8 @@ class fs_timing_entry(ctypes.Structure):
 
 class fs_timing(ctypes.Structure):
     _fields_ = [("lse_pass", fs_timing_entry), ("grad_pass", fs_timing_entry),
-                ("marg_pass", fs_timing_entry), ("combine", fs_timing_entry)]
+                ("marg_pass", fs_timing_entry), ("combine", fs_timing_entry),
+                ("screen", fs_timing_entry)]
 
 
 _lib = None

@@ -9,6 +9,7 @@
 #include <vector>
 
 #include "../../include/fs.h"
+#include "fs_screen.cuh"
 #include "fs_tc.cuh"
 
 namespace fs {
@@ -32,7 +33,7 @@ std::mutex g_timing_mu;
 bool g_timing_on = false;
 fs_timing g_timing = {};
 
-enum TimedKind { kTLse = 0, kTGrad = 1, kTMarg = 2, kTCombine = 3 };
+enum TimedKind { kTLse = 0, kTGrad = 1, kTMarg = 2, kTCombine = 3, kTScreen = 4 };
 
 struct TimedLaunch {
   cudaEvent_t start, stop;
@@ -81,6 +82,7 @@ class Timer {
       fs_timing_entry* e = t.kind == kTLse    ? &g_timing.lse_pass
                            : t.kind == kTGrad ? &g_timing.grad_pass
                            : t.kind == kTMarg ? &g_timing.marg_pass
+                           : t.kind == kTScreen ? &g_timing.screen
                                               : &g_timing.combine;
       e->launches += 1;
       e->total_ms += ms;
@@ -212,6 +214,41 @@ int64_t partial_floats(const Plan& p, int D, bool grad) {
   return static_cast<int64_t>(p.n_splits) * p.rows_pad * (2 + (grad ? D : 0));
 }
 
+// Queue mode: passes on sorted clouds whose key tiles are whole screening tiles run on the
+// unit plan of fs_screen.cuh. The kept-tile masks take one bit per (row block, key tile),
+// capped at kMaskCapWords words; larger problems run unscreened in split mode.
+constexpr int64_t kMaskCapWords = int64_t(64) << 20;  // 256 MiB
+constexpr int kUnitWaves = 8;  // unit budget, in waves of resident CTAs
+
+struct QPlan {
+  bool on;
+  int64_t rb;         // row blocks
+  int RB;             // rows per row block
+  int mask_words;     // 32-tile mask words per row block
+  int64_t budget;     // C = max(1, ceil(kept / budget)) tiles per unit
+  int64_t units_max;  // budget + rb bounds the number of units
+};
+
+QPlan make_qplan(const Plan& pl, int64_t key_pairs, int D, bool grad, int sms, bool sorted) {
+  QPlan q{};
+  const int64_t tiles = key_pairs / (kScreenTile / 2);
+  q.RB = pl.R * pl.NT;
+  q.rb = pl.row_blocks;
+  q.mask_words = static_cast<int>(ceil_div(tiles, 32));
+  q.on = sorted && D <= 16 && pl.tile_pairs == kScreenTile / 2 && tiles >= 2 &&
+         q.rb * q.mask_words <= kMaskCapWords;
+  if (!q.on) return q;
+  const int64_t slots =
+      static_cast<int64_t>(sms) * occupancy_for(D, grad, pl.variant, pass_smem_bytes(D, pl.tile_pairs));
+  q.budget = kUnitWaves * slots;
+  q.units_max = q.budget + q.rb;
+  return q;
+}
+
+int64_t queue_partial_floats(const QPlan& q, int D, bool grad) {
+  return q.on ? q.units_max * q.RB * (2 + (grad ? D : 0)) : 0;
+}
+
 // Points wider than 16 coordinates take the tensor-core pass for potential and marginal
 // passes (the gradient pass stays on the FMA path); its padded width is 32, 48 or 64.
 int tc_dim(int d) { return d <= 16 ? 0 : (d <= 32 ? 32 : (d <= 48 ? 48 : 64)); }
@@ -269,6 +306,8 @@ constexpr int kMaxAbs = 142;  // unsigned: float bits of the largest |coordinate
 constexpr int kBox = 144;     // ints: ordered lo[3], hi[3] of the first three coordinates
 constexpr int kDmin = 147;    // ints: ordered smallest key-bias change of x, of y
 constexpr int kEval = 148;    // uint64[3]: pairs evaluated by sorted passes, by TimedKind
+constexpr int kQueue = 151;   // ints: tiles per unit C and unit count U of the last queue plan
+constexpr int kKept = 152;    // int64: kept tiles K of the last queue plan
 
 struct Layout {
   int D;       // padded dimension of the FMA path
@@ -285,6 +324,8 @@ struct Layout {
   int64_t sort_n;  // keys of the bitonic sort (power of two, >= kSortSmem)
   size_t off_perm_x, off_perm_y, off_sortkeys, off_box_x, off_box_y, off_hmax_x, off_hmax_y,
       off_lse_x, off_lse_y;
+  // queue mode: kept-tile masks, kept counts, unit starts and unit -> row block
+  size_t off_kmask, off_kcount, off_ustart, off_unit_rb;
   int64_t part_floats;
 };
 
@@ -296,12 +337,23 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms) {
   L.KP = key_pair_floats(L.D);
   L.px = pairs_pad(n);
   L.py = pairs_pad(m);
-  int64_t pf = 0;
-  for (int grad = 0; grad < 2; ++grad) {
-    pf = std::max(pf, partial_floats(make_plan(n, L.py, L.D, grad, sms), L.D, grad));
-    pf = std::max(pf, partial_floats(make_plan(m, L.px, L.D, grad, sms), L.D, grad));
-  }
   L.Dtc = tc_dim(d);
+  L.sorted = L.Dtc == 0;
+  int64_t pf = 0, mask_words = 0, rb_max = 0, units_max = 0;
+  for (int grad = 0; grad < 2; ++grad) {
+    for (int rows_x = 0; rows_x < 2; ++rows_x) {
+      const int64_t key_pairs = rows_x ? L.py : L.px;
+      const Plan pl = make_plan(rows_x ? n : m, key_pairs, L.D, grad, sms);
+      pf = std::max(pf, partial_floats(pl, L.D, grad));
+      const QPlan q = make_qplan(pl, key_pairs, L.D, grad, sms, L.sorted);
+      if (q.on) {
+        pf = std::max(pf, queue_partial_floats(q, L.D, grad));
+        mask_words = std::max(mask_words, q.rb * q.mask_words);
+        rb_max = std::max(rb_max, q.rb);
+        units_max = std::max(units_max, q.units_max);
+      }
+    }
+  }
   L.tx = tc_pad(n);
   L.ty = tc_pad(m);
   if (L.Dtc) {
@@ -341,7 +393,6 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms) {
     L.off_hy_y = o;
     o = align_up(o + static_cast<size_t>(L.ty) * sizeof(float));
   }
-  L.sorted = L.Dtc == 0;
   if (L.sorted) {
     int64_t sn = kSortSmem;
     while (sn < std::max(n, m)) sn <<= 1;
@@ -365,6 +416,14 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms) {
     o = align_up(o + static_cast<size_t>(n) * sizeof(float));
     L.off_lse_y = o;
     o = align_up(o + static_cast<size_t>(m) * sizeof(float));
+    L.off_kmask = o;
+    o = align_up(o + static_cast<size_t>(mask_words) * sizeof(unsigned));
+    L.off_kcount = o;
+    o = align_up(o + static_cast<size_t>(rb_max) * sizeof(int));
+    L.off_ustart = o;
+    o = align_up(o + static_cast<size_t>(rb_max + 1) * sizeof(int));
+    L.off_unit_rb = o;
+    o = align_up(o + static_cast<size_t>(units_max) * sizeof(int));
   }
   L.total = o;
   return L;
@@ -396,6 +455,21 @@ struct PassKernel {
     fn<<<grid, NT, pass_smem_bytes(D, pl.tile_pairs), st>>>(P);
     CK(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  static void launch_queue(const PassParams& P, int64_t units, cudaStream_t st) {
+    set_smem_attr();
+    fn<<<static_cast<unsigned>(units), NT, pass_smem_bytes(D, kScreenTile / 2), st>>>(P);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  static void screen(const PassParams& P, int64_t rb, unsigned* kmask, int* kcount,
+                     cudaStream_t st) {
+    if constexpr (D <= 16) {  // screening runs on the FMA path's widths only
+      const size_t smem = static_cast<size_t>(kScreenTile / 2) * key_pair_floats(D) * sizeof(float);
+      screen_kernel<D, R, NT><<<static_cast<unsigned>(rb), NT, smem, st>>>(P, kmask, kcount);
+      CK(cudaGetLastError());
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+    }
   }
   static int occupancy(size_t smem) {
     int n = 0;
@@ -439,6 +513,24 @@ struct LaunchOp {
   void run() { K::launch(P, pl, st); }
 };
 
+struct QueueOp {
+  const PassParams& P;
+  int64_t units;
+  cudaStream_t st;
+  template <typename K>
+  void run() { K::launch_queue(P, units, st); }
+};
+
+struct ScreenOp {
+  const PassParams& P;
+  int64_t rb;
+  unsigned* kmask;
+  int* kcount;
+  cudaStream_t st;
+  template <typename K>
+  void run() { K::screen(P, rb, kmask, kcount, st); }
+};
+
 struct OccupancyOp {
   size_t smem;
   int result = 1;
@@ -449,6 +541,17 @@ struct OccupancyOp {
 template <int D>
 void launch_pass_d(const PassParams& P, const Plan& pl, bool grad, cudaStream_t st) {
   with_pass_kernel<D>(grad, pl.variant, LaunchOp{P, pl, st});
+}
+
+template <int D>
+void launch_queue_d(const PassParams& P, const Plan& pl, int64_t units, bool grad, cudaStream_t st) {
+  with_pass_kernel<D>(grad, pl.variant, QueueOp{P, units, st});
+}
+
+template <int D>
+void launch_screen_d(const PassParams& P, const Plan& pl, unsigned* kmask, int* kcount, bool grad,
+                     cudaStream_t st) {
+  with_pass_kernel<D>(grad, pl.variant, ScreenOp{P, pl.row_blocks, kmask, kcount, st});
 }
 
 template <int D>
@@ -638,6 +741,9 @@ struct Ctx {
   int *perm_x, *perm_y;         // sorted slot -> original index (NULL when unsorted)
   uint64_t* sortkeys;
   float *box_x, *box_y, *hmax_x, *hmax_y, *lse_x, *lse_y;
+  unsigned* kmask;
+  int *kcount, *ustart, *unit_rb;
+  bool no_screen;  // screening found to keep most tiles: the rest of the call runs unscreened
 };
 
 fs_status check_common(const fs_problem* p, void* ws, size_t ws_bytes, size_t* need_out,
@@ -684,6 +790,10 @@ void carve(Ctx& c, void* ws) {
     c.hmax_y = reinterpret_cast<float*>(c.ws + c.L.off_hmax_y);
     c.lse_x = reinterpret_cast<float*>(c.ws + c.L.off_lse_x);
     c.lse_y = reinterpret_cast<float*>(c.ws + c.L.off_lse_y);
+    c.kmask = reinterpret_cast<unsigned*>(c.ws + c.L.off_kmask);
+    c.kcount = reinterpret_cast<int*>(c.ws + c.L.off_kcount);
+    c.ustart = reinterpret_cast<int*>(c.ws + c.L.off_ustart);
+    c.unit_rb = reinterpret_cast<int*>(c.ws + c.L.off_unit_rb);
   }
 }
 
@@ -947,38 +1057,85 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
   P.err = err_ptr(c.scal);
   int* dmin_slots = reinterpret_cast<int*>(c.scal + kDmin);
   const int tk = grad ? kTGrad : (kind == kMarg ? kTMarg : kTLse);
+  const QPlan q = make_qplan(pl, key_pairs, c.L.D, grad, c.sms, c.L.sorted && !c.no_screen);
   if (c.L.sorted) {
     P.perm = rows_x ? c.perm_x : c.perm_y;
-    P.screen = 1;
-    P.key_box = rows_x ? c.box_y : c.box_x;
-    P.key_hmax = rows_x ? c.hmax_y : c.hmax_x;
     P.evaluated = reinterpret_cast<unsigned long long*>(c.scal + kEval + tk);
     if (kind == kPot) {
       // this pass writes the query cloud's biases: record their change and its LSE2
       P.lse_out = rows_x ? c.lse_x : c.lse_y;
       P.dmin_out = dmin_slots + (rows_x ? 0 : 1);
       CK(cudaMemsetAsync(P.dmin_out, 0x7F, sizeof(int), c.st));
-      if (history) {
-        P.key_dmin = dmin_slots + (rows_x ? 1 : 0);
-        P.lse_prev = rows_x ? c.lse_x : c.lse_y;
-        P.log2_keys = static_cast<float>(std::log2(static_cast<double>(rows_x ? p->m : p->n)));
-      }
     }
   }
   const double pairs = static_cast<double>(n_rows) * static_cast<double>(rows_x ? p->m : p->n);
-  int ti = c.timer->begin();
-  FS_DISPATCH_D(c.L.D, launch_pass_d, P, pl, grad, c.st);
-  c.timer->end(ti, tk, pairs);
-  if (pl.n_splits > 1) {
+  if (q.on) {
+    const int64_t n_keys = rows_x ? p->m : p->n;
+    P.key_box = rows_x ? c.box_y : c.box_x;
+    P.key_hmax = rows_x ? c.hmax_y : c.hmax_x;
+    P.log2_keys = static_cast<float>(std::log2(static_cast<double>(n_keys)));
+    P.skip_margin = kSkipBits + P.log2_keys;
+    if (history && kind == kPot) {
+      P.key_dmin = dmin_slots + (rows_x ? 1 : 0);
+      P.lse_prev = rows_x ? c.lse_x : c.lse_y;
+    }
+    P.part_l = c.part + q.units_max * q.RB;
+    P.part_a = c.part + 2 * q.units_max * q.RB;
+    P.mask_words = q.mask_words;
+    P.rb_rows = q.RB;
+    P.kcount = c.kcount;
+    P.unit_start = c.ustart;
+    P.unit_rb = c.unit_rb;
+    P.qscal = reinterpret_cast<const int*>(c.scal + kQueue);
+    int ti = c.timer->begin();
+    FS_DISPATCH_D(c.L.D, launch_screen_d, P, pl, c.kmask, c.kcount, grad, c.st);
+    plan_units_kernel<<<1, 1024, 0, c.st>>>(c.kcount, static_cast<int>(q.rb), q.budget, q.RB,
+                                            c.ustart, c.unit_rb,
+                                            reinterpret_cast<int*>(c.scal + kQueue),
+                                            reinterpret_cast<long long*>(c.scal + kKept),
+                                            P.evaluated);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    c.timer->end(ti, kTScreen, 0.0);
+    P.kmask = c.kmask;
+    P.evaluated = nullptr;  // counted by the plan
+    ti = c.timer->begin();
+    FS_DISPATCH_D(c.L.D, launch_queue_d, P, pl, q.units_max, grad, c.st);
+    c.timer->end(ti, tk, pairs);
     ti = c.timer->begin();
     FS_DISPATCH_D(c.L.D, launch_combine_d, P, grad, c.st);
     c.timer->end(ti, kTCombine, 0.0);
+  } else {
+    int ti = c.timer->begin();
+    FS_DISPATCH_D(c.L.D, launch_pass_d, P, pl, grad, c.st);
+    c.timer->end(ti, tk, pairs);
+    if (pl.n_splits > 1) {
+      ti = c.timer->begin();
+      FS_DISPATCH_D(c.L.D, launch_combine_d, P, grad, c.st);
+      c.timer->end(ti, kTCombine, 0.0);
+    }
   }
   if (c.L.sorted && kind == kPot) {
     // largest bias per tile of the cloud just updated: the next pass screens against it
     FS_DISPATCH_D(c.L.D, launch_tile_hmax_d, rows_x ? c.kx : c.ky, n_rows,
                   (rows_x ? c.L.px : c.L.py) / kPairPad, rows_x ? c.hmax_x : c.hmax_y, c.st);
   }
+}
+
+// After a solve's first iteration: if the last screened pass (rows from x when rows_x, else
+// from y) kept more than half of all (row block, key tile) pairs, screening cannot pay for
+// its planning and merging, and the remaining passes of the call run unscreened.
+void screening_probe(Ctx& c, bool rows_x) {
+  const int64_t n_rows = rows_x ? c.p->n : c.p->m;
+  const int64_t key_pairs = rows_x ? c.L.py : c.L.px;
+  const Plan pl = make_plan(n_rows, key_pairs, c.L.D, false, c.sms);
+  const QPlan q = make_qplan(pl, key_pairs, c.L.D, false, c.sms, c.L.sorted && !c.no_screen);
+  if (!q.on) return;
+  long long kept = 0;
+  CK(cudaMemcpyAsync(&kept, c.scal + kKept, sizeof(kept), cudaMemcpyDeviceToHost, c.st));
+  CK(cudaStreamSynchronize(c.st));
+  const double all = static_cast<double>(q.rb) * static_cast<double>(key_pairs / (kScreenTile / 2));
+  if (static_cast<double>(kept) > 0.5 * all) c.no_screen = true;
 }
 
 // Drains the stream and reads the kernels' error word.
@@ -1043,6 +1200,7 @@ fs_status potentials_impl(const fs_problem* p, int32_t n_iters, const float* g_i
     for (int32_t it = 0; it < n_iters; ++it) {
       run_pass(c, true, kPot, nullptr, f, nullptr, nullptr, nullptr, it > 0);   // f <- F(g)
       run_pass(c, false, kPot, nullptr, g, nullptr, nullptr, nullptr, it > 0);  // g <- G(f)
+      if (it == 0 && n_iters > 2) screening_probe(c, false);
     }
     return finish(c);
   });

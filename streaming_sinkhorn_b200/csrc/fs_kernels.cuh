@@ -83,21 +83,31 @@ struct PassParams {
   const float* nrm;
   // spatially sorted clouds: sorted row -> original index of the query cloud (NULL: identity)
   const int* perm;
-  // block screening (potential passes after the first two)
-  int32_t screen;           // 1: skip key tiles whose every term is provably negligible
+  // block screening (sorted clouds): the inputs of screen_kernel
   const float* key_box;     // [tile][2D]: bounding box of each 256-point key tile
   const float* key_hmax;    // [tile]: largest key bias H of each key tile
-  const int* key_dmin;      // ordered int: smallest change of the key biases since the last pass
+  const int* key_dmin;      // ordered int: smallest change of the key biases since the last
+                            // pass, or NULL (no history bound)
   const float* lse_prev;    // LSE2 of every query row in its previous pass (sorted order)
   float log2_keys;          // log2(number of keys)
+  float skip_margin;        // log2 units below a row's lower bound under which tiles drop
   float* lse_out;           // kPot: LSE2 of every query row (sorted order)
   int* dmin_out;            // kPot: ordered int, smallest change of the H this pass writes
-  unsigned long long* evaluated;  // pairs evaluated after screening
+  unsigned long long* evaluated;  // pairs evaluated (after screening)
+  // queue mode (screened passes): kept-tile bit masks and the unit plan
+  const unsigned* kmask;    // [row block][mask_words], or NULL for split mode
+  int32_t mask_words;       // 32-tile words per row block
+  int32_t rb_rows;          // rows of a row block (R * NT of the pass)
+  const int* kcount;        // [row block] kept tiles
+  const int* unit_start;    // [row block + 1] first unit of each row block
+  const int* unit_rb;       // [unit] row block of each unit
+  const int* qscal;         // [0] tiles per unit C, [1] number of units U
 };
 
-constexpr int kScreenTile = 256;      // points per screening tile (= kPairPad pairs)
-constexpr int kScreenMaxTiles = 4096; // tiles one CTA can screen (list in shared memory)
-constexpr float kSkipMargin = 150.0f; // skipped terms are below 2^-150 of the row's largest
+constexpr int kScreenTile = 256;  // points per screening tile (= kPairPad pairs)
+// Relative size, in log2 units, below which the omitted part of a row's sum is kept: the
+// skip margin is kSkipBits + log2(number of keys) (the tolerance of the screening).
+constexpr float kSkipBits = 32.0f;
 
 // Offset of coordinate slot k (k == D is the bias H) of point i in packed keys.
 template <int D>
@@ -204,25 +214,106 @@ template <int D, int R, int NT, int G, bool GRAD, int MINB>
 __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) {
   constexpr int KP = key_pair_floats(D);
   constexpr int NA = GRAD ? D : 1;
+  constexpr int RB = R * NT;  // rows of one row block
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ uint64_t bars[kStages];
+  __shared__ int s_walk[2];
 
   float* stages = reinterpret_cast<float*>(smem_raw);
   const int tid = threadIdx.x;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (NT * R);
-  const int split = blockIdx.y;
-  const int64_t p_begin = static_cast<int64_t>(split) * P.pairs_per_split;
-  int64_t p_end = p_begin + P.pairs_per_split;
-  if (p_end > P.key_pairs) p_end = P.key_pairs;
-  const int n_tiles = static_cast<int>((p_end - p_begin) / P.tile_pairs);
   const uint32_t stage_floats = static_cast<uint32_t>(P.tile_pairs) * KP;
   const uint32_t stage_bytes = stage_floats * 4u;
-  const float* key_src = P.keys + p_begin * KP;
+
+  // The work of this CTA: rows row0 .. row0 + RB and a list of key tiles. Split mode: the
+  // tiles of column split blockIdx.y, in order. Queue mode (screened, sorted clouds): unit
+  // blockIdx.x of the screening plan, i.e. the kept tiles with ordinals [k0, k0 + n_work)
+  // of row block b, read from the row block's bit mask.
+  const bool queue = P.kmask != nullptr;
+  int64_t row0, unit;
+  int n_work, n_units = 1;
+  const float* key_src;
+  const unsigned* mrow = nullptr;
+  if (queue) {
+    unit = blockIdx.x;
+    if (unit >= P.qscal[1]) return;  // past the plan's unit count
+    const int b = P.unit_rb[unit];
+    const int first = P.unit_start[b];
+    n_units = P.unit_start[b + 1] - first;
+    const int C = P.qscal[0];
+    const int k0 = static_cast<int>(unit - first) * C;
+    n_work = min(C, P.kcount[b] - k0);
+    row0 = static_cast<int64_t>(b) * RB;
+    key_src = P.keys;
+    mrow = P.kmask + static_cast<int64_t>(b) * P.mask_words;
+    // Locate ordinal k0: the mask word holding it and how many set bits of that word precede it.
+    if (tid < 32) {
+      int before = 0;
+      bool found = false;
+      for (int w0 = 0; w0 < P.mask_words && !found; w0 += 32) {
+        const int w = w0 + tid;
+        const int cnt = w < P.mask_words ? __popc(mrow[w]) : 0;
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (tid >= o) incl += v;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, before + incl > k0);
+        if (hit) {
+          const int lane = __ffs(hit) - 1;
+          if (tid == lane) {
+            s_walk[0] = w;
+            s_walk[1] = k0 - (before + incl - cnt);
+          }
+          found = true;
+        }
+        before += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (!found && tid == 0) {  // inconsistent plan: no tile is read, the rows get no result
+        s_walk[0] = -1;
+        s_walk[1] = 0;
+        atomicOr(P.err, kErrTimeout);
+      }
+    }
+  } else {
+    unit = blockIdx.y;
+    row0 = static_cast<int64_t>(blockIdx.x) * RB;
+    const int64_t p_begin = static_cast<int64_t>(blockIdx.y) * P.pairs_per_split;
+    int64_t p_end = p_begin + P.pairs_per_split;
+    if (p_end > P.key_pairs) p_end = P.key_pairs;
+    n_work = static_cast<int>((p_end - p_begin) / P.tile_pairs);
+    n_units = P.n_splits;
+    key_src = P.keys + p_begin * KP;
+    if (tid == 0 && P.evaluated)
+      atomicAdd(P.evaluated, static_cast<unsigned long long>(n_work) * P.tile_pairs * 2 * RB);
+  }
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
   }
+  __syncthreads();
+  if (queue && s_walk[0] < 0) n_work = 0;
+
+  // Thread 0 issues the copies in order; in queue mode it walks the set bits of the mask
+  // from the located start (the plan guarantees n_work of them; the walk stays inside the
+  // row's words regardless and falls back to tile 0 if they run out).
+  int walk_w = 0;
+  unsigned walk_bits = 0u;
+  if (queue && tid == 0 && n_work > 0) {
+    walk_w = s_walk[0];
+    walk_bits = mrow[walk_w];
+    for (int s = 0; s < s_walk[1]; ++s) walk_bits &= walk_bits - 1u;
+  }
+  auto tile_src = [&](int e) -> const float* {
+    int tt = e;
+    if (queue) {
+      while (walk_bits == 0u && walk_w + 1 < P.mask_words) walk_bits = mrow[++walk_w];
+      tt = walk_bits ? walk_w * 32 + __ffs(walk_bits) - 1 : 0;
+      walk_bits &= walk_bits - 1u;
+    }
+    return key_src + static_cast<int64_t>(tt) * stage_floats;
+  };
 
   // Row state: coordinates duplicated into both lanes of a packed register; the running
   // offset m (log2 units), `base` (m, or 0 while no column has set it) and mk = base/kappa
@@ -248,110 +339,6 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
 #pragma unroll
     for (int k = 0; k < NA; ++k) A[r][k] = pk(0.0f, 0.0f);
   }
-
-  // Block screening (sorted clouds). Every pass first processes an anchor tile: the key
-  // tile whose exponents have the largest upper bound (its largest bias minus kappa times
-  // the squared distance between the CTA's row box and the tile's box). The running offset
-  // it leaves is a value some term of the row reaches, hence a lower bound on the row's
-  // largest exponent; a potential pass with history also has the bound "previous LSE2 plus
-  // the smallest change of the key biases, minus log2(#keys)" (the largest term is at least
-  // the sum over the count). Every other tile whose upper bound lies more than kSkipMargin
-  // below the smallest of those bounds over the CTA's rows is skipped: each omitted term is
-  // under 2^-kSkipMargin of its row's largest. The kept tiles form a list in shared memory.
-  __shared__ unsigned short tlist[kScreenMaxTiles];
-  __shared__ unsigned smask[kScreenMaxTiles / 32];
-  __shared__ int s_box[2 * D];
-  __shared__ int s_mlb, s_count;
-  __shared__ unsigned long long s_best;
-  const bool screening = P.screen && P.tile_pairs == kScreenTile / 2 && n_tiles > 1 &&
-                         n_tiles <= kScreenMaxTiles;
-  const bool history = screening && P.lse_prev && P.key_dmin;
-  const int64_t T0 = p_begin / (kScreenTile / 2);
-  int n_work = n_tiles;
-  // Upper bound of the exponents of key tile tt for any row of this CTA.
-  auto tile_ub = [&](int tt) -> float {
-    const float* bx = P.key_box + (T0 + tt) * 2 * D;
-    float d2 = 0.0f;
-#pragma unroll
-    for (int k = 0; k < D; ++k) {
-      const float gap =
-          fmaxf(fmaxf(bx[k] - ord_float(s_box[D + k]), ord_float(s_box[k]) - bx[D + k]), 0.0f);
-      d2 = fmaf(gap, gap, d2);
-    }
-    return P.key_hmax[T0 + tt] - P.kappa_f * d2;
-  };
-  if (screening) {
-    if (tid < D) {
-      s_box[tid] = 0x7FFFFFFF;
-      s_box[D + tid] = static_cast<int>(0x80000000u);
-    }
-    if (tid == 0) {
-      s_mlb = 0x7FFFFFFF;
-      s_best = 0ull;
-    }
-    __syncthreads();
-    float lo[D], hi[D];
-#pragma unroll
-    for (int k = 0; k < D; ++k) {
-      lo[k] = INFINITY;
-      hi[k] = -INFINITY;
-    }
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int64_t i = row0 + r * NT + tid;
-      if (i < P.n_rows) {
-#pragma unroll
-        for (int k = 0; k < D; ++k) {
-          float c0, c1;
-          upk(X[r][k], c0, c1);
-          lo[k] = fminf(lo[k], c0);
-          hi[k] = fmaxf(hi[k], c0);
-        }
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-      for (int k = 0; k < D; ++k) {
-        lo[k] = fminf(lo[k], __shfl_xor_sync(0xffffffffu, lo[k], o));
-        hi[k] = fmaxf(hi[k], __shfl_xor_sync(0xffffffffu, hi[k], o));
-      }
-    }
-    if ((tid & 31) == 0) {
-#pragma unroll
-      for (int k = 0; k < D; ++k) {
-        atomicMin(&s_box[k], float_ord(lo[k]));
-        atomicMax(&s_box[D + k], float_ord(hi[k]));
-      }
-    }
-    __syncthreads();
-    // anchor: largest upper bound, ties to the lower tile (key = ordered ub, then ~index)
-    unsigned long long best = 0ull;
-    for (int tt = tid; tt < n_tiles; tt += NT) {
-      const unsigned ub = static_cast<unsigned>(float_ord(tile_ub(tt))) ^ 0x80000000u;
-      const unsigned long long key =
-          (static_cast<unsigned long long>(ub) << 32) | static_cast<unsigned>(0xFFFF - tt);
-      best = best > key ? best : key;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-      best = best > other ? best : other;
-    }
-    if ((tid & 31) == 0) atomicMax(&s_best, best);
-    __syncthreads();
-    if (tid == 0) tlist[0] = static_cast<unsigned short>(0xFFFF - (s_best & 0xFFFFull));
-    __syncthreads();
-    n_work = 1;  // the anchor; the kept tiles are appended once it is processed
-  } else {
-    __syncthreads();
-    if (tid == 0 && P.evaluated)
-      atomicAdd(P.evaluated, static_cast<unsigned long long>(n_tiles) * P.tile_pairs * 2 * (R * NT));
-  }
-  auto tile_src = [&](int e) -> const float* {
-    const int tt = screening ? static_cast<int>(tlist[e]) : e;
-    return key_src + static_cast<int64_t>(tt) * stage_floats;
-  };
 
   // Online max/sum of this thread's rows over one key tile in shared memory.
   auto process_tile = [&](const float* tile) {
@@ -417,71 +404,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
           }
         }
       }
-    }
-  };
-
-  // After the anchor: the lower bounds, the screen of the other tiles, the list, and the
-  // first copies of the kept tiles.
-  auto screen_rest = [&]() {
-    const int anchor = tlist[0];
-    const float dmin = history ? ord_float(*P.key_dmin) : 0.0f;
-    float mlb = INFINITY;
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int64_t i = row0 + r * NT + tid;
-      if (i < P.n_rows) {
-        float b = m[r];
-        if (history) b = fmaxf(b, P.lse_prev[i] + dmin - P.log2_keys);
-        mlb = fminf(mlb, b);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mlb = fminf(mlb, __shfl_xor_sync(0xffffffffu, mlb, o));
-    const int nwords = (n_tiles + 31) / 32;
-    for (int w = tid; w < nwords; w += NT) smask[w] = 0u;
-    if ((tid & 31) == 0) atomicMin(&s_mlb, float_ord(mlb));
-    __syncthreads();
-    const float mlb_min = ord_float(s_mlb);
-    for (int tt = tid; tt < n_tiles; tt += NT) {
-      if (tt != anchor && tile_ub(tt) >= mlb_min - kSkipMargin)
-        atomicOr(&smask[tt >> 5], 1u << (tt & 31));
-    }
-    __syncthreads();
-    if (tid < 32) {
-      int running = 1;  // slot 0 holds the anchor
-      for (int w0 = 0; w0 < nwords; w0 += 32) {
-        const int w = w0 + tid;
-        unsigned word = w < nwords ? smask[w] : 0u;
-        const int cnt = __popc(word);
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (tid >= o) incl += v;
-        }
-        int pos = running + incl - cnt;
-        while (word) {
-          const int bit = __ffs(word) - 1;
-          tlist[pos++] = static_cast<unsigned short>(w * 32 + bit);
-          word &= word - 1u;
-        }
-        running += __shfl_sync(0xffffffffu, incl, 31);
-      }
-      if (tid == 0) {
-        s_count = running;
-        if (P.evaluated)
-          atomicAdd(P.evaluated, static_cast<unsigned long long>(running) * kScreenTile * (R * NT));
-      }
-    }
-    __syncthreads();
-    n_work = s_count;
-    if (tid == 0) {
-      for (int e = 1; e < kStages && e < n_work; ++e) {
-        mbar_expect_tx(&bars[e], stage_bytes);
-        bulk_g2s(stages + e * stage_floats, tile_src(e), stage_bytes, &bars[e]);
-      }
-    }
-  };
+    }  };
 
   if (tid == 0) {
     for (int s = 0; s < kStages && s < n_work; ++s) {
@@ -509,7 +432,6 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       bulk_g2s(stages + ps * stage_floats, tile_src(t - 1 + kStages), stage_bytes, &bars[ps]);
     }
     process_tile(stages + st * stage_floats);
-    if (screening && t == 0) screen_rest();
   }
 
   if (aborted) {
@@ -524,7 +446,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     return;
   }
 
-  if (P.n_splits == 1) {
+  if (n_units == 1) {
     double dev_sum = 0.0, dev_max = 0.0, mass = 0.0;
     float dmin = INFINITY;
 #pragma unroll
@@ -559,13 +481,17 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     if (!GRAD && P.kind == kMarg) block_reduce_marg(dev_sum, dev_max, mass, P.acc);
     if (!GRAD && P.kind == kPot) reduce_dmin(dmin, P.dmin_out);
   } else {
+    // Partials of this unit: split mode at [split][rows_pad] (global row index), queue mode
+    // at [unit][RB] (row index within the block).
+    const int64_t pstride = queue ? RB : P.rows_pad;
+    const int64_t poff = queue ? -row0 : 0;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int64_t i = row0 + r * NT + tid;
       if (i >= P.n_rows) continue;
       float l0, l1;
       upk(L[r], l0, l1);
-      const int64_t o = static_cast<int64_t>(split) * P.rows_pad + i;
+      const int64_t o = unit * pstride + poff + i;
       P.part_m[o] = m[r];
       P.part_l[o] = l0 + l1;
       if (GRAD) {
@@ -573,36 +499,46 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
         for (int k = 0; k < NA; ++k) {
           float a0, a1;
           upk(A[r][k], a0, a1);
-          P.part_a[(static_cast<int64_t>(split) * D + k) * P.rows_pad + i] = a0 + a1;
+          P.part_a[(unit * D + k) * pstride + poff + i] = a0 + a1;
         }
       }
     }
   }
 }
 
-// Second-level LSE over the split partials of each row, then the row completion. A split
-// whose columns were all zero-weight or padding left m = -inf and sum 0 and drops out.
+// Second-level LSE over the partials of each row, then the row completion. Split mode: the
+// n_splits partials at [split][rows_pad]. Queue mode: the units of the row's block at
+// [unit][rb_rows]; a block with one unit was completed by the pass itself. A partial whose
+// columns were all zero-weight or padding left m = -inf and sum 0 and drops out.
 template <int D, bool GRAD>
 __global__ void __launch_bounds__(256) combine_kernel(const PassParams P) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   double dev = 0.0, mass = 0.0;
   float dmin = INFINITY;
-  if (i < P.n_rows) {
+  int64_t s0 = 0, ns = P.n_splits, stride = P.rows_pad, off = i;
+  if (P.kmask && i < P.n_rows) {
+    const int64_t b = i / P.rb_rows;
+    s0 = P.unit_start[b];
+    ns = P.unit_start[b + 1] - s0;
+    stride = P.rb_rows;
+    off = i - b * P.rb_rows;
+  }
+  if (i < P.n_rows && (ns > 1 || !P.kmask)) {
     float mx = -INFINITY;
-    for (int s = 0; s < P.n_splits; ++s) mx = fmaxf(mx, P.part_m[s * P.rows_pad + i]);
+    for (int64_t s = s0; s < s0 + ns; ++s) mx = fmaxf(mx, P.part_m[s * stride + off]);
     double l = 0.0;
     float a[GRAD ? D : 1];
     if (GRAD) {
       for (int k = 0; k < D; ++k) a[k] = 0.0f;
     }
-    for (int s = 0; s < P.n_splits; ++s) {
-      const int64_t o = s * P.rows_pad + i;
+    for (int64_t s = s0; s < s0 + ns; ++s) {
+      const int64_t o = s * stride + off;
       const float pm = P.part_m[o];
       if (pm == -INFINITY) continue;
       const float w = ex2(pm - mx);
       l += static_cast<double>(P.part_l[o]) * w;
       if (GRAD) {
-        for (int k = 0; k < D; ++k) a[k] += P.part_a[(static_cast<int64_t>(s) * D + k) * P.rows_pad + i] * w;
+        for (int k = 0; k < D; ++k) a[k] += P.part_a[(s * D + k) * stride + off] * w;
       }
     }
     if (GRAD) {

@@ -146,6 +146,6 @@ def test_timing_api_roundtrip():
     fs.timing_enable(True)
     fs.timing_reset()
     t = fs.timing_get()
-    assert set(t) == {"lse_pass", "grad_pass", "marg_pass", "combine"}
+    assert set(t) == {"lse_pass", "grad_pass", "marg_pass", "combine", "screen"}
     assert all(v["launches"] == 0 for v in t.values())
     fs.timing_enable(False)
