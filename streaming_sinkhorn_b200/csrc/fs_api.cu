@@ -123,10 +123,15 @@ struct Variant {
 constexpr Variant kLseVariants[2] = {{2, 128}, {1, 128}};
 constexpr Variant kGradVariants[2] = {{2, 128}, {1, 128}};
 constexpr Variant kWideVariant = {1, 128};
+// Queue mode: one warp per CTA, 64 rows, so each warp screens, streams and merges on its own
+// and no warp waits at a barrier for another warp's tiles.
+constexpr int kQueueVariant = 2;
+constexpr Variant kQueueShape = {2, 32};
 
 struct Plan {
   int variant;  // index into the variant table of this pass type
   int R, NT;
+  int64_t n_rows;
   int64_t row_blocks, rows_pad;
   int tile_pairs;
   int n_splits;
@@ -163,6 +168,7 @@ Plan make_plan(int64_t n_rows, int64_t key_pairs, int D, bool grad, int sms) {
     nv = 2;
   }
   Plan p{};
+  p.n_rows = n_rows;
   // Most rows per CTA whose (row blocks x tiles) still fills the machine; else the smallest.
   int chosen = nv - 1;
   for (int v = 0; v < nv; ++v) {
@@ -232,14 +238,14 @@ struct QPlan {
 QPlan make_qplan(const Plan& pl, int64_t key_pairs, int D, bool grad, int sms, bool sorted) {
   QPlan q{};
   const int64_t tiles = key_pairs / (kScreenTile / 2);
-  q.RB = pl.R * pl.NT;
-  q.rb = pl.row_blocks;
+  q.RB = kQueueShape.R * kQueueShape.NT;
+  q.rb = ceil_div(pl.n_rows, q.RB);
   q.mask_words = static_cast<int>(ceil_div(tiles, 32));
   q.on = sorted && D <= 16 && pl.tile_pairs == kScreenTile / 2 && tiles >= 2 &&
          q.rb * q.mask_words <= kMaskCapWords;
   if (!q.on) return q;
-  const int64_t slots =
-      static_cast<int64_t>(sms) * occupancy_for(D, grad, pl.variant, pass_smem_bytes(D, pl.tile_pairs));
+  const int64_t slots = static_cast<int64_t>(sms) *
+                        occupancy_for(D, grad, kQueueVariant, pass_smem_bytes(D, kScreenTile / 2));
   q.budget = kUnitWaves * slots;
   q.units_max = q.budget + q.rb;
   return q;
@@ -325,7 +331,7 @@ struct Layout {
   size_t off_perm_x, off_perm_y, off_sortkeys, off_box_x, off_box_y, off_hmax_x, off_hmax_y,
       off_lse_x, off_lse_y;
   // queue mode: kept-tile masks, kept counts, unit starts and unit -> row block
-  size_t off_kmask, off_kcount, off_ustart, off_unit_rb;
+  size_t off_kmask, off_kcount, off_ustart, off_unit_rb, off_rmlb;
   int64_t part_floats;
 };
 
@@ -404,14 +410,16 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms) {
     o = align_up(o + static_cast<size_t>(m) * sizeof(int));
     L.off_sortkeys = o;
     o = align_up(o + static_cast<size_t>(sn) * sizeof(uint64_t));
+    // tile summaries followed by their super-tile summaries
+    const int64_t sx = tiles_x + ceil_div(tiles_x, kSuper), sy = tiles_y + ceil_div(tiles_y, kSuper);
     L.off_box_x = o;
-    o = align_up(o + static_cast<size_t>(tiles_x) * 2 * L.D * sizeof(float));
+    o = align_up(o + static_cast<size_t>(sx) * 2 * L.D * sizeof(float));
     L.off_box_y = o;
-    o = align_up(o + static_cast<size_t>(tiles_y) * 2 * L.D * sizeof(float));
+    o = align_up(o + static_cast<size_t>(sy) * 2 * L.D * sizeof(float));
     L.off_hmax_x = o;
-    o = align_up(o + static_cast<size_t>(tiles_x) * sizeof(float));
+    o = align_up(o + static_cast<size_t>(sx) * sizeof(float));
     L.off_hmax_y = o;
-    o = align_up(o + static_cast<size_t>(tiles_y) * sizeof(float));
+    o = align_up(o + static_cast<size_t>(sy) * sizeof(float));
     L.off_lse_x = o;
     o = align_up(o + static_cast<size_t>(n) * sizeof(float));
     L.off_lse_y = o;
@@ -424,6 +432,8 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms) {
     o = align_up(o + static_cast<size_t>(rb_max + 1) * sizeof(int));
     L.off_unit_rb = o;
     o = align_up(o + static_cast<size_t>(units_max) * sizeof(int));
+    L.off_rmlb = o;
+    o = align_up(o + static_cast<size_t>(std::max(n, m)) * sizeof(float));
   }
   L.total = o;
   return L;
@@ -464,9 +474,8 @@ struct PassKernel {
   }
   static void screen(const PassParams& P, int64_t rb, unsigned* kmask, int* kcount,
                      cudaStream_t st) {
-    if constexpr (D <= 16) {  // screening runs on the FMA path's widths only
-      const size_t smem = static_cast<size_t>(kScreenTile / 2) * key_pair_floats(D) * sizeof(float);
-      screen_kernel<D, R, NT><<<static_cast<unsigned>(rb), NT, smem, st>>>(P, kmask, kcount);
+    if constexpr (D <= 16 && NT == 32) {  // one warp per row block, FMA-path widths only
+      screen_kernel<D, R><<<static_cast<unsigned>(rb), 32, 0, st>>>(P, kmask, kcount);
       CK(cudaGetLastError());
       g_launches.fetch_add(1, std::memory_order_relaxed);
     }
@@ -494,13 +503,17 @@ void with_pass_kernel(bool grad, int variant, Op&& op) {
     if (grad) {
       if (variant == 0)
         op.template run<PassKernel<D, 2, 128, true, 8, 3>>();
-      else
+      else if (variant == 1)
         op.template run<PassKernel<D, 1, 128, true, 8, 4>>();
+      else
+        op.template run<PassKernel<D, 2, 32, true, 8, 12>>();
     } else {
       if (variant == 0)
         op.template run<PassKernel<D, 2, 128, false, 8, 6>>();
-      else
+      else if (variant == 1)
         op.template run<PassKernel<D, 1, 128, false, 8, 8>>();
+      else
+        op.template run<PassKernel<D, 2, 32, false, 8, 24>>();
     }
   }
 }
@@ -544,14 +557,14 @@ void launch_pass_d(const PassParams& P, const Plan& pl, bool grad, cudaStream_t 
 }
 
 template <int D>
-void launch_queue_d(const PassParams& P, const Plan& pl, int64_t units, bool grad, cudaStream_t st) {
-  with_pass_kernel<D>(grad, pl.variant, QueueOp{P, units, st});
+void launch_queue_d(const PassParams& P, int64_t units, bool grad, cudaStream_t st) {
+  with_pass_kernel<D>(grad, kQueueVariant, QueueOp{P, units, st});
 }
 
 template <int D>
-void launch_screen_d(const PassParams& P, const Plan& pl, unsigned* kmask, int* kcount, bool grad,
+void launch_screen_d(const PassParams& P, int64_t rb, unsigned* kmask, int* kcount, bool grad,
                      cudaStream_t st) {
-  with_pass_kernel<D>(grad, pl.variant, ScreenOp{P, pl.row_blocks, kmask, kcount, st});
+  with_pass_kernel<D>(grad, kQueueVariant, ScreenOp{P, rb, kmask, kcount, st});
 }
 
 template <int D>
@@ -676,9 +689,14 @@ void launch_bias_d(float* keys, int64_t count, const float* pot, const int* perm
 template <int D>
 void launch_tile_box_d(const float* keys, int64_t count, int64_t tiles, float* box,
                        cudaStream_t st) {
-  tile_box_kernel<D><<<static_cast<unsigned>(tiles), 256, 0, st>>>(keys, count, box);
+  // tile boxes, then super-tile boxes behind them (lower corners by min, upper by max)
+  tile_box_kernel<D><<<static_cast<unsigned>(tiles), 256, 0, st>>>(keys, count, box, tiles);
   CK(cudaGetLastError());
-  g_launches.fetch_add(1, std::memory_order_relaxed);
+  const int64_t supers = ceil_div(tiles, kSuper);
+  super_reduce_kernel<<<static_cast<unsigned>(ceil_div(supers, 256)), 256, 0, st>>>(
+      box, tiles, box + 2 * D * tiles, supers, 2 * D, D);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(2, std::memory_order_relaxed);
 }
 
 template <int D>
@@ -686,7 +704,11 @@ void launch_tile_hmax_d(const float* keys, int64_t count, int64_t tiles, float* 
                         cudaStream_t st) {
   tile_hmax_kernel<D><<<static_cast<unsigned>(tiles), 256, 0, st>>>(keys, count, hmax);
   CK(cudaGetLastError());
-  g_launches.fetch_add(1, std::memory_order_relaxed);
+  const int64_t supers = ceil_div(tiles, kSuper);
+  super_reduce_kernel<<<static_cast<unsigned>(ceil_div(supers, 256)), 256, 0, st>>>(
+      hmax, tiles, hmax + tiles, supers, 1, 0);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(2, std::memory_order_relaxed);
 }
 
 // Morton order of one cloud: keys (code << 32 | index), bitonic sort, permutation.
@@ -743,6 +765,7 @@ struct Ctx {
   float *box_x, *box_y, *hmax_x, *hmax_y, *lse_x, *lse_y;
   unsigned* kmask;
   int *kcount, *ustart, *unit_rb;
+  float* rmlb;     // per-row lower bounds written by the screening kernel
   bool no_screen;  // screening found to keep most tiles: the rest of the call runs unscreened
 };
 
@@ -794,6 +817,7 @@ void carve(Ctx& c, void* ws) {
     c.kcount = reinterpret_cast<int*>(c.ws + c.L.off_kcount);
     c.ustart = reinterpret_cast<int*>(c.ws + c.L.off_ustart);
     c.unit_rb = reinterpret_cast<int*>(c.ws + c.L.off_unit_rb);
+    c.rmlb = reinterpret_cast<float*>(c.ws + c.L.off_rmlb);
   }
 }
 
@@ -1071,8 +1095,13 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
   const double pairs = static_cast<double>(n_rows) * static_cast<double>(rows_x ? p->m : p->n);
   if (q.on) {
     const int64_t n_keys = rows_x ? p->m : p->n;
+    const int64_t T = key_pairs / kPairPad, S = ceil_div(T, kSuper);
+    P.key_tiles = static_cast<int32_t>(T);
+    P.key_supers = static_cast<int32_t>(S);
     P.key_box = rows_x ? c.box_y : c.box_x;
     P.key_hmax = rows_x ? c.hmax_y : c.hmax_x;
+    P.key_sbox = P.key_box + 2 * c.L.D * T;
+    P.key_shmax = P.key_hmax + T;
     P.log2_keys = static_cast<float>(std::log2(static_cast<double>(n_keys)));
     P.skip_margin = kSkipBits + P.log2_keys;
     if (history && kind == kPot) {
@@ -1087,20 +1116,20 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
     P.unit_start = c.ustart;
     P.unit_rb = c.unit_rb;
     P.qscal = reinterpret_cast<const int*>(c.scal + kQueue);
+    P.row_mlb = c.rmlb;
     int ti = c.timer->begin();
-    FS_DISPATCH_D(c.L.D, launch_screen_d, P, pl, c.kmask, c.kcount, grad, c.st);
+    FS_DISPATCH_D(c.L.D, launch_screen_d, P, q.rb, c.kmask, c.kcount, grad, c.st);
     plan_units_kernel<<<1, 1024, 0, c.st>>>(c.kcount, static_cast<int>(q.rb), q.budget, q.RB,
                                             c.ustart, c.unit_rb,
                                             reinterpret_cast<int*>(c.scal + kQueue),
                                             reinterpret_cast<long long*>(c.scal + kKept),
-                                            P.evaluated);
+                                            nullptr);
     CK(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
     c.timer->end(ti, kTScreen, 0.0);
-    P.kmask = c.kmask;
-    P.evaluated = nullptr;  // counted by the plan
+    P.kmask = c.kmask;  // the pass counts the tiles each warp evaluates
     ti = c.timer->begin();
-    FS_DISPATCH_D(c.L.D, launch_queue_d, P, pl, q.units_max, grad, c.st);
+    FS_DISPATCH_D(c.L.D, launch_queue_d, P, q.units_max, grad, c.st);
     c.timer->end(ti, tk, pairs);
     ti = c.timer->begin();
     FS_DISPATCH_D(c.L.D, launch_combine_d, P, grad, c.st);

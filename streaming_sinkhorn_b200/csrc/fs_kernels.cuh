@@ -84,8 +84,11 @@ struct PassParams {
   // spatially sorted clouds: sorted row -> original index of the query cloud (NULL: identity)
   const int* perm;
   // block screening (sorted clouds): the inputs of screen_kernel
-  const float* key_box;     // [tile][2D]: bounding box of each 256-point key tile
-  const float* key_hmax;    // [tile]: largest key bias H of each key tile
+  const float* key_box;     // [2D][key_tiles]: box of each 256-point key tile (lo, then hi)
+  const float* key_hmax;    // [key_tiles]: largest key bias H of each key tile
+  const float* key_sbox;    // [2D][key_supers]: the same for runs of kSuper tiles
+  const float* key_shmax;   // [key_supers]
+  int32_t key_tiles, key_supers;
   const int* key_dmin;      // ordered int: smallest change of the key biases since the last
                             // pass, or NULL (no history bound)
   const float* lse_prev;    // LSE2 of every query row in its previous pass (sorted order)
@@ -102,6 +105,7 @@ struct PassParams {
   const int* unit_start;    // [row block + 1] first unit of each row block
   const int* unit_rb;       // [unit] row block of each unit
   const int* qscal;         // [0] tiles per unit C, [1] number of units U
+  float* row_mlb;           // [row]: lower bound on each row's largest exponent (screening)
 };
 
 constexpr int kScreenTile = 256;  // points per screening tile (= kPairPad pairs)
@@ -433,6 +437,8 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     }
     process_tile(stages + st * stage_floats);
   }
+  if (queue && P.evaluated && tid == 0 && n_work > 0)
+    atomicAdd(P.evaluated, static_cast<unsigned long long>(n_work) * kScreenTile * RB);
 
   if (aborted) {
     // Record the timeout, let this CTA's own copies still in flight land (bounded), leave.

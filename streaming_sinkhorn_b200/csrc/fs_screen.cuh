@@ -29,33 +29,23 @@
 
 namespace fs {
 
-// One CTA per row block: the bit mask of kept key tiles and its population count.
-template <int D, int R, int NT>
-__global__ void __launch_bounds__(NT) screen_kernel(const PassParams P, unsigned* kmask,
+// One warp (one CTA) per row block of 32 R rows: the bit mask of kept key tiles and its
+// population count. Tiles are tested through their super-tiles first: a super-tile's box
+// contains its tiles' boxes and its bias maximum bounds theirs, so its upper bound bounds
+// theirs, and a rejected super-tile rejects all of its tiles.
+template <int D, int R>
+__global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned* kmask,
                                                     int* kcount) {
   constexpr int KP = key_pair_floats(D);
-  constexpr int RB = R * NT;
+  constexpr int RB = R * 32;
   constexpr int TP = kScreenTile / 2;  // key pairs per tile
-  extern __shared__ __align__(16) float anchor_tile[];  // TP * KP floats
-  __shared__ int s_box[2 * D];
-  __shared__ int s_mlb, s_cnt;
-  __shared__ unsigned long long s_best;
-  const int tid = threadIdx.x;
+  __shared__ __align__(16) float anchor_tile[TP * KP];
+  const int lane = threadIdx.x;
   const int64_t b = blockIdx.x;
   const int64_t row0 = b * RB;
-  const int n_tiles = static_cast<int>(P.key_pairs / TP);
-  if (tid < D) {
-    s_box[tid] = 0x7FFFFFFF;
-    s_box[D + tid] = static_cast<int>(0x80000000u);
-  }
-  if (tid == 0) {
-    s_mlb = 0x7FFFFFFF;
-    s_cnt = 0;
-    s_best = 0ull;
-  }
-  __syncthreads();
+  const int T = P.key_tiles, S = P.key_supers;
 
-  // rows of the block and their box
+  // rows of the block and their box (every lane ends with the block's box)
   float x[R][D];
   bool valid[R];
   float lo[D], hi[D];
@@ -66,7 +56,7 @@ __global__ void __launch_bounds__(NT) screen_kernel(const PassParams P, unsigned
   }
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    const int64_t i = row0 + r * NT + tid;
+    const int64_t i = row0 + r * 32 + lane;
     valid[r] = i < P.n_rows;
 #pragma unroll
     for (int k = 0; k < D; ++k) {
@@ -85,72 +75,94 @@ __global__ void __launch_bounds__(NT) screen_kernel(const PassParams P, unsigned
       hi[k] = fmaxf(hi[k], __shfl_xor_sync(0xffffffffu, hi[k], o));
     }
   }
-  if ((tid & 31) == 0) {
-#pragma unroll
-    for (int k = 0; k < D; ++k) {
-      atomicMin(&s_box[k], float_ord(lo[k]));
-      atomicMax(&s_box[D + k], float_ord(hi[k]));
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int k = 0; k < D; ++k) {
-    lo[k] = ord_float(s_box[k]);
-    hi[k] = ord_float(s_box[D + k]);
-  }
-  auto tile_ub = [&](int tt) -> float {
-    const float* bx = P.key_box + static_cast<int64_t>(tt) * 2 * D;
+  // upper bound of the exponents of entry idx of a component-major summary (stride n)
+  auto ub_of = [&](const float* box, const float* hm, int n, int idx) -> float {
     float d2 = 0.0f;
 #pragma unroll
     for (int k = 0; k < D; ++k) {
-      const float gap = fmaxf(fmaxf(bx[k] - hi[k], lo[k] - bx[D + k]), 0.0f);
+      const float gap = fmaxf(fmaxf(box[k * n + idx] - hi[k], lo[k] - box[(D + k) * n + idx]), 0.0f);
       d2 = fmaf(gap, gap, d2);
     }
-    return P.key_hmax[tt] - P.kappa_f * d2;
+    return hm[idx] - P.kappa_f * d2;
+  };
+  // warp argmax of (ub, -index): key = ordered ub << 32 | ~index
+  auto best_of = [&](float ub, int idx, bool ok) -> unsigned long long {
+    unsigned long long key =
+        ok ? (static_cast<unsigned long long>(static_cast<unsigned>(float_ord(ub)) ^ 0x80000000u) << 32) |
+                 static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<unsigned>(idx))
+           : 0ull;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
+      key = key > other ? key : other;
+    }
+    return key;
   };
 
-  // anchor: the largest upper bound, ties to the lower tile index
+  // anchor: the tile with the largest upper bound (ties to the lower index), found through
+  // the super-tiles: the best tile of the best super-tile gives a bound L, and only
+  // super-tiles whose own bound exceeds L can hold a better tile.
   unsigned long long best = 0ull;
-  for (int tt = tid; tt < n_tiles; tt += NT) {
-    const unsigned ub = static_cast<unsigned>(float_ord(tile_ub(tt))) ^ 0x80000000u;
-    const unsigned long long key = (static_cast<unsigned long long>(ub) << 32) |
-                                   static_cast<unsigned long long>(0xFFFFFFFFu - tt);
-    best = best > key ? best : key;
+  for (int s0 = 0; s0 < S; s0 += 32) {
+    const int sidx = s0 + lane;
+    const unsigned long long k = best_of(sidx < S ? ub_of(P.key_sbox, P.key_shmax, S, sidx) : 0.0f,
+                                         sidx, sidx < S);
+    best = best > k ? best : k;
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-    best = best > other ? best : other;
+  const int sstar = static_cast<int>(0xFFFFFFFFu - static_cast<unsigned>(best & 0xFFFFFFFFull));
+  {
+    const int t = sstar * kSuper + lane;
+    const bool ok = lane < kSuper && t < T;
+    best = best_of(ok ? ub_of(P.key_box, P.key_hmax, T, t) : 0.0f, t, ok);
   }
-  if ((tid & 31) == 0) atomicMax(&s_best, best);
-  __syncthreads();
-  const int anchor = static_cast<int>(0xFFFFFFFFu - static_cast<unsigned>(s_best & 0xFFFFFFFFull));
+  for (int s0 = 0; s0 < S; s0 += 32) {
+    const int sidx = s0 + lane;
+    const float lbest = ord_float(static_cast<int>(static_cast<unsigned>(best >> 32) ^ 0x80000000u));
+    unsigned sbits = __ballot_sync(
+        0xffffffffu, sidx < S && sidx != sstar && ub_of(P.key_sbox, P.key_shmax, S, sidx) >= lbest);
+    while (sbits) {
+      const int sl = __ffs(sbits) - 1;
+      sbits &= sbits - 1u;
+      const int t = (s0 + sl) * kSuper + lane;
+      const bool ok = lane < kSuper && t < T;
+      const unsigned long long k = best_of(ok ? ub_of(P.key_box, P.key_hmax, T, t) : 0.0f, t, ok);
+      best = best > k ? best : k;
+    }
+  }
+  const int anchor = static_cast<int>(0xFFFFFFFFu - static_cast<unsigned>(best & 0xFFFFFFFFull));
 
-  // the anchor's keys, then each row's largest exponent over them
+  // the anchor's keys, then each row's largest exponent over them (packed, direct form)
   {
     const float4* src = reinterpret_cast<const float4*>(P.keys + static_cast<int64_t>(anchor) * TP * KP);
     float4* dst = reinterpret_cast<float4*>(anchor_tile);
-    for (int q = tid; q < TP * KP / 4; q += NT) dst[q] = src[q];
+    for (int q = lane; q < TP * KP / 4; q += 32) dst[q] = src[q];
   }
-  __syncthreads();
+  __syncwarp();
+  u64 xp[R][D];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+#pragma unroll
+    for (int k = 0; k < D; ++k) xp[r][k] = pk(x[r][k], x[r][k]);
+  }
+  const u64 nkappa = pk(-P.kappa_f, -P.kappa_f);
   float zmax[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) zmax[r] = -INFINITY;
+#pragma unroll 4
   for (int p = 0; p < TP; ++p) {
-    const float* kp = anchor_tile + p * KP;
+    u64 comp[KP / 2];
+    load_pair<D>(anchor_tile, p, comp);
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float h = kp[2 * D + e];
+    for (int r = 0; r < R; ++r) {
+      u64 acc = pk(0.0f, 0.0f);
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        float d2 = 0.0f;
-#pragma unroll
-        for (int k = 0; k < D; ++k) {
-          const float dk = x[r][k] - kp[2 * k + e];
-          d2 = fmaf(dk, dk, d2);
-        }
-        zmax[r] = fmaxf(zmax[r], fmaf(-P.kappa_f, d2, h));
+      for (int k = 0; k < D; ++k) {
+        const u64 dk = sub2(xp[r][k], comp[k]);
+        acc = fma2(dk, dk, acc);
       }
+      float z0, z1;
+      upk(fma2(nkappa, acc, comp[D]), z0, z1);
+      zmax[r] = max3(zmax[r], z0, z1);
     }
   }
   const bool history = P.lse_prev && P.key_dmin;
@@ -159,32 +171,43 @@ __global__ void __launch_bounds__(NT) screen_kernel(const PassParams P, unsigned
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     if (!valid[r]) continue;
+    const int64_t i = row0 + r * 32 + lane;
     float v = zmax[r];
-    if (history) v = fmaxf(v, P.lse_prev[row0 + r * NT + tid] + dmin - P.log2_keys);
+    if (history) v = fmaxf(v, P.lse_prev[i] + dmin - P.log2_keys);
+    if (P.row_mlb) P.row_mlb[i] = v;
     mlb = fminf(mlb, v);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mlb = fminf(mlb, __shfl_xor_sync(0xffffffffu, mlb, o));
-  if ((tid & 31) == 0) atomicMin(&s_mlb, float_ord(mlb));
-  __syncthreads();
-  const float thr = ord_float(s_mlb) - P.skip_margin;
+  const float thr = mlb - P.skip_margin;
 
-  // the mask: one warp writes 32 consecutive tiles per word
+  // the mask, 32 super-tiles (8 mask words) per round; lane j < 8 assembles word j
   unsigned* mrow = kmask + b * P.mask_words;
   int cnt = 0;
-  for (int base = 0; base < n_tiles; base += NT) {
-    const int tt = base + tid;
-    const bool keep = tt < n_tiles && (tt == anchor || tile_ub(tt) >= thr);
-    const unsigned word = __ballot_sync(0xffffffffu, keep);
-    const int w = (base + (tid & ~31)) >> 5;
-    if ((tid & 31) == 0 && w < P.mask_words) {
+  for (int s0 = 0; s0 < S; s0 += 32) {
+    const int sidx = s0 + lane;
+    const bool keep_s =
+        sidx < S && (sidx == anchor / kSuper || ub_of(P.key_sbox, P.key_shmax, S, sidx) >= thr);
+    unsigned sbits = __ballot_sync(0xffffffffu, keep_s);
+    unsigned word = 0u;
+    while (sbits) {
+      const int sl = __ffs(sbits) - 1;
+      sbits &= sbits - 1u;
+      const int t = (s0 + sl) * kSuper + lane;
+      const bool keep_t =
+          lane < kSuper && t < T && (t == anchor || ub_of(P.key_box, P.key_hmax, T, t) >= thr);
+      const unsigned pat = __ballot_sync(0xffffffffu, keep_t) & 0xFFu;
+      if (lane == sl / 4) word |= pat << ((sl % 4) * kSuper);
+    }
+    const int w = s0 / 4 + lane;
+    if (lane < 8 && w < P.mask_words) {
       mrow[w] = word;
       cnt += __popc(word);
     }
   }
-  if ((tid & 31) == 0) atomicAdd(&s_cnt, cnt);
-  __syncthreads();
-  if (tid == 0) kcount[b] = s_cnt;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if (lane == 0) kcount[b] = cnt;
 }
 
 // One CTA of 1024 threads: C = max(1, ceil(K / budget)) for K kept tiles in all, the units
@@ -198,43 +221,41 @@ __global__ void __launch_bounds__(1024) plan_units_kernel(const int* kcount, int
   __shared__ long long s_part[32];
   __shared__ int s_scan[32];
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  // thread t owns row blocks [t * per, (t + 1) * per)
+  const int per = (rb + 1023) / 1024;
+  const int b0 = min(rb, tid * per), b1 = min(rb, b0 + per);
   long long k = 0;
-  for (int b = tid; b < rb; b += 1024) k += kcount[b];
+  for (int b = b0; b < b1; ++b) k += kcount[b];
+  long long kw = k;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
-  if (lane == 0) s_part[wid] = k;
+  for (int o = 16; o > 0; o >>= 1) kw += __shfl_xor_sync(0xffffffffu, kw, o);
+  if (lane == 0) s_part[wid] = kw;
   __syncthreads();
   long long total = 0;
   for (int q = 0; q < 32; ++q) total += s_part[q];
   const long long C = total > budget ? (total + budget - 1) / budget : 1;
-  int carry = 0;
-  for (int base = 0; base < rb; base += 1024) {
-    const int b = base + tid;
-    const int nu = b < rb ? static_cast<int>((kcount[b] + C - 1) / C) : 0;
-    int incl = nu;
+  int nu = 0;
+  for (int b = b0; b < b1; ++b) nu += static_cast<int>((kcount[b] + C - 1) / C);
+  int incl = nu;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    __syncthreads();  // s_scan free from the previous round
-    if (lane == 31) s_scan[wid] = incl;
-    __syncthreads();
-    int wbase = 0;
-    for (int q = 0; q < wid; ++q) wbase += s_scan[q];
-    int all = 0;
-    for (int q = 0; q < 32; ++q) all += s_scan[q];
-    const int start = carry + wbase + incl - nu;
-    if (b < rb) {
-      unit_start[b] = start;
-      for (int j = 0; j < nu; ++j) unit_rb[start + j] = b;
-    }
-    carry += all;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
   }
-  if (tid == 0) {
-    unit_start[rb] = carry;
+  if (lane == 31) s_scan[wid] = incl;
+  __syncthreads();
+  int start = incl - nu;
+  for (int q = 0; q < wid; ++q) start += s_scan[q];
+  for (int b = b0; b < b1; ++b) {
+    const int n = static_cast<int>((kcount[b] + C - 1) / C);
+    unit_start[b] = start;
+    for (int j = 0; j < n; ++j) unit_rb[start + j] = b;
+    start += n;
+  }
+  if (tid == 1023) {
+    unit_start[rb] = start;
     qscal[0] = static_cast<int>(C);
-    qscal[1] = carry;
+    qscal[1] = start;
     *kept_out = total;
     if (evaluated)
       atomicAdd(evaluated, static_cast<unsigned long long>(total) * kScreenTile * rb_rows);

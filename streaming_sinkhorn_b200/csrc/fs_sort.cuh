@@ -149,13 +149,16 @@ __global__ void __launch_bounds__(256) perm_from_keys_kernel(const uint64_t* key
   if (j < count) perm[j] = static_cast<int>(keys[j] & 0xFFFFFFFFull);
 }
 
-// Bounding box (all D coordinates) of each 256-point tile of a packed cloud, as floats
-// box[T][0..D) = lo, box[T][D..2D) = hi. Only real points count.
+// Bounding box (all D coordinates) of each 256-point tile of a packed cloud, stored by
+// component: box[k * T + t] = lo_k, box[(D + k) * T + t] = hi_k of tile t (T tiles), so that
+// a warp scanning consecutive tiles reads each component in one coalesced request. Only
+// real points count.
 template <int D>
-__global__ void __launch_bounds__(256) tile_box_kernel(const float* keys, int64_t count, float* box) {
+__global__ void __launch_bounds__(256) tile_box_kernel(const float* keys, int64_t count, float* box,
+                                                       int64_t T) {
   constexpr int KP = ((2 * (D + 1) + 3) / 4) * 4;
-  const int64_t T = blockIdx.x;
-  const int64_t j = T * 256 + threadIdx.x;
+  const int64_t t = blockIdx.x;
+  const int64_t j = t * 256 + threadIdx.x;
   __shared__ float red[2][D][8];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
 #pragma unroll
@@ -182,8 +185,8 @@ __global__ void __launch_bounds__(256) tile_box_kernel(const float* keys, int64_
       v = fminf(v, red[0][k][q]);
       u = fmaxf(u, red[1][k][q]);
     }
-    box[T * 2 * D + k] = v;
-    box[T * 2 * D + D + k] = u;
+    box[k * T + t] = v;
+    box[(D + k) * T + t] = u;
   }
 }
 
@@ -205,6 +208,28 @@ __global__ void __launch_bounds__(256) tile_hmax_kernel(const float* keys, int64
     float m = red[0];
     for (int q = 1; q < 8; ++q) m = fmaxf(m, red[q]);
     hmax[T] = m;
+  }
+}
+
+// Super-tiles: runs of kSuper consecutive tiles (2048 points), summarised the same way, so
+// that screening can reject a whole run with one test. One thread per super-tile; `nc`
+// components of stride T (tiles) and S (super-tiles); `take_max` picks max over the run
+// (biases, upper box corners) or min (lower corners) per component.
+constexpr int kSuper = 8;
+
+__global__ void __launch_bounds__(256) super_reduce_kernel(const float* v, int64_t T, float* out,
+                                                           int64_t S, int nc, int n_min) {
+  const int64_t s = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (s >= S) return;
+  const int64_t t0 = s * kSuper, t1 = t0 + kSuper < T ? t0 + kSuper : T;
+  for (int c = 0; c < nc; ++c) {
+    const bool take_min = c < n_min;
+    float r = take_min ? INFINITY : -INFINITY;
+    for (int64_t t = t0; t < t1; ++t) {
+      const float x = v[c * T + t];
+      r = take_min ? fminf(r, x) : fmaxf(r, x);
+    }
+    out[c * S + s] = r;
   }
 }
 
