@@ -127,6 +127,7 @@ constexpr Variant kWideVariant = {1, 128};
 // and no warp waits at a barrier for another warp's tiles.
 constexpr int kQueueVariant = 2;
 constexpr Variant kQueueShape = {2, 32};
+constexpr int kQueueStages = 2;  // one tile in flight while one is consumed
 
 struct Plan {
   int variant;  // index into the variant table of this pass type
@@ -146,8 +147,8 @@ int num_sms_current() {
   return sms > 0 ? sms : 148;
 }
 
-size_t pass_smem_bytes(int D, int tile_pairs) {
-  return static_cast<size_t>(kStages) * tile_pairs * key_pair_floats(D) * 4;
+size_t pass_smem_bytes(int D, int tile_pairs, int stages = kStages) {
+  return static_cast<size_t>(stages) * tile_pairs * key_pair_floats(D) * 4;
 }
 
 int occupancy_for(int D, bool grad, int variant, size_t smem);  // defined after the kernels
@@ -245,7 +246,8 @@ QPlan make_qplan(const Plan& pl, int64_t key_pairs, int D, bool grad, int sms, b
          q.rb * q.mask_words <= kMaskCapWords;
   if (!q.on) return q;
   const int64_t slots = static_cast<int64_t>(sms) *
-                        occupancy_for(D, grad, kQueueVariant, pass_smem_bytes(D, kScreenTile / 2));
+                        occupancy_for(D, grad, kQueueVariant,
+                                      pass_smem_bytes(D, kScreenTile / 2, kQueueStages));
   q.budget = kUnitWaves * slots;
   q.units_max = q.budget + q.rb;
   return q;
@@ -448,27 +450,27 @@ inline bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr)
 
 // ---------------- kernel dispatch ----------------
 
-template <int D, int R, int NT, bool GRAD, int G, int MINB>
+template <int D, int R, int NT, bool GRAD, int G, int MINB, int ST = kStages>
 struct PassKernel {
-  static constexpr auto fn = lse_pass_kernel<D, R, NT, G, GRAD, MINB>;
+  static constexpr auto fn = lse_pass_kernel<D, R, NT, G, GRAD, MINB, ST>;
   static void set_smem_attr() {
     static bool done = false;  // idempotent, so a race between threads is harmless
     if (!done) {
       CK(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(pass_smem_bytes(D, 128))));
+                              static_cast<int>(pass_smem_bytes(D, 128, ST))));
       done = true;
     }
   }
   static void launch(const PassParams& P, const Plan& pl, cudaStream_t st) {
     set_smem_attr();
     dim3 grid(static_cast<unsigned>(pl.row_blocks), static_cast<unsigned>(pl.n_splits));
-    fn<<<grid, NT, pass_smem_bytes(D, pl.tile_pairs), st>>>(P);
+    fn<<<grid, NT, pass_smem_bytes(D, pl.tile_pairs, ST), st>>>(P);
     CK(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
   static void launch_queue(const PassParams& P, int64_t units, cudaStream_t st) {
     set_smem_attr();
-    fn<<<static_cast<unsigned>(units), NT, pass_smem_bytes(D, kScreenTile / 2), st>>>(P);
+    fn<<<static_cast<unsigned>(units), NT, pass_smem_bytes(D, kScreenTile / 2, ST), st>>>(P);
     CK(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
@@ -506,14 +508,14 @@ void with_pass_kernel(bool grad, int variant, Op&& op) {
       else if (variant == 1)
         op.template run<PassKernel<D, 1, 128, true, 8, 4>>();
       else
-        op.template run<PassKernel<D, 2, 32, true, 8, 12>>();
+        op.template run<PassKernel<D, 2, 32, true, 8, 12, kQueueStages>>();
     } else {
       if (variant == 0)
         op.template run<PassKernel<D, 2, 128, false, 8, 6>>();
       else if (variant == 1)
         op.template run<PassKernel<D, 1, 128, false, 8, 8>>();
       else
-        op.template run<PassKernel<D, 2, 32, false, 8, 24>>();
+        op.template run<PassKernel<D, 2, 32, false, 8, 24, kQueueStages>>();
     }
   }
 }

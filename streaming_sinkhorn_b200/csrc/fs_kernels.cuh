@@ -214,8 +214,9 @@ __device__ __forceinline__ void load_pair(const float* tile, int p, u64 (&comp)[
   }
 }
 
-template <int D, int R, int NT, int G, bool GRAD, int MINB>
+template <int D, int R, int NT, int G, bool GRAD, int MINB, int ST>
 __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) {
+  constexpr int kStages = ST;  // depth of the copy ring
   constexpr int KP = key_pair_floats(D);
   constexpr int NA = GRAD ? D : 1;
   constexpr int RB = R * NT;  // rows of one row block
@@ -323,10 +324,22 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
   // offset m (log2 units), `base` (m, or 0 while no column has set it) and mk = base/kappa
   // folded into the distance accumulator; the running sums L (two lanes: even and odd
   // columns) and, for the gradient, the weighted differences A = sum p (x - y).
+  //
+  // One-warp CTAs (CEN) use the centred expanded form instead. With c the centre of the
+  // warp's row box, x' = x - c and y' = y - c,
+  //   z - base = (H - kappa |y'|^2) - (base + kappa |x'|^2) + sum_k (2 kappa x'_k) y'_k,
+  // so each tile is rewritten once in place to (y', H' = H - kappa |y'|^2), X holds
+  // 2 kappa x', mk holds -(base + kappa |x'|^2), and a pair costs D + 1 packed operations
+  // instead of 2D + 1. Centring keeps every magnitude at the scale of the row box and the
+  // kept tiles around it, where the direct form's rounding also lives. The gradient then
+  // accumulates A = sum p y' and forms sum p (x - y) = x' L - A at the end.
+  constexpr bool CEN = NT == 32;
   u64 X[R][D];
   float m[R], base[R];
   u64 mk[R], L[R];
   u64 A[R][NA];
+  float q[R];        // CEN: kappa |x'|^2
+  u64 cpk[D];        // CEN: the centre, in both lanes
   const u64 nkappa = pk(-P.kappa_f, -P.kappa_f);
 #pragma unroll
   for (int r = 0; r < R; ++r) {
@@ -343,6 +356,64 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
 #pragma unroll
     for (int k = 0; k < NA; ++k) A[r][k] = pk(0.0f, 0.0f);
   }
+  if constexpr (CEN) {
+#pragma unroll
+    for (int k = 0; k < D; ++k) {
+      float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (row0 + r * NT + tid < P.n_rows) {
+          float c0, c1;
+          upk(X[r][k], c0, c1);
+          lo = fminf(lo, c0);
+          hi = fmaxf(hi, c0);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+      }
+      const float c = lo <= hi ? 0.5f * (lo + hi) : 0.0f;
+      cpk[k] = pk(c, c);
+    }
+    const float k2 = 2.0f * P.kappa_f;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float s2 = 0.0f;
+#pragma unroll
+      for (int k = 0; k < D; ++k) {
+        float c0, c1, cc, cd;
+        upk(X[r][k], c0, c1);
+        upk(cpk[k], cc, cd);
+        const float xs = c0 - cc;
+        s2 = fmaf(xs, xs, s2);
+        X[r][k] = pk(k2 * xs, k2 * xs);
+      }
+      q[r] = P.kappa_f * s2;
+      mk[r] = pk(-q[r], -q[r]);
+    }
+  }
+  // CEN: rewrite a tile in place to (y', H'); pairs are spread over the warp's lanes.
+  auto centre_tile = [&](float* tile) {
+    if constexpr (CEN) {
+      for (int p = tid; p < P.tile_pairs; p += 32) {
+        u64 comp[KP / 2];
+        load_pair<D>(tile, p, comp);
+        u64 s2 = pk(0.0f, 0.0f);
+#pragma unroll
+        for (int k = 0; k < D; ++k) {
+          comp[k] = sub2(comp[k], cpk[k]);
+          s2 = fma2(comp[k], comp[k], s2);
+        }
+        comp[D] = fma2(nkappa, s2, comp[D]);
+        ulonglong2* pv = reinterpret_cast<ulonglong2*>(tile + p * KP);
+#pragma unroll
+        for (int v = 0; v < KP / 4; ++v) pv[v] = make_ulonglong2(comp[2 * v], comp[2 * v + 1]);
+      }
+      __syncwarp();
+    }
+  };
 
   // Online max/sum of this thread's rows over one key tile in shared memory.
   auto process_tile = [&](const float* tile) {
@@ -354,13 +425,20 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
         load_pair<D>(tile, pg + g, comp);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          u64 acc = mk[r];
+          if constexpr (CEN) {
+            u64 acc = add2(comp[D], mk[r]);  // H' - base - kappa |x'|^2
 #pragma unroll
-          for (int k = 0; k < D; ++k) {
-            const u64 dk = sub2(X[r][k], comp[k]);
-            acc = fma2(dk, dk, acc);
+            for (int k = 0; k < D; ++k) acc = fma2(X[r][k], comp[k], acc);
+            tv[r][g] = acc;
+          } else {
+            u64 acc = mk[r];
+#pragma unroll
+            for (int k = 0; k < D; ++k) {
+              const u64 dk = sub2(X[r][k], comp[k]);
+              acc = fma2(dk, dk, acc);
+            }
+            tv[r][g] = fma2(nkappa, acc, comp[D]);  // H - kappa (m/kappa + |x - y|^2)
           }
-          tv[r][g] = fma2(nkappa, acc, comp[D]);  // H - kappa (m/kappa + |x - y|^2)
         }
       }
       // Group max; lazy rescale of the running sums (always on a row's first real group).
@@ -388,8 +466,13 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
           for (int g = 0; g < G; ++g) tv[r][g] = add2(tv[r][g], sh);
           m[r] = mx_abs;
           base[r] = mx_abs;
-          const float q = mx_abs * P.inv_kappa_f;
-          mk[r] = pk(q, q);
+          if constexpr (CEN) {
+            const float nb = -(mx_abs + q[r]);
+            mk[r] = pk(nb, nb);
+          } else {
+            const float qb = mx_abs * P.inv_kappa_f;
+            mk[r] = pk(qb, qb);
+          }
         }
       }
 #pragma unroll
@@ -404,7 +487,8 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
           L[r] = add2(L[r], e);
           if (GRAD) {
 #pragma unroll
-            for (int k = 0; k < NA; ++k) A[r][k] = fma2(e, sub2(X[r][k], comp[k]), A[r][k]);
+            for (int k = 0; k < NA; ++k)
+              A[r][k] = CEN ? fma2(e, comp[k], A[r][k]) : fma2(e, sub2(X[r][k], comp[k]), A[r][k]);
           }
         }
       }
@@ -435,7 +519,10 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       mbar_expect_tx(&bars[ps], stage_bytes);
       bulk_g2s(stages + ps * stage_floats, tile_src(t - 1 + kStages), stage_bytes, &bars[ps]);
     }
+    if constexpr (CEN) centre_tile(stages + st * stage_floats);
     process_tile(stages + st * stage_floats);
+    // the stage was written by this (generic) proxy: order that before its next copy
+    if constexpr (CEN) fence_proxy_async_smem();
   }
   if (queue && P.evaluated && tid == 0 && n_work > 0)
     atomicAdd(P.evaluated, static_cast<unsigned long long>(n_work) * kScreenTile * RB);
@@ -452,6 +539,18 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     return;
   }
 
+  // sum_j p_ij (x_i - y_j) of row r, component k, for row sum l (same offset)
+  auto diff_sum = [&](int r, int k, float l) -> float {
+    float a0, a1;
+    upk(A[r][k], a0, a1);
+    if constexpr (CEN) {
+      float x0, x1;
+      upk(X[r][k], x0, x1);
+      return x0 * (0.5f * P.inv_kappa_f) * l - (a0 + a1);
+    }
+    return a0 + a1;
+  };
+
   if (n_units == 1) {
     double dev_sum = 0.0, dev_max = 0.0, mass = 0.0;
     float dmin = INFINITY;
@@ -465,11 +564,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       if (GRAD) {
         float a[NA];
 #pragma unroll
-        for (int k = 0; k < NA; ++k) {
-          float a0, a1;
-          upk(A[r][k], a0, a1);
-          a[k] = a0 + a1;
-        }
+        for (int k = 0; k < NA; ++k) a[k] = diff_sum(r, k, l);
         finish_grad(P, i, a, l);
       } else {
         const double lse2 = static_cast<double>(m[r]) + log2(static_cast<double>(l));
@@ -502,11 +597,8 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       P.part_l[o] = l0 + l1;
       if (GRAD) {
 #pragma unroll
-        for (int k = 0; k < NA; ++k) {
-          float a0, a1;
-          upk(A[r][k], a0, a1);
-          P.part_a[(unit * D + k) * pstride + poff + i] = a0 + a1;
-        }
+        for (int k = 0; k < NA; ++k)
+          P.part_a[(unit * D + k) * pstride + poff + i] = diff_sum(r, k, l0 + l1);
       }
     }
   }
