@@ -120,14 +120,16 @@ int64_t pairs_pad(int64_t count) { return round_up(ceil_div(count, 2), kPairPad)
 struct Variant {
   int R, NT;
 };
-constexpr Variant kLseVariants[2] = {{2, 128}, {1, 128}};
-constexpr Variant kGradVariants[2] = {{2, 128}, {1, 128}};
+// d <= 16: one warp per CTA over 64 rows, so each warp centres, streams (and, screened,
+// screens and merges) on its own and never waits at a barrier for another warp's tiles.
+constexpr Variant kNarrowVariant = {2, 32};
+constexpr int kNarrowStages = 2;  // one tile in flight while one is consumed
+// d > 16 (the gradient pass of wide points): four warps share each tile.
 constexpr Variant kWideVariant = {1, 128};
-// Queue mode: one warp per CTA, 64 rows, so each warp screens, streams and merges on its own
-// and no warp waits at a barrier for another warp's tiles.
-constexpr int kQueueVariant = 2;
-constexpr Variant kQueueShape = {2, 32};
-constexpr int kQueueStages = 2;  // one tile in flight while one is consumed
+constexpr int kQueueVariant = 0;
+constexpr Variant kQueueShape = kNarrowVariant;
+constexpr int kQueueStages = kNarrowStages;
+inline int stages_for(int D) { return D > 16 ? kStages : kNarrowStages; }
 
 struct Plan {
   int variant;  // index into the variant table of this pass type
@@ -154,20 +156,10 @@ size_t pass_smem_bytes(int D, int tile_pairs, int stages = kStages) {
 int occupancy_for(int D, bool grad, int variant, size_t smem);  // defined after the kernels
 
 Plan make_plan(int64_t n_rows, int64_t key_pairs, int D, bool grad, int sms) {
-  const int64_t fill = static_cast<int64_t>(sms) * 4;
+  const int64_t fill = static_cast<int64_t>(sms) * (D > 16 ? 4 : 16);
   const int max_tile = D > 16 ? 32 : 128;
-  const Variant* vars;
-  int nv;
-  if (D > 16) {
-    vars = &kWideVariant;
-    nv = 1;
-  } else if (grad) {
-    vars = kGradVariants;
-    nv = 2;
-  } else {
-    vars = kLseVariants;
-    nv = 2;
-  }
+  const Variant* vars = D > 16 ? &kWideVariant : &kNarrowVariant;
+  const int nv = 1;
   Plan p{};
   p.n_rows = n_rows;
   // Most rows per CTA whose (row blocks x tiles) still fills the machine; else the smallest.
@@ -193,7 +185,8 @@ Plan make_plan(int64_t n_rows, int64_t key_pairs, int D, bool grad, int sms) {
   // Take the fewest splits whose last wave is at least 97 % full, else the best one within
   // max(4 waves, 3 splits per row block) units (which bounds the partial buffers).
   const int64_t slots =
-      static_cast<int64_t>(sms) * occupancy_for(D, grad, chosen, pass_smem_bytes(D, tile));
+      static_cast<int64_t>(sms) *
+      occupancy_for(D, grad, chosen, pass_smem_bytes(D, tile, stages_for(D)));
   const int64_t max_units = std::max<int64_t>(4 * slots, 3 * p.row_blocks);
   int64_t best_s = 1;
   double best_eff = -1.0;
@@ -502,21 +495,11 @@ void with_pass_kernel(bool grad, int variant, Op&& op) {
     else
       op.template run<PassKernel<D, 1, 128, false, 4, 1>>();
   } else {
-    if (grad) {
-      if (variant == 0)
-        op.template run<PassKernel<D, 2, 128, true, 8, 3>>();
-      else if (variant == 1)
-        op.template run<PassKernel<D, 1, 128, true, 8, 4>>();
-      else
-        op.template run<PassKernel<D, 2, 32, true, 8, 12, kQueueStages>>();
-    } else {
-      if (variant == 0)
-        op.template run<PassKernel<D, 2, 128, false, 8, 6>>();
-      else if (variant == 1)
-        op.template run<PassKernel<D, 1, 128, false, 8, 8>>();
-      else
-        op.template run<PassKernel<D, 2, 32, false, 8, 24, kQueueStages>>();
-    }
+    (void)variant;
+    if (grad)
+      op.template run<PassKernel<D, 2, 32, true, 8, 12, kNarrowStages>>();
+    else
+      op.template run<PassKernel<D, 2, 32, false, 8, 24, kNarrowStages>>();
   }
 }
 
