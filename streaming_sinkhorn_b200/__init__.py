@@ -18,7 +18,8 @@ import ctypes
 from . import _lib
 
 __all__ = ["potentials", "cost", "grad_x", "marginal_residual", "solve_host", "workspace_bytes",
-           "FsError", "timing_enable", "timing_reset", "timing_get", "launch_count"]
+           "FsError", "timing_enable", "timing_reset", "timing_get", "launch_count",
+           "screening_enable"]
 
 
 class FsError(RuntimeError):
@@ -239,6 +240,11 @@ def timing_enable(on: bool = True) -> None:
 
 def timing_reset() -> None:
     _lib.load().fs_timing_reset()
+
+
+def screening_enable(on: bool = True) -> None:
+    """Turns block screening on or off for later calls (fs_screening_enable)."""
+    _lib.load().fs_screening_enable(1 if on else 0)
 
 
 def launch_count() -> int:

@@ -25,7 +25,7 @@ EXPORTS = (
     "fs_status_string", "fs_last_cuda_error", "fs_workspace_bytes", "fs_potentials", "fs_cost",
     "fs_grad_x", "fs_marginal_residual", "fs_solve_host_workspace_bytes", "fs_solve_host",
     "fs_timing_enable", "fs_timing_reset", "fs_timing_get", "fs_launch_count",
-    "fs_potentials_noalloc",
+    "fs_potentials_noalloc", "fs_screening_enable",
 )
 
 
@@ -79,6 +79,8 @@ def load():
         fn.restype = ctypes.c_int
     lib.fs_timing_enable.argtypes = [ctypes.c_int]
     lib.fs_timing_enable.restype = None
+    lib.fs_screening_enable.argtypes = [ctypes.c_int]
+    lib.fs_screening_enable.restype = None
     lib.fs_timing_reset.argtypes = []
     lib.fs_timing_reset.restype = None
     lib.fs_timing_get.argtypes = [ctypes.POINTER(fs_timing)]

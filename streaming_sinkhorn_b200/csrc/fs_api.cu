@@ -31,6 +31,7 @@ inline void ck(cudaError_t e, const char* what) {
 // ---------------- kernel timing ----------------
 std::mutex g_timing_mu;
 bool g_timing_on = false;
+std::atomic<bool> g_screening{true};
 fs_timing g_timing = {};
 
 enum TimedKind { kTLse = 0, kTGrad = 1, kTMarg = 2, kTCombine = 3, kTScreen = 4 };
@@ -1066,7 +1067,8 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
   P.err = err_ptr(c.scal);
   int* dmin_slots = reinterpret_cast<int*>(c.scal + kDmin);
   const int tk = grad ? kTGrad : (kind == kMarg ? kTMarg : kTLse);
-  const QPlan q = make_qplan(pl, key_pairs, c.L.D, grad, c.sms, c.L.sorted && !c.no_screen);
+  const QPlan q = make_qplan(pl, key_pairs, c.L.D, grad, c.sms,
+                             c.L.sorted && !c.no_screen && g_screening.load());
   if (c.L.sorted) {
     P.perm = rows_x ? c.perm_x : c.perm_y;
     P.evaluated = reinterpret_cast<unsigned long long*>(c.scal + kEval + tk);
@@ -1429,6 +1431,8 @@ fs_status fs_solve_host(const fs_problem* hp, int32_t n_iters, float* f, float* 
 }
 
 int64_t fs_launch_count(void) { return fs::g_launches.load(std::memory_order_relaxed); }
+
+void fs_screening_enable(int on) { fs::g_screening.store(on != 0); }
 
 void fs_timing_enable(int on) {
   std::lock_guard<std::mutex> lk(fs::g_timing_mu);

@@ -331,8 +331,9 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
   // so each tile is rewritten once in place to (y', H' = H - kappa |y'|^2), X holds
   // 2 kappa x', mk holds -(base + kappa |x'|^2), and a pair costs D + 1 packed operations
   // instead of 2D + 1. Centring keeps every magnitude at the scale of the row box and the
-  // kept tiles around it, where the direct form's rounding also lives. The gradient then
-  // accumulates A = sum p y' and forms sum p (x - y) = x' L - A at the end.
+  // kept tiles around it, where the direct form's rounding also lives. The gradient
+  // accumulates sum p (y' - x') term by term (x' recovered from X), not x' L - sum p y',
+  // whose cancellation would cost digits when x is close to its barycentre.
   constexpr bool CEN = NT == 32;
   u64 X[R][D];
   float m[R], base[R];
@@ -341,6 +342,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
   float q[R];        // CEN: kappa |x'|^2
   u64 cpk[D];        // CEN: the centre, in both lanes
   const u64 nkappa = pk(-P.kappa_f, -P.kappa_f);
+  const u64 nhalf_ik = pk(-0.5f * P.inv_kappa_f, -0.5f * P.inv_kappa_f);  // X -> -x'
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     const int64_t i = row0 + r * NT + tid;
@@ -488,7 +490,8 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
           if (GRAD) {
 #pragma unroll
             for (int k = 0; k < NA; ++k)
-              A[r][k] = CEN ? fma2(e, comp[k], A[r][k]) : fma2(e, sub2(X[r][k], comp[k]), A[r][k]);
+              A[r][k] = CEN ? fma2(e, fma2(X[r][k], nhalf_ik, comp[k]), A[r][k])  // e (y' - x')
+                            : fma2(e, sub2(X[r][k], comp[k]), A[r][k]);
           }
         }
       }
@@ -539,16 +542,11 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     return;
   }
 
-  // sum_j p_ij (x_i - y_j) of row r, component k, for row sum l (same offset)
-  auto diff_sum = [&](int r, int k, float l) -> float {
+  // sum_j p_ij (x_i - y_j) of row r, component k (CEN accumulates its negative)
+  auto diff_sum = [&](int r, int k) -> float {
     float a0, a1;
     upk(A[r][k], a0, a1);
-    if constexpr (CEN) {
-      float x0, x1;
-      upk(X[r][k], x0, x1);
-      return x0 * (0.5f * P.inv_kappa_f) * l - (a0 + a1);
-    }
-    return a0 + a1;
+    return CEN ? -(a0 + a1) : a0 + a1;
   };
 
   if (n_units == 1) {
@@ -564,7 +562,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       if (GRAD) {
         float a[NA];
 #pragma unroll
-        for (int k = 0; k < NA; ++k) a[k] = diff_sum(r, k, l);
+        for (int k = 0; k < NA; ++k) a[k] = diff_sum(r, k);
         finish_grad(P, i, a, l);
       } else {
         const double lse2 = static_cast<double>(m[r]) + log2(static_cast<double>(l));
@@ -598,7 +596,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       if (GRAD) {
 #pragma unroll
         for (int k = 0; k < NA; ++k)
-          P.part_a[(unit * D + k) * pstride + poff + i] = diff_sum(r, k, l0 + l1);
+          P.part_a[(unit * D + k) * pstride + poff + i] = diff_sum(r, k);
       }
     }
   }
