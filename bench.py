@@ -67,19 +67,8 @@ def workload(cfg: str, rank: int, n_override=None):
             raise SystemExit("--n applies to the clustered workload (c5) only")
         w = workloads.clustered_cube(n=n_override, seed=4 + 1000 * rank, n_iters=20)
         return dataclasses.replace(w, name=f"clustered_cube_n{n_override}")
-    w = workloads.config(CONFIG_INDEX[cfg])
-    if rank:
-        # an independently seeded replica of the same recipe
-        base = {0: workloads.gaussian_shifted, 1: workloads.gaussian_pair}
-        idx = CONFIG_INDEX[cfg]
-        if idx == 4:
-            w = dataclasses.replace(workloads.clustered_cube(n=w.n, seed=w.seed + 1000 * rank,
-                                                             eps=w.eps, n_iters=w.n_iters),
-                                    name=w.name)
-        elif idx in base:
-            w = dataclasses.replace(base[idx](n=w.n, d=w.d, seed=w.seed + 1000 * rank, eps=w.eps,
-                                              n_iters=w.n_iters), name=w.name)
-    return w
+    # rank r > 0 runs an independently seeded replica of the same recipe
+    return workloads.config(CONFIG_INDEX[cfg], seed_offset=1000 * rank)
 
 
 # ---------------------------------------------------------------- clocks ----------
@@ -207,6 +196,23 @@ def oracle_sample(w, target_s: float):
     return value, oracle.threads(), desc, dt
 
 
+# ---------------------------------------------------------------- ranks ------------
+
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The slowest rank's time; every rank returns it (a MAX all-reduce, or ms alone)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(pairs_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the pairs all ranks processed per step over the slowest time."""
+    return pairs_per_rank_step * world / (ms_per_step / 1e3)
+
+
 # ---------------------------------------------------------------- native arm -------
 
 def run_native(args, rank, world, local_rank):
@@ -270,13 +276,9 @@ def run_native(args, rank, world, local_rank):
     timing = fs.timing_get()
     fs.timing_enable(False)
     clk = clocks.stop()
-    ms_per_step = total_ms / args.steps
-    if dist is not None:
-        t = torch.tensor([ms_per_step], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_per_step = float(t.item())
+    ms_per_step = max_over_ranks(total_ms / args.steps, dist, dev)
     pairs_per_step = float(w.n) * w.m * w.n_iters
-    value = pairs_per_step * world / (ms_per_step / 1e3)
+    value = job_value(pairs_per_step, world, ms_per_step)
 
     # roofline of the dominant kernel: the potential-update pass
     lse = timing["lse_pass"]
@@ -386,14 +388,10 @@ def run_e2e(args, w, dev, world, dist):
         fs.solve_host(xh, yh, ah, bh, eps=w.eps, n_iters=w.n_iters, device=dev, workspace=ws, out=out)
     e1.record(stream)
     e1.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dist, dev)
     h2d = (w.n * w.d + w.m * w.d + w.n + w.m) * 4
     d2h = (w.n + w.m + w.n * w.d) * 4 + 5 * 8
-    return {"value": float(w.n) * w.m * w.n_iters * world / (ms / 1e3), "unit": UNIT,
+    return {"value": job_value(float(w.n) * w.m * w.n_iters, world, ms), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
             "steps": steps, "api": "fs_solve_host (pinned host buffers)"}
 

@@ -145,20 +145,26 @@ CONFIG_NAMES = ("c1_gauss_shift_1k_d2", "c2_gauss_10k_d2", "c3_cube_mix_20k30k_d
                 "c4_mix_50k_d64", "c5_cluster_1m_d3")
 
 
-def config(i: int) -> Workload:
-    """Configuration ``i`` (0-based) of the five named workloads, at full size."""
+def config(i: int, seed_offset: int = 0) -> Workload:
+    """Configuration ``i`` (0-based) of the five named workloads, at full size.
+
+    ``seed_offset`` draws an independent instance of the same recipe (replicas of a
+    multi-process run); 0 is the configuration itself.
+    """
+    o = seed_offset
     if i == 0:
-        w = gaussian_shifted(n=1000, d=2, shift=3.0, seed=0, eps=0.05, n_iters=100)
+        w = gaussian_shifted(n=1000, d=2, shift=3.0, seed=0 + o, eps=0.05, n_iters=100)
     elif i == 1:
-        w = gaussian_pair(n=10000, d=2, seed=1, eps=0.05, n_iters=200)
+        w = gaussian_pair(n=10000, d=2, seed=1 + o, eps=0.05, n_iters=200)
     elif i == 2:
-        w = cube_to_mixture(n=20000, m=30000, d=3, k=8, std=0.05, seed=2, eps=0.01, n_iters=200)
+        w = cube_to_mixture(n=20000, m=30000, d=3, k=8, std=0.05, seed=2 + o, eps=0.01,
+                            n_iters=200)
     elif i == 3:
-        w = mixture_pair(n=50000, d=64, k=10, mean_scale=2.0, std=1.0, seed=3, eps=1.0,
+        w = mixture_pair(n=50000, d=64, k=10, mean_scale=2.0, std=1.0, seed=3 + o, eps=1.0,
                          n_iters=100)
     elif i == 4:
-        w = clustered_cube(n=1 << 20, d=3, k=1000, std=0.01, seed=4, eps=2.0 ** (-40.0 / 3.0),
-                           n_iters=20)
+        w = clustered_cube(n=1 << 20, d=3, k=1000, std=0.01, seed=4 + o,
+                           eps=2.0 ** (-40.0 / 3.0), n_iters=20)
     else:
         raise IndexError(f"no configuration {i}")
     return dataclasses.replace(w, name=CONFIG_NAMES[i])
