@@ -62,6 +62,9 @@ def _load():
     lib.oracle_plan_row_sums.argtypes = [dp, i64, dp, i64, i32, dp, dp, dbl, dp, dp, lp, i64, dp]
     lib.oracle_cost.argtypes = [dp, i64, dp, i64, i32, dp, dp, dbl, dp, dp, dp]
     lib.oracle_grad_x.argtypes = [dp, i64, dp, i64, i32, dp, dp, dbl, dp, lp, i64, dp]
+    lib.oracle_solve.argtypes = [dp, i64, dp, i64, i32, dp, dp, dbl, i32, dbl, i32, i32, i32,
+                                 dbl, i32, dp, dp, dp, ctypes.POINTER(ctypes.c_int32),
+                                 ctypes.POINTER(ctypes.c_int32), dp]
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
     lib.oracle_threads.restype = ctypes.c_int
     for fn in (lib.oracle_lse_update, lib.oracle_potentials, lib.oracle_plan_row_sums,
@@ -175,3 +178,31 @@ def marginal_residual(x, y, a, b, eps: float, f, g) -> np.ndarray:
     dr = np.abs(r - _d(a))
     dc = np.abs(c - _d(b))
     return np.array([dr.sum(), dr.max(), dc.sum(), dc.max()], dtype=np.float64)
+
+
+VARIANTS = {"alternating": 0, "symmetric": 1}
+STOP_MODES = {"fixed": 0, "marginal": 1, "potential": 2}
+
+
+def solve(x, y, a, b, eps: float, *, n_iters: int = 200, variant: str = "alternating",
+          alpha: float = 0.5, stop_mode: str = "fixed", stop_max_iter: int = 20000,
+          stop_tol: float = 1e-6, stop_check_every: int = 5, g_init=None):
+    """The general solve: (f, g, iters_run, converged, final_viol).
+
+    converged is None and final_viol NaN under stop_mode "fixed".
+    """
+    x, y, a, b = _d(x), _d(y), _d(a), _d(b)
+    n, m, d = x.shape[0], y.shape[0], x.shape[1]
+    f = np.empty(n, dtype=np.float64)
+    g = np.empty(m, dtype=np.float64)
+    gi = None if g_init is None else _d(g_init)
+    it = ctypes.c_int32(0)
+    conv = ctypes.c_int32(0)
+    viol = np.zeros(1, dtype=np.float64)
+    _check(_load().oracle_solve(_p(x), n, _p(y), m, d, _p(a), _p(b), float(eps),
+                                VARIANTS[variant], float(alpha), STOP_MODES[stop_mode],
+                                int(n_iters), int(stop_max_iter), float(stop_tol),
+                                int(stop_check_every), None if gi is None else _p(gi), _p(f),
+                                _p(g), ctypes.byref(it), ctypes.byref(conv), _p(viol)))
+    converged = None if conv.value < 0 else bool(conv.value)
+    return f, g, int(it.value), converged, float(viol[0])

@@ -30,6 +30,17 @@
  *  - Plan row sums r_i = sum_j P_ij (column sums by swapping the roles of the
  *    clouds), from which the marginal residuals are formed (SinkSLOT README,
  *    stop_mode "marginal").
+ *  - The general solve (SinkSLOT README, API Reference: variant, alpha, stop_mode,
+ *    stop_max_iter, stop_tol, stop_check_every; iters_run, converged, final_viol):
+ *    variant "alternating" (Gauss-Seidel) is the schedule above; variant "symmetric"
+ *    (Jacobi) computes both updates from the previous iterate and blends them,
+ *    f' = (1 - alpha) f + alpha F(g), g' = (1 - alpha) g + alpha G(f), from f = 0 and
+ *    g = g_init (or 0). Stop mode "fixed" runs n_iters iterations; "marginal" stops at
+ *    the first check where max(|P1 - a|_inf, |P^T 1 - b|_inf) <= stop_tol; "potential"
+ *    at the first check where max(|f - f_prev|_inf, |g - g_prev|_inf) < stop_tol, the
+ *    previous values being those of the last check (of the start for the first one;
+ *    eps * |delta phi| with phi = f / eps is |delta f|). Checks run after every
+ *    stop_check_every-th iteration and after the last one allowed (stop_max_iter).
  *
  * Every function returns 0 on success or a negative code on invalid arguments.
  */
@@ -250,4 +261,114 @@ int oracle_grad_x(const double* x, int64_t n, const double* y, int64_t m, int32_
   }
   free(ft);
   return bad ? ORC_ERR_ALLOC : ORC_OK;
+}
+
+/* max(|P1 - a|_inf, |P^T 1 - b|_inf) at (f, g), from the explicit row and column sums. */
+static int marginal_violation(const double* x, int64_t n, const double* y, int64_t m, int32_t d,
+                              const double* a, const double* b, double eps, const double* f,
+                              const double* g, double* out) {
+  double* r = (double*)malloc(sizeof(double) * (size_t)n);
+  double* c = (double*)malloc(sizeof(double) * (size_t)m);
+  if (!r || !c) {
+    free(r);
+    free(c);
+    return ORC_ERR_ALLOC;
+  }
+  int rc = oracle_plan_row_sums(x, n, y, m, d, a, b, eps, f, g, NULL, n, r);
+  if (!rc) rc = oracle_plan_row_sums(y, m, x, n, d, b, a, eps, g, f, NULL, m, c);
+  double v = 0.0;
+  if (!rc) {
+    for (int64_t i = 0; i < n; ++i) v = fmax(v, fabs(r[i] - a[i]));
+    for (int64_t j = 0; j < m; ++j) v = fmax(v, fabs(c[j] - b[j]));
+  }
+  free(r);
+  free(c);
+  *out = v;
+  return rc;
+}
+
+#define ORC_ALTERNATING 0
+#define ORC_SYMMETRIC 1
+#define ORC_STOP_FIXED 0
+#define ORC_STOP_MARGINAL 1
+#define ORC_STOP_POTENTIAL 2
+
+/*
+ * The general solve. Under stop_mode fixed it runs n_iters iterations and reports
+ * iters_run = n_iters, converged = -1, final_viol = NaN; otherwise at most stop_max_iter
+ * iterations with a check after every stop_check_every-th one and after the last one.
+ */
+int oracle_solve(const double* x, int64_t n, const double* y, int64_t m, int32_t d,
+                 const double* a, const double* b, double eps, int32_t variant, double alpha,
+                 int32_t stop_mode, int32_t n_iters, int32_t stop_max_iter, double stop_tol,
+                 int32_t stop_check_every, const double* g_init, double* f_out, double* g_out,
+                 int32_t* iters_run, int32_t* converged, double* final_viol) {
+  if (!x || !y || !a || !b || !f_out || !g_out || !iters_run || !converged || !final_viol ||
+      n < 1 || m < 1 || d < 1 || !(eps > 0.0) || isinf(eps))
+    return ORC_ERR_ARG;
+  if (variant != ORC_ALTERNATING && variant != ORC_SYMMETRIC) return ORC_ERR_ARG;
+  if (variant == ORC_SYMMETRIC && !(alpha > 0.0 && alpha <= 1.0)) return ORC_ERR_ARG;
+  if (stop_mode < ORC_STOP_FIXED || stop_mode > ORC_STOP_POTENTIAL) return ORC_ERR_ARG;
+  if (stop_mode == ORC_STOP_FIXED ? n_iters < 1
+                                  : (stop_max_iter < 1 || stop_check_every < 1 || !(stop_tol >= 0.0)))
+    return ORC_ERR_ARG;
+  int rc = check_mass(a, n, b, m);
+  if (rc) return rc;
+  const int32_t total = stop_mode == ORC_STOP_FIXED ? n_iters : stop_max_iter;
+  double* fn = (double*)malloc(sizeof(double) * (size_t)n);
+  double* gn = (double*)malloc(sizeof(double) * (size_t)m);
+  double* fp = (double*)malloc(sizeof(double) * (size_t)n);
+  double* gp = (double*)malloc(sizeof(double) * (size_t)m);
+  if (!fn || !gn || !fp || !gp) {
+    free(fn);
+    free(gn);
+    free(fp);
+    free(gp);
+    return ORC_ERR_ALLOC;
+  }
+  for (int64_t i = 0; i < n; ++i) f_out[i] = fp[i] = 0.0;
+  for (int64_t j = 0; j < m; ++j) g_out[j] = gp[j] = g_init ? g_init[j] : 0.0;
+  *iters_run = 0;
+  *converged = stop_mode == ORC_STOP_FIXED ? -1 : 0;
+  *final_viol = NAN;
+  for (int32_t it = 1; it <= total && !rc; ++it) {
+    if (variant == ORC_ALTERNATING) {
+      rc = oracle_lse_update(x, n, y, m, d, b, g_out, eps, NULL, n, f_out);
+      if (!rc) rc = oracle_lse_update(y, m, x, n, d, a, f_out, eps, NULL, m, g_out);
+    } else {
+      rc = oracle_lse_update(x, n, y, m, d, b, g_out, eps, NULL, n, fn);
+      if (!rc) rc = oracle_lse_update(y, m, x, n, d, a, f_out, eps, NULL, m, gn);
+      if (!rc) {
+        for (int64_t i = 0; i < n; ++i) f_out[i] = (1.0 - alpha) * f_out[i] + alpha * fn[i];
+        for (int64_t j = 0; j < m; ++j) g_out[j] = (1.0 - alpha) * g_out[j] + alpha * gn[j];
+      }
+    }
+    if (rc) break;
+    *iters_run = it;
+    if (stop_mode == ORC_STOP_FIXED || (it % stop_check_every != 0 && it != total)) continue;
+    double v = 0.0;
+    if (stop_mode == ORC_STOP_MARGINAL) {
+      rc = marginal_violation(x, n, y, m, d, a, b, eps, f_out, g_out, &v);
+      if (rc) break;
+    } else {
+      for (int64_t i = 0; i < n; ++i) {
+        v = fmax(v, fabs(f_out[i] - fp[i]));
+        fp[i] = f_out[i];
+      }
+      for (int64_t j = 0; j < m; ++j) {
+        v = fmax(v, fabs(g_out[j] - gp[j]));
+        gp[j] = g_out[j];
+      }
+    }
+    *final_viol = v;
+    if (stop_mode == ORC_STOP_MARGINAL ? v <= stop_tol : v < stop_tol) {
+      *converged = 1;
+      break;
+    }
+  }
+  free(fn);
+  free(gn);
+  free(fp);
+  free(gp);
+  return rc;
 }

@@ -44,6 +44,15 @@ MUTANTS = {
         "    rc = oracle_lse_update(x, n, y, m, d, b, g_out, eps, NULL, n, f_out);"),
     "grad_uses_f_pass_weights": ("double p = a[i] * b[j] * exp((ft[k] + g[j] - cij) / eps);",
                                  "double p = b[j] * exp((ft[k] + g[j] - cij) / eps);"),
+    "symmetric_blend_swapped": ("f_out[i] = (1.0 - alpha) * f_out[i] + alpha * fn[i];",
+                                "f_out[i] = alpha * f_out[i] + (1.0 - alpha) * fn[i];"),
+    "symmetric_g_from_new_f": (
+        "if (!rc) rc = oracle_lse_update(y, m, x, n, d, a, f_out, eps, NULL, m, gn);",
+        "if (!rc) rc = oracle_lse_update(y, m, x, n, d, a, fn, eps, NULL, m, gn);"),
+    "potential_reference_not_moved": ("fp[i] = f_out[i];", ";"),
+    "check_cadence_off_by_one": ("it % stop_check_every != 0", "(it + 1) % stop_check_every != 0"),
+    "no_check_at_the_cap": ("(it % stop_check_every != 0 && it != total)",
+                            "(it % stop_check_every != 0)"),
 }
 
 

@@ -282,3 +282,114 @@ def test_zero_mass_and_negative_weight_raise():
         oracle.potentials(x, y, a, b, 0.0, 1)
     with pytest.raises(oracle.OracleError):
         oracle.potentials(x, y, a, b, eps, 0)
+
+
+# --- the general solve: symmetric variant and stop modes ---------------------------------
+
+def jacobi_scaling(x, y, a, b, eps, n_iters, alpha, g0=None):
+    """The symmetric (Jacobi) blend in multiplicative form on the explicit Gibbs kernel:
+    with U = exp(f/eps), V = b exp(g/eps), both new values come from the old pair,
+    U' = U^(1-alpha) (K V)^(-alpha) and exp(g'/eps) = exp(g/eps)^(1-alpha) (K^T (a U))^(-alpha),
+    from f = 0. Returns the list of (f, g) after each iteration."""
+    C = dense_cost(x, y)
+    K = np.exp(-C / eps)
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    U = np.ones(len(a))
+    E = np.ones(len(b)) if g0 is None else np.exp(np.asarray(g0, np.float64) / eps)
+    out = []
+    for _ in range(n_iters):
+        KV = K @ (b * E)
+        KtU = K.T @ (a * U)
+        U, E = U ** (1.0 - alpha) * KV ** (-alpha), E ** (1.0 - alpha) * KtU ** (-alpha)
+        out.append((eps * np.log(U), eps * np.log(E)))
+    return out
+
+
+def dense_violation(x, y, a, b, eps, f, g):
+    P = dense_plan(x, y, a, b, eps, f, g)
+    return max(np.abs(P.sum(1) - a).max(), np.abs(P.sum(0) - b).max())
+
+
+@pytest.mark.parametrize("alpha", [0.3, 0.5, 1.0])
+@pytest.mark.parametrize("n,m,d,seed", [(7, 5, 2, 0), (40, 33, 3, 1)])
+def test_symmetric_matches_jacobi_scaling(alpha, n, m, d, seed):
+    x, y, a, b, _ = small(n, m, d, seed)
+    eps = float(dense_cost(x, y).max()) / 25.0
+    ref = jacobi_scaling(x, y, a, b, eps, 6, alpha)
+    for iters in (1, 2, 6):
+        f, g, it, conv, viol = oracle.solve(x, y, a, b, eps, n_iters=iters, variant="symmetric",
+                                            alpha=alpha)
+        assert it == iters and conv is None and np.isnan(viol)
+        np.testing.assert_allclose(f, ref[iters - 1][0], rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(g, ref[iters - 1][1], rtol=1e-11, atol=1e-12)
+
+
+def test_symmetric_and_alternating_share_the_fixed_point():
+    """Both schedules converge to the unique optimal plan (the potentials may differ by a
+    constant (f + c, g - c), which leaves the plan and the cost unchanged)."""
+    x, y, a, b, _ = small(30, 24, 2, 4)
+    eps = float(dense_cost(x, y).max()) / 15.0
+    fa, ga, *_ = oracle.solve(x, y, a, b, eps, n_iters=400)
+    fs_, gs_, *_ = oracle.solve(x, y, a, b, eps, n_iters=1500, variant="symmetric", alpha=0.5)
+    Pa = dense_plan(x, y, a, b, eps, fa, ga)
+    Ps = dense_plan(x, y, a, b, eps, fs_, gs_)
+    np.testing.assert_allclose(Ps, Pa, rtol=1e-7, atol=1e-12)
+    shift = fs_ - fa
+    assert np.ptp(shift) < 1e-7 and np.abs((gs_ - ga) + shift.mean()).max() < 1e-7
+
+
+@pytest.mark.parametrize("variant", ["alternating", "symmetric"])
+def test_marginal_stop_is_the_first_passing_check(variant):
+    x, y, a, b, _ = small(25, 31, 2, 7)
+    eps = float(dense_cost(x, y).max()) / 20.0
+    tol, every = 1e-7, 4
+    f, g, it, conv, viol = oracle.solve(x, y, a, b, eps, variant=variant, stop_mode="marginal",
+                                        stop_tol=tol, stop_check_every=every, stop_max_iter=5000)
+    assert conv is True and it % every == 0 and viol <= tol
+    assert viol == pytest.approx(dense_violation(x, y, a, b, eps, f, g), rel=1e-9, abs=1e-15)
+    # the check before it did not pass: rerun that many iterations with the fixed schedule
+    if variant == "alternating":
+        fp, gp = scaling_sinkhorn(x, y, a, b, eps, it - every)
+    else:
+        fp, gp = jacobi_scaling(x, y, a, b, eps, it - every, 0.5)[-1]
+    assert dense_violation(x, y, a, b, eps, fp, gp) > tol
+
+
+def test_potential_stop_measures_change_since_last_check():
+    x, y, a, b, _ = small(20, 18, 3, 8)
+    eps = float(dense_cost(x, y).max()) / 20.0
+    tol, every = 1e-9, 3
+    f, g, it, conv, viol = oracle.solve(x, y, a, b, eps, variant="symmetric", alpha=0.5,
+                                        stop_mode="potential", stop_tol=tol,
+                                        stop_check_every=every, stop_max_iter=5000)
+    traj = jacobi_scaling(x, y, a, b, eps, it, 0.5)
+    assert conv is True and it % every == 0 and viol < tol
+    f0, g0 = traj[it - every - 1]
+    expect = max(np.abs(traj[-1][0] - f0).max(), np.abs(traj[-1][1] - g0).max())
+    assert viol == pytest.approx(expect, rel=1e-6, abs=1e-14)
+    f1, g1 = traj[it - 2 * every - 1]
+    assert max(np.abs(f0 - f1).max(), np.abs(g0 - g1).max()) >= tol
+
+
+def test_stop_cap_reports_the_last_check():
+    """A tolerance no check can meet: converged is False, iters_run is the cap, and the
+    last check (after the capped iteration, 10 is not a multiple of 4) is reported."""
+    x, y, a, b, _ = small(12, 9, 2, 9)
+    eps = float(dense_cost(x, y).max()) / 10.0
+    f, g, it, conv, viol = oracle.solve(x, y, a, b, eps, stop_mode="marginal", stop_tol=0.0,
+                                        stop_check_every=4, stop_max_iter=10)
+    assert conv is False and it == 10
+    fs, gs = scaling_sinkhorn(x, y, a, b, eps, 10)
+    np.testing.assert_allclose(f, fs, rtol=1e-11, atol=1e-12)
+    assert viol == pytest.approx(dense_violation(x, y, a, b, eps, f, g), rel=1e-9, abs=1e-15)
+
+
+def test_solve_argument_errors():
+    x, y, a, b, eps = small(5, 6, 2, 10)
+    for kw in ({"n_iters": 0}, {"variant": "symmetric", "alpha": 0.0},
+               {"variant": "symmetric", "alpha": 1.5}, {"stop_mode": "marginal", "stop_max_iter": 0},
+               {"stop_mode": "potential", "stop_check_every": 0},
+               {"stop_mode": "marginal", "stop_tol": -1.0}):
+        with pytest.raises(oracle.OracleError):
+            oracle.solve(x, y, a, b, eps, **kw)
