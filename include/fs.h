@@ -77,7 +77,8 @@ typedef enum {
   FS_ERR_WORKSPACE = 10,       /* ws NULL, misaligned or smaller than required */
   FS_ERR_TIMEOUT = 11,         /* a kernel's bounded wait expired; outputs invalid */
   FS_ERR_CUDA = 12,            /* a CUDA runtime call failed (see fs_last_cuda_error) */
-  FS_ERR_ALIGNMENT = 13        /* a device pointer is not 4-byte aligned */
+  FS_ERR_ALIGNMENT = 13,       /* a device pointer is not 4-byte aligned */
+  FS_ERR_OPTION = 14           /* an fs_solve_options field is out of range */
 } fs_status;
 
 /* Human-readable name of a status code (static storage, never NULL). */
@@ -106,6 +107,55 @@ FS_API size_t fs_workspace_bytes(const fs_problem* p);
  */
 FS_API fs_status fs_potentials(const fs_problem* p, int32_t n_iters, const float* g_init, float* f,
                         float* g, void* ws, size_t ws_bytes, fs_stream_t stream);
+
+/*
+ * The general solve (SinkSLOT README, API Reference: variant, alpha, stop_mode,
+ * stop_max_iter, stop_tol, stop_check_every; the result's iters_run, converged and
+ * final_viol).
+ *   variant FS_VARIANT_ALTERNATING (Gauss-Seidel): the schedule of fs_potentials.
+ *   variant FS_VARIANT_SYMMETRIC (Jacobi): from f = 0 and g = g_init (or 0), both updates
+ *     come from the previous iterate and are blended:
+ *       f <- (1 - alpha) f + alpha F(g),   g <- (1 - alpha) g + alpha G(f).
+ *   stop_mode FS_STOP_FIXED: exactly n_iters iterations, no check.
+ *   stop_mode FS_STOP_MARGINAL: at most stop_max_iter iterations; after every
+ *     stop_check_every-th one (and after the last allowed one) the plan's marginal
+ *     violation max(|P1 - a|_inf, |P^T 1 - b|_inf) is computed (two extra passes) and
+ *     the solve stops once it is <= stop_tol.
+ *   stop_mode FS_STOP_POTENTIAL: the same cadence; stops once
+ *     max(|f - f_prev|_inf, |g - g_prev|_inf) < stop_tol, the previous values being those of
+ *     the last check (of the start for the first one). This is eps * max |delta phi| for
+ *     the absorbed potentials phi = f / eps.
+ * Each check reads one scalar back to the host (a stream synchronisation).
+ * report (host, may be NULL): iters_run; converged (1 or 0; -1 under FS_STOP_FIXED);
+ * final_viol (the last check's value; NaN under FS_STOP_FIXED).
+ * Errors as fs_potentials (FS_ERR_ITERS for n_iters < 1 under FS_STOP_FIXED), plus
+ * FS_ERR_NULL for a NULL opt and FS_ERR_OPTION for an option out of range: an unknown
+ * variant or stop mode, alpha outside (0, 1] for the symmetric variant, and under the
+ * checked modes stop_max_iter < 1, stop_check_every < 1 or stop_tol < 0 (or NaN).
+ */
+typedef enum { FS_VARIANT_ALTERNATING = 0, FS_VARIANT_SYMMETRIC = 1 } fs_variant;
+typedef enum { FS_STOP_FIXED = 0, FS_STOP_MARGINAL = 1, FS_STOP_POTENTIAL = 2 } fs_stop_mode;
+
+typedef struct {
+  int32_t n_iters;          /* iterations under FS_STOP_FIXED */
+  int32_t variant;          /* fs_variant */
+  float alpha;              /* blend weight of the symmetric variant */
+  int32_t stop_mode;        /* fs_stop_mode */
+  int32_t stop_max_iter;    /* iteration cap of the checked modes */
+  int32_t stop_check_every; /* iterations between checks */
+  double stop_tol;          /* threshold of the checks */
+  const float* g_init;      /* initial g (m floats, device; may alias g) or NULL */
+} fs_solve_options;
+
+typedef struct {
+  int32_t iters_run;
+  int32_t converged;
+  double final_viol;
+} fs_solve_report;
+
+FS_API fs_status fs_solve(const fs_problem* p, const fs_solve_options* opt, float* f, float* g,
+                          fs_solve_report* report, void* ws, size_t ws_bytes,
+                          fs_stream_t stream);
 
 /*
  * Dual objective at (f, g):

@@ -19,7 +19,7 @@ from . import _lib
 
 __all__ = ["potentials", "cost", "grad_x", "marginal_residual", "solve_host", "workspace_bytes",
            "FsError", "timing_enable", "timing_reset", "timing_get", "launch_count",
-           "screening_enable"]
+           "screening_enable", "solve"]
 
 
 class FsError(RuntimeError):
@@ -139,6 +139,43 @@ def potentials(x, y, a=None, b=None, *, eps: float, n_iters: int, g_init=None, o
                                      f.data_ptr(), g.data_ptr(), ws.data_ptr(), ws.numel(),
                                      P.stream()))
     return f, g
+
+
+def solve(x, y, a=None, b=None, *, eps: float, n_iters: int = 200, variant: str = "alternating",
+          alpha: float = 0.5, stop_mode: str = "fixed", stop_max_iter: int = 20000,
+          stop_tol: float = 1e-6, stop_check_every: int = 5, g_init=None, out=None,
+          workspace=None):
+    """The general solve (fs_solve): (f, g, report).
+
+    SinkSLOT README, API Reference: ``variant`` "alternating" (Gauss-Seidel) or "symmetric"
+    (Jacobi, blended with ``alpha``); ``stop_mode`` "fixed" (``n_iters`` iterations),
+    "marginal" or "potential" (at most ``stop_max_iter``, checked every
+    ``stop_check_every`` against ``stop_tol``). ``report`` holds iters_run, converged (None
+    under "fixed") and final_viol (NaN under "fixed").
+    """
+    torch = _torch()
+    P = _Problem(x, y, a, b, eps)
+    if out is None:
+        f = torch.empty(P.n, dtype=torch.float32, device=P.device)
+        g = torch.empty(P.m, dtype=torch.float32, device=P.device)
+    else:
+        f = _check_tensor(out[0], "f", (P.n,), P.device)
+        g = _check_tensor(out[1], "g", (P.m,), P.device)
+    gi = None if g_init is None else _check_tensor(g_init, "g_init", (P.m,), P.device)
+    if variant not in _lib.VARIANTS or stop_mode not in _lib.STOP_MODES:
+        raise ValueError(f"unknown variant {variant!r} or stop_mode {stop_mode!r}")
+    opt = _lib.fs_solve_options(int(n_iters), _lib.VARIANTS[variant], float(alpha),
+                                _lib.STOP_MODES[stop_mode], int(stop_max_iter),
+                                int(stop_check_every), float(stop_tol),
+                                None if gi is None else gi.data_ptr())
+    rep = _lib.fs_solve_report()
+    ws = P.workspace() if workspace is None else workspace
+    _raise(_lib.load().fs_solve(P.ref, ctypes.byref(opt), f.data_ptr(), g.data_ptr(),
+                                ctypes.byref(rep), ws.data_ptr(), ws.numel(), P.stream()))
+    report = {"iters_run": int(rep.iters_run),
+              "converged": None if rep.converged < 0 else bool(rep.converged),
+              "final_viol": float(rep.final_viol)}
+    return f, g, report
 
 
 def cost(x, y, f, g, a=None, b=None, *, eps: float, workspace=None):

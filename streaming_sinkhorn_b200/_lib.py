@@ -16,7 +16,7 @@ STATUS = {
     0: "FS_OK", 1: "FS_ERR_NULL", 2: "FS_ERR_SHAPE", 3: "FS_ERR_EPS", 4: "FS_ERR_ITERS",
     5: "FS_ERR_NEGATIVE_WEIGHT", 6: "FS_ERR_NONFINITE_INPUT", 7: "FS_ERR_MASS_MISMATCH",
     8: "FS_ERR_ZERO_MASS", 9: "FS_ERR_UNSUPPORTED_D", 10: "FS_ERR_WORKSPACE",
-    11: "FS_ERR_TIMEOUT", 12: "FS_ERR_CUDA", 13: "FS_ERR_ALIGNMENT",
+    11: "FS_ERR_TIMEOUT", 12: "FS_ERR_CUDA", 13: "FS_ERR_ALIGNMENT", 14: "FS_ERR_OPTION",
 }
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
@@ -25,14 +25,29 @@ EXPORTS = (
     "fs_status_string", "fs_last_cuda_error", "fs_workspace_bytes", "fs_potentials", "fs_cost",
     "fs_grad_x", "fs_marginal_residual", "fs_solve_host_workspace_bytes", "fs_solve_host",
     "fs_timing_enable", "fs_timing_reset", "fs_timing_get", "fs_launch_count",
-    "fs_potentials_noalloc", "fs_screening_enable",
+    "fs_potentials_noalloc", "fs_screening_enable", "fs_solve",
 )
+
+VARIANTS = {"alternating": 0, "symmetric": 1}
+STOP_MODES = {"fixed": 0, "marginal": 1, "potential": 2}
 
 
 class fs_problem(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("y", ctypes.c_void_p), ("a", ctypes.c_void_p),
                 ("b", ctypes.c_void_p), ("n", ctypes.c_int64), ("m", ctypes.c_int64),
                 ("d", ctypes.c_int32), ("eps", ctypes.c_float)]
+
+
+class fs_solve_options(ctypes.Structure):
+    _fields_ = [("n_iters", ctypes.c_int32), ("variant", ctypes.c_int32),
+                ("alpha", ctypes.c_float), ("stop_mode", ctypes.c_int32),
+                ("stop_max_iter", ctypes.c_int32), ("stop_check_every", ctypes.c_int32),
+                ("stop_tol", ctypes.c_double), ("g_init", ctypes.c_void_p)]
+
+
+class fs_solve_report(ctypes.Structure):
+    _fields_ = [("iters_run", ctypes.c_int32), ("converged", ctypes.c_int32),
+                ("final_viol", ctypes.c_double)]
 
 
 class fs_timing_entry(ctypes.Structure):
@@ -74,8 +89,10 @@ def load():
     lib.fs_solve_host_workspace_bytes.argtypes = [P]
     lib.fs_solve_host_workspace_bytes.restype = sz
     lib.fs_solve_host.argtypes = [P, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.fs_solve.argtypes = [P, ctypes.POINTER(fs_solve_options), vp, vp,
+                             ctypes.POINTER(fs_solve_report), vp, sz, vp]
     for fn in (lib.fs_potentials, lib.fs_cost, lib.fs_grad_x, lib.fs_marginal_residual,
-               lib.fs_solve_host):
+               lib.fs_solve_host, lib.fs_solve):
         fn.restype = ctypes.c_int
     lib.fs_timing_enable.argtypes = [ctypes.c_int]
     lib.fs_timing_enable.restype = None

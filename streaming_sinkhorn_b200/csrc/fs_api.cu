@@ -310,6 +310,7 @@ constexpr int kDmin = 147;    // ints: ordered smallest key-bias change of x, of
 constexpr int kEval = 148;    // uint64[3]: pairs evaluated by sorted passes, by TimedKind
 constexpr int kQueue = 151;   // ints: tiles per unit C and unit count U of the last queue plan
 constexpr int kKept = 152;    // int64: kept tiles K of the last queue plan
+constexpr int kPotChange = 153;  // unsigned: float bits of the largest potential change
 
 struct Layout {
   int D;       // padded dimension of the FMA path
@@ -328,6 +329,8 @@ struct Layout {
       off_lse_x, off_lse_y;
   // queue mode: kept-tile masks, kept counts, unit starts and unit -> row block
   size_t off_kmask, off_kcount, off_ustart, off_unit_rb, off_rmlb;
+  // general solve: deferred biases of x (symmetric schedule), potentials at the last check
+  size_t off_defer, off_fprev, off_gprev;
   int64_t part_floats;
 };
 
@@ -431,6 +434,12 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms) {
     L.off_rmlb = o;
     o = align_up(o + static_cast<size_t>(std::max(n, m)) * sizeof(float));
   }
+  L.off_defer = o;
+  o = align_up(o + static_cast<size_t>(std::max(n, L.tx)) * sizeof(float));
+  L.off_fprev = o;
+  o = align_up(o + static_cast<size_t>(n) * sizeof(float));
+  L.off_gprev = o;
+  o = align_up(o + static_cast<size_t>(m) * sizeof(float));
   L.total = o;
   return L;
 }
@@ -664,6 +673,15 @@ void launch_pack_d(const float* pts, int64_t count, int d, const float* w, float
 }
 
 template <int D>
+void launch_apply_bias_d(float* keys, const float* defer_h, int64_t count, int* dmin,
+                         cudaStream_t st) {
+  apply_bias_kernel<D><<<static_cast<unsigned>(ceil_div(count, 256)), 256, 0, st>>>(keys, defer_h,
+                                                                                    count, dmin);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
+template <int D>
 void launch_bias_d(float* keys, int64_t count, const float* pot, const int* perm, const float* lw,
                    double kappa, cudaStream_t st) {
   const unsigned blocks = static_cast<unsigned>(ceil_div(count, 256));
@@ -752,6 +770,9 @@ struct Ctx {
   unsigned* kmask;
   int *kcount, *ustart, *unit_rb;
   float* rmlb;     // per-row lower bounds written by the screening kernel
+  float *defer, *fprev, *gprev;
+  float alpha;    // symmetric schedule: blend weight of the potential passes (0: plain)
+  bool defer_x;   // the next x-row potential pass leaves its biases in `defer`
   bool no_screen;  // screening found to keep most tiles: the rest of the call runs unscreened
 };
 
@@ -779,6 +800,9 @@ void carve(Ctx& c, void* ws) {
   c.lwx = reinterpret_cast<float*>(c.ws + c.L.off_lwx);
   c.lwy = reinterpret_cast<float*>(c.ws + c.L.off_lwy);
   c.part = reinterpret_cast<float*>(c.ws + c.L.off_part);
+  c.defer = reinterpret_cast<float*>(c.ws + c.L.off_defer);
+  c.fprev = reinterpret_cast<float*>(c.ws + c.L.off_fprev);
+  c.gprev = reinterpret_cast<float*>(c.ws + c.L.off_gprev);
   if (c.L.Dtc) {
     c.rimg_x = c.ws + c.L.off_rimg_x;
     c.kimg_x = c.ws + c.L.off_kimg_x;
@@ -1006,6 +1030,10 @@ void run_pass_tc(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_
   P.err = err_ptr(c.scal);
   P.hy_out = rows_x ? c.hy_x : c.hy_y;
   P.nrm = rows_x ? c.nrm_x : c.nrm_y;
+  if (kind == kPot) {
+    P.alpha = c.alpha;
+    if (rows_x && c.defer_x) P.defer_h = c.defer;  // installed after the other pass
+  }
   TcParams T{};
   T.row_img = rows_x ? c.rimg_x : c.rimg_y;
   T.key_img = rows_x ? c.kimg_y : c.kimg_x;
@@ -1075,8 +1103,15 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
     if (kind == kPot) {
       // this pass writes the query cloud's biases: record their change and its LSE2
       P.lse_out = rows_x ? c.lse_x : c.lse_y;
-      P.dmin_out = dmin_slots + (rows_x ? 0 : 1);
-      CK(cudaMemsetAsync(P.dmin_out, 0x7F, sizeof(int), c.st));
+      P.alpha = c.alpha;
+      if (rows_x && c.defer_x) {
+        // installed, and its change recorded, after the other pass of the iteration: the
+        // change recorded for x so far must survive until that pass has screened with it
+        P.defer_h = c.defer;
+      } else {
+        P.dmin_out = dmin_slots + (rows_x ? 0 : 1);
+        CK(cudaMemsetAsync(P.dmin_out, 0x7F, sizeof(int), c.st));
+      }
     }
   }
   const double pairs = static_cast<double>(n_rows) * static_cast<double>(rows_x ? p->m : p->n);
@@ -1131,7 +1166,7 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
       c.timer->end(ti, kTCombine, 0.0);
     }
   }
-  if (c.L.sorted && kind == kPot) {
+  if (c.L.sorted && kind == kPot && !(rows_x && c.defer_x)) {
     // largest bias per tile of the cloud just updated: the next pass screens against it
     FS_DISPATCH_D(c.L.D, launch_tile_hmax_d, rows_x ? c.kx : c.ky, n_rows,
                   (rows_x ? c.L.px : c.L.py) / kPairPad, rows_x ? c.hmax_x : c.hmax_y, c.st);
@@ -1191,35 +1226,137 @@ fs_status begin(Ctx& c, const fs_problem* p, void* ws, size_t ws_bytes, fs_strea
   return FS_OK;
 }
 
+// Symmetric schedule: install x's deferred biases once the y pass of the iteration has
+// read the previous ones.
+void apply_deferred_x(Ctx& c) {
+  const int64_t n = c.p->n;
+  if (c.use_tc) {
+    CK(cudaMemcpyAsync(c.hy_x, c.defer, static_cast<size_t>(n) * sizeof(float),
+                       cudaMemcpyDeviceToDevice, c.st));
+    return;
+  }
+  int* dmin = reinterpret_cast<int*>(c.scal + kDmin);  // slot 0: x
+  CK(cudaMemsetAsync(dmin, 0x7F, sizeof(int), c.st));
+  FS_DISPATCH_D(c.L.D, launch_apply_bias_d, c.kx, c.defer, n, dmin, c.st);
+  FS_DISPATCH_D(c.L.D, launch_tile_hmax_d, c.kx, n, c.L.px / kPairPad, c.hmax_x, c.st);
+}
+
+// max(|P1 - a|_inf, |P^T 1 - b|_inf) at (f, g): two marginal passes, one read-back.
+double check_marginal(Ctx& c, const float* f, const float* g) {
+  CK(cudaMemsetAsync(c.scal + kAccRow, 0, 6 * sizeof(double), c.st));
+  run_pass(c, true, kMarg, f, nullptr, nullptr, nullptr, c.scal + kAccRow);
+  run_pass(c, false, kMarg, g, nullptr, nullptr, nullptr, c.scal + kAccCol);
+  double acc[6];
+  CK(cudaMemcpyAsync(acc, c.scal + kAccRow, sizeof(acc), cudaMemcpyDeviceToHost, c.st));
+  CK(cudaStreamSynchronize(c.st));
+  return std::max(acc[1], acc[4]);
+}
+
+// max(|f - f_prev|_inf, |g - g_prev|_inf), then prev <- current; one read-back.
+double check_potential(Ctx& c, const float* f, const float* g) {
+  unsigned* mb = reinterpret_cast<unsigned*>(c.scal + kPotChange);
+  CK(cudaMemsetAsync(mb, 0, sizeof(unsigned), c.st));
+  pot_change_kernel<<<reduce_blocks(c.p->n, c.sms), 256, 0, c.st>>>(f, c.fprev, c.p->n, mb);
+  CK(cudaGetLastError());
+  pot_change_kernel<<<reduce_blocks(c.p->m, c.sms), 256, 0, c.st>>>(g, c.gprev, c.p->m, mb);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(2, std::memory_order_relaxed);
+  unsigned bits = 0;
+  CK(cudaMemcpyAsync(&bits, mb, sizeof(bits), cudaMemcpyDeviceToHost, c.st));
+  CK(cudaStreamSynchronize(c.st));
+  float v;
+  memcpy(&v, &bits, sizeof(v));
+  return static_cast<double>(v);
+}
+
+fs_status check_options(const fs_solve_options& o) {
+  if (o.variant != FS_VARIANT_ALTERNATING && o.variant != FS_VARIANT_SYMMETRIC) return FS_ERR_OPTION;
+  if (o.variant == FS_VARIANT_SYMMETRIC && !(o.alpha > 0.0f && o.alpha <= 1.0f)) return FS_ERR_OPTION;
+  if (o.stop_mode == FS_STOP_FIXED) return o.n_iters < 1 ? FS_ERR_ITERS : FS_OK;
+  if (o.stop_mode != FS_STOP_MARGINAL && o.stop_mode != FS_STOP_POTENTIAL) return FS_ERR_OPTION;
+  if (o.stop_max_iter < 1 || o.stop_check_every < 1 || !(o.stop_tol >= 0.0)) return FS_ERR_OPTION;
+  return FS_OK;
+}
+
 }  // namespace
+
+fs_status solve_impl(const fs_problem* p, const fs_solve_options* opt, float* f, float* g,
+                     fs_solve_report* report, void* ws, size_t ws_bytes, fs_stream_t stream) {
+  Ctx c{};
+  fs_status s = begin(c, p, ws, ws_bytes, stream);
+  if (s != FS_OK) return s;
+  if (!opt || !f || !g) return FS_ERR_NULL;
+  const fs_solve_options o = *opt;
+  if (!aligned4(f) || !aligned4(g) || !aligned4(o.g_init)) return FS_ERR_ALIGNMENT;
+  s = check_options(o);
+  if (s != FS_OK) return s;
+  Timer timer(c.st);
+  c.timer = &timer;
+  return guarded(c.st, [&]() -> fs_status {
+    std::vector<std::pair<const float*, int64_t>> pots;
+    if (o.g_init) pots.push_back({o.g_init, p->m});
+    fs_status r = prepare_all(c, pots, true);
+    if (r != FS_OK) return r;
+    const bool sym = o.variant == FS_VARIANT_SYMMETRIC;
+    const bool fixed = o.stop_mode == FS_STOP_FIXED;
+    const size_t fb = static_cast<size_t>(p->n) * sizeof(float);
+    const size_t gb = static_cast<size_t>(p->m) * sizeof(float);
+    if (sym || o.stop_mode == FS_STOP_POTENTIAL) {
+      // the blend and the first potential check read the starting point f = 0, g = g_init
+      if (o.g_init && o.g_init != g)
+        CK(cudaMemcpyAsync(g, o.g_init, gb, cudaMemcpyDeviceToDevice, c.st));
+      else if (!o.g_init)
+        CK(cudaMemsetAsync(g, 0, gb, c.st));
+      CK(cudaMemsetAsync(f, 0, fb, c.st));
+    }
+    if (o.stop_mode == FS_STOP_POTENTIAL) {
+      CK(cudaMemsetAsync(c.fprev, 0, fb, c.st));
+      CK(cudaMemcpyAsync(c.gprev, g, gb, cudaMemcpyDeviceToDevice, c.st));
+    }
+    if (sym) set_bias(c, true, nullptr);  // x carries f = 0
+    set_bias(c, false, o.g_init);
+    c.alpha = sym ? o.alpha : 0.0f;
+    const int32_t total = fixed ? o.n_iters : o.stop_max_iter;
+    int32_t iters = 0, conv = fixed ? -1 : 0;
+    double viol = NAN;
+    // From the second iteration on every row has a previous LSE2 and the keys a recorded
+    // bias change, so the passes can screen key tiles by history as well.
+    for (int32_t it = 1; it <= total; ++it) {
+      c.defer_x = sym;
+      run_pass(c, true, kPot, nullptr, f, nullptr, nullptr, nullptr, it > 1);   // f <- F(g)
+      c.defer_x = false;
+      run_pass(c, false, kPot, nullptr, g, nullptr, nullptr, nullptr, it > 1);  // g <- G(f)
+      if (sym) apply_deferred_x(c);
+      iters = it;
+      if (it == 1 && total > 2) screening_probe(c, false);
+      if (fixed || (it % o.stop_check_every != 0 && it != total)) continue;
+      viol = o.stop_mode == FS_STOP_MARGINAL ? check_marginal(c, f, g) : check_potential(c, f, g);
+      if (o.stop_mode == FS_STOP_MARGINAL ? viol <= o.stop_tol : viol < o.stop_tol) {
+        conv = 1;
+        break;
+      }
+    }
+    c.alpha = 0.0f;
+    r = finish(c);
+    if (report) {
+      report->iters_run = iters;
+      report->converged = conv;
+      report->final_viol = viol;
+    }
+    return r;
+  });
+}
 
 // ---------------- entry points ----------------
 
 fs_status potentials_impl(const fs_problem* p, int32_t n_iters, const float* g_init, float* f,
                           float* g, void* ws, size_t ws_bytes, fs_stream_t stream) {
-  Ctx c{};
-  fs_status s = begin(c, p, ws, ws_bytes, stream);
-  if (s != FS_OK) return s;
-  if (!f || !g) return FS_ERR_NULL;
-  if (!aligned4(f) || !aligned4(g) || !aligned4(g_init)) return FS_ERR_ALIGNMENT;
-  if (n_iters < 1) return FS_ERR_ITERS;
-  Timer timer(c.st);
-  c.timer = &timer;
-  return guarded(c.st, [&]() -> fs_status {
-    std::vector<std::pair<const float*, int64_t>> pots;
-    if (g_init) pots.push_back({g_init, p->m});
-    fs_status r = prepare_all(c, pots, true);
-    if (r != FS_OK) return r;
-    set_bias(c, false, g_init);
-    // From the second iteration on every row has a previous LSE2 and the keys a recorded
-    // bias change, so the passes can screen key tiles.
-    for (int32_t it = 0; it < n_iters; ++it) {
-      run_pass(c, true, kPot, nullptr, f, nullptr, nullptr, nullptr, it > 0);   // f <- F(g)
-      run_pass(c, false, kPot, nullptr, g, nullptr, nullptr, nullptr, it > 0);  // g <- G(f)
-      if (it == 0 && n_iters > 2) screening_probe(c, false);
-    }
-    return finish(c);
-  });
+  fs_solve_options o{};
+  o.n_iters = n_iters;
+  o.variant = FS_VARIANT_ALTERNATING;
+  o.stop_mode = FS_STOP_FIXED;
+  o.g_init = g_init;
+  return solve_impl(p, &o, f, g, nullptr, ws, ws_bytes, stream);
 }
 
 }  // namespace fs
@@ -1241,6 +1378,7 @@ const char* fs_status_string(fs_status s) {
     case FS_ERR_WORKSPACE: return "FS_ERR_WORKSPACE: workspace missing, misaligned or too small";
     case FS_ERR_TIMEOUT: return "FS_ERR_TIMEOUT: a kernel's bounded wait expired";
     case FS_ERR_CUDA: return "FS_ERR_CUDA: a CUDA runtime call failed";
+    case FS_ERR_OPTION: return "FS_ERR_OPTION: a solve option is out of range";
     case FS_ERR_ALIGNMENT: return "FS_ERR_ALIGNMENT: device pointers must be 4-byte aligned";
   }
   return "unknown fs_status";
@@ -1256,6 +1394,11 @@ size_t fs_workspace_bytes(const fs_problem* p) {
 fs_status fs_potentials(const fs_problem* p, int32_t n_iters, const float* g_init, float* f,
                         float* g, void* ws, size_t ws_bytes, fs_stream_t stream) {
   return fs::potentials_impl(p, n_iters, g_init, f, g, ws, ws_bytes, stream);
+}
+
+fs_status fs_solve(const fs_problem* p, const fs_solve_options* opt, float* f, float* g,
+                   fs_solve_report* report, void* ws, size_t ws_bytes, fs_stream_t stream) {
+  return fs::solve_impl(p, opt, f, g, report, ws, ws_bytes, stream);
 }
 
 fs_status fs_grad_x(const fs_problem* p, const float* g, float* grad_x, void* ws, size_t ws_bytes,

@@ -106,6 +106,10 @@ struct PassParams {
   const int* unit_rb;       // [unit] row block of each unit
   const int* qscal;         // [0] tiles per unit C, [1] number of units U
   float* row_mlb;           // [row]: lower bound on each row's largest exponent (screening)
+  // symmetric (Jacobi) schedule: blend weight (0: plain update) and, for the pass whose
+  // biases the other pass of the same iteration must not see yet, where to leave them
+  float alpha;
+  float* defer_h;           // kPot: new bias of every query row (sorted order), or NULL
 };
 
 constexpr int kScreenTile = 256;  // points per screening tile (= kPairPad pairs)
@@ -124,18 +128,36 @@ __device__ __forceinline__ int64_t key_slot(int64_t i, int k) {
 // kPot: the new potential and the bias this row carries as a key into the next pass:
 //   pot_i = -LSE2_i / kappa,   H_i = kappa pot_i + log2 w_i = log2 w_i - LSE2_i.
 // Returns the change of the row's key bias (new - previous), for the screening bound.
+// Symmetric schedule: pot_i = (1 - alpha) pot_prev_i + alpha F_i (pot_prev read from
+// pot_out before it is overwritten) and H_i = kappa pot_i + log2 w_i; the bias goes to
+// defer_h when the other pass of the iteration still needs the previous one (the change
+// is then recorded when it is applied).
 template <int D>
 __device__ __forceinline__ float finish_pot(const PassParams& P, int64_t i, double lse2) {
   const int64_t oi = P.perm ? P.perm[i] : i;
-  P.pot_out[oi] = static_cast<float>(-lse2 * P.eps_ln2);
+  double pot = -lse2 * P.eps_ln2;
+  double h = static_cast<double>(P.lw[i]) - lse2;
+  if (P.alpha > 0.0f) {
+    const double a = static_cast<double>(P.alpha);
+    pot = (1.0 - a) * static_cast<double>(P.pot_out[oi]) + a * pot;
+    h = P.kappa * pot + static_cast<double>(P.lw[i]);
+  }
+  P.pot_out[oi] = static_cast<float>(pot);
   if (P.lse_out) P.lse_out[i] = static_cast<float>(lse2);
-  const double h = static_cast<double>(P.lw[i]) - lse2;
   if (P.hy_out) {
-    P.hy_out[i] = static_cast<float>(h - P.kappa * static_cast<double>(P.nrm[i]));
+    const float hy = static_cast<float>(h - P.kappa * static_cast<double>(P.nrm[i]));
+    if (P.defer_h)
+      P.defer_h[i] = hy;
+    else
+      P.hy_out[i] = hy;
+    return 0.0f;
+  }
+  const float hn = static_cast<float>(h);
+  if (P.defer_h) {
+    P.defer_h[i] = hn;
     return 0.0f;
   }
   const int64_t slot = key_slot<D>(i, D);
-  const float hn = static_cast<float>(h);
   const float delta = hn - P.qkeys[slot];
   P.qkeys[slot] = hn;
   return delta;
@@ -749,6 +771,38 @@ __global__ void __launch_bounds__(256) dot_kernel(const float* v, const float* w
 __global__ void cost_finish_kernel(const double* fa, const double* gb, const double* mass,
                                    double eps, double mamb, double* out) {
   if (threadIdx.x == 0 && blockIdx.x == 0) out[0] = fa[0] + gb[0] - eps * (mass[0] - mamb);
+}
+
+// Symmetric schedule: install the deferred biases of a cloud into its packed keys and
+// record the smallest change (for the screening history bound of the next pass).
+template <int D>
+__global__ void __launch_bounds__(256) apply_bias_kernel(float* keys, const float* defer_h,
+                                                         int64_t count, int* dmin_out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  float delta = INFINITY;
+  if (i < count) {
+    const int64_t slot = key_slot<D>(i, D);
+    const float hn = defer_h[i];
+    delta = hn - keys[slot];
+    keys[slot] = hn;
+  }
+  reduce_dmin(delta, dmin_out);
+}
+
+// Potential stop check: the largest |v - prev| over a vector, then prev <- v. The maximum
+// is kept as the bits of a non-negative float (ordered like unsigned ints).
+__global__ void __launch_bounds__(256) pot_change_kernel(const float* v, float* prev, int64_t count,
+                                                         unsigned* max_bits) {
+  float mx = 0.0f;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float x = v[i];
+    mx = fmaxf(mx, fabsf(x - prev[i]));
+    prev[i] = x;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(max_bits, __float_as_uint(mx));
 }
 
 __global__ void residual_finish_kernel(const double* row_acc, const double* col_acc, double* out) {

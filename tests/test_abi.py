@@ -149,3 +149,34 @@ def test_timing_api_roundtrip():
     assert set(t) == {"lse_pass", "grad_pass", "marg_pass", "combine", "screen"}
     assert all(v["launches"] == 0 for v in t.values())
     fs.timing_enable(False)
+
+
+def test_solve_option_errors():
+    lib = _lib.load()
+    p = ctypes.byref(prob())
+    need = lib.fs_workspace_bytes(p)
+    st = lambda c: _lib.STATUS[c]  # noqa: E731
+
+    def opts(**kw):
+        o = dict(n_iters=5, variant=0, alpha=0.5, stop_mode=0, stop_max_iter=100,
+                 stop_check_every=5, stop_tol=1e-6, g_init=None)
+        o.update(kw)
+        return _lib.fs_solve_options(o["n_iters"], o["variant"], o["alpha"], o["stop_mode"],
+                                     o["stop_max_iter"], o["stop_check_every"], o["stop_tol"],
+                                     o["g_init"])
+
+    rep = _lib.fs_solve_report()
+    call = lambda o: st(lib.fs_solve(p, ctypes.byref(o), FAKE, FAKE, ctypes.byref(rep), FAKE,  # noqa: E731
+                                     need, None))
+    assert st(lib.fs_solve(p, None, FAKE, FAKE, None, FAKE, need, None)) == "FS_ERR_NULL"
+    assert call(opts(n_iters=0)) == "FS_ERR_ITERS"
+    assert call(opts(variant=2)) == "FS_ERR_OPTION"
+    assert call(opts(variant=1, alpha=0.0)) == "FS_ERR_OPTION"
+    assert call(opts(variant=1, alpha=1.5)) == "FS_ERR_OPTION"
+    assert call(opts(stop_mode=3)) == "FS_ERR_OPTION"
+    assert call(opts(stop_mode=1, stop_max_iter=0)) == "FS_ERR_OPTION"
+    assert call(opts(stop_mode=2, stop_check_every=0)) == "FS_ERR_OPTION"
+    assert call(opts(stop_mode=1, stop_tol=-1.0)) == "FS_ERR_OPTION"
+    assert call(opts(stop_mode=1, stop_tol=float("nan"))) == "FS_ERR_OPTION"
+    assert st(lib.fs_solve(p, ctypes.byref(opts()), FAKE + 2, FAKE, None, FAKE, need,
+                           None)) == "FS_ERR_ALIGNMENT"
