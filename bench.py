@@ -52,8 +52,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-dense", action="store_true",
-                    help="skip the unscreened pass measured after the timed region")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the measurements after the timed region (the unscreened pass "
+                         "and the solve variants)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU seconds of the oracle sample")
     return ap.parse_args()
@@ -306,7 +307,7 @@ def run_native(args, rank, world, local_rank):
     # The same pass with screening off, outside the timed region: one solve iteration (an
     # f pass and a g pass over all N x M pairs) on the same inputs, so the kernel's roofline
     # is also shown on dense work.
-    if not args.no_dense:
+    if not args.no_extras:
         fs.screening_enable(False)
         fd, gd = torch.empty_like(f), torch.empty_like(g)
         fs.potentials(x, y, a, b, eps=w.eps, n_iters=1, out=(fd, gd), workspace=ws)
@@ -325,6 +326,32 @@ def run_native(args, rank, world, local_rank):
             "ms_per_launch": d_ms, "executed_ex2_per_launch": d_exec,
             "achieved": d_exec / (d_ms / 1e3) / 1e12, "frac": d_exec / (d_ms / 1e3) / peak}
 
+    # The general solve on the same inputs, outside the timed region: the symmetric
+    # (Jacobi) schedule for the same iteration count, and the alternating schedule stopped
+    # by the marginal check.
+    solve_extras = None
+    if not args.no_extras:
+        solve_extras = {}
+        for name, kw in (("symmetric_fixed", dict(n_iters=w.n_iters, variant="symmetric",
+                                                  alpha=0.5)),
+                         ("alternating_marginal_stop",
+                          dict(stop_mode="marginal", stop_tol=0.25 * float(w.a.max()),
+                               stop_check_every=5, stop_max_iter=100))):
+            fs.solve(x, y, a, b, eps=w.eps, out=(f, g), workspace=ws, **kw)
+            torch.cuda.synchronize(dev)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            _, _, rep = fs.solve(x, y, a, b, eps=w.eps, out=(f, g), workspace=ws, **kw)
+            e1.record(stream)
+            e1.synchronize()
+            ms = e0.elapsed_time(e1)
+            solve_extras[name] = {
+                "options": {k: v for k, v in kw.items()}, "ms": ms,
+                "iters_run": rep["iters_run"], "converged": rep["converged"],
+                "final_viol": None if rep["final_viol"] != rep["final_viol"] else rep["final_viol"],
+                "pair_evals_per_s": float(w.n) * w.m * rep["iters_run"] / (ms / 1e3)}
+
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -340,6 +367,7 @@ def run_native(args, rank, world, local_rank):
         "roofline": roofline,
         "clocks": clk,
         "kernel_timing": timing,
+        "solve_variants": solve_extras,
         "check": {"residual": [float(v) for v in res.cpu().numpy()], "cost": float(c.item())},
     }
 
