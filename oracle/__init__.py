@@ -18,6 +18,11 @@ Each function names the passage of the pages it follows:
   section 3 and SinkSLOT README "Basic Usage".
 * ``plan_row_sums`` / ``plan_col_sums`` / ``marginal_residual`` -- plan marginals and their
   deviation from (a, b), SinkSLOT README stop_mode "marginal".
+* ``solve`` -- the general solve: symmetric (Jacobi) schedule and the marginal / potential
+  stop modes, SinkSLOT README API Reference.
+* ``transport_apply`` / ``transport_apply_t`` / ``hvp`` (numpy, ``transport.py``) -- the
+  transport-vector and transport-matrix products and the Hessian-vector product of the
+  loss, FlashSinkhorn summary section 3.
 
 Pins: every function here is checked against closed forms, brute force and
 invariants in ``tests/test_oracle_pins.py``; none is left unpinned.
@@ -29,6 +34,8 @@ import os
 import subprocess
 
 import numpy as np
+
+from .transport import hvp, plan, transport_apply, transport_apply_t  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")

@@ -87,10 +87,49 @@ def test_pins_catch_mutant(mutant, tmp_path, monkeypatch):
     real = oracle._load()
     lib = ctypes.CDLL(str(lib_path))
     for fname in ("oracle_lse_update", "oracle_potentials", "oracle_plan_row_sums", "oracle_cost",
-                  "oracle_grad_x", "oracle_set_threads", "oracle_threads"):
+                  "oracle_grad_x", "oracle_solve", "oracle_set_threads", "oracle_threads"):
         getattr(lib, fname).argtypes = getattr(real, fname).argtypes
         getattr(lib, fname).restype = getattr(real, fname).restype
     monkeypatch.setattr(oracle, "_lib", lib)
+    caught = []
+    with np.errstate(all="ignore"):
+        for name, fn, kwargs in _pin_calls():
+            try:
+                fn(**kwargs)
+            except Exception:  # noqa: BLE001 - any failure of a pin counts as a catch
+                caught.append(name)
+    assert caught, f"no pin caught mutant {mutant}"
+
+
+# Mutants of the numpy transport products and Hessian-vector product (oracle/transport.py),
+# loaded from an edited copy and swapped into the oracle package for the pin run.
+PY_SRC = os.path.join(os.path.dirname(oracle.__file__), "transport.py")
+PY_MUTANTS = {
+    "hvp_dropped_direct_term": ("return 2.0 * a[:, None] * v + (2.0 / eps)",
+                                "return (2.0 / eps)"),
+    "hvp_flipped_cost_change": ("w = P * (df[:, None] + dg[None, :] - dC)",
+                                "w = P * (df[:, None] + dg[None, :] + dC)"),
+    "hvp_column_rhs_from_rows": ("s = (P * dC).sum(axis=0)", "s = (P * dC).sum(axis=0) * 0.0"),
+    "hvp_plan_of_given_g_only": ("ft = f_update(x, y, b, eps, g)", "ft = np.zeros(len(x))"),
+    "plan_missing_row_weight": (
+        "return _d(a)[:, None] * _d(b)[None, :] * np.exp(",
+        "return _d(b)[None, :] * np.exp("),
+}
+
+
+@pytest.mark.parametrize("mutant", sorted(PY_MUTANTS))
+def test_pins_catch_python_mutant(mutant, tmp_path, monkeypatch):
+    import importlib.util
+    before, after = PY_MUTANTS[mutant]
+    src = open(PY_SRC).read()
+    assert src.count(before) == 1, f"mutation site for {mutant} not unique"
+    mpath = tmp_path / "transport_mutant.py"
+    mpath.write_text(src.replace(before, after))
+    spec = importlib.util.spec_from_file_location("transport_mutant", mpath)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    for fname in ("hvp", "plan", "transport_apply", "transport_apply_t"):
+        monkeypatch.setattr(oracle, fname, getattr(mod, fname))
     caught = []
     with np.errstate(all="ignore"):
         for name, fn, kwargs in _pin_calls():

@@ -393,3 +393,75 @@ def test_solve_argument_errors():
                {"stop_mode": "marginal", "stop_tol": -1.0}):
         with pytest.raises(oracle.OracleError):
             oracle.solve(x, y, a, b, eps, **kw)
+
+
+# --- transport products and the Hessian-vector product -----------------------------------
+
+def converged(x, y, a, b, eps):
+    f, g, it, conv, viol = oracle.solve(x, y, a, b, eps, stop_mode="marginal", stop_tol=1e-13,
+                                        stop_check_every=10, stop_max_iter=200000)
+    assert conv
+    return f, g
+
+
+def test_transport_products_against_plan_sums_and_gradient():
+    x, y, a, b, _ = small(23, 17, 3, 11)
+    eps = float(dense_cost(x, y).max()) / 8.0
+    f, g = oracle.potentials(x, y, a, b, eps, 5)
+    # P 1 and P^T 1 against the C oracle's plan sums (an independent code path)
+    np.testing.assert_allclose(oracle.transport_apply(x, y, a, b, eps, f, g, np.ones(17)),
+                               oracle.plan_row_sums(x, y, a, b, eps, f, g), rtol=1e-12)
+    np.testing.assert_allclose(oracle.transport_apply_t(x, y, a, b, eps, f, g, np.ones(23)),
+                               oracle.plan_col_sums(x, y, a, b, eps, f, g), rtol=1e-12)
+    # P Y at the plan of (F(g), g) gives the gradient 2 (a x - P Y)
+    ft = oracle.lse_update(x, y, b, g, eps)
+    PY = oracle.transport_apply(x, y, a, b, eps, ft, g, y)
+    np.testing.assert_allclose(2.0 * (a[:, None] * x - PY), oracle.grad_x(x, y, a, b, eps, g),
+                               rtol=1e-10, atol=1e-13)
+
+
+@pytest.mark.parametrize("n,m,d,seed,div", [(12, 10, 2, 12, 4.0), (9, 14, 3, 13, 2.0)])
+def test_hvp_matches_gradient_finite_differences(n, m, d, seed, div):
+    """The derivative of the converged gradient along v, by central differences of two
+    fully converged solves at x +- h v."""
+    x, y, a, b, _ = small(n, m, d, seed)
+    eps = float(dense_cost(x, y).max()) / div
+    v = np.random.default_rng(seed).standard_normal(x.shape)
+    h = 1e-4
+
+    def grad_at(xx):
+        _, g = converged(xx, y, a, b, eps)
+        return oracle.grad_x(xx, y, a, b, eps, g)
+
+    fd = (grad_at(x + h * v) - grad_at(x - h * v)) / (2.0 * h)
+    _, g = converged(x, y, a, b, eps)
+    hv = oracle.hvp(x, y, a, b, eps, g, v)
+    np.testing.assert_allclose(hv, fd, rtol=1e-5, atol=1e-6 * np.abs(fd).max())
+
+
+def test_hvp_is_symmetric_and_gauge_invariant():
+    x, y, a, b, _ = small(15, 11, 2, 14)
+    eps = float(dense_cost(x, y).max()) / 5.0
+    _, g = converged(x, y, a, b, eps)
+    rng = np.random.default_rng(3)
+    u, v = rng.standard_normal(x.shape), rng.standard_normal(x.shape)
+    Hu = oracle.hvp(x, y, a, b, eps, g, u)
+    Hv = oracle.hvp(x, y, a, b, eps, g, v)
+    assert (u * Hv).sum() == pytest.approx((v * Hu).sum(), rel=1e-9, abs=1e-14)
+    # F(g + c) = F(g) - c: the plan, hence H v, does not move
+    np.testing.assert_allclose(oracle.hvp(x, y, a, b, eps, g + 0.37, v), Hv, rtol=1e-9,
+                               atol=1e-12 * np.abs(Hv).max())
+
+
+def test_hvp_large_eps_limit():
+    """As eps grows the plan tends to a (x) b, which does not depend on x, and
+    H v -> 2 a v, with an O(1/eps) remainder."""
+    x, y, a, b, _ = small(10, 12, 2, 15)
+    v = np.random.default_rng(4).standard_normal(x.shape)
+    errs = []
+    for eps in (1e2, 1e3, 1e4):
+        _, g = converged(x, y, a, b, eps)
+        errs.append(np.abs(oracle.hvp(x, y, a, b, eps, g, v) - 2.0 * a[:, None] * v).max())
+    assert errs[2] < errs[1] < errs[0]
+    assert errs[2] < 1e-3 * np.abs(2.0 * a[:, None] * v).max()
+    assert errs[1] / errs[2] == pytest.approx(10.0, rel=0.2)
