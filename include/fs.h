@@ -158,6 +158,55 @@ FS_API fs_status fs_solve(const fs_problem* p, const fs_solve_options* opt, floa
                           fs_stream_t stream);
 
 /*
+ * Transport products and the Hessian-vector product (FlashSinkhorn summary, section 3:
+ * transport-matrix application; an HVP decomposed into transport-vector and
+ * transport-matrix products), for d <= 16 (FS_ERR_UNSUPPORTED_D otherwise). Both stream the
+ * plan P_ij = a_i b_j exp((f_i + g_j - C_ij)/eps) like the potential passes (and screen it
+ * the same way) and never store it.
+ *
+ * Their workspace is fs_transport_workspace_bytes(p) (0 for an invalid shape or d > 16),
+ * larger than fs_workspace_bytes(p): keys with up to 16 payload channels and the HVP's
+ * vectors.
+ */
+FS_API size_t fs_transport_workspace_bytes(const fs_problem* p);
+
+/*
+ * transpose == 0: out (n x k) = P u for u (m x k); transpose == 1: out (m x k) = P^T u for
+ * u (n x k); row-major, device, 4-byte aligned. P is the plan of the given (f, g). k >= 1
+ * (FS_ERR_OPTION otherwise); channels are streamed 16 at a time.
+ */
+FS_API fs_status fs_transport_apply(const fs_problem* p, const float* f, const float* g,
+                                    int32_t transpose, int32_t k, const float* u, float* out,
+                                    void* ws, size_t ws_bytes, fs_stream_t stream);
+
+/*
+ * Hessian-vector product of the loss L(x) = OT_eps at the plan of (F(g), g) (exact at a
+ * converged g), for one vector v_i per point x_i (v and out: n x d, row-major, device):
+ *   (H v)_i = 2 a_i v_i + (2/eps) sum_j P_ij (x_i - y_j)(df_i + dg_j - 2 (x_i - y_j).v_i),
+ * where (df, dg) solves [diag(P1) P; P^T diag(P^T 1)] (df, dg) = (r, s) with
+ * r_i = sum_j P_ij 2 (x_i - y_j).v_i, s_j = sum_i P_ij 2 (x_i - y_j).v_i: the derivative of
+ * the gradient 2 (a_i x_i - sum_j P_ij y_j) when the potentials follow x through the
+ * marginal constraints. The system (positive semi-definite, singular along the gauge
+ * direction (1, -1)) is solved by conjugate gradients on the device, two transport passes
+ * and one host read-back per iteration. opt may be NULL (cg_max_iter 200, cg_tol 1e-6, a
+ * relative residual); report (host, may be NULL) receives the iterations run and the final
+ * relative residual.
+ */
+typedef struct {
+  int32_t cg_max_iter;  /* >= 1 */
+  double cg_tol;        /* >= 0: stop once |residual| <= cg_tol |right-hand side| */
+} fs_hvp_options;
+
+typedef struct {
+  int32_t cg_iters;
+  double cg_rel_residual;
+} fs_hvp_report;
+
+FS_API fs_status fs_hvp(const fs_problem* p, const float* g, const float* v, float* out,
+                        const fs_hvp_options* opt, fs_hvp_report* report, void* ws,
+                        size_t ws_bytes, fs_stream_t stream);
+
+/*
  * Dual objective at (f, g):
  *   D(f, g) = <f, a> + <g, b> - eps * (sum_ij P_ij - m_a * m_b),
  *   P_ij = a_i b_j exp((f_i + g_j - C_ij)/eps),  m_a = sum a, m_b = sum b.

@@ -19,7 +19,7 @@ from . import _lib
 
 __all__ = ["potentials", "cost", "grad_x", "marginal_residual", "solve_host", "workspace_bytes",
            "FsError", "timing_enable", "timing_reset", "timing_get", "launch_count",
-           "screening_enable", "solve"]
+           "screening_enable", "solve", "transport_apply", "hvp"]
 
 
 class FsError(RuntimeError):
@@ -176,6 +176,53 @@ def solve(x, y, a=None, b=None, *, eps: float, n_iters: int = 200, variant: str 
               "converged": None if rep.converged < 0 else bool(rep.converged),
               "final_viol": float(rep.final_viol)}
     return f, g, report
+
+
+def _transport_workspace(P):
+    nbytes = int(_lib.load().fs_transport_workspace_bytes(P.ref))
+    if nbytes == 0:
+        raise ValueError("transport products need 1 <= d <= 16")
+    return _torch().empty(nbytes, dtype=_torch().uint8, device=P.device)
+
+
+def transport_apply(x, y, f, g, u, a=None, b=None, *, eps: float, transpose: bool = False,
+                    workspace=None):
+    """P u (u: (M,) or (M, k)) or, with ``transpose``, P^T u (u: (N,) or (N, k)), with
+    P_ij = a_i b_j exp((f_i + g_j - |x_i - y_j|^2)/eps) streamed, never stored
+    (fs_transport_apply; FlashSinkhorn summary section 3, transport-matrix application)."""
+    torch = _torch()
+    P = _Problem(x, y, a, b, eps)
+    f = _check_tensor(f, "f", (P.n,), P.device)
+    g = _check_tensor(g, "g", (P.m,), P.device)
+    rows_in = P.n if transpose else P.m
+    rows_out = P.m if transpose else P.n
+    vec = u.dim() == 1
+    u2 = u.reshape(-1, 1) if vec else u
+    k = int(u2.shape[1])
+    u2 = _check_tensor(u2, "u", (rows_in, k), P.device)
+    out = torch.empty((rows_out, k), dtype=torch.float32, device=P.device)
+    ws = _transport_workspace(P) if workspace is None else workspace
+    _raise(_lib.load().fs_transport_apply(P.ref, f.data_ptr(), g.data_ptr(), 1 if transpose else 0,
+                                          k, u2.data_ptr(), out.data_ptr(), ws.data_ptr(),
+                                          ws.numel(), P.stream()))
+    return out.reshape(-1) if vec else out
+
+
+def hvp(x, y, g, v, a=None, b=None, *, eps: float, cg_max_iter: int = 200, cg_tol: float = 1e-6,
+        workspace=None):
+    """Hessian-vector product of OT_eps with respect to x at the plan of (F(g), g), v of
+    shape (N, d) (fs_hvp; FlashSinkhorn summary section 3). Returns (H v, report)."""
+    torch = _torch()
+    P = _Problem(x, y, a, b, eps)
+    g = _check_tensor(g, "g", (P.m,), P.device)
+    v = _check_tensor(v, "v", (P.n, P.d), P.device)
+    out = torch.empty((P.n, P.d), dtype=torch.float32, device=P.device)
+    opt = _lib.fs_hvp_options(int(cg_max_iter), float(cg_tol))
+    rep = _lib.fs_hvp_report()
+    ws = _transport_workspace(P) if workspace is None else workspace
+    _raise(_lib.load().fs_hvp(P.ref, g.data_ptr(), v.data_ptr(), out.data_ptr(), ctypes.byref(opt),
+                              ctypes.byref(rep), ws.data_ptr(), ws.numel(), P.stream()))
+    return out, {"cg_iters": int(rep.cg_iters), "cg_rel_residual": float(rep.cg_rel_residual)}
 
 
 def cost(x, y, f, g, a=None, b=None, *, eps: float, workspace=None):

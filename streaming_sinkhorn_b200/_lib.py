@@ -25,7 +25,8 @@ EXPORTS = (
     "fs_status_string", "fs_last_cuda_error", "fs_workspace_bytes", "fs_potentials", "fs_cost",
     "fs_grad_x", "fs_marginal_residual", "fs_solve_host_workspace_bytes", "fs_solve_host",
     "fs_timing_enable", "fs_timing_reset", "fs_timing_get", "fs_launch_count",
-    "fs_potentials_noalloc", "fs_screening_enable", "fs_solve",
+    "fs_potentials_noalloc", "fs_screening_enable", "fs_solve", "fs_transport_workspace_bytes",
+    "fs_transport_apply", "fs_hvp",
 )
 
 VARIANTS = {"alternating": 0, "symmetric": 1}
@@ -48,6 +49,14 @@ class fs_solve_options(ctypes.Structure):
 class fs_solve_report(ctypes.Structure):
     _fields_ = [("iters_run", ctypes.c_int32), ("converged", ctypes.c_int32),
                 ("final_viol", ctypes.c_double)]
+
+
+class fs_hvp_options(ctypes.Structure):
+    _fields_ = [("cg_max_iter", ctypes.c_int32), ("cg_tol", ctypes.c_double)]
+
+
+class fs_hvp_report(ctypes.Structure):
+    _fields_ = [("cg_iters", ctypes.c_int32), ("cg_rel_residual", ctypes.c_double)]
 
 
 class fs_timing_entry(ctypes.Structure):
@@ -91,8 +100,13 @@ def load():
     lib.fs_solve_host.argtypes = [P, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.fs_solve.argtypes = [P, ctypes.POINTER(fs_solve_options), vp, vp,
                              ctypes.POINTER(fs_solve_report), vp, sz, vp]
+    lib.fs_transport_workspace_bytes.argtypes = [P]
+    lib.fs_transport_workspace_bytes.restype = sz
+    lib.fs_transport_apply.argtypes = [P, vp, vp, i32, i32, vp, vp, vp, sz, vp]
+    lib.fs_hvp.argtypes = [P, vp, vp, vp, ctypes.POINTER(fs_hvp_options),
+                           ctypes.POINTER(fs_hvp_report), vp, sz, vp]
     for fn in (lib.fs_potentials, lib.fs_cost, lib.fs_grad_x, lib.fs_marginal_residual,
-               lib.fs_solve_host, lib.fs_solve):
+               lib.fs_solve_host, lib.fs_solve, lib.fs_transport_apply, lib.fs_hvp):
         fn.restype = ctypes.c_int
     lib.fs_timing_enable.argtypes = [ctypes.c_int]
     lib.fs_timing_enable.restype = None

@@ -10,6 +10,7 @@
 
 #include "../../include/fs.h"
 #include "fs_screen.cuh"
+#include "fs_transport.cuh"
 #include "fs_tc.cuh"
 
 namespace fs {
@@ -150,8 +151,16 @@ int num_sms_current() {
   return sms > 0 ? sms : 148;
 }
 
-size_t pass_smem_bytes(int D, int tile_pairs, int stages = kStages) {
-  return static_cast<size_t>(stages) * tile_pairs * key_pair_floats(D) * 4;
+size_t pass_smem_bytes(int D, int tile_pairs, int stages = kStages, int np = 0) {
+  return static_cast<size_t>(stages) * tile_pairs * pair_floats(D, np) * 4;
+}
+
+// Pass kernel selector: what the pass accumulates (PassMode) and, for transport products,
+// how many payload channels its key tiles carry.
+enum PassSel : int { kSelLse = 0, kSelGrad = 1, kSelPay1 = 2, kSelPay4 = 3, kSelPay16 = 4,
+                     kSelDiff = 5 };
+inline int sel_channels(int sel) {
+  return sel == kSelPay1 ? 1 : sel == kSelPay4 ? 4 : sel == kSelPay16 ? 16 : sel == kSelDiff ? 1 : 0;
 }
 
 int occupancy_for(int D, bool grad, int variant, size_t smem);  // defined after the kernels
@@ -311,6 +320,7 @@ constexpr int kEval = 148;    // uint64[3]: pairs evaluated by sorted passes, by
 constexpr int kQueue = 151;   // ints: tiles per unit C and unit count U of the last queue plan
 constexpr int kKept = 152;    // int64: kept tiles K of the last queue plan
 constexpr int kPotChange = 153;  // unsigned: float bits of the largest potential change
+constexpr int kCgDots = 156;     // [4] float64: the HVP solve's dot products and sums
 
 struct Layout {
   int D;       // padded dimension of the FMA path
@@ -331,12 +341,23 @@ struct Layout {
   size_t off_kmask, off_kcount, off_ustart, off_unit_rb, off_rmlb;
   // general solve: deferred biases of x (symmetric schedule), potentials at the last check
   size_t off_defer, off_fprev, off_gprev;
+  // transport products and the Hessian-vector product (layouts asked with acc_ch > 0):
+  // keys with payload channels and the vectors of the HVP's conjugate-gradient solve
+  size_t off_paykeys, off_hvp;
   int64_t part_floats;
 };
 
+constexpr int kTransportChannels = 16;  // payload channels of one transport pass, at most
+
+// Floats of the HVP's vectors: ft, r, df, (u, w, r, p, Ap) over n + m, grad and the final
+// accumulations (n x d), the column data (m x (d + 2)) and the column sums.
+inline int64_t hvp_floats(int64_t n, int64_t m, int d) {
+  return 3 * n + 5 * (n + m) + 3 * n * d + m * (d + 2) + 2 * m + 64;
+}
+
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
-Layout make_layout(int64_t n, int64_t m, int d, int sms) {
+Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0) {
   Layout L{};
   L.D = padded_dim(d);
   L.KP = key_pair_floats(L.D);
@@ -349,10 +370,11 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms) {
     for (int rows_x = 0; rows_x < 2; ++rows_x) {
       const int64_t key_pairs = rows_x ? L.py : L.px;
       const Plan pl = make_plan(rows_x ? n : m, key_pairs, L.D, grad, sms);
-      pf = std::max(pf, partial_floats(pl, L.D, grad));
+      const int ch = std::max(L.D, acc_ch);  // accumulated channels of a gradient-like pass
+      pf = std::max(pf, partial_floats(pl, ch, grad));
       const QPlan q = make_qplan(pl, key_pairs, L.D, grad, sms, L.sorted);
       if (q.on) {
-        pf = std::max(pf, queue_partial_floats(q, L.D, grad));
+        pf = std::max(pf, queue_partial_floats(q, ch, grad));
         mask_words = std::max(mask_words, q.rb * q.mask_words);
         rb_max = std::max(rb_max, q.rb);
         units_max = std::max(units_max, q.units_max);
@@ -440,6 +462,13 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms) {
   o = align_up(o + static_cast<size_t>(n) * sizeof(float));
   L.off_gprev = o;
   o = align_up(o + static_cast<size_t>(m) * sizeof(float));
+  if (acc_ch > 0) {
+    L.off_paykeys = o;
+    o = align_up(o + static_cast<size_t>(std::max(L.px, L.py)) * pair_floats(L.D, acc_ch) *
+                         sizeof(float));
+    L.off_hvp = o;
+    o = align_up(o + static_cast<size_t>(hvp_floats(n, m, d)) * sizeof(float));
+  }
   L.total = o;
   return L;
 }
@@ -453,27 +482,27 @@ inline bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr)
 
 // ---------------- kernel dispatch ----------------
 
-template <int D, int R, int NT, bool GRAD, int G, int MINB, int ST = kStages>
+template <int D, int R, int NT, int MODE, int NP, int G, int MINB, int ST = kStages>
 struct PassKernel {
-  static constexpr auto fn = lse_pass_kernel<D, R, NT, G, GRAD, MINB, ST>;
+  static constexpr auto fn = lse_pass_kernel<D, R, NT, G, MODE, NP, MINB, ST>;
   static void set_smem_attr() {
     static bool done = false;  // idempotent, so a race between threads is harmless
     if (!done) {
       CK(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(pass_smem_bytes(D, 128, ST))));
+                              static_cast<int>(pass_smem_bytes(D, 128, ST, NP))));
       done = true;
     }
   }
   static void launch(const PassParams& P, const Plan& pl, cudaStream_t st) {
     set_smem_attr();
     dim3 grid(static_cast<unsigned>(pl.row_blocks), static_cast<unsigned>(pl.n_splits));
-    fn<<<grid, NT, pass_smem_bytes(D, pl.tile_pairs, ST), st>>>(P);
+    fn<<<grid, NT, pass_smem_bytes(D, pl.tile_pairs, ST, NP), st>>>(P);
     CK(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
   static void launch_queue(const PassParams& P, int64_t units, cudaStream_t st) {
     set_smem_attr();
-    fn<<<static_cast<unsigned>(units), NT, pass_smem_bytes(D, kScreenTile / 2, ST), st>>>(P);
+    fn<<<static_cast<unsigned>(units), NT, pass_smem_bytes(D, kScreenTile / 2, ST, NP), st>>>(P);
     CK(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
@@ -498,18 +527,23 @@ struct PassKernel {
 
 // The kernel of (D, pass type, variant): calls op.template run<Kernel>().
 template <int D, typename Op>
-void with_pass_kernel(bool grad, int variant, Op&& op) {
-  if constexpr (D > 16) {
-    if (grad)
-      op.template run<PassKernel<D, 1, 128, true, 4, 1>>();
+void with_pass_kernel(int sel, int variant, Op&& op) {
+  (void)variant;
+  if constexpr (D > 16) {  // the gradient of wide points; potentials run on the tensor cores
+    if (sel == kSelGrad)
+      op.template run<PassKernel<D, 1, 128, kModeGrad, 0, 4, 1>>();
     else
-      op.template run<PassKernel<D, 1, 128, false, 4, 1>>();
+      op.template run<PassKernel<D, 1, 128, kModeLse, 0, 4, 1>>();
   } else {
-    (void)variant;
-    if (grad)
-      op.template run<PassKernel<D, 2, 32, true, 8, 12, kNarrowStages>>();
-    else
-      op.template run<PassKernel<D, 2, 32, false, 8, 24, kNarrowStages>>();
+    constexpr int S = kNarrowStages;
+    switch (sel) {
+      case kSelGrad: op.template run<PassKernel<D, 2, 32, kModeGrad, 0, 8, 12, S>>(); break;
+      case kSelPay1: op.template run<PassKernel<D, 2, 32, kModePay, 1, 8, 20, S>>(); break;
+      case kSelPay4: op.template run<PassKernel<D, 2, 32, kModePay, 4, 8, 16, S>>(); break;
+      case kSelPay16: op.template run<PassKernel<D, 2, 32, kModePay, 16, 8, 8, S>>(); break;
+      case kSelDiff: op.template run<PassKernel<D, 2, 32, kModeDiff, 1, 8, 8, S>>(); break;
+      default: op.template run<PassKernel<D, 2, 32, kModeLse, 0, 8, 24, S>>(); break;
+    }
   }
 }
 
@@ -547,33 +581,37 @@ struct OccupancyOp {
 };
 
 template <int D>
-void launch_pass_d(const PassParams& P, const Plan& pl, bool grad, cudaStream_t st) {
-  with_pass_kernel<D>(grad, pl.variant, LaunchOp{P, pl, st});
+void launch_pass_d(const PassParams& P, const Plan& pl, int sel, cudaStream_t st) {
+  with_pass_kernel<D>(sel, pl.variant, LaunchOp{P, pl, st});
 }
 
 template <int D>
-void launch_queue_d(const PassParams& P, int64_t units, bool grad, cudaStream_t st) {
-  with_pass_kernel<D>(grad, kQueueVariant, QueueOp{P, units, st});
+void launch_queue_d(const PassParams& P, int64_t units, int sel, cudaStream_t st) {
+  with_pass_kernel<D>(sel, kQueueVariant, QueueOp{P, units, st});
 }
 
 template <int D>
-void launch_screen_d(const PassParams& P, int64_t rb, unsigned* kmask, int* kcount, bool grad,
+void launch_screen_d(const PassParams& P, int64_t rb, unsigned* kmask, int* kcount,
                      cudaStream_t st) {
-  with_pass_kernel<D>(grad, kQueueVariant, ScreenOp{P, rb, kmask, kcount, st});
+  with_pass_kernel<D>(kSelLse, kQueueVariant, ScreenOp{P, rb, kmask, kcount, st});
 }
 
 template <int D>
 void occupancy_d(bool grad, int variant, OccupancyOp* op) {
-  with_pass_kernel<D>(grad, variant, *op);
+  with_pass_kernel<D>(grad ? kSelGrad : kSelLse, variant, *op);
 }
 
 template <int D>
-void launch_combine_d(const PassParams& P, bool grad, cudaStream_t st) {
+void launch_combine_d(const PassParams& P, int sel, cudaStream_t st) {
   const unsigned blocks = static_cast<unsigned>(ceil_div(P.n_rows, 256));
-  if (grad)
-    combine_kernel<D, true><<<blocks, 256, 0, st>>>(P);
-  else
-    combine_kernel<D, false><<<blocks, 256, 0, st>>>(P);
+  switch (sel) {
+    case kSelGrad: combine_kernel<D, kModeGrad, D><<<blocks, 256, 0, st>>>(P); break;
+    case kSelPay1: combine_kernel<D, kModePay, 1><<<blocks, 256, 0, st>>>(P); break;
+    case kSelPay4: combine_kernel<D, kModePay, 4><<<blocks, 256, 0, st>>>(P); break;
+    case kSelPay16: combine_kernel<D, kModePay, 16><<<blocks, 256, 0, st>>>(P); break;
+    case kSelDiff: combine_kernel<D, kModeDiff, D><<<blocks, 256, 0, st>>>(P); break;
+    default: combine_kernel<D, kModeLse, 1><<<blocks, 256, 0, st>>>(P); break;
+  }
   CK(cudaGetLastError());
   g_launches.fetch_add(1, std::memory_order_relaxed);
 }
@@ -670,6 +708,22 @@ void launch_pack_d(const float* pts, int64_t count, int d, const float* w, float
   pack_kernel<D><<<blocks, 256, 0, st>>>(pts, count, d, w, wu, perm, keys, lw, pp);
   CK(cudaGetLastError());
   g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
+template <int D>
+void launch_payload_keys_d(const float* keys, int64_t count, int64_t pairs, const float* pay, int k,
+                           int stride, const int* perm, float* out, int np, cudaStream_t st) {
+  const unsigned blocks = static_cast<unsigned>(ceil_div(2 * pairs, 256));
+  if constexpr (D <= 16) {
+    if (np == 1)
+      payload_keys_kernel<D, 1><<<blocks, 256, 0, st>>>(keys, count, pairs, pay, k, stride, perm, out);
+    else if (np == 4)
+      payload_keys_kernel<D, 4><<<blocks, 256, 0, st>>>(keys, count, pairs, pay, k, stride, perm, out);
+    else
+      payload_keys_kernel<D, 16><<<blocks, 256, 0, st>>>(keys, count, pairs, pay, k, stride, perm, out);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
 }
 
 template <int D>
@@ -771,13 +825,16 @@ struct Ctx {
   int *kcount, *ustart, *unit_rb;
   float* rmlb;     // per-row lower bounds written by the screening kernel
   float *defer, *fprev, *gprev;
+  float* paykeys; // transport passes: keys with payload channels
+  float* hvp;     // the HVP's vectors
+  float ctr[3];   // centre of the clouds' box (first three coordinates)
   float alpha;    // symmetric schedule: blend weight of the potential passes (0: plain)
   bool defer_x;   // the next x-row potential pass leaves its biases in `defer`
   bool no_screen;  // screening found to keep most tiles: the rest of the call runs unscreened
 };
 
 fs_status check_common(const fs_problem* p, void* ws, size_t ws_bytes, size_t* need_out,
-                       int sms) {
+                       int sms, int acc_ch = 0) {
   if (!p) return FS_ERR_NULL;
   if (!shape_ok(p)) return FS_ERR_SHAPE;
   if (p->d > FS_MAX_D) return FS_ERR_UNSUPPORTED_D;
@@ -785,7 +842,7 @@ fs_status check_common(const fs_problem* p, void* ws, size_t ws_bytes, size_t* n
   if (!p->x || !p->y) return FS_ERR_NULL;
   if (!aligned4(p->x) || !aligned4(p->y) || !aligned4(p->a) || !aligned4(p->b))
     return FS_ERR_ALIGNMENT;
-  const Layout L = make_layout(p->n, p->m, p->d, sms);
+  const Layout L = make_layout(p->n, p->m, p->d, sms, acc_ch);
   *need_out = L.total;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || ws_bytes < L.total)
     return FS_ERR_WORKSPACE;
@@ -803,6 +860,10 @@ void carve(Ctx& c, void* ws) {
   c.defer = reinterpret_cast<float*>(c.ws + c.L.off_defer);
   c.fprev = reinterpret_cast<float*>(c.ws + c.L.off_fprev);
   c.gprev = reinterpret_cast<float*>(c.ws + c.L.off_gprev);
+  if (c.L.off_paykeys) {
+    c.paykeys = reinterpret_cast<float*>(c.ws + c.L.off_paykeys);
+    c.hvp = reinterpret_cast<float*>(c.ws + c.L.off_hvp);
+  }
   if (c.L.Dtc) {
     c.rimg_x = c.ws + c.L.off_rimg_x;
     c.kimg_x = c.ws + c.L.off_kimg_x;
@@ -916,6 +977,7 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
     F.bits = sdims == 3 ? 10 : (sdims == 2 ? 16 : 30);
     for (int k = 0; k < sdims; ++k) {
       const float lo = ord_float(boxi[k]), hi = ord_float(boxi[kSortDims + k]);
+      c.ctr[k] = 0.5f * (lo + hi);
       F.lo[k] = lo;
       F.scale[k] = hi > lo ? static_cast<float>(((1u << F.bits) - 1u) / (static_cast<double>(hi) - lo))
                            : 0.0f;
@@ -1053,20 +1115,39 @@ void run_pass_tc(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_
   }
 }
 
+// A transport or Hessian-vector pass: what it accumulates, the streamed keys with their
+// payload, the row vectors (kModeDiff) and where the results go.
+struct PassExtra {
+  int sel;
+  const float* tile_keys;
+  const float* row_v;
+  float* out;
+  int k, stride;
+};
+
 // Sorted FMA passes screen key tiles (see the kernel); `history` adds the bound from the
 // rows' previous LSE2 and the keys' bias change, which exists from a solve's second iteration.
 void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out, float* marg_out,
-              float* grad_out, double* acc, bool history = false) {
+              float* grad_out, double* acc, bool history = false, const PassExtra* ex = nullptr) {
   if (c.use_tc && kind != kGrad) {
     run_pass_tc(c, rows_x, kind, pot_in, pot_out, marg_out, acc);
     return;
   }
   const fs_problem* p = c.p;
-  const bool grad = kind == kGrad;
+  // transport passes are planned (and their partials sized) like the gradient pass
+  const bool grad = kind == kGrad || ex != nullptr;
+  const int sel = ex ? ex->sel : (kind == kGrad ? kSelGrad : kSelLse);
   const int64_t n_rows = rows_x ? p->n : p->m;
   const int64_t key_pairs = rows_x ? c.L.py : c.L.px;
   const Plan pl = make_plan(n_rows, key_pairs, c.L.D, grad, c.sms);
   PassParams P{};
+  if (ex) {
+    P.tile_keys = ex->tile_keys;
+    P.row_v = ex->row_v;
+    P.acc_out = ex->out;
+    P.acc_k = ex->k;
+    P.acc_stride = ex->stride;
+  }
   P.keys = rows_x ? c.ky : c.kx;
   P.qkeys = rows_x ? c.kx : c.ky;
   P.n_rows = n_rows;
@@ -1140,7 +1221,7 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
     P.qscal = reinterpret_cast<const int*>(c.scal + kQueue);
     P.row_mlb = c.rmlb;
     int ti = c.timer->begin();
-    FS_DISPATCH_D(c.L.D, launch_screen_d, P, q.rb, c.kmask, c.kcount, grad, c.st);
+    FS_DISPATCH_D(c.L.D, launch_screen_d, P, q.rb, c.kmask, c.kcount, c.st);
     plan_units_kernel<<<1, 1024, 0, c.st>>>(c.kcount, static_cast<int>(q.rb), q.budget, q.RB,
                                             c.ustart, c.unit_rb,
                                             reinterpret_cast<int*>(c.scal + kQueue),
@@ -1151,18 +1232,18 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
     c.timer->end(ti, kTScreen, 0.0);
     P.kmask = c.kmask;  // the pass counts the tiles each warp evaluates
     ti = c.timer->begin();
-    FS_DISPATCH_D(c.L.D, launch_queue_d, P, q.units_max, grad, c.st);
+    FS_DISPATCH_D(c.L.D, launch_queue_d, P, q.units_max, sel, c.st);
     c.timer->end(ti, tk, pairs);
     ti = c.timer->begin();
-    FS_DISPATCH_D(c.L.D, launch_combine_d, P, grad, c.st);
+    FS_DISPATCH_D(c.L.D, launch_combine_d, P, sel, c.st);
     c.timer->end(ti, kTCombine, 0.0);
   } else {
     int ti = c.timer->begin();
-    FS_DISPATCH_D(c.L.D, launch_pass_d, P, pl, grad, c.st);
+    FS_DISPATCH_D(c.L.D, launch_pass_d, P, pl, sel, c.st);
     c.timer->end(ti, tk, pairs);
     if (pl.n_splits > 1) {
       ti = c.timer->begin();
-      FS_DISPATCH_D(c.L.D, launch_combine_d, P, grad, c.st);
+      FS_DISPATCH_D(c.L.D, launch_combine_d, P, sel, c.st);
       c.timer->end(ti, kTCombine, 0.0);
     }
   }
@@ -1213,14 +1294,15 @@ fs_status guarded(cudaStream_t st, F&& body) {
   }
 }
 
-fs_status begin(Ctx& c, const fs_problem* p, void* ws, size_t ws_bytes, fs_stream_t stream) {
+fs_status begin(Ctx& c, const fs_problem* p, void* ws, size_t ws_bytes, fs_stream_t stream,
+                int acc_ch = 0) {
   c.sms = num_sms_current();
   size_t need = 0;
-  const fs_status s = check_common(p, ws, ws_bytes, &need, c.sms);
+  const fs_status s = check_common(p, ws, ws_bytes, &need, c.sms, acc_ch);
   if (s != FS_OK) return s;
   c.p = p;
   c.st = reinterpret_cast<cudaStream_t>(stream);
-  c.L = make_layout(p->n, p->m, p->d, c.sms);
+  c.L = make_layout(p->n, p->m, p->d, c.sms, acc_ch);
   c.kappa = 1.4426950408889634 / static_cast<double>(p->eps);
   carve(c, ws);
   return FS_OK;
@@ -1267,6 +1349,24 @@ double check_potential(Ctx& c, const float* f, const float* g) {
   float v;
   memcpy(&v, &bits, sizeof(v));
   return static_cast<double>(v);
+}
+
+// out(i, c) = sum_j P_ij pay(j, c) for the rows of one cloud (rows_x: rows x, keys y), c < k,
+// P the plan of (pot_in, key potentials) when pot_in is given, else of (F(g), g) (each row's
+// mass is then its weight). The keys must carry their biases. Channels go 16 at a time.
+void transport_pass(Ctx& c, bool rows_x, const float* pot_in, const float* pay, int k, int stride,
+                    float* out, int out_stride, const float* row_v = nullptr) {
+  const int64_t n_keys = rows_x ? c.p->m : c.p->n;
+  const int64_t pairs = rows_x ? c.L.py : c.L.px;
+  for (int c0 = 0; c0 < k; c0 += kTransportChannels) {
+    const int kc = std::min(kTransportChannels, k - c0);
+    const int np = row_v ? 1 : (kc == 1 ? 1 : (kc <= 4 ? 4 : 16));
+    const int sel = row_v ? kSelDiff : (np == 1 ? kSelPay1 : (np == 4 ? kSelPay4 : kSelPay16));
+    FS_DISPATCH_D(c.L.D, launch_payload_keys_d, rows_x ? c.ky : c.kx, n_keys, pairs, pay + c0, kc,
+                  stride, rows_x ? c.perm_y : c.perm_x, c.paykeys, np, c.st);
+    PassExtra ex{sel, c.paykeys, row_v, out + c0, row_v ? c.p->d : kc, out_stride};
+    run_pass(c, rows_x, kMarg, pot_in, nullptr, nullptr, nullptr, nullptr, false, &ex);
+  }
 }
 
 fs_status check_options(const fs_solve_options& o) {
@@ -1347,6 +1447,142 @@ fs_status solve_impl(const fs_problem* p, const fs_solve_options* opt, float* f,
   });
 }
 
+fs_status transport_impl(const fs_problem* p, const float* f, const float* g, int32_t transpose,
+                         int32_t k, const float* u, float* out, void* ws, size_t ws_bytes,
+                         fs_stream_t stream) {
+  Ctx c{};
+  fs_status s = begin(c, p, ws, ws_bytes, stream, kTransportChannels);
+  if (s != FS_OK) return s;
+  if (p->d > 16) return FS_ERR_UNSUPPORTED_D;
+  if (!f || !g || !u || !out) return FS_ERR_NULL;
+  if (!aligned4(f) || !aligned4(g) || !aligned4(u) || !aligned4(out)) return FS_ERR_ALIGNMENT;
+  if (k < 1 || (transpose != 0 && transpose != 1)) return FS_ERR_OPTION;
+  Timer timer(c.st);
+  c.timer = &timer;
+  return guarded(c.st, [&]() -> fs_status {
+    fs_status r = prepare_all(c, {{f, p->n}, {g, p->m}}, false);
+    if (r != FS_OK) return r;
+    if (!transpose) {
+      set_bias(c, false, g);  // keys y carry g; rows x carry f
+      transport_pass(c, true, f, u, k, k, out, k);
+    } else {
+      set_bias(c, true, f);  // keys x carry f; rows y carry g
+      transport_pass(c, false, g, u, k, k, out, k);
+    }
+    return finish(c);
+  });
+}
+
+fs_status hvp_impl(const fs_problem* p, const float* g, const float* v, float* out,
+                   const fs_hvp_options* opt, fs_hvp_report* report, void* ws, size_t ws_bytes,
+                   fs_stream_t stream) {
+  Ctx c{};
+  fs_status s = begin(c, p, ws, ws_bytes, stream, kTransportChannels);
+  if (s != FS_OK) return s;
+  if (p->d > 16) return FS_ERR_UNSUPPORTED_D;
+  if (!g || !v || !out) return FS_ERR_NULL;
+  if (!aligned4(g) || !aligned4(v) || !aligned4(out)) return FS_ERR_ALIGNMENT;
+  const int32_t max_iter = opt ? opt->cg_max_iter : 200;
+  const double tol = opt ? opt->cg_tol : 1e-6;
+  if (max_iter < 1 || !(tol >= 0.0)) return FS_ERR_OPTION;
+  Timer timer(c.st);
+  c.timer = &timer;
+  return guarded(c.st, [&]() -> fs_status {
+    fs_status r = prepare_all(c, {{g, p->m}}, false);
+    if (r != FS_OK) return r;
+    const int64_t n = p->n, m = p->m, nm = n + m;
+    const int32_t d = p->d;
+    // vectors
+    float* ft = c.hvp;
+    float* rv = ft + n;
+    float* zu = rv + n;               // (df, dg) = z
+    float* res = zu + nm;
+    float* dir = res + nm;
+    float* ap = dir + nm;
+    float* prod = ap + nm;            // P w (n) then P^T u (m)
+    float* grad = prod + nm;
+    float* diffsum = grad + n * d;
+    float* v2 = diffsum + n * d;
+    float* colpay = v2 + n * d;        // (n, d + 2)
+    float* coldata = colpay + n * (d + 2);  // (m, d + 2)
+    float* csum = coldata + m * (d + 2);
+    double* dots = c.scal + kCgDots;
+    const unsigned blk = static_cast<unsigned>(ceil_div(nm, 256));
+    const float a_uni = static_cast<float>(1.0 / n);
+    auto launched = [](int k) { g_launches.fetch_add(k, std::memory_order_relaxed); };
+    auto read = [&](double* h, int count) {
+      CK(cudaMemcpyAsync(h, dots, count * sizeof(double), cudaMemcpyDeviceToHost, c.st));
+      CK(cudaStreamSynchronize(c.st));
+    };
+    // 1. keys y carry g; ft = F(g) gives keys x their biases kappa ft + log2 a
+    set_bias(c, false, g);
+    run_pass(c, true, kPot, nullptr, ft, nullptr, nullptr, nullptr);
+    // 2. the gradient at the plan of (ft, g), r and the column pass's payload
+    run_pass(c, true, kGrad, nullptr, nullptr, nullptr, grad, nullptr);
+    hvp_row_prep_kernel<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, c.st>>>(
+        p->x, v, grad, n, d, c.ctr[0], c.ctr[1], c.ctr[2], res, colpay);
+    CK(cudaGetLastError());
+    transport_pass(c, false, g, colpay, d + 2, d + 2, coldata, d + 2);  // column sums and data
+    hvp_col_rhs_kernel<<<static_cast<unsigned>(ceil_div(m, 256)), 256, 0, c.st>>>(
+        p->y, coldata, m, d, c.ctr[0], c.ctr[1], c.ctr[2], res + n, csum);
+    CK(cudaGetLastError());
+    launched(2);
+    // 3. conjugate gradients on [diag(P1) P; P^T diag(P^T 1)] z = (r, s), from z = 0, with
+    //    the gauge direction (1, -1) removed from the right-hand side
+    CK(cudaMemsetAsync(dots, 0, 4 * sizeof(double), c.st));
+    cg_split_sum_kernel<<<reduce_blocks(nm, c.sms), 256, 0, c.st>>>(res, n, m, dots);
+    cg_project_kernel<<<blk, 256, 0, c.st>>>(res, n, m, dots);
+    CK(cudaMemsetAsync(zu, 0, nm * sizeof(float), c.st));
+    CK(cudaMemcpyAsync(dir, res, nm * sizeof(float), cudaMemcpyDeviceToDevice, c.st));
+    cg_dot_kernel<<<reduce_blocks(nm, c.sms), 256, 0, c.st>>>(res, res, nm, dots + 2);
+    CK(cudaGetLastError());
+    launched(3);
+    double h[4];
+    read(h, 4);
+    const double bb = h[2];
+    double rr = bb;
+    int32_t it = 0;
+    while (it < max_iter && rr > tol * tol * bb && rr > 0.0) {
+      transport_pass(c, true, nullptr, dir + n, 1, 1, prod, 1);      // P w
+      transport_pass(c, false, g, dir, 1, 1, prod + n, 1);           // P^T u
+      cg_apply_kernel<<<blk, 256, 0, c.st>>>(dir, p->a, a_uni, csum, prod, prod + n, n, m, ap);
+      CK(cudaMemsetAsync(dots, 0, 2 * sizeof(double), c.st));
+      cg_dot_kernel<<<reduce_blocks(nm, c.sms), 256, 0, c.st>>>(dir, ap, nm, dots);
+      CK(cudaGetLastError());
+      launched(2);
+      read(h, 1);
+      if (!(h[0] > 0.0)) break;
+      const double alpha = rr / h[0];
+      cg_step_kernel<<<blk, 256, 0, c.st>>>(zu, res, dir, ap, nm, static_cast<float>(alpha));
+      cg_dot_kernel<<<reduce_blocks(nm, c.sms), 256, 0, c.st>>>(res, res, nm, dots + 1);
+      CK(cudaGetLastError());
+      launched(2);
+      read(h, 2);
+      const double rr_new = h[1];
+      cg_dir_kernel<<<blk, 256, 0, c.st>>>(dir, res, nm, static_cast<float>(rr_new / rr));
+      CK(cudaGetLastError());
+      launched(1);
+      rr = rr_new;
+      ++it;
+    }
+    // 4. the difference pass with payload dg and row vectors 2 v, then the combination
+    scale_kernel<<<static_cast<unsigned>(ceil_div(n * d, 256)), 256, 0, c.st>>>(v, n * d, 2.0f, v2);
+    CK(cudaGetLastError());
+    launched(1);
+    transport_pass(c, true, nullptr, zu + n, 1, 1, diffsum, d, v2);
+    hvp_final_kernel<<<static_cast<unsigned>(ceil_div(n * d, 256)), 256, 0, c.st>>>(
+        v, p->a, a_uni, zu, grad, diffsum, n, d, 2.0 / static_cast<double>(p->eps), out);
+    CK(cudaGetLastError());
+    launched(1);
+    r = finish(c);
+    if (report) {
+      report->cg_iters = it;
+      report->cg_rel_residual = bb > 0.0 ? std::sqrt(rr / bb) : 0.0;
+    }
+    return r;
+  });
+}
+
 // ---------------- entry points ----------------
 
 fs_status potentials_impl(const fs_problem* p, int32_t n_iters, const float* g_init, float* f,
@@ -1399,6 +1635,23 @@ fs_status fs_potentials(const fs_problem* p, int32_t n_iters, const float* g_ini
 fs_status fs_solve(const fs_problem* p, const fs_solve_options* opt, float* f, float* g,
                    fs_solve_report* report, void* ws, size_t ws_bytes, fs_stream_t stream) {
   return fs::solve_impl(p, opt, f, g, report, ws, ws_bytes, stream);
+}
+
+size_t fs_transport_workspace_bytes(const fs_problem* p) {
+  if (!fs::shape_ok(p) || p->d > 16) return 0;
+  return fs::make_layout(p->n, p->m, p->d, fs::num_sms_current(), fs::kTransportChannels).total;
+}
+
+fs_status fs_transport_apply(const fs_problem* p, const float* f, const float* g,
+                             int32_t transpose, int32_t k, const float* u, float* out, void* ws,
+                             size_t ws_bytes, fs_stream_t stream) {
+  return fs::transport_impl(p, f, g, transpose, k, u, out, ws, ws_bytes, stream);
+}
+
+fs_status fs_hvp(const fs_problem* p, const float* g, const float* v, float* out,
+                 const fs_hvp_options* opt, fs_hvp_report* report, void* ws, size_t ws_bytes,
+                 fs_stream_t stream) {
+  return fs::hvp_impl(p, g, v, out, opt, report, ws, ws_bytes, stream);
 }
 
 fs_status fs_grad_x(const fs_problem* p, const float* g, float* grad_x, void* ws, size_t ws_bytes,

@@ -40,6 +40,17 @@ namespace fs {
 
 // Floats per packed key pair for padded dimension D: 2(D+1) rounded up to 4.
 __host__ __device__ constexpr int key_pair_floats(int D) { return ((2 * (D + 1) + 3) / 4) * 4; }
+// The same with NP payload channels after the bias: [c0 c0' .. h h' p0 p0' .. pad].
+__host__ __device__ constexpr int pair_floats(int D, int NP) {
+  return ((2 * (D + 1 + NP) + 3) / 4) * 4;
+}
+
+// What a pass accumulates next to its row sums (the weights e = 2^(z - m)):
+//   kModeLse  nothing (potential and marginal passes)
+//   kModeGrad sum e (y' - x')                                     (gradient)
+//   kModePay  sum e p_c over NP key payload channels               (transport products)
+//   kModeDiff sum e (p_0 + (y' - x').v_i) (y' - x'), v_i per row   (Hessian-vector product)
+enum PassMode : int { kModeLse = 0, kModeGrad = 1, kModePay = 2, kModeDiff = 3 };
 
 constexpr int kStages = 3;
 constexpr float kLazyThr = 8.0f;
@@ -110,6 +121,12 @@ struct PassParams {
   // biases the other pass of the same iteration must not see yet, where to leave them
   float alpha;
   float* defer_h;           // kPot: new bias of every query row (sorted order), or NULL
+  // transport products and the Hessian-vector product (kModePay, kModeDiff)
+  const float* tile_keys;   // the streamed cloud with payload channels, or NULL (keys)
+  const float* row_v;       // kModeDiff: v_i per query row, (n_rows, d_real), caller order
+  float* acc_out;           // results, caller order: row i at acc_out + i * acc_stride
+  int32_t acc_k;            // channels written (<= the kernel's channel count)
+  int32_t acc_stride;
 };
 
 constexpr int kScreenTile = 256;  // points per screening tile (= kPairPad pairs)
@@ -184,6 +201,19 @@ __device__ __forceinline__ void finish_grad(const PassParams& P, int64_t i, cons
   for (int k = 0; k < P.d_real; ++k) P.grad_out[oi * P.d_real + k] = s * dsum[k];
 }
 
+// kModePay / kModeDiff: out_i = mass_i * (sum_j e_ij acc_ij) / (sum_j e_ij), mass_i the row's
+// plan mass: its weight w_i on the plan of (F(g), g) (pot_in NULL), else the plan marginal
+// w_i 2^(kappa pot_i + LSE2_i) of the given potentials (as finish_marg).
+__device__ __forceinline__ void finish_acc(const PassParams& P, int64_t i, const float* a,
+                                           double l, double lse2) {
+  const int64_t oi = P.perm ? P.perm[i] : i;
+  const double w = P.w ? static_cast<double>(P.w[oi]) : static_cast<double>(P.w_uniform);
+  double mass = w;
+  if (P.pot_in) mass = w > 0.0 ? w * exp2(P.kappa * static_cast<double>(P.pot_in[oi]) + lse2) : 0.0;
+  const double s = l > 0.0 ? mass / l : 0.0;
+  for (int c = 0; c < P.acc_k; ++c) P.acc_out[oi * P.acc_stride + c] = static_cast<float>(s * a[c]);
+}
+
 // Warp-wide minimum of the bias changes, one atomic per warp (NaN never wins fminf).
 __device__ __forceinline__ void reduce_dmin(float v, int* out) {
 #pragma unroll
@@ -224,10 +254,10 @@ __device__ __forceinline__ void block_reduce_marg(double dev_sum, double dev_max
 // ---- the fused streaming pass -------------------------------------------------------------
 
 // Loads the packed components of key pair p of a shared-memory tile.
-template <int D>
-__device__ __forceinline__ void load_pair(const float* tile, int p, u64 (&comp)[key_pair_floats(D) / 2]) {
-  constexpr int NV = key_pair_floats(D) / 4;
-  const ulonglong2* pv = reinterpret_cast<const ulonglong2*>(tile + p * key_pair_floats(D));
+template <int KP>
+__device__ __forceinline__ void load_pair(const float* tile, int p, u64 (&comp)[KP / 2]) {
+  constexpr int NV = KP / 4;
+  const ulonglong2* pv = reinterpret_cast<const ulonglong2*>(tile + p * KP);
 #pragma unroll
   for (int v = 0; v < NV; ++v) {
     const ulonglong2 q = pv[v];
@@ -236,11 +266,14 @@ __device__ __forceinline__ void load_pair(const float* tile, int p, u64 (&comp)[
   }
 }
 
-template <int D, int R, int NT, int G, bool GRAD, int MINB, int ST>
+template <int D, int R, int NT, int G, int MODE, int NP, int MINB, int ST>
 __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) {
   constexpr int kStages = ST;  // depth of the copy ring
-  constexpr int KP = key_pair_floats(D);
-  constexpr int NA = GRAD ? D : 1;
+  constexpr bool GRAD = MODE == kModeGrad;
+  constexpr bool ACC = MODE != kModeLse;   // accumulates more than the row sums
+  constexpr int KP = pair_floats(D, NP);   // key tile layout (payload channels after H)
+  constexpr int NA = (MODE == kModeGrad || MODE == kModeDiff) ? D : (MODE == kModePay ? NP : 1);
+  static_assert(MODE != kModeDiff || NP == 1, "the difference mode reads one payload channel");
   constexpr int RB = R * NT;  // rows of one row block
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ uint64_t bars[kStages];
@@ -270,7 +303,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     const int k0 = static_cast<int>(unit - first) * C;
     n_work = min(C, P.kcount[b] - k0);
     row0 = static_cast<int64_t>(b) * RB;
-    key_src = P.keys;
+    key_src = P.tile_keys ? P.tile_keys : P.keys;
     mrow = P.kmask + static_cast<int64_t>(b) * P.mask_words;
     // Locate ordinal k0: the mask word holding it and how many set bits of that word precede it.
     if (tid < 32) {
@@ -310,7 +343,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     if (p_end > P.key_pairs) p_end = P.key_pairs;
     n_work = static_cast<int>((p_end - p_begin) / P.tile_pairs);
     n_units = P.n_splits;
-    key_src = P.keys + p_begin * KP;
+    key_src = (P.tile_keys ? P.tile_keys : P.keys) + p_begin * KP;
     if (tid == 0 && P.evaluated)
       atomicAdd(P.evaluated, static_cast<unsigned long long>(n_work) * P.tile_pairs * 2 * RB);
   }
@@ -361,6 +394,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
   float m[R], base[R];
   u64 mk[R], L[R];
   u64 A[R][NA];
+  u64 V[R][MODE == kModeDiff ? D : 1];  // kModeDiff: the row's vector v_i, in both lanes
   float q[R];        // CEN: kappa |x'|^2
   u64 cpk[D];        // CEN: the centre, in both lanes
   const u64 nkappa = pk(-P.kappa_f, -P.kappa_f);
@@ -379,6 +413,14 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     L[r] = pk(0.0f, 0.0f);
 #pragma unroll
     for (int k = 0; k < NA; ++k) A[r][k] = pk(0.0f, 0.0f);
+    if constexpr (MODE == kModeDiff) {
+      const int64_t oi = i < P.n_rows ? (P.perm ? P.perm[i] : i) : -1;
+#pragma unroll
+      for (int k = 0; k < D; ++k) {
+        const float v = (oi >= 0 && k < P.d_real) ? P.row_v[oi * P.d_real + k] : 0.0f;
+        V[r][k] = pk(v, v);
+      }
+    }
   }
   if constexpr (CEN) {
 #pragma unroll
@@ -423,7 +465,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     if constexpr (CEN) {
       for (int p = tid; p < P.tile_pairs; p += 32) {
         u64 comp[KP / 2];
-        load_pair<D>(tile, p, comp);
+        load_pair<KP>(tile, p, comp);
         u64 s2 = pk(0.0f, 0.0f);
 #pragma unroll
         for (int k = 0; k < D; ++k) {
@@ -446,7 +488,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         u64 comp[KP / 2];
-        load_pair<D>(tile, pg + g, comp);
+        load_pair<KP>(tile, pg + g, comp);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           if constexpr (CEN) {
@@ -481,7 +523,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
           const float sc = ex2(m[r] - mx_abs);
           const u64 sc2 = pk(sc, sc);
           L[r] = mul2(L[r], sc2);
-          if (GRAD) {
+          if (ACC) {
 #pragma unroll
             for (int k = 0; k < NA; ++k) A[r][k] = mul2(A[r][k], sc2);
           }
@@ -502,18 +544,32 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         u64 comp[KP / 2];
-        if (GRAD) load_pair<D>(tile, pg + g, comp);
+        if (ACC) load_pair<KP>(tile, pg + g, comp);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           float t0, t1;
           upk(tv[r][g], t0, t1);
           const u64 e = pk(ex2(t0), ex2(t1));
           L[r] = add2(L[r], e);
-          if (GRAD) {
+          if constexpr (MODE == kModeGrad) {
 #pragma unroll
             for (int k = 0; k < NA; ++k)
               A[r][k] = CEN ? fma2(e, fma2(X[r][k], nhalf_ik, comp[k]), A[r][k])  // e (y' - x')
                             : fma2(e, sub2(X[r][k], comp[k]), A[r][k]);
+          } else if constexpr (MODE == kModePay) {
+#pragma unroll
+            for (int c = 0; c < NA; ++c) A[r][c] = fma2(e, comp[D + 1 + c], A[r][c]);
+          } else if constexpr (MODE == kModeDiff) {
+            u64 dk[D];
+            u64 w = comp[D + 1];  // p_0 + (y' - x').v_i
+#pragma unroll
+            for (int k = 0; k < D; ++k) {
+              dk[k] = fma2(X[r][k], nhalf_ik, comp[k]);
+              w = fma2(dk[k], V[r][k], w);
+            }
+            const u64 ew = mul2(e, w);
+#pragma unroll
+            for (int k = 0; k < D; ++k) A[r][k] = fma2(ew, dk[k], A[r][k]);
           }
         }
       }
@@ -586,6 +642,16 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
 #pragma unroll
         for (int k = 0; k < NA; ++k) a[k] = diff_sum(r, k);
         finish_grad(P, i, a, l);
+      } else if (ACC) {
+        float a[NA];
+#pragma unroll
+        for (int k = 0; k < NA; ++k) {
+          float a0, a1;
+          upk(A[r][k], a0, a1);
+          a[k] = a0 + a1;
+        }
+        finish_acc(P, i, a, static_cast<double>(l),
+                   static_cast<double>(m[r]) + log2(static_cast<double>(l)));
       } else {
         const double lse2 = static_cast<double>(m[r]) + log2(static_cast<double>(l));
         if (P.kind == kPot) {
@@ -599,8 +665,8 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
         }
       }
     }
-    if (!GRAD && P.kind == kMarg) block_reduce_marg(dev_sum, dev_max, mass, P.acc);
-    if (!GRAD && P.kind == kPot) reduce_dmin(dmin, P.dmin_out);
+    if (!ACC && P.kind == kMarg) block_reduce_marg(dev_sum, dev_max, mass, P.acc);
+    if (!ACC && P.kind == kPot) reduce_dmin(dmin, P.dmin_out);
   } else {
     // Partials of this unit: split mode at [split][rows_pad] (global row index), queue mode
     // at [unit][RB] (row index within the block).
@@ -615,10 +681,13 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       const int64_t o = unit * pstride + poff + i;
       P.part_m[o] = m[r];
       P.part_l[o] = l0 + l1;
-      if (GRAD) {
+      if (ACC) {
 #pragma unroll
-        for (int k = 0; k < NA; ++k)
-          P.part_a[(unit * D + k) * pstride + poff + i] = diff_sum(r, k);
+        for (int k = 0; k < NA; ++k) {
+          float a0, a1;
+          upk(A[r][k], a0, a1);
+          P.part_a[(unit * NA + k) * pstride + poff + i] = GRAD ? diff_sum(r, k) : a0 + a1;
+        }
       }
     }
   }
@@ -628,8 +697,10 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
 // n_splits partials at [split][rows_pad]. Queue mode: the units of the row's block at
 // [unit][rb_rows]; a block with one unit was completed by the pass itself. A partial whose
 // columns were all zero-weight or padding left m = -inf and sum 0 and drops out.
-template <int D, bool GRAD>
+template <int D, int MODE, int NA>
 __global__ void __launch_bounds__(256) combine_kernel(const PassParams P) {
+  constexpr bool GRAD = MODE == kModeGrad;
+  constexpr bool ACC = MODE != kModeLse;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   double dev = 0.0, mass = 0.0;
   float dmin = INFINITY;
@@ -645,33 +716,31 @@ __global__ void __launch_bounds__(256) combine_kernel(const PassParams P) {
     float mx = -INFINITY;
     for (int64_t s = s0; s < s0 + ns; ++s) mx = fmaxf(mx, P.part_m[s * stride + off]);
     double l = 0.0;
-    float a[GRAD ? D : 1];
-    if (GRAD) {
-      for (int k = 0; k < D; ++k) a[k] = 0.0f;
-    }
+    float a[NA];
+    for (int k = 0; k < NA; ++k) a[k] = 0.0f;
     for (int64_t s = s0; s < s0 + ns; ++s) {
       const int64_t o = s * stride + off;
       const float pm = P.part_m[o];
       if (pm == -INFINITY) continue;
       const float w = ex2(pm - mx);
       l += static_cast<double>(P.part_l[o]) * w;
-      if (GRAD) {
-        for (int k = 0; k < D; ++k) a[k] += P.part_a[(s * D + k) * stride + off] * w;
+      if (ACC) {
+        for (int k = 0; k < NA; ++k) a[k] += P.part_a[(s * NA + k) * stride + off] * w;
       }
     }
+    const double lse2 = static_cast<double>(mx) + log2(l);
     if (GRAD) {
       finish_grad(P, i, a, static_cast<float>(l));
+    } else if (ACC) {
+      finish_acc(P, i, a, l, lse2);
+    } else if (P.kind == kPot) {
+      dmin = finish_pot<D>(P, i, lse2);
     } else {
-      const double lse2 = static_cast<double>(mx) + log2(l);
-      if (P.kind == kPot) {
-        dmin = finish_pot<D>(P, i, lse2);
-      } else {
-        finish_marg(P, i, lse2, dev, mass);
-      }
+      finish_marg(P, i, lse2, dev, mass);
     }
   }
-  if (!GRAD && P.kind == kMarg) block_reduce_marg(dev, dev, mass, P.acc);
-  if (!GRAD && P.kind == kPot) reduce_dmin(dmin, P.dmin_out);
+  if (!ACC && P.kind == kMarg) block_reduce_marg(dev, dev, mass, P.acc);
+  if (!ACC && P.kind == kPot) reduce_dmin(dmin, P.dmin_out);
 }
 
 // ---- preparation kernels --------------------------------------------------------------
@@ -771,6 +840,30 @@ __global__ void __launch_bounds__(256) dot_kernel(const float* v, const float* w
 __global__ void cost_finish_kernel(const double* fa, const double* gb, const double* mass,
                                    double eps, double mamb, double* out) {
   if (threadIdx.x == 0 && blockIdx.x == 0) out[0] = fa[0] + gb[0] - eps * (mass[0] - mamb);
+}
+
+// Key tiles with payload: coordinates and bias of every packed pair copied from the
+// standard layout, then NP payload channels, pay[caller index * stride + c] for c < k (0
+// beyond k and for padding points). One thread per point.
+template <int D, int NP>
+__global__ void __launch_bounds__(256) payload_keys_kernel(const float* keys, int64_t count,
+                                                           int64_t pairs, const float* pay,
+                                                           int k, int stride, const int* perm,
+                                                           float* out) {
+  constexpr int K0 = key_pair_floats(D), K1 = pair_floats(D, NP);
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j >= 2 * pairs) return;
+  const int64_t p = j >> 1;
+  const int e = static_cast<int>(j & 1);
+  const float* src = keys + p * K0;
+  float* dst = out + p * K1;
+#pragma unroll
+  for (int c = 0; c <= D; ++c) dst[2 * c + e] = src[2 * c + e];
+  const int64_t oi = j < count ? (perm ? perm[j] : j) : -1;
+#pragma unroll
+  for (int c = 0; c < NP; ++c)
+    dst[2 * (D + 1 + c) + e] = (oi >= 0 && c < k) ? pay[oi * stride + c] : 0.0f;
+  for (int q = 2 * (D + 1 + NP) + e; q < K1; q += 2) dst[q] = 0.0f;
 }
 
 // Symmetric schedule: install the deferred biases of a cloud into its packed keys and

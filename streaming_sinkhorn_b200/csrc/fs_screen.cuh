@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
 #pragma unroll 4
   for (int p = 0; p < TP; ++p) {
     u64 comp[KP / 2];
-    load_pair<D>(anchor_tile, p, comp);
+    load_pair<KP>(anchor_tile, p, comp);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       u64 acc = pk(0.0f, 0.0f);

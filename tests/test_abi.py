@@ -180,3 +180,29 @@ def test_solve_option_errors():
     assert call(opts(stop_mode=1, stop_tol=float("nan"))) == "FS_ERR_OPTION"
     assert st(lib.fs_solve(p, ctypes.byref(opts()), FAKE + 2, FAKE, None, FAKE, need,
                            None)) == "FS_ERR_ALIGNMENT"
+
+
+def test_transport_and_hvp_argument_errors():
+    lib = _lib.load()
+    p = ctypes.byref(prob())
+    base = lib.fs_workspace_bytes(p)
+    need = lib.fs_transport_workspace_bytes(p)
+    assert need > base and need % 256 == 0
+    assert lib.fs_transport_workspace_bytes(ctypes.byref(prob(d=17))) == 0
+    assert lib.fs_transport_workspace_bytes(None) == 0
+    st = lambda c: _lib.STATUS[c]  # noqa: E731
+    ta = lambda *a: st(lib.fs_transport_apply(*a))  # noqa: E731
+    assert ta(p, FAKE, FAKE, 0, 0, FAKE, FAKE, FAKE, need, None) == "FS_ERR_OPTION"
+    assert ta(p, FAKE, FAKE, 2, 3, FAKE, FAKE, FAKE, need, None) == "FS_ERR_OPTION"
+    assert ta(p, None, FAKE, 0, 3, FAKE, FAKE, FAKE, need, None) == "FS_ERR_NULL"
+    assert ta(p, FAKE, FAKE, 0, 3, FAKE + 2, FAKE, FAKE, need, None) == "FS_ERR_ALIGNMENT"
+    assert ta(p, FAKE, FAKE, 0, 3, FAKE, FAKE, FAKE, need - 256, None) == "FS_ERR_WORKSPACE"
+    wide = ctypes.byref(prob(d=17))
+    assert ta(wide, FAKE, FAKE, 0, 3, FAKE, FAKE, FAKE, BIG, None) == "FS_ERR_UNSUPPORTED_D"
+    hv = lambda *a: st(lib.fs_hvp(*a))  # noqa: E731
+    bad_iter = _lib.fs_hvp_options(0, 1e-6)
+    bad_tol = _lib.fs_hvp_options(10, -1.0)
+    assert hv(p, FAKE, FAKE, FAKE, ctypes.byref(bad_iter), None, FAKE, need, None) == "FS_ERR_OPTION"
+    assert hv(p, FAKE, FAKE, FAKE, ctypes.byref(bad_tol), None, FAKE, need, None) == "FS_ERR_OPTION"
+    assert hv(p, FAKE, None, FAKE, None, None, FAKE, need, None) == "FS_ERR_NULL"
+    assert hv(wide, FAKE, FAKE, FAKE, None, None, FAKE, BIG, None) == "FS_ERR_UNSUPPORTED_D"

@@ -1,0 +1,102 @@
+"""GPU parity of the transport products (fs_transport_apply) and the Hessian-vector product
+(fs_hvp) against the fp64 oracle's dense definitions, and of the screened HVP against the
+unscreened one on a clustered problem."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import streaming_sinkhorn_b200 as fs
+from streaming_sinkhorn_b200 import workloads
+from tests.parity_util import dev, inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def problem(n, m, d, eps, seed):
+    return workloads.random_small(n, m, d, seed=seed, eps=eps, n_iters=8)
+
+
+def close(got, ref, rel):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    scale = max(np.abs(ref).max(), 1e-30)
+    err = np.abs(got - ref).max()
+    assert err <= rel * scale, f"max err {err:.3e} vs {rel:.0e} * {scale:.3e}"
+
+
+@pytest.mark.parametrize("k", [1, 3, 5, 16, 20])
+@pytest.mark.parametrize("transpose", [False, True])
+@pytest.mark.parametrize("shape", [(300, 257, 2, 0.1), (129, 700, 3, 0.05), (200, 150, 8, 0.5),
+                                   (90, 100, 16, 1.0)], ids=lambda s: "n{}-m{}-d{}".format(*s[:3]))
+def test_transport_apply_matches_dense_plan(shape, transpose, k):
+    n, m, d, eps = shape
+    w = problem(n, m, d, eps, seed=n + m + d + k)
+    x, y, a, b = inputs(w)
+    f, g = oracle.potentials(w.x, w.y, w.a, w.b, w.eps, 5)
+    f32, g32 = f.astype(np.float32), g.astype(np.float32)
+    rng = np.random.default_rng(k)
+    u = rng.standard_normal(((n if transpose else m), k)).astype(np.float32)
+    out = fs.transport_apply(x, y, dev(f32), dev(g32), dev(u), a, b, eps=w.eps,
+                             transpose=transpose).cpu().numpy()
+    fn = oracle.transport_apply_t if transpose else oracle.transport_apply
+    ref = fn(w.x, w.y, w.a, w.b, w.eps, f32, g32, u)
+    close(out, ref, 1e-4)
+
+
+def test_transport_apply_vector_form():
+    w = problem(100, 80, 3, 0.2, seed=5)
+    x, y, a, b = inputs(w)
+    f, g = oracle.potentials(w.x, w.y, w.a, w.b, w.eps, 5)
+    f32, g32 = f.astype(np.float32), g.astype(np.float32)
+    u = np.random.default_rng(1).standard_normal(80).astype(np.float32)
+    out = fs.transport_apply(x, y, dev(f32), dev(g32), dev(u), a, b, eps=w.eps)
+    assert out.shape == (100,)
+    close(out.cpu().numpy(), oracle.transport_apply(w.x, w.y, w.a, w.b, w.eps, f32, g32, u), 1e-4)
+
+
+@pytest.mark.parametrize("shape", [(120, 90, 2, 0.3), (250, 300, 3, 0.1), (80, 70, 8, 1.0)],
+                         ids=lambda s: "n{}-m{}-d{}".format(*s[:3]))
+def test_hvp_matches_oracle(shape):
+    n, m, d, eps = shape
+    w = problem(n, m, d, eps, seed=7 * n + m)
+    x, y, a, b = inputs(w)
+    # the HVP is defined at any g (the plan of (F(g), g)); both sides use the same one
+    _, g = oracle.potentials(w.x, w.y, w.a, w.b, w.eps, 60)
+    g32 = g.astype(np.float32)
+    v = np.random.default_rng(n).standard_normal((n, d)).astype(np.float32)
+    hv, rep = fs.hvp(x, y, dev(g32), dev(v), a, b, eps=w.eps, cg_max_iter=500, cg_tol=1e-7)
+    ref = oracle.hvp(w.x, w.y, w.a, w.b, w.eps, g32, v)
+    assert rep["cg_iters"] >= 1
+    close(hv.cpu().numpy(), ref, 2e-3)
+
+
+def test_hvp_is_symmetric_on_the_gpu():
+    w = problem(200, 180, 3, 0.2, seed=17)
+    x, y, a, b = inputs(w)
+    _, g = oracle.potentials(w.x, w.y, w.a, w.b, w.eps, 60)
+    gd = dev(g.astype(np.float32))
+    rng = np.random.default_rng(2)
+    u = rng.standard_normal((200, 3)).astype(np.float32)
+    v = rng.standard_normal((200, 3)).astype(np.float32)
+    hu, _ = fs.hvp(x, y, gd, dev(u), a, b, eps=w.eps, cg_max_iter=500, cg_tol=1e-7)
+    hv, _ = fs.hvp(x, y, gd, dev(v), a, b, eps=w.eps, cg_max_iter=500, cg_tol=1e-7)
+    lhs = float((u * hv.cpu().numpy()).sum())
+    rhs = float((v * hu.cpu().numpy()).sum())
+    assert lhs == pytest.approx(rhs, rel=2e-3)
+
+
+def test_hvp_screened_equals_dense():
+    w = workloads.clustered_cube(n=16384, seed=31, n_iters=10, eps=2e-4)
+    x, y, a, b = inputs(w)
+    f, g = fs.potentials(x, y, a, b, eps=w.eps, n_iters=10)
+    v = torch.from_numpy(np.random.default_rng(3).standard_normal((w.n, 3)).astype(np.float32)).cuda()
+    out = {}
+    for screening in (False, True):
+        fs.screening_enable(screening)
+        try:
+            hv, rep = fs.hvp(x, y, g, v, a, b, eps=w.eps, cg_max_iter=60, cg_tol=1e-6)
+        finally:
+            fs.screening_enable(True)
+        out[screening] = (hv.cpu().numpy(), rep)
+    close(out[True][0], out[False][0], 5e-3)
