@@ -351,6 +351,32 @@ def run_native(args, rank, world, local_rank):
                 "iters_run": rep["iters_run"], "converged": rep["converged"],
                 "final_viol": None if rep["final_viol"] != rep["final_viol"] else rep["final_viol"],
                 "pair_evals_per_s": float(w.n) * w.m * rep["iters_run"] / (ms / 1e3)}
+        # a transport-matrix product (P Y, 3 channels) and a Hessian-vector product at the
+        # potentials just solved
+        if w.d <= 16:
+            from streaming_sinkhorn_b200 import _lib
+            p_ = _lib.fs_problem(x.data_ptr(), y.data_ptr(), a.data_ptr(), b.data_ptr(), w.n, w.m,
+                                 w.d, w.eps)
+            import ctypes
+            twork = torch.empty(int(_lib.load().fs_transport_workspace_bytes(ctypes.byref(p_))),
+                                dtype=torch.uint8, device=dev)
+            v = torch.randn((w.n, w.d), generator=torch.Generator().manual_seed(5)).to(dev)
+            for name, call in (
+                    ("transport_apply_PY", lambda: (fs.transport_apply(
+                        x, y, f, g, y, a, b, eps=w.eps, workspace=twork), None)),
+                    ("hvp", lambda: fs.hvp(x, y, g, v, a, b, eps=w.eps, cg_max_iter=50,
+                                           cg_tol=1e-4, workspace=twork))):
+                call()
+                torch.cuda.synchronize(dev)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                _, rep = call()
+                e1.record(stream)
+                e1.synchronize()
+                solve_extras[name] = {"ms": e0.elapsed_time(e1)}
+                if rep is not None:
+                    solve_extras[name].update(rep)
 
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -349,10 +349,12 @@ struct Layout {
 
 constexpr int kTransportChannels = 16;  // payload channels of one transport pass, at most
 
-// Floats of the HVP's vectors: ft, r, df, (u, w, r, p, Ap) over n + m, grad and the final
-// accumulations (n x d), the column data (m x (d + 2)) and the column sums.
+// Floats of the HVP's vectors, in the order hvp_impl carves them: ft and a spare row vector
+// (2n); the solution, residual, direction, product and transport output over n + m (5);
+// the gradient, the difference sums and 2v (3 n d); the column pass's payload (n (d + 2))
+// and output (m (d + 2)); the column sums (m).
 inline int64_t hvp_floats(int64_t n, int64_t m, int d) {
-  return 3 * n + 5 * (n + m) + 3 * n * d + m * (d + 2) + 2 * m + 64;
+  return 2 * n + 5 * (n + m) + 3 * n * d + (n + m) * (d + 2) + m + 64;
 }
 
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
@@ -1505,7 +1507,7 @@ fs_status hvp_impl(const fs_problem* p, const float* g, const float* v, float* o
     float* v2 = diffsum + n * d;
     float* colpay = v2 + n * d;        // (n, d + 2)
     float* coldata = colpay + n * (d + 2);  // (m, d + 2)
-    float* csum = coldata + m * (d + 2);
+    float* csum = coldata + m * (d + 2);      // ends at hvp_floats(n, m, d) - 64
     double* dots = c.scal + kCgDots;
     const unsigned blk = static_cast<unsigned>(ceil_div(nm, 256));
     const float a_uni = static_cast<float>(1.0 / n);
