@@ -19,7 +19,7 @@ from . import _lib
 
 __all__ = ["potentials", "cost", "grad_x", "marginal_residual", "solve_host", "workspace_bytes",
            "FsError", "timing_enable", "timing_reset", "timing_get", "launch_count",
-           "screening_enable", "solve", "transport_apply", "hvp"]
+           "screening_enable", "solve", "transport_apply", "hvp", "SamplesLoss"]
 
 
 class FsError(RuntimeError):
@@ -344,3 +344,6 @@ def timing_get() -> dict:
                    "pairs": float(getattr(t, name).pairs),
                    "evaluated": float(getattr(t, name).evaluated)}
             for name in ("lse_pass", "grad_pass", "marg_pass", "combine", "screen")}
+
+
+from .loss import SamplesLoss  # noqa: E402  (uses the functions above)
