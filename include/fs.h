@@ -61,7 +61,18 @@ typedef struct {
   int64_t m;      /* number of target points, >= 1 */
   int32_t d;      /* dimension, 1..FS_MAX_D */
   float eps;      /* entropic regularisation, finite and > 0, in cost units */
+  int32_t cost;   /* fs_cost_kind; 0 (the default of a zeroed struct) is squared Euclidean */
 } fs_problem;
+
+/*
+ * Ground costs. FS_COST_SQEUCLIDEAN: C_ij = |x_i - y_j|^2. FS_COST_COSINE:
+ * C_ij = 1 - cos(x_i, y_j) = |x_i/|x_i| - y_j/|y_j||^2 / 2 (FlashSinkhorn summary: the cosine
+ * distance after normalisation is the other cost of this structure); the library
+ * normalises the points (scaled by sqrt(1/2)) into its workspace, so every pass is the
+ * squared-Euclidean one, and fs_grad_x applies the normalisation's Jacobian. A zero vector
+ * has no direction: FS_ERR_NONFINITE_INPUT. fs_hvp supports the squared-Euclidean cost only.
+ */
+typedef enum { FS_COST_SQEUCLIDEAN = 0, FS_COST_COSINE = 1 } fs_cost_kind;
 
 typedef enum {
   FS_OK = 0,
@@ -70,7 +81,8 @@ typedef enum {
   FS_ERR_EPS = 3,              /* eps not finite or <= 0 */
   FS_ERR_ITERS = 4,            /* n_iters < 1 */
   FS_ERR_NEGATIVE_WEIGHT = 5,  /* a weight is negative or not finite */
-  FS_ERR_NONFINITE_INPUT = 6,  /* a coordinate (or a given potential) is not finite */
+  FS_ERR_NONFINITE_INPUT = 6,  /* a coordinate (or a given potential) is not finite, or a
+                                  point is zero under the cosine cost */
   FS_ERR_MASS_MISMATCH = 7,    /* |sum a - sum b| > 1e-5 * max(sum a, sum b) */
   FS_ERR_ZERO_MASS = 8,        /* sum a == 0 (so every weight is zero) */
   FS_ERR_UNSUPPORTED_D = 9,    /* d > FS_MAX_D */

@@ -20,6 +20,11 @@ Each function names the passage of the pages it follows:
   deviation from (a, b), SinkSLOT README stop_mode "marginal".
 * ``solve`` -- the general solve: symmetric (Jacobi) schedule and the marginal / potential
   stop modes, SinkSLOT README API Reference.
+* ``cosine_inputs`` / ``grad_x_cosine`` -- the cosine cost C = 1 - cos(x, y), which equals
+  |x/|x| - y/|y||^2 / 2: every function above applies to the normalised points scaled by
+  sqrt(1/2), and the gradient with respect to x is the one with respect to those points
+  times the normalisation's Jacobian (FlashSinkhorn summary: "cosine distance after
+  normalization" shares the squared-Euclidean structure).
 * ``transport_apply`` / ``transport_apply_t`` / ``hvp`` (numpy, ``transport.py``) -- the
   transport-vector and transport-matrix products and the Hessian-vector product of the
   loss, FlashSinkhorn summary section 3.
@@ -213,3 +218,24 @@ def solve(x, y, a, b, eps: float, *, n_iters: int = 200, variant: str = "alterna
                                 _p(g), ctypes.byref(it), ctypes.byref(conv), _p(viol)))
     converged = None if conv.value < 0 else bool(conv.value)
     return f, g, int(it.value), converged, float(viol[0])
+
+
+def cosine_inputs(x, y):
+    """The points on which the squared-Euclidean cost is 1 - cos(x, y): sqrt(1/2) x / |x|."""
+    x, y = _d(x), _d(y)
+    s = np.sqrt(0.5)
+    return (s * x / np.linalg.norm(x, axis=1, keepdims=True),
+            s * y / np.linalg.norm(y, axis=1, keepdims=True))
+
+
+def grad_x_cosine(x, y, a, b, eps: float, g, rows=None) -> np.ndarray:
+    """Envelope gradient of OT_eps with respect to x under the cosine cost: the gradient
+    with respect to u = sqrt(1/2) x / |x| times du/dx = sqrt(1/2) (I - e e^T) / |x|,
+    e = x / |x|."""
+    x = _d(x)
+    xs, ys = cosine_inputs(x, y)
+    gu = grad_x(xs, ys, a, b, eps, g, rows=rows)
+    xr = x if rows is None else x[np.asarray(rows)]
+    nrm = np.linalg.norm(xr, axis=1, keepdims=True)
+    e = xr / nrm
+    return np.sqrt(0.5) / nrm * (gu - e * (e * gu).sum(axis=1, keepdims=True))

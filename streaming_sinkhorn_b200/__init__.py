@@ -74,7 +74,7 @@ def _check_tensor(t, name, shape=None, device=None):
 class _Problem:
     """Validated tensors plus the fs_problem struct that points at them."""
 
-    def __init__(self, x, y, a, b, eps):
+    def __init__(self, x, y, a, b, eps, cost="sqeuclidean"):
         torch = _torch()
         if not isinstance(x, torch.Tensor) or x.dim() != 2:
             raise ValueError("x must be a 2-D tensor (N, d)")
@@ -91,10 +91,13 @@ class _Problem:
         self.b = None if b is None else _check_tensor(b, "b", (m,), self.device)
         self.n, self.m, self.d = int(n), int(m), int(d)
         self.eps = float(eps)
+        if cost not in _lib.COSTS:
+            raise ValueError(f"unknown cost {cost!r}: {sorted(_lib.COSTS)}")
+        self.cost = cost
         self.s = _lib.fs_problem(self.x.data_ptr(), self.y.data_ptr(),
                                  None if self.a is None else self.a.data_ptr(),
                                  None if self.b is None else self.b.data_ptr(),
-                                 self.n, self.m, self.d, self.eps)
+                                 self.n, self.m, self.d, self.eps, _lib.COSTS[cost])
 
     @property
     def ref(self):
@@ -104,21 +107,22 @@ class _Problem:
         return _torch().cuda.current_stream(self.device).cuda_stream
 
     def workspace(self):
-        nbytes = workspace_bytes(self.n, self.m, self.d, self.device)
+        nbytes = workspace_bytes(self.n, self.m, self.d, self.device, cost=self.cost)
         # torch's caching allocator returns 512-byte aligned blocks
         return _torch().empty(max(nbytes, 1), dtype=_torch().uint8, device=self.device)
 
 
-def workspace_bytes(n: int, m: int, d: int, device=None) -> int:
+def workspace_bytes(n: int, m: int, d: int, device=None, cost: str = "sqeuclidean") -> int:
     """fs_workspace_bytes for an (n, m, d) problem on ``device`` (the current one if None)."""
     torch = _torch()
     lib = _lib.load()
-    p = _lib.fs_problem(None, None, None, None, int(n), int(m), int(d), 1.0)
+    p = _lib.fs_problem(None, None, None, None, int(n), int(m), int(d), 1.0, _lib.COSTS[cost])
     with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
         return int(lib.fs_workspace_bytes(ctypes.byref(p)))
 
 
-def potentials(x, y, a=None, b=None, *, eps: float, n_iters: int, g_init=None, out=None,
+def potentials(x, y, a=None, b=None, *, eps: float, ground_cost: str = "sqeuclidean",
+               n_iters: int, g_init=None, out=None,
                workspace=None):
     """(f, g) after ``n_iters`` alternating f/g updates starting from g = g_init (or 0).
 
@@ -126,7 +130,7 @@ def potentials(x, y, a=None, b=None, *, eps: float, n_iters: int, g_init=None, o
     (alternating variant, fixed iteration count). ``out`` may pass preallocated (f, g).
     """
     torch = _torch()
-    P = _Problem(x, y, a, b, eps)
+    P = _Problem(x, y, a, b, eps, ground_cost)
     if out is None:
         f = torch.empty(P.n, dtype=torch.float32, device=P.device)
         g = torch.empty(P.m, dtype=torch.float32, device=P.device)
@@ -141,7 +145,8 @@ def potentials(x, y, a=None, b=None, *, eps: float, n_iters: int, g_init=None, o
     return f, g
 
 
-def solve(x, y, a=None, b=None, *, eps: float, n_iters: int = 200, variant: str = "alternating",
+def solve(x, y, a=None, b=None, *, eps: float, ground_cost: str = "sqeuclidean",
+          n_iters: int = 200, variant: str = "alternating",
           alpha: float = 0.5, stop_mode: str = "fixed", stop_max_iter: int = 20000,
           stop_tol: float = 1e-6, stop_check_every: int = 5, g_init=None, out=None,
           workspace=None):
@@ -154,7 +159,7 @@ def solve(x, y, a=None, b=None, *, eps: float, n_iters: int = 200, variant: str 
     under "fixed") and final_viol (NaN under "fixed").
     """
     torch = _torch()
-    P = _Problem(x, y, a, b, eps)
+    P = _Problem(x, y, a, b, eps, ground_cost)
     if out is None:
         f = torch.empty(P.n, dtype=torch.float32, device=P.device)
         g = torch.empty(P.m, dtype=torch.float32, device=P.device)
@@ -185,13 +190,14 @@ def _transport_workspace(P):
     return _torch().empty(nbytes, dtype=_torch().uint8, device=P.device)
 
 
-def transport_apply(x, y, f, g, u, a=None, b=None, *, eps: float, transpose: bool = False,
+def transport_apply(x, y, f, g, u, a=None, b=None, *, eps: float, ground_cost: str = "sqeuclidean",
+                    transpose: bool = False,
                     workspace=None):
     """P u (u: (M,) or (M, k)) or, with ``transpose``, P^T u (u: (N,) or (N, k)), with
     P_ij = a_i b_j exp((f_i + g_j - |x_i - y_j|^2)/eps) streamed, never stored
     (fs_transport_apply; FlashSinkhorn summary section 3, transport-matrix application)."""
     torch = _torch()
-    P = _Problem(x, y, a, b, eps)
+    P = _Problem(x, y, a, b, eps, ground_cost)
     f = _check_tensor(f, "f", (P.n,), P.device)
     g = _check_tensor(g, "g", (P.m,), P.device)
     rows_in = P.n if transpose else P.m
@@ -208,12 +214,13 @@ def transport_apply(x, y, f, g, u, a=None, b=None, *, eps: float, transpose: boo
     return out.reshape(-1) if vec else out
 
 
-def hvp(x, y, g, v, a=None, b=None, *, eps: float, cg_max_iter: int = 200, cg_tol: float = 1e-6,
+def hvp(x, y, g, v, a=None, b=None, *, eps: float, ground_cost: str = "sqeuclidean",
+        cg_max_iter: int = 200, cg_tol: float = 1e-6,
         workspace=None):
     """Hessian-vector product of OT_eps with respect to x at the plan of (F(g), g), v of
     shape (N, d) (fs_hvp; FlashSinkhorn summary section 3). Returns (H v, report)."""
     torch = _torch()
-    P = _Problem(x, y, a, b, eps)
+    P = _Problem(x, y, a, b, eps, ground_cost)
     g = _check_tensor(g, "g", (P.m,), P.device)
     v = _check_tensor(v, "v", (P.n, P.d), P.device)
     out = torch.empty((P.n, P.d), dtype=torch.float32, device=P.device)
@@ -225,10 +232,11 @@ def hvp(x, y, g, v, a=None, b=None, *, eps: float, cg_max_iter: int = 200, cg_to
     return out, {"cg_iters": int(rep.cg_iters), "cg_rel_residual": float(rep.cg_rel_residual)}
 
 
-def cost(x, y, f, g, a=None, b=None, *, eps: float, workspace=None):
+def cost(x, y, f, g, a=None, b=None, *, eps: float, ground_cost: str = "sqeuclidean",
+         workspace=None):
     """Dual objective <f,a> + <g,b> - eps (sum_ij P_ij - m_a m_b) as a 0-d float64 tensor."""
     torch = _torch()
-    P = _Problem(x, y, a, b, eps)
+    P = _Problem(x, y, a, b, eps, ground_cost)
     f = _check_tensor(f, "f", (P.n,), P.device)
     g = _check_tensor(g, "g", (P.m,), P.device)
     out = torch.empty((), dtype=torch.float64, device=P.device)
@@ -238,10 +246,11 @@ def cost(x, y, f, g, a=None, b=None, *, eps: float, workspace=None):
     return out
 
 
-def grad_x(x, y, g, a=None, b=None, *, eps: float, out=None, workspace=None):
+def grad_x(x, y, g, a=None, b=None, *, eps: float, ground_cost: str = "sqeuclidean",
+           out=None, workspace=None):
     """Envelope gradient 2 (a_i x_i - sum_j P_ij y_j) with the plan of (F(g), g), (N, d)."""
     torch = _torch()
-    P = _Problem(x, y, a, b, eps)
+    P = _Problem(x, y, a, b, eps, ground_cost)
     g = _check_tensor(g, "g", (P.m,), P.device)
     gr = (torch.empty((P.n, P.d), dtype=torch.float32, device=P.device) if out is None
           else _check_tensor(out, "out", (P.n, P.d), P.device))
@@ -251,14 +260,15 @@ def grad_x(x, y, g, a=None, b=None, *, eps: float, out=None, workspace=None):
     return gr
 
 
-def marginal_residual(x, y, f, g, a=None, b=None, *, eps: float, marginals: bool = False,
+def marginal_residual(x, y, f, g, a=None, b=None, *, eps: float, ground_cost: str = "sqeuclidean",
+                      marginals: bool = False,
                       workspace=None):
     """[sum|P1 - a|, max|P1 - a|, sum|P^T 1 - b|, max|P^T 1 - b|] (float64, device).
 
     With ``marginals=True`` also returns the plan marginals r = P 1 and c = P^T 1.
     """
     torch = _torch()
-    P = _Problem(x, y, a, b, eps)
+    P = _Problem(x, y, a, b, eps, ground_cost)
     f = _check_tensor(f, "f", (P.n,), P.device)
     g = _check_tensor(g, "g", (P.m,), P.device)
     out = torch.empty(4, dtype=torch.float64, device=P.device)
@@ -272,7 +282,8 @@ def marginal_residual(x, y, f, g, a=None, b=None, *, eps: float, marginals: bool
 
 
 def solve_host(x, y, a=None, b=None, *, eps: float, n_iters: int, grad: bool = True,
-               residual: bool = True, cost: bool = True, device=None, workspace=None, out=None):
+               residual: bool = True, cost: bool = True, device=None, workspace=None, out=None,
+               ground_cost: str = "sqeuclidean"):
     """One fs_solve_host call on host arrays (numpy or CPU tensors, float32).
 
     Copies the inputs to the device, solves, and copies f, g and the requested extras
@@ -296,7 +307,8 @@ def solve_host(x, y, a=None, b=None, *, eps: float, n_iters: int, grad: bool = T
     m = yh.shape[0]
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     p = _lib.fs_problem(xh.data_ptr(), yh.data_ptr(), None if ah is None else ah.data_ptr(),
-                        None if bh is None else bh.data_ptr(), n, m, d, float(eps))
+                        None if bh is None else bh.data_ptr(), n, m, d, float(eps),
+                        _lib.COSTS[ground_cost])
     lib = _lib.load()
     with torch.cuda.device(dev):
         nbytes = int(lib.fs_solve_host_workspace_bytes(ctypes.byref(p)))

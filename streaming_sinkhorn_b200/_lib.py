@@ -36,7 +36,10 @@ STOP_MODES = {"fixed": 0, "marginal": 1, "potential": 2}
 class fs_problem(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("y", ctypes.c_void_p), ("a", ctypes.c_void_p),
                 ("b", ctypes.c_void_p), ("n", ctypes.c_int64), ("m", ctypes.c_int64),
-                ("d", ctypes.c_int32), ("eps", ctypes.c_float)]
+                ("d", ctypes.c_int32), ("eps", ctypes.c_float), ("cost", ctypes.c_int32)]
+
+
+COSTS = {"sqeuclidean": 0, "cosine": 1}
 
 
 class fs_solve_options(ctypes.Structure):

@@ -344,6 +344,8 @@ struct Layout {
   // transport products and the Hessian-vector product (layouts asked with acc_ch > 0):
   // keys with payload channels and the vectors of the HVP's conjugate-gradient solve
   size_t off_paykeys, off_hvp;
+  // cosine cost: the normalised copies of x and y
+  size_t off_cos;
   int64_t part_floats;
 };
 
@@ -359,7 +361,7 @@ inline int64_t hvp_floats(int64_t n, int64_t m, int d) {
 
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
-Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0) {
+Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0, bool cosine = false) {
   Layout L{};
   L.D = padded_dim(d);
   L.KP = key_pair_floats(L.D);
@@ -470,6 +472,10 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0) {
                          sizeof(float));
     L.off_hvp = o;
     o = align_up(o + static_cast<size_t>(hvp_floats(n, m, d)) * sizeof(float));
+  }
+  if (cosine) {
+    L.off_cos = o;
+    o = align_up(o + static_cast<size_t>(n + m) * d * sizeof(float));
   }
   L.total = o;
   return L;
@@ -830,6 +836,8 @@ struct Ctx {
   float* paykeys; // transport passes: keys with payload channels
   float* hvp;     // the HVP's vectors
   float ctr[3];   // centre of the clouds' box (first three coordinates)
+  fs_problem pn;  // cosine cost: the problem on the normalised copies (c.p points here)
+  float *cos_x, *cos_y;
   float alpha;    // symmetric schedule: blend weight of the potential passes (0: plain)
   bool defer_x;   // the next x-row potential pass leaves its biases in `defer`
   bool no_screen;  // screening found to keep most tiles: the rest of the call runs unscreened
@@ -841,10 +849,11 @@ fs_status check_common(const fs_problem* p, void* ws, size_t ws_bytes, size_t* n
   if (!shape_ok(p)) return FS_ERR_SHAPE;
   if (p->d > FS_MAX_D) return FS_ERR_UNSUPPORTED_D;
   if (!(std::isfinite(p->eps) && p->eps > 0.0f)) return FS_ERR_EPS;
+  if (p->cost != FS_COST_SQEUCLIDEAN && p->cost != FS_COST_COSINE) return FS_ERR_OPTION;
   if (!p->x || !p->y) return FS_ERR_NULL;
   if (!aligned4(p->x) || !aligned4(p->y) || !aligned4(p->a) || !aligned4(p->b))
     return FS_ERR_ALIGNMENT;
-  const Layout L = make_layout(p->n, p->m, p->d, sms, acc_ch);
+  const Layout L = make_layout(p->n, p->m, p->d, sms, acc_ch, p->cost == FS_COST_COSINE);
   *need_out = L.total;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || ws_bytes < L.total)
     return FS_ERR_WORKSPACE;
@@ -862,6 +871,10 @@ void carve(Ctx& c, void* ws) {
   c.defer = reinterpret_cast<float*>(c.ws + c.L.off_defer);
   c.fprev = reinterpret_cast<float*>(c.ws + c.L.off_fprev);
   c.gprev = reinterpret_cast<float*>(c.ws + c.L.off_gprev);
+  if (c.L.off_cos) {
+    c.cos_x = reinterpret_cast<float*>(c.ws + c.L.off_cos);
+    c.cos_y = c.cos_x + c.p->n * c.p->d;
+  }
   if (c.L.off_paykeys) {
     c.paykeys = reinterpret_cast<float*>(c.ws + c.L.off_paykeys);
     c.hvp = reinterpret_cast<float*>(c.ws + c.L.off_hvp);
@@ -905,6 +918,22 @@ unsigned reduce_blocks(int64_t count, int sms) {
 // `pots` lists potentials to check for finiteness (device pointers with their lengths).
 fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& pots,
                   bool need_tc) {
+  if (c.p->cost == FS_COST_COSINE) {
+    // every pass below runs on the normalised copies, under the squared-Euclidean cost
+    const fs_problem* p0 = c.p;
+    normalize_kernel<<<static_cast<unsigned>(ceil_div(p0->n, 256)), 256, 0, c.st>>>(
+        p0->x, p0->n, p0->d, c.cos_x);
+    CK(cudaGetLastError());
+    normalize_kernel<<<static_cast<unsigned>(ceil_div(p0->m, 256)), 256, 0, c.st>>>(
+        p0->y, p0->m, p0->d, c.cos_y);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(2, std::memory_order_relaxed);
+    c.pn = *p0;
+    c.pn.x = c.cos_x;
+    c.pn.y = c.cos_y;
+    c.pn.cost = FS_COST_SQEUCLIDEAN;
+    c.p = &c.pn;
+  }
   const fs_problem* p = c.p;
   c.use_tc = need_tc && c.L.Dtc > 0;
   CK(cudaMemsetAsync(c.scal, 0, kScalarDoubles * sizeof(double), c.st));
@@ -1304,7 +1333,7 @@ fs_status begin(Ctx& c, const fs_problem* p, void* ws, size_t ws_bytes, fs_strea
   if (s != FS_OK) return s;
   c.p = p;
   c.st = reinterpret_cast<cudaStream_t>(stream);
-  c.L = make_layout(p->n, p->m, p->d, c.sms, acc_ch);
+  c.L = make_layout(p->n, p->m, p->d, c.sms, acc_ch, p->cost == FS_COST_COSINE);
   c.kappa = 1.4426950408889634 / static_cast<double>(p->eps);
   carve(c, ws);
   return FS_OK;
@@ -1482,6 +1511,7 @@ fs_status hvp_impl(const fs_problem* p, const float* g, const float* v, float* o
   fs_status s = begin(c, p, ws, ws_bytes, stream, kTransportChannels);
   if (s != FS_OK) return s;
   if (p->d > 16) return FS_ERR_UNSUPPORTED_D;
+  if (p->cost != FS_COST_SQEUCLIDEAN) return FS_ERR_OPTION;
   if (!g || !v || !out) return FS_ERR_NULL;
   if (!aligned4(g) || !aligned4(v) || !aligned4(out)) return FS_ERR_ALIGNMENT;
   const int32_t max_iter = opt ? opt->cg_max_iter : 200;
@@ -1626,7 +1656,8 @@ const char* fs_last_cuda_error(void) { return fs::g_cuda_err; }
 
 size_t fs_workspace_bytes(const fs_problem* p) {
   if (!fs::shape_ok(p) || p->d > FS_MAX_D) return 0;
-  return fs::make_layout(p->n, p->m, p->d, fs::num_sms_current()).total;
+  return fs::make_layout(p->n, p->m, p->d, fs::num_sms_current(), 0,
+                         p->cost == FS_COST_COSINE).total;
 }
 
 fs_status fs_potentials(const fs_problem* p, int32_t n_iters, const float* g_init, float* f,
@@ -1641,7 +1672,8 @@ fs_status fs_solve(const fs_problem* p, const fs_solve_options* opt, float* f, f
 
 size_t fs_transport_workspace_bytes(const fs_problem* p) {
   if (!fs::shape_ok(p) || p->d > 16) return 0;
-  return fs::make_layout(p->n, p->m, p->d, fs::num_sms_current(), fs::kTransportChannels).total;
+  return fs::make_layout(p->n, p->m, p->d, fs::num_sms_current(), fs::kTransportChannels,
+                         p->cost == FS_COST_COSINE).total;
 }
 
 fs_status fs_transport_apply(const fs_problem* p, const float* f, const float* g,
@@ -1671,6 +1703,12 @@ fs_status fs_grad_x(const fs_problem* p, const float* g, float* grad_x, void* ws
     if (r != FS_OK) return r;
     set_bias(c, false, g);
     run_pass(c, true, kGrad, nullptr, nullptr, nullptr, grad_x, nullptr);
+    if (p->cost == FS_COST_COSINE) {
+      cosine_grad_kernel<<<static_cast<unsigned>(ceil_div(p->n, 256)), 256, 0, c.st>>>(
+          p->x, p->n, p->d, grad_x);
+      CK(cudaGetLastError());
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+    }
     return finish(c);
   });
 }

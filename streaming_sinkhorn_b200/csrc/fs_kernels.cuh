@@ -866,6 +866,32 @@ __global__ void __launch_bounds__(256) payload_keys_kernel(const float* keys, in
   for (int q = 2 * (D + 1 + NP) + e; q < K1; q += 2) dst[q] = 0.0f;
 }
 
+// Cosine cost: x_i sqrt(1/2) / |x_i|, so that |x~_i - y~_j|^2 = 1 - cos(x_i, y_j). A zero
+// point gives non-finite coordinates, which the coordinate check then reports.
+__global__ void __launch_bounds__(256) normalize_kernel(const float* pts, int64_t count, int32_t d,
+                                                        float* out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= count) return;
+  float s2 = 0.0f;
+  for (int k = 0; k < d; ++k) s2 = fmaf(pts[i * d + k], pts[i * d + k], s2);
+  const float sc = 0.70710678118654752f / sqrtf(s2);
+  for (int k = 0; k < d; ++k) out[i * d + k] = pts[i * d + k] * sc;
+}
+
+// Cosine cost: the gradient with respect to x from the one with respect to
+// x~ = sqrt(1/2) x / |x|: multiply by the Jacobian sqrt(1/2) (I - u u^T) / |x|, u = x / |x|.
+__global__ void __launch_bounds__(256) cosine_grad_kernel(const float* pts, int64_t count, int32_t d,
+                                                          float* grad) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= count) return;
+  float s2 = 0.0f, ug = 0.0f;
+  for (int k = 0; k < d; ++k) s2 = fmaf(pts[i * d + k], pts[i * d + k], s2);
+  const float inv = 1.0f / sqrtf(s2);
+  for (int k = 0; k < d; ++k) ug = fmaf(pts[i * d + k] * inv, grad[i * d + k], ug);
+  const float sc = 0.70710678118654752f * inv;
+  for (int k = 0; k < d; ++k) grad[i * d + k] = sc * (grad[i * d + k] - pts[i * d + k] * inv * ug);
+}
+
 // Symmetric schedule: install the deferred biases of a cloud into its packed keys and
 // record the smallest change (for the screening history bound of the next pass).
 template <int D>

@@ -23,13 +23,15 @@ class _OTLoss:
 
             class OTLossFunction(torch.autograd.Function):
                 @staticmethod
-                def forward(ctx, x, y, a, b, eps, options):
+                def forward(ctx, x, y, a, b, eps, ground_cost, options):
                     xd, yd = x.detach(), y.detach()
-                    f, g, report = solve(xd, yd, a, b, eps=eps, **options)
-                    value = cost(xd, yd, f, g, a, b, eps=eps)
+                    f, g, report = solve(xd, yd, a, b, eps=eps, ground_cost=ground_cost,
+                                         **options)
+                    value = cost(xd, yd, f, g, a, b, eps=eps, ground_cost=ground_cost)
                     ctx.save_for_backward(xd, yd, f, g)
                     ctx.weights = (a, b)
                     ctx.eps = eps
+                    ctx.ground_cost = ground_cost
                     ctx.report = report
                     return value.to(x.dtype)
 
@@ -40,11 +42,13 @@ class _OTLoss:
                     gx = gy = None
                     if ctx.needs_input_grad[0]:
                         # 2 (a_i x_i - sum_j P_ij y_j), the plan of (F(g), g)
-                        gx = grad_x(x, y, g, a, b, eps=ctx.eps) * grad_out
+                        gx = grad_x(x, y, g, a, b, eps=ctx.eps,
+                                    ground_cost=ctx.ground_cost) * grad_out
                     if ctx.needs_input_grad[1]:
                         # the same with the clouds' roles swapped: the plan of (f, G(f))
-                        gy = grad_x(y, x, f, b, a, eps=ctx.eps) * grad_out
-                    return gx, gy, None, None, None, None
+                        gy = grad_x(y, x, f, b, a, eps=ctx.eps,
+                                    ground_cost=ctx.ground_cost) * grad_out
+                    return gx, gy, None, None, None, None, None
 
             cls.fn = OTLossFunction
         return cls.fn
@@ -54,7 +58,8 @@ class SamplesLoss:
     """Entropic optimal transport loss between two weighted point clouds.
 
     ``SamplesLoss(eps, n_iters=200, variant="alternating", alpha=0.5, stop_mode="fixed",
-    stop_max_iter=20000, stop_tol=1e-6, stop_check_every=5)``; ``loss(x, y, a=None, b=None)``
+    stop_max_iter=20000, stop_tol=1e-6, stop_check_every=5, ground_cost="sqeuclidean")``
+    (or "cosine"); ``loss(x, y, a=None, b=None)``
     returns OT_eps as a 0-d tensor (the dual objective <f,a> + <g,b> - eps (sum P - m_a m_b)
     at the solved potentials) with gradients for x and y; ``loss(x, y, potentials=True)``
     returns the potentials (f, g) in cost units instead. ``last_report`` holds the solve's
@@ -63,8 +68,10 @@ class SamplesLoss:
 
     def __init__(self, eps: float = 0.05, n_iters: int = 200, variant: str = "alternating",
                  alpha: float = 0.5, stop_mode: str = "fixed", stop_max_iter: int = 20000,
-                 stop_tol: float = 1e-6, stop_check_every: int = 5):
+                 stop_tol: float = 1e-6, stop_check_every: int = 5,
+                 ground_cost: str = "sqeuclidean"):
         self.eps = float(eps)
+        self.ground_cost = ground_cost
         self.options = dict(n_iters=n_iters, variant=variant, alpha=alpha, stop_mode=stop_mode,
                             stop_max_iter=stop_max_iter, stop_tol=stop_tol,
                             stop_check_every=stop_check_every)
@@ -73,7 +80,7 @@ class SamplesLoss:
     def __call__(self, x, y, a=None, b=None, potentials: bool = False):
         if potentials:
             f, g, self.last_report = solve(x.detach(), y.detach(), a, b, eps=self.eps,
-                                           **self.options)
+                                           ground_cost=self.ground_cost, **self.options)
             return f, g
         fn = _OTLoss.get()
-        return fn.apply(x, y, a, b, self.eps, self.options)
+        return fn.apply(x, y, a, b, self.eps, self.ground_cost, self.options)

@@ -465,3 +465,53 @@ def test_hvp_large_eps_limit():
     assert errs[2] < errs[1] < errs[0]
     assert errs[2] < 1e-3 * np.abs(2.0 * a[:, None] * v).max()
     assert errs[1] / errs[2] == pytest.approx(10.0, rel=0.2)
+
+
+# --- the cosine cost -------------------------------------------------------------------------
+
+def cosine_cost_matrix(x, y):
+    x = np.asarray(x, np.float64)
+    y = np.asarray(y, np.float64)
+    return 1.0 - (x @ y.T) / np.outer(np.linalg.norm(x, axis=1), np.linalg.norm(y, axis=1))
+
+
+def test_cosine_matches_scaling_on_the_cosine_matrix():
+    """Sinkhorn-Knopp on exp(-(1 - cos)/eps), computed from the cosines directly."""
+    x, y, a, b, _ = small(19, 23, 4, 21)
+    C = cosine_cost_matrix(x, y)
+    eps = 0.05
+    K = np.exp(-C / eps)
+    v = b.copy()
+    for _ in range(7):
+        Kv = K @ v
+        u = a / Kv
+        Ktu = K.T @ u
+        v = b / Ktu
+    xs, ys = oracle.cosine_inputs(x, y)
+    f, g = oracle.potentials(xs, ys, a, b, eps, 7)
+    np.testing.assert_allclose(f, -eps * np.log(Kv), rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(g, -eps * np.log(Ktu), rtol=1e-11, atol=1e-13)
+    # the identity behind it
+    np.testing.assert_allclose(dense_cost(xs, ys), C, rtol=1e-12, atol=1e-14)
+
+
+def test_cosine_gradient_matches_finite_differences():
+    x, y, a, b, _ = small(11, 9, 3, 22)
+    eps = 0.1
+    # a direction not drawn like x (the same draws would be parallel to each point, along
+    # which the cosine cost does not move)
+    v = np.random.default_rng(1022).standard_normal(x.shape)
+    h = 1e-5
+
+    def loss_at(xx):
+        xs, ys = oracle.cosine_inputs(xx, y)
+        f, g = converged(xs, ys, a, b, eps)
+        return oracle.cost(xs, ys, a, b, eps, f, g)
+
+    fd = (loss_at(x + h * v) - loss_at(x - h * v)) / (2.0 * h)
+    xs, ys = oracle.cosine_inputs(x, y)
+    _, g = converged(xs, ys, a, b, eps)
+    gr = oracle.grad_x_cosine(x, y, a, b, eps, g)
+    assert (gr * v).sum() == pytest.approx(fd, rel=1e-6, abs=1e-12)
+    # the gradient is orthogonal to each point: scaling a point leaves its cosines alone
+    np.testing.assert_allclose((gr * x).sum(axis=1), 0.0, atol=1e-12)
