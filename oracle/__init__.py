@@ -25,6 +25,11 @@ Each function names the passage of the pages it follows:
   sqrt(1/2), and the gradient with respect to x is the one with respect to those points
   times the normalisation's Jacobian (FlashSinkhorn summary: "cosine distance after
   normalization" shares the squared-Euclidean structure).
+* ``divergence`` -- the debiased (Sinkhorn) divergence
+  S = OT(a, b) - OT(a, a)/2 - OT(b, b)/2, each term the dual objective of its own solve with
+  the same schedule, and its gradients: grad_x S = grad_x OT(x, y) - (G1 + G2)/2 with G1, G2
+  the envelope gradients of OT(x, x) from each side (FlashSinkhorn 2 abstract and SinkSLOT
+  README: the debiased "divergence" the losses report).
 * ``transport_apply`` / ``transport_apply_t`` / ``hvp`` (numpy, ``transport.py``) -- the
   transport-vector and transport-matrix products and the Hessian-vector product of the
   loss, FlashSinkhorn summary section 3.
@@ -239,3 +244,21 @@ def grad_x_cosine(x, y, a, b, eps: float, g, rows=None) -> np.ndarray:
     nrm = np.linalg.norm(xr, axis=1, keepdims=True)
     e = xr / nrm
     return np.sqrt(0.5) / nrm * (gu - e * (e * gu).sum(axis=1, keepdims=True))
+
+
+def divergence(x, y, a, b, eps: float, grads: bool = False, **solve_options):
+    """S = OT(x, y) - OT(x, x)/2 - OT(y, y)/2, each solved by ``solve`` with the same
+    options; with ``grads`` also (grad_x S, grad_y S)."""
+    x, y, a, b = _d(x), _d(y), _d(a), _d(b)
+    fxy, gxy, *_ = solve(x, y, a, b, eps, **solve_options)
+    fxx, gxx, *_ = solve(x, x, a, a, eps, **solve_options)
+    fyy, gyy, *_ = solve(y, y, b, b, eps, **solve_options)
+    value = (cost(x, y, a, b, eps, fxy, gxy) - 0.5 * cost(x, x, a, a, eps, fxx, gxx)
+             - 0.5 * cost(y, y, b, b, eps, fyy, gyy))
+    if not grads:
+        return value
+    gx = grad_x(x, y, a, b, eps, gxy) - 0.5 * (grad_x(x, x, a, a, eps, gxx)
+                                               + grad_x(x, x, a, a, eps, fxx))
+    gy = grad_x(y, x, b, a, eps, fxy) - 0.5 * (grad_x(y, y, b, b, eps, gyy)
+                                               + grad_x(y, y, b, b, eps, fyy))
+    return value, gx, gy

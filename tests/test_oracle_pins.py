@@ -515,3 +515,45 @@ def test_cosine_gradient_matches_finite_differences():
     assert (gr * v).sum() == pytest.approx(fd, rel=1e-6, abs=1e-12)
     # the gradient is orthogonal to each point: scaling a point leaves its cosines alone
     np.testing.assert_allclose((gr * x).sum(axis=1), 0.0, atol=1e-12)
+
+
+# --- the debiased divergence ---------------------------------------------------------------
+
+CONV = dict(stop_mode="marginal", stop_tol=1e-13, stop_check_every=10, stop_max_iter=200000)
+
+
+@pytest.mark.parametrize("seed", [30, 31, 32])
+def test_divergence_is_nonnegative_and_zero_on_equal_clouds(seed):
+    """At convergence the Sinkhorn divergence of the squared-Euclidean cost (a positive
+    Gibbs kernel) is nonnegative, and zero for equal measures (Feydy et al. 2019, cited
+    among the FS2 page's references for the debiased loss)."""
+    x, y, a, b, _ = small(13, 17, 2, seed)
+    eps = float(dense_cost(x, y).max()) / 6.0
+    assert oracle.divergence(x, y, a, b, eps, **CONV) > 0.0
+    assert abs(oracle.divergence(x, x, a, a, eps, **CONV)) < 1e-12
+
+
+def test_divergence_large_eps_limit():
+    """As eps grows each plan tends to the product of the marginals, and
+    S -> int C d(a b) - int C d(a a)/2 - int C d(b b)/2 = |mean_a x - mean_b y|^2."""
+    x, y, a, b, _ = small(10, 12, 3, 33)
+    mx = (a[:, None] * x).sum(0) / a.sum()
+    my = (b[:, None] * y).sum(0) / b.sum()
+    target = float(((mx - my) ** 2).sum())
+    errs = [abs(oracle.divergence(x, y, a, b, eps, **CONV) - target) for eps in (1e2, 1e3)]
+    assert errs[1] < errs[0] and errs[1] < 1e-2 * target
+
+
+def test_divergence_gradients_match_finite_differences():
+    x, y, a, b, _ = small(9, 8, 2, 34)
+    eps = float(dense_cost(x, y).max()) / 4.0
+    rng = np.random.default_rng(340)
+    vx, vy = rng.standard_normal(x.shape), rng.standard_normal(y.shape)
+    h = 1e-5
+    _, gx, gy = oracle.divergence(x, y, a, b, eps, grads=True, **CONV)
+    fdx = (oracle.divergence(x + h * vx, y, a, b, eps, **CONV)
+           - oracle.divergence(x - h * vx, y, a, b, eps, **CONV)) / (2 * h)
+    fdy = (oracle.divergence(x, y + h * vy, a, b, eps, **CONV)
+           - oracle.divergence(x, y - h * vy, a, b, eps, **CONV)) / (2 * h)
+    assert (gx * vx).sum() == pytest.approx(fdx, rel=1e-6, abs=1e-11)
+    assert (gy * vy).sum() == pytest.approx(fdy, rel=1e-6, abs=1e-11)
