@@ -362,6 +362,9 @@ def run_native(args, rank, world, local_rank):
                                 dtype=torch.uint8, device=dev)
             v = torch.randn((w.n, w.d), generator=torch.Generator().manual_seed(5)).to(dev)
             for name, call in (
+                    ("debiased_divergence_with_grads", lambda: (None, {"value": float(
+                        fs.sinkhorn_divergence(x, y, a, b, eps=w.eps, n_iters=w.n_iters,
+                                               grads=True)[0])})),
                     ("transport_apply_PY", lambda: (fs.transport_apply(
                         x, y, f, g, y, a, b, eps=w.eps, workspace=twork), None)),
                     ("hvp", lambda: fs.hvp(x, y, g, v, a, b, eps=w.eps, cg_max_iter=50,

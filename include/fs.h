@@ -170,6 +170,20 @@ FS_API fs_status fs_solve(const fs_problem* p, const fs_solve_options* opt, floa
                           fs_stream_t stream);
 
 /*
+ * Debiased (Sinkhorn) divergence S = OT(a, b) - OT(a, a)/2 - OT(b, b)/2 (the "divergence"
+ * the pages' losses report): three fs_solve runs with the same options (g_init ignored) and
+ * their dual objectives, value (device, one double) = S. grad_x (n x d) and grad_y (m x d),
+ * device or NULL, receive grad_x S = grad_x OT(x, y) - (G1 + G2)/2 with G1, G2 the envelope
+ * gradients of OT(x, x) from its two sides (they coincide at convergence), and the same for
+ * y. Workspace: fs_divergence_workspace_bytes(p) (the largest of the three problems' plus
+ * the divergence's own vectors). Errors as fs_solve.
+ */
+FS_API size_t fs_divergence_workspace_bytes(const fs_problem* p);
+FS_API fs_status fs_divergence(const fs_problem* p, const fs_solve_options* opt, double* value,
+                               float* grad_x, float* grad_y, void* ws, size_t ws_bytes,
+                               fs_stream_t stream);
+
+/*
  * Transport products and the Hessian-vector product (FlashSinkhorn summary, section 3:
  * transport-matrix application; an HVP decomposed into transport-vector and
  * transport-matrix products), for d <= 16 (FS_ERR_UNSUPPORTED_D otherwise). Both stream the

@@ -19,7 +19,8 @@ from . import _lib
 
 __all__ = ["potentials", "cost", "grad_x", "marginal_residual", "solve_host", "workspace_bytes",
            "FsError", "timing_enable", "timing_reset", "timing_get", "launch_count",
-           "screening_enable", "solve", "transport_apply", "hvp", "SamplesLoss"]
+           "screening_enable", "solve", "transport_apply", "hvp", "SamplesLoss",
+           "sinkhorn_divergence"]
 
 
 class FsError(RuntimeError):
@@ -181,6 +182,30 @@ def solve(x, y, a=None, b=None, *, eps: float, ground_cost: str = "sqeuclidean",
               "converged": None if rep.converged < 0 else bool(rep.converged),
               "final_viol": float(rep.final_viol)}
     return f, g, report
+
+
+def sinkhorn_divergence(x, y, a=None, b=None, *, eps: float, ground_cost: str = "sqeuclidean",
+                        grads: bool = False, n_iters: int = 200, variant: str = "alternating",
+                        alpha: float = 0.5, stop_mode: str = "fixed", stop_max_iter: int = 20000,
+                        stop_tol: float = 1e-6, stop_check_every: int = 5, workspace=None):
+    """Debiased divergence OT(a, b) - OT(a, a)/2 - OT(b, b)/2 (fs_divergence) as a 0-d
+    float64 tensor; with ``grads`` also its gradients for x (N, d) and y (M, d)."""
+    torch = _torch()
+    P = _Problem(x, y, a, b, eps, ground_cost)
+    opt = _lib.fs_solve_options(int(n_iters), _lib.VARIANTS[variant], float(alpha),
+                                _lib.STOP_MODES[stop_mode], int(stop_max_iter),
+                                int(stop_check_every), float(stop_tol), None)
+    value = torch.empty((), dtype=torch.float64, device=P.device)
+    gx = torch.empty((P.n, P.d), dtype=torch.float32, device=P.device) if grads else None
+    gy = torch.empty((P.m, P.d), dtype=torch.float32, device=P.device) if grads else None
+    if workspace is None:
+        nbytes = int(_lib.load().fs_divergence_workspace_bytes(P.ref))
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=P.device)
+    _raise(_lib.load().fs_divergence(P.ref, ctypes.byref(opt), value.data_ptr(),
+                                     None if gx is None else gx.data_ptr(),
+                                     None if gy is None else gy.data_ptr(), workspace.data_ptr(),
+                                     workspace.numel(), P.stream()))
+    return (value, gx, gy) if grads else value
 
 
 def _transport_workspace(P):

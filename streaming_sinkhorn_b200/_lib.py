@@ -26,7 +26,7 @@ EXPORTS = (
     "fs_grad_x", "fs_marginal_residual", "fs_solve_host_workspace_bytes", "fs_solve_host",
     "fs_timing_enable", "fs_timing_reset", "fs_timing_get", "fs_launch_count",
     "fs_potentials_noalloc", "fs_screening_enable", "fs_solve", "fs_transport_workspace_bytes",
-    "fs_transport_apply", "fs_hvp",
+    "fs_transport_apply", "fs_hvp", "fs_divergence_workspace_bytes", "fs_divergence",
 )
 
 VARIANTS = {"alternating": 0, "symmetric": 1}
@@ -108,8 +108,12 @@ def load():
     lib.fs_transport_apply.argtypes = [P, vp, vp, i32, i32, vp, vp, vp, sz, vp]
     lib.fs_hvp.argtypes = [P, vp, vp, vp, ctypes.POINTER(fs_hvp_options),
                            ctypes.POINTER(fs_hvp_report), vp, sz, vp]
+    lib.fs_divergence_workspace_bytes.argtypes = [P]
+    lib.fs_divergence_workspace_bytes.restype = sz
+    lib.fs_divergence.argtypes = [P, ctypes.POINTER(fs_solve_options), vp, vp, vp, vp, sz, vp]
     for fn in (lib.fs_potentials, lib.fs_cost, lib.fs_grad_x, lib.fs_marginal_residual,
-               lib.fs_solve_host, lib.fs_solve, lib.fs_transport_apply, lib.fs_hvp):
+               lib.fs_solve_host, lib.fs_solve, lib.fs_transport_apply, lib.fs_hvp,
+               lib.fs_divergence):
         fn.restype = ctypes.c_int
     lib.fs_timing_enable.argtypes = [ctypes.c_int]
     lib.fs_timing_enable.restype = None

@@ -1670,6 +1670,113 @@ fs_status fs_solve(const fs_problem* p, const fs_solve_options* opt, float* f, f
   return fs::solve_impl(p, opt, f, g, report, ws, ws_bytes, stream);
 }
 
+namespace {
+// The two self problems of the divergence: (x, x, a, a) and (y, y, b, b).
+void self_problems(const fs_problem* p, fs_problem* pxx, fs_problem* pyy) {
+  *pxx = *p;
+  pxx->y = p->x;
+  pxx->b = p->a;
+  pxx->m = p->n;
+  *pyy = *p;
+  pyy->x = p->y;
+  pyy->a = p->b;
+  pyy->n = p->m;
+}
+// The problem with the clouds' roles swapped.
+fs_problem transposed(const fs_problem* p) {
+  fs_problem t = *p;
+  t.x = p->y;
+  t.y = p->x;
+  t.a = p->b;
+  t.b = p->a;
+  t.n = p->m;
+  t.m = p->n;
+  return t;
+}
+// Inner workspace of the divergence (the largest of its three problems), then its vectors:
+// six potentials, two gradient buffers, three costs.
+size_t divergence_inner_bytes(const fs_problem* p) {
+  fs_problem pxx, pyy;
+  self_problems(p, &pxx, &pyy);
+  return std::max({fs_workspace_bytes(p), fs_workspace_bytes(&pxx), fs_workspace_bytes(&pyy)});
+}
+size_t divergence_tail_bytes(const fs_problem* p) {
+  const size_t n = static_cast<size_t>(p->n), m = static_cast<size_t>(p->m),
+               d = static_cast<size_t>(p->d);
+  return fs::align_up((3 * n + 3 * m) * sizeof(float)) + fs::align_up(2 * std::max(n, m) * d * 4) +
+         fs::align_up(3 * sizeof(double));
+}
+}  // namespace
+
+size_t fs_divergence_workspace_bytes(const fs_problem* p) {
+  if (!fs::shape_ok(p) || p->d > FS_MAX_D) return 0;
+  return divergence_inner_bytes(p) + divergence_tail_bytes(p);
+}
+
+fs_status fs_divergence(const fs_problem* p, const fs_solve_options* opt, double* value,
+                        float* grad_x, float* grad_y, void* ws, size_t ws_bytes,
+                        fs_stream_t stream) {
+  using namespace fs;
+  if (!p || !opt || !value) return FS_ERR_NULL;
+  if (!shape_ok(p)) return FS_ERR_SHAPE;
+  if (p->d > FS_MAX_D) return FS_ERR_UNSUPPORTED_D;
+  if ((reinterpret_cast<uintptr_t>(value) & 7u) || !aligned4(grad_x) || !aligned4(grad_y))
+    return FS_ERR_ALIGNMENT;
+  const size_t inner = divergence_inner_bytes(p);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 ||
+      ws_bytes < inner + divergence_tail_bytes(p))
+    return FS_ERR_WORKSPACE;
+  const int64_t n = p->n, m = p->m, d = p->d;
+  unsigned char* tail = static_cast<unsigned char*>(ws) + inner;
+  float* fxy = reinterpret_cast<float*>(tail);
+  float* gxy = fxy + n;
+  float* fxx = gxy + m;
+  float* gxx = fxx + n;
+  float* fyy = gxx + n;
+  float* gyy = fyy + m;
+  float* tmp1 = reinterpret_cast<float*>(tail + align_up((3 * n + 3 * m) * sizeof(float)));
+  float* tmp2 = tmp1 + std::max(n, m) * d;
+  double* costs = reinterpret_cast<double*>(
+      tail + align_up((3 * n + 3 * m) * sizeof(float)) +
+      align_up(2 * static_cast<size_t>(std::max(n, m) * d) * 4));
+  fs_problem pxx, pyy;
+  self_problems(p, &pxx, &pyy);
+  const fs_problem pyx = transposed(p);
+  fs_solve_options o = *opt;
+  o.g_init = nullptr;  // the three problems start alike
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  fs_status s;
+  if ((s = solve_impl(p, &o, fxy, gxy, nullptr, ws, inner, stream)) != FS_OK) return s;
+  if ((s = solve_impl(&pxx, &o, fxx, gxx, nullptr, ws, inner, stream)) != FS_OK) return s;
+  if ((s = solve_impl(&pyy, &o, fyy, gyy, nullptr, ws, inner, stream)) != FS_OK) return s;
+  if ((s = fs_cost(p, fxy, gxy, costs, ws, inner, stream)) != FS_OK) return s;
+  if ((s = fs_cost(&pxx, fxx, gxx, costs + 1, ws, inner, stream)) != FS_OK) return s;
+  if ((s = fs_cost(&pyy, fyy, gyy, costs + 2, ws, inner, stream)) != FS_OK) return s;
+  divergence_finish_kernel<<<1, 32, 0, st>>>(costs, value);
+  if (cudaGetLastError() != cudaSuccess) return FS_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  // grad_x S = grad_x OT(x, y) - (the self problem's gradients from both sides) / 2
+  if (grad_x) {
+    if ((s = fs_grad_x(p, gxy, grad_x, ws, inner, stream)) != FS_OK) return s;
+    if ((s = fs_grad_x(&pxx, gxx, tmp1, ws, inner, stream)) != FS_OK) return s;
+    if ((s = fs_grad_x(&pxx, fxx, tmp2, ws, inner, stream)) != FS_OK) return s;
+    sub_half_sum_kernel<<<static_cast<unsigned>(ceil_div(n * d, 256)), 256, 0, st>>>(grad_x, tmp1,
+                                                                                     tmp2, n * d);
+    if (cudaGetLastError() != cudaSuccess) return FS_ERR_CUDA;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  if (grad_y) {
+    if ((s = fs_grad_x(&pyx, fxy, grad_y, ws, inner, stream)) != FS_OK) return s;
+    if ((s = fs_grad_x(&pyy, gyy, tmp1, ws, inner, stream)) != FS_OK) return s;
+    if ((s = fs_grad_x(&pyy, fyy, tmp2, ws, inner, stream)) != FS_OK) return s;
+    sub_half_sum_kernel<<<static_cast<unsigned>(ceil_div(m * d, 256)), 256, 0, st>>>(grad_y, tmp1,
+                                                                                     tmp2, m * d);
+    if (cudaGetLastError() != cudaSuccess) return FS_ERR_CUDA;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  return FS_OK;
+}
+
 size_t fs_transport_workspace_bytes(const fs_problem* p) {
   if (!fs::shape_ok(p) || p->d > 16) return 0;
   return fs::make_layout(p->n, p->m, p->d, fs::num_sms_current(), fs::kTransportChannels,

@@ -866,6 +866,18 @@ __global__ void __launch_bounds__(256) payload_keys_kernel(const float* keys, in
   for (int q = 2 * (D + 1 + NP) + e; q < K1; q += 2) dst[q] = 0.0f;
 }
 
+// Debiased divergence: S = c[0] - c[1]/2 - c[2]/2.
+__global__ void divergence_finish_kernel(const double* c, double* out) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) *out = c[0] - 0.5 * c[1] - 0.5 * c[2];
+}
+
+// grad -= (u + v) / 2 (the self problem's two one-sided gradients).
+__global__ void __launch_bounds__(256) sub_half_sum_kernel(float* grad, const float* u,
+                                                           const float* v, int64_t len) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < len) grad[i] -= 0.5f * (u[i] + v[i]);
+}
+
 // Cosine cost: x_i sqrt(1/2) / |x_i|, so that |x~_i - y~_j|^2 = 1 - cos(x_i, y_j). A zero
 // point gives non-finite coordinates, which the coordinate check then reports.
 __global__ void __launch_bounds__(256) normalize_kernel(const float* pts, int64_t count, int32_t d,

@@ -7,7 +7,7 @@ Only argument marshalling happens here: every number comes from the C ABI.
 """
 from __future__ import annotations
 
-from . import _torch, cost, grad_x, solve
+from . import _torch, cost, grad_x, sinkhorn_divergence, solve
 
 
 class _OTLoss:
@@ -15,6 +15,7 @@ class _OTLoss:
     does not import torch)."""
 
     fn = None
+    div = None
 
     @classmethod
     def get(cls):
@@ -50,7 +51,22 @@ class _OTLoss:
                                     ground_cost=ctx.ground_cost) * grad_out
                     return gx, gy, None, None, None, None, None
 
+            class DivergenceFunction(torch.autograd.Function):
+                @staticmethod
+                def forward(ctx, x, y, a, b, eps, ground_cost, options):
+                    value, gx, gy = sinkhorn_divergence(x.detach(), y.detach(), a, b, eps=eps,
+                                                        ground_cost=ground_cost, grads=True,
+                                                        **options)
+                    ctx.save_for_backward(gx, gy)
+                    return value.to(x.dtype)
+
+                @staticmethod
+                def backward(ctx, grad_out):
+                    gx, gy = ctx.saved_tensors
+                    return gx * grad_out, gy * grad_out, None, None, None, None, None
+
             cls.fn = OTLossFunction
+            cls.div = DivergenceFunction
         return cls.fn
 
 
@@ -59,7 +75,8 @@ class SamplesLoss:
 
     ``SamplesLoss(eps, n_iters=200, variant="alternating", alpha=0.5, stop_mode="fixed",
     stop_max_iter=20000, stop_tol=1e-6, stop_check_every=5, ground_cost="sqeuclidean")``
-    (or "cosine"); ``loss(x, y, a=None, b=None)``
+    (or "cosine"), ``debias=False`` (True: the debiased divergence
+    OT(a, b) - OT(a, a)/2 - OT(b, b)/2 and its gradients); ``loss(x, y, a=None, b=None)``
     returns OT_eps as a 0-d tensor (the dual objective <f,a> + <g,b> - eps (sum P - m_a m_b)
     at the solved potentials) with gradients for x and y; ``loss(x, y, potentials=True)``
     returns the potentials (f, g) in cost units instead. ``last_report`` holds the solve's
@@ -69,9 +86,10 @@ class SamplesLoss:
     def __init__(self, eps: float = 0.05, n_iters: int = 200, variant: str = "alternating",
                  alpha: float = 0.5, stop_mode: str = "fixed", stop_max_iter: int = 20000,
                  stop_tol: float = 1e-6, stop_check_every: int = 5,
-                 ground_cost: str = "sqeuclidean"):
+                 ground_cost: str = "sqeuclidean", debias: bool = False):
         self.eps = float(eps)
         self.ground_cost = ground_cost
+        self.debias = debias
         self.options = dict(n_iters=n_iters, variant=variant, alpha=alpha, stop_mode=stop_mode,
                             stop_max_iter=stop_max_iter, stop_tol=stop_tol,
                             stop_check_every=stop_check_every)
@@ -83,4 +101,6 @@ class SamplesLoss:
                                            ground_cost=self.ground_cost, **self.options)
             return f, g
         fn = _OTLoss.get()
+        if self.debias:
+            fn = _OTLoss.div
         return fn.apply(x, y, a, b, self.eps, self.ground_cost, self.options)

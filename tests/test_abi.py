@@ -206,3 +206,21 @@ def test_transport_and_hvp_argument_errors():
     assert hv(p, FAKE, FAKE, FAKE, ctypes.byref(bad_tol), None, FAKE, need, None) == "FS_ERR_OPTION"
     assert hv(p, FAKE, None, FAKE, None, None, FAKE, need, None) == "FS_ERR_NULL"
     assert hv(wide, FAKE, FAKE, FAKE, None, None, FAKE, BIG, None) == "FS_ERR_UNSUPPORTED_D"
+
+
+def test_divergence_argument_errors():
+    lib = _lib.load()
+    p = ctypes.byref(prob())
+    need = lib.fs_divergence_workspace_bytes(p)
+    assert need > lib.fs_workspace_bytes(p)
+    assert lib.fs_divergence_workspace_bytes(ctypes.byref(prob(d=65))) == 0
+    st = lambda c: _lib.STATUS[c]  # noqa: E731
+    o = _lib.fs_solve_options(5, 0, 0.5, 0, 100, 5, 1e-6, None)
+    assert st(lib.fs_divergence(p, None, FAKE, None, None, FAKE, need, None)) == "FS_ERR_NULL"
+    assert st(lib.fs_divergence(p, ctypes.byref(o), None, None, None, FAKE, need, None)) == "FS_ERR_NULL"
+    assert st(lib.fs_divergence(p, ctypes.byref(o), FAKE + 4, None, None, FAKE, need,
+                                None)) == "FS_ERR_ALIGNMENT"
+    assert st(lib.fs_divergence(p, ctypes.byref(o), FAKE, None, None, FAKE, need - 256,
+                                None)) == "FS_ERR_WORKSPACE"
+    assert st(lib.fs_divergence(ctypes.byref(prob(n=0)), ctypes.byref(o), FAKE, None, None, FAKE,
+                                need, None)) == "FS_ERR_SHAPE"

@@ -399,7 +399,7 @@ def test_solve_argument_errors():
 
 def converged(x, y, a, b, eps):
     f, g, it, conv, viol = oracle.solve(x, y, a, b, eps, stop_mode="marginal", stop_tol=1e-13,
-                                        stop_check_every=10, stop_max_iter=200000)
+                                        stop_check_every=10, stop_max_iter=20000)
     assert conv
     return f, g
 
@@ -519,7 +519,7 @@ def test_cosine_gradient_matches_finite_differences():
 
 # --- the debiased divergence ---------------------------------------------------------------
 
-CONV = dict(stop_mode="marginal", stop_tol=1e-13, stop_check_every=10, stop_max_iter=200000)
+CONV = dict(stop_mode="marginal", stop_tol=1e-13, stop_check_every=10, stop_max_iter=20000)
 
 
 @pytest.mark.parametrize("seed", [30, 31, 32])
