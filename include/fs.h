@@ -170,6 +170,41 @@ FS_API fs_status fs_solve(const fs_problem* p, const fs_solve_options* opt, floa
                           fs_stream_t stream);
 
 /*
+ * Coarse-to-fine solve (FlashSinkhorn 2 abstract, the coarse stage), squared-Euclidean cost
+ * and d <= 16 (FS_ERR_OPTION / FS_ERR_UNSUPPORTED_D otherwise). Each cloud is cut into cells
+ * of cell_points (1 to 256) points consecutive in its Morton order; a cell is its weighted
+ * centroid with its total mass. Rounds of coarse_iters alternating iterations run on the cell problem; after
+ * each round its potentials are lifted to every point of y (g_j = G(f_cells)(y_j), one pass
+ * of the fine y against the cells) and checked: one fine iteration from the lift and the
+ * marginal violation max(|P1 - a|_inf, |P^T 1 - b|_inf) after it. The lift is accepted when
+ * that violation is <= lift_tol, when a round shrank it by less than the factor lift_shrink,
+ * or after max_rounds rounds; otherwise the coarse iterations continue. The fine stage is
+ * then fs_solve with opt from the accepted lift (opt->g_init is ignored). Workspace:
+ * fs_multiscale_workspace_bytes(p, cell_points). report (host, may be NULL): rounds, coarse iterations,
+ * the accepted lift's violation and the fine solve's report.
+ */
+typedef struct {
+  int32_t cell_points;   /* points per cell, 1..256 */
+  int32_t coarse_iters;  /* coarse iterations per round, >= 1 */
+  int32_t max_rounds;    /* >= 1 */
+  double lift_tol;       /* >= 0 */
+  double lift_shrink;    /* in (0, 1] */
+} fs_multiscale_options;
+
+typedef struct {
+  int32_t rounds;
+  int32_t coarse_iters;
+  double lift_viol;
+  fs_solve_report fine;
+} fs_multiscale_report;
+
+FS_API size_t fs_multiscale_workspace_bytes(const fs_problem* p, int32_t cell_points);
+FS_API fs_status fs_solve_multiscale(const fs_problem* p, const fs_solve_options* opt,
+                                     const fs_multiscale_options* mo, float* f, float* g,
+                                     fs_multiscale_report* report, void* ws, size_t ws_bytes,
+                                     fs_stream_t stream);
+
+/*
  * Debiased (Sinkhorn) divergence S = OT(a, b) - OT(a, a)/2 - OT(b, b)/2 (the "divergence"
  * the pages' losses report): three fs_solve runs with the same options (g_init ignored) and
  * their dual objectives, value (device, one double) = S. grad_x (n x d) and grad_y (m x d),

@@ -20,7 +20,7 @@ from . import _lib
 __all__ = ["potentials", "cost", "grad_x", "marginal_residual", "solve_host", "workspace_bytes",
            "FsError", "timing_enable", "timing_reset", "timing_get", "launch_count",
            "screening_enable", "solve", "transport_apply", "hvp", "SamplesLoss",
-           "sinkhorn_divergence"]
+           "sinkhorn_divergence", "solve_multiscale"]
 
 
 class FsError(RuntimeError):
@@ -181,6 +181,43 @@ def solve(x, y, a=None, b=None, *, eps: float, ground_cost: str = "sqeuclidean",
     report = {"iters_run": int(rep.iters_run),
               "converged": None if rep.converged < 0 else bool(rep.converged),
               "final_viol": float(rep.final_viol)}
+    return f, g, report
+
+
+def solve_multiscale(x, y, a=None, b=None, *, eps: float, cell_points: int = 8,
+                     coarse_iters: int = 50,
+                     max_rounds: int = 8, lift_tol: float = 0.0, lift_shrink: float = 0.5,
+                     n_iters: int = 200, stop_mode: str = "fixed", stop_max_iter: int = 20000,
+                     stop_tol: float = 1e-6, stop_check_every: int = 5, variant: str = "alternating",
+                     alpha: float = 0.5, workspace=None):
+    """Coarse-to-fine solve (fs_solve_multiscale): rounds on Morton cells of ``cell_points``
+    consecutive points, lifts to
+    the fine y checked by one fine iteration, then fs_solve from the accepted lift.
+    Returns (f, g, report)."""
+    torch = _torch()
+    P = _Problem(x, y, a, b, eps)
+    f = torch.empty(P.n, dtype=torch.float32, device=P.device)
+    g = torch.empty(P.m, dtype=torch.float32, device=P.device)
+    opt = _lib.fs_solve_options(int(n_iters), _lib.VARIANTS[variant], float(alpha),
+                                _lib.STOP_MODES[stop_mode], int(stop_max_iter),
+                                int(stop_check_every), float(stop_tol), None)
+    mo = _lib.fs_multiscale_options(int(cell_points), int(coarse_iters), int(max_rounds),
+                                    float(lift_tol), float(lift_shrink))
+    rep = _lib.fs_multiscale_report()
+    if workspace is None:
+        nbytes = int(_lib.load().fs_multiscale_workspace_bytes(P.ref, int(cell_points)))
+        if nbytes == 0:
+            raise ValueError("the coarse-to-fine solve needs 1 <= d <= 16")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=P.device)
+    _raise(_lib.load().fs_solve_multiscale(P.ref, ctypes.byref(opt), ctypes.byref(mo),
+                                           f.data_ptr(), g.data_ptr(), ctypes.byref(rep),
+                                           workspace.data_ptr(), workspace.numel(), P.stream()))
+    fine = rep.fine
+    report = {"rounds": int(rep.rounds), "coarse_iters": int(rep.coarse_iters),
+              "lift_viol": float(rep.lift_viol),
+              "fine": {"iters_run": int(fine.iters_run),
+                       "converged": None if fine.converged < 0 else bool(fine.converged),
+                       "final_viol": float(fine.final_viol)}}
     return f, g, report
 
 

@@ -27,6 +27,7 @@ EXPORTS = (
     "fs_timing_enable", "fs_timing_reset", "fs_timing_get", "fs_launch_count",
     "fs_potentials_noalloc", "fs_screening_enable", "fs_solve", "fs_transport_workspace_bytes",
     "fs_transport_apply", "fs_hvp", "fs_divergence_workspace_bytes", "fs_divergence",
+    "fs_multiscale_workspace_bytes", "fs_solve_multiscale",
 )
 
 VARIANTS = {"alternating": 0, "symmetric": 1}
@@ -52,6 +53,17 @@ class fs_solve_options(ctypes.Structure):
 class fs_solve_report(ctypes.Structure):
     _fields_ = [("iters_run", ctypes.c_int32), ("converged", ctypes.c_int32),
                 ("final_viol", ctypes.c_double)]
+
+
+class fs_multiscale_options(ctypes.Structure):
+    _fields_ = [("cell_points", ctypes.c_int32), ("coarse_iters", ctypes.c_int32),
+                ("max_rounds", ctypes.c_int32), ("lift_tol", ctypes.c_double),
+                ("lift_shrink", ctypes.c_double)]
+
+
+class fs_multiscale_report(ctypes.Structure):
+    _fields_ = [("rounds", ctypes.c_int32), ("coarse_iters", ctypes.c_int32),
+                ("lift_viol", ctypes.c_double), ("fine", fs_solve_report)]
 
 
 class fs_hvp_options(ctypes.Structure):
@@ -108,6 +120,12 @@ def load():
     lib.fs_transport_apply.argtypes = [P, vp, vp, i32, i32, vp, vp, vp, sz, vp]
     lib.fs_hvp.argtypes = [P, vp, vp, vp, ctypes.POINTER(fs_hvp_options),
                            ctypes.POINTER(fs_hvp_report), vp, sz, vp]
+    lib.fs_multiscale_workspace_bytes.argtypes = [P, i32]
+    lib.fs_multiscale_workspace_bytes.restype = sz
+    lib.fs_solve_multiscale.argtypes = [P, ctypes.POINTER(fs_solve_options),
+                                        ctypes.POINTER(fs_multiscale_options), vp, vp,
+                                        ctypes.POINTER(fs_multiscale_report), vp, sz, vp]
+    lib.fs_solve_multiscale.restype = ctypes.c_int
     lib.fs_divergence_workspace_bytes.argtypes = [P]
     lib.fs_divergence_workspace_bytes.restype = sz
     lib.fs_divergence.argtypes = [P, ctypes.POINTER(fs_solve_options), vp, vp, vp, vp, sz, vp]

@@ -735,6 +735,18 @@ void launch_payload_keys_d(const float* keys, int64_t count, int64_t pairs, cons
 }
 
 template <int D>
+void launch_cells_d(const float* keys, int64_t count, int32_t d, const float* w, float wu,
+                    const int* perm, int cell_points, float* pts, float* mass, int64_t cells,
+                    cudaStream_t st) {
+  if constexpr (D <= 16) {
+    cell_kernel<D><<<static_cast<unsigned>(cells), 256, 0, st>>>(keys, count, d, w, wu, perm,
+                                                                 cell_points, pts, mass);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+}
+
+template <int D>
 void launch_apply_bias_d(float* keys, const float* defer_h, int64_t count, int* dmin,
                          cudaStream_t st) {
   apply_bias_kernel<D><<<static_cast<unsigned>(ceil_div(count, 256)), 256, 0, st>>>(keys, defer_h,
@@ -1773,6 +1785,142 @@ fs_status fs_divergence(const fs_problem* p, const fs_solve_options* opt, double
                                                                                      tmp2, m * d);
     if (cudaGetLastError() != cudaSuccess) return FS_ERR_CUDA;
     g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  return FS_OK;
+}
+
+namespace {
+// The coarse stage's problems: the cell clouds (cx, ca; cy, cb) and the lift problem, fine y
+// against the x cells; cells per cloud, and the tail of the workspace after the largest
+// inner workspace of the fine, cell and lift problems.
+struct Multiscale {
+  int64_t ncx, ncy;
+  fs_problem cells, lift;
+  size_t inner, tail;
+  float *cx, *cy, *ca, *cb, *fc, *gc, *gl, *tmp;
+};
+
+Multiscale multiscale_layout(const fs_problem* p, int cell_points, unsigned char* ws) {
+  Multiscale M{};
+  M.ncx = fs::ceil_div(p->n, cell_points);
+  M.ncy = fs::ceil_div(p->m, cell_points);
+  const int64_t d = p->d;
+  M.cells = *p;
+  M.cells.n = M.ncx;
+  M.cells.m = M.ncy;
+  M.lift = *p;  // rows: the fine y; keys: the x cells
+  M.lift.n = p->m;
+  M.lift.m = M.ncx;
+  M.inner = std::max({fs_workspace_bytes(p), fs_workspace_bytes(&M.cells), fs_workspace_bytes(&M.lift)});
+  size_t o = M.inner;
+  auto take = [&](int64_t floats) {
+    float* ptr = ws ? reinterpret_cast<float*>(ws + o) : nullptr;
+    o = fs::align_up(o + static_cast<size_t>(floats) * sizeof(float));
+    return ptr;
+  };
+  M.cx = take(M.ncx * d);
+  M.cy = take(M.ncy * d);
+  M.ca = take(M.ncx);
+  M.cb = take(M.ncy);
+  M.fc = take(M.ncx);
+  M.gc = take(M.ncy);
+  M.gl = take(p->m);
+  M.tmp = take(M.ncx);
+  M.tail = o - M.inner;
+  M.cells.x = M.cx;
+  M.cells.y = M.cy;
+  M.cells.a = M.ca;
+  M.cells.b = M.cb;
+  M.lift.x = p->y;
+  M.lift.y = M.cx;
+  M.lift.a = p->b;
+  M.lift.b = M.ca;
+  return M;
+}
+}  // namespace
+
+size_t fs_multiscale_workspace_bytes(const fs_problem* p, int32_t cell_points) {
+  if (!fs::shape_ok(p) || p->d > 16 || cell_points < 1 || cell_points > fs::kScreenTile) return 0;
+  const Multiscale M = multiscale_layout(p, cell_points, nullptr);
+  return M.inner + M.tail;
+}
+
+fs_status fs_solve_multiscale(const fs_problem* p, const fs_solve_options* opt,
+                              const fs_multiscale_options* mo, float* f, float* g,
+                              fs_multiscale_report* report, void* ws, size_t ws_bytes,
+                              fs_stream_t stream) {
+  using namespace fs;
+  if (!p || !opt || !mo || !f || !g) return FS_ERR_NULL;
+  if (!shape_ok(p)) return FS_ERR_SHAPE;
+  if (p->d > 16) return FS_ERR_UNSUPPORTED_D;
+  if (p->cost != FS_COST_SQEUCLIDEAN) return FS_ERR_OPTION;
+  fs_status s = check_options(*opt);
+  if (s != FS_OK) return s;
+  if (mo->coarse_iters < 1 || mo->max_rounds < 1 || !(mo->lift_tol >= 0.0) ||
+      !(mo->lift_shrink > 0.0 && mo->lift_shrink <= 1.0) || mo->cell_points < 1 ||
+      mo->cell_points > kScreenTile)
+    return FS_ERR_OPTION;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return FS_ERR_WORKSPACE;
+  const Multiscale M = multiscale_layout(p, mo->cell_points, static_cast<unsigned char*>(ws));
+  if (ws_bytes < M.inner + M.tail) return FS_ERR_WORKSPACE;
+  // cells of both clouds, from their Morton-sorted packed copies
+  {
+    Ctx c{};
+    s = begin(c, p, ws, M.inner, stream);
+    if (s != FS_OK) return s;
+    Timer timer(c.st);
+    c.timer = &timer;
+    s = guarded(c.st, [&]() -> fs_status {
+      const fs_status r = prepare_all(c, {}, false);
+      if (r != FS_OK) return r;
+      FS_DISPATCH_D(c.L.D, launch_cells_d, c.kx, p->n, p->d, p->a,
+                    static_cast<float>(1.0 / p->n), c.perm_x, mo->cell_points, M.cx, M.ca, M.ncx,
+                    c.st);
+      FS_DISPATCH_D(c.L.D, launch_cells_d, c.ky, p->m, p->d, p->b,
+                    static_cast<float>(1.0 / p->m), c.perm_y, mo->cell_points, M.cy, M.cb, M.ncy,
+                    c.st);
+      return finish(c);
+    });
+    if (s != FS_OK) return s;
+  }
+  // rounds on the cells, each followed by a lift and its check
+  fs_solve_options co{};
+  co.n_iters = mo->coarse_iters;
+  co.variant = FS_VARIANT_ALTERNATING;
+  co.stop_mode = FS_STOP_FIXED;
+  fs_solve_options chk{};
+  chk.variant = FS_VARIANT_ALTERNATING;
+  chk.stop_mode = FS_STOP_MARGINAL;
+  chk.stop_max_iter = 1;
+  chk.stop_check_every = 1;
+  chk.stop_tol = 0.0;
+  chk.g_init = M.gl;
+  int32_t rounds = 0;
+  double viol = NAN, prev = NAN;
+  for (int32_t r = 1; r <= mo->max_rounds; ++r) {
+    co.g_init = r == 1 ? nullptr : M.gc;  // continue from the last round
+    if ((s = solve_impl(&M.cells, &co, M.fc, M.gc, nullptr, ws, M.inner, stream)) != FS_OK) return s;
+    // lift: g_j = G(f_cells)(y_j), the f-update of the problem (y, x cells) from f_cells
+    if ((s = potentials_impl(&M.lift, 1, M.fc, M.gl, M.tmp, ws, M.inner, stream)) != FS_OK)
+      return s;
+    fs_solve_report cr{};
+    if ((s = solve_impl(p, &chk, f, g, &cr, ws, M.inner, stream)) != FS_OK) return s;
+    rounds = r;
+    viol = cr.final_viol;
+    const bool shrank_little = r > 1 && !(viol < mo->lift_shrink * prev);
+    if (viol <= mo->lift_tol || shrank_little) break;
+    prev = viol;
+  }
+  // the fine stage from the accepted lift
+  fs_solve_options fo = *opt;
+  fo.g_init = M.gl;
+  fs_solve_report fr{};
+  if ((s = solve_impl(p, &fo, f, g, &fr, ws, M.inner, stream)) != FS_OK) return s;
+  if (report) {
+    report->rounds = rounds;
+    report->coarse_iters = rounds * mo->coarse_iters;
+    report->lift_viol = viol;
+    report->fine = fr;
   }
   return FS_OK;
 }

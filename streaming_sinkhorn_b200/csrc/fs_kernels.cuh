@@ -866,6 +866,62 @@ __global__ void __launch_bounds__(256) payload_keys_kernel(const float* keys, in
   for (int q = 2 * (D + 1 + NP) + e; q < K1; q += 2) dst[q] = 0.0f;
 }
 
+// Coarse stage: one cell per `cell_points` consecutive points of a sorted cloud (consecutive
+// in Morton order, so spatially compact; cell_points <= 256): its mass sum_j w_j and its
+// weighted centroid. One CTA per cell. A cell without mass takes the plain mean of its
+// points (it then carries no weight).
+template <int D>
+__global__ void __launch_bounds__(256) cell_kernel(const float* keys, int64_t count, int32_t d_real,
+                                                   const float* w, float w_uniform,
+                                                   const int* perm, int cell_points,
+                                                   float* cell_pts, float* cell_mass) {
+  __shared__ double red[8][D + 2];
+  __shared__ double pred[8][D];
+  const int64_t c = blockIdx.x;
+  const int64_t j = c * cell_points + threadIdx.x;
+  const bool mine = static_cast<int>(threadIdx.x) < cell_points && j < count;
+  double acc[D + 2];
+#pragma unroll
+  for (int k = 0; k < D + 2; ++k) acc[k] = 0.0;
+  if (mine) {
+    const int64_t oi = perm ? perm[j] : j;
+    const double wj = w ? static_cast<double>(w[oi]) : static_cast<double>(w_uniform);
+#pragma unroll
+    for (int k = 0; k < D; ++k) acc[k] = wj * static_cast<double>(keys[key_slot<D>(j, k)]);
+    acc[D] = wj;
+    acc[D + 1] = 1.0;
+  }
+  double plain[D];
+#pragma unroll
+  for (int k = 0; k < D; ++k) plain[k] = mine ? static_cast<double>(keys[key_slot<D>(j, k)]) : 0.0;
+#pragma unroll
+  for (int k = 0; k < D + 2; ++k) acc[k] = warp_sum(acc[k]);
+#pragma unroll
+  for (int k = 0; k < D; ++k) plain[k] = warp_sum(plain[k]);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (lane == 0) {
+#pragma unroll
+    for (int k = 0; k < D + 2; ++k) red[wid][k] = acc[k];
+#pragma unroll
+    for (int k = 0; k < D; ++k) pred[wid][k] = plain[k];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t[D + 2], q[D];
+    for (int k = 0; k < D + 2; ++k) t[k] = 0.0;
+    for (int k = 0; k < D; ++k) q[k] = 0.0;
+    for (int r = 0; r < 8; ++r) {
+      for (int k = 0; k < D + 2; ++k) t[k] += red[r][k];
+      for (int k = 0; k < D; ++k) q[k] += pred[r][k];
+    }
+    const double mass = t[D], pts = t[D + 1];
+    for (int k = 0; k < d_real; ++k)
+      cell_pts[c * d_real + k] =
+          static_cast<float>(mass > 0.0 ? t[k] / mass : (pts > 0.0 ? q[k] / pts : 0.0));
+    cell_mass[c] = static_cast<float>(mass);
+  }
+}
+
 // Debiased divergence: S = c[0] - c[1]/2 - c[2]/2.
 __global__ void divergence_finish_kernel(const double* c, double* out) {
   if (threadIdx.x == 0 && blockIdx.x == 0) *out = c[0] - 0.5 * c[1] - 0.5 * c[2];

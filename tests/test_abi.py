@@ -224,3 +224,28 @@ def test_divergence_argument_errors():
                                 None)) == "FS_ERR_WORKSPACE"
     assert st(lib.fs_divergence(ctypes.byref(prob(n=0)), ctypes.byref(o), FAKE, None, None, FAKE,
                                 need, None)) == "FS_ERR_SHAPE"
+
+
+def test_multiscale_argument_errors():
+    lib = _lib.load()
+    p = ctypes.byref(prob())
+    need = lib.fs_multiscale_workspace_bytes(p, 32)
+    assert need > lib.fs_workspace_bytes(p)
+    assert lib.fs_multiscale_workspace_bytes(ctypes.byref(prob(d=17)), 32) == 0
+    assert lib.fs_multiscale_workspace_bytes(p, 0) == 0
+    assert lib.fs_multiscale_workspace_bytes(p, 257) == 0
+    st = lambda c: _lib.STATUS[c]  # noqa: E731
+    o = _lib.fs_solve_options(5, 0, 0.5, 0, 100, 5, 1e-6, None)
+    call = lambda mo, ws=need: st(lib.fs_solve_multiscale(  # noqa: E731
+        p, ctypes.byref(o), ctypes.byref(mo), FAKE, FAKE, None, FAKE, ws, None))
+    assert call(_lib.fs_multiscale_options(32, 0, 4, 0.0, 0.5)) == "FS_ERR_OPTION"
+    assert call(_lib.fs_multiscale_options(32, 5, 0, 0.0, 0.5)) == "FS_ERR_OPTION"
+    assert call(_lib.fs_multiscale_options(32, 5, 4, -1.0, 0.5)) == "FS_ERR_OPTION"
+    assert call(_lib.fs_multiscale_options(32, 5, 4, 0.0, 0.0)) == "FS_ERR_OPTION"
+    assert call(_lib.fs_multiscale_options(0, 5, 4, 0.0, 0.5)) == "FS_ERR_OPTION"
+    assert call(_lib.fs_multiscale_options(300, 5, 4, 0.0, 0.5)) == "FS_ERR_OPTION"
+    assert call(_lib.fs_multiscale_options(32, 5, 4, 0.0, 0.5), need - 256) == "FS_ERR_WORKSPACE"
+    cos = _lib.fs_problem(FAKE, FAKE + 4096, None, None, 10, 12, 3, 0.1, 1)
+    assert st(lib.fs_solve_multiscale(ctypes.byref(cos), ctypes.byref(o),
+                                      ctypes.byref(_lib.fs_multiscale_options(32, 5, 4, 0.0, 0.5)),
+                                      FAKE, FAKE, None, FAKE, BIG, None)) == "FS_ERR_OPTION"
