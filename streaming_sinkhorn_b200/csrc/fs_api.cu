@@ -338,7 +338,7 @@ struct Layout {
   size_t off_perm_x, off_perm_y, off_sortkeys, off_box_x, off_box_y, off_hmax_x, off_hmax_y,
       off_lse_x, off_lse_y;
   // queue mode: kept-tile masks, kept counts, unit starts and unit -> row block
-  size_t off_kmask, off_kcount, off_ustart, off_unit_rb, off_rmlb;
+  size_t off_kmask, off_kcount, off_ustart, off_unit_rb, off_unit_j, off_rmlb;
   // general solve: deferred biases of x (symmetric schedule), potentials at the last check
   size_t off_defer, off_fprev, off_gprev;
   // transport products and the Hessian-vector product (layouts asked with acc_ch > 0):
@@ -456,6 +456,8 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0, bool co
     L.off_ustart = o;
     o = align_up(o + static_cast<size_t>(rb_max + 1) * sizeof(int));
     L.off_unit_rb = o;
+    o = align_up(o + static_cast<size_t>(units_max) * sizeof(int));
+    L.off_unit_j = o;
     o = align_up(o + static_cast<size_t>(units_max) * sizeof(int));
     L.off_rmlb = o;
     o = align_up(o + static_cast<size_t>(std::max(n, m)) * sizeof(float));
@@ -842,7 +844,7 @@ struct Ctx {
   uint64_t* sortkeys;
   float *box_x, *box_y, *hmax_x, *hmax_y, *lse_x, *lse_y;
   unsigned* kmask;
-  int *kcount, *ustart, *unit_rb;
+  int *kcount, *ustart, *unit_rb, *unit_j;
   float* rmlb;     // per-row lower bounds written by the screening kernel
   float *defer, *fprev, *gprev;
   float* paykeys; // transport passes: keys with payload channels
@@ -915,6 +917,7 @@ void carve(Ctx& c, void* ws) {
     c.kcount = reinterpret_cast<int*>(c.ws + c.L.off_kcount);
     c.ustart = reinterpret_cast<int*>(c.ws + c.L.off_ustart);
     c.unit_rb = reinterpret_cast<int*>(c.ws + c.L.off_unit_rb);
+    c.unit_j = reinterpret_cast<int*>(c.ws + c.L.off_unit_j);
     c.rmlb = reinterpret_cast<float*>(c.ws + c.L.off_rmlb);
   }
 }
@@ -1261,12 +1264,13 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
     P.kcount = c.kcount;
     P.unit_start = c.ustart;
     P.unit_rb = c.unit_rb;
+    P.unit_j = c.unit_j;
     P.qscal = reinterpret_cast<const int*>(c.scal + kQueue);
     P.row_mlb = c.rmlb;
     int ti = c.timer->begin();
     FS_DISPATCH_D(c.L.D, launch_screen_d, P, q.rb, c.kmask, c.kcount, c.st);
     plan_units_kernel<<<1, 1024, 0, c.st>>>(c.kcount, static_cast<int>(q.rb), q.budget, q.RB,
-                                            c.ustart, c.unit_rb,
+                                            c.ustart, c.unit_rb, c.unit_j,
                                             reinterpret_cast<int*>(c.scal + kQueue),
                                             reinterpret_cast<long long*>(c.scal + kKept),
                                             nullptr);

@@ -114,7 +114,8 @@ struct PassParams {
   int32_t rb_rows;          // rows of a row block (R * NT of the pass)
   const int* kcount;        // [row block] kept tiles
   const int* unit_start;    // [row block + 1] first unit of each row block
-  const int* unit_rb;       // [unit] row block of each unit
+  const int* unit_rb;       // [unit] row block of each unit (launch order)
+  const int* unit_j;        // [unit] its index among its row block's units
   const int* qscal;         // [0] tiles per unit C, [1] number of units U
   float* row_mlb;           // [row]: lower bound on each row's largest exponent (screening)
   // symmetric (Jacobi) schedule: blend weight (0: plain update) and, for the pass whose
@@ -294,13 +295,15 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
   const float* key_src;
   const unsigned* mrow = nullptr;
   if (queue) {
-    unit = blockIdx.x;
-    if (unit >= P.qscal[1]) return;  // past the plan's unit count
-    const int b = P.unit_rb[unit];
+    if (static_cast<int>(blockIdx.x) >= P.qscal[1]) return;  // past the plan's unit count
+    // unit blockIdx.x is the j-th unit of row block b; its partials go to slot first + j
+    const int b = P.unit_rb[blockIdx.x];
+    const int j = P.unit_j[blockIdx.x];
     const int first = P.unit_start[b];
     n_units = P.unit_start[b + 1] - first;
+    unit = first + j;
     const int C = P.qscal[0];
-    const int k0 = static_cast<int>(unit - first) * C;
+    const int k0 = j * C;
     n_work = min(C, P.kcount[b] - k0);
     row0 = static_cast<int64_t>(b) * RB;
     key_src = P.tile_keys ? P.tile_keys : P.keys;

@@ -210,16 +210,20 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
   if (lane == 0) kcount[b] = cnt;
 }
 
-// One CTA of 1024 threads: C = max(1, ceil(K / budget)) for K kept tiles in all, the units
-// of each row block (ceil(kept / C)), their prefix, the row block of every unit, K itself
-// and the evaluated-pair count (kept tiles x 256 keys x rows per block).
+// One CTA of 1024 threads: C = max(1, ceil(K / budget)) for K kept tiles in all; each row
+// block's kept tiles in units of C (floor(kept / C) full units and one shorter tail unit when
+// C does not divide kept); the prefix of units per block (partial slots and unit counts for
+// the merge); and the launch order: every full unit first, in block order, then the tails,
+// so that the last CTAs the hardware schedules are the shortest ones. Also K itself and the
+// evaluated-pair count (kept tiles x 256 keys x rows per block).
 __global__ void __launch_bounds__(1024) plan_units_kernel(const int* kcount, int rb,
                                                           long long budget, int rb_rows,
                                                           int* unit_start, int* unit_rb,
-                                                          int* qscal, long long* kept_out,
+                                                          int* unit_j, int* qscal,
+                                                          long long* kept_out,
                                                           unsigned long long* evaluated) {
   __shared__ long long s_part[32];
-  __shared__ int s_scan[32];
+  __shared__ int s_scan[3][32];
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   // thread t owns row blocks [t * per, (t + 1) * per)
   const int per = (rb + 1023) / 1024;
@@ -233,28 +237,57 @@ __global__ void __launch_bounds__(1024) plan_units_kernel(const int* kcount, int
   __syncthreads();
   long long total = 0;
   for (int q = 0; q < 32; ++q) total += s_part[q];
-  const long long C = total > budget ? (total + budget - 1) / budget : 1;
-  int nu = 0;
-  for (int b = b0; b < b1; ++b) nu += static_cast<int>((kcount[b] + C - 1) / C);
-  int incl = nu;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) s_scan[wid] = incl;
-  __syncthreads();
-  int start = incl - nu;
-  for (int q = 0; q < wid; ++q) start += s_scan[q];
+  const int C = static_cast<int>(total > budget ? (total + budget - 1) / budget : 1);
+  // per thread: units, full units and tail units of its blocks
+  int v[3] = {0, 0, 0};
   for (int b = b0; b < b1; ++b) {
-    const int n = static_cast<int>((kcount[b] + C - 1) / C);
+    const int kc = kcount[b];
+    v[1] += kc / C;
+    v[2] += kc % C ? 1 : 0;
+  }
+  v[0] = v[1] + v[2];
+  int incl[3], excl[3], all[3];
+#pragma unroll
+  for (int q = 0; q < 3; ++q) {
+    incl[q] = v[q];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl[q], o);
+      if (lane >= o) incl[q] += t;
+    }
+    if (lane == 31) s_scan[q][wid] = incl[q];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 3; ++q) {
+    int wbase = 0;
+    all[q] = 0;
+    for (int w = 0; w < 32; ++w) {
+      if (w < wid) wbase += s_scan[q][w];
+      all[q] += s_scan[q][w];
+    }
+    excl[q] = wbase + incl[q] - v[q];
+  }
+  int start = excl[0], full = excl[1], tail = all[1] + excl[2];
+  for (int b = b0; b < b1; ++b) {
+    const int kc = kcount[b];
+    const int nf = kc / C;
     unit_start[b] = start;
-    for (int j = 0; j < n; ++j) unit_rb[start + j] = b;
-    start += n;
+    start += nf + (kc % C ? 1 : 0);
+    for (int j = 0; j < nf; ++j) {
+      unit_rb[full + j] = b;
+      unit_j[full + j] = j;
+    }
+    full += nf;
+    if (kc % C) {
+      unit_rb[tail] = b;
+      unit_j[tail] = nf;
+      ++tail;
+    }
   }
   if (tid == 1023) {
     unit_start[rb] = start;
-    qscal[0] = static_cast<int>(C);
+    qscal[0] = C;
     qscal[1] = start;
     *kept_out = total;
     if (evaluated)
