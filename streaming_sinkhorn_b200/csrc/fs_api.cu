@@ -228,7 +228,11 @@ int64_t partial_floats(const Plan& p, int D, bool grad) {
 // unit plan of fs_screen.cuh. The kept-tile masks take one bit per (row block, key tile),
 // capped at kMaskCapWords words; larger problems run unscreened in split mode.
 constexpr int64_t kMaskCapWords = int64_t(64) << 20;  // 256 MiB
-constexpr int kUnitWaves = 8;  // unit budget, in waves of resident CTAs
+// Unit budget: up to kUnitWaves waves of resident CTAs (many short units balance the SMs),
+// but at most kUnitsPerBlock per row block, which keeps the partials' memory in proportion
+// to the problem (4 x the rows' own (2 + channels) floats).
+constexpr int kUnitWaves = 32;
+constexpr int kUnitsPerBlock = 4;
 
 struct QPlan {
   bool on;
@@ -251,7 +255,7 @@ QPlan make_qplan(const Plan& pl, int64_t key_pairs, int D, bool grad, int sms, b
   const int64_t slots = static_cast<int64_t>(sms) *
                         occupancy_for(D, grad, kQueueVariant,
                                       pass_smem_bytes(D, kScreenTile / 2, kQueueStages));
-  q.budget = kUnitWaves * slots;
+  q.budget = std::max<int64_t>(1, std::min<int64_t>(kUnitWaves * slots, kUnitsPerBlock * q.rb));
   q.units_max = q.budget + q.rb;
   return q;
 }

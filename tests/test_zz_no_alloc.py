@@ -58,3 +58,13 @@ def test_noalloc_matches_workspace_entry_point():
         assert np.isfinite(f.cpu().numpy()).all() and np.isfinite(g.cpu().numpy()).all()
         assert_potential_close(f.cpu().numpy(), f_ref, "f")
         assert_potential_close(g.cpu().numpy(), g_ref, "g")
+
+
+@pytest.mark.gpu
+def test_documented_size_fits_the_static_scratch():
+    """The header promises that every d = 3 problem with n, m <= 80000 fits; the workspace
+    depends on the device's occupancy, so this is checked on the GPU."""
+    lib = _lib.load()
+    for n, m in ((80000, 80000), (80000, 1), (1, 80000), (65536, 80000)):
+        p = _lib.fs_problem(FAKE, FAKE, None, None, n, m, 3, 0.1)
+        assert lib.fs_workspace_bytes(ctypes.byref(p)) <= 16 << 20, (n, m)
