@@ -250,8 +250,11 @@ FS_API fs_status fs_transport_apply(const fs_problem* p, const float* f, const f
  * marginal constraints. The system (positive semi-definite, singular along the gauge
  * direction (1, -1)) is solved by conjugate gradients on the device, two transport passes
  * and one host read-back per iteration. opt may be NULL (cg_max_iter 200, cg_tol 1e-6, a
- * relative residual); report (host, may be NULL) receives the iterations run and the final
- * relative residual.
+ * relative residual). The iteration runs in fp32 and returns the iterate with the smallest
+ * residual it has seen; it also stops after 50 iterations without a new smallest residual
+ * (a tolerance below fp32 rounding is never reached, and past that point the recurrence
+ * only drifts). report (host, may be NULL) receives the iterations run and the relative
+ * residual of the returned iterate.
  */
 typedef struct {
   int32_t cg_max_iter;  /* >= 1 */

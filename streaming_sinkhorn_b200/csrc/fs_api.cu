@@ -358,9 +358,9 @@ constexpr int kTransportChannels = 16;  // payload channels of one transport pas
 // Floats of the HVP's vectors, in the order hvp_impl carves them: ft and a spare row vector
 // (2n); the solution, residual, direction, product and transport output over n + m (5);
 // the gradient, the difference sums and 2v (3 n d); the column pass's payload (n (d + 2))
-// and output (m (d + 2)); the column sums (m).
+// and output (m (d + 2)); the column sums (m); the best solution so far (n + m).
 inline int64_t hvp_floats(int64_t n, int64_t m, int d) {
-  return 2 * n + 5 * (n + m) + 3 * n * d + (n + m) * (d + 2) + m + 64;
+  return 2 * n + 6 * (n + m) + 3 * n * d + (n + m) * (d + 2) + m + 64;
 }
 
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
@@ -523,7 +523,8 @@ struct PassKernel {
   static void screen(const PassParams& P, int64_t rb, unsigned* kmask, int* kcount,
                      cudaStream_t st) {
     if constexpr (D <= 16 && NT == 32) {  // one warp per row block, FMA-path widths only
-      screen_kernel<D, R><<<static_cast<unsigned>(rb), 32, 0, st>>>(P, kmask, kcount);
+      const size_t smem = P.key_supers <= kSupCache ? P.key_supers * sizeof(float) : 0;
+      screen_kernel<D, R><<<static_cast<unsigned>(rb), 32, smem, st>>>(P, kmask, kcount);
       CK(cudaGetLastError());
       g_launches.fetch_add(1, std::memory_order_relaxed);
     }
@@ -1557,7 +1558,8 @@ fs_status hvp_impl(const fs_problem* p, const float* g, const float* v, float* o
     float* v2 = diffsum + n * d;
     float* colpay = v2 + n * d;        // (n, d + 2)
     float* coldata = colpay + n * (d + 2);  // (m, d + 2)
-    float* csum = coldata + m * (d + 2);      // ends at hvp_floats(n, m, d) - 64
+    float* csum = coldata + m * (d + 2);      // (m)
+    float* zbest = csum + m;                  // (n + m), ends at hvp_floats(n, m, d) - 64
     double* dots = c.scal + kCgDots;
     const unsigned blk = static_cast<unsigned>(ceil_div(nm, 256));
     const float a_uni = static_cast<float>(1.0 / n);
@@ -1594,6 +1596,11 @@ fs_status hvp_impl(const fs_problem* p, const float* g, const float* v, float* o
     const double bb = h[2];
     double rr = bb;
     int32_t it = 0;
+    // the iterate with the smallest residual so far (z = 0 to begin with)
+    constexpr int32_t kCgPatience = 50;
+    double best = bb;
+    int32_t best_it = 0;
+    CK(cudaMemsetAsync(zbest, 0, nm * sizeof(float), c.st));
     while (it < max_iter && rr > tol * tol * bb && rr > 0.0) {
       transport_pass(c, true, nullptr, dir + n, 1, 1, prod, 1);      // P w
       transport_pass(c, false, g, dir, 1, 1, prod + n, 1);           // P^T u
@@ -1616,20 +1623,27 @@ fs_status hvp_impl(const fs_problem* p, const float* g, const float* v, float* o
       launched(1);
       rr = rr_new;
       ++it;
+      if (rr < best) {
+        best = rr;
+        best_it = it;
+        CK(cudaMemcpyAsync(zbest, zu, nm * sizeof(float), cudaMemcpyDeviceToDevice, c.st));
+      } else if (it - best_it >= kCgPatience) {
+        break;
+      }
     }
     // 4. the difference pass with payload dg and row vectors 2 v, then the combination
     scale_kernel<<<static_cast<unsigned>(ceil_div(n * d, 256)), 256, 0, c.st>>>(v, n * d, 2.0f, v2);
     CK(cudaGetLastError());
     launched(1);
-    transport_pass(c, true, nullptr, zu + n, 1, 1, diffsum, d, v2);
+    transport_pass(c, true, nullptr, zbest + n, 1, 1, diffsum, d, v2);
     hvp_final_kernel<<<static_cast<unsigned>(ceil_div(n * d, 256)), 256, 0, c.st>>>(
-        v, p->a, a_uni, zu, grad, diffsum, n, d, 2.0 / static_cast<double>(p->eps), out);
+        v, p->a, a_uni, zbest, grad, diffsum, n, d, 2.0 / static_cast<double>(p->eps), out);
     CK(cudaGetLastError());
     launched(1);
     r = finish(c);
     if (report) {
       report->cg_iters = it;
-      report->cg_rel_residual = bb > 0.0 ? std::sqrt(rr / bb) : 0.0;
+      report->cg_rel_residual = bb > 0.0 ? std::sqrt(best / bb) : 0.0;
     }
     return r;
   });

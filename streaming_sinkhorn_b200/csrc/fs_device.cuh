@@ -57,6 +57,11 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Asks L2 to fetch the line holding p (no register result, nothing waits for it).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));

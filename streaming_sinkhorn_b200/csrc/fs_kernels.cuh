@@ -252,6 +252,69 @@ __device__ __forceinline__ void block_reduce_marg(double dev_sum, double dev_max
   }
 }
 
+// Second-level LSE of row i over its ns partials (slots s0 .. s0 + ns - 1, row offset off
+// within a slot of `stride` rows), then the row's completion. The partials are read
+// kMergeChunk at a time, all loads of a chunk issued before any is used, so that a row
+// costs one memory round trip per chunk rather than one per partial. A partial whose
+// columns were all zero-weight or padding left m = -inf and sum 0 and drops out.
+constexpr int kMergeChunk = 8;
+template <int D, int MODE, int NA>
+__device__ __forceinline__ void merge_row(const PassParams& P, int64_t i, int64_t s0, int64_t ns,
+                                          int64_t stride, int64_t off, double& dev_sum,
+                                          double& dev_max, double& mass, float& dmin) {
+  constexpr bool GRAD = MODE == kModeGrad;
+  constexpr bool ACC = MODE != kModeLse;
+  float mx = -INFINITY;
+  double l = 0.0;
+  float a[NA];
+#pragma unroll
+  for (int k = 0; k < NA; ++k) a[k] = 0.0f;
+  for (int64_t c0 = s0; c0 < s0 + ns; c0 += kMergeChunk) {
+    float pm[kMergeChunk], pl[kMergeChunk];
+#pragma unroll
+    for (int u = 0; u < kMergeChunk; ++u) {
+      const bool ok = c0 + u < s0 + ns;
+      const int64_t o = (c0 + u) * stride + off;
+      pm[u] = ok ? P.part_m[o] : -INFINITY;
+      pl[u] = ok ? P.part_l[o] : 0.0f;
+    }
+    float cm = mx;
+#pragma unroll
+    for (int u = 0; u < kMergeChunk; ++u) cm = fmaxf(cm, pm[u]);
+    if (cm == -INFINITY) continue;
+    if (cm > mx) {  // rescale what was merged so far to the new maximum
+      const float sc = ex2(mx - cm);
+      l *= sc;
+#pragma unroll
+      for (int k = 0; k < NA; ++k) a[k] *= sc;
+      mx = cm;
+    }
+#pragma unroll
+    for (int u = 0; u < kMergeChunk; ++u) {
+      const float w = pm[u] == -INFINITY ? 0.0f : ex2(pm[u] - mx);
+      l += static_cast<double>(pl[u]) * w;
+      if (ACC && c0 + u < s0 + ns) {
+#pragma unroll
+        for (int k = 0; k < NA; ++k) a[k] += P.part_a[((c0 + u) * NA + k) * stride + off] * w;
+      }
+    }
+  }
+  const double lse2 = static_cast<double>(mx) + log2(l);
+  if (GRAD) {
+    finish_grad(P, i, a, static_cast<float>(l));
+  } else if (ACC) {
+    finish_acc(P, i, a, l, lse2);
+  } else if (P.kind == kPot) {
+    dmin = fminf(dmin, finish_pot<D>(P, i, lse2));
+  } else {
+    double dv, ms;
+    finish_marg(P, i, lse2, dv, ms);
+    dev_sum += dv;
+    dev_max = fmax(dev_max, dv);
+    mass += ms;
+  }
+}
+
 // ---- the fused streaming pass -------------------------------------------------------------
 
 // Loads the packed components of key pair p of a shared-memory tile.
@@ -698,51 +761,32 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
 
 // Second-level LSE over the partials of each row, then the row completion. Split mode: the
 // n_splits partials at [split][rows_pad]. Queue mode: the units of the row's block at
-// [unit][rb_rows]; a block with one unit was completed by the pass itself. A partial whose
-// columns were all zero-weight or padding left m = -inf and sum 0 and drops out.
+// [unit][rb_rows]; a block with one unit was completed by the pass itself. The loads the
+// row's completion will need are sent to L2 first, so they overlap the partials' loads.
 template <int D, int MODE, int NA>
 __global__ void __launch_bounds__(256) combine_kernel(const PassParams P) {
-  constexpr bool GRAD = MODE == kModeGrad;
   constexpr bool ACC = MODE != kModeLse;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  double dev = 0.0, mass = 0.0;
+  double dev_sum = 0.0, dev_max = 0.0, mass = 0.0;
   float dmin = INFINITY;
-  int64_t s0 = 0, ns = P.n_splits, stride = P.rows_pad, off = i;
-  if (P.kmask && i < P.n_rows) {
-    const int64_t b = i / P.rb_rows;
-    s0 = P.unit_start[b];
-    ns = P.unit_start[b + 1] - s0;
-    stride = P.rb_rows;
-    off = i - b * P.rb_rows;
-  }
-  if (i < P.n_rows && (ns > 1 || !P.kmask)) {
-    float mx = -INFINITY;
-    for (int64_t s = s0; s < s0 + ns; ++s) mx = fmaxf(mx, P.part_m[s * stride + off]);
-    double l = 0.0;
-    float a[NA];
-    for (int k = 0; k < NA; ++k) a[k] = 0.0f;
-    for (int64_t s = s0; s < s0 + ns; ++s) {
-      const int64_t o = s * stride + off;
-      const float pm = P.part_m[o];
-      if (pm == -INFINITY) continue;
-      const float w = ex2(pm - mx);
-      l += static_cast<double>(P.part_l[o]) * w;
-      if (ACC) {
-        for (int k = 0; k < NA; ++k) a[k] += P.part_a[(s * NA + k) * stride + off] * w;
-      }
+  if (i < P.n_rows) {
+    if (P.perm) prefetch_l2(P.perm + i);
+    if (!ACC && P.kind == kPot) {
+      prefetch_l2(P.lw + i);
+      if (!P.hy_out && !P.defer_h) prefetch_l2(P.qkeys + key_slot<D>(i, D));
     }
-    const double lse2 = static_cast<double>(mx) + log2(l);
-    if (GRAD) {
-      finish_grad(P, i, a, static_cast<float>(l));
-    } else if (ACC) {
-      finish_acc(P, i, a, l, lse2);
-    } else if (P.kind == kPot) {
-      dmin = finish_pot<D>(P, i, lse2);
-    } else {
-      finish_marg(P, i, lse2, dev, mass);
+    int64_t s0 = 0, ns = P.n_splits, stride = P.rows_pad, off = i;
+    if (P.kmask) {
+      const int64_t b = i / P.rb_rows;
+      s0 = P.unit_start[b];
+      ns = P.unit_start[b + 1] - s0;
+      stride = P.rb_rows;
+      off = i - b * P.rb_rows;
     }
+    if (ns > 1 || !P.kmask)
+      merge_row<D, MODE, NA>(P, i, s0, ns, stride, off, dev_sum, dev_max, mass, dmin);
   }
-  if (!ACC && P.kind == kMarg) block_reduce_marg(dev, dev, mass, P.acc);
+  if (!ACC && P.kind == kMarg) block_reduce_marg(dev_sum, dev_max, mass, P.acc);
   if (!ACC && P.kind == kPot) reduce_dmin(dmin, P.dmin_out);
 }
 

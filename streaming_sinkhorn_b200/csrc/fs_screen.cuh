@@ -29,6 +29,10 @@
 
 namespace fs {
 
+// Super-tile bounds a screening warp keeps in shared memory (4 KiB); beyond this many
+// super-tiles (2^21 keys) it recomputes them where they are used.
+constexpr int kSupCache = 1024;
+
 // One warp (one CTA) per row block of 32 R rows: the bit mask of kept key tiles and its
 // population count. Tiles are tested through their super-tiles first: a super-tile's box
 // contains its tiles' boxes and its bias maximum bounds theirs, so its upper bound bounds
@@ -40,6 +44,7 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
   constexpr int RB = R * 32;
   constexpr int TP = kScreenTile / 2;  // key pairs per tile
   __shared__ __align__(16) float anchor_tile[TP * KP];
+  extern __shared__ float s_sub[];  // kSupCache bounds at most (dynamic size)
   const int lane = threadIdx.x;
   const int64_t b = blockIdx.x;
   const int64_t row0 = b * RB;
@@ -99,16 +104,27 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
     return key;
   };
 
+  // Super-tile bounds, kept in shared memory when they fit (every lane reads back only the
+  // entries it wrote, so no barrier is needed); otherwise recomputed where used.
+  const bool cached = S <= kSupCache;
+  auto sub_ub = [&](int sidx) -> float {
+    return cached ? s_sub[sidx] : ub_of(P.key_sbox, P.key_shmax, S, sidx);
+  };
+
   // anchor: the tile with the largest upper bound (ties to the lower index), found through
   // the super-tiles: the best tile of the best super-tile gives a bound L, and only
   // super-tiles whose own bound exceeds L can hold a better tile.
-  unsigned long long best = 0ull;
-  for (int s0 = 0; s0 < S; s0 += 32) {
-    const int sidx = s0 + lane;
-    const unsigned long long k = best_of(sidx < S ? ub_of(P.key_sbox, P.key_shmax, S, sidx) : 0.0f,
-                                         sidx, sidx < S);
-    best = best > k ? best : k;
+  float bub = -INFINITY;
+  int bidx = -1;
+  for (int sidx = lane; sidx < S; sidx += 32) {
+    const float u = ub_of(P.key_sbox, P.key_shmax, S, sidx);
+    if (cached) s_sub[sidx] = u;
+    if (bidx < 0 || u > bub) {  // a lane's indices rise, so ties keep the lower one
+      bub = u;
+      bidx = sidx;
+    }
   }
+  unsigned long long best = best_of(bub, bidx, bidx >= 0);
   const int sstar = static_cast<int>(0xFFFFFFFFu - static_cast<unsigned>(best & 0xFFFFFFFFull));
   {
     const int t = sstar * kSuper + lane;
@@ -118,8 +134,8 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
   for (int s0 = 0; s0 < S; s0 += 32) {
     const int sidx = s0 + lane;
     const float lbest = ord_float(static_cast<int>(static_cast<unsigned>(best >> 32) ^ 0x80000000u));
-    unsigned sbits = __ballot_sync(
-        0xffffffffu, sidx < S && sidx != sstar && ub_of(P.key_sbox, P.key_shmax, S, sidx) >= lbest);
+    unsigned sbits =
+        __ballot_sync(0xffffffffu, sidx < S && sidx != sstar && sub_ub(sidx) >= lbest);
     while (sbits) {
       const int sl = __ffs(sbits) - 1;
       sbits &= sbits - 1u;
@@ -131,20 +147,49 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
   }
   const int anchor = static_cast<int>(0xFFFFFFFFu - static_cast<unsigned>(best & 0xFFFFFFFFull));
 
-  // the anchor's keys, then each row's largest exponent over them (packed, direct form)
-  {
-    const float4* src = reinterpret_cast<const float4*>(P.keys + static_cast<int64_t>(anchor) * TP * KP);
-    float4* dst = reinterpret_cast<float4*>(anchor_tile);
-    for (int q = lane; q < TP * KP / 4; q += 32) dst[q] = src[q];
-  }
-  __syncwarp();
-  u64 xp[R][D];
+  // The anchor's keys about the block's centre c (y' = y - c, H' = H - kappa |y'|^2), then
+  // each row's largest exponent over them: z = H' - kappa |x'|^2 + 2 kappa x'.y' (packed).
+  u64 cpk[D];
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-#pragma unroll
-    for (int k = 0; k < D; ++k) xp[r][k] = pk(x[r][k], x[r][k]);
+  for (int k = 0; k < D; ++k) {
+    const float c = lo[k] <= hi[k] ? 0.5f * (lo[k] + hi[k]) : 0.0f;
+    cpk[k] = pk(c, c);
   }
   const u64 nkappa = pk(-P.kappa_f, -P.kappa_f);
+  {
+    const float* src = P.keys + static_cast<int64_t>(anchor) * TP * KP;
+    for (int p = lane; p < TP; p += 32) {
+      u64 comp[KP / 2];
+      load_pair<KP>(src, p, comp);
+      u64 s2 = pk(0.0f, 0.0f);
+#pragma unroll
+      for (int k = 0; k < D; ++k) {
+        comp[k] = sub2(comp[k], cpk[k]);
+        s2 = fma2(comp[k], comp[k], s2);
+      }
+      comp[D] = fma2(nkappa, s2, comp[D]);
+      ulonglong2* pv = reinterpret_cast<ulonglong2*>(anchor_tile + p * KP);
+#pragma unroll
+      for (int v = 0; v < KP / 4; ++v) pv[v] = make_ulonglong2(comp[2 * v], comp[2 * v + 1]);
+    }
+  }
+  __syncwarp();
+  u64 xp[R][D], mk[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    float s2 = 0.0f;
+#pragma unroll
+    for (int k = 0; k < D; ++k) {
+      float cc, cd;
+      upk(cpk[k], cc, cd);
+      const float xs = x[r][k] - cc;
+      s2 = fmaf(xs, xs, s2);
+      const float x2 = 2.0f * P.kappa_f * xs;
+      xp[r][k] = pk(x2, x2);
+    }
+    const float q = -P.kappa_f * s2;
+    mk[r] = pk(q, q);
+  }
   float zmax[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) zmax[r] = -INFINITY;
@@ -154,14 +199,11 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
     load_pair<KP>(anchor_tile, p, comp);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      u64 acc = pk(0.0f, 0.0f);
+      u64 acc = add2(comp[D], mk[r]);
 #pragma unroll
-      for (int k = 0; k < D; ++k) {
-        const u64 dk = sub2(xp[r][k], comp[k]);
-        acc = fma2(dk, dk, acc);
-      }
+      for (int k = 0; k < D; ++k) acc = fma2(xp[r][k], comp[k], acc);
       float z0, z1;
-      upk(fma2(nkappa, acc, comp[D]), z0, z1);
+      upk(acc, z0, z1);
       zmax[r] = max3(zmax[r], z0, z1);
     }
   }
@@ -186,8 +228,7 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
   int cnt = 0;
   for (int s0 = 0; s0 < S; s0 += 32) {
     const int sidx = s0 + lane;
-    const bool keep_s =
-        sidx < S && (sidx == anchor / kSuper || ub_of(P.key_sbox, P.key_shmax, S, sidx) >= thr);
+    const bool keep_s = sidx < S && (sidx == anchor / kSuper || sub_ub(sidx) >= thr);
     unsigned sbits = __ballot_sync(0xffffffffu, keep_s);
     unsigned word = 0u;
     while (sbits) {
@@ -222,73 +263,93 @@ __global__ void __launch_bounds__(1024) plan_units_kernel(const int* kcount, int
                                                           int* unit_j, int* qscal,
                                                           long long* kept_out,
                                                           unsigned long long* evaluated) {
-  __shared__ long long s_part[32];
-  __shared__ int s_scan[3][32];
+  __shared__ long long s_kept[32];
+  __shared__ int s_cnt[3][32];
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  // thread t owns row blocks [t * per, (t + 1) * per)
-  const int per = (rb + 1023) / 1024;
-  const int b0 = min(rb, tid * per), b1 = min(rb, b0 + per);
+  // warp w owns the run of row blocks [w0, w1), read 32 consecutive blocks at a time
+  const int per_w = (rb + 31) / 32;
+  const int w0 = min(rb, wid * per_w), w1 = min(rb, w0 + per_w);
   long long k = 0;
-  for (int b = b0; b < b1; ++b) k += kcount[b];
-  long long kw = k;
+#pragma unroll 4
+  for (int b = w0 + lane; b < w1; b += 32) k += kcount[b];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) kw += __shfl_xor_sync(0xffffffffu, kw, o);
-  if (lane == 0) s_part[wid] = kw;
+  for (int o = 16; o > 0; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+  if (lane == 0) s_kept[wid] = k;
   __syncthreads();
   long long total = 0;
-  for (int q = 0; q < 32; ++q) total += s_part[q];
+  for (int q = 0; q < 32; ++q) total += s_kept[q];
   const int C = static_cast<int>(total > budget ? (total + budget - 1) / budget : 1);
-  // per thread: units, full units and tail units of its blocks
+  // per warp: units, full units and tail units of its run
   int v[3] = {0, 0, 0};
-  for (int b = b0; b < b1; ++b) {
-    const int kc = kcount[b];
-    v[1] += kc / C;
-    v[2] += kc % C ? 1 : 0;
-  }
-  v[0] = v[1] + v[2];
-  int incl[3], excl[3], all[3];
-#pragma unroll
-  for (int q = 0; q < 3; ++q) {
-    incl[q] = v[q];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl[q], o);
-      if (lane >= o) incl[q] += t;
-    }
-    if (lane == 31) s_scan[q][wid] = incl[q];
-  }
-  __syncthreads();
-#pragma unroll
-  for (int q = 0; q < 3; ++q) {
-    int wbase = 0;
-    all[q] = 0;
-    for (int w = 0; w < 32; ++w) {
-      if (w < wid) wbase += s_scan[q][w];
-      all[q] += s_scan[q][w];
-    }
-    excl[q] = wbase + incl[q] - v[q];
-  }
-  int start = excl[0], full = excl[1], tail = all[1] + excl[2];
-  for (int b = b0; b < b1; ++b) {
+#pragma unroll 4
+  for (int b = w0 + lane; b < w1; b += 32) {
     const int kc = kcount[b];
     const int nf = kc / C;
-    unit_start[b] = start;
-    start += nf + (kc % C ? 1 : 0);
-    for (int j = 0; j < nf; ++j) {
-      unit_rb[full + j] = b;
-      unit_j[full + j] = j;
-    }
-    full += nf;
-    if (kc % C) {
-      unit_rb[tail] = b;
-      unit_j[tail] = nf;
-      ++tail;
-    }
+    v[1] += nf;
+    v[2] += kc - nf * C ? 1 : 0;
   }
-  if (tid == 1023) {
-    unit_start[rb] = start;
+  v[0] = v[1] + v[2];
+#pragma unroll
+  for (int q = 0; q < 3; ++q) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v[q] += __shfl_xor_sync(0xffffffffu, v[q], o);
+    if (lane == 0) s_cnt[q][wid] = v[q];
+  }
+  __syncthreads();
+  // exclusive prefix of the warps' counts (lane l holds warp l's) and the totals
+  int base[3], all[3];
+#pragma unroll
+  for (int q = 0; q < 3; ++q) {
+    const int own = s_cnt[q][lane];
+    int incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    base[q] = __shfl_sync(0xffffffffu, incl - own, wid);
+    all[q] = __shfl_sync(0xffffffffu, incl, 31);
+  }
+  // the run's units in rounds of 32 blocks: a scan within the round gives each block its
+  // first unit (merge order), its full units' slots and its tail's slot (launch order)
+  int start = base[0], full = base[1], tail = all[1] + base[2];
+  for (int r0 = w0; r0 < w1; r0 += 32) {
+    const int b = r0 + lane;
+    const int kc = b < w1 ? kcount[b] : 0;
+    const int nf = kc / C;
+    const int tl = kc - nf * C ? 1 : 0;
+    int iu = nf + tl, ifl = nf, itl = tl;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, iu, o);
+      const int f = __shfl_up_sync(0xffffffffu, ifl, o);
+      const int t = __shfl_up_sync(0xffffffffu, itl, o);
+      if (lane >= o) {
+        iu += a;
+        ifl += f;
+        itl += t;
+      }
+    }
+    if (b < w1) {
+      unit_start[b] = start + iu - (nf + tl);
+      const int f0 = full + ifl - nf;
+      for (int j = 0; j < nf; ++j) {
+        unit_rb[f0 + j] = b;
+        unit_j[f0 + j] = j;
+      }
+      if (tl) {
+        unit_rb[tail + itl - 1] = b;
+        unit_j[tail + itl - 1] = nf;
+      }
+    }
+    start += __shfl_sync(0xffffffffu, iu, 31);
+    full += __shfl_sync(0xffffffffu, ifl, 31);
+    tail += __shfl_sync(0xffffffffu, itl, 31);
+  }
+  if (tid == 0) {
+    unit_start[rb] = all[0];
     qscal[0] = C;
-    qscal[1] = start;
+    qscal[1] = all[0];
     *kept_out = total;
     if (evaluated)
       atomicAdd(evaluated, static_cast<unsigned long long>(total) * kScreenTile * rb_rows);
