@@ -379,8 +379,8 @@ FS_API int64_t fs_launch_count(void);
 /*
  * Block screening, on by default (point clouds with d <= 16, which the library puts in a
  * spatial order). A pass skips a 256-point key tile when a bound shows that each of its
- * terms is below 2^-(32 + log2 M) times the largest term of every row it meets, so that
- * the omitted part of each row's sum is below 2^-32 of the sum (FlashSinkhorn 2 abstract,
+ * terms is below 2^-(24 + log2 M) times the largest term of every row it meets, so that
+ * the omitted part of each row's sum is below 2^-24 of the sum (FlashSinkhorn 2 abstract,
  * block-sparse screening, here with a provable bound). fs_screening_enable(0) makes every
  * later call evaluate all N x M pairs; the results agree to fp32 rounding either way.
  * Process-wide; takes effect at the next call.

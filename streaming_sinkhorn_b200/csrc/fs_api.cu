@@ -159,9 +159,6 @@ size_t pass_smem_bytes(int D, int tile_pairs, int stages = kStages, int np = 0) 
 // how many payload channels its key tiles carry.
 enum PassSel : int { kSelLse = 0, kSelGrad = 1, kSelPay1 = 2, kSelPay4 = 3, kSelPay16 = 4,
                      kSelDiff = 5 };
-inline int sel_channels(int sel) {
-  return sel == kSelPay1 ? 1 : sel == kSelPay4 ? 4 : sel == kSelPay16 ? 16 : sel == kSelDiff ? 1 : 0;
-}
 
 int occupancy_for(int D, bool grad, int variant, size_t smem);  // defined after the kernels
 
@@ -339,7 +336,7 @@ struct Layout {
   // maxima, and the LSE2 of every row in its last pass
   bool sorted;
   int64_t sort_n;  // keys of the bitonic sort (power of two, >= kSortSmem)
-  size_t off_perm_x, off_perm_y, off_sortkeys, off_box_x, off_box_y, off_hmax_x, off_hmax_y,
+  size_t off_perm_x, off_perm_y, off_code_x, off_code_y, off_sortkeys, off_box_x, off_box_y, off_hmax_x, off_hmax_y,
       off_lse_x, off_lse_y;
   // queue mode: kept-tile masks, kept counts, unit starts and unit -> row block
   size_t off_kmask, off_kcount, off_ustart, off_unit_rb, off_unit_j, off_rmlb;
@@ -437,6 +434,10 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0, bool co
     o = align_up(o + static_cast<size_t>(n) * sizeof(int));
     L.off_perm_y = o;
     o = align_up(o + static_cast<size_t>(m) * sizeof(int));
+    L.off_code_x = o;
+    o = align_up(o + static_cast<size_t>(n) * sizeof(unsigned));
+    L.off_code_y = o;
+    o = align_up(o + static_cast<size_t>(m) * sizeof(unsigned));
     L.off_sortkeys = o;
     o = align_up(o + static_cast<size_t>(sn) * sizeof(uint64_t));
     // tile summaries followed by their super-tile summaries
@@ -798,7 +799,7 @@ void launch_tile_hmax_d(const float* keys, int64_t count, int64_t tiles, float* 
 
 // Morton order of one cloud: keys (code << 32 | index), bitonic sort, permutation.
 void sort_cloud(const float* pts, int64_t count, int d, const MortonFrame& F, uint64_t* keys,
-                int64_t sort_n, int* perm, cudaStream_t st) {
+                int64_t sort_n, int* perm, unsigned* codes, cudaStream_t st) {
   morton_keys_kernel<<<static_cast<unsigned>(ceil_div(sort_n, 256)), 256, 0, st>>>(
       pts, count, d, F, keys, sort_n);
   CK(cudaGetLastError());
@@ -819,7 +820,7 @@ void sort_cloud(const float* pts, int64_t count, int d, const MortonFrame& F, ui
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
   perm_from_keys_kernel<<<static_cast<unsigned>(ceil_div(count, 256)), 256, 0, st>>>(keys, count,
-                                                                                      perm);
+                                                                                      perm, codes);
   CK(cudaGetLastError());
   g_launches.fetch_add(1, std::memory_order_relaxed);
 }
@@ -846,6 +847,7 @@ struct Ctx {
   float *nrm_x, *nrm_y, *hy_x, *hy_y;
   float c2;       // 2 kappa / s^2
   int *perm_x, *perm_y;         // sorted slot -> original index (NULL when unsorted)
+  unsigned *code_x, *code_y;    // Morton codes in sorted order (NULL when unsorted)
   uint64_t* sortkeys;
   float *box_x, *box_y, *hmax_x, *hmax_y, *lse_x, *lse_y;
   unsigned* kmask;
@@ -911,6 +913,8 @@ void carve(Ctx& c, void* ws) {
   if (c.L.sorted) {
     c.perm_x = reinterpret_cast<int*>(c.ws + c.L.off_perm_x);
     c.perm_y = reinterpret_cast<int*>(c.ws + c.L.off_perm_y);
+    c.code_x = reinterpret_cast<unsigned*>(c.ws + c.L.off_code_x);
+    c.code_y = reinterpret_cast<unsigned*>(c.ws + c.L.off_code_y);
     c.sortkeys = reinterpret_cast<uint64_t*>(c.ws + c.L.off_sortkeys);
     c.box_x = reinterpret_cast<float*>(c.ws + c.L.off_box_x);
     c.box_y = reinterpret_cast<float*>(c.ws + c.L.off_box_y);
@@ -1033,8 +1037,8 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
       F.scale[k] = hi > lo ? static_cast<float>(((1u << F.bits) - 1u) / (static_cast<double>(hi) - lo))
                            : 0.0f;
     }
-    sort_cloud(p->x, p->n, p->d, F, c.sortkeys, c.L.sort_n, c.perm_x, c.st);
-    sort_cloud(p->y, p->m, p->d, F, c.sortkeys, c.L.sort_n, c.perm_y, c.st);
+    sort_cloud(p->x, p->n, p->d, F, c.sortkeys, c.L.sort_n, c.perm_x, c.code_x, c.st);
+    sort_cloud(p->y, p->m, p->d, F, c.sortkeys, c.L.sort_n, c.perm_y, c.code_y, c.st);
   }
   const float wu_x = static_cast<float>(1.0 / p->n), wu_y = static_cast<float>(1.0 / p->m);
   FS_DISPATCH_D(c.L.D, launch_pack_d, p->x, p->n, p->d, p->a, wu_x, c.perm_x, c.kx, c.lwx, c.L.px,
@@ -1272,6 +1276,9 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
     P.unit_j = c.unit_j;
     P.qscal = reinterpret_cast<const int*>(c.scal + kQueue);
     P.row_mlb = c.rmlb;
+    P.key_codes = rows_x ? c.code_y : c.code_x;
+    P.row_codes = rows_x ? c.code_x : c.code_y;
+    P.key_count = n_keys;
     int ti = c.timer->begin();
     FS_DISPATCH_D(c.L.D, launch_screen_d, P, q.rb, c.kmask, c.kcount, c.st);
     plan_units_kernel<<<1, 1024, 0, c.st>>>(c.kcount, static_cast<int>(q.rb), q.budget, q.RB,

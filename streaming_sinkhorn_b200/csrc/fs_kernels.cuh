@@ -118,6 +118,9 @@ struct PassParams {
   const int* unit_j;        // [unit] its index among its row block's units
   const int* qscal;         // [0] tiles per unit C, [1] number of units U
   float* row_mlb;           // [row]: lower bound on each row's largest exponent (screening)
+  const unsigned* key_codes; // Morton codes of the key cloud in sorted order (key_count)
+  const unsigned* row_codes; // Morton codes of the query cloud in sorted order
+  int64_t key_count;         // real keys
   // symmetric (Jacobi) schedule: blend weight (0: plain update) and, for the pass whose
   // biases the other pass of the same iteration must not see yet, where to leave them
   float alpha;
@@ -132,8 +135,9 @@ struct PassParams {
 
 constexpr int kScreenTile = 256;  // points per screening tile (= kPairPad pairs)
 // Relative size, in log2 units, below which the omitted part of a row's sum is kept: the
-// skip margin is kSkipBits + log2(number of keys) (the tolerance of the screening).
-constexpr float kSkipBits = 32.0f;
+// skip margin is kSkipBits + log2(number of keys) (the tolerance of the screening). 24 bits
+// is the fp32 unit roundoff: the omitted mass is at most one rounding of the row's sum.
+constexpr float kSkipBits = 24.0f;
 
 // Offset of coordinate slot k (k == D is the bias H) of point i in packed keys.
 template <int D>

@@ -14,7 +14,8 @@
 // A tile with ub(T) < min_i mlb_i - margin is skipped. Each of its terms is below
 // 2^-margin times its row's largest term, so with margin = kSkipBits + log2(m) the whole
 // omitted part of a row's sum is below 2^-kSkipBits of that sum (the largest term is at
-// most the sum). With kSkipBits = 32 this is under the rounding of the fp32 sums. The
+// most the sum). With kSkipBits = 24, the fp32 unit roundoff, the omitted mass is at most
+// one rounding of the row's sum (the fp32 accumulation itself errs by more). The
 // anchor is always kept, so every row block has work.
 //
 // The plan. The kept tiles of a row block are cut into units of at most C tiles, with C
@@ -32,6 +33,9 @@ namespace fs {
 // Super-tile bounds a screening warp keeps in shared memory (4 KiB); beyond this many
 // super-tiles (2^21 keys) it recomputes them where they are used.
 constexpr int kSupCache = 1024;
+// Key tiles from the block's stretch of the Morton order that the screen evaluates besides
+// the anchor.
+constexpr int kMortonAnchors = 4;
 
 // One warp (one CTA) per row block of 32 R rows: the bit mask of kept key tiles and its
 // population count. Tiles are tested through their super-tiles first: a super-tile's box
@@ -147,8 +151,9 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
   }
   const int anchor = static_cast<int>(0xFFFFFFFFu - static_cast<unsigned>(best & 0xFFFFFFFFull));
 
-  // The anchor's keys about the block's centre c (y' = y - c, H' = H - kappa |y'|^2), then
-  // each row's largest exponent over them: z = H' - kappa |x'|^2 + 2 kappa x'.y' (packed).
+  // Each row's largest exponent over the keys of a few tiles is a value the row reaches.
+  // A tile's keys are taken about the block's centre c (y' = y - c, H' = H - kappa |y'|^2):
+  // z = H' - kappa |x'|^2 + 2 kappa x'.y' (packed).
   u64 cpk[D];
 #pragma unroll
   for (int k = 0; k < D; ++k) {
@@ -156,24 +161,6 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
     cpk[k] = pk(c, c);
   }
   const u64 nkappa = pk(-P.kappa_f, -P.kappa_f);
-  {
-    const float* src = P.keys + static_cast<int64_t>(anchor) * TP * KP;
-    for (int p = lane; p < TP; p += 32) {
-      u64 comp[KP / 2];
-      load_pair<KP>(src, p, comp);
-      u64 s2 = pk(0.0f, 0.0f);
-#pragma unroll
-      for (int k = 0; k < D; ++k) {
-        comp[k] = sub2(comp[k], cpk[k]);
-        s2 = fma2(comp[k], comp[k], s2);
-      }
-      comp[D] = fma2(nkappa, s2, comp[D]);
-      ulonglong2* pv = reinterpret_cast<ulonglong2*>(anchor_tile + p * KP);
-#pragma unroll
-      for (int v = 0; v < KP / 4; ++v) pv[v] = make_ulonglong2(comp[2 * v], comp[2 * v + 1]);
-    }
-  }
-  __syncwarp();
   u64 xp[R][D], mk[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
@@ -193,18 +180,74 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
   float zmax[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) zmax[r] = -INFINITY;
+  auto eval_tile = [&](int t) {
+    __syncwarp();  // every lane is done with the previous tile
+    const float* src = P.keys + static_cast<int64_t>(t) * TP * KP;
+    for (int p = lane; p < TP; p += 32) {
+      u64 comp[KP / 2];
+      load_pair<KP>(src, p, comp);
+      u64 s2 = pk(0.0f, 0.0f);
+#pragma unroll
+      for (int k = 0; k < D; ++k) {
+        comp[k] = sub2(comp[k], cpk[k]);
+        s2 = fma2(comp[k], comp[k], s2);
+      }
+      comp[D] = fma2(nkappa, s2, comp[D]);
+      ulonglong2* pv = reinterpret_cast<ulonglong2*>(anchor_tile + p * KP);
+#pragma unroll
+      for (int v = 0; v < KP / 4; ++v) pv[v] = make_ulonglong2(comp[2 * v], comp[2 * v + 1]);
+    }
+    __syncwarp();
 #pragma unroll 4
-  for (int p = 0; p < TP; ++p) {
-    u64 comp[KP / 2];
-    load_pair<KP>(anchor_tile, p, comp);
+    for (int p = 0; p < TP; ++p) {
+      u64 comp[KP / 2];
+      load_pair<KP>(anchor_tile, p, comp);
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      u64 acc = add2(comp[D], mk[r]);
+      for (int r = 0; r < R; ++r) {
+        u64 acc = add2(comp[D], mk[r]);
 #pragma unroll
-      for (int k = 0; k < D; ++k) acc = fma2(xp[r][k], comp[k], acc);
-      float z0, z1;
-      upk(acc, z0, z1);
-      zmax[r] = max3(zmax[r], z0, z1);
+        for (int k = 0; k < D; ++k) acc = fma2(xp[r][k], comp[k], acc);
+        float z0, z1;
+        upk(acc, z0, z1);
+        zmax[r] = max3(zmax[r], z0, z1);
+      }
+    }
+  };
+  eval_tile(anchor);
+
+  // Morton anchors: the key tiles that hold the block's stretch of the shared space-filling
+  // order (the keys whose codes lie between the block's first and last row codes, and one
+  // key on either side). They hold most rows' nearest keys even where the anchor, chosen
+  // for the block's box as a whole, is far from some of its rows; at most kMortonAnchors
+  // of them, spread over the stretch.
+  if (P.key_codes) {
+    const int64_t nk = P.key_count;
+    // first position in the sorted key codes whose code is >= target (warp-wide search)
+    auto lower_bound = [&](uint64_t target) -> int64_t {
+      int64_t lo_p = 0, hi_p = nk;
+      while (hi_p - lo_p > 32) {
+        const int64_t q = lo_p + (static_cast<int64_t>(lane) + 1) * (hi_p - lo_p) / 33;
+        const unsigned below = __ballot_sync(0xffffffffu, P.key_codes[q] < target);
+        const int c = __popc(below);
+        const int64_t nlo = c == 0 ? lo_p : __shfl_sync(0xffffffffu, q, c - 1) + 1;
+        const int64_t nhi = c == 32 ? hi_p : __shfl_sync(0xffffffffu, q, c & 31);
+        lo_p = nlo;
+        hi_p = nhi;
+      }
+      const int64_t q = lo_p + lane;
+      return lo_p + __popc(__ballot_sync(0xffffffffu, q < hi_p && P.key_codes[q] < target));
+    };
+    const int64_t last = (row0 + RB < P.n_rows ? row0 + RB : P.n_rows) - 1;
+    const int64_t p0 = lower_bound(P.row_codes[row0]);
+    const int64_t p1 = lower_bound(static_cast<uint64_t>(P.row_codes[last]) + 1u);
+    const int64_t q0 = p0 > 0 ? p0 - 1 : 0;
+    const int64_t q1 = p1 < nk - 1 ? p1 : nk - 1;
+    const int t0 = static_cast<int>(q0 / kScreenTile), t1 = static_cast<int>(q1 / kScreenTile);
+    const int span = t1 - t0 + 1;
+    const int na = span < kMortonAnchors ? span : kMortonAnchors;
+    for (int e = 0; e < na; ++e) {
+      const int t = na == span ? t0 + e : t0 + static_cast<int>(static_cast<int64_t>(e) * (span - 1) / (na - 1));
+      if (t != anchor) eval_tile(t);
     }
   }
   const bool history = P.lse_prev && P.key_dmin;

@@ -143,10 +143,14 @@ __global__ void __launch_bounds__(256) bitonic_global_kernel(uint64_t* keys, int
   }
 }
 
+// The permutation (original index of each sorted position) and the sorted Morton codes.
 __global__ void __launch_bounds__(256) perm_from_keys_kernel(const uint64_t* keys, int64_t count,
-                                                             int* perm) {
+                                                             int* perm, unsigned* codes) {
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (j < count) perm[j] = static_cast<int>(keys[j] & 0xFFFFFFFFull);
+  if (j >= count) return;
+  const uint64_t k = keys[j];
+  perm[j] = static_cast<int>(k & 0xFFFFFFFFull);
+  codes[j] = static_cast<unsigned>(k >> 32);
 }
 
 // Bounding box (all D coordinates) of each 256-point tile of a packed cloud, stored by

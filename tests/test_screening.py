@@ -1,7 +1,7 @@
 """Block screening on the GPU: a clustered problem solved with screening on and off gives
 the same potentials, gradient and marginals to fp32 rounding, and the screened run
 evaluates far fewer pairs. Screening drops only tiles whose terms are all below
-2^-(32 + log2 M) of their rows' largest term, so any larger difference is a bug in the
+2^-(24 + log2 M) of their rows' largest term, so any larger difference is a bug in the
 bound, the kept-tile masks, the unit plan or the merge of a row block's units."""
 import numpy as np
 import pytest

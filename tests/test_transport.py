@@ -93,6 +93,9 @@ def test_hvp_is_symmetric_on_the_gpu():
 
 
 def test_hvp_screened_equals_dense():
+    """Screened and unscreened transport passes differ by fp32 rounding (at eps = 2e-4 the
+    fp32 potentials alone fix each plan entry to ~1e-4); conjugate gradients stopped early
+    amplify that, so both solves run until they stagnate at the same residual level."""
     w = workloads.clustered_cube(n=16384, seed=31, n_iters=10, eps=2e-4)
     x, y, a, b = inputs(w)
     f, g = fs.potentials(x, y, a, b, eps=w.eps, n_iters=10)
@@ -101,8 +104,9 @@ def test_hvp_screened_equals_dense():
     for screening in (False, True):
         fs.screening_enable(screening)
         try:
-            hv, rep = fs.hvp(x, y, g, v, a, b, eps=w.eps, cg_max_iter=60, cg_tol=1e-6)
+            hv, rep = fs.hvp(x, y, g, v, a, b, eps=w.eps, cg_max_iter=1000, cg_tol=1e-5)
         finally:
             fs.screening_enable(True)
         out[screening] = (hv.cpu().numpy(), rep)
+    assert out[True][1]["cg_rel_residual"] < 2e-3 and out[False][1]["cg_rel_residual"] < 2e-3
     close(out[True][0], out[False][0], 5e-3)
