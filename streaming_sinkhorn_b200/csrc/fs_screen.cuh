@@ -6,8 +6,11 @@
 // with bounding box B and a key tile T with box B_T and largest bias Hmax_T,
 //   z_ij <= Hmax_T - kappa dist(B, B_T)^2 =: ub(T)          for all i in the block, j in T.
 // A lower bound mlb_i on each row's largest exponent max_j z_ij comes from
-//   (a) an anchor tile: max over the anchor's keys of the computed z_ij is a value the row
-//       reaches (the anchor is the tile with the largest ub);
+//   (a) anchor tiles: the max over an anchor's keys of the computed z_ij is a value the row
+//       reaches. The anchors are the key tiles that hold the row block's stretch of the
+//       Morton order both clouds share (the keys whose codes lie between the block's first
+//       and last row codes, and one key on either side): they hold most rows' nearest keys,
+//       so the bound is close to each row's true maximum, at most kMortonAnchors of them;
 //   (b) history (potential passes after the first two): the largest term of a sum of m terms
 //       is at least the sum over m, and every bias moved by at least dmin since the row's
 //       previous pass, so max_j z_ij >= LSE2_prev_i + dmin - log2(m).
@@ -15,7 +18,7 @@
 // 2^-margin times its row's largest term, so with margin = kSkipBits + log2(m) the whole
 // omitted part of a row's sum is below 2^-kSkipBits of that sum (the largest term is at
 // most the sum). With kSkipBits = 24, the fp32 unit roundoff, the omitted mass is at most
-// one rounding of the row's sum (the fp32 accumulation itself errs by more). The
+// one rounding of the row's sum (the fp32 accumulation itself errs by more). The first
 // anchor is always kept, so every row block has work.
 //
 // The plan. The kept tiles of a row block are cut into units of at most C tiles, with C
@@ -33,8 +36,7 @@ namespace fs {
 // Super-tile bounds a screening warp keeps in shared memory (4 KiB); beyond this many
 // super-tiles (2^21 keys) it recomputes them where they are used.
 constexpr int kSupCache = 1024;
-// Key tiles from the block's stretch of the Morton order that the screen evaluates besides
-// the anchor.
+// Anchor tiles a screening warp evaluates at most (spread over the block's Morton stretch).
 constexpr int kMortonAnchors = 4;
 
 // One warp (one CTA) per row block of 32 R rows: the bit mask of kept key tiles and its
@@ -94,20 +96,6 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
     }
     return hm[idx] - P.kappa_f * d2;
   };
-  // warp argmax of (ub, -index): key = ordered ub << 32 | ~index
-  auto best_of = [&](float ub, int idx, bool ok) -> unsigned long long {
-    unsigned long long key =
-        ok ? (static_cast<unsigned long long>(static_cast<unsigned>(float_ord(ub)) ^ 0x80000000u) << 32) |
-                 static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<unsigned>(idx))
-           : 0ull;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
-      key = key > other ? key : other;
-    }
-    return key;
-  };
-
   // Super-tile bounds, kept in shared memory when they fit (every lane reads back only the
   // entries it wrote, so no barrier is needed); otherwise recomputed where used.
   const bool cached = S <= kSupCache;
@@ -115,41 +103,8 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
     return cached ? s_sub[sidx] : ub_of(P.key_sbox, P.key_shmax, S, sidx);
   };
 
-  // anchor: the tile with the largest upper bound (ties to the lower index), found through
-  // the super-tiles: the best tile of the best super-tile gives a bound L, and only
-  // super-tiles whose own bound exceeds L can hold a better tile.
-  float bub = -INFINITY;
-  int bidx = -1;
-  for (int sidx = lane; sidx < S; sidx += 32) {
-    const float u = ub_of(P.key_sbox, P.key_shmax, S, sidx);
-    if (cached) s_sub[sidx] = u;
-    if (bidx < 0 || u > bub) {  // a lane's indices rise, so ties keep the lower one
-      bub = u;
-      bidx = sidx;
-    }
-  }
-  unsigned long long best = best_of(bub, bidx, bidx >= 0);
-  const int sstar = static_cast<int>(0xFFFFFFFFu - static_cast<unsigned>(best & 0xFFFFFFFFull));
-  {
-    const int t = sstar * kSuper + lane;
-    const bool ok = lane < kSuper && t < T;
-    best = best_of(ok ? ub_of(P.key_box, P.key_hmax, T, t) : 0.0f, t, ok);
-  }
-  for (int s0 = 0; s0 < S; s0 += 32) {
-    const int sidx = s0 + lane;
-    const float lbest = ord_float(static_cast<int>(static_cast<unsigned>(best >> 32) ^ 0x80000000u));
-    unsigned sbits =
-        __ballot_sync(0xffffffffu, sidx < S && sidx != sstar && sub_ub(sidx) >= lbest);
-    while (sbits) {
-      const int sl = __ffs(sbits) - 1;
-      sbits &= sbits - 1u;
-      const int t = (s0 + sl) * kSuper + lane;
-      const bool ok = lane < kSuper && t < T;
-      const unsigned long long k = best_of(ok ? ub_of(P.key_box, P.key_hmax, T, t) : 0.0f, t, ok);
-      best = best > k ? best : k;
-    }
-  }
-  const int anchor = static_cast<int>(0xFFFFFFFFu - static_cast<unsigned>(best & 0xFFFFFFFFull));
+  if (cached)
+    for (int sidx = lane; sidx < S; sidx += 32) s_sub[sidx] = ub_of(P.key_sbox, P.key_shmax, S, sidx);
 
   // Each row's largest exponent over the keys of a few tiles is a value the row reaches.
   // A tile's keys are taken about the block's centre c (y' = y - c, H' = H - kappa |y'|^2):
@@ -213,13 +168,12 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
       }
     }
   };
-  eval_tile(anchor);
 
-  // Morton anchors: the key tiles that hold the block's stretch of the shared space-filling
-  // order (the keys whose codes lie between the block's first and last row codes, and one
-  // key on either side). They hold most rows' nearest keys even where the anchor, chosen
-  // for the block's box as a whole, is far from some of its rows; at most kMortonAnchors
-  // of them, spread over the stretch.
+  // The anchors: the key tiles that hold the block's stretch of the shared Morton order
+  // (from one key before the block's first row code to one key after its last), at most
+  // kMortonAnchors of them, spread over the stretch. Without codes no tile is evaluated,
+  // every bound stays -inf and every tile is kept.
+  int anchor = -1;
   if (P.key_codes) {
     const int64_t nk = P.key_count;
     // first position in the sorted key codes whose code is >= target (warp-wide search)
@@ -247,7 +201,8 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
     const int na = span < kMortonAnchors ? span : kMortonAnchors;
     for (int e = 0; e < na; ++e) {
       const int t = na == span ? t0 + e : t0 + static_cast<int>(static_cast<int64_t>(e) * (span - 1) / (na - 1));
-      if (t != anchor) eval_tile(t);
+      if (e == 0) anchor = t;
+      eval_tile(t);
     }
   }
   const bool history = P.lse_prev && P.key_dmin;
