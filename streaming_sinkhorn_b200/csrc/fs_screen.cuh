@@ -14,7 +14,9 @@
 //   (b) history (potential passes after the first two): the largest term of a sum of m terms
 //       is at least the sum over m, and every bias moved by at least dmin since the row's
 //       previous pass, so max_j z_ij >= LSE2_prev_i + dmin - log2(m).
-// A tile with ub(T) < min_i mlb_i - margin is skipped. Each of its terms is below
+// A tile with ub(T) < min_i mlb_i - margin is skipped, and so is a tile for which every row
+// i of the block has ub_i(T) = Hmax_T - kappa dist(x_i, B_T)^2 < mlb_i - margin (the same
+// bound for the row alone). Each of its terms is below
 // 2^-margin times its row's largest term, so with margin = kSkipBits + log2(m) the whole
 // omitted part of a row's sum is below 2^-kSkipBits of that sum (the largest term is at
 // most the sum). With kSkipBits = 24, the fp32 unit roundoff, the omitted mass is at most
@@ -46,6 +48,7 @@ constexpr int kMortonAnchors = 4;
 template <int D, int R>
 __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned* kmask,
                                                     int* kcount) {
+  static_assert(R == 2, "the per-row tile test packs a lane's two rows");
   constexpr int KP = key_pair_floats(D);
   constexpr int RB = R * 32;
   constexpr int TP = kScreenTile / 2;  // key pairs per tile
@@ -208,20 +211,31 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
   const bool history = P.lse_prev && P.key_dmin;
   const float dmin = history ? ord_float(*P.key_dmin) : 0.0f;
   float mlb = INFINITY;
+  float rthr[R];  // each row's own threshold (+inf for rows past the end)
 #pragma unroll
   for (int r = 0; r < R; ++r) {
+    rthr[r] = INFINITY;
     if (!valid[r]) continue;
     const int64_t i = row0 + r * 32 + lane;
     float v = zmax[r];
     if (history) v = fmaxf(v, P.lse_prev[i] + dmin - P.log2_keys);
     if (P.row_mlb) P.row_mlb[i] = v;
     mlb = fminf(mlb, v);
+    rthr[r] = v - P.skip_margin;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mlb = fminf(mlb, __shfl_xor_sync(0xffffffffu, mlb, o));
   const float thr = mlb - P.skip_margin;
 
-  // the mask, 32 super-tiles (8 mask words) per round; lane j < 8 assembles word j
+  // The mask, 32 super-tiles (8 mask words) per round; lane j < 8 assembles word j. A tile
+  // is tested against the block's box and smallest bound, then each tile that passes row by
+  // row: it stays only if some row i has Hmax_t - kappa dist(x_i, B_t)^2 >= its own bound
+  // - margin. A block whose box spans two clusters, or that holds a row far below the
+  // others, keeps many tiles under the block test; the per-row test removes most of them.
+  // A lane tests its two rows at once in packed arithmetic.
+  u64 xr[D];
+#pragma unroll
+  for (int k = 0; k < D; ++k) xr[k] = pk(x[0][k], x[1][k]);
   unsigned* mrow = kmask + b * P.mask_words;
   int cnt = 0;
   for (int s0 = 0; s0 < S; s0 += 32) {
@@ -232,10 +246,43 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
     while (sbits) {
       const int sl = __ffs(sbits) - 1;
       sbits &= sbits - 1u;
-      const int t = (s0 + sl) * kSuper + lane;
-      const bool keep_t =
-          lane < kSuper && t < T && (t == anchor || ub_of(P.key_box, P.key_hmax, T, t) >= thr);
-      const unsigned pat = __ballot_sync(0xffffffffu, keep_t) & 0xFFu;
+      const int tbase = (s0 + sl) * kSuper;
+      const int t = tbase + lane;
+      // lanes 0-7 load the run's tiles (box and Hmax) once; the per-row tests below take
+      // them by shuffles
+      const bool okl = lane < kSuper && t < T;
+      float blo[D], bhi[D];
+      float d2b = 0.0f;
+#pragma unroll
+      for (int k = 0; k < D; ++k) {
+        blo[k] = okl ? P.key_box[k * T + t] : 0.0f;
+        bhi[k] = okl ? P.key_box[(D + k) * T + t] : 0.0f;
+        const float gap = fmaxf(fmaxf(blo[k] - hi[k], lo[k] - bhi[k]), 0.0f);
+        d2b = fmaf(gap, gap, d2b);
+      }
+      const float thm = okl ? P.key_hmax[t] : -INFINITY;
+      const bool keep_t = okl && (t == anchor || thm - P.kappa_f * d2b >= thr);
+      unsigned pat = __ballot_sync(0xffffffffu, keep_t) & 0xFFu;
+#pragma unroll
+      for (int tl = 0; tl < kSuper; ++tl) {
+        if (!((pat >> tl) & 1u) || tbase + tl == anchor) continue;
+        u64 d2 = pk(0.0f, 0.0f);
+#pragma unroll
+        for (int k = 0; k < D; ++k) {
+          const float lk = __shfl_sync(0xffffffffu, blo[k], tl);
+          const float hk = __shfl_sync(0xffffffffu, bhi[k], tl);
+          float a0, a1, c0, c1;
+          upk(sub2(pk(lk, lk), xr[k]), a0, a1);
+          upk(sub2(xr[k], pk(hk, hk)), c0, c1);
+          const u64 gap = pk(max3(a0, c0, 0.0f), max3(a1, c1, 0.0f));
+          d2 = fma2(gap, gap, d2);
+        }
+        float e0, e1;
+        upk(d2, e0, e1);
+        const float hm = __shfl_sync(0xffffffffu, thm, tl);
+        const bool need = hm - P.kappa_f * e0 >= rthr[0] || hm - P.kappa_f * e1 >= rthr[1];
+        if (!__any_sync(0xffffffffu, need)) pat &= ~(1u << tl);
+      }
       if (lane == sl / 4) word |= pat << ((sl % 4) * kSuper);
     }
     const int w = s0 / 4 + lane;
