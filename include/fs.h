@@ -108,6 +108,20 @@ FS_API const char* fs_last_cuda_error(void);
 FS_API size_t fs_workspace_bytes(const fs_problem* p);
 
 /*
+ * What a workspace carries from one call to the next. Every call on sorted clouds (d <= 16)
+ * puts both clouds in Morton order; the workspace keeps that order and a record of it (the
+ * shapes, a 64-bit fingerprint of each cloud's coordinates, the sort's frame and where the
+ * order lies). A later call with the same workspace whose record matches reuses the order
+ * instead of sorting again: fs_potentials, fs_grad_x, fs_marginal_residual and fs_cost on
+ * the same clouds sort once. A stale or colliding record cannot make results wrong, only
+ * screening less effective, since every pass is correct under any order.
+ * fs_workspace_invalidate (ws: device, 256-byte aligned, ws_bytes >= 2048, else
+ * FS_ERR_WORKSPACE; stream: as for the other calls) drops the record, so the next call
+ * sorts; enqueued on `stream`, FS_ERR_CUDA if that fails.
+ */
+FS_API fs_status fs_workspace_invalidate(void* ws, size_t ws_bytes, fs_stream_t stream);
+
+/*
  * Fixed-count alternating Sinkhorn (SinkSLOT README, API Reference: variant
  * "alternating", stop_mode "fixed"; FlashSinkhorn summary, section 1 for the update):
  *   g <- g_init (or 0 when g_init is NULL)

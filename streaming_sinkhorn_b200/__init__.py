@@ -18,6 +18,7 @@ import ctypes
 from . import _lib
 
 __all__ = ["potentials", "cost", "grad_x", "marginal_residual", "solve_host", "workspace_bytes",
+           "workspace_invalidate",
            "FsError", "timing_enable", "timing_reset", "timing_get", "launch_count",
            "screening_enable", "solve", "transport_apply", "hvp", "SamplesLoss",
            "sinkhorn_divergence", "solve_multiscale"]
@@ -403,6 +404,15 @@ def timing_reset() -> None:
 def screening_enable(on: bool = True) -> None:
     """Turns block screening on or off for later calls (fs_screening_enable)."""
     _lib.load().fs_screening_enable(1 if on else 0)
+
+
+def workspace_invalidate(workspace) -> None:
+    """Drops what ``workspace`` (a device uint8 tensor) remembers from earlier calls: the
+    Morton order of the last clouds it sorted, which later calls on the same clouds reuse
+    (fs_workspace_invalidate). Never needed for correct results."""
+    torch = _torch()
+    st = torch.cuda.current_stream(workspace.device).cuda_stream
+    _raise(_lib.load().fs_workspace_invalidate(workspace.data_ptr(), workspace.numel(), st))
 
 
 def launch_count() -> int:

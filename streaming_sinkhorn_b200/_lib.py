@@ -27,7 +27,7 @@ EXPORTS = (
     "fs_timing_enable", "fs_timing_reset", "fs_timing_get", "fs_launch_count",
     "fs_potentials_noalloc", "fs_screening_enable", "fs_solve", "fs_transport_workspace_bytes",
     "fs_transport_apply", "fs_hvp", "fs_divergence_workspace_bytes", "fs_divergence",
-    "fs_multiscale_workspace_bytes", "fs_solve_multiscale",
+    "fs_multiscale_workspace_bytes", "fs_solve_multiscale", "fs_workspace_invalidate",
 )
 
 VARIANTS = {"alternating": 0, "symmetric": 1}
@@ -137,6 +137,8 @@ def load():
     lib.fs_timing_enable.restype = None
     lib.fs_screening_enable.argtypes = [ctypes.c_int]
     lib.fs_screening_enable.restype = None
+    lib.fs_workspace_invalidate.argtypes = [vp, sz, vp]
+    lib.fs_workspace_invalidate.restype = ctypes.c_int
     lib.fs_timing_reset.argtypes = []
     lib.fs_timing_reset.restype = None
     lib.fs_timing_get.argtypes = [ctypes.POINTER(fs_timing)]

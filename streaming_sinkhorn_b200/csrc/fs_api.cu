@@ -312,6 +312,8 @@ constexpr int kAccRow = 130;  // [3]
 constexpr int kAccCol = 133;  // [3]
 constexpr int kDotFA = 136;
 constexpr int kDotGB = 137;
+constexpr int kHashX = 138;    // uint64: fingerprint of x's coordinates
+constexpr int kHashY = 139;    // uint64: fingerprint of y's coordinates
 constexpr int kFlags = 140;   // unsigned, in the bytes of this double
 constexpr int kErr = 141;     // unsigned
 constexpr int kMaxAbs = 142;  // unsigned: float bits of the largest |coordinate| of x and y
@@ -322,6 +324,11 @@ constexpr int kQueue = 151;   // ints: tiles per unit C and unit count U of the 
 constexpr int kKept = 152;    // int64: kept tiles K of the last queue plan
 constexpr int kPotChange = 153;  // unsigned: float bits of the largest potential change
 constexpr int kCgDots = 156;     // [4] float64: the HVP solve's dot products and sums
+// [kSortMemoWords] uint64 from here: the record of the last sort done in this workspace,
+// which prepare() does not clear (everything before it is cleared at every call)
+constexpr int kSortMemo = 240;
+constexpr unsigned long long kSortMagic = 0x536f72744d656d6full;  // "SortMemo"
+static_assert(kSortMemo + kSortMemoWords <= kScalarDoubles, "sort record outside the scalar block");
 
 struct Layout {
   int D;       // padded dimension of the FMA path
@@ -960,7 +967,7 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
   }
   const fs_problem* p = c.p;
   c.use_tc = need_tc && c.L.Dtc > 0;
-  CK(cudaMemsetAsync(c.scal, 0, kScalarDoubles * sizeof(double), c.st));
+  CK(cudaMemsetAsync(c.scal, 0, kSortMemo * sizeof(double), c.st));
   const int sdims = std::min(p->d, kSortDims);
   if (c.L.sorted) {
     // bounding box of both clouds: lo starts at +3.4e38, hi at -3.4e38 (as ordered ints)
@@ -985,12 +992,12 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
     CK(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
-  check_coords_kernel<<<reduce_blocks(p->n * p->d, c.sms), 256, 0, c.st>>>(p->x, p->n * p->d,
-                                                                           flags_ptr(c.scal));
+  check_coords_kernel<<<reduce_blocks(p->n * p->d, c.sms), 256, 0, c.st>>>(
+      p->x, p->n * p->d, flags_ptr(c.scal), reinterpret_cast<unsigned long long*>(c.scal + kHashX));
   CK(cudaGetLastError());
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  check_coords_kernel<<<reduce_blocks(p->m * p->d, c.sms), 256, 0, c.st>>>(p->y, p->m * p->d,
-                                                                           flags_ptr(c.scal));
+  check_coords_kernel<<<reduce_blocks(p->m * p->d, c.sms), 256, 0, c.st>>>(
+      p->y, p->m * p->d, flags_ptr(c.scal), reinterpret_cast<unsigned long long*>(c.scal + kHashY));
   CK(cudaGetLastError());
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (p->a) {
@@ -1012,7 +1019,9 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
   double host[kBox + 3];  // through the bounding box (6 ints at kBox)
+  unsigned long long memo[kSortMemoWords];
   CK(cudaMemcpyAsync(host, c.scal, sizeof(host), cudaMemcpyDeviceToHost, c.st));
+  CK(cudaMemcpyAsync(memo, c.scal + kSortMemo, sizeof(memo), cudaMemcpyDeviceToHost, c.st));
   CK(cudaStreamSynchronize(c.st));
   unsigned flags;
   memcpy(&flags, &host[kFlags], sizeof(unsigned));
@@ -1037,8 +1046,31 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
       F.scale[k] = hi > lo ? static_cast<float>(((1u << F.bits) - 1u) / (static_cast<double>(hi) - lo))
                            : 0.0f;
     }
-    sort_cloud(p->x, p->n, p->d, F, c.sortkeys, c.L.sort_n, c.perm_x, c.code_x, c.st);
-    sort_cloud(p->y, p->m, p->d, F, c.sortkeys, c.L.sort_n, c.perm_y, c.code_y, c.st);
+    // The sort depends only on the coordinates (through them, on the frame). A workspace
+    // keeps a record of its last sort: the shapes, both clouds' fingerprints, the frame and
+    // where the permutations and codes lie; a call that matches it reuses them. (Any
+    // permutation gives correct results; the order only decides how well screening works.)
+    unsigned long long hx, hy;
+    memcpy(&hx, &host[kHashX], sizeof(hx));
+    memcpy(&hy, &host[kHashY], sizeof(hy));
+    unsigned long long frame = static_cast<unsigned long long>(F.dims) | (static_cast<unsigned long long>(F.bits) << 8);
+    for (int k = 0; k < 2 * kSortDims; ++k)
+      frame = (frame * 0x100000001b3ull) ^ static_cast<unsigned>(boxi[k]);
+    const SortMemo want{{kSortMagic, static_cast<unsigned long long>(p->n),
+                         static_cast<unsigned long long>(p->m), static_cast<unsigned long long>(p->d),
+                         hx, hy, c.L.off_perm_x, c.L.off_perm_y, c.L.off_code_x, c.L.off_code_y,
+                         static_cast<unsigned long long>(c.L.sort_n), frame}};
+    if (memcmp(want.v, memo, sizeof(memo)) != 0) {
+      sort_cloud(p->x, p->n, p->d, F, c.sortkeys, c.L.sort_n, c.perm_x, c.code_x, c.st);
+      sort_cloud(p->y, p->m, p->d, F, c.sortkeys, c.L.sort_n, c.perm_y, c.code_y, c.st);
+      sort_memo_kernel<<<1, 32, 0, c.st>>>(
+          reinterpret_cast<unsigned long long*>(c.scal + kSortMemo), want);
+      CK(cudaGetLastError());
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+    }
+  } else {
+    // this layout may overwrite where a sorted layout keeps its permutations
+    CK(cudaMemsetAsync(c.scal + kSortMemo, 0, sizeof(unsigned long long), c.st));
   }
   const float wu_x = static_cast<float>(1.0 / p->n), wu_y = static_cast<float>(1.0 / p->m);
   FS_DISPATCH_D(c.L.D, launch_pack_d, p->x, p->n, p->d, p->a, wu_x, c.perm_x, c.kx, c.lwx, c.L.px,
@@ -2153,6 +2185,22 @@ fs_status fs_solve_host(const fs_problem* hp, int32_t n_iters, float* f, float* 
 int64_t fs_launch_count(void) { return fs::g_launches.load(std::memory_order_relaxed); }
 
 void fs_screening_enable(int on) { fs::g_screening.store(on != 0); }
+
+fs_status fs_workspace_invalidate(void* ws, size_t ws_bytes, fs_stream_t stream) {
+  using namespace fs;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 ||
+      ws_bytes < kScalarDoubles * sizeof(double))
+    return FS_ERR_WORKSPACE;
+  // the scalar block opens every layout; the record's first word is its marker
+  double* scal = static_cast<double*>(ws);
+  try {
+    CK(cudaMemsetAsync(scal + kSortMemo, 0, sizeof(unsigned long long),
+                       static_cast<cudaStream_t>(stream)));
+  } catch (const CudaFail&) {
+    return FS_ERR_CUDA;
+  }
+  return FS_OK;
+}
 
 void fs_timing_enable(int on) {
   std::lock_guard<std::mutex> lk(fs::g_timing_mu);

@@ -134,6 +134,7 @@ struct PassParams {
 };
 
 constexpr int kScreenTile = 256;  // points per screening tile (= kPairPad pairs)
+constexpr int kSortMemoWords = 12;  // words of the sort record a workspace keeps
 // Relative size, in log2 units, below which the omitted part of a row's sum is kept: the
 // skip margin is kSkipBits + log2(number of keys) (the tolerance of the screening). 24 bits
 // is the fp32 unit roundoff: the omitted mass is at most one rounding of the row's sum.
@@ -796,15 +797,43 @@ __global__ void __launch_bounds__(256) combine_kernel(const PassParams P) {
 
 // ---- preparation kernels --------------------------------------------------------------
 
-// Flags bit 1 for a non-finite coordinate.
+// The splitmix64 output mixer (Steele, Lea and Flood, "Fast splittable pseudorandom number
+// generators", 2014, with the "variant 13" constants of D. Stafford that Vigna's splitmix64
+// uses): a bijective 64-bit mixer.
+__device__ __forceinline__ unsigned long long mix64(unsigned long long z) {
+  z = (z ^ (z >> 30)) * 0xbf58476d1ce4e5b9ull;
+  z = (z ^ (z >> 27)) * 0x94d049bb133111ebull;
+  return z ^ (z >> 31);
+}
+
+// Flags bit 1 for a non-finite coordinate; adds a fingerprint of the coordinates (the sum
+// over entries of mix64(index, bits), so it does not depend on the reduction order) to *hash.
 __global__ void __launch_bounds__(256) check_coords_kernel(const float* pts, int64_t count,
-                                                           unsigned* flags) {
+                                                           unsigned* flags,
+                                                           unsigned long long* hash) {
   int bad = 0;
+  unsigned long long h = 0ull;
   for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < count;
-       j += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    bad |= !isfinite(pts[j]);
+       j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float v = pts[j];
+    bad |= !isfinite(v);
+    h += mix64((static_cast<unsigned long long>(j) << 32) ^ __float_as_uint(v));
+  }
   bad = warp_or(bad);
-  if ((threadIdx.x & 31) == 0 && bad) atomicOr(flags, 1u);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) h += __shfl_xor_sync(0xffffffffu, h, o);
+  if ((threadIdx.x & 31) == 0) {
+    if (bad) atomicOr(flags, 1u);
+    atomicAdd(hash, h);
+  }
+}
+
+// The record of the last sort kept in a workspace (see prepare()).
+struct SortMemo {
+  unsigned long long v[kSortMemoWords];
+};
+__global__ void sort_memo_kernel(unsigned long long* memo, const SortMemo m) {
+  if (threadIdx.x < kSortMemoWords) memo[threadIdx.x] = m.v[threadIdx.x];
 }
 
 // Weight sum (float64); flags bit 2 for a negative or non-finite weight.

@@ -249,3 +249,13 @@ def test_multiscale_argument_errors():
     assert st(lib.fs_solve_multiscale(ctypes.byref(cos), ctypes.byref(o),
                                       ctypes.byref(_lib.fs_multiscale_options(32, 5, 4, 0.0, 0.5)),
                                       FAKE, FAKE, None, FAKE, BIG, None)) == "FS_ERR_OPTION"
+
+
+def test_workspace_invalidate_argument_errors():
+    """Rejected before any CUDA call: no workspace, a misaligned one, one too small to hold
+    the scalar block."""
+    lib = _lib.load()
+    code = _lib.STATUS_CODE["FS_ERR_WORKSPACE"]
+    assert lib.fs_workspace_invalidate(None, 4096, None) == code
+    assert lib.fs_workspace_invalidate(FAKE + 16, 4096, None) == code
+    assert lib.fs_workspace_invalidate(FAKE, 1024, None) == code
