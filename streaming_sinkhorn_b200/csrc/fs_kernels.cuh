@@ -262,7 +262,7 @@ __device__ __forceinline__ void block_reduce_marg(double dev_sum, double dev_max
 // kMergeChunk at a time, all loads of a chunk issued before any is used, so that a row
 // costs one memory round trip per chunk rather than one per partial. A partial whose
 // columns were all zero-weight or padding left m = -inf and sum 0 and drops out.
-constexpr int kMergeChunk = 8;
+constexpr int kMergeChunk = 4;
 template <int D, int MODE, int NA>
 __device__ __forceinline__ void merge_row(const PassParams& P, int64_t i, int64_t s0, int64_t ns,
                                           int64_t stride, int64_t off, double& dev_sum,
