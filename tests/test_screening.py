@@ -77,3 +77,25 @@ def test_screened_equals_dense(n, m):
     # sums), where any change of summation order shows at ~1e-6 of the mass
     np.testing.assert_allclose(ress, resd, rtol=1e-3, atol=2e-5 * float(w.b.sum()))
     assert costs == pytest.approx(costd, rel=1e-4)
+
+
+@pytest.mark.parametrize("d", [2, 5, 8])
+def test_screened_equals_dense_other_dims(d):
+    """Other widths: 16-bit Morton codes at d = 2, codes of the first three coordinates at
+    d = 5 and 8 (so the anchors come from a projection of the points), ragged row blocks
+    and key tiles (n, m not multiples of 64 and 256)."""
+    w = workloads.mixture_pair(n=24001, m=30011, d=d, k=40, std=0.03, seed=13 + d, eps=1e-3,
+                               n_iters=6, clip_unit_cube=True)
+    fd, gd, td = solve(w, False)
+    fsc, gsc, ts = solve(w, True)
+    kappa = 1.0 / (w.eps * np.log(2.0))
+    df = np.abs(fsc.astype(np.float64) - fd).max() * kappa
+    dg = np.abs(gsc.astype(np.float64) - gd).max() * kappa
+    assert df < 1e-2 and dg < 1e-2, (df, dg)
+    assert ts["screen"]["launches"] > 0
+    assert ts["lse_pass"]["evaluated"] < 0.9 * ts["lse_pass"]["pairs"]
+    gxd, rd, cd, resd, costd = passes(w, fd, gd, False)
+    gxs, rs, cs, ress, costs = passes(w, fd, gd, True)
+    assert_grad_close(gxs, gxd, rel=1e-3)
+    np.testing.assert_allclose(rs, rd, rtol=1e-3, atol=1e-7 * float(w.a.max()))
+    assert costs == pytest.approx(costd, rel=1e-4)
