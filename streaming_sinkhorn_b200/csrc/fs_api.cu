@@ -346,7 +346,7 @@ struct Layout {
   size_t off_perm_x, off_perm_y, off_code_x, off_code_y, off_sortkeys, off_box_x, off_box_y, off_hmax_x, off_hmax_y,
       off_lse_x, off_lse_y;
   // queue mode: kept-tile masks, kept counts, unit starts and unit -> row block
-  size_t off_kmask, off_kcount, off_ustart, off_unit_rb, off_unit_j, off_rmlb;
+  size_t off_kmask, off_kcount, off_ustart, off_unit_rb, off_unit_j;
   // general solve: deferred biases of x (symmetric schedule), potentials at the last check
   size_t off_defer, off_fprev, off_gprev;
   // transport products and the Hessian-vector product (layouts asked with acc_ch > 0):
@@ -471,8 +471,6 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0, bool co
     o = align_up(o + static_cast<size_t>(units_max) * sizeof(int));
     L.off_unit_j = o;
     o = align_up(o + static_cast<size_t>(units_max) * sizeof(int));
-    L.off_rmlb = o;
-    o = align_up(o + static_cast<size_t>(std::max(n, m)) * sizeof(float));
   }
   L.off_defer = o;
   o = align_up(o + static_cast<size_t>(std::max(n, L.tx)) * sizeof(float));
@@ -859,7 +857,6 @@ struct Ctx {
   float *box_x, *box_y, *hmax_x, *hmax_y, *lse_x, *lse_y;
   unsigned* kmask;
   int *kcount, *ustart, *unit_rb, *unit_j;
-  float* rmlb;     // per-row lower bounds written by the screening kernel
   float *defer, *fprev, *gprev;
   float* paykeys; // transport passes: keys with payload channels
   float* hvp;     // the HVP's vectors
@@ -934,7 +931,6 @@ void carve(Ctx& c, void* ws) {
     c.ustart = reinterpret_cast<int*>(c.ws + c.L.off_ustart);
     c.unit_rb = reinterpret_cast<int*>(c.ws + c.L.off_unit_rb);
     c.unit_j = reinterpret_cast<int*>(c.ws + c.L.off_unit_j);
-    c.rmlb = reinterpret_cast<float*>(c.ws + c.L.off_rmlb);
   }
 }
 
@@ -1307,7 +1303,6 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
     P.unit_rb = c.unit_rb;
     P.unit_j = c.unit_j;
     P.qscal = reinterpret_cast<const int*>(c.scal + kQueue);
-    P.row_mlb = c.rmlb;
     P.key_codes = rows_x ? c.code_y : c.code_x;
     P.row_codes = rows_x ? c.code_x : c.code_y;
     P.key_count = n_keys;

@@ -117,7 +117,6 @@ struct PassParams {
   const int* unit_rb;       // [unit] row block of each unit (launch order)
   const int* unit_j;        // [unit] its index among its row block's units
   const int* qscal;         // [0] tiles per unit C, [1] number of units U
-  float* row_mlb;           // [row]: lower bound on each row's largest exponent (screening)
   const unsigned* key_codes; // Morton codes of the key cloud in sorted order (key_count)
   const unsigned* row_codes; // Morton codes of the query cloud in sorted order
   int64_t key_count;         // real keys

@@ -219,7 +219,6 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
     const int64_t i = row0 + r * 32 + lane;
     float v = zmax[r];
     if (history) v = fmaxf(v, P.lse_prev[i] + dmin - P.log2_keys);
-    if (P.row_mlb) P.row_mlb[i] = v;
     mlb = fminf(mlb, v);
     rthr[r] = v - P.skip_margin;
   }
