@@ -558,7 +558,7 @@ void with_pass_kernel(int sel, int variant, Op&& op) {
   } else {
     constexpr int S = kNarrowStages;
     switch (sel) {
-      case kSelGrad: op.template run<PassKernel<D, 2, 32, kModeGrad, 0, 8, 12, S>>(); break;
+      case kSelGrad: op.template run<PassKernel<D, 2, 32, kModeGrad, 0, 8, 16, S>>(); break;
       case kSelPay1: op.template run<PassKernel<D, 2, 32, kModePay, 1, 8, 20, S>>(); break;
       case kSelPay4: op.template run<PassKernel<D, 2, 32, kModePay, 4, 8, 16, S>>(); break;
       case kSelPay16: op.template run<PassKernel<D, 2, 32, kModePay, 16, 8, 8, S>>(); break;
