@@ -343,7 +343,7 @@ FS_API fs_status fs_marginal_residual(const fs_problem* p, const float* f, const
  *    wrong results. Serialise them.
  * Other errors are those of fs_potentials.
  */
-#define FS_NOALLOC_SCRATCH_BYTES (16u << 20)
+#define FS_NOALLOC_SCRATCH_BYTES (20u << 20)
 FS_API fs_status fs_potentials_noalloc(const fs_problem* p, int32_t n_iters, const float* g_init,
                                        float* f, float* g, fs_stream_t stream);
 
