@@ -55,6 +55,7 @@ class Timer {
       cudaEventDestroy(t.stop);
     }
   }
+  bool on() const { return on_; }
   int begin() {
     if (!on_) return -1;
     TimedLaunch t{};
@@ -1466,6 +1467,67 @@ fs_status check_options(const fs_solve_options& o) {
 
 }  // namespace
 
+// A stream the library captures graphs on: the caller's stream may be the legacy default
+// stream, which cannot be captured. One per device, created on first use.
+cudaStream_t capture_stream() {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {};
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!streams[dev]) CK(cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking));
+  return streams[dev];
+}
+
+// Runs body() `count` times on c.st as one CUDA graph: body's launches are captured once
+// (on the capture stream, so nothing runs during the capture) and the graph is replayed on
+// the caller's stream, one launch instead of ~15 per replay. body() must issue the same
+// launches with the same arguments every time and read nothing back. Returns false, having
+// run nothing, when the capture is unavailable or refused one of body's calls; the caller
+// then issues the work itself.
+template <typename Body>
+bool replay_as_graph(Ctx& c, int32_t count, Body&& body) {
+  cudaStream_t cap = capture_stream();
+  if (!cap) return false;
+  const cudaStream_t user = c.st;
+  if (cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  const int64_t l0 = g_launches.load();
+  cudaGraph_t graph = nullptr;
+  c.st = cap;
+  bool ok = true;
+  try {
+    body();
+  } catch (const CudaFail&) {
+    ok = false;  // a call the capture refused: nothing ran, so the caller issues it all
+  }
+  c.st = user;
+  const int64_t per = g_launches.load() - l0;  // counted while capturing, not yet run
+  g_launches.fetch_sub(per);
+  if (cudaStreamEndCapture(cap, &graph) != cudaSuccess || !ok) {
+    if (graph) cudaGraphDestroy(graph);
+    cudaGetLastError();
+    return false;
+  }
+  cudaGraphExec_t exec = nullptr;
+  cudaError_t e = cudaGraphInstantiate(&exec, graph, 0);
+  for (int32_t k = 0; e == cudaSuccess && k < count; ++k) {
+    e = cudaGraphLaunch(exec, user);
+    if (e == cudaSuccess) g_launches.fetch_add(per);
+  }
+  if (exec) {
+    const cudaError_t se = cudaStreamSynchronize(user);  // the launches are done with it
+    if (e == cudaSuccess) e = se;
+    cudaGraphExecDestroy(exec);
+  }
+  cudaGraphDestroy(graph);
+  CK(e);
+  return true;
+}
+
 fs_status solve_impl(const fs_problem* p, const fs_solve_options* opt, float* f, float* g,
                      fs_solve_report* report, void* ws, size_t ws_bytes, fs_stream_t stream) {
   Ctx c{};
@@ -1507,12 +1569,23 @@ fs_status solve_impl(const fs_problem* p, const fs_solve_options* opt, float* f,
     double viol = NAN;
     // From the second iteration on every row has a previous LSE2 and the keys a recorded
     // bias change, so the passes can screen key tiles by history as well.
-    for (int32_t it = 1; it <= total; ++it) {
+    auto iteration = [&](int32_t it) {
       c.defer_x = sym;
       run_pass(c, true, kPot, nullptr, f, nullptr, nullptr, nullptr, it > 1);   // f <- F(g)
       c.defer_x = false;
       run_pass(c, false, kPot, nullptr, g, nullptr, nullptr, nullptr, it > 1);  // g <- G(f)
       if (sym) apply_deferred_x(c);
+    };
+    // A fixed count issues the same launches in every iteration from the second on (the
+    // screening decision is taken after the first): those run as replays of one CUDA graph,
+    // unless per-kernel timing is on (it records events around each launch).
+    const bool graphs = fixed && total >= 3 && !c.timer->on();
+    for (int32_t it = 1; it <= total; ++it) {
+      if (graphs && it == 2 && replay_as_graph(c, total - 1, [&] { iteration(2); })) {
+        iters = total;
+        break;
+      }
+      iteration(it);
       iters = it;
       if (it == 1 && total > 2) screening_probe(c, false);
       if (fixed || (it % o.stop_check_every != 0 && it != total)) continue;
