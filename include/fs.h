@@ -134,8 +134,9 @@ FS_API fs_status fs_workspace_invalidate(void* ws, size_t ws_bytes, fs_stream_t 
  * fs_solve with stop_mode FS_STOP_FIXED) are captured once as a CUDA graph and replayed on
  * `stream`. The capture runs on a non-blocking stream the library creates once per device
  * and keeps until exit (so `stream` may be the legacy default stream); a capture that
- * fails falls back to plain launches. Per-kernel timing (fs_timing_enable) turns it off.
- * The call returns once the replays have finished.
+ * fails falls back to plain launches. Per-kernel timing (fs_timing_enable) turns it off,
+ * and fs_potentials_noalloc never uses it (instantiating a graph may allocate). The call
+ * returns once the replays have finished.
  */
 FS_API fs_status fs_potentials(const fs_problem* p, int32_t n_iters, const float* g_init, float* f,
                         float* g, void* ws, size_t ws_bytes, fs_stream_t stream);

@@ -1529,7 +1529,8 @@ bool replay_as_graph(Ctx& c, int32_t count, Body&& body) {
 }
 
 fs_status solve_impl(const fs_problem* p, const fs_solve_options* opt, float* f, float* g,
-                     fs_solve_report* report, void* ws, size_t ws_bytes, fs_stream_t stream) {
+                     fs_solve_report* report, void* ws, size_t ws_bytes, fs_stream_t stream,
+                     bool graphs_allowed = true) {
   Ctx c{};
   fs_status s = begin(c, p, ws, ws_bytes, stream);
   if (s != FS_OK) return s;
@@ -1579,7 +1580,7 @@ fs_status solve_impl(const fs_problem* p, const fs_solve_options* opt, float* f,
     // A fixed count issues the same launches in every iteration from the second on (the
     // screening decision is taken after the first): those run as replays of one CUDA graph,
     // unless per-kernel timing is on (it records events around each launch).
-    const bool graphs = fixed && total >= 3 && !c.timer->on();
+    const bool graphs = graphs_allowed && fixed && total >= 3 && !c.timer->on();
     for (int32_t it = 1; it <= total; ++it) {
       if (graphs && it == 2 && replay_as_graph(c, total - 1, [&] { iteration(2); })) {
         iters = total;
@@ -1759,13 +1760,14 @@ fs_status hvp_impl(const fs_problem* p, const float* g, const float* v, float* o
 // ---------------- entry points ----------------
 
 fs_status potentials_impl(const fs_problem* p, int32_t n_iters, const float* g_init, float* f,
-                          float* g, void* ws, size_t ws_bytes, fs_stream_t stream) {
+                          float* g, void* ws, size_t ws_bytes, fs_stream_t stream,
+                          bool graphs_allowed = true) {
   fs_solve_options o{};
   o.n_iters = n_iters;
   o.variant = FS_VARIANT_ALTERNATING;
   o.stop_mode = FS_STOP_FIXED;
   o.g_init = g_init;
-  return solve_impl(p, &o, f, g, nullptr, ws, ws_bytes, stream);
+  return solve_impl(p, &o, f, g, nullptr, ws, ws_bytes, stream, graphs_allowed);
 }
 
 }  // namespace fs

@@ -6,9 +6,12 @@
 #include "../../include/fs.h"
 
 namespace fs {
-// Defined in fs_api.cu: the body of fs_potentials, which takes its scratch space as an argument.
+// Defined in fs_api.cu: the body of fs_potentials, which takes its scratch space as an
+// argument; graphs_allowed = false keeps it to plain launches (instantiating a CUDA graph
+// may allocate device memory, which this entry point promises not to do).
 fs_status potentials_impl(const fs_problem* p, int32_t n_iters, const float* g_init, float* f,
-                          float* g, void* ws, size_t ws_bytes, fs_stream_t stream);
+                          float* g, void* ws, size_t ws_bytes, fs_stream_t stream,
+                          bool graphs_allowed);
 }
 
 namespace {
@@ -58,5 +61,6 @@ extern "C" fs_status fs_potentials_noalloc(const fs_problem* p, int32_t n_iters,
   // The solve clears the part of the scratch that must start at zero (its float64
   // accumulators and error word) and writes every other byte it reads, so what an
   // earlier call left there does not matter.
-  return fs::potentials_impl(p, n_iters, g_init, f, g, scratch, FS_NOALLOC_SCRATCH_BYTES, stream);
+  return fs::potentials_impl(p, n_iters, g_init, f, g, scratch, FS_NOALLOC_SCRATCH_BYTES, stream,
+                             false);
 }
