@@ -403,6 +403,25 @@ def run_native(args, rank, world, local_rank):
                 if rep is not None:
                     solve_extras[name].update(rep)
 
+    # Work the kernels actually did: pairs evaluated per step by every pass of the step (after
+    # screening; the tensor-core path does not screen, so there it is the nominal count),
+    # and the metric rate the unscreened pass sustains.
+    evaluated = 0.0
+    for k in ("lse_pass", "grad_pass", "marg_pass"):
+        t = timing[k]
+        evaluated += t["evaluated"] if t["evaluated"] > 0 else t["pairs"]
+    executed = {
+        "pairs_evaluated_per_step": evaluated / args.steps,
+        "executed_pair_evals_per_s": evaluated / args.steps / (ms_per_step / 1e3),
+        "what": "pairs the kernels evaluated per step (all passes: 2 x iters potential passes, "
+                "gradient, marginal and plan-mass passes) over the step time"}
+    if "dense_pass" in roofline:
+        dp = roofline["dense_pass"]
+        # one iteration = two N x M passes; N*M*iters/s of the pass run unscreened
+        executed["dense_metric_rate"] = float(w.n) * w.m / (dp["ms_per_launch"] / 1e3) / 2.0
+        executed["dense_metric_rate_what"] = ("N*M*iters/s of the potential pass with screening "
+                                              "off (N*M pairs per launch, two per iteration)")
+
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -415,6 +434,7 @@ def run_native(args, rank, world, local_rank):
                    "screening": "on: value counts all N*M*iters pairs; roofline.executed_ex2 "
                                 "counts the exponentials the kernels issued"},
         "gpu_launches": int(launches),
+        "executed": executed,
         "roofline": roofline,
         "clocks": clk,
         "kernel_timing": timing,
@@ -438,7 +458,10 @@ def run_native(args, rank, world, local_rank):
 
 def run_e2e(args, w, dev, world, dist):
     """Same metric through fs_solve_host: host inputs copied in and results copied out
-    inside every timed step."""
+    inside every timed step. Each step drops the workspace's sort record first, so it sorts
+    once as the device-timed step does, and runs in the same mode (per-kernel timing on, so
+    no CUDA graph replay); the same loop with timing off (graph replay of the iterations)
+    is reported beside it."""
     import torch
     import streaming_sinkhorn_b200 as fs
     pin = lambda v: torch.from_numpy(v).pin_memory()  # noqa: E731
@@ -455,24 +478,40 @@ def run_e2e(args, w, dev, world, dist):
     nbytes = int(_lib.load().fs_solve_host_workspace_bytes(ctypes.byref(p)))
     ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     steps = args.e2e_steps if args.e2e_steps is not None else args.steps
-    fs.solve_host(xh, yh, ah, bh, eps=w.eps, n_iters=w.n_iters, device=dev, workspace=ws, out=out)
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
     stream = torch.cuda.current_stream(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        fs.solve_host(xh, yh, ah, bh, eps=w.eps, n_iters=w.n_iters, device=dev, workspace=ws, out=out)
-    e1.record(stream)
-    e1.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dist, dev)
+
+    def one():
+        fs.workspace_invalidate(ws)
+        fs.solve_host(xh, yh, ah, bh, eps=w.eps, n_iters=w.n_iters, device=dev, workspace=ws,
+                      out=out)
+
+    def timed(per_kernel_timing: bool) -> float:
+        fs.timing_enable(per_kernel_timing)
+        one()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            one()
+        e1.record(stream)
+        e1.synchronize()
+        fs.timing_enable(False)
+        return max_over_ranks(e0.elapsed_time(e1) / steps, dist, dev)
+
+    ms = timed(True)
+    ms_graphs = timed(False)
     h2d = (w.n * w.d + w.m * w.d + w.n + w.m) * 4
     d2h = (w.n + w.m + w.n * w.d) * 4 + 5 * 8
-    return {"value": job_value(float(w.n) * w.m * w.n_iters, world, ms), "unit": UNIT,
+    pairs = float(w.n) * w.m * w.n_iters
+    return {"value": job_value(pairs, world, ms), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
-            "steps": steps, "api": "fs_solve_host (pinned host buffers)"}
+            "steps": steps, "api": "fs_solve_host (pinned host buffers)",
+            "mode": "per-kernel timing on, no graph replay, one sort per step (as the device leg)",
+            "graph_replay": {"value": job_value(pairs, world, ms_graphs), "ms_per_step": ms_graphs,
+                             "mode": "timing off: iterations 2.. replayed as one CUDA graph"}}
 
 
 # ---------------------------------------------------------------- reference arm ----

@@ -90,7 +90,9 @@ typedef enum {
   FS_ERR_TIMEOUT = 11,         /* a kernel's bounded wait expired; outputs invalid */
   FS_ERR_CUDA = 12,            /* a CUDA runtime call failed (see fs_last_cuda_error) */
   FS_ERR_ALIGNMENT = 13,       /* a device pointer is not 4-byte aligned */
-  FS_ERR_OPTION = 14           /* an fs_solve_options field is out of range */
+  FS_ERR_OPTION = 14,          /* an fs_solve_options field is out of range */
+  FS_ERR_DEVICE_MEMORY = 15    /* the device could not commit the static scratch array of
+                                  fs_potentials_noalloc when its module was loaded */
 } fs_status;
 
 /* Human-readable name of a status code (static storage, never NULL). */
@@ -340,9 +342,18 @@ FS_API fs_status fs_marginal_residual(const fs_problem* p, const float* f, const
  *  - Problems whose fs_workspace_bytes() exceeds FS_NOALLOC_SCRATCH_BYTES are rejected
  *    with FS_ERR_WORKSPACE before any device work. At d = 3 every problem with
  *    n, m <= 80000 fits; larger d needs more scratch per point.
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call before any
- *    stream capture on the device.
+ *  - Every call looks up the array's device address (cudaGetSymbolAddress) in the context
+ *    current on the calling thread; nothing is cached, so the call stays correct after
+ *    cudaDeviceReset or under a context of the caller's own.
+ *  - When that memory is committed depends on the CUDA module loading mode. Under lazy
+ *    loading (CUDA_MODULE_LOADING=LAZY, the default since CUDA 12.2) the FIRST call in a
+ *    context loads the module that holds the array: that call commits
+ *    FS_NOALLOC_SCRATCH_BYTES of device memory (plus the module's code) and may
+ *    synchronise the device. Make it during initialisation, before a pool allocator
+ *    reserves the device's memory and before any stream capture. If the device cannot
+ *    provide the memory the call returns FS_ERR_DEVICE_MEMORY (other failures of the
+ *    lookup: FS_ERR_CUDA). Under eager loading the array is committed when the context is
+ *    created. Later calls commit nothing.
  *  - No call allocates or frees device memory (no cudaMalloc, cudaFree or allocating
  *    library routine).
  *  - All calls on a device share the one array and it keeps what the last call wrote:
@@ -353,6 +364,30 @@ FS_API fs_status fs_marginal_residual(const fs_problem* p, const float* f, const
 #define FS_NOALLOC_SCRATCH_BYTES (20u << 20)
 FS_API fs_status fs_potentials_noalloc(const fs_problem* p, int32_t n_iters, const float* g_init,
                                        float* f, float* g, fs_stream_t stream);
+
+/*
+ * Checks of the error path (SinkSLOT README, "Tensor Contract": bad states raise rather than
+ * return wrong results). Every pass kernel bounds its waits (2 s of %globaltimer) and, when
+ * one expires, sets a bit in the call's device error word, waits (bounded) for its own
+ * copies in flight and returns; the entry point then returns FS_ERR_TIMEOUT.
+ *
+ * fs_inject_error_word arms a one-shot injection: the next entry point call (any host
+ * thread) that reads its kernels' error word first ORs `bits` into that word on the device,
+ * by a kernel launched on the call's stream after its passes, where an expired wait would
+ * have set it. That call then returns FS_ERR_TIMEOUT (for any non-zero bits) and its
+ * outputs are invalid; the injection is disarmed, and later calls are unaffected
+ * (0 disarms without injecting). Process-wide, for tests of the error path.
+ *
+ * fs_check_bounded_wait runs the bounded mbarrier wait of the pass kernels, with a limit of
+ * limit_ns (1e3 .. 2e9 ns, else FS_ERR_OPTION), on a barrier that nothing arrives at, with
+ * no copy or MMA in flight. The wait expires, the kernel sets the error word (held in `ws`:
+ * device, 256-byte aligned, >= 2048 bytes, else FS_ERR_WORKSPACE) and returns, so the call
+ * returns FS_ERR_TIMEOUT after about limit_ns, the context still usable. FS_OK would mean a
+ * wait that ended although nothing arrived.
+ */
+FS_API void fs_inject_error_word(unsigned bits);
+FS_API fs_status fs_check_bounded_wait(int64_t limit_ns, void* ws, size_t ws_bytes,
+                                       fs_stream_t stream);
 
 /*
  * One call for callers whose data live in HOST memory: copies x, y, a, b (and nothing

@@ -17,6 +17,7 @@ STATUS = {
     5: "FS_ERR_NEGATIVE_WEIGHT", 6: "FS_ERR_NONFINITE_INPUT", 7: "FS_ERR_MASS_MISMATCH",
     8: "FS_ERR_ZERO_MASS", 9: "FS_ERR_UNSUPPORTED_D", 10: "FS_ERR_WORKSPACE",
     11: "FS_ERR_TIMEOUT", 12: "FS_ERR_CUDA", 13: "FS_ERR_ALIGNMENT", 14: "FS_ERR_OPTION",
+    15: "FS_ERR_DEVICE_MEMORY",
 }
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
@@ -28,6 +29,7 @@ EXPORTS = (
     "fs_potentials_noalloc", "fs_screening_enable", "fs_solve", "fs_transport_workspace_bytes",
     "fs_transport_apply", "fs_hvp", "fs_divergence_workspace_bytes", "fs_divergence",
     "fs_multiscale_workspace_bytes", "fs_solve_multiscale", "fs_workspace_invalidate",
+    "fs_inject_error_word", "fs_check_bounded_wait",
 )
 
 VARIANTS = {"alternating": 0, "symmetric": 1}
@@ -145,6 +147,10 @@ def load():
     lib.fs_timing_get.restype = None
     lib.fs_potentials_noalloc.argtypes = [P, i32, vp, vp, vp, vp]
     lib.fs_potentials_noalloc.restype = ctypes.c_int
+    lib.fs_inject_error_word.argtypes = [ctypes.c_uint]
+    lib.fs_inject_error_word.restype = None
+    lib.fs_check_bounded_wait.argtypes = [ctypes.c_int64, vp, sz, vp]
+    lib.fs_check_bounded_wait.restype = ctypes.c_int
     lib.fs_launch_count.argtypes = []
     lib.fs_launch_count.restype = ctypes.c_int64
     _lib = lib

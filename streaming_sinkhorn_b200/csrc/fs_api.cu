@@ -18,6 +18,8 @@ namespace {
 
 thread_local char g_cuda_err[256] = "";
 std::atomic<int64_t> g_launches{0};
+// Error bits the next call ORs into its error word (fs_inject_error_word), 0 = none.
+std::atomic<unsigned> g_inject{0};
 
 struct CudaFail {};
 
@@ -1357,8 +1359,14 @@ void screening_probe(Ctx& c, bool rows_x) {
   if (static_cast<double>(kept) > 0.5 * all) c.no_screen = true;
 }
 
-// Drains the stream and reads the kernels' error word.
+// Drains the stream and reads the kernels' error word (after ORing in an armed injection).
 fs_status finish(Ctx& c) {
+  const unsigned inject = g_inject.exchange(0u);
+  if (inject) {
+    or_error_word_kernel<<<1, 32, 0, c.st>>>(err_ptr(c.scal), inject);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
   double tail[kEval + 3 - kErr];
   CK(cudaMemcpyAsync(tail, c.scal + kErr, sizeof(tail), cudaMemcpyDeviceToHost, c.st));
   CK(cudaStreamSynchronize(c.st));
@@ -1770,6 +1778,11 @@ fs_status potentials_impl(const fs_problem* p, int32_t n_iters, const float* g_i
   return solve_impl(p, &o, f, g, nullptr, ws, ws_bytes, stream, graphs_allowed);
 }
 
+// Records a CUDA error of another translation unit of the library for fs_last_cuda_error.
+void record_cuda_error(const char* what, cudaError_t e) {
+  snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", what, cudaGetErrorString(e));
+}
+
 }  // namespace fs
 
 extern "C" {
@@ -1791,6 +1804,8 @@ const char* fs_status_string(fs_status s) {
     case FS_ERR_CUDA: return "FS_ERR_CUDA: a CUDA runtime call failed";
     case FS_ERR_OPTION: return "FS_ERR_OPTION: a solve option is out of range";
     case FS_ERR_ALIGNMENT: return "FS_ERR_ALIGNMENT: device pointers must be 4-byte aligned";
+    case FS_ERR_DEVICE_MEMORY:
+      return "FS_ERR_DEVICE_MEMORY: the device could not commit the library's static scratch array";
   }
   return "unknown fs_status";
 }
@@ -2270,6 +2285,28 @@ fs_status fs_workspace_invalidate(void* ws, size_t ws_bytes, fs_stream_t stream)
     return FS_ERR_CUDA;
   }
   return FS_OK;
+}
+
+void fs_inject_error_word(unsigned bits) { fs::g_inject.store(bits); }
+
+fs_status fs_check_bounded_wait(int64_t limit_ns, void* ws, size_t ws_bytes, fs_stream_t stream) {
+  using namespace fs;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 ||
+      ws_bytes < kScalarDoubles * sizeof(double))
+    return FS_ERR_WORKSPACE;
+  if (limit_ns < 1000 || limit_ns > static_cast<int64_t>(kWaitLimitNs)) return FS_ERR_OPTION;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned* err = err_ptr(static_cast<double*>(ws));
+  return guarded(st, [&]() -> fs_status {
+    CK(cudaMemsetAsync(err, 0, sizeof(unsigned), st));
+    bounded_wait_check_kernel<<<1, 32, 0, st>>>(err, static_cast<unsigned long long>(limit_ns));
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    unsigned h = 0;
+    CK(cudaMemcpyAsync(&h, err, sizeof(h), cudaMemcpyDeviceToHost, st));
+    CK(cudaStreamSynchronize(st));
+    return h ? FS_ERR_TIMEOUT : FS_OK;
+  });
 }
 
 void fs_timing_enable(int on) {

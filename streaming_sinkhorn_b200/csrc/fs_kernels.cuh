@@ -1080,4 +1080,23 @@ __global__ void residual_finish_kernel(const double* row_acc, const double* col_
   }
 }
 
+// ---- error-path checks -------------------------------------------------------------------
+
+// ORs `bits` into a call's error word from the device, where a kernel whose bounded wait
+// expired would have set it (fault injection for the error path; no wait is involved).
+__global__ void or_error_word_kernel(unsigned* err, unsigned bits) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(err, bits);
+}
+
+// Self-check of the bounded mbarrier wait every pass kernel uses: one thread waits for the
+// first phase of a barrier that nothing arrives at (no copy or MMA is in flight), gives up
+// after limit_ns and sets kErrTimeout in the error word, as a pass kernel would.
+__global__ void bounded_wait_check_kernel(unsigned* err, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  if (!mbar_wait_bounded(&bar, 0, limit_ns)) atomicOr(err, kErrTimeout);
+}
+
 }  // namespace fs

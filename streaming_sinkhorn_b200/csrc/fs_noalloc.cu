@@ -1,8 +1,6 @@
 // fs_noalloc.cu -- fs_potentials_noalloc: the alternating solve with its scratch space taken
 // from a fixed-size array in device global memory that the library owns, so the caller
 // never has to allocate anything beyond its own inputs and outputs.
-#include <mutex>
-
 #include "../../include/fs.h"
 
 namespace fs {
@@ -12,37 +10,34 @@ namespace fs {
 fs_status potentials_impl(const fs_problem* p, int32_t n_iters, const float* g_init, float* f,
                           float* g, void* ws, size_t ws_bytes, fs_stream_t stream,
                           bool graphs_allowed);
+// Defined in fs_api.cu: keeps the text of a CUDA error for fs_last_cuda_error.
+void record_cuda_error(const char* what, cudaError_t e);
 }
 
 namespace {
 
-// The scratch space. Every device that loads the library holds these bytes until the
-// process exits; every call on a device reuses them.
+// The scratch space. Every device whose context has loaded this file's module holds these
+// bytes until the process exits; every call on a device reuses them.
 static __device__ __align__(256) unsigned char fs_noalloc_scratch[FS_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 128;
-std::mutex g_mu;
-void* g_scratch[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device, looked up once per device.
-// The array's name in host code is only a stand-in handle, so the address must come from
-// cudaGetSymbolAddress with that device current.
+// Device address of the scratch array in the current context. The array's name in host
+// code is only a stand-in handle, so the address must come from cudaGetSymbolAddress with
+// the device (and context) current that the kernels will run in. It is looked up on every
+// call, never cached: after cudaDeviceReset, or under another context of the same device,
+// the module is loaded anew and the array may sit at another address. Once the module is
+// loaded the lookup is a host-side table query. Under lazy module loading (the default
+// since CUDA 12.2) the first lookup in a context loads the module, which commits the
+// array's device memory; when the device cannot provide it the call returns
+// FS_ERR_DEVICE_MEMORY.
 fs_status scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  void* ptr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&ptr, fs_noalloc_scratch);
+  if (e != cudaSuccess || !ptr) {
+    fs::record_cuda_error("cudaGetSymbolAddress(fs_noalloc_scratch)", e);
     cudaGetLastError();
-    return FS_ERR_CUDA;
+    return e == cudaErrorMemoryAllocation ? FS_ERR_DEVICE_MEMORY : FS_ERR_CUDA;
   }
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, fs_noalloc_scratch) != cudaSuccess || !ptr) {
-      cudaGetLastError();
-      return FS_ERR_CUDA;
-    }
-    g_scratch[dev] = ptr;
-  }
-  *out = g_scratch[dev];
+  *out = ptr;
   return FS_OK;
 }
 

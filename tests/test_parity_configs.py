@@ -10,6 +10,7 @@ the iterate one step earlier), the gradient and the plan marginals on sampled ro
 properties that hold at any size (the column residual vanishes after a g-update).
 """
 import hashlib
+import math
 import os
 
 import numpy as np
@@ -83,6 +84,24 @@ def test_c5_full_run_matches_warm_restart(c5_run):
     assert_potential_close(g20.cpu().numpy(), g, "g", rel=1e-6)
 
 
+# Bound in exponent units (log2) for the clustered workloads at eps = 2^(-40/3), where the
+# potential bar 1e-4 max(1, |f|) is about 1.4 kappa^-1 and would hide the loss of a third of
+# a row's mass. One pass rounds each score z_ij = H_j - kappa |x_i - y_j|^2 a few times in
+# fp32 (|H| and the kept kappa-scaled distances stay below ~60 log2 units: log2 of the
+# weights ~ -20, kappa g within tens), about 8 * 2^-24 * 60 ~ 3e-5 per pass; the update is
+# non-expansive in the sup norm (|F(g) - F(g')| <= |g - g'|), so 40 passes add at most
+# ~1.2e-3; screening omits under 2^-24 of each row's sum (1e-7 log2 units). 1e-2 leaves
+# eight times that.
+KAPPA_BOUND_LOG2 = 1e-2
+
+
+def assert_exponent_close(got, ref, eps, name):
+    kappa = math.log2(math.e) / eps
+    err = kappa * np.abs(np.asarray(got, np.float64) - np.asarray(ref, np.float64))
+    assert err.max() <= KAPPA_BOUND_LOG2, (f"{name}: kappa |d{name}| = {err.max():.3e} log2 "
+                                           f"units at index {int(np.argmax(err))}")
+
+
 def test_c5_sampled_updates(c5_run):
     w, _, f, g, g_prev = c5_run
     rng = np.random.default_rng(0)
@@ -90,8 +109,42 @@ def test_c5_sampled_updates(c5_run):
     cols = np.sort(rng.choice(w.m, 1024, replace=False))
     f_ref = oracle.lse_update(w.x, w.y, w.b, g_prev, w.eps, rows=rows)
     assert_potential_close(f[rows], f_ref, "f")
+    assert_exponent_close(f[rows], f_ref, w.eps, "f")
     g_ref = oracle.lse_update(w.y, w.x, w.a, f, w.eps, rows=cols)
     assert_potential_close(g[cols], g_ref, "g")
+    assert_exponent_close(g[cols], g_ref, w.eps, "g")
+
+
+def test_clustered_32k_twenty_iterations_against_stored_oracle():
+    """The 2^20-point recipe (1000 clusters of std 0.01, eps = 2^(-40/3), 20 iterations,
+    screened) at 2^15 points, where the oracle runs all 20 iterations: the drift of the
+    screened fp32 iterate against the fp64 one over the whole solve, element by element."""
+    path = os.path.join(GOLDEN, "cluster_32k_d3.npz")
+    z = np.load(path)
+    w = workloads.clustered_cube(n=1 << 15, d=3, k=1000, std=0.01, seed=4,
+                                 eps=2.0 ** (-40.0 / 3.0), n_iters=20)
+    assert str(z["digest"]) == digest(w), "inputs drifted from the stored oracle run"
+    assert int(z["n_iters"]) == w.n_iters and float(z["eps"]) == w.eps
+    x, y, a, b = inputs(w)
+    fs.timing_enable(True)
+    fs.timing_reset()
+    try:
+        f, g = fs.potentials(x, y, a, b, eps=w.eps, n_iters=w.n_iters)
+        t = fs.timing_get()["lse_pass"]
+    finally:
+        fs.timing_enable(False)
+    assert 0 < t["evaluated"] < 0.5 * t["pairs"], "the solve did not screen"
+    fn, gn = f.cpu().numpy(), g.cpu().numpy()
+    assert_potential_close(fn, z["f"], "f")
+    assert_potential_close(gn, z["g"], "g")
+    assert_exponent_close(fn, z["f"], w.eps, "f")
+    assert_exponent_close(gn, z["g"], w.eps, "g")
+    c = fs.cost(x, y, f, g, a, b, eps=w.eps).item()
+    assert_cost_close(c, float(z["cost"]))
+    gx = fs.grad_x(x, y, g, a, b, eps=w.eps).cpu().numpy()
+    assert_grad_close(gx[z["grad_rows"]], z["grad"])
+    res = fs.marginal_residual(x, y, f, g, a, b, eps=w.eps).cpu().numpy()
+    np.testing.assert_allclose(res[:2], z["residual"][:2], rtol=2e-2, atol=residual_tolerance(w))
 
 
 def test_c5_sampled_grad_and_marginals(c5_run):

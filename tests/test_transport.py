@@ -69,27 +69,45 @@ def test_hvp_matches_oracle(shape):
     hv, rep = fs.hvp(x, y, dev(g32), dev(v), a, b, eps=w.eps, cg_max_iter=500, cg_tol=1e-7)
     ref = oracle.hvp(w.x, w.y, w.a, w.b, w.eps, g32, v)
     assert rep["cg_iters"] >= 1
-    close(hv.cpu().numpy(), ref, 2e-3)
+    close(hv.cpu().numpy(), ref, HVP_TOL)
+
+
+HVP_TOL = 2e-3  # elementwise, relative to the largest |(Hv)_i|: test_hvp_matches_oracle
 
 
 def test_hvp_is_symmetric_on_the_gpu():
+    """u.(Hv) = v.(Hu) (the Hessian is symmetric) and both equal the oracle's value.
+
+    Error model: every entry of the GPU's Hv is within HVP_TOL max|H_ref v| of the oracle's
+    (the bar of test_hvp_matches_oracle), so |u.(Hv) - u.(H_ref v)| <= HVP_TOL max|H_ref v|
+    |u|_1, and the GPU's asymmetry |u.(Hv) - v.(Hu)| is at most the sum of that bound for
+    (u, v) and for (v, u) plus the oracle's own (fp64) asymmetry. u is taken correlated with
+    v (u = v + w / 2), so that u.(Hv) ~ v.(Hv) > 0 sums coherently and the bound is a few
+    1e-3 of the value, while a dropped or one-sided term of H changes it by O(1).
+    """
     w = problem(200, 180, 3, 0.2, seed=17)
     x, y, a, b = inputs(w)
     _, g = oracle.potentials(w.x, w.y, w.a, w.b, w.eps, 400)
-    gd = dev(g.astype(np.float32))
+    g32 = g.astype(np.float32)
+    gd = dev(g32)
     rng = np.random.default_rng(2)
-    u = rng.standard_normal((200, 3)).astype(np.float32)
     v = rng.standard_normal((200, 3)).astype(np.float32)
+    u = (v + 0.5 * rng.standard_normal((200, 3))).astype(np.float32)
     hu, _ = fs.hvp(x, y, gd, dev(u), a, b, eps=w.eps, cg_max_iter=500, cg_tol=1e-7)
     hv, _ = fs.hvp(x, y, gd, dev(v), a, b, eps=w.eps, cg_max_iter=500, cg_tol=1e-7)
-    lhs = float((u * hv.cpu().numpy()).sum())
-    rhs = float((v * hu.cpu().numpy()).sum())
-    # a sum of 600 products of entries accurate to ~1e-3 of the largest (fp32 conjugate
-    # gradients): agreement to a few 1e-3 of the value, while a dropped or one-sided term
-    # breaks the symmetry by O(1)
-    ref = float((u * oracle.hvp(w.x, w.y, w.a, w.b, w.eps, g.astype(np.float32), v)).sum())
-    assert lhs == pytest.approx(rhs, rel=3e-2)
-    assert lhs == pytest.approx(ref, rel=3e-2) and rhs == pytest.approx(ref, rel=3e-2)
+    hu, hv = hu.cpu().numpy().astype(np.float64), hv.cpu().numpy().astype(np.float64)
+    hu_ref = oracle.hvp(w.x, w.y, w.a, w.b, w.eps, g32, u)
+    hv_ref = oracle.hvp(w.x, w.y, w.a, w.b, w.eps, g32, v)
+    u64, v64 = u.astype(np.float64), v.astype(np.float64)
+    b_uv = HVP_TOL * np.abs(hv_ref).max() * np.abs(u64).sum()
+    b_vu = HVP_TOL * np.abs(hu_ref).max() * np.abs(v64).sum()
+    ref_uv, ref_vu = float((u64 * hv_ref).sum()), float((v64 * hu_ref).sum())
+    lhs, rhs = float((u64 * hv).sum()), float((v64 * hu).sum())
+    assert abs(ref_uv - ref_vu) <= 1e-9 * abs(ref_uv)  # the oracle is symmetric
+    assert abs(lhs - ref_uv) <= b_uv, (lhs, ref_uv, b_uv)
+    assert abs(rhs - ref_vu) <= b_vu, (rhs, ref_vu, b_vu)
+    assert abs(lhs - rhs) <= b_uv + b_vu + abs(ref_uv - ref_vu), (lhs, rhs)
+    assert b_uv + b_vu <= 0.03 * abs(ref_uv)  # the check can see an O(1) asymmetry
 
 
 def test_hvp_screened_equals_dense():
