@@ -327,6 +327,8 @@ constexpr int kQueue = 151;   // ints: tiles per unit C and unit count U of the 
 constexpr int kKept = 152;    // int64: kept tiles K of the last queue plan
 constexpr int kPotChange = 153;  // unsigned: float bits of the largest potential change
 constexpr int kCgDots = 156;     // [4] float64: the HVP solve's dot products and sums
+constexpr int kPayMax = 160;     // unsigned: float bits of the largest |payload| of an apply pass
+constexpr int kPayInv = 161;     // float: 1 / s of that pass's payload image
 // [kSortMemoWords] uint64 from here: the record of the last sort done in this workspace,
 // which prepare() does not clear (everything before it is cleared at every call)
 constexpr int kSortMemo = 240;
@@ -341,7 +343,9 @@ struct Layout {
   int Dtc;     // padded dimension of the tensor-core path, 0 if unused
   int64_t tx, ty;  // points of x and y padded to whole 128-point tiles (tensor-core path)
   size_t off_scalars, off_kx, off_ky, off_lwx, off_lwy, off_part, total;
-  size_t off_rimg_x, off_kimg_x, off_rimg_y, off_kimg_y, off_nrm_x, off_nrm_y, off_hy_x, off_hy_y;
+  size_t off_img_x, off_img_y, off_nrm_x, off_nrm_y, off_hy_x, off_hy_y;
+  // apply passes (d > 16): the rows' LSE2 offsets and plan masses, a payload image
+  size_t off_tc_lse, off_tc_mass, off_tc_pay;
   // spatial order and screening (FMA path): permutations, sort keys, per-tile boxes and bias
   // maxima, and the LSE2 of every row in its last pass
   bool sorted;
@@ -399,8 +403,10 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0, bool co
   L.tx = tc_pad(n);
   L.ty = tc_pad(m);
   if (L.Dtc) {
+    // potential passes: (max, sum) per split and row; apply passes: (sum, NC channels)
+    const int64_t nc = std::max<int64_t>(L.Dtc, kPayChannels);
     for (const TcPlan& tp : {make_tc_plan(n, m, L.Dtc, sms), make_tc_plan(m, n, L.Dtc, sms)})
-      if (tp.n_splits > 1) pf = std::max<int64_t>(pf, 2 * tp.n_splits * tp.rows_pad);
+      if (tp.n_splits > 1) pf = std::max<int64_t>(pf, (1 + nc) * tp.n_splits * tp.rows_pad);
   }
   L.part_floats = pf;
   size_t o = 0;
@@ -417,14 +423,10 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0, bool co
   L.off_part = o;
   o = align_up(o + static_cast<size_t>(pf) * sizeof(float));
   if (L.Dtc) {
-    const size_t kbytes = static_cast<size_t>(3 * L.Dtc) * 2;  // fp16 per point per image
-    L.off_rimg_x = o;
+    const size_t kbytes = static_cast<size_t>(2 * L.Dtc) * 2;  // [hi | lo] fp16 per point
+    L.off_img_x = o;
     o = align_up(o + static_cast<size_t>(L.tx) * kbytes);
-    L.off_kimg_x = o;
-    o = align_up(o + static_cast<size_t>(L.tx) * kbytes);
-    L.off_rimg_y = o;
-    o = align_up(o + static_cast<size_t>(L.ty) * kbytes);
-    L.off_kimg_y = o;
+    L.off_img_y = o;
     o = align_up(o + static_cast<size_t>(L.ty) * kbytes);
     L.off_nrm_x = o;
     o = align_up(o + static_cast<size_t>(L.tx) * sizeof(float));
@@ -434,6 +436,15 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0, bool co
     o = align_up(o + static_cast<size_t>(L.tx) * sizeof(float));
     L.off_hy_y = o;
     o = align_up(o + static_cast<size_t>(L.ty) * sizeof(float));
+    const int64_t tmax = std::max(L.tx, L.ty);
+    L.off_tc_lse = o;
+    o = align_up(o + static_cast<size_t>(tmax) * sizeof(float));
+    L.off_tc_mass = o;
+    o = align_up(o + static_cast<size_t>(tmax) * sizeof(float));
+    if (acc_ch > 0) {
+      L.off_tc_pay = o;
+      o = align_up(o + static_cast<size_t>(tmax) * 2 * kPayChannels * 2);
+    }
   }
   if (L.sorted) {
     int64_t sn = kSortSmem;
@@ -688,12 +699,17 @@ struct TcKernel {
   }
 };
 
+// Resident CTAs per SM of the potential pass: shared memory's limit, and TMEM's (each CTA
+// allocates kTcTmemCols of the SM's 512 columns; a CTA beyond that would wait in its
+// allocation).
 int occupancy_tc(int Dtc) {
+  int n = 1;
   switch (Dtc) {
-    case 32: return TcKernel<32>::occupancy();
-    case 48: return TcKernel<48>::occupancy();
-    default: return TcKernel<64>::occupancy();
+    case 32: n = TcKernel<32>::occupancy(); break;
+    case 48: n = TcKernel<48>::occupancy(); break;
+    default: n = TcKernel<64>::occupancy(); break;
   }
+  return std::max(1, std::min(n, static_cast<int>(512u / kTcTmemCols)));
 }
 
 void launch_tc(int Dtc, const PassParams& P, const TcParams& T, const TcPlan& pl, cudaStream_t st) {
@@ -704,12 +720,53 @@ void launch_tc(int Dtc, const PassParams& P, const TcParams& T, const TcPlan& pl
   }
 }
 
+template <int Dtc, int NC, int MODE>
+struct TcApplyKernel {
+  static constexpr auto fn = lse_apply_tc_kernel<Dtc, NC, MODE>;
+  static constexpr size_t SMEM = TcApplyShape<Dtc, NC, MODE>::SMEM;
+  static void launch(const PassParams& P, const TcParams& T, const TcApply& A, const TcPlan& pl,
+                     cudaStream_t st) {
+    static bool done = false;  // idempotent, so a race between threads is harmless
+    if (!done) {
+      CK(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(SMEM)));
+      done = true;
+    }
+    dim3 grid(static_cast<unsigned>(pl.row_blocks), static_cast<unsigned>(pl.n_splits));
+    fn<<<grid, kTcThreads, SMEM, st>>>(P, T, A);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (pl.n_splits > 1) {
+      tc_apply_combine_kernel<NC, MODE><<<static_cast<unsigned>(ceil_div(P.n_rows, 256)), 256, 0,
+                                          st>>>(P, A);
+      CK(cudaGetLastError());
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+    }
+  }
+};
+
+void launch_apply_tc(int Dtc, int mode, const PassParams& P, const TcParams& T, const TcApply& A,
+                     const TcPlan& pl, cudaStream_t st) {
+  if (mode == kApplyGrad) {
+    switch (Dtc) {
+      case 32: TcApplyKernel<32, 32, kApplyGrad>::launch(P, T, A, pl, st); break;
+      case 48: TcApplyKernel<48, 48, kApplyGrad>::launch(P, T, A, pl, st); break;
+      default: TcApplyKernel<64, 64, kApplyGrad>::launch(P, T, A, pl, st); break;
+    }
+  } else {
+    switch (Dtc) {
+      case 32: TcApplyKernel<32, kPayChannels, kApplyPay>::launch(P, T, A, pl, st); break;
+      case 48: TcApplyKernel<48, kPayChannels, kApplyPay>::launch(P, T, A, pl, st); break;
+      default: TcApplyKernel<64, kPayChannels, kApplyPay>::launch(P, T, A, pl, st); break;
+    }
+  }
+}
+
 template <int Dtc>
-void launch_images(const float* pts, int64_t count, int d, const TcCenter& ctr, float scale,
-                   unsigned char* rimg, unsigned char* kimg, float* nrm, int64_t pad,
-                   cudaStream_t st) {
-  build_images_kernel<Dtc><<<static_cast<unsigned>(ceil_div(pad, 256)), 256, 0, st>>>(
-      pts, count, d, ctr, scale, rimg, kimg, nrm, pad);
+void launch_image(const float* pts, int64_t count, int d, const TcCenter& ctr, float scale,
+                  unsigned char* img, float* nrm, int64_t pad, cudaStream_t st) {
+  build_image_kernel<Dtc><<<static_cast<unsigned>(ceil_div(pad, 256)), 256, 0, st>>>(
+      pts, count, d, ctr, scale, img, nrm, pad);
   CK(cudaGetLastError());
   g_launches.fetch_add(1, std::memory_order_relaxed);
 }
@@ -851,9 +908,13 @@ struct Ctx {
   double kappa;
   Timer* timer;
   bool use_tc;    // potential and marginal passes on the tensor cores
-  unsigned char *rimg_x, *kimg_x, *rimg_y, *kimg_y;
+  unsigned char *img_x, *img_y;
   float *nrm_x, *nrm_y, *hy_x, *hy_y;
+  float *tc_lse, *tc_mass;      // apply passes: the rows' LSE2 offsets and plan masses
+  unsigned char* tc_pay;        // apply passes: payload image
   float c2;       // 2 kappa / s^2
+  float tc_scale;  // s: the images' power-of-two scale
+  TcCenter tc_ctr;  // the centre the images were built about
   int *perm_x, *perm_y;         // sorted slot -> original index (NULL when unsorted)
   unsigned *code_x, *code_y;    // Morton codes in sorted order (NULL when unsorted)
   uint64_t* sortkeys;
@@ -908,10 +969,11 @@ void carve(Ctx& c, void* ws) {
     c.hvp = reinterpret_cast<float*>(c.ws + c.L.off_hvp);
   }
   if (c.L.Dtc) {
-    c.rimg_x = c.ws + c.L.off_rimg_x;
-    c.kimg_x = c.ws + c.L.off_kimg_x;
-    c.rimg_y = c.ws + c.L.off_rimg_y;
-    c.kimg_y = c.ws + c.L.off_kimg_y;
+    c.img_x = c.ws + c.L.off_img_x;
+    c.img_y = c.ws + c.L.off_img_y;
+    c.tc_lse = reinterpret_cast<float*>(c.ws + c.L.off_tc_lse);
+    c.tc_mass = reinterpret_cast<float*>(c.ws + c.L.off_tc_mass);
+    if (c.L.off_tc_pay) c.tc_pay = c.ws + c.L.off_tc_pay;
     c.nrm_x = reinterpret_cast<float*>(c.ws + c.L.off_nrm_x);
     c.nrm_y = reinterpret_cast<float*>(c.ws + c.L.off_nrm_y);
     c.hy_x = reinterpret_cast<float*>(c.ws + c.L.off_hy_x);
@@ -1096,18 +1158,21 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
     const double bound = static_cast<double>(fmaxabs) + cmax;
     const double scale = bound > 0.0 ? std::exp2(std::floor(std::log2(16384.0 / bound))) : 1.0;
     c.c2 = static_cast<float>(2.0 * c.kappa / (scale * scale));
+    c.tc_ctr = ctr;
+    c.tc_scale = static_cast<float>(scale);
+    const float sc = static_cast<float>(scale);
     switch (c.L.Dtc) {
       case 32:
-        launch_images<32>(p->x, p->n, p->d, ctr, static_cast<float>(scale), c.rimg_x, c.kimg_x, c.nrm_x, c.L.tx, c.st);
-        launch_images<32>(p->y, p->m, p->d, ctr, static_cast<float>(scale), c.rimg_y, c.kimg_y, c.nrm_y, c.L.ty, c.st);
+        launch_image<32>(p->x, p->n, p->d, ctr, sc, c.img_x, c.nrm_x, c.L.tx, c.st);
+        launch_image<32>(p->y, p->m, p->d, ctr, sc, c.img_y, c.nrm_y, c.L.ty, c.st);
         break;
       case 48:
-        launch_images<48>(p->x, p->n, p->d, ctr, static_cast<float>(scale), c.rimg_x, c.kimg_x, c.nrm_x, c.L.tx, c.st);
-        launch_images<48>(p->y, p->m, p->d, ctr, static_cast<float>(scale), c.rimg_y, c.kimg_y, c.nrm_y, c.L.ty, c.st);
+        launch_image<48>(p->x, p->n, p->d, ctr, sc, c.img_x, c.nrm_x, c.L.tx, c.st);
+        launch_image<48>(p->y, p->m, p->d, ctr, sc, c.img_y, c.nrm_y, c.L.ty, c.st);
         break;
       default:
-        launch_images<64>(p->x, p->n, p->d, ctr, static_cast<float>(scale), c.rimg_x, c.kimg_x, c.nrm_x, c.L.tx, c.st);
-        launch_images<64>(p->y, p->m, p->d, ctr, static_cast<float>(scale), c.rimg_y, c.kimg_y, c.nrm_y, c.L.ty, c.st);
+        launch_image<64>(p->x, p->n, p->d, ctr, sc, c.img_x, c.nrm_x, c.L.tx, c.st);
+        launch_image<64>(p->y, p->m, p->d, ctr, sc, c.img_y, c.nrm_y, c.L.ty, c.st);
         break;
     }
   }
@@ -1152,7 +1217,7 @@ void set_bias(Ctx& c, bool cloud_x, const float* pot) {
 
 // One streaming pass with rows from cloud x (rows_x) or y, keys from the other cloud.
 void run_pass_tc(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out,
-                 float* marg_out, double* acc) {
+                 float* marg_out, double* acc, float* lse_out = nullptr, int timed_kind = -1) {
   const fs_problem* p = c.p;
   const int64_t n_rows = rows_x ? p->n : p->m, n_keys = rows_x ? p->m : p->n;
   const TcPlan pl = make_tc_plan(n_rows, n_keys, c.L.Dtc, c.sms);
@@ -1178,13 +1243,14 @@ void run_pass_tc(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_
   P.err = err_ptr(c.scal);
   P.hy_out = rows_x ? c.hy_x : c.hy_y;
   P.nrm = rows_x ? c.nrm_x : c.nrm_y;
+  P.lse_out = lse_out;
   if (kind == kPot) {
     P.alpha = c.alpha;
     if (rows_x && c.defer_x) P.defer_h = c.defer;  // installed after the other pass
   }
   TcParams T{};
-  T.row_img = rows_x ? c.rimg_x : c.rimg_y;
-  T.key_img = rows_x ? c.kimg_y : c.kimg_x;
+  T.row_img = rows_x ? c.img_x : c.img_y;
+  T.key_img = rows_x ? c.img_y : c.img_x;
   T.key_hy = rows_x ? c.hy_y : c.hy_x;
   T.row_nrm = rows_x ? c.nrm_x : c.nrm_y;
   T.key_tiles = pl.key_tiles;
@@ -1193,11 +1259,91 @@ void run_pass_tc(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_
   const double pairs = static_cast<double>(n_rows) * static_cast<double>(n_keys);
   int ti = c.timer->begin();
   launch_tc(c.L.Dtc, P, T, pl, c.st);
-  c.timer->end(ti, kind == kMarg ? kTMarg : kTLse, pairs);
+  c.timer->end(ti, timed_kind >= 0 ? timed_kind : (kind == kMarg ? kTMarg : kTLse), pairs);
   if (pl.n_splits > 1) {
     ti = c.timer->begin();
     FS_DISPATCH_D(c.L.D, launch_combine_d, P, false, c.st);
     c.timer->end(ti, kTCombine, 0.0);
+  }
+}
+
+// An apply pass on the tensor cores (d > 16), rows from cloud x (rows_x) or y:
+//   mode kApplyGrad: out = grad (n_rows x d) at the plan of (F(g), g), g carried by the keys;
+//   mode kApplyPay:  out (n_rows x k, row stride out_stride) = P pay, pay (n_keys x k, row
+//     stride pay_stride), P the plan of (pot_in, key potentials), or of (F(g), g) when pot_in
+//     is NULL; channels go kPayChannels at a time.
+// First a potential-type pass writes every row's LSE2 (and, with pot_in, its plan mass),
+// then the apply pass streams the keys again at those fixed offsets.
+void run_apply_tc(Ctx& c, bool rows_x, int mode, const float* pot_in, const float* pay, int k,
+                  int pay_stride, float* out, int out_stride) {
+  const fs_problem* p = c.p;
+  const int64_t n_rows = rows_x ? p->n : p->m, n_keys = rows_x ? p->m : p->n;
+  const int tk = mode == kApplyGrad ? kTGrad : kTMarg;
+  if (pot_in)
+    run_pass_tc(c, rows_x, kMarg, pot_in, nullptr, c.tc_mass, nullptr, c.tc_lse, tk);
+  else
+    run_pass_tc(c, rows_x, kLse, nullptr, nullptr, nullptr, nullptr, c.tc_lse, tk);
+  const TcPlan pl = make_tc_plan(n_rows, n_keys, c.L.Dtc, c.sms);
+  PassParams P{};
+  P.n_rows = n_rows;
+  P.n_splits = pl.n_splits;
+  P.rows_pad = pl.rows_pad;
+  P.kind = kGrad;
+  P.d_real = p->d;
+  P.kappa = c.kappa;
+  P.kappa_f = static_cast<float>(c.kappa);
+  P.inv_kappa_f = static_cast<float>(1.0 / c.kappa);
+  P.eps_ln2 = 1.0 / c.kappa;
+  P.w = rows_x ? p->a : p->b;
+  P.w_uniform = static_cast<float>(1.0 / n_rows);
+  P.part_l = c.part;
+  P.part_a = c.part + static_cast<int64_t>(pl.n_splits) * pl.rows_pad;
+  P.err = err_ptr(c.scal);
+  TcParams T{};
+  T.row_img = rows_x ? c.img_x : c.img_y;
+  T.key_img = rows_x ? c.img_y : c.img_x;
+  T.key_hy = rows_x ? c.hy_y : c.hy_x;
+  T.row_nrm = rows_x ? c.nrm_x : c.nrm_y;
+  T.key_tiles = pl.key_tiles;
+  T.tiles_per_split = pl.tiles_per_split;
+  T.c2 = c.c2;
+  TcApply A{};
+  A.row_lse = c.tc_lse;
+  A.row_mass = pot_in ? c.tc_mass : nullptr;
+  A.x = rows_x ? p->x : p->y;
+  A.inv_key_scale = 1.0f / c.tc_scale;
+  memcpy(A.ctr, c.tc_ctr.c, sizeof(A.ctr));
+  const double pairs = static_cast<double>(n_rows) * static_cast<double>(n_keys);
+  if (mode == kApplyGrad) {
+    A.out = out;
+    A.out_stride = out_stride;
+    int ti = c.timer->begin();
+    launch_apply_tc(c.L.Dtc, mode, P, T, A, pl, c.st);
+    c.timer->end(ti, tk, pairs);
+    return;
+  }
+  unsigned* mx = reinterpret_cast<unsigned*>(c.scal + kPayMax);
+  float* inv = reinterpret_cast<float*>(c.scal + kPayInv);
+  const int64_t kpad = rows_x ? c.L.ty : c.L.tx;
+  A.pay_img = c.tc_pay;
+  A.pay_inv_scale = inv;
+  for (int c0 = 0; c0 < k; c0 += kPayChannels) {
+    const int kc = std::min(kPayChannels, k - c0);
+    CK(cudaMemsetAsync(mx, 0, sizeof(unsigned), c.st));
+    pay_maxabs_kernel<<<reduce_blocks(n_keys * kc, c.sms), 256, 0, c.st>>>(pay + c0, n_keys, kc,
+                                                                          pay_stride, mx);
+    CK(cudaGetLastError());
+    build_pay_image_kernel<kPayChannels><<<static_cast<unsigned>(ceil_div(kpad, 256)), 256, 0,
+                                           c.st>>>(pay + c0, n_keys, kpad, kc, pay_stride, mx,
+                                                   c.tc_pay, inv);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(2, std::memory_order_relaxed);
+    A.out = out + c0;
+    A.out_k = kc;
+    A.out_stride = out_stride;
+    int ti = c.timer->begin();
+    launch_apply_tc(c.L.Dtc, mode, P, T, A, pl, c.st);
+    c.timer->end(ti, tk, pairs);
   }
 }
 
@@ -1217,6 +1363,10 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
               float* grad_out, double* acc, bool history = false, const PassExtra* ex = nullptr) {
   if (c.use_tc && kind != kGrad) {
     run_pass_tc(c, rows_x, kind, pot_in, pot_out, marg_out, acc);
+    return;
+  }
+  if (c.use_tc && kind == kGrad && !ex) {
+    run_apply_tc(c, rows_x, kApplyGrad, nullptr, nullptr, 0, 0, grad_out, c.p->d);
     return;
   }
   const fs_problem* p = c.p;
@@ -1451,6 +1601,10 @@ double check_potential(Ctx& c, const float* f, const float* g) {
 // mass is then its weight). The keys must carry their biases. Channels go 16 at a time.
 void transport_pass(Ctx& c, bool rows_x, const float* pot_in, const float* pay, int k, int stride,
                     float* out, int out_stride, const float* row_v = nullptr) {
+  if (c.use_tc && !row_v) {
+    run_apply_tc(c, rows_x, kApplyPay, pot_in, pay, k, stride, out, out_stride);
+    return;
+  }
   const int64_t n_keys = rows_x ? c.p->m : c.p->n;
   const int64_t pairs = rows_x ? c.L.py : c.L.px;
   for (int c0 = 0; c0 < k; c0 += kTransportChannels) {
@@ -1621,14 +1775,13 @@ fs_status transport_impl(const fs_problem* p, const float* f, const float* g, in
   Ctx c{};
   fs_status s = begin(c, p, ws, ws_bytes, stream, kTransportChannels);
   if (s != FS_OK) return s;
-  if (p->d > 16) return FS_ERR_UNSUPPORTED_D;
   if (!f || !g || !u || !out) return FS_ERR_NULL;
   if (!aligned4(f) || !aligned4(g) || !aligned4(u) || !aligned4(out)) return FS_ERR_ALIGNMENT;
   if (k < 1 || (transpose != 0 && transpose != 1)) return FS_ERR_OPTION;
   Timer timer(c.st);
   c.timer = &timer;
   return guarded(c.st, [&]() -> fs_status {
-    fs_status r = prepare_all(c, {{f, p->n}, {g, p->m}}, false);
+    fs_status r = prepare_all(c, {{f, p->n}, {g, p->m}}, true);
     if (r != FS_OK) return r;
     if (!transpose) {
       set_bias(c, false, g);  // keys y carry g; rows x carry f
@@ -2072,7 +2225,7 @@ fs_status fs_solve_multiscale(const fs_problem* p, const fs_solve_options* opt,
 }
 
 size_t fs_transport_workspace_bytes(const fs_problem* p) {
-  if (!fs::shape_ok(p) || p->d > 16) return 0;
+  if (!fs::shape_ok(p) || p->d > FS_MAX_D) return 0;
   return fs::make_layout(p->n, p->m, p->d, fs::num_sms_current(), fs::kTransportChannels,
                          p->cost == FS_COST_COSINE).total;
 }
@@ -2100,7 +2253,7 @@ fs_status fs_grad_x(const fs_problem* p, const float* g, float* grad_x, void* ws
   Timer timer(c.st);
   c.timer = &timer;
   return guarded(c.st, [&]() -> fs_status {
-    fs_status r = prepare_all(c, {{g, p->m}}, false);
+    fs_status r = prepare_all(c, {{g, p->m}}, true);
     if (r != FS_OK) return r;
     set_bias(c, false, g);
     run_pass(c, true, kGrad, nullptr, nullptr, nullptr, grad_x, nullptr);

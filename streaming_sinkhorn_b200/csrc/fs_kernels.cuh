@@ -59,7 +59,8 @@ constexpr int kPairPad = 128;  // key pairs are padded to a multiple of this
 // columns; it never sets the running offset.
 constexpr float kEmptyCut = -1.0e29f;
 
-enum PassKind : int { kPot = 0, kMarg = 1, kGrad = 2 };
+// kLse: the row's LSE2 only (to lse_out), the fixed offset of a tensor-core apply pass.
+enum PassKind : int { kPot = 0, kMarg = 1, kGrad = 2, kLse = 3 };
 
 struct PassParams {
   const float* keys;        // streamed cloud, packed
@@ -105,7 +106,8 @@ struct PassParams {
   const float* lse_prev;    // LSE2 of every query row in its previous pass (sorted order)
   float log2_keys;          // log2(number of keys)
   float skip_margin;        // log2 units below a row's lower bound under which tiles drop
-  float* lse_out;           // kPot: LSE2 of every query row (sorted order)
+  float* lse_out;           // kPot, kLse (and kMarg when set): LSE2 of every query row
+                            // (sorted order)
   int* dmin_out;            // kPot: ordered int, smallest change of the H this pass writes
   unsigned long long* evaluated;  // pairs evaluated (after screening)
   // queue mode (screened passes): kept-tile bit masks and the unit plan
@@ -193,6 +195,7 @@ __device__ __forceinline__ void finish_marg(const PassParams& P, int64_t i, doub
   double r = 0.0;
   if (w > 0.0) r = w * exp2(P.kappa * static_cast<double>(P.pot_in[oi]) + lse2);
   if (P.marg_out) P.marg_out[oi] = static_cast<float>(r);
+  if (P.lse_out) P.lse_out[i] = static_cast<float>(lse2);
   dev = fabs(r - w);
   mass = r;
 }
@@ -226,7 +229,8 @@ __device__ __forceinline__ void reduce_dmin(float v, int* out) {
   if ((threadIdx.x & 31) == 0 && out) atomicMin(out, float_ord(v));
 }
 
-// Block-wide sum/max of the marginal deviations, then one atomic per block.
+// Block-wide sum/max of the marginal deviations, then one atomic per block (none when acc is
+// NULL: a pass that only wants the per-row marginals). Every thread of the block calls it.
 __device__ __forceinline__ void block_reduce_marg(double dev_sum, double dev_max, double mass,
                                                   double* acc) {
   __shared__ double sh[3][32];
@@ -248,7 +252,7 @@ __device__ __forceinline__ void block_reduce_marg(double dev_sum, double dev_max
     s = warp_sum(s);
     mx = warp_max(mx);
     ms = warp_sum(ms);
-    if (lane == 0) {
+    if (lane == 0 && acc) {
       atomicAdd(&acc[0], s);
       atomic_max_nonneg(&acc[1], mx);
       atomicAdd(&acc[2], ms);
@@ -310,6 +314,8 @@ __device__ __forceinline__ void merge_row(const PassParams& P, int64_t i, int64_
     finish_acc(P, i, a, l, lse2);
   } else if (P.kind == kPot) {
     dmin = fminf(dmin, finish_pot<D>(P, i, lse2));
+  } else if (P.kind == kLse) {
+    P.lse_out[i] = static_cast<float>(lse2);
   } else {
     double dv, ms;
     finish_marg(P, i, lse2, dv, ms);

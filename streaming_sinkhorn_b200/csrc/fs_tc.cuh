@@ -1,30 +1,40 @@
-// fs_tc.cuh -- the streaming pass for d > 16 on the tcgen05 tensor cores (sm_100a).
+// fs_tc.cuh -- the streaming passes for d > 16 on the tcgen05 tensor cores (sm_100a).
 //
-// For wide points the score is a real contraction, so the pass uses the attention form of
+// For wide points the score is a real contraction, so the passes use the attention form of
 // the update (FlashSinkhorn summary, Methodology section 1): with the clouds centred,
 //     z_ij = hy_j + 2 kappa x_i.y_j - kappa |x_i|^2,    hy_j = H_j - kappa |y_j|^2,
 // and x.y is computed by the tensor cores for a 128-row block against 128-column key
 // tiles. To keep float32-level accuracy the inputs are scaled by a power of two s and
-// split into fp16 halves, u = hi + lo (hi = fp16(u), lo = fp16(u - hi)); the MMA takes
-//     A = [hi_x | lo_x | hi_x],  B = [hi_y | hi_y | lo_y]   (K = 3D),
-// so one K = 3D product gives hi.hi + lo.hi + hi.lo = s^2 x.y up to ~2^-22 relative, with
-// fp32 accumulation in tensor memory.
+// split into fp16 halves, u = hi + lo (hi = fp16(u), lo = fp16(u - hi)); each 16-wide
+// K-step issues three MMAs, hi_x.hi_y + lo_x.hi_y + hi_x.lo_y = s^2 x.y up to ~2^-22
+// relative, with fp32 accumulation in tensor memory.
 //
-// Operand images. Each cloud is stored twice in global memory (as rows with the A order,
-// as keys with the B order), already in the shared-memory layout the MMA reads: per tile of
-// 128 points, 8x8-element core matrices (8 points x 16 bytes of K) stored K-block-major,
-// core(g, kb) at byte (kb * 16 + g) * 128. A K-step of 16 elements is two consecutive
-// K-blocks (leading-byte offset 16 * 128 B); consecutive 8-point groups are 128 B apart
-// (stride-byte offset). A tile is therefore one contiguous block that a single TMA bulk copy
-// moves into shared memory.
+// Operand images. Each cloud is stored once in global memory as [hi | lo] (K = 2D fp16 per
+// point), already in the shared-memory layout the MMA reads: per tile of 128 points,
+// 8x8-element core matrices (8 points x 16 bytes of K) stored K-block-major, core(g, kb) at
+// byte (kb * 16 + g) * 128. For the score MMA (points along M or N, coordinates along K)
+// that is the K-major layout: a K-step of 16 elements is two consecutive K-blocks
+// (leading-byte offset 16 * 128 B), consecutive 8-point groups are 128 B apart (stride-byte
+// offset). Read the other way (points along K, coordinates along N) the same bytes are the
+// MN-major layout: 8 consecutive points of one core matrix are 16-byte rows, the next 8
+// points are 128 B on (leading-byte offset), the next 8 coordinates 16 * 128 B on
+// (stride-byte offset). The apply pass uses it so as the B operand of sum_j p_ij y_j. A
+// tile is one contiguous block that a single TMA bulk copy moves into shared memory.
 //
-// Kernel: one CTA per 128-row block and column split, 10 warps with fixed roles. Warp 8
-// streams key tiles (B image + hy) through a 3-stage ring with TMA bulk copies; warp 9
-// issues the MMAs of tile t into one of two TMEM accumulators; warps 0-7 run the online
-// max/sum (warp w reads TMEM lanes 32 (w % 4) .. +31, the columns of half w / 4 of each
-// tile). Roles hand off through mbarriers only: a tile's stage is free once its MMAs have
-// completed (tcgen05.commit) and the 8 epilogue warps have read its biases; an accumulator
-// is free once the 8 epilogue warps have loaded it. No CTA barrier runs per tile.
+// Potential pass (lse_pass_tc_kernel): one CTA per 128-row block and column split, 10 warps
+// with fixed roles. Warp 8 streams key tiles (image + hy) through a 3-stage ring with TMA
+// bulk copies; warp 9 issues the MMAs of tile t into one of two TMEM accumulators; warps
+// 0-7 run the online max/sum (warp w reads TMEM lanes 32 (w % 4) .. +31, the columns of
+// half w / 4 of each tile). Roles hand off through mbarriers only.
+//
+// Apply pass (lse_apply_tc_kernel, FlashSinkhorn summary, section 3, "Transport Matrix
+// Application"): out_i = sum_j p_ij U_j / sum_j p_ij with p_ij = 2^(z_ij - LSE2_i), the
+// offset LSE2_i taken from a potential-type pass run just before (so p <= 1, no running
+// rescale of a TMEM accumulator is needed). The epilogue writes 2^15 p as fp16 into a
+// shared-memory weight tile, the MMA warp multiplies it by the key tile's U (the key
+// coordinates for the gradient, a payload image for transport products), hi and lo halves,
+// into a third TMEM accumulator, and the epilogue sums the same rounded weights, so the
+// result is an exact convex combination of U up to fp16 weight rounding.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -33,21 +43,26 @@
 namespace fs {
 
 constexpr int kTcRows = 128;     // rows per CTA (MMA M)
-constexpr int kTcCols = 128;     // key columns per tile (MMA N)
+constexpr int kTcCols = 128;     // key columns per tile (MMA N of the score)
 constexpr int kTcStages = 3;
 constexpr int kTcEpiWarps = 8;  // epilogue warps: 4 TMEM lane quarters x 2 column halves
 constexpr int kTcThreads = (kTcEpiWarps + 2) * 32;  // + a producer warp and an MMA warp
-constexpr uint32_t kTcTmemCols = 256;  // two accumulators of kTcCols fp32 columns
+constexpr uint32_t kTcTmemCols = 256;  // potential pass: two accumulators of kTcCols columns
+constexpr uint32_t kTcApplyTmemCols = 512;  // apply pass: two score accumulators + the result
+constexpr uint32_t kCoreLBO = 16u * 128u;  // next K-block of a core-matrix tile
+constexpr uint32_t kCoreSBO = 128u;        // next 8-point group
+// Dynamic shared memory a tensor-core pass may take (the opt-in limit is 227 KB; the
+// kernels' static shared memory is under 2 KB).
+constexpr size_t kTcSmemBudget = 225u * 1024u;
 
 template <int D>
 struct TcShape {
-  static constexpr int K = 3 * D;                  // split-operand K extent
-  static constexpr int KSTEPS = K / 16;            // MMA K = 16 for fp16
+  static constexpr int K = 2 * D;                  // [hi | lo] elements per point
+  static constexpr int KSTEPS = D / 16;            // MMA K = 16 for fp16
   static constexpr uint32_t TILE_BYTES = 128u * K * 2u;
+  static constexpr uint32_t LO_OFF = (D / 8) * kCoreLBO;  // first K-block of the lo half
   static constexpr uint32_t HY_BYTES = kTcCols * 4u;
   static constexpr uint32_t STAGE_BYTES = TILE_BYTES + 1024u;  // hy, padded to keep stages aligned
-  static constexpr uint32_t LBO = 16u * 128u;      // next K-block (second half of a K-step)
-  static constexpr uint32_t SBO = 128u;            // next 8-point group
   static constexpr size_t SMEM = static_cast<size_t>(TILE_BYTES) + kTcStages * STAGE_BYTES;
 };
 
@@ -59,7 +74,9 @@ __host__ __device__ __forceinline__ int64_t tc_image_offset(int64_t i, int kk, i
          (r & 7) * 16 + (kk & 7) * 2;
 }
 
-// Shared-memory matrix descriptor: K-major, no swizzle, sm_100 version field.
+// Shared-memory matrix descriptor: no swizzle, sm_100 version field. For K-major operands
+// lbo steps along K and sbo along M/N; for MN-major operands lbo steps along K (the next 8
+// rows of K) and sbo along M/N (the next 8 elements).
 __device__ __forceinline__ uint64_t tc_smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
@@ -69,9 +86,11 @@ __device__ __forceinline__ uint64_t tc_smem_desc(uint32_t addr, uint32_t lbo, ui
   return d;
 }
 
-// Instruction descriptor of kind::f16: fp16 A and B (K-major), fp32 accumulate, M x N.
-__host__ __device__ constexpr uint32_t tc_instr_desc(int M, int N) {
-  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+// Instruction descriptor of kind::f16: fp16 A and B, fp32 accumulate, M x N; A K-major,
+// B K-major (b_mn = false) or MN-major (b_mn = true).
+__host__ __device__ constexpr uint32_t tc_instr_desc(int M, int N, bool b_mn = false) {
+  return (1u << 4) | (b_mn ? (1u << 16) : 0u) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -97,6 +116,25 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
       : "memory");
 }
 
+// The score tile of one 128-row block against one 128-key tile: three MMAs per 16-wide
+// K-step (hi.hi, lo.hi, hi.lo) into the accumulator at tmem_d. a0 and b0 are the
+// shared-memory addresses of the row and key images ([hi | lo], K-major).
+template <int D>
+__device__ __forceinline__ void tc_issue_scores(uint32_t tmem_d, uint32_t a0, uint32_t b0,
+                                                uint32_t idesc) {
+  using S = TcShape<D>;
+#pragma unroll
+  for (int s = 0; s < S::KSTEPS; ++s) {
+    const uint32_t o = static_cast<uint32_t>(s) * 2u * kCoreLBO;
+    tc_mma_f16(tmem_d, tc_smem_desc(a0 + o, kCoreLBO, kCoreSBO),
+               tc_smem_desc(b0 + o, kCoreLBO, kCoreSBO), idesc, s > 0 ? 1u : 0u);
+    tc_mma_f16(tmem_d, tc_smem_desc(a0 + S::LO_OFF + o, kCoreLBO, kCoreSBO),
+               tc_smem_desc(b0 + o, kCoreLBO, kCoreSBO), idesc, 1u);
+    tc_mma_f16(tmem_d, tc_smem_desc(a0 + o, kCoreLBO, kCoreSBO),
+               tc_smem_desc(b0 + S::LO_OFF + o, kCoreLBO, kCoreSBO), idesc, 1u);
+  }
+}
+
 // 32 consecutive fp32 columns of this thread's TMEM lane; the caller waits (tcgen05.wait::ld).
 __device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, float* v) {
   uint32_t r[32];
@@ -113,26 +151,25 @@ __device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, float* v) {
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
+// 8 consecutive fp32 columns of this thread's TMEM lane; the caller waits.
+__device__ __forceinline__ void tc_ld8_nowait(uint32_t taddr, float* v) {
+  uint32_t r[8];
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        "=r"(r[7])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+__device__ __forceinline__ void tc_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
 struct TcParams {
-  const unsigned char* row_img;  // query cloud as rows (A order), tiles of 128 points
-  const unsigned char* key_img;  // streamed cloud as keys (B order)
+  const unsigned char* row_img;  // query cloud's image, tiles of 128 points
+  const unsigned char* key_img;  // streamed cloud's image
   const float* key_hy;           // hy of the streamed cloud, padded to whole tiles
   const float* row_nrm;          // |x_i|^2 of the query cloud (centred)
   int64_t key_tiles;             // tiles of 128 keys
@@ -218,16 +255,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
   if (warp == kTcEpiWarps) {
     // ---- producer: the row block once, then key tiles through the stage ring ----------
     if (lane == 0) {
-      int issued = 0, waited_free = 0;
+      int issued = 0;
       mbar_expect_tx(&a_bar, S::TILE_BYTES);
       bulk_g2s(sA, T.row_img + (row0 >> 7) * S::TILE_BYTES, S::TILE_BYTES, &a_bar);
       for (int t = 0; t < n_tiles; ++t) {
         const int st = t % kTcStages;
-        if (t >= kTcStages) {
-          if (!tc_wait(&free_bar[st], static_cast<uint32_t>((t - kTcStages) / kTcStages) & 1u, abort))
-            break;
-          ++waited_free;
-        }
+        if (t >= kTcStages &&
+            !tc_wait(&free_bar[st], static_cast<uint32_t>((t - kTcStages) / kTcStages) & 1u, abort))
+          break;
         unsigned char* dst = sStage + st * S::STAGE_BYTES;
         const int64_t kt = t_begin + t;
         fence_proxy_async_smem();
@@ -236,7 +271,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
         bulk_g2s(dst + S::TILE_BYTES, T.key_hy + kt * kTcCols, S::HY_BYTES, &full_bar[st]);
         ++issued;
       }
-      (void)waited_free;
       // Copies never waited for by the MMA role: let them land before the CTA exits.
       if (*abort) {
         (void)mbar_wait_bounded(&a_bar, 0);
@@ -256,14 +290,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
         if (t >= 2 && !tc_wait(&acc_free_bar[b], static_cast<uint32_t>((t - 2) >> 1) & 1u, abort))
           break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA);
-        const uint32_t b0 = smem_u32(sStage + st * S::STAGE_BYTES);
-        const uint32_t d = tmem + static_cast<uint32_t>(b) * kTcCols;
-#pragma unroll
-        for (int s = 0; s < S::KSTEPS; ++s) {
-          tc_mma_f16(d, tc_smem_desc(a0 + s * 2 * S::LBO, S::LBO, S::SBO),
-                     tc_smem_desc(b0 + s * 2 * S::LBO, S::LBO, S::SBO), idesc, s > 0 ? 1u : 0u);
-        }
+        tc_issue_scores<D>(tmem + static_cast<uint32_t>(b) * kTcCols, smem_u32(sA),
+                           smem_u32(sStage + st * S::STAGE_BYTES), idesc);
         tc_commit(&mma_bar[b]);
         tc_commit(&free_bar[st]);
         ++committed;
@@ -288,7 +316,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
       float v[64];
       tc_ld32_nowait(tbase, v);
       tc_ld32_nowait(tbase + 32, v + 32);
-      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_free_bar[b]);
@@ -349,6 +377,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
         const double lse2 = static_cast<double>(mm) + log2(static_cast<double>(l));
         if (P.kind == kPot) {
           finish_pot<D>(P, i, lse2);
+        } else if (P.kind == kLse) {
+          P.lse_out[i] = static_cast<float>(lse2);
         } else {
           finish_marg(P, i, lse2, dev, mass);
         }
@@ -368,7 +398,311 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
                  "r"(kTcTmemCols));
 }
 
-// ---- preparation for the tensor-core pass -----------------------------------------------
+// ---- the apply pass: sum_j p_ij U_j at fixed row offsets ------------------------------------
+
+enum TcApplyMode : int { kApplyGrad = 0, kApplyPay = 1 };
+// Weights p <= 1 are stored as fp16(2^15 p): the largest lands below fp16's maximum and
+// weights down to 2^-39 keep their leading bits.
+constexpr float kPScale = 32768.0f;
+constexpr int kPayChannels = 16;  // payload channels of one transport apply pass
+
+struct TcApply {
+  const float* row_lse;          // LSE2 of every query row (the offset), padding rows unread
+  const float* row_mass;         // kApplyPay: plan mass of each row, or NULL (the row weight)
+  const unsigned char* pay_img;  // kApplyPay: payload image, tiles of 128 keys x [hi | lo]
+  const float* pay_inv_scale;    // kApplyPay: device scalar 1 / s_u of the payload image
+  const float* x;                // kApplyGrad: query cloud (n_rows, d_real), caller order
+  float* out;                    // results: row i, channel c at out[i * out_stride + c]
+  int32_t out_k;                 // kApplyPay: channels written
+  int32_t out_stride;
+  float inv_key_scale;           // kApplyGrad: 1 / s of the key image
+  double ctr[64];                // kApplyGrad: the centre the images were built about
+};
+
+template <int D, int NC, int MODE>
+struct TcApplyShape {
+  using S = TcShape<D>;
+  static constexpr uint32_t PAY_BYTES = MODE == kApplyPay ? 128u * 2u * NC * 2u : 0u;
+  static constexpr uint32_t HY_OFF = S::TILE_BYTES + PAY_BYTES;
+  static constexpr uint32_t STAGE_BYTES = HY_OFF + 1024u;
+  static constexpr uint32_t P_BYTES = 128u * 128u * 2u;  // one fp16 weight tile
+  static constexpr size_t BASE = static_cast<size_t>(S::TILE_BYTES) + 2u * P_BYTES;
+  static constexpr int STAGES = BASE + 3u * STAGE_BYTES <= kTcSmemBudget ? 3 : 2;
+  static constexpr size_t SMEM = BASE + static_cast<size_t>(STAGES) * STAGE_BYTES;
+  static constexpr uint32_t U_LO_OFF = (NC / 8) * kCoreLBO;  // lo half of the U operand
+  static_assert(NC % 16 == 0 && NC >= 16 && NC <= 128, "MMA N of the result");
+  static_assert(SMEM <= kTcSmemBudget, "shared memory");
+};
+
+// Completes channel c of row i from its sums: a = sum_j q_ij U_jc and l = sum_j q_ij (the
+// rounded, 2^15-scaled weights of the row).
+template <int MODE>
+__device__ __forceinline__ void tc_apply_finish(const PassParams& P, const TcApply& A, int64_t i,
+                                                int c, double a, double l) {
+  if constexpr (MODE == kApplyGrad) {
+    if (c >= P.d_real) return;
+    const double w = P.w ? static_cast<double>(P.w[i]) : static_cast<double>(P.w_uniform);
+    const double t = A.ctr[c] + a / l;  // the barycentric projection T_i
+    A.out[i * A.out_stride + c] =
+        static_cast<float>(2.0 * w * (static_cast<double>(A.x[i * P.d_real + c]) - t));
+  } else {
+    if (c >= A.out_k) return;
+    const double mass = A.row_mass ? static_cast<double>(A.row_mass[i])
+                                   : (P.w ? static_cast<double>(P.w[i])
+                                          : static_cast<double>(P.w_uniform));
+    A.out[i * A.out_stride + c] = static_cast<float>(l > 0.0 ? mass * a / l : 0.0);
+  }
+}
+
+template <int D, int NC, int MODE>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    lse_apply_tc_kernel(const PassParams P, const TcParams T, const TcApply A) {
+  using S = TcShape<D>;
+  using Sh = TcApplyShape<D, NC, MODE>;
+  constexpr int ST = Sh::STAGES;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  __shared__ uint64_t full_bar[ST];   // tile landed
+  __shared__ uint64_t free_bar[ST];   // stage reusable: result MMA commit + 8 epilogue warps
+  __shared__ uint64_t mma_bar[2];     // score accumulator ready
+  __shared__ uint64_t acc_free_bar[2];  // score accumulator read by the 8 epilogue warps
+  __shared__ uint64_t p_full[2];      // weight tile written by the 8 epilogue warps
+  __shared__ uint64_t p_free[2];      // weight tile read by its result MMAs
+  __shared__ uint64_t a_bar, o_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  __shared__ float lsum[2][kTcRows];
+
+  unsigned char* sA = smem;
+  unsigned char* sP = smem + S::TILE_BYTES;
+  unsigned char* sStage = sP + 2 * Sh::P_BYTES;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kTcRows;
+  const int split = blockIdx.y;
+  const int64_t t_begin = static_cast<int64_t>(split) * T.tiles_per_split;
+  int64_t t_end = t_begin + T.tiles_per_split;
+  if (t_end > T.key_tiles) t_end = T.key_tiles;
+  const int n_tiles = static_cast<int>(t_end - t_begin);
+  volatile int* abort = &abort_sh;
+
+  if (tid == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&free_bar[s], kTcEpiWarps + 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&mma_bar[b], 1);
+      mbar_init(&acc_free_bar[b], kTcEpiWarps);
+      mbar_init(&p_full[b], kTcEpiWarps);
+      mbar_init(&p_free[b], 1);
+    }
+    mbar_init(&a_bar, 1);
+    mbar_init(&o_bar, 1);
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tmem_base_sh)),
+                 "r"(kTcApplyTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const uint32_t tmem_o = tmem + 2u * kTcCols;  // the result accumulator, NC columns
+
+  const int quarter = warp & 3, half = (warp >> 2) & 1;
+  const int r = quarter * 32 + lane;
+  const int64_t i = row0 + r;
+  u64 L = pk(0.0f, 0.0f);  // epilogue: sum of this row's rounded weights over its half
+
+  if (warp == kTcEpiWarps) {
+    // ---- producer ---------------------------------------------------------------------
+    if (lane == 0) {
+      int issued = 0;
+      mbar_expect_tx(&a_bar, S::TILE_BYTES);
+      bulk_g2s(sA, T.row_img + (row0 >> 7) * S::TILE_BYTES, S::TILE_BYTES, &a_bar);
+      for (int t = 0; t < n_tiles; ++t) {
+        const int st = t % ST;
+        if (t >= ST && !tc_wait(&free_bar[st], static_cast<uint32_t>((t - ST) / ST) & 1u, abort))
+          break;
+        unsigned char* dst = sStage + st * Sh::STAGE_BYTES;
+        const int64_t kt = t_begin + t;
+        fence_proxy_async_smem();
+        mbar_expect_tx(&full_bar[st], S::TILE_BYTES + Sh::PAY_BYTES + S::HY_BYTES);
+        bulk_g2s(dst, T.key_img + kt * S::TILE_BYTES, S::TILE_BYTES, &full_bar[st]);
+        if constexpr (MODE == kApplyPay)
+          bulk_g2s(dst + S::TILE_BYTES, A.pay_img + kt * Sh::PAY_BYTES, Sh::PAY_BYTES,
+                   &full_bar[st]);
+        bulk_g2s(dst + Sh::HY_OFF, T.key_hy + kt * kTcCols, S::HY_BYTES, &full_bar[st]);
+        ++issued;
+      }
+      if (*abort) {
+        (void)mbar_wait_bounded(&a_bar, 0);
+        for (int t = (issued > ST ? issued - ST : 0); t < issued; ++t)
+          (void)mbar_wait_bounded(&full_bar[t % ST], static_cast<uint32_t>(t / ST) & 1u);
+      }
+    }
+  } else if (warp == kTcEpiWarps + 1) {
+    // ---- MMA issuer: scores of tile t, then the result MMAs of tile t - 1 ---------------
+    if (lane == 0) {
+      const uint32_t idesc_s = tc_instr_desc(kTcRows, kTcCols);
+      const uint32_t idesc_o = tc_instr_desc(kTcRows, NC, true);
+      bool ok = tc_wait(&a_bar, 0, abort);
+      for (int t = 0; ok && t <= n_tiles; ++t) {
+        if (t < n_tiles) {
+          const int st = t % ST, b = t & 1;
+          if (!tc_wait(&full_bar[st], static_cast<uint32_t>(t / ST) & 1u, abort)) break;
+          if (t >= 2 && !tc_wait(&acc_free_bar[b], static_cast<uint32_t>((t - 2) >> 1) & 1u, abort))
+            break;
+          tc_fence_after();
+          tc_issue_scores<D>(tmem + static_cast<uint32_t>(b) * kTcCols, smem_u32(sA),
+                             smem_u32(sStage + st * Sh::STAGE_BYTES), idesc_s);
+          tc_commit(&mma_bar[b]);
+        }
+        if (t >= 1) {
+          const int u = t - 1, su = u % ST, pb = u & 1;
+          if (!tc_wait(&p_full[pb], static_cast<uint32_t>(u >> 1) & 1u, abort)) break;
+          tc_fence_after();
+          const uint32_t pa = smem_u32(sP + pb * Sh::P_BYTES);
+          const uint32_t ub = smem_u32(sStage + su * Sh::STAGE_BYTES) +
+                              (MODE == kApplyPay ? S::TILE_BYTES : 0u);
+          // U along N (coordinates or channels), keys along K: MN-major
+#pragma unroll
+          for (int s = 0; s < kTcCols / 16; ++s) {
+            const uint64_t ad = tc_smem_desc(pa + s * 2u * kCoreLBO, kCoreLBO, kCoreSBO);
+            const uint32_t ko = static_cast<uint32_t>(s) * 2u * kCoreSBO;  // next 16 keys
+            tc_mma_f16(tmem_o, ad, tc_smem_desc(ub + ko, kCoreSBO, kCoreLBO), idesc_o,
+                       (u > 0 || s > 0) ? 1u : 0u);
+            tc_mma_f16(tmem_o, ad, tc_smem_desc(ub + Sh::U_LO_OFF + ko, kCoreSBO, kCoreLBO),
+                       idesc_o, 1u);
+          }
+          tc_commit(&free_bar[su]);
+          tc_commit(&p_free[pb]);
+        }
+      }
+      // Every MMA this thread issued has completed once o_bar fires; wait for it here so
+      // that TMEM is never released under a running MMA, whatever the other roles did.
+      tc_commit(&o_bar);
+      (void)mbar_wait_bounded(&o_bar, 0);
+    }
+  } else {
+    // ---- epilogue warps: weights of one row over half of every tile --------------------
+    float off = 1.0e30f;  // padding rows: every weight is 0
+    if (i < P.n_rows) off = P.kappa_f * T.row_nrm[i] + A.row_lse[i];
+    const u64 c2 = pk(T.c2, T.c2);
+    const u64 noff = pk(-off, -off);
+    for (int u = 0; u < n_tiles; ++u) {
+      const int b = u & 1, st = u % ST, pb = u & 1;
+      if (!tc_wait(&mma_bar[b], static_cast<uint32_t>(u >> 1) & 1u, abort)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(b) * kTcCols + half * 64;
+      float v[64];
+      tc_ld32_nowait(tbase, v);
+      tc_ld32_nowait(tbase + 32, v + 32);
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_free_bar[b]);
+      const u64* hv = reinterpret_cast<const u64*>(sStage + st * Sh::STAGE_BYTES + Sh::HY_OFF) +
+                      half * 32;
+      uint32_t h2[32];  // fp16 pairs of 2^15 p
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float t0, t1;
+        upk(add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), hv[j]), noff), t0, t1);
+        const __half2 h = __floats2half2_rn(ex2(t0) * kPScale, ex2(t1) * kPScale);
+        const float2 back = __half22float2(h);
+        L = add2(L, pk(back.x, back.y));
+        h2[j] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&free_bar[st]);  // its hy has been read
+      if (u >= 2 && !tc_wait(&p_free[pb], static_cast<uint32_t>((u - 2) >> 1) & 1u, abort)) break;
+      // K-major weight tile: core(row group, key block) at (kb * 16 + r / 8) * 128 + (r % 8) * 16
+      unsigned char* pt = sP + pb * Sh::P_BYTES + (r >> 3) * 128 + (r & 7) * 16;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int kb = half * 8 + c;
+        *reinterpret_cast<uint4*>(pt + kb * 16 * 128) =
+            make_uint4(h2[4 * c], h2[4 * c + 1], h2[4 * c + 2], h2[4 * c + 3]);
+      }
+      fence_proxy_async_smem();  // the generic-proxy writes, before the MMA reads them
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[pb]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  {
+    float l0, l1;
+    upk(L, l0, l1);
+    if (warp < kTcEpiWarps) lsum[half][r] = l0 + l1;
+  }
+  __syncthreads();
+  if (abort_sh) {
+    if (tid == 0) atomicOr(P.err, kErrTimeout);
+  } else if (warp < kTcEpiWarps) {
+    // The result accumulator: this warp's rows, channels [half * NC / 2, (half + 1) * NC / 2).
+    if (mbar_wait_bounded(&o_bar, 0)) {
+      tc_fence_after();
+      constexpr int NH = NC / 2;
+      float o[NH];
+      const uint32_t obase = tmem_o + (static_cast<uint32_t>(quarter * 32) << 16) + half * NH;
+#pragma unroll
+      for (int c = 0; c < NH; c += 8) tc_ld8_nowait(obase + c, o + c);
+      tc_wait_ld();
+      const double l = static_cast<double>(lsum[0][r]) + static_cast<double>(lsum[1][r]);
+      const double inv = MODE == kApplyGrad ? static_cast<double>(A.inv_key_scale)
+                                            : static_cast<double>(*A.pay_inv_scale);
+      if (i < P.n_rows) {
+        if (P.n_splits == 1) {
+#pragma unroll
+          for (int c = 0; c < NH; ++c)
+            tc_apply_finish<MODE>(P, A, i, half * NH + c, static_cast<double>(o[c]) * inv, l);
+        } else {
+          const int64_t ps = static_cast<int64_t>(split);
+          if (half == 0) P.part_l[ps * P.rows_pad + i] = static_cast<float>(l);
+#pragma unroll
+          for (int c = 0; c < NH; ++c)
+            P.part_a[(ps * NC + half * NH + c) * P.rows_pad + i] =
+                static_cast<float>(static_cast<double>(o[c]) * inv);
+        }
+      }
+    } else {
+      atomicOr(P.err, kErrTimeout);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTcApplyTmemCols));
+}
+
+// Sums the column splits' partials of an apply pass (the offsets are fixed, so partials
+// add) and completes each row.
+template <int NC, int MODE>
+__global__ void __launch_bounds__(256) tc_apply_combine_kernel(const PassParams P, const TcApply A) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= P.n_rows) return;
+  double l = 0.0;
+  for (int s = 0; s < P.n_splits; ++s) l += P.part_l[static_cast<int64_t>(s) * P.rows_pad + i];
+  for (int c = 0; c < NC; ++c) {
+    double a = 0.0;
+    for (int s = 0; s < P.n_splits; ++s)
+      a += P.part_a[(static_cast<int64_t>(s) * NC + c) * P.rows_pad + i];
+    tc_apply_finish<MODE>(P, A, i, c, a, l);
+  }
+}
+
+// ---- preparation for the tensor-core passes -----------------------------------------------
 
 // Per-coordinate sums (float64) and the largest |coordinate| of one cloud.
 __global__ void __launch_bounds__(256) coord_stats_kernel(const float* pts, int64_t count,
@@ -396,14 +730,14 @@ struct TcCenter {
   double c[64];
 };
 
-// Both operand images of one cloud and its centred squared norms, for all padded points.
+// The operand image of one cloud ([hi | lo] of the centred, scaled coordinates) and its
+// centred squared norms, for all padded points.
 template <int D>
-__global__ void __launch_bounds__(256) build_images_kernel(const float* pts, int64_t count,
-                                                           int32_t d_real, const TcCenter ctr,
-                                                           float scale, unsigned char* row_img,
-                                                           unsigned char* key_img, float* nrm,
-                                                           int64_t count_pad) {
-  constexpr int K = 3 * D;
+__global__ void __launch_bounds__(256) build_image_kernel(const float* pts, int64_t count,
+                                                          int32_t d_real, const TcCenter ctr,
+                                                          float scale, unsigned char* img,
+                                                          float* nrm, int64_t count_pad) {
+  constexpr int K = 2 * D;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= count_pad) return;
   double n2 = 0.0;
@@ -417,12 +751,8 @@ __global__ void __launch_bounds__(256) build_images_kernel(const float* pts, int
     }
     const __half hi = __float2half_rn(u);
     const __half lo = __float2half_rn(u - __half2float(hi));
-    *reinterpret_cast<__half*>(row_img + tc_image_offset(i, k, K)) = hi;
-    *reinterpret_cast<__half*>(row_img + tc_image_offset(i, D + k, K)) = lo;
-    *reinterpret_cast<__half*>(row_img + tc_image_offset(i, 2 * D + k, K)) = hi;
-    *reinterpret_cast<__half*>(key_img + tc_image_offset(i, k, K)) = hi;
-    *reinterpret_cast<__half*>(key_img + tc_image_offset(i, D + k, K)) = hi;
-    *reinterpret_cast<__half*>(key_img + tc_image_offset(i, 2 * D + k, K)) = lo;
+    *reinterpret_cast<__half*>(img + tc_image_offset(i, k, K)) = hi;
+    *reinterpret_cast<__half*>(img + tc_image_offset(i, D + k, K)) = lo;
   }
   nrm[i] = static_cast<float>(n2);
 }
@@ -442,6 +772,47 @@ __global__ void __launch_bounds__(256) tc_key_bias_kernel(float* hy, int64_t cou
   const double p = pot ? static_cast<double>(pot[j]) : 0.0;
   hy[j] = static_cast<float>(kappa * p + static_cast<double>(lw[j]) -
                              kappa * static_cast<double>(nrm[j]));
+}
+
+// Largest |u| over channels [0, k) of a row-major (count, stride) array, as float bits.
+__global__ void __launch_bounds__(256) pay_maxabs_kernel(const float* u, int64_t count, int k,
+                                                         int stride, unsigned* maxabs_bits) {
+  float mx = 0.0f;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < count * k;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    mx = fmaxf(mx, fabsf(u[(t / k) * stride + t % k]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(maxabs_bits, __float_as_uint(mx));
+}
+
+// Payload image of a transport apply pass: channels [0, k) of u scaled by the power of two
+// s = 2^floor(log2(16384 / max|u|)) and split into [hi | lo] fp16 (NC channels per point,
+// padding channels and points zero), in the core-matrix layout of the key images. Thread 0
+// of block 0 also stores 1 / s.
+template <int NC>
+__global__ void __launch_bounds__(256) build_pay_image_kernel(const float* u, int64_t count,
+                                                              int64_t count_pad, int k,
+                                                              int stride,
+                                                              const unsigned* maxabs_bits,
+                                                              unsigned char* img,
+                                                              float* inv_scale) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const float mx = __uint_as_float(*maxabs_bits);
+  int e = 0;
+  if (mx > 0.0f) e = static_cast<int>(floorf(log2f(16384.0f / mx)));
+  e = max(-120, min(120, e));
+  const float scale = exp2f(static_cast<float>(e));
+  if (i == 0) *inv_scale = exp2f(static_cast<float>(-e));
+  if (i >= count_pad) return;
+#pragma unroll 4
+  for (int c = 0; c < NC; ++c) {
+    const float v = (i < count && c < k) ? u[i * stride + c] * scale : 0.0f;
+    const __half hi = __float2half_rn(v);
+    const __half lo = __float2half_rn(v - __half2float(hi));
+    *reinterpret_cast<__half*>(img + tc_image_offset(i, c, 2 * NC)) = hi;
+    *reinterpret_cast<__half*>(img + tc_image_offset(i, NC + c, 2 * NC)) = lo;
+  }
 }
 
 }  // namespace fs

@@ -84,6 +84,6 @@ def test_injected_error_word_is_reported_once():
         assert ei.value.status == "FS_ERR_TIMEOUT"
         gx = fs.grad_x(x, y, g, a, b, eps=w.eps).cpu().numpy()
         gxr = oracle.grad_x(w.x, w.y, w.a, w.b, w.eps, g.cpu().numpy())
-        assert np.abs(gx - gxr).max() <= 1e-3 * np.abs(gxr).max()
+        assert np.abs(gx - gxr).max() <= 1e-4 * np.abs(gxr).max()
     finally:
         lib.fs_inject_error_word(0)

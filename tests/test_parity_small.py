@@ -8,7 +8,7 @@ import oracle
 import streaming_sinkhorn_b200 as fs
 from streaming_sinkhorn_b200 import workloads
 from tests.parity_util import (assert_cost_close, assert_grad_close, assert_potential_close,
-                               dev, inputs, residual_tolerance)
+                               dev, grad_rel, inputs, residual_tolerance)
 
 pytestmark = pytest.mark.gpu
 
@@ -53,7 +53,7 @@ def test_potentials_cost_grad_residual(shape):
 
     gx = fs.grad_x(x, y, g, a, b, eps=w.eps).cpu().numpy()
     gxr = oracle.grad_x(w.x, w.y, w.a, w.b, w.eps, g.cpu().numpy())
-    assert_grad_close(gx, gxr)
+    assert_grad_close(gx, gxr, rel=grad_rel(w.d))
 
     res, r, cc = fs.marginal_residual(x, y, f, g, a, b, eps=w.eps, marginals=True)
     fn, gn = f.cpu().numpy(), g.cpu().numpy()

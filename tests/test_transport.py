@@ -25,10 +25,20 @@ def close(got, ref, rel):
     assert err <= rel * scale, f"max err {err:.3e} vs {rel:.0e} * {scale:.3e}"
 
 
+# Relative bar of a transport product against the oracle's dense one. The float32 path
+# (d <= 16) meets 1e-4 of the largest entry. The tensor-core path (d > 16) forms
+# P u / (P 1) with the plan weights rounded to fp16 (2^-11 relative each) and u to a
+# [hi | lo] fp16 pair (2^-22 relative): each entry moves by at most 2^-11 of the row's
+# mean |u_j - (P u)_i / (P 1)_i| (below max|u|) times the row mass, which bounds the error
+# by 2^-11 max|u| a_i against entries of size ~ a_i |u|: 1e-3 of the largest entry.
+TRANSPORT_REL = {False: 1e-4, True: 1e-3}
+
+
 @pytest.mark.parametrize("k", [1, 3, 5, 16, 20])
 @pytest.mark.parametrize("transpose", [False, True])
 @pytest.mark.parametrize("shape", [(300, 257, 2, 0.1), (129, 700, 3, 0.05), (200, 150, 8, 0.5),
-                                   (90, 100, 16, 1.0)], ids=lambda s: "n{}-m{}-d{}".format(*s[:3]))
+                                   (90, 100, 16, 1.0), (200, 170, 32, 4.0), (130, 300, 64, 8.0)],
+                         ids=lambda s: "n{}-m{}-d{}".format(*s[:3]))
 def test_transport_apply_matches_dense_plan(shape, transpose, k):
     n, m, d, eps = shape
     w = problem(n, m, d, eps, seed=n + m + d + k)
@@ -41,7 +51,7 @@ def test_transport_apply_matches_dense_plan(shape, transpose, k):
                              transpose=transpose).cpu().numpy()
     fn = oracle.transport_apply_t if transpose else oracle.transport_apply
     ref = fn(w.x, w.y, w.a, w.b, w.eps, f32, g32, u)
-    close(out, ref, 1e-4)
+    close(out, ref, TRANSPORT_REL[d > 16])
 
 
 def test_transport_apply_vector_form():
@@ -53,6 +63,14 @@ def test_transport_apply_vector_form():
     out = fs.transport_apply(x, y, dev(f32), dev(g32), dev(u), a, b, eps=w.eps)
     assert out.shape == (100,)
     close(out.cpu().numpy(), oracle.transport_apply(w.x, w.y, w.a, w.b, w.eps, f32, g32, u), 1e-4)
+
+
+# Bar of the HVP against the oracle, relative to the largest entry and, as a whole vector,
+# in the 2-norm. fp32 conjugate gradients return an iterate at a relative residual of a few
+# 1e-7 (the fp32 floor; reported by fs_hvp) and the transport passes are accurate to fp32
+# rounding, so the entries agree to ~1e-5 of the largest (measured worst 1.1e-5); 1e-4
+# leaves ten times that.
+HVP_TOL = 1e-4
 
 
 @pytest.mark.parametrize("shape", [(120, 90, 2, 0.3), (250, 300, 3, 0.1), (80, 70, 8, 1.0)],
@@ -69,21 +87,23 @@ def test_hvp_matches_oracle(shape):
     hv, rep = fs.hvp(x, y, dev(g32), dev(v), a, b, eps=w.eps, cg_max_iter=500, cg_tol=1e-7)
     ref = oracle.hvp(w.x, w.y, w.a, w.b, w.eps, g32, v)
     assert rep["cg_iters"] >= 1
-    close(hv.cpu().numpy(), ref, HVP_TOL)
+    hv = hv.cpu().numpy().astype(np.float64)
+    close(hv, ref, HVP_TOL)
+    assert np.linalg.norm(hv - ref) <= HVP_TOL * np.linalg.norm(ref)
 
 
-HVP_TOL = 2e-3  # elementwise, relative to the largest |(Hv)_i|: test_hvp_matches_oracle
 
 
 def test_hvp_is_symmetric_on_the_gpu():
     """u.(Hv) = v.(Hu) (the Hessian is symmetric) and both equal the oracle's value.
 
-    Error model: every entry of the GPU's Hv is within HVP_TOL max|H_ref v| of the oracle's
-    (the bar of test_hvp_matches_oracle), so |u.(Hv) - u.(H_ref v)| <= HVP_TOL max|H_ref v|
-    |u|_1, and the GPU's asymmetry |u.(Hv) - v.(Hu)| is at most the sum of that bound for
-    (u, v) and for (v, u) plus the oracle's own (fp64) asymmetry. u is taken correlated with
-    v (u = v + w / 2), so that u.(Hv) ~ v.(Hv) > 0 sums coherently and the bound is a few
-    1e-3 of the value, while a dropped or one-sided term of H changes it by O(1).
+    Error model: the GPU's Hv is within HVP_TOL |H_ref v|_2 of the oracle's in the 2-norm (the
+    bar of test_hvp_matches_oracle), so by Cauchy-Schwarz |u.(Hv) - u.(H_ref v)| <= HVP_TOL
+    |u|_2 |H_ref v|_2, and the GPU's asymmetry |u.(Hv) - v.(Hu)| is at most that bound for
+    (u, v) plus the one for (v, u) plus the oracle's own (fp64) asymmetry. u is taken
+    correlated with v (u = v + w / 2), so that u.(Hv) ~ v.(Hv) > 0 (H is positive
+    semi-definite) and the bound is well under 1e-2 of the value, while a dropped or
+    one-sided term of H changes it by O(1).
     """
     w = problem(200, 180, 3, 0.2, seed=17)
     x, y, a, b = inputs(w)
@@ -99,15 +119,15 @@ def test_hvp_is_symmetric_on_the_gpu():
     hu_ref = oracle.hvp(w.x, w.y, w.a, w.b, w.eps, g32, u)
     hv_ref = oracle.hvp(w.x, w.y, w.a, w.b, w.eps, g32, v)
     u64, v64 = u.astype(np.float64), v.astype(np.float64)
-    b_uv = HVP_TOL * np.abs(hv_ref).max() * np.abs(u64).sum()
-    b_vu = HVP_TOL * np.abs(hu_ref).max() * np.abs(v64).sum()
+    b_uv = HVP_TOL * np.linalg.norm(u64) * np.linalg.norm(hv_ref)
+    b_vu = HVP_TOL * np.linalg.norm(v64) * np.linalg.norm(hu_ref)
     ref_uv, ref_vu = float((u64 * hv_ref).sum()), float((v64 * hu_ref).sum())
     lhs, rhs = float((u64 * hv).sum()), float((v64 * hu).sum())
     assert abs(ref_uv - ref_vu) <= 1e-9 * abs(ref_uv)  # the oracle is symmetric
+    assert b_uv + b_vu <= 1e-2 * abs(ref_uv)  # the check can see an O(1) asymmetry
     assert abs(lhs - ref_uv) <= b_uv, (lhs, ref_uv, b_uv)
     assert abs(rhs - ref_vu) <= b_vu, (rhs, ref_vu, b_vu)
     assert abs(lhs - rhs) <= b_uv + b_vu + abs(ref_uv - ref_vu), (lhs, rhs)
-    assert b_uv + b_vu <= 0.03 * abs(ref_uv)  # the check can see an O(1) asymmetry
 
 
 def test_hvp_screened_equals_dense():
