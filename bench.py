@@ -373,9 +373,9 @@ def run_native(args, rank, world, local_rank):
             for k in ("coarse_rounds", "lift_viol"):
                 if k in rep:
                     solve_extras[name][k] = rep[k]
-        # a transport-matrix product (P Y, 3 channels) and a Hessian-vector product at the
+        # a transport-matrix product (P Y, d channels) and a Hessian-vector product at the
         # potentials just solved
-        if w.d <= 16:
+        if True:
             from streaming_sinkhorn_b200 import _lib
             p_ = _lib.fs_problem(x.data_ptr(), y.data_ptr(), a.data_ptr(), b.data_ptr(), w.n, w.m,
                                  w.d, w.eps)

@@ -329,6 +329,9 @@ constexpr int kPotChange = 153;  // unsigned: float bits of the largest potentia
 constexpr int kCgDots = 156;     // [4] float64: the HVP solve's dot products and sums
 constexpr int kPayMax = 160;     // unsigned: float bits of the largest |payload| of an apply pass
 constexpr int kPayInv = 161;     // float: 1 / s of that pass's payload image
+constexpr int kVMax = 162;       // unsigned: float bits of max |v| (HVP difference pass)
+constexpr int kVInv = 163;       // float: 1 / s_v of its vector image
+constexpr int kDgMax = 164;      // unsigned: float bits of max |dg|
 // [kSortMemoWords] uint64 from here: the record of the last sort done in this workspace,
 // which prepare() does not clear (everything before it is cleared at every call)
 constexpr int kSortMemo = 240;
@@ -344,8 +347,10 @@ struct Layout {
   int64_t tx, ty;  // points of x and y padded to whole 128-point tiles (tensor-core path)
   size_t off_scalars, off_kx, off_ky, off_lwx, off_lwy, off_part, total;
   size_t off_img_x, off_img_y, off_nrm_x, off_nrm_y, off_hy_x, off_hy_y;
-  // apply passes (d > 16): the rows' LSE2 offsets and plan masses, a payload image
-  size_t off_tc_lse, off_tc_mass, off_tc_pay;
+  // apply passes (d > 16): the rows' LSE2 offsets and plan masses (rows x, then rows y), a
+  // payload image; the HVP's difference pass: the rows' vector image, per-row (qs, x'.v),
+  // the keys' padded dg
+  size_t off_tc_lse, off_tc_mass, off_tc_pay, off_tc_vimg, off_tc_vrow, off_tc_dg;
   // spatial order and screening (FMA path): permutations, sort keys, per-tile boxes and bias
   // maxima, and the LSE2 of every row in its last pass
   bool sorted;
@@ -403,10 +408,11 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0, bool co
   L.tx = tc_pad(n);
   L.ty = tc_pad(m);
   if (L.Dtc) {
-    // potential passes: (max, sum) per split and row; apply passes: (sum, NC channels)
+    // potential passes: (max, sum) per split and row; apply passes: (sum, NC channels and,
+    // for the difference pass, a second sum)
     const int64_t nc = std::max<int64_t>(L.Dtc, kPayChannels);
     for (const TcPlan& tp : {make_tc_plan(n, m, L.Dtc, sms), make_tc_plan(m, n, L.Dtc, sms)})
-      if (tp.n_splits > 1) pf = std::max<int64_t>(pf, (1 + nc) * tp.n_splits * tp.rows_pad);
+      if (tp.n_splits > 1) pf = std::max<int64_t>(pf, (2 + nc) * tp.n_splits * tp.rows_pad);
   }
   L.part_floats = pf;
   size_t o = 0;
@@ -438,12 +444,18 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0, bool co
     o = align_up(o + static_cast<size_t>(L.ty) * sizeof(float));
     const int64_t tmax = std::max(L.tx, L.ty);
     L.off_tc_lse = o;
-    o = align_up(o + static_cast<size_t>(tmax) * sizeof(float));
+    o = align_up(o + static_cast<size_t>(2 * tmax) * sizeof(float));
     L.off_tc_mass = o;
-    o = align_up(o + static_cast<size_t>(tmax) * sizeof(float));
+    o = align_up(o + static_cast<size_t>(2 * tmax) * sizeof(float));
     if (acc_ch > 0) {
       L.off_tc_pay = o;
       o = align_up(o + static_cast<size_t>(tmax) * 2 * kPayChannels * 2);
+      L.off_tc_vimg = o;
+      o = align_up(o + static_cast<size_t>(L.tx) * 2 * L.Dtc * 2);
+      L.off_tc_vrow = o;
+      o = align_up(o + static_cast<size_t>(2 * L.tx) * sizeof(float));
+      L.off_tc_dg = o;
+      o = align_up(o + static_cast<size_t>(tmax) * sizeof(float));
     }
   }
   if (L.sorted) {
@@ -493,9 +505,11 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0, bool co
   L.off_gprev = o;
   o = align_up(o + static_cast<size_t>(m) * sizeof(float));
   if (acc_ch > 0) {
-    L.off_paykeys = o;
-    o = align_up(o + static_cast<size_t>(std::max(L.px, L.py)) * pair_floats(L.D, acc_ch) *
-                         sizeof(float));
+    if (!L.Dtc) {  // payload keys of the FMA transport passes
+      L.off_paykeys = o;
+      o = align_up(o + static_cast<size_t>(std::max(L.px, L.py)) * pair_floats(L.D, acc_ch) *
+                           sizeof(float));
+    }
     L.off_hvp = o;
     o = align_up(o + static_cast<size_t>(hvp_floats(n, m, d)) * sizeof(float));
   }
@@ -753,11 +767,17 @@ void launch_apply_tc(int Dtc, int mode, const PassParams& P, const TcParams& T, 
       case 48: TcApplyKernel<48, 48, kApplyGrad>::launch(P, T, A, pl, st); break;
       default: TcApplyKernel<64, 64, kApplyGrad>::launch(P, T, A, pl, st); break;
     }
-  } else {
+  } else if (mode == kApplyPay) {
     switch (Dtc) {
       case 32: TcApplyKernel<32, kPayChannels, kApplyPay>::launch(P, T, A, pl, st); break;
       case 48: TcApplyKernel<48, kPayChannels, kApplyPay>::launch(P, T, A, pl, st); break;
       default: TcApplyKernel<64, kPayChannels, kApplyPay>::launch(P, T, A, pl, st); break;
+    }
+  } else {
+    switch (Dtc) {
+      case 32: TcApplyKernel<32, 32, kApplyDiff>::launch(P, T, A, pl, st); break;
+      case 48: TcApplyKernel<48, 48, kApplyDiff>::launch(P, T, A, pl, st); break;
+      default: TcApplyKernel<64, 64, kApplyDiff>::launch(P, T, A, pl, st); break;
     }
   }
 }
@@ -911,7 +931,13 @@ struct Ctx {
   unsigned char *img_x, *img_y;
   float *nrm_x, *nrm_y, *hy_x, *hy_y;
   float *tc_lse, *tc_mass;      // apply passes: the rows' LSE2 offsets and plan masses
+                                // ([0, tmax): rows x; [tmax, 2 tmax): rows y)
   unsigned char* tc_pay;        // apply passes: payload image
+  unsigned char* tc_vimg;       // difference pass: the rows' vector image
+  float *tc_vrow, *tc_dg;       // difference pass: per-row (qs, x'.v); the keys' padded dg
+  double tc_rkey;               // a bound on |y'_j| and |x'_i| (centred points)
+  bool tc_reuse;                // apply passes keep the offsets of their first pre-pass
+  bool tc_valid[2];             // ... per direction (rows x, rows y)
   float c2;       // 2 kappa / s^2
   float tc_scale;  // s: the images' power-of-two scale
   TcCenter tc_ctr;  // the centre the images were built about
@@ -964,16 +990,19 @@ void carve(Ctx& c, void* ws) {
     c.cos_x = reinterpret_cast<float*>(c.ws + c.L.off_cos);
     c.cos_y = c.cos_x + c.p->n * c.p->d;
   }
-  if (c.L.off_paykeys) {
-    c.paykeys = reinterpret_cast<float*>(c.ws + c.L.off_paykeys);
-    c.hvp = reinterpret_cast<float*>(c.ws + c.L.off_hvp);
-  }
+  if (c.L.off_paykeys) c.paykeys = reinterpret_cast<float*>(c.ws + c.L.off_paykeys);
+  if (c.L.off_hvp) c.hvp = reinterpret_cast<float*>(c.ws + c.L.off_hvp);
   if (c.L.Dtc) {
     c.img_x = c.ws + c.L.off_img_x;
     c.img_y = c.ws + c.L.off_img_y;
     c.tc_lse = reinterpret_cast<float*>(c.ws + c.L.off_tc_lse);
     c.tc_mass = reinterpret_cast<float*>(c.ws + c.L.off_tc_mass);
-    if (c.L.off_tc_pay) c.tc_pay = c.ws + c.L.off_tc_pay;
+    if (c.L.off_tc_pay) {
+      c.tc_pay = c.ws + c.L.off_tc_pay;
+      c.tc_vimg = c.ws + c.L.off_tc_vimg;
+      c.tc_vrow = reinterpret_cast<float*>(c.ws + c.L.off_tc_vrow);
+      c.tc_dg = reinterpret_cast<float*>(c.ws + c.L.off_tc_dg);
+    }
     c.nrm_x = reinterpret_cast<float*>(c.ws + c.L.off_nrm_x);
     c.nrm_y = reinterpret_cast<float*>(c.ws + c.L.off_nrm_y);
     c.hy_x = reinterpret_cast<float*>(c.ws + c.L.off_hy_x);
@@ -1160,6 +1189,7 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
     c.c2 = static_cast<float>(2.0 * c.kappa / (scale * scale));
     c.tc_ctr = ctr;
     c.tc_scale = static_cast<float>(scale);
+    c.tc_rkey = std::sqrt(static_cast<double>(p->d)) * bound;
     const float sc = static_cast<float>(scale);
     switch (c.L.Dtc) {
       case 32:
@@ -1271,18 +1301,28 @@ void run_pass_tc(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_
 //   mode kApplyGrad: out = grad (n_rows x d) at the plan of (F(g), g), g carried by the keys;
 //   mode kApplyPay:  out (n_rows x k, row stride out_stride) = P pay, pay (n_keys x k, row
 //     stride pay_stride), P the plan of (pot_in, key potentials), or of (F(g), g) when pot_in
-//     is NULL; channels go kPayChannels at a time.
+//     is NULL; channels go kPayChannels at a time;
+//   mode kApplyDiff: out (n_rows x d) = sum_j P_ij (pay_j + (y_j - x_i).row_v_i)(y_j - x_i),
+//     pay one value per key (dg), row_v (n_rows x d) one vector per row.
 // First a potential-type pass writes every row's LSE2 (and, with pot_in, its plan mass),
-// then the apply pass streams the keys again at those fixed offsets.
+// then the apply pass streams the keys again at those fixed offsets. With c.tc_reuse the
+// first pre-pass of each direction serves every later apply pass of the call.
 void run_apply_tc(Ctx& c, bool rows_x, int mode, const float* pot_in, const float* pay, int k,
-                  int pay_stride, float* out, int out_stride) {
+                  int pay_stride, float* out, int out_stride, const float* row_v = nullptr) {
   const fs_problem* p = c.p;
   const int64_t n_rows = rows_x ? p->n : p->m, n_keys = rows_x ? p->m : p->n;
   const int tk = mode == kApplyGrad ? kTGrad : kTMarg;
-  if (pot_in)
-    run_pass_tc(c, rows_x, kMarg, pot_in, nullptr, c.tc_mass, nullptr, c.tc_lse, tk);
-  else
-    run_pass_tc(c, rows_x, kLse, nullptr, nullptr, nullptr, nullptr, c.tc_lse, tk);
+  const int64_t half = std::max(c.L.tx, c.L.ty);
+  float* lse = c.tc_lse + (rows_x ? 0 : half);
+  float* mass = c.tc_mass + (rows_x ? 0 : half);
+  const int dir = rows_x ? 0 : 1;
+  if (!(c.tc_reuse && c.tc_valid[dir])) {
+    if (pot_in)
+      run_pass_tc(c, rows_x, kMarg, pot_in, nullptr, mass, nullptr, lse, tk);
+    else
+      run_pass_tc(c, rows_x, kLse, nullptr, nullptr, nullptr, nullptr, lse, tk);
+    c.tc_valid[dir] = true;
+  }
   const TcPlan pl = make_tc_plan(n_rows, n_keys, c.L.Dtc, c.sms);
   PassParams P{};
   P.n_rows = n_rows;
@@ -1308,13 +1348,49 @@ void run_apply_tc(Ctx& c, bool rows_x, int mode, const float* pot_in, const floa
   T.tiles_per_split = pl.tiles_per_split;
   T.c2 = c.c2;
   TcApply A{};
-  A.row_lse = c.tc_lse;
-  A.row_mass = pot_in ? c.tc_mass : nullptr;
+  A.row_lse = lse;
+  A.row_mass = pot_in ? mass : nullptr;
   A.x = rows_x ? p->x : p->y;
   A.inv_key_scale = 1.0f / c.tc_scale;
   memcpy(A.ctr, c.tc_ctr.c, sizeof(A.ctr));
   const double pairs = static_cast<double>(n_rows) * static_cast<double>(n_keys);
-  if (mode == kApplyGrad) {
+  if (mode == kApplyDiff) {
+    const int64_t rpad = rows_x ? c.L.tx : c.L.ty, kpad = rows_x ? c.L.ty : c.L.tx;
+    unsigned* vmax = reinterpret_cast<unsigned*>(c.scal + kVMax);
+    unsigned* dgmax = reinterpret_cast<unsigned*>(c.scal + kDgMax);
+    float* vinv = reinterpret_cast<float*>(c.scal + kVInv);
+    CK(cudaMemsetAsync(vmax, 0, sizeof(unsigned), c.st));
+    CK(cudaMemsetAsync(dgmax, 0, sizeof(unsigned), c.st));
+    dg_prep_kernel<<<reduce_blocks(kpad, c.sms), 256, 0, c.st>>>(pay, n_keys, kpad, c.tc_dg, dgmax);
+    CK(cudaGetLastError());
+    pay_maxabs_kernel<<<reduce_blocks(n_rows * p->d, c.sms), 256, 0, c.st>>>(row_v, n_rows, p->d,
+                                                                            p->d, vmax);
+    CK(cudaGetLastError());
+    const unsigned vb = static_cast<unsigned>(ceil_div(rpad, 256));
+    const float rk = static_cast<float>(c.tc_rkey);
+    const float* xr = rows_x ? p->x : p->y;
+    switch (c.L.Dtc) {
+      case 32:
+        build_vrow_image_kernel<32><<<vb, 256, 0, c.st>>>(row_v, xr, n_rows, rpad, p->d, c.tc_ctr,
+                                                          vmax, dgmax, rk, c.tc_vimg, c.tc_vrow, vinv);
+        break;
+      case 48:
+        build_vrow_image_kernel<48><<<vb, 256, 0, c.st>>>(row_v, xr, n_rows, rpad, p->d, c.tc_ctr,
+                                                          vmax, dgmax, rk, c.tc_vimg, c.tc_vrow, vinv);
+        break;
+      default:
+        build_vrow_image_kernel<64><<<vb, 256, 0, c.st>>>(row_v, xr, n_rows, rpad, p->d, c.tc_ctr,
+                                                          vmax, dgmax, rk, c.tc_vimg, c.tc_vrow, vinv);
+        break;
+    }
+    CK(cudaGetLastError());
+    g_launches.fetch_add(3, std::memory_order_relaxed);
+    A.v_img = c.tc_vimg;
+    A.v_row = c.tc_vrow;
+    A.key_dg = c.tc_dg;
+    A.v_inv_scale = vinv;
+  }
+  if (mode != kApplyPay) {
     A.out = out;
     A.out_stride = out_stride;
     int ti = c.timer->begin();
@@ -1601,8 +1677,11 @@ double check_potential(Ctx& c, const float* f, const float* g) {
 // mass is then its weight). The keys must carry their biases. Channels go 16 at a time.
 void transport_pass(Ctx& c, bool rows_x, const float* pot_in, const float* pay, int k, int stride,
                     float* out, int out_stride, const float* row_v = nullptr) {
-  if (c.use_tc && !row_v) {
-    run_apply_tc(c, rows_x, kApplyPay, pot_in, pay, k, stride, out, out_stride);
+  if (c.use_tc) {
+    if (row_v)
+      run_apply_tc(c, rows_x, kApplyDiff, pot_in, pay, 1, stride, out, out_stride, row_v);
+    else
+      run_apply_tc(c, rows_x, kApplyPay, pot_in, pay, k, stride, out, out_stride);
     return;
   }
   const int64_t n_keys = rows_x ? c.p->m : c.p->n;
@@ -1800,7 +1879,6 @@ fs_status hvp_impl(const fs_problem* p, const float* g, const float* v, float* o
   Ctx c{};
   fs_status s = begin(c, p, ws, ws_bytes, stream, kTransportChannels);
   if (s != FS_OK) return s;
-  if (p->d > 16) return FS_ERR_UNSUPPORTED_D;
   if (p->cost != FS_COST_SQEUCLIDEAN) return FS_ERR_OPTION;
   if (!g || !v || !out) return FS_ERR_NULL;
   if (!aligned4(g) || !aligned4(v) || !aligned4(out)) return FS_ERR_ALIGNMENT;
@@ -1810,7 +1888,7 @@ fs_status hvp_impl(const fs_problem* p, const float* g, const float* v, float* o
   Timer timer(c.st);
   c.timer = &timer;
   return guarded(c.st, [&]() -> fs_status {
-    fs_status r = prepare_all(c, {{g, p->m}}, false);
+    fs_status r = prepare_all(c, {{g, p->m}}, true);
     if (r != FS_OK) return r;
     const int64_t n = p->n, m = p->m, nm = n + m;
     const int32_t d = p->d;
@@ -1840,6 +1918,9 @@ fs_status hvp_impl(const fs_problem* p, const float* g, const float* v, float* o
     // 1. keys y carry g; ft = F(g) gives keys x their biases kappa ft + log2 a
     set_bias(c, false, g);
     run_pass(c, true, kPot, nullptr, ft, nullptr, nullptr, nullptr);
+    // From here on every bias is fixed: the tensor-core apply passes compute each
+    // direction's row offsets once.
+    c.tc_reuse = true;
     // 2. the gradient at the plan of (ft, g), r and the column pass's payload
     run_pass(c, true, kGrad, nullptr, nullptr, nullptr, grad, nullptr);
     hvp_row_prep_kernel<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, c.st>>>(

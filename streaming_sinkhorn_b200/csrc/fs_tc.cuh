@@ -400,7 +400,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
 
 // ---- the apply pass: sum_j p_ij U_j at fixed row offsets ------------------------------------
 
-enum TcApplyMode : int { kApplyGrad = 0, kApplyPay = 1 };
+//   kApplyGrad: U = the key coordinates, q = p; out = the gradient 2 w_i (x_i - T_i).
+//   kApplyPay:  U = a payload image (kPayChannels channels), q = p; out = mass_i sum q U / sum p.
+//   kApplyDiff: U = the key coordinates, q = p (dg_j + (y_j - x_i).v_i) with a second score
+//               W = V Y^T on the tensor cores; out = mass_i sum_j q_ij (y_j - x_i) / sum_j p_ij
+//               (the difference pass of the Hessian-vector product).
+enum TcApplyMode : int { kApplyGrad = 0, kApplyPay = 1, kApplyDiff = 2 };
 // Weights p <= 1 are stored as fp16(2^15 p): the largest lands below fp16's maximum and
 // weights down to 2^-39 keep their leading bits.
 constexpr float kPScale = 32768.0f;
@@ -415,8 +420,15 @@ struct TcApply {
   float* out;                    // results: row i, channel c at out[i * out_stride + c]
   int32_t out_k;                 // kApplyPay: channels written
   int32_t out_stride;
-  float inv_key_scale;           // kApplyGrad: 1 / s of the key image
-  double ctr[64];                // kApplyGrad: the centre the images were built about
+  float inv_key_scale;           // kApplyGrad, kApplyDiff: 1 / s of the key image
+  double ctr[64];                // kApplyGrad, kApplyDiff: the centre the images were built about
+  // kApplyDiff: the rows' vectors v_i as an image ([hi | lo], scaled by s_v), per row
+  // (qs_i, x'_i.v_i) with q stored as fp16(qs_i q), the keys' dg padded to whole tiles, and
+  // the device scalar 1 / s_v (the second score is W / (s_v s))
+  const unsigned char* v_img;
+  const float* v_row;
+  const float* key_dg;
+  const float* v_inv_scale;
 };
 
 template <int D, int NC, int MODE>
@@ -424,14 +436,21 @@ struct TcApplyShape {
   using S = TcShape<D>;
   static constexpr uint32_t PAY_BYTES = MODE == kApplyPay ? 128u * 2u * NC * 2u : 0u;
   static constexpr uint32_t HY_OFF = S::TILE_BYTES + PAY_BYTES;
+  static constexpr uint32_t DG_OFF = HY_OFF + S::HY_BYTES;  // kApplyDiff: the keys' dg
   static constexpr uint32_t STAGE_BYTES = HY_OFF + 1024u;
   static constexpr uint32_t P_BYTES = 128u * 128u * 2u;  // one fp16 weight tile
-  static constexpr size_t BASE = static_cast<size_t>(S::TILE_BYTES) + 2u * P_BYTES;
+  // the row image (and for kApplyDiff the rows' vector image) and two weight tiles
+  static constexpr size_t BASE =
+      static_cast<size_t>(S::TILE_BYTES) * (MODE == kApplyDiff ? 2u : 1u) + 2u * P_BYTES;
+  // TMEM columns: two score accumulators, the second score (kApplyDiff), the result
+  static constexpr uint32_t W_COL = 2u * kTcCols;
+  static constexpr uint32_t O_COL = W_COL + (MODE == kApplyDiff ? kTcCols : 0u);
   static constexpr int STAGES = BASE + 3u * STAGE_BYTES <= kTcSmemBudget ? 3 : 2;
   static constexpr size_t SMEM = BASE + static_cast<size_t>(STAGES) * STAGE_BYTES;
   static constexpr uint32_t U_LO_OFF = (NC / 8) * kCoreLBO;  // lo half of the U operand
   static_assert(NC % 16 == 0 && NC >= 16 && NC <= 128, "MMA N of the result");
   static_assert(SMEM <= kTcSmemBudget, "shared memory");
+  static_assert(O_COL + NC <= kTcApplyTmemCols, "tensor memory");
 };
 
 // Completes channel c of row i from its sums: a = sum_j q_ij U_jc and l = sum_j q_ij (the
@@ -445,13 +464,27 @@ __device__ __forceinline__ void tc_apply_finish(const PassParams& P, const TcApp
     const double t = A.ctr[c] + a / l;  // the barycentric projection T_i
     A.out[i * A.out_stride + c] =
         static_cast<float>(2.0 * w * (static_cast<double>(A.x[i * P.d_real + c]) - t));
-  } else {
+  } else if constexpr (MODE == kApplyPay) {
     if (c >= A.out_k) return;
     const double mass = A.row_mass ? static_cast<double>(A.row_mass[i])
                                    : (P.w ? static_cast<double>(P.w[i])
                                           : static_cast<double>(P.w_uniform));
     A.out[i * A.out_stride + c] = static_cast<float>(l > 0.0 ? mass * a / l : 0.0);
   }
+}
+
+// kApplyDiff: channel c of row i from a = sum_j q'_ij y'_jc, lq = sum_j q'_ij (q' = qs_i q,
+// fp16-rounded) and lp = sum_j p_ij: mass_i (a - x'_ic lq) / (qs_i lp).
+__device__ __forceinline__ void tc_diff_finish(const PassParams& P, const TcApply& A, int64_t i,
+                                               int c, double a, double lq, double lp) {
+  if (c >= P.d_real) return;
+  const double mass = A.row_mass ? static_cast<double>(A.row_mass[i])
+                                 : (P.w ? static_cast<double>(P.w[i])
+                                        : static_cast<double>(P.w_uniform));
+  const double qs = static_cast<double>(A.v_row[2 * i]);
+  const double xc = static_cast<double>(A.x[i * P.d_real + c]) - A.ctr[c];
+  A.out[i * A.out_stride + c] =
+      static_cast<float>(lp > 0.0 && qs > 0.0 ? mass * (a - xc * lq) / (qs * lp) : 0.0);
 }
 
 template <int D, int NC, int MODE>
@@ -467,13 +500,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ uint64_t acc_free_bar[2];  // score accumulator read by the 8 epilogue warps
   __shared__ uint64_t p_full[2];      // weight tile written by the 8 epilogue warps
   __shared__ uint64_t p_free[2];      // weight tile read by its result MMAs
+  __shared__ uint64_t w_free;         // kApplyDiff: second score read by the 8 epilogue warps
   __shared__ uint64_t a_bar, o_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
-  __shared__ float lsum[2][kTcRows];
+  __shared__ float lsum[2][kTcRows];   // per column half: sum of the rounded weights q'
+  __shared__ float lpsum[2][kTcRows];  // kApplyDiff: sum of the weights p
 
+  constexpr bool DIFF = MODE == kApplyDiff;
   unsigned char* sA = smem;
-  unsigned char* sP = smem + S::TILE_BYTES;
+  unsigned char* sV = smem + S::TILE_BYTES;  // kApplyDiff: the rows' vector image
+  unsigned char* sP = smem + S::TILE_BYTES * (DIFF ? 2 : 1);
   unsigned char* sStage = sP + 2 * Sh::P_BYTES;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -496,6 +533,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&p_full[b], kTcEpiWarps);
       mbar_init(&p_free[b], 1);
     }
+    mbar_init(&w_free, kTcEpiWarps);
     mbar_init(&a_bar, 1);
     mbar_init(&o_bar, 1);
     abort_sh = 0;
@@ -511,19 +549,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t tmem_o = tmem + 2u * kTcCols;  // the result accumulator, NC columns
+  const uint32_t tmem_w = tmem + Sh::W_COL;  // kApplyDiff: the second score
+  const uint32_t tmem_o = tmem + Sh::O_COL;  // the result accumulator, NC columns
 
   const int quarter = warp & 3, half = (warp >> 2) & 1;
   const int r = quarter * 32 + lane;
   const int64_t i = row0 + r;
-  u64 L = pk(0.0f, 0.0f);  // epilogue: sum of this row's rounded weights over its half
+  u64 L = pk(0.0f, 0.0f);   // epilogue: sum of this row's rounded weights q' over its half
+  u64 Lp = pk(0.0f, 0.0f);  // kApplyDiff: sum of the weights p
 
   if (warp == kTcEpiWarps) {
     // ---- producer ---------------------------------------------------------------------
     if (lane == 0) {
       int issued = 0;
-      mbar_expect_tx(&a_bar, S::TILE_BYTES);
+      mbar_expect_tx(&a_bar, S::TILE_BYTES * (DIFF ? 2u : 1u));
       bulk_g2s(sA, T.row_img + (row0 >> 7) * S::TILE_BYTES, S::TILE_BYTES, &a_bar);
+      if constexpr (DIFF)
+        bulk_g2s(sV, A.v_img + (row0 >> 7) * S::TILE_BYTES, S::TILE_BYTES, &a_bar);
       for (int t = 0; t < n_tiles; ++t) {
         const int st = t % ST;
         if (t >= ST && !tc_wait(&free_bar[st], static_cast<uint32_t>((t - ST) / ST) & 1u, abort))
@@ -531,12 +573,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         unsigned char* dst = sStage + st * Sh::STAGE_BYTES;
         const int64_t kt = t_begin + t;
         fence_proxy_async_smem();
-        mbar_expect_tx(&full_bar[st], S::TILE_BYTES + Sh::PAY_BYTES + S::HY_BYTES);
+        mbar_expect_tx(&full_bar[st], S::TILE_BYTES + Sh::PAY_BYTES + S::HY_BYTES *
+                                                                     (DIFF ? 2u : 1u));
         bulk_g2s(dst, T.key_img + kt * S::TILE_BYTES, S::TILE_BYTES, &full_bar[st]);
         if constexpr (MODE == kApplyPay)
           bulk_g2s(dst + S::TILE_BYTES, A.pay_img + kt * Sh::PAY_BYTES, Sh::PAY_BYTES,
                    &full_bar[st]);
         bulk_g2s(dst + Sh::HY_OFF, T.key_hy + kt * kTcCols, S::HY_BYTES, &full_bar[st]);
+        if constexpr (DIFF)
+          bulk_g2s(dst + Sh::DG_OFF, A.key_dg + kt * kTcCols, S::HY_BYTES, &full_bar[st]);
         ++issued;
       }
       if (*abort) {
@@ -560,6 +605,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc_fence_after();
           tc_issue_scores<D>(tmem + static_cast<uint32_t>(b) * kTcCols, smem_u32(sA),
                              smem_u32(sStage + st * Sh::STAGE_BYTES), idesc_s);
+          if constexpr (DIFF) {
+            // the second score W = V Y^T, single-buffered: tile t - 1's must have been read
+            if (t >= 1 && !tc_wait(&w_free, static_cast<uint32_t>(t - 1) & 1u, abort)) break;
+            tc_fence_after();
+            tc_issue_scores<D>(tmem_w, smem_u32(sV), smem_u32(sStage + st * Sh::STAGE_BYTES),
+                               idesc_s);
+          }
           tc_commit(&mma_bar[b]);
         }
         if (t >= 1) {
@@ -594,30 +646,74 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (i < P.n_rows) off = P.kappa_f * T.row_nrm[i] + A.row_lse[i];
     const u64 c2 = pk(T.c2, T.c2);
     const u64 noff = pk(-off, -off);
+    // kApplyDiff: q'_ij = qs_i p_ij (dg_j + w_scale W_ij - x'_i.v_i)
+    float qs = 0.0f, xv = 0.0f;
+    if (DIFF && i < P.n_rows) {
+      qs = A.v_row[2 * i];
+      xv = A.v_row[2 * i + 1];
+    }
+    const float w_scale = DIFF ? *A.v_inv_scale * A.inv_key_scale : 0.0f;
+    const u64 wsc = pk(w_scale, w_scale);
+    const u64 nxv = pk(-xv, -xv);
     for (int u = 0; u < n_tiles; ++u) {
       const int b = u & 1, st = u % ST, pb = u & 1;
       if (!tc_wait(&mma_bar[b], static_cast<uint32_t>(u >> 1) & 1u, abort)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             static_cast<uint32_t>(b) * kTcCols + half * 64;
-      float v[64];
-      tc_ld32_nowait(tbase, v);
-      tc_ld32_nowait(tbase + 32, v + 32);
-      tc_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_free_bar[b]);
+      const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+      const uint32_t tbase = tmem + lane_off + static_cast<uint32_t>(b) * kTcCols + half * 64;
       const u64* hv = reinterpret_cast<const u64*>(sStage + st * Sh::STAGE_BYTES + Sh::HY_OFF) +
                       half * 32;
-      uint32_t h2[32];  // fp16 pairs of 2^15 p
+      uint32_t h2[32];  // fp16 pairs of the weights q' (2^15 p unless kApplyDiff)
+      if constexpr (!DIFF) {
+        float v[64];
+        tc_ld32_nowait(tbase, v);
+        tc_ld32_nowait(tbase + 32, v + 32);
+        tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_free_bar[b]);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        float t0, t1;
-        upk(add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), hv[j]), noff), t0, t1);
-        const __half2 h = __floats2half2_rn(ex2(t0) * kPScale, ex2(t1) * kPScale);
-        const float2 back = __half22float2(h);
-        L = add2(L, pk(back.x, back.y));
-        h2[j] = *reinterpret_cast<const uint32_t*>(&h);
+        for (int j = 0; j < 32; ++j) {
+          float t0, t1;
+          upk(add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), hv[j]), noff), t0, t1);
+          const __half2 h = __floats2half2_rn(ex2(t0) * kPScale, ex2(t1) * kPScale);
+          const float2 back = __half22float2(h);
+          L = add2(L, pk(back.x, back.y));
+          h2[j] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+      } else {
+        const u64* dv = reinterpret_cast<const u64*>(sStage + st * Sh::STAGE_BYTES + Sh::DG_OFF) +
+                        half * 32;
+        const uint32_t wbase = tmem_w + lane_off + half * 64;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // two chunks of 32 columns
+          float v[32], wv[32];
+          tc_ld32_nowait(tbase + 32 * h, v);
+          tc_ld32_nowait(wbase + 32 * h, wv);
+          tc_wait_ld();
+          if (h == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(&acc_free_bar[b]);
+              mbar_arrive(&w_free);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int jj = 16 * h + j;
+            float t0, t1, p0, p1, f0, f1;
+            upk(add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), hv[jj]), noff), t0, t1);
+            p0 = ex2(t0);
+            p1 = ex2(t1);
+            Lp = add2(Lp, pk(p0, p1));
+            upk(add2(fma2(wsc, pk(wv[2 * j], wv[2 * j + 1]), dv[jj]), nxv), f0, f1);
+            const __half2 hq = __floats2half2_rn(qs * p0 * f0, qs * p1 * f1);
+            const float2 back = __half22float2(hq);
+            L = add2(L, pk(back.x, back.y));
+            h2[jj] = *reinterpret_cast<const uint32_t*>(&hq);
+          }
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&free_bar[st]);  // its hy has been read
@@ -640,9 +736,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   {
-    float l0, l1;
+    float l0, l1, p0, p1;
     upk(L, l0, l1);
-    if (warp < kTcEpiWarps) lsum[half][r] = l0 + l1;
+    upk(Lp, p0, p1);
+    if (warp < kTcEpiWarps) {
+      lsum[half][r] = l0 + l1;
+      lpsum[half][r] = p0 + p1;
+    }
   }
   __syncthreads();
   if (abort_sh) {
@@ -658,19 +758,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int c = 0; c < NH; c += 8) tc_ld8_nowait(obase + c, o + c);
       tc_wait_ld();
       const double l = static_cast<double>(lsum[0][r]) + static_cast<double>(lsum[1][r]);
-      const double inv = MODE == kApplyGrad ? static_cast<double>(A.inv_key_scale)
-                                            : static_cast<double>(*A.pay_inv_scale);
+      const double lp = static_cast<double>(lpsum[0][r]) + static_cast<double>(lpsum[1][r]);
+      const double inv = MODE == kApplyPay ? static_cast<double>(*A.pay_inv_scale)
+                                           : static_cast<double>(A.inv_key_scale);
       if (i < P.n_rows) {
         if (P.n_splits == 1) {
 #pragma unroll
-          for (int c = 0; c < NH; ++c)
-            tc_apply_finish<MODE>(P, A, i, half * NH + c, static_cast<double>(o[c]) * inv, l);
+          for (int c = 0; c < NH; ++c) {
+            const double a = static_cast<double>(o[c]) * inv;
+            if constexpr (DIFF)
+              tc_diff_finish(P, A, i, half * NH + c, a, l, lp);
+            else
+              tc_apply_finish<MODE>(P, A, i, half * NH + c, a, l);
+          }
         } else {
+          // partials: [sum q'][channels][sum p (kApplyDiff)], split-major
+          constexpr int NP = NC + (DIFF ? 1 : 0);
           const int64_t ps = static_cast<int64_t>(split);
           if (half == 0) P.part_l[ps * P.rows_pad + i] = static_cast<float>(l);
+          if (DIFF && half == 0) P.part_a[(ps * NP + NC) * P.rows_pad + i] = static_cast<float>(lp);
 #pragma unroll
           for (int c = 0; c < NH; ++c)
-            P.part_a[(ps * NC + half * NH + c) * P.rows_pad + i] =
+            P.part_a[(ps * NP + half * NH + c) * P.rows_pad + i] =
                 static_cast<float>(static_cast<double>(o[c]) * inv);
         }
       }
@@ -690,15 +799,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // add) and completes each row.
 template <int NC, int MODE>
 __global__ void __launch_bounds__(256) tc_apply_combine_kernel(const PassParams P, const TcApply A) {
+  constexpr bool DIFF = MODE == kApplyDiff;
+  constexpr int NP = NC + (DIFF ? 1 : 0);
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= P.n_rows) return;
-  double l = 0.0;
-  for (int s = 0; s < P.n_splits; ++s) l += P.part_l[static_cast<int64_t>(s) * P.rows_pad + i];
+  double l = 0.0, lp = 0.0;
+  for (int s = 0; s < P.n_splits; ++s) {
+    l += P.part_l[static_cast<int64_t>(s) * P.rows_pad + i];
+    if (DIFF) lp += P.part_a[(static_cast<int64_t>(s) * NP + NC) * P.rows_pad + i];
+  }
   for (int c = 0; c < NC; ++c) {
     double a = 0.0;
     for (int s = 0; s < P.n_splits; ++s)
-      a += P.part_a[(static_cast<int64_t>(s) * NC + c) * P.rows_pad + i];
-    tc_apply_finish<MODE>(P, A, i, c, a, l);
+      a += P.part_a[(static_cast<int64_t>(s) * NP + c) * P.rows_pad + i];
+    if constexpr (DIFF)
+      tc_diff_finish(P, A, i, c, a, l, lp);
+    else
+      tc_apply_finish<MODE>(P, A, i, c, a, l);
   }
 }
 
@@ -813,6 +930,63 @@ __global__ void __launch_bounds__(256) build_pay_image_kernel(const float* u, in
     *reinterpret_cast<__half*>(img + tc_image_offset(i, c, 2 * NC)) = hi;
     *reinterpret_cast<__half*>(img + tc_image_offset(i, NC + c, 2 * NC)) = lo;
   }
+}
+
+// The difference pass's key column dg, zero-padded to whole tiles, and max |dg| (float bits).
+__global__ void __launch_bounds__(256) dg_prep_kernel(const float* dg, int64_t count,
+                                                      int64_t count_pad, float* dg_pad,
+                                                      unsigned* maxabs_bits) {
+  float mx = 0.0f;
+  for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < count_pad;
+       j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float v = j < count ? dg[j] : 0.0f;
+    dg_pad[j] = v;
+    mx = fmaxf(mx, fabsf(v));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(maxabs_bits, __float_as_uint(mx));
+}
+
+// The difference pass's row side: the image of the vectors v_i (scaled by the power of two
+// s_v = 2^floor(log2(16384 / max|v|)), [hi | lo]), 1 / s_v, and per row
+//   qs_i = 2^14 / (max|dg| + |v_i| (r_key + |x'_i|))   and   x'_i.v_i,
+// where |dg_j + (y'_j - x'_i).v_i| <= max|dg| + |v_i| (|y'_j| + |x'_i|) and r_key bounds
+// |y'_j|, so |qs_i p_ij (dg_j + (y'_j - x'_i).v_i)| <= 2^14 for p <= 1 (fp16 range).
+template <int D>
+__global__ void __launch_bounds__(256) build_vrow_image_kernel(
+    const float* v, const float* x, int64_t count, int64_t count_pad, int32_t d_real,
+    const TcCenter ctr, const unsigned* vmax_bits, const unsigned* dgmax_bits, float r_key,
+    unsigned char* img, float* v_row, float* inv_scale) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const float mx = __uint_as_float(*vmax_bits);
+  int e = 0;
+  if (mx > 0.0f) e = static_cast<int>(floorf(log2f(16384.0f / mx)));
+  e = max(-120, min(120, e));
+  const float scale = exp2f(static_cast<float>(e));
+  if (i == 0) *inv_scale = exp2f(static_cast<float>(-e));
+  if (i >= count_pad) return;
+  double vv = 0.0, xx = 0.0, xv = 0.0;
+#pragma unroll 4
+  for (int k = 0; k < D; ++k) {
+    float u = 0.0f;
+    if (i < count && k < d_real) {
+      const double vk = static_cast<double>(v[i * d_real + k]);
+      const double xk = static_cast<double>(x[i * d_real + k]) - ctr.c[k];
+      vv += vk * vk;
+      xx += xk * xk;
+      xv += xk * vk;
+      u = static_cast<float>(vk * scale);
+    }
+    const __half hi = __float2half_rn(u);
+    const __half lo = __float2half_rn(u - __half2float(hi));
+    *reinterpret_cast<__half*>(img + tc_image_offset(i, k, 2 * D)) = hi;
+    *reinterpret_cast<__half*>(img + tc_image_offset(i, D + k, 2 * D)) = lo;
+  }
+  const double bound = static_cast<double>(__uint_as_float(*dgmax_bits)) +
+                       sqrt(vv) * (static_cast<double>(r_key) + sqrt(xx));
+  v_row[2 * i] = i < count && bound > 0.0 ? static_cast<float>(16384.0 / bound) : 0.0f;
+  v_row[2 * i + 1] = static_cast<float>(xv);
 }
 
 }  // namespace fs

@@ -200,14 +200,13 @@ def test_transport_and_hvp_argument_errors():
     assert ta(p, FAKE, FAKE, 0, 3, FAKE, FAKE, FAKE, need - 256, None) == "FS_ERR_WORKSPACE"
     too_wide = ctypes.byref(prob(d=65))
     assert ta(too_wide, FAKE, FAKE, 0, 3, FAKE, FAKE, FAKE, BIG, None) == "FS_ERR_UNSUPPORTED_D"
-    wide = ctypes.byref(prob(d=17))  # the HVP's difference pass has no tensor-core form yet
     hv = lambda *a: st(lib.fs_hvp(*a))  # noqa: E731
     bad_iter = _lib.fs_hvp_options(0, 1e-6)
     bad_tol = _lib.fs_hvp_options(10, -1.0)
     assert hv(p, FAKE, FAKE, FAKE, ctypes.byref(bad_iter), None, FAKE, need, None) == "FS_ERR_OPTION"
     assert hv(p, FAKE, FAKE, FAKE, ctypes.byref(bad_tol), None, FAKE, need, None) == "FS_ERR_OPTION"
     assert hv(p, FAKE, None, FAKE, None, None, FAKE, need, None) == "FS_ERR_NULL"
-    assert hv(wide, FAKE, FAKE, FAKE, None, None, FAKE, BIG, None) == "FS_ERR_UNSUPPORTED_D"
+    assert hv(too_wide, FAKE, FAKE, FAKE, None, None, FAKE, BIG, None) == "FS_ERR_UNSUPPORTED_D"
 
 
 def test_divergence_argument_errors():

@@ -71,9 +71,13 @@ def test_transport_apply_vector_form():
 # rounding, so the entries agree to ~1e-5 of the largest (measured worst 1.1e-5); 1e-4
 # leaves ten times that.
 HVP_TOL = 1e-4
+# d > 16: every transport product of the solve and the difference pass carry the fp16
+# rounding of the plan weights (2^-11 relative each, see TRANSPORT_REL); the tensor-core bar.
+HVP_TOL_TC = 5e-3
 
 
-@pytest.mark.parametrize("shape", [(120, 90, 2, 0.3), (250, 300, 3, 0.1), (80, 70, 8, 1.0)],
+@pytest.mark.parametrize("shape", [(120, 90, 2, 0.3), (250, 300, 3, 0.1), (80, 70, 8, 1.0),
+                                   (120, 100, 32, 4.0), (90, 110, 64, 8.0)],
                          ids=lambda s: "n{}-m{}-d{}".format(*s[:3]))
 def test_hvp_matches_oracle(shape):
     n, m, d, eps = shape
@@ -88,8 +92,9 @@ def test_hvp_matches_oracle(shape):
     ref = oracle.hvp(w.x, w.y, w.a, w.b, w.eps, g32, v)
     assert rep["cg_iters"] >= 1
     hv = hv.cpu().numpy().astype(np.float64)
-    close(hv, ref, HVP_TOL)
-    assert np.linalg.norm(hv - ref) <= HVP_TOL * np.linalg.norm(ref)
+    tol = HVP_TOL if d <= 16 else HVP_TOL_TC
+    close(hv, ref, tol)
+    assert np.linalg.norm(hv - ref) <= tol * np.linalg.norm(ref)
 
 
 
