@@ -244,13 +244,18 @@ FS_API fs_status fs_divergence(const fs_problem* p, const fs_solve_options* opt,
 /*
  * Transport products and the Hessian-vector product (FlashSinkhorn summary, section 3:
  * transport-matrix application; an HVP decomposed into transport-vector and
- * transport-matrix products), for d <= 16 (FS_ERR_UNSUPPORTED_D otherwise). Both stream the
- * plan P_ij = a_i b_j exp((f_i + g_j - C_ij)/eps) like the potential passes (and screen it
- * the same way) and never store it.
+ * transport-matrix products), for every d <= FS_MAX_D. Both stream the plan
+ * P_ij = a_i b_j exp((f_i + g_j - C_ij)/eps) like the potential passes and never store it.
+ * For d <= 16 the passes run on the FMA path in float32 (and screen the plan the same way
+ * as the potential passes). For d > 16 they run on the tensor cores: a first pass takes
+ * each row's log-sum-exp, a second forms the weights p_ij = P_ij / (P 1)_i <= 1, stores
+ * them as fp16 (2^-11 relative rounding each) and multiplies them by the payload (a [hi |
+ * lo] fp16 pair, ~2^-22 relative) with fp32 accumulation, and divides by the sum of the
+ * same rounded weights; the HVP's difference pass also takes v_i.y_j on the tensor cores.
  *
- * Their workspace is fs_transport_workspace_bytes(p) (0 for an invalid shape or d > 16),
- * larger than fs_workspace_bytes(p): keys with up to 16 payload channels and the HVP's
- * vectors.
+ * Their workspace is fs_transport_workspace_bytes(p) (0 for an invalid shape or
+ * d > FS_MAX_D), larger than fs_workspace_bytes(p): payload keys or images with up to 16
+ * channels and the HVP's vectors.
  */
 FS_API size_t fs_transport_workspace_bytes(const fs_problem* p);
 
@@ -306,7 +311,9 @@ FS_API fs_status fs_cost(const fs_problem* p, const float* f, const float* g, do
 
 /*
  * Envelope gradient of the cost with respect to x (FlashSinkhorn summary, section 3:
- * transport-matrix application without materialising P):
+ * transport-matrix application without materialising P). For d > 16 it runs on the tensor
+ * cores as two streaming passes (the rows' log-sum-exp, then sum_j Pt_ij y_j with the
+ * weights in fp16 as for the transport products):
  *   ft = F(g) (a fresh f-update, fused into the same pass), Pt_ij = a_i b_j
  *   exp((ft_i + g_j - C_ij)/eps), so sum_j Pt_ij = a_i and
  *   grad_x[i, :] = 2 * (a_i x_i - sum_j Pt_ij y_j) = 2 a_i (x_i - T_i),

@@ -21,11 +21,12 @@
 // (stride-byte offset). The apply pass uses it so as the B operand of sum_j p_ij y_j. A
 // tile is one contiguous block that a single TMA bulk copy moves into shared memory.
 //
-// Potential pass (lse_pass_tc_kernel): one CTA per 128-row block and column split, 10 warps
-// with fixed roles. Warp 8 streams key tiles (image + hy) through a 3-stage ring with TMA
-// bulk copies; warp 9 issues the MMAs of tile t into one of two TMEM accumulators; warps
-// 0-7 run the online max/sum (warp w reads TMEM lanes 32 (w % 4) .. +31, the columns of
-// half w / 4 of each tile). Roles hand off through mbarriers only.
+// Potential pass (lse_pass_tc_kernel): one CTA per 128-row block and column split, 18 warps
+// with fixed roles. Warp 16 streams key tiles (image + hy) through a 3-stage ring with TMA
+// bulk copies; warp 17 issues the MMAs of tile t into one of two TMEM accumulators; warps
+// 0-15 run the online max/sum (warp w reads TMEM lanes 32 (w % 4) .. +31, the 32 columns of
+// group w / 4 of each tile: sixteen warps keep enough exponentials in flight for the MUFU
+// unit). Roles hand off through mbarriers only.
 //
 // Apply pass (lse_apply_tc_kernel, FlashSinkhorn summary, section 3, "Transport Matrix
 // Application"): out_i = sum_j p_ij U_j / sum_j p_ij with p_ij = 2^(z_ij - LSE2_i), the
@@ -45,15 +46,18 @@ namespace fs {
 constexpr int kTcRows = 128;     // rows per CTA (MMA M)
 constexpr int kTcCols = 128;     // key columns per tile (MMA N of the score)
 constexpr int kTcStages = 3;
-constexpr int kTcEpiWarps = 8;  // epilogue warps: 4 TMEM lane quarters x 2 column halves
+constexpr int kTcEpiWarps = 16;  // epilogue warps: 4 TMEM lane quarters x 4 column groups
+constexpr int kTcGroups = kTcEpiWarps / 4;  // column groups of a tile
+constexpr int kTcGC = kTcCols / kTcGroups;  // columns of one group
 constexpr int kTcThreads = (kTcEpiWarps + 2) * 32;  // + a producer warp and an MMA warp
+static_assert(kTcGC % 32 == 0, "whole 32-column TMEM loads per group");
 constexpr uint32_t kTcTmemCols = 256;  // potential pass: two accumulators of kTcCols columns
 constexpr uint32_t kTcApplyTmemCols = 512;  // apply pass: two score accumulators + the result
 constexpr uint32_t kCoreLBO = 16u * 128u;  // next K-block of a core-matrix tile
 constexpr uint32_t kCoreSBO = 128u;        // next 8-point group
 // Dynamic shared memory a tensor-core pass may take (the opt-in limit is 227 KB; the
-// kernels' static shared memory is under 2 KB).
-constexpr size_t kTcSmemBudget = 225u * 1024u;
+// kernels' static shared memory is at most 5 KB).
+constexpr size_t kTcSmemBudget = 222u * 1024u;
 
 template <int D>
 struct TcShape {
@@ -178,16 +182,21 @@ struct TcParams {
 };
 
 // Waits for phase `parity` of `bar`, giving up after kWaitLimitNs or as soon as another
-// role of the CTA has raised `abort`.
+// role of the CTA has raised `abort`. Between checks the thread sleeps in the barrier wait
+// (up to 2 us per try), and the abort flag and the clock are read only every 16th try, so
+// waiting warps leave the shared-memory and special-function issue queues to the warps
+// that are computing.
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (global_ns() - t0 > kWaitLimitNs) {
-      *abort = 1;
-      return false;
+  for (uint32_t k = 1;; ++k) {
+    if (mbar_try_wait_sleep(bar, parity, 2000u)) return true;
+    if ((k & 15u) == 0u) {
+      if (*abort) return false;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        return false;
+      }
     }
   }
 }
@@ -208,7 +217,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
   __shared__ uint64_t a_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
-  __shared__ float2 merge[kTcRows];
+  __shared__ float2 merge[kTcGroups][kTcRows];
 
   unsigned char* sA = smem;
   unsigned char* sStage = smem + S::TILE_BYTES;
@@ -248,7 +257,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
 
   float m = -INFINITY;  // epilogue row state (origin-free running offset) ...
   u64 L = pk(0.0f, 0.0f);
-  const int quarter = warp & 3, half = (warp >> 2) & 1;
+  const int quarter = warp & 3, grp = warp >> 2;
   const int r = quarter * 32 + lane;
   const int64_t i = row0 + r;
 
@@ -302,7 +311,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
                                 static_cast<uint32_t>((committed - 1) >> 1) & 1u);
     }
   } else {
-    // ---- epilogue warps: online max/sum of one row over half of every tile ------------
+    // ---- epilogue warps: online max/sum of one row over one column group of every tile --
+    constexpr int GP = kTcGC / 2;  // column pairs of a group
     const float knrm = (i < P.n_rows) ? P.kappa_f * T.row_nrm[i] : 0.0f;
     float base = 0.0f, mo = knrm;
     const u64 c2 = pk(T.c2, T.c2);
@@ -312,26 +322,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
       tc_fence_after();
       const float* hy = reinterpret_cast<const float*>(sStage + st * S::STAGE_BYTES + S::TILE_BYTES);
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             static_cast<uint32_t>(b) * kTcCols + half * 64;
-      float v[64];
-      tc_ld32_nowait(tbase, v);
-      tc_ld32_nowait(tbase + 32, v + 32);
+                             static_cast<uint32_t>(b) * kTcCols + grp * kTcGC;
+      float v[kTcGC];
+#pragma unroll
+      for (int c = 0; c < kTcGC; c += 32) tc_ld32_nowait(tbase + c, v + c);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_free_bar[b]);
-      const u64* hv = reinterpret_cast<const u64*>(hy + half * 64);
-      u64 tv[32];
+      const ulonglong2* hv = reinterpret_cast<const ulonglong2*>(hy + grp * kTcGC);
+      u64 tv[GP];
       const u64 nmo = pk(-mo, -mo);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) tv[j] = add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), hv[j]), nmo);
+      for (int j = 0; j < GP; j += 2) {
+        const ulonglong2 h = hv[j / 2];  // four biases in one 16-byte (broadcast) load
+        tv[j] = add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), h.x), nmo);
+        tv[j + 1] = add2(fma2(c2, pk(v[2 * j + 2], v[2 * j + 3]), h.y), nmo);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&free_bar[st]);
       float a0, a1;
       upk(tv[0], a0, a1);
       float mx = fmaxf(a0, a1);
 #pragma unroll
-      for (int j = 1; j < 32; ++j) {
+      for (int j = 1; j < GP; ++j) {
         upk(tv[j], a0, a1);
         mx = max3(mx, a0, a1);
       }
@@ -341,13 +355,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
         L = mul2(L, pk(sc, sc));
         const u64 sh = pk(-mx, -mx);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) tv[j] = add2(tv[j], sh);
+        for (int j = 0; j < GP; ++j) tv[j] = add2(tv[j], sh);
         m = mx_abs;
         base = mx_abs;
         mo = knrm + m;
       }
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
+      for (int j = 0; j < GP; ++j) {
         float t0, t1;
         upk(tv[j], t0, t1);
         L = add2(L, pk(ex2(t0), ex2(t1)));
@@ -361,18 +375,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
   if (abort_sh) {
     if (tid == 0) atomicOr(P.err, kErrTimeout);
   } else {
-    // Merge the two column halves of each row, then finish the row.
+    // Merge the column groups of each row, then finish the row.
     float l0, l1;
     upk(L, l0, l1);
-    if (warp < kTcEpiWarps && half == 1) merge[r] = make_float2(m, l0 + l1);
+    if (warp < kTcEpiWarps) merge[grp][r] = make_float2(m, l0 + l1);
     __syncthreads();
     double dev = 0.0, mass = 0.0;
-    if (warp < kTcEpiWarps && half == 0 && i < P.n_rows) {
-      const float2 o = merge[r];
-      const float mm = fmaxf(m, o.x);
+    if (warp < kTcEpiWarps && grp == 0 && i < P.n_rows) {
+      float mm = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < kTcGroups; ++q) mm = fmaxf(mm, merge[q][r].x);
       float l = 0.0f;
-      if (m != -INFINITY) l += (l0 + l1) * ex2(m - mm);
-      if (o.x != -INFINITY) l += o.y * ex2(o.x - mm);
+#pragma unroll
+      for (int q = 0; q < kTcGroups; ++q) {
+        const float2 o = merge[q][r];
+        if (o.x != -INFINITY) l += o.y * ex2(o.x - mm);
+      }
       if (P.n_splits == 1) {
         const double lse2 = static_cast<double>(mm) + log2(static_cast<double>(l));
         if (P.kind == kPot) {
@@ -504,8 +522,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ uint64_t a_bar, o_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
-  __shared__ float lsum[2][kTcRows];   // per column half: sum of the rounded weights q'
-  __shared__ float lpsum[2][kTcRows];  // kApplyDiff: sum of the weights p
+  __shared__ float lsum[kTcGroups][kTcRows];   // per column group: sum of the rounded q'
+  __shared__ float lpsum[kTcGroups][kTcRows];  // kApplyDiff: sum of the weights p
 
   constexpr bool DIFF = MODE == kApplyDiff;
   unsigned char* sA = smem;
@@ -552,10 +570,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem_w = tmem + Sh::W_COL;  // kApplyDiff: the second score
   const uint32_t tmem_o = tmem + Sh::O_COL;  // the result accumulator, NC columns
 
-  const int quarter = warp & 3, half = (warp >> 2) & 1;
+  const int quarter = warp & 3, grp = warp >> 2;
   const int r = quarter * 32 + lane;
   const int64_t i = row0 + r;
-  u64 L = pk(0.0f, 0.0f);   // epilogue: sum of this row's rounded weights q' over its half
+  u64 L = pk(0.0f, 0.0f);   // epilogue: sum of this row's rounded weights q' over its group
   u64 Lp = pk(0.0f, 0.0f);  // kApplyDiff: sum of the weights p
 
   if (warp == kTcEpiWarps) {
@@ -641,7 +659,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       (void)mbar_wait_bounded(&o_bar, 0);
     }
   } else {
-    // ---- epilogue warps: weights of one row over half of every tile --------------------
+    // ---- epilogue warps: weights of one row over one column group of every tile ---------
+    constexpr int GP = kTcGC / 2;  // column pairs of a group
     float off = 1.0e30f;  // padding rows: every weight is 0
     if (i < P.n_rows) off = P.kappa_f * T.row_nrm[i] + A.row_lse[i];
     const u64 c2 = pk(T.c2, T.c2);
@@ -660,22 +679,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!tc_wait(&mma_bar[b], static_cast<uint32_t>(u >> 1) & 1u, abort)) break;
       tc_fence_after();
       const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-      const uint32_t tbase = tmem + lane_off + static_cast<uint32_t>(b) * kTcCols + half * 64;
+      const uint32_t tbase = tmem + lane_off + static_cast<uint32_t>(b) * kTcCols + grp * kTcGC;
       const u64* hv = reinterpret_cast<const u64*>(sStage + st * Sh::STAGE_BYTES + Sh::HY_OFF) +
-                      half * 32;
-      uint32_t h2[32];  // fp16 pairs of the weights q' (2^15 p unless kApplyDiff)
+                      grp * GP;
+      uint32_t h2[GP];  // fp16 pairs of the weights q' (2^15 p unless kApplyDiff)
       if constexpr (!DIFF) {
-        float v[64];
-        tc_ld32_nowait(tbase, v);
-        tc_ld32_nowait(tbase + 32, v + 32);
+        float v[kTcGC];
+#pragma unroll
+        for (int c = 0; c < kTcGC; c += 32) tc_ld32_nowait(tbase + c, v + c);
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_free_bar[b]);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < GP; ++j) {
           float t0, t1;
-          upk(add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), hv[j]), noff), t0, t1);
+          const ulonglong2 h4 = reinterpret_cast<const ulonglong2*>(hv)[j / 2];
+          upk(add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), (j & 1) ? h4.y : h4.x), noff), t0, t1);
           const __half2 h = __floats2half2_rn(ex2(t0) * kPScale, ex2(t1) * kPScale);
           const float2 back = __half22float2(h);
           L = add2(L, pk(back.x, back.y));
@@ -683,15 +703,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       } else {
         const u64* dv = reinterpret_cast<const u64*>(sStage + st * Sh::STAGE_BYTES + Sh::DG_OFF) +
-                        half * 32;
-        const uint32_t wbase = tmem_w + lane_off + half * 64;
+                        grp * GP;
+        const uint32_t wbase = tmem_w + lane_off + grp * kTcGC;
+        constexpr int NCH = kTcGC / 32;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {  // two chunks of 32 columns
+        for (int h = 0; h < NCH; ++h) {  // chunks of 32 columns
           float v[32], wv[32];
           tc_ld32_nowait(tbase + 32 * h, v);
           tc_ld32_nowait(wbase + 32 * h, wv);
           tc_wait_ld();
-          if (h == 1) {
+          if (h == NCH - 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -721,8 +742,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // K-major weight tile: core(row group, key block) at (kb * 16 + r / 8) * 128 + (r % 8) * 16
       unsigned char* pt = sP + pb * Sh::P_BYTES + (r >> 3) * 128 + (r & 7) * 16;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int kb = half * 8 + c;
+      for (int c = 0; c < kTcGC / 8; ++c) {
+        const int kb = grp * (kTcGC / 8) + c;
         *reinterpret_cast<uint4*>(pt + kb * 16 * 128) =
             make_uint4(h2[4 * c], h2[4 * c + 1], h2[4 * c + 2], h2[4 * c + 3]);
       }
@@ -740,15 +761,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     upk(L, l0, l1);
     upk(Lp, p0, p1);
     if (warp < kTcEpiWarps) {
-      lsum[half][r] = l0 + l1;
-      lpsum[half][r] = p0 + p1;
+      lsum[grp][r] = l0 + l1;
+      lpsum[grp][r] = p0 + p1;
     }
   }
   __syncthreads();
   if (abort_sh) {
     if (tid == 0) atomicOr(P.err, kErrTimeout);
-  } else if (warp < kTcEpiWarps) {
-    // The result accumulator: this warp's rows, channels [half * NC / 2, (half + 1) * NC / 2).
+  } else if (warp < 8) {
+    // The result accumulator: this warp's rows, channels [half * NC / 2, (half + 1) * NC / 2)
+    // (the warps of the first two column groups).
+    const int half = grp;
     if (mbar_wait_bounded(&o_bar, 0)) {
       tc_fence_after();
       constexpr int NH = NC / 2;
@@ -757,8 +780,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int c = 0; c < NH; c += 8) tc_ld8_nowait(obase + c, o + c);
       tc_wait_ld();
-      const double l = static_cast<double>(lsum[0][r]) + static_cast<double>(lsum[1][r]);
-      const double lp = static_cast<double>(lpsum[0][r]) + static_cast<double>(lpsum[1][r]);
+      double l = 0.0, lp = 0.0;
+#pragma unroll
+      for (int q = 0; q < kTcGroups; ++q) {
+        l += static_cast<double>(lsum[q][r]);
+        lp += static_cast<double>(lpsum[q][r]);
+      }
       const double inv = MODE == kApplyPay ? static_cast<double>(*A.pay_inv_scale)
                                            : static_cast<double>(A.inv_key_scale);
       if (i < P.n_rows) {
