@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--n", type=int, default=None,
                     help="clustered workload only: use n = m points (eps by the same spacing rule)")
+    ap.add_argument("--d", type=int, default=None,
+                    help="50k-point mixture workload (c4) only: use d coordinates, eps = d / 64")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -60,9 +62,17 @@ def parse():
     return ap.parse_args()
 
 
-def workload(cfg: str, rank: int, n_override=None):
+def workload(cfg: str, rank: int, n_override=None, d_override=None):
     from streaming_sinkhorn_b200 import workloads
     import dataclasses
+    if d_override is not None:
+        if cfg != "c4":
+            raise SystemExit("--d applies to the 50k-point mixture workload (c4) only")
+        # the same recipe at another width; eps grows with d so that kappa |x - y|^2 keeps the
+        # scale it has at d = 64, eps = 1
+        w = workloads.mixture_pair(n=50000, d=d_override, k=10, mean_scale=2.0, std=1.0,
+                                   seed=3 + 1000 * rank, eps=d_override / 64.0, n_iters=100)
+        return dataclasses.replace(w, name=f"mix_50k_d{d_override}")
     if n_override is not None:
         if cfg != "c5":
             raise SystemExit("--n applies to the clustered workload (c5) only")
@@ -227,7 +237,7 @@ def run_native(args, rank, world, local_rank):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local_rank))
-    w = workload(args.config, rank, args.n)
+    w = workload(args.config, rank, args.n, args.d)
     dev = torch.device("cuda", local_rank)
     x = torch.from_numpy(w.x).to(dev)
     y = torch.from_numpy(w.y).to(dev)
@@ -519,7 +529,7 @@ def run_e2e(args, w, dev, world, dist):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    w = workload(args.config, 0, args.n)
+    w = workload(args.config, 0, args.n, args.d)
     per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample(w, min(per_step, 3.0))

@@ -49,7 +49,9 @@ extern "C" {
 /* Same type as cudaStream_t; NULL selects the legacy default stream. */
 typedef struct CUstream_st* fs_stream_t;
 
-#define FS_MAX_D 64
+/* Widest points: d <= 16 runs on the FMA path, 16 < d <= 64 on the tensor cores with the
+ * operand images resident, 64 < d <= 1024 on the tensor cores in 64-coordinate K-chunks. */
+#define FS_MAX_D 1024
 
 /* One OT problem. Pointer fields are device pointers (host pointers for fs_solve_host). */
 typedef struct {
@@ -270,7 +272,8 @@ FS_API fs_status fs_transport_apply(const fs_problem* p, const float* f, const f
 
 /*
  * Hessian-vector product of the loss L(x) = OT_eps at the plan of (F(g), g) (exact at a
- * converged g), for one vector v_i per point x_i (v and out: n x d, row-major, device):
+ * converged g), for one vector v_i per point x_i (v and out: n x d, row-major, device);
+ * d <= 64 (FS_ERR_UNSUPPORTED_D above: its difference pass has no K-chunked form):
  *   (H v)_i = 2 a_i v_i + (2/eps) sum_j P_ij (x_i - y_j)(df_i + dg_j - 2 (x_i - y_j).v_i),
  * where (df, dg) solves [diag(P1) P; P^T diag(P^T 1)] (df, dg) = (r, s) with
  * r_i = sum_j P_ij 2 (x_i - y_j).v_i, s_j = sum_i P_ij 2 (x_i - y_j).v_i: the derivative of

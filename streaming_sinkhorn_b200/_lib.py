@@ -10,7 +10,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfs.so")
 
-FS_MAX_D = 64
+FS_MAX_D = 1024
 
 STATUS = {
     0: "FS_OK", 1: "FS_ERR_NULL", 2: "FS_ERR_SHAPE", 3: "FS_ERR_EPS", 4: "FS_ERR_ITERS",

@@ -12,6 +12,7 @@
 #include "fs_screen.cuh"
 #include "fs_transport.cuh"
 #include "fs_tc.cuh"
+#include "fs_tc_wide.cuh"
 
 namespace fs {
 namespace {
@@ -264,9 +265,14 @@ int64_t queue_partial_floats(const QPlan& q, int D, bool grad) {
   return q.on ? q.units_max * q.RB * (2 + (grad ? D : 0)) : 0;
 }
 
-// Points wider than 16 coordinates take the tensor-core pass for potential and marginal
-// passes (the gradient pass stays on the FMA path); its padded width is 32, 48 or 64.
-int tc_dim(int d) { return d <= 16 ? 0 : (d <= 32 ? 32 : (d <= 48 ? 48 : 64)); }
+// Points wider than 16 coordinates take the tensor-core passes; the padded width is 32, 48
+// or 64, and above 64 a multiple of 64 (the K-chunks of the wide passes).
+int tc_dim(int d) {
+  if (d <= 16) return 0;
+  if (d <= 64) return d <= 32 ? 32 : (d <= 48 ? 48 : 64);
+  return static_cast<int>(round_up(d, kTcChunk));
+}
+inline bool tc_wide(int Dtc) { return Dtc > 64; }
 int64_t tc_pad(int64_t count) { return round_up(count, kTcRows); }
 
 struct TcPlan {
@@ -351,6 +357,8 @@ struct Layout {
   // payload image; the HVP's difference pass: the rows' vector image, per-row (qs, x'.v),
   // the keys' padded dg
   size_t off_tc_lse, off_tc_mass, off_tc_pay, off_tc_vimg, off_tc_vrow, off_tc_dg;
+  // wide layouts (d > 64): per-coordinate sums of both clouds and the centre
+  size_t off_tc_sums, off_tc_ctr;
   // spatial order and screening (FMA path): permutations, sort keys, per-tile boxes and bias
   // maxima, and the LSE2 of every row in its last pass
   bool sorted;
@@ -410,7 +418,7 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0, bool co
   if (L.Dtc) {
     // potential passes: (max, sum) per split and row; apply passes: (sum, NC channels and,
     // for the difference pass, a second sum)
-    const int64_t nc = std::max<int64_t>(L.Dtc, kPayChannels);
+    const int64_t nc = tc_wide(L.Dtc) ? kPayChannels : std::max<int64_t>(L.Dtc, kPayChannels);
     for (const TcPlan& tp : {make_tc_plan(n, m, L.Dtc, sms), make_tc_plan(m, n, L.Dtc, sms)})
       if (tp.n_splits > 1) pf = std::max<int64_t>(pf, (2 + nc) * tp.n_splits * tp.rows_pad);
   }
@@ -442,14 +450,23 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0, bool co
     o = align_up(o + static_cast<size_t>(L.tx) * sizeof(float));
     L.off_hy_y = o;
     o = align_up(o + static_cast<size_t>(L.ty) * sizeof(float));
+    if (tc_wide(L.Dtc)) {
+      L.off_tc_sums = o;
+      o = align_up(o + static_cast<size_t>(2 * L.Dtc) * sizeof(double));
+      L.off_tc_ctr = o;
+      o = align_up(o + static_cast<size_t>(L.Dtc) * sizeof(double));
+    }
     const int64_t tmax = std::max(L.tx, L.ty);
     L.off_tc_lse = o;
     o = align_up(o + static_cast<size_t>(2 * tmax) * sizeof(float));
     L.off_tc_mass = o;
     o = align_up(o + static_cast<size_t>(2 * tmax) * sizeof(float));
-    if (acc_ch > 0) {
+    if (acc_ch > 0 || tc_wide(L.Dtc)) {
+      // the payload image: transport products, and the gradient of wide points (P y)
       L.off_tc_pay = o;
       o = align_up(o + static_cast<size_t>(tmax) * 2 * kPayChannels * 2);
+    }
+    if (acc_ch > 0) {
       L.off_tc_vimg = o;
       o = align_up(o + static_cast<size_t>(L.tx) * 2 * L.Dtc * 2);
       L.off_tc_vrow = o;
@@ -718,6 +735,7 @@ struct TcKernel {
 // allocation).
 int occupancy_tc(int Dtc) {
   int n = 1;
+  if (tc_wide(Dtc)) return 1;  // one 194 KB CTA per SM
   switch (Dtc) {
     case 32: n = TcKernel<32>::occupancy(); break;
     case 48: n = TcKernel<48>::occupancy(); break;
@@ -726,7 +744,24 @@ int occupancy_tc(int Dtc) {
   return std::max(1, std::min(n, static_cast<int>(512u / kTcTmemCols)));
 }
 
+void launch_tc_wide(const PassParams& P, const TcParams& T, const TcPlan& pl, cudaStream_t st) {
+  static bool done = false;  // idempotent, so a race between threads is harmless
+  if (!done) {
+    CK(cudaFuncSetAttribute(lse_pass_tcw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            static_cast<int>(TcWideShape::SMEM)));
+    done = true;
+  }
+  dim3 grid(static_cast<unsigned>(pl.row_blocks), static_cast<unsigned>(pl.n_splits));
+  lse_pass_tcw_kernel<<<grid, kTcThreads, TcWideShape::SMEM, st>>>(P, T);
+  CK(cudaGetLastError());
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
 void launch_tc(int Dtc, const PassParams& P, const TcParams& T, const TcPlan& pl, cudaStream_t st) {
+  if (tc_wide(Dtc)) {
+    launch_tc_wide(P, T, pl, st);
+    return;
+  }
   switch (Dtc) {
     case 32: TcKernel<32>::launch(P, T, pl, st); break;
     case 48: TcKernel<48>::launch(P, T, pl, st); break;
@@ -761,6 +796,25 @@ struct TcApplyKernel {
 
 void launch_apply_tc(int Dtc, int mode, const PassParams& P, const TcParams& T, const TcApply& A,
                      const TcPlan& pl, cudaStream_t st) {
+  if (tc_wide(Dtc)) {  // transport products only (the gradient runs as one)
+    static bool done = false;
+    if (!done) {
+      CK(cudaFuncSetAttribute(lse_apply_tcw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(TcWideShape::APPLY_SMEM)));
+      done = true;
+    }
+    dim3 grid(static_cast<unsigned>(pl.row_blocks), static_cast<unsigned>(pl.n_splits));
+    lse_apply_tcw_kernel<<<grid, kTcThreads, TcWideShape::APPLY_SMEM, st>>>(P, T, A);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (pl.n_splits > 1) {
+      tc_apply_combine_kernel<kPayChannels, kApplyPay>
+          <<<static_cast<unsigned>(ceil_div(P.n_rows, 256)), 256, 0, st>>>(P, A);
+      CK(cudaGetLastError());
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+    }
+    return;
+  }
   if (mode == kApplyGrad) {
     switch (Dtc) {
       case 32: TcApplyKernel<32, 32, kApplyGrad>::launch(P, T, A, pl, st); break;
@@ -936,6 +990,9 @@ struct Ctx {
   unsigned char* tc_vimg;       // difference pass: the rows' vector image
   float *tc_vrow, *tc_dg;       // difference pass: per-row (qs, x'.v); the keys' padded dg
   double tc_rkey;               // a bound on |y'_j| and |x'_i| (centred points)
+  double* tc_sums;              // wide layouts: coordinate sums of x then y (2 Dtc doubles)
+  double* tc_ctr_dev;           // wide layouts: the centre (Dtc doubles)
+  std::vector<double> tc_ctr_host;
   bool tc_reuse;                // apply passes keep the offsets of their first pre-pass
   bool tc_valid[2];             // ... per direction (rows x, rows y)
   float c2;       // 2 kappa / s^2
@@ -996,9 +1053,13 @@ void carve(Ctx& c, void* ws) {
     c.img_x = c.ws + c.L.off_img_x;
     c.img_y = c.ws + c.L.off_img_y;
     c.tc_lse = reinterpret_cast<float*>(c.ws + c.L.off_tc_lse);
+    if (c.L.off_tc_sums) {
+      c.tc_sums = reinterpret_cast<double*>(c.ws + c.L.off_tc_sums);
+      c.tc_ctr_dev = reinterpret_cast<double*>(c.ws + c.L.off_tc_ctr);
+    }
     c.tc_mass = reinterpret_cast<float*>(c.ws + c.L.off_tc_mass);
-    if (c.L.off_tc_pay) {
-      c.tc_pay = c.ws + c.L.off_tc_pay;
+    if (c.L.off_tc_pay) c.tc_pay = c.ws + c.L.off_tc_pay;
+    if (c.L.off_tc_vimg) {
       c.tc_vimg = c.ws + c.L.off_tc_vimg;
       c.tc_vrow = reinterpret_cast<float*>(c.ws + c.L.off_tc_vrow);
       c.tc_dg = reinterpret_cast<float*>(c.ws + c.L.off_tc_dg);
@@ -1072,13 +1133,17 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
     CK(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
+  const bool wide = c.use_tc && tc_wide(c.L.Dtc);
+  double* sum_x = wide ? c.tc_sums : c.scal + kSumX;
+  double* sum_y = wide ? c.tc_sums + c.L.Dtc : c.scal + kSumY;
+  if (wide) CK(cudaMemsetAsync(c.tc_sums, 0, 2 * c.L.Dtc * sizeof(double), c.st));
   if (c.use_tc) {
     unsigned* mx = reinterpret_cast<unsigned*>(c.scal + kMaxAbs);
     dim3 gx(reduce_blocks(p->n, c.sms), p->d), gy(reduce_blocks(p->m, c.sms), p->d);
-    coord_stats_kernel<<<gx, 256, 0, c.st>>>(p->x, p->n, p->d, c.scal + kSumX, mx);
+    coord_stats_kernel<<<gx, 256, 0, c.st>>>(p->x, p->n, p->d, sum_x, mx);
     CK(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    coord_stats_kernel<<<gy, 256, 0, c.st>>>(p->y, p->m, p->d, c.scal + kSumY, mx);
+    coord_stats_kernel<<<gy, 256, 0, c.st>>>(p->y, p->m, p->d, sum_y, mx);
     CK(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
@@ -1110,8 +1175,12 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
   }
   double host[kBox + 3];  // through the bounding box (6 ints at kBox)
   unsigned long long memo[kSortMemoWords];
+  std::vector<double> wide_sums(wide ? 2 * c.L.Dtc : 0);
   CK(cudaMemcpyAsync(host, c.scal, sizeof(host), cudaMemcpyDeviceToHost, c.st));
   CK(cudaMemcpyAsync(memo, c.scal + kSortMemo, sizeof(memo), cudaMemcpyDeviceToHost, c.st));
+  if (wide)
+    CK(cudaMemcpyAsync(wide_sums.data(), c.tc_sums, wide_sums.size() * sizeof(double),
+                       cudaMemcpyDeviceToHost, c.st));
   CK(cudaStreamSynchronize(c.st));
   unsigned flags;
   memcpy(&flags, &host[kFlags], sizeof(unsigned));
@@ -1176,9 +1245,16 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
     // two that puts the largest centred coordinate near 2^14, well inside fp16 range.
     TcCenter ctr{};
     double cmax = 0.0;
+    if (wide) c.tc_ctr_host.assign(c.L.Dtc, 0.0);
     for (int k = 0; k < p->d; ++k) {
-      ctr.c[k] = (host[kSumX + k] + host[kSumY + k]) / static_cast<double>(p->n + p->m);
-      cmax = std::max(cmax, std::fabs(ctr.c[k]));
+      const double sx = wide ? wide_sums[k] : host[kSumX + k];
+      const double sy = wide ? wide_sums[c.L.Dtc + k] : host[kSumY + k];
+      const double ck = (sx + sy) / static_cast<double>(p->n + p->m);
+      if (wide)
+        c.tc_ctr_host[k] = ck;
+      else
+        ctr.c[k] = ck;
+      cmax = std::max(cmax, std::fabs(ck));
     }
     unsigned bits;
     memcpy(&bits, &host[kMaxAbs], sizeof(unsigned));
@@ -1191,7 +1267,18 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
     c.tc_scale = static_cast<float>(scale);
     c.tc_rkey = std::sqrt(static_cast<double>(p->d)) * bound;
     const float sc = static_cast<float>(scale);
-    switch (c.L.Dtc) {
+    if (wide) {
+      CK(cudaMemcpyAsync(c.tc_ctr_dev, c.tc_ctr_host.data(), c.L.Dtc * sizeof(double),
+                         cudaMemcpyHostToDevice, c.st));
+      const int kc = c.L.Dtc / kTcChunk;
+      build_wide_image_kernel<<<static_cast<unsigned>(ceil_div(c.L.tx, 256)), 256, 0, c.st>>>(
+          p->x, p->n, p->d, kc, c.tc_ctr_dev, sc, c.img_x, c.nrm_x, c.L.tx);
+      CK(cudaGetLastError());
+      build_wide_image_kernel<<<static_cast<unsigned>(ceil_div(c.L.ty, 256)), 256, 0, c.st>>>(
+          p->y, p->m, p->d, kc, c.tc_ctr_dev, sc, c.img_y, c.nrm_y, c.L.ty);
+      CK(cudaGetLastError());
+      g_launches.fetch_add(2, std::memory_order_relaxed);
+    } else switch (c.L.Dtc) {
       case 32:
         launch_image<32>(p->x, p->n, p->d, ctr, sc, c.img_x, c.nrm_x, c.L.tx, c.st);
         launch_image<32>(p->y, p->m, p->d, ctr, sc, c.img_y, c.nrm_y, c.L.ty, c.st);
@@ -1286,6 +1373,7 @@ void run_pass_tc(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_
   T.key_tiles = pl.key_tiles;
   T.tiles_per_split = pl.tiles_per_split;
   T.c2 = c.c2;
+  T.kc = c.L.Dtc / kTcChunk;
   const double pairs = static_cast<double>(n_rows) * static_cast<double>(n_keys);
   int ti = c.timer->begin();
   launch_tc(c.L.Dtc, P, T, pl, c.st);
@@ -1310,6 +1398,18 @@ void run_pass_tc(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_
 void run_apply_tc(Ctx& c, bool rows_x, int mode, const float* pot_in, const float* pay, int k,
                   int pay_stride, float* out, int out_stride, const float* row_v = nullptr) {
   const fs_problem* p = c.p;
+  if (mode == kApplyGrad && tc_wide(c.L.Dtc)) {
+    // Wide points: P y as a transport product at the plan of (F(g), g) (row masses w), in
+    // the gradient's buffer, then grad = 2 (w x - P y) in place.
+    const int64_t n_rows = rows_x ? p->n : p->m;
+    run_apply_tc(c, rows_x, kApplyPay, nullptr, rows_x ? p->y : p->x, p->d, p->d, out, out_stride);
+    grad_from_py_kernel<<<static_cast<unsigned>(ceil_div(n_rows * p->d, 256)), 256, 0, c.st>>>(
+        rows_x ? p->x : p->y, rows_x ? p->a : p->b, static_cast<float>(1.0 / n_rows), out, n_rows,
+        p->d, out);
+    CK(cudaGetLastError());
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return;
+  }
   const int64_t n_rows = rows_x ? p->n : p->m, n_keys = rows_x ? p->m : p->n;
   const int tk = mode == kApplyGrad ? kTGrad : kTMarg;
   const int64_t half = std::max(c.L.tx, c.L.ty);
@@ -1347,6 +1447,7 @@ void run_apply_tc(Ctx& c, bool rows_x, int mode, const float* pot_in, const floa
   T.key_tiles = pl.key_tiles;
   T.tiles_per_split = pl.tiles_per_split;
   T.c2 = c.c2;
+  T.kc = c.L.Dtc / kTcChunk;
   TcApply A{};
   A.row_lse = lse;
   A.row_mass = pot_in ? mass : nullptr;
@@ -1879,6 +1980,7 @@ fs_status hvp_impl(const fs_problem* p, const float* g, const float* v, float* o
   Ctx c{};
   fs_status s = begin(c, p, ws, ws_bytes, stream, kTransportChannels);
   if (s != FS_OK) return s;
+  if (p->d > 64) return FS_ERR_UNSUPPORTED_D;  // no wide form of the difference pass
   if (p->cost != FS_COST_SQEUCLIDEAN) return FS_ERR_OPTION;
   if (!g || !v || !out) return FS_ERR_NULL;
   if (!aligned4(g) || !aligned4(v) || !aligned4(out)) return FS_ERR_ALIGNMENT;

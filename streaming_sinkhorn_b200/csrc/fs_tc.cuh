@@ -53,6 +53,9 @@ constexpr int kTcThreads = (kTcEpiWarps + 2) * 32;  // + a producer warp and an 
 static_assert(kTcGC % 32 == 0, "whole 32-column TMEM loads per group");
 constexpr uint32_t kTcTmemCols = 256;  // potential pass: two accumulators of kTcCols columns
 constexpr uint32_t kTcApplyTmemCols = 512;  // apply pass: two score accumulators + the result
+// Weights p <= 1 of the apply passes are stored as fp16(2^15 p): the largest lands below
+// fp16's maximum and weights down to 2^-39 keep their leading bits.
+constexpr float kPScale = 32768.0f;
 constexpr uint32_t kCoreLBO = 16u * 128u;  // next K-block of a core-matrix tile
 constexpr uint32_t kCoreSBO = 128u;        // next 8-point group
 // Dynamic shared memory a tensor-core pass may take (the opt-in limit is 227 KB; the
@@ -123,15 +126,18 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
 // The score tile of one 128-row block against one 128-key tile: three MMAs per 16-wide
 // K-step (hi.hi, lo.hi, hi.lo) into the accumulator at tmem_d. a0 and b0 are the
 // shared-memory addresses of the row and key images ([hi | lo], K-major).
+// With accumulate set, the first MMA adds to the accumulator too (a later K-chunk of one
+// score tile).
 template <int D>
 __device__ __forceinline__ void tc_issue_scores(uint32_t tmem_d, uint32_t a0, uint32_t b0,
-                                                uint32_t idesc) {
+                                                uint32_t idesc, bool accumulate = false) {
   using S = TcShape<D>;
 #pragma unroll
   for (int s = 0; s < S::KSTEPS; ++s) {
     const uint32_t o = static_cast<uint32_t>(s) * 2u * kCoreLBO;
     tc_mma_f16(tmem_d, tc_smem_desc(a0 + o, kCoreLBO, kCoreSBO),
-               tc_smem_desc(b0 + o, kCoreLBO, kCoreSBO), idesc, s > 0 ? 1u : 0u);
+               tc_smem_desc(b0 + o, kCoreLBO, kCoreSBO), idesc,
+               (s > 0 || accumulate) ? 1u : 0u);
     tc_mma_f16(tmem_d, tc_smem_desc(a0 + S::LO_OFF + o, kCoreLBO, kCoreSBO),
                tc_smem_desc(b0 + o, kCoreLBO, kCoreSBO), idesc, 1u);
     tc_mma_f16(tmem_d, tc_smem_desc(a0 + o, kCoreLBO, kCoreSBO),
@@ -179,6 +185,7 @@ struct TcParams {
   int64_t key_tiles;             // tiles of 128 keys
   int64_t tiles_per_split;
   float c2;                      // 2 kappa / s^2: scale of the MMA result
+  int32_t kc;                    // wide images (d > 64): 64-coordinate chunks per point
 };
 
 // Waits for phase `parity` of `bar`, giving up after kWaitLimitNs or as soon as another
@@ -203,6 +210,137 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// ---- epilogue pieces shared by the tensor-core kernels ------------------------------------
+
+// Online max/sum of one row (its column group) over the score tiles: running offset m
+// (log2 units, -inf until a real column sets it), base (m, or 0 before), mo = kappa |x|^2 + m
+// subtracted from each score, and the running sums L (two lanes).
+struct TcRowLse {
+  float m, base, mo, knrm;
+  u64 L;
+};
+
+__device__ __forceinline__ TcRowLse tc_row_lse_init(float knrm) {
+  TcRowLse s;
+  s.m = -INFINITY;
+  s.base = 0.0f;
+  s.mo = knrm;
+  s.knrm = knrm;
+  s.L = pk(0.0f, 0.0f);
+  return s;
+}
+
+// Folds one tile into the row state: v holds the group's kTcGC raw scores (the MMA result),
+// hy the group's key biases (shared memory, 16-byte aligned), c2 the score scale.
+__device__ __forceinline__ void tc_lse_tile(TcRowLse& s, const float* v, const float* hy,
+                                            u64 c2) {
+  constexpr int GP = kTcGC / 2;  // column pairs of a group
+  const ulonglong2* hv = reinterpret_cast<const ulonglong2*>(hy);
+  u64 tv[GP];
+  const u64 nmo = pk(-s.mo, -s.mo);
+#pragma unroll
+  for (int j = 0; j < GP; j += 2) {
+    const ulonglong2 h = hv[j / 2];  // four biases in one 16-byte (broadcast) load
+    tv[j] = add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), h.x), nmo);
+    tv[j + 1] = add2(fma2(c2, pk(v[2 * j + 2], v[2 * j + 3]), h.y), nmo);
+  }
+  float a0, a1;
+  upk(tv[0], a0, a1);
+  float mx = fmaxf(a0, a1);
+#pragma unroll
+  for (int j = 1; j < GP; ++j) {
+    upk(tv[j], a0, a1);
+    mx = max3(mx, a0, a1);
+  }
+  const float mx_abs = mx + s.base;
+  if (mx_abs > s.m + kLazyThr && mx > kEmptyCut) {
+    const float sc = ex2(s.m - mx_abs);
+    s.L = mul2(s.L, pk(sc, sc));
+    const u64 sh = pk(-mx, -mx);
+#pragma unroll
+    for (int j = 0; j < GP; ++j) tv[j] = add2(tv[j], sh);
+    s.m = mx_abs;
+    s.base = mx_abs;
+    s.mo = s.knrm + s.m;
+  }
+#pragma unroll
+  for (int j = 0; j < GP; ++j) {
+    float t0, t1;
+    upk(tv[j], t0, t1);
+    s.L = add2(s.L, pk(ex2(t0), ex2(t1)));
+  }
+}
+
+// Merges the column groups' states of every row and completes the row: the pass kind's
+// finish (split mode: the row's partial). Called by every thread of the CTA once all roles
+// are done; `merge` is shared scratch of kTcGroups x kTcRows entries.
+template <int D>
+__device__ __forceinline__ void tc_lse_finish(const PassParams& P, float2 (*merge)[kTcRows],
+                                              const TcRowLse& s, bool epi, int grp, int r,
+                                              int64_t i, int split) {
+  float l0, l1;
+  upk(s.L, l0, l1);
+  if (epi) merge[grp][r] = make_float2(s.m, l0 + l1);
+  __syncthreads();
+  double dev = 0.0, mass = 0.0;
+  if (epi && grp == 0 && i < P.n_rows) {
+    float mm = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < kTcGroups; ++q) mm = fmaxf(mm, merge[q][r].x);
+    float l = 0.0f;
+#pragma unroll
+    for (int q = 0; q < kTcGroups; ++q) {
+      const float2 o = merge[q][r];
+      if (o.x != -INFINITY) l += o.y * ex2(o.x - mm);
+    }
+    if (P.n_splits == 1) {
+      const double lse2 = static_cast<double>(mm) + log2(static_cast<double>(l));
+      if (P.kind == kPot) {
+        finish_pot<D>(P, i, lse2);
+      } else if (P.kind == kLse) {
+        P.lse_out[i] = static_cast<float>(lse2);
+      } else {
+        finish_marg(P, i, lse2, dev, mass);
+      }
+    } else {
+      const int64_t o2 = static_cast<int64_t>(split) * P.rows_pad + i;
+      P.part_m[o2] = mm;
+      P.part_l[o2] = l;
+    }
+  }
+  if (P.n_splits == 1 && P.kind == kMarg) block_reduce_marg(dev, dev, mass, P.acc);
+}
+
+// The weights of one tile for the apply passes: q = 2^15 2^(score - offset) rounded to fp16,
+// as packed pairs h2; L sums the rounded values.
+__device__ __forceinline__ void tc_weights_tile(const float* v, const float* hy, u64 c2, u64 noff,
+                                                u64& L, uint32_t* h2) {
+  constexpr int GP = kTcGC / 2;
+#pragma unroll
+  for (int j = 0; j < GP; ++j) {
+    float t0, t1;
+    const ulonglong2 h4 = reinterpret_cast<const ulonglong2*>(hy)[j / 2];
+    upk(add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), (j & 1) ? h4.y : h4.x), noff), t0, t1);
+    const __half2 h = __floats2half2_rn(ex2(t0) * kPScale, ex2(t1) * kPScale);
+    const float2 back = __half22float2(h);
+    L = add2(L, pk(back.x, back.y));
+    h2[j] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+}
+
+// Stores this thread's kTcGC weights (row r, column group grp) into a K-major weight tile:
+// core(row group, key block) at (kb * 16 + r / 8) * 128 + (r % 8) * 16.
+__device__ __forceinline__ void tc_store_weights(unsigned char* tile, int r, int grp,
+                                                 const uint32_t* h2) {
+  unsigned char* pt = tile + (r >> 3) * 128 + (r & 7) * 16;
+#pragma unroll
+  for (int c = 0; c < kTcGC / 8; ++c) {
+    const int kb = grp * (kTcGC / 8) + c;
+    *reinterpret_cast<uint4*>(pt + kb * 16 * 128) =
+        make_uint4(h2[4 * c], h2[4 * c + 1], h2[4 * c + 2], h2[4 * c + 3]);
+  }
 }
 
 template <int D>
@@ -255,11 +393,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  float m = -INFINITY;  // epilogue row state (origin-free running offset) ...
-  u64 L = pk(0.0f, 0.0f);
   const int quarter = warp & 3, grp = warp >> 2;
   const int r = quarter * 32 + lane;
   const int64_t i = row0 + r;
+  TcRowLse rs = tc_row_lse_init((i < P.n_rows) ? P.kappa_f * T.row_nrm[i] : 0.0f);
 
   if (warp == kTcEpiWarps) {
     // ---- producer: the row block once, then key tiles through the stage ring ----------
@@ -312,9 +449,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
     }
   } else {
     // ---- epilogue warps: online max/sum of one row over one column group of every tile --
-    constexpr int GP = kTcGC / 2;  // column pairs of a group
-    const float knrm = (i < P.n_rows) ? P.kappa_f * T.row_nrm[i] : 0.0f;
-    float base = 0.0f, mo = knrm;
     const u64 c2 = pk(T.c2, T.c2);
     for (int u = 0; u < n_tiles; ++u) {
       const int b = u & 1, st = u % kTcStages;
@@ -330,42 +464,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_free_bar[b]);
-      const ulonglong2* hv = reinterpret_cast<const ulonglong2*>(hy + grp * kTcGC);
-      u64 tv[GP];
-      const u64 nmo = pk(-mo, -mo);
-#pragma unroll
-      for (int j = 0; j < GP; j += 2) {
-        const ulonglong2 h = hv[j / 2];  // four biases in one 16-byte (broadcast) load
-        tv[j] = add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), h.x), nmo);
-        tv[j + 1] = add2(fma2(c2, pk(v[2 * j + 2], v[2 * j + 3]), h.y), nmo);
-      }
+      tc_lse_tile(rs, v, hy + grp * kTcGC, c2);
+      // the stage is released once its biases have been read
       __syncwarp();
       if (lane == 0) mbar_arrive(&free_bar[st]);
-      float a0, a1;
-      upk(tv[0], a0, a1);
-      float mx = fmaxf(a0, a1);
-#pragma unroll
-      for (int j = 1; j < GP; ++j) {
-        upk(tv[j], a0, a1);
-        mx = max3(mx, a0, a1);
-      }
-      const float mx_abs = mx + base;
-      if (mx_abs > m + kLazyThr && mx > kEmptyCut) {
-        const float sc = ex2(m - mx_abs);
-        L = mul2(L, pk(sc, sc));
-        const u64 sh = pk(-mx, -mx);
-#pragma unroll
-        for (int j = 0; j < GP; ++j) tv[j] = add2(tv[j], sh);
-        m = mx_abs;
-        base = mx_abs;
-        mo = knrm + m;
-      }
-#pragma unroll
-      for (int j = 0; j < GP; ++j) {
-        float t0, t1;
-        upk(tv[j], t0, t1);
-        L = add2(L, pk(ex2(t0), ex2(t1)));
-      }
     }
   }
 
@@ -375,38 +477,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
   if (abort_sh) {
     if (tid == 0) atomicOr(P.err, kErrTimeout);
   } else {
-    // Merge the column groups of each row, then finish the row.
-    float l0, l1;
-    upk(L, l0, l1);
-    if (warp < kTcEpiWarps) merge[grp][r] = make_float2(m, l0 + l1);
-    __syncthreads();
-    double dev = 0.0, mass = 0.0;
-    if (warp < kTcEpiWarps && grp == 0 && i < P.n_rows) {
-      float mm = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < kTcGroups; ++q) mm = fmaxf(mm, merge[q][r].x);
-      float l = 0.0f;
-#pragma unroll
-      for (int q = 0; q < kTcGroups; ++q) {
-        const float2 o = merge[q][r];
-        if (o.x != -INFINITY) l += o.y * ex2(o.x - mm);
-      }
-      if (P.n_splits == 1) {
-        const double lse2 = static_cast<double>(mm) + log2(static_cast<double>(l));
-        if (P.kind == kPot) {
-          finish_pot<D>(P, i, lse2);
-        } else if (P.kind == kLse) {
-          P.lse_out[i] = static_cast<float>(lse2);
-        } else {
-          finish_marg(P, i, lse2, dev, mass);
-        }
-      } else {
-        const int64_t o2 = static_cast<int64_t>(split) * P.rows_pad + i;
-        P.part_m[o2] = mm;
-        P.part_l[o2] = l;
-      }
-    }
-    if (P.n_splits == 1 && P.kind == kMarg) block_reduce_marg(dev, dev, mass, P.acc);
+    tc_lse_finish<D>(P, merge, rs, warp < kTcEpiWarps, grp, r, i, split);
   }
   tc_fence_before();
   __syncthreads();
@@ -424,9 +495,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) lse_pass_tc_kernel(const PassPa
 //               W = V Y^T on the tensor cores; out = mass_i sum_j q_ij (y_j - x_i) / sum_j p_ij
 //               (the difference pass of the Hessian-vector product).
 enum TcApplyMode : int { kApplyGrad = 0, kApplyPay = 1, kApplyDiff = 2 };
-// Weights p <= 1 are stored as fp16(2^15 p): the largest lands below fp16's maximum and
-// weights down to 2^-39 keep their leading bits.
-constexpr float kPScale = 32768.0f;
 constexpr int kPayChannels = 16;  // payload channels of one transport apply pass
 
 struct TcApply {
@@ -691,16 +759,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_free_bar[b]);
-#pragma unroll
-        for (int j = 0; j < GP; ++j) {
-          float t0, t1;
-          const ulonglong2 h4 = reinterpret_cast<const ulonglong2*>(hv)[j / 2];
-          upk(add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), (j & 1) ? h4.y : h4.x), noff), t0, t1);
-          const __half2 h = __floats2half2_rn(ex2(t0) * kPScale, ex2(t1) * kPScale);
-          const float2 back = __half22float2(h);
-          L = add2(L, pk(back.x, back.y));
-          h2[j] = *reinterpret_cast<const uint32_t*>(&h);
-        }
+        tc_weights_tile(v, reinterpret_cast<const float*>(hv), c2, noff, L, h2);
       } else {
         const u64* dv = reinterpret_cast<const u64*>(sStage + st * Sh::STAGE_BYTES + Sh::DG_OFF) +
                         grp * GP;
@@ -739,14 +798,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&free_bar[st]);  // its hy has been read
       if (u >= 2 && !tc_wait(&p_free[pb], static_cast<uint32_t>((u - 2) >> 1) & 1u, abort)) break;
-      // K-major weight tile: core(row group, key block) at (kb * 16 + r / 8) * 128 + (r % 8) * 16
-      unsigned char* pt = sP + pb * Sh::P_BYTES + (r >> 3) * 128 + (r & 7) * 16;
-#pragma unroll
-      for (int c = 0; c < kTcGC / 8; ++c) {
-        const int kb = grp * (kTcGC / 8) + c;
-        *reinterpret_cast<uint4*>(pt + kb * 16 * 128) =
-            make_uint4(h2[4 * c], h2[4 * c + 1], h2[4 * c + 2], h2[4 * c + 3]);
-      }
+      tc_store_weights(sP + pb * Sh::P_BYTES, r, grp, h2);
       fence_proxy_async_smem();  // the generic-proxy writes, before the MMA reads them
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[pb]);

@@ -54,7 +54,7 @@ def test_workspace_bytes():
     assert big > small
     # packed keys alone: 2 clouds x (2^19 pairs x 8 floats x 4 B) = 32 MiB for d = 3
     assert big >= 2 * (1 << 19) * 8 * 4
-    for bad in (prob(n=0), prob(m=0), prob(d=0), prob(d=65)):
+    for bad in (prob(n=0), prob(m=0), prob(d=0), prob(d=1025)):
         assert lib.fs_workspace_bytes(ctypes.byref(bad)) == 0
     assert lib.fs_workspace_bytes(None) == 0
 
@@ -64,7 +64,7 @@ def test_workspace_bytes():
     (prob(n=0), "FS_ERR_SHAPE"),
     (prob(m=-3), "FS_ERR_SHAPE"),
     (prob(d=0), "FS_ERR_SHAPE"),
-    (prob(d=65), "FS_ERR_UNSUPPORTED_D"),
+    (prob(d=1025), "FS_ERR_UNSUPPORTED_D"),
     (prob(eps=0.0), "FS_ERR_EPS"),
     (prob(eps=-1.0), "FS_ERR_EPS"),
     (prob(eps=float("nan")), "FS_ERR_EPS"),
@@ -189,7 +189,7 @@ def test_transport_and_hvp_argument_errors():
     need = lib.fs_transport_workspace_bytes(p)
     assert need > base and need % 256 == 0
     assert lib.fs_transport_workspace_bytes(ctypes.byref(prob(d=17))) > 0  # tensor-core path
-    assert lib.fs_transport_workspace_bytes(ctypes.byref(prob(d=65))) == 0
+    assert lib.fs_transport_workspace_bytes(ctypes.byref(prob(d=1025))) == 0
     assert lib.fs_transport_workspace_bytes(None) == 0
     st = lambda c: _lib.STATUS[c]  # noqa: E731
     ta = lambda *a: st(lib.fs_transport_apply(*a))  # noqa: E731
@@ -198,7 +198,7 @@ def test_transport_and_hvp_argument_errors():
     assert ta(p, None, FAKE, 0, 3, FAKE, FAKE, FAKE, need, None) == "FS_ERR_NULL"
     assert ta(p, FAKE, FAKE, 0, 3, FAKE + 2, FAKE, FAKE, need, None) == "FS_ERR_ALIGNMENT"
     assert ta(p, FAKE, FAKE, 0, 3, FAKE, FAKE, FAKE, need - 256, None) == "FS_ERR_WORKSPACE"
-    too_wide = ctypes.byref(prob(d=65))
+    too_wide = ctypes.byref(prob(d=1025))
     assert ta(too_wide, FAKE, FAKE, 0, 3, FAKE, FAKE, FAKE, BIG, None) == "FS_ERR_UNSUPPORTED_D"
     hv = lambda *a: st(lib.fs_hvp(*a))  # noqa: E731
     bad_iter = _lib.fs_hvp_options(0, 1e-6)
@@ -207,6 +207,9 @@ def test_transport_and_hvp_argument_errors():
     assert hv(p, FAKE, FAKE, FAKE, ctypes.byref(bad_tol), None, FAKE, need, None) == "FS_ERR_OPTION"
     assert hv(p, FAKE, None, FAKE, None, None, FAKE, need, None) == "FS_ERR_NULL"
     assert hv(too_wide, FAKE, FAKE, FAKE, None, None, FAKE, BIG, None) == "FS_ERR_UNSUPPORTED_D"
+    # the HVP's difference pass has no wide form: d > 64 is refused before any device work
+    hvp_wide = ctypes.byref(prob(d=65))
+    assert hv(hvp_wide, FAKE, FAKE, FAKE, None, None, FAKE, BIG, None) == "FS_ERR_UNSUPPORTED_D"
 
 
 def test_divergence_argument_errors():
@@ -214,7 +217,7 @@ def test_divergence_argument_errors():
     p = ctypes.byref(prob())
     need = lib.fs_divergence_workspace_bytes(p)
     assert need > lib.fs_workspace_bytes(p)
-    assert lib.fs_divergence_workspace_bytes(ctypes.byref(prob(d=65))) == 0
+    assert lib.fs_divergence_workspace_bytes(ctypes.byref(prob(d=1025))) == 0
     st = lambda c: _lib.STATUS[c]  # noqa: E731
     o = _lib.fs_solve_options(5, 0, 0.5, 0, 100, 5, 1e-6, None)
     assert st(lib.fs_divergence(p, None, FAKE, None, None, FAKE, need, None)) == "FS_ERR_NULL"

@@ -28,6 +28,10 @@ SHAPES = [  # (n, m, d, zero_frac, mass, eps)
     (100, 120, 17, 0.0, 1.0, 2.0),
     (96, 160, 32, 0.0, 1.0, 4.0),
     (130, 70, 64, 0.1, 1.0, 8.0),
+    (96, 120, 96, 0.0, 1.0, 12.0),     # wide points: 64-coordinate K-chunks from here on
+    (140, 130, 128, 0.1, 1.0, 16.0),
+    (130, 100, 512, 0.0, 1.0, 64.0),
+    (100, 90, 1024, 0.0, 1.0, 128.0),
 ]
 
 

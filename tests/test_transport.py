@@ -37,7 +37,8 @@ TRANSPORT_REL = {False: 1e-4, True: 1e-3}
 @pytest.mark.parametrize("k", [1, 3, 5, 16, 20])
 @pytest.mark.parametrize("transpose", [False, True])
 @pytest.mark.parametrize("shape", [(300, 257, 2, 0.1), (129, 700, 3, 0.05), (200, 150, 8, 0.5),
-                                   (90, 100, 16, 1.0), (200, 170, 32, 4.0), (130, 300, 64, 8.0)],
+                                   (90, 100, 16, 1.0), (200, 170, 32, 4.0), (130, 300, 64, 8.0),
+                                   (150, 140, 256, 32.0)],
                          ids=lambda s: "n{}-m{}-d{}".format(*s[:3]))
 def test_transport_apply_matches_dense_plan(shape, transpose, k):
     n, m, d, eps = shape
