@@ -13,6 +13,7 @@
 #include "fs_transport.cuh"
 #include "fs_tc.cuh"
 #include "fs_tc_wide.cuh"
+#include "fs_small.cuh"
 
 namespace fs {
 namespace {
@@ -1822,6 +1823,95 @@ cudaStream_t capture_stream() {
   return streams[dev];
 }
 
+// ---- small problems: the whole fixed-count solve in one cluster launch ----------------------
+
+template <int D>
+struct SmallKernel {
+  static constexpr auto fn = small_solve_kernel<D>;
+  // Launches one cluster of 16 CTAs (a non-portable size) if the device co-schedules it,
+  // else of 8, 4, 2 or 1; the size that worked is remembered.
+  static bool launch(const SmallParams& S, cudaStream_t st) {
+    static int best = 0;  // 0: not tried yet; -1: unavailable
+    static bool attr = false;
+    if (!attr) {
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
+          cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kSmallSmemBudget)) != cudaSuccess) {
+        cudaGetLastError();
+        best = -1;
+      }
+      attr = true;
+    }
+    if (best < 0) return false;
+    const size_t smem = small_smem_bytes(S.n, S.m, D);
+    for (int cs = best ? best : kSmallMaxCluster; cs >= 1; cs /= 2) {
+      cudaLaunchConfig_t cfg{};
+      cudaLaunchAttribute at[1];
+      cfg.gridDim = dim3(cs);
+      cfg.blockDim = dim3(kSmallThreads);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = st;
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = cs;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      if (cudaLaunchKernelEx(&cfg, fn, S) == cudaSuccess) {
+        best = cs;
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        return true;
+      }
+      cudaGetLastError();  // a cluster this device cannot co-schedule: try a smaller one
+    }
+    best = -1;
+    return false;
+  }
+};
+
+// Whether the fixed-count alternating solve of this problem runs in one cluster launch:
+// points of at most 16 coordinates, at most kSmallMaxPairs pairs, and both clouds staged in
+// shared memory.
+bool small_solve_fits(const fs_problem* p) {
+  if (p->d > 16 || p->n * p->m > kSmallMaxPairs) return false;
+  return small_smem_bytes(p->n, p->m, padded_dim(p->d)) <= kSmallSmemBudget;
+}
+
+// Runs the solve in one cluster launch; false (nothing launched) when the device cannot
+// co-schedule a cluster for it.
+bool run_small_solve(Ctx& c, int32_t n_iters, const float* g_init, float* f, float* g) {
+  const fs_problem* p = c.p;
+  SmallParams S{};
+  S.x = p->x;
+  S.y = p->y;
+  S.a = p->a;
+  S.b = p->b;
+  S.wa = static_cast<float>(1.0 / p->n);
+  S.wb = static_cast<float>(1.0 / p->m);
+  S.g_init = g_init;
+  S.f = f;
+  S.g = g;
+  S.n = static_cast<int32_t>(p->n);  // n * m <= kSmallMaxPairs
+  S.m = static_cast<int32_t>(p->m);
+  S.d = p->d;
+  S.n_iters = n_iters;
+  S.kappa = c.kappa;
+  S.inv_kappa = 1.0 / c.kappa;
+  const double pairs = 2.0 * static_cast<double>(p->n) * static_cast<double>(p->m) * n_iters;
+  const int ti = c.timer->begin();
+  bool ok = false;
+  switch (padded_dim(p->d)) {
+    case 1: ok = SmallKernel<1>::launch(S, c.st); break;
+    case 2: ok = SmallKernel<2>::launch(S, c.st); break;
+    case 3: ok = SmallKernel<3>::launch(S, c.st); break;
+    case 4: ok = SmallKernel<4>::launch(S, c.st); break;
+    case 8: ok = SmallKernel<8>::launch(S, c.st); break;
+    default: ok = SmallKernel<16>::launch(S, c.st); break;
+  }
+  c.timer->end(ti, kTLse, ok ? pairs : 0.0);
+  return ok;
+}
+
 // Runs body() `count` times on c.st as one CUDA graph: body's launches are captured once
 // (on the capture stream, so nothing runs during the capture) and the graph is replayed on
 // the caller's stream, one launch instead of ~15 per replay. body() must issue the same
@@ -1903,6 +1993,15 @@ fs_status solve_impl(const fs_problem* p, const fs_solve_options* opt, float* f,
     if (o.stop_mode == FS_STOP_POTENTIAL) {
       CK(cudaMemsetAsync(c.fprev, 0, fb, c.st));
       CK(cudaMemcpyAsync(c.gprev, g, gb, cudaMemcpyDeviceToDevice, c.st));
+    }
+    if (!sym && fixed && small_solve_fits(c.p) && run_small_solve(c, o.n_iters, o.g_init, f, g)) {
+      r = finish(c);
+      if (report) {
+        report->iters_run = o.n_iters;
+        report->converged = -1;
+        report->final_viol = NAN;
+      }
+      return r;
     }
     if (sym) set_bias(c, true, nullptr);  // x carries f = 0
     set_bias(c, false, o.g_init);

@@ -57,6 +57,34 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^t of both lanes on the FMA and integer pipes instead of the MUFU unit, for kernels whose
+// MUFU unit is the bound while issue slots are free. t is clamped to [-125, ...) (smaller
+// exponents give 2^-125 where ex2.approx.ftz gives 0: a term below 2^-125 of any sum that
+// matters), rounded to the nearest integer j by adding 1.5 * 2^23 (j then sits in the low
+// mantissa bits), and 2^(t - j), t - j in [-1/2, 1/2], is a degree-5 polynomial fitted to
+// 2^f on that interval by iteratively reweighted least squares at Chebyshev nodes (relative
+// error 2.1e-7 evaluated in fp32 by Horner's rule, checked over [-125, 9]); 2^j is added to
+// its exponent field.
+__device__ __forceinline__ u64 ex2_poly2(u64 t) {
+  float a, b;
+  upk(t, a, b);
+  t = pk(fmaxf(a, -125.0f), fmaxf(b, -125.0f));
+  const u64 magic = pk(12582912.0f, 12582912.0f);
+  const u64 tm = add2(t, magic);
+  const u64 f = sub2(t, sub2(tm, magic));
+  u64 p = pk(1.327645150013268e-3f, 1.327645150013268e-3f);
+  p = fma2(p, f, pk(9.675540961325169e-3f, 9.675540961325169e-3f));
+  p = fma2(p, f, pk(5.550713464617729e-2f, 5.550713464617729e-2f));
+  p = fma2(p, f, pk(2.4022120237350464e-1f, 2.4022120237350464e-1f));
+  p = fma2(p, f, pk(6.931469440460205e-1f, 6.931469440460205e-1f));
+  p = fma2(p, f, pk(1.0000001192092896f, 1.0000001192092896f));
+  float pa, pb, ma, mb;
+  upk(p, pa, pb);
+  upk(tm, ma, mb);
+  return pk(__uint_as_float(__float_as_uint(pa) + (__float_as_uint(ma) << 23)),
+            __uint_as_float(__float_as_uint(pb) + (__float_as_uint(mb) << 23)));
+}
+
 // Asks L2 to fetch the line holding p (no register result, nothing waits for it).
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));

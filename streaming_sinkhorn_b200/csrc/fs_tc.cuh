@@ -214,6 +214,10 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 
 // ---- epilogue pieces shared by the tensor-core kernels ------------------------------------
 
+// Column pairs per pair whose exponentials the LSE epilogue computes on the FMA pipe
+// (0: all on the MUFU unit).
+constexpr int kTcPolyEvery = 4;
+
 // Online max/sum of one row (its column group) over the score tiles: running offset m
 // (log2 units, -inf until a real column sets it), base (m, or 0 before), mo = kappa |x|^2 + m
 // subtracted from each score, and the running sums L (two lanes).
@@ -265,11 +269,17 @@ __device__ __forceinline__ void tc_lse_tile(TcRowLse& s, const float* v, const f
     s.base = mx_abs;
     s.mo = s.knrm + s.m;
   }
+  // One column pair in kTcPolyEvery takes its exponentials on the FMA pipe (ex2_poly2), the
+  // rest on the MUFU unit, which is this pass's bound while issue slots are free.
 #pragma unroll
   for (int j = 0; j < GP; ++j) {
-    float t0, t1;
-    upk(tv[j], t0, t1);
-    s.L = add2(s.L, pk(ex2(t0), ex2(t1)));
+    if (kTcPolyEvery > 0 && j % kTcPolyEvery == kTcPolyEvery - 1) {
+      s.L = add2(s.L, ex2_poly2(tv[j]));
+    } else {
+      float t0, t1;
+      upk(tv[j], t0, t1);
+      s.L = add2(s.L, pk(ex2(t0), ex2(t1)));
+    }
   }
 }
 

@@ -168,16 +168,23 @@ def test_repeated_calls_are_deterministic():
     assert bool((f1 == f2).all()) and bool((g1 == g2).all())
 
 
-def test_kernel_timing_counts_launches():
-    w = problem(1000, 800, 3, 0.0, 1.0, 0.05)
+@pytest.mark.parametrize("n,m,launches", [
+    (1000, 800, 1),    # at most 2^22 pairs: the whole solve in one cluster launch
+    (3000, 2500, 8),   # above: one streaming pass per half-iteration
+])
+def test_kernel_timing_counts_launches(n, m, launches):
+    w = problem(n, m, 3, 0.0, 1.0, 0.05)
     x, y, a, b = inputs(w)
     fs.timing_enable(True)
     fs.timing_reset()
     try:
-        fs.potentials(x, y, a, b, eps=w.eps, n_iters=4)
+        f, g = fs.potentials(x, y, a, b, eps=w.eps, n_iters=4)
         t = fs.timing_get()
     finally:
         fs.timing_enable(False)
-    assert t["lse_pass"]["launches"] == 8
-    assert t["lse_pass"]["pairs"] == pytest.approx(8 * 1000 * 800)
+    assert t["lse_pass"]["launches"] == launches
+    assert t["lse_pass"]["pairs"] == pytest.approx(8 * n * m)
     assert t["lse_pass"]["total_ms"] > 0
+    fr, gr = oracle.potentials(w.x, w.y, w.a, w.b, w.eps, 4)
+    assert_potential_close(f.cpu().numpy(), fr, "f")
+    assert_potential_close(g.cpu().numpy(), gr, "g")
