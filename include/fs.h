@@ -134,7 +134,7 @@ FS_API fs_status fs_workspace_invalidate(void* ws, size_t ws_bytes, fs_stream_t 
  *     g_j <- -eps * LSE_i[(f_i - C_ij)/eps + log a_i]       (one fused streaming pass)
  * Outputs: f (n floats) and g (m floats), the iterate after the last g-update.
  * g_init (m floats, device) may alias g.
- * From the second iteration on, the iterations of a fixed-count solve (this call, and
+ * From the third iteration on, the iterations of a fixed-count solve (this call, and
  * fs_solve with stop_mode FS_STOP_FIXED) are captured once as a CUDA graph and replayed on
  * `stream`. The capture runs on a non-blocking stream the library creates once per device
  * and keeps until exit (so `stream` may be the legacy default stream); a capture that

@@ -226,6 +226,10 @@ int64_t partial_floats(const Plan& p, int D, bool grad) {
   return static_cast<int64_t>(p.n_splits) * p.rows_pad * (2 + (grad ? D : 0));
 }
 
+// Screens per direction and call that evaluate the anchor tiles (and record each row's best
+// anchor key) before the later screens use the recorded keys.
+constexpr int kAnchorRecords = 2;
+
 // Queue mode: passes on sorted clouds whose key tiles are whole screening tiles run on the
 // unit plan of fs_screen.cuh. The kept-tile masks take one bit per (row block, key tile),
 // capped at kMaskCapWords words; larger problems run unscreened in split mode.
@@ -368,6 +372,8 @@ struct Layout {
       off_lse_x, off_lse_y;
   // queue mode: kept-tile masks, kept counts, unit starts and unit -> row block
   size_t off_kmask, off_kcount, off_ustart, off_unit_rb, off_unit_j;
+  // screening: each row's recorded anchor key (rows x, rows y)
+  size_t off_akey_x, off_akey_y;
   // general solve: deferred biases of x (symmetric schedule), potentials at the last check
   size_t off_defer, off_fprev, off_gprev;
   // transport products and the Hessian-vector product (layouts asked with acc_ch > 0):
@@ -505,6 +511,10 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0, bool co
     o = align_up(o + static_cast<size_t>(n) * sizeof(float));
     L.off_lse_y = o;
     o = align_up(o + static_cast<size_t>(m) * sizeof(float));
+    L.off_akey_x = o;
+    o = align_up(o + static_cast<size_t>(n) * sizeof(int));
+    L.off_akey_y = o;
+    o = align_up(o + static_cast<size_t>(m) * sizeof(int));
     L.off_kmask = o;
     o = align_up(o + static_cast<size_t>(mask_words) * sizeof(unsigned));
     L.off_kcount = o;
@@ -1005,6 +1015,8 @@ struct Ctx {
   float *box_x, *box_y, *hmax_x, *hmax_y, *lse_x, *lse_y;
   unsigned* kmask;
   int *kcount, *ustart, *unit_rb, *unit_j;
+  int *akey_x, *akey_y;  // screening: each row's recorded anchor key
+  int anchor_records[2];  // screens that recorded anchor keys in this call (rows x, rows y)
   float *defer, *fprev, *gprev;
   float* paykeys; // transport passes: keys with payload channels
   float* hvp;     // the HVP's vectors
@@ -1083,6 +1095,8 @@ void carve(Ctx& c, void* ws) {
     c.lse_x = reinterpret_cast<float*>(c.ws + c.L.off_lse_x);
     c.lse_y = reinterpret_cast<float*>(c.ws + c.L.off_lse_y);
     c.kmask = reinterpret_cast<unsigned*>(c.ws + c.L.off_kmask);
+    c.akey_x = reinterpret_cast<int*>(c.ws + c.L.off_akey_x);
+    c.akey_y = reinterpret_cast<int*>(c.ws + c.L.off_akey_y);
     c.kcount = reinterpret_cast<int*>(c.ws + c.L.off_kcount);
     c.ustart = reinterpret_cast<int*>(c.ws + c.L.off_ustart);
     c.unit_rb = reinterpret_cast<int*>(c.ws + c.L.off_unit_rb);
@@ -1637,6 +1651,12 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
     P.key_codes = rows_x ? c.code_y : c.code_x;
     P.row_codes = rows_x ? c.code_x : c.code_y;
     P.key_count = n_keys;
+    // The first kAnchorRecords screens of each direction in a call evaluate the anchor tiles
+    // and record each row's best key; later ones evaluate only that key.
+    const int dir = rows_x ? 0 : 1;
+    P.anchor_key = rows_x ? c.akey_x : c.akey_y;
+    P.anchor_mode = c.anchor_records[dir] >= kAnchorRecords ? 2 : 1;
+    if (P.anchor_mode == 1) ++c.anchor_records[dir];
     int ti = c.timer->begin();
     FS_DISPATCH_D(c.L.D, launch_screen_d, P, q.rb, c.kmask, c.kcount, c.st);
     plan_units_kernel<<<1, 1024, 0, c.st>>>(c.kcount, static_cast<int>(q.rb), q.budget, q.RB,
@@ -2018,12 +2038,15 @@ fs_status solve_impl(const fs_problem* p, const fs_solve_options* opt, float* f,
       run_pass(c, false, kPot, nullptr, g, nullptr, nullptr, nullptr, it > 1);  // g <- G(f)
       if (sym) apply_deferred_x(c);
     };
-    // A fixed count issues the same launches in every iteration from the second on (the
-    // screening decision is taken after the first): those run as replays of one CUDA graph,
-    // unless per-kernel timing is on (it records events around each launch).
-    const bool graphs = graphs_allowed && fixed && total >= 3 && !c.timer->on();
+    // A fixed count issues the same launches in every iteration from the third on (the
+    // screening decision is taken after the first, the screens record their anchor keys in
+    // the first two): those run as replays of one CUDA graph, unless per-kernel timing is on
+    // (it records events around each launch).
+    constexpr int32_t kGraphFrom = kAnchorRecords + 1;
+    const bool graphs = graphs_allowed && fixed && total > kGraphFrom && !c.timer->on();
     for (int32_t it = 1; it <= total; ++it) {
-      if (graphs && it == 2 && replay_as_graph(c, total - 1, [&] { iteration(2); })) {
+      if (graphs && it == kGraphFrom &&
+          replay_as_graph(c, total - kGraphFrom + 1, [&] { iteration(kGraphFrom); })) {
         iters = total;
         break;
       }

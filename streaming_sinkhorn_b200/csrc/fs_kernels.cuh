@@ -119,6 +119,11 @@ struct PassParams {
   const int* unit_rb;       // [unit] row block of each unit (launch order)
   const int* unit_j;        // [unit] its index among its row block's units
   const int* qscal;         // [0] tiles per unit C, [1] number of units U
+  // anchor record of the screen: per query row (sorted order) the key (sorted order) that
+  // gave its largest anchor exponent; anchor_mode 1 evaluates the anchor tiles and records
+  // it, 2 evaluates only the recorded key (0: anchor tiles, no record)
+  int* anchor_key;
+  int32_t anchor_mode;
   const unsigned* key_codes; // Morton codes of the key cloud in sorted order (key_count)
   const unsigned* row_codes; // Morton codes of the query cloud in sorted order
   int64_t key_count;         // real keys

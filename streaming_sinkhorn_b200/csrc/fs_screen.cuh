@@ -10,7 +10,10 @@
 //       reaches. The anchors are the key tiles that hold the row block's stretch of the
 //       Morton order both clouds share (the keys whose codes lie between the block's first
 //       and last row codes, and one key on either side): they hold most rows' nearest keys,
-//       so the bound is close to each row's true maximum, at most kMortonAnchors of them;
+//       so the bound is close to each row's true maximum, at most kMortonAnchors of them.
+//       A screen may record, per row, the key that gave this maximum; a later screen of the
+//       same call evaluates z_ij at that key alone (only the biases H changed in between,
+//       and any key's exponent is a value the row reaches);
 //   (b) history (potential passes after the first two): the largest term of a sum of m terms
 //       is at least the sum over m, and every bias moved by at least dmin since the row's
 //       previous pass, so max_j z_ij >= LSE2_prev_i + dmin - log2(m).
@@ -136,8 +139,13 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
     mk[r] = pk(q, q);
   }
   float zmax[R];
+  int zarg[R];  // anchor_mode 1: the key (sorted order) of each row's largest anchor exponent
 #pragma unroll
-  for (int r = 0; r < R; ++r) zmax[r] = -INFINITY;
+  for (int r = 0; r < R; ++r) {
+    zmax[r] = -INFINITY;
+    zarg[r] = -1;
+  }
+  const bool record = P.anchor_key && P.anchor_mode == 1;
   auto eval_tile = [&](int t) {
     __syncwarp();  // every lane is done with the previous tile
     const float* src = P.keys + static_cast<int64_t>(t) * TP * KP;
@@ -167,7 +175,19 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
         for (int k = 0; k < D; ++k) acc = fma2(xp[r][k], comp[k], acc);
         float z0, z1;
         upk(acc, z0, z1);
-        zmax[r] = max3(zmax[r], z0, z1);
+        if (record) {
+          const int key0 = t * kScreenTile + 2 * p;
+          if (z0 > zmax[r]) {
+            zmax[r] = z0;
+            zarg[r] = key0;
+          }
+          if (z1 > zmax[r]) {
+            zmax[r] = z1;
+            zarg[r] = key0 + 1;
+          }
+        } else {
+          zmax[r] = max3(zmax[r], z0, z1);
+        }
       }
     }
   };
@@ -177,7 +197,25 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
   // kMortonAnchors of them, spread over the stretch. Without codes no tile is evaluated,
   // every bound stays -inf and every tile is kept.
   int anchor = -1;
-  if (P.key_codes) {
+  if (P.anchor_key && P.anchor_mode == 2) {
+    // the recorded key of each row: its exponent now (direct difference)
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (!valid[r]) continue;
+      // a recorded key index; clamped so that even a stale one stays inside the keys
+      const int j = min(max(P.anchor_key[row0 + r * 32 + lane], 0),
+                        static_cast<int>(P.key_count) - 1);
+      float d2 = 0.0f;
+#pragma unroll
+      for (int k = 0; k < D; ++k) {
+        const float dk = x[r][k] - P.keys[key_slot<D>(j, k)];
+        d2 = fmaf(dk, dk, d2);
+      }
+      zmax[r] = P.keys[key_slot<D>(j, D)] - P.kappa_f * d2;
+    }
+    // the tile of the first row's key is always kept, so the block has work
+    anchor = min(max(P.anchor_key[row0], 0), static_cast<int>(P.key_count) - 1) / kScreenTile;
+  } else if (P.key_codes) {
     const int64_t nk = P.key_count;
     // first position in the sorted key codes whose code is >= target (warp-wide search)
     auto lower_bound = [&](uint64_t target) -> int64_t {
@@ -207,6 +245,11 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
       if (e == 0) anchor = t;
       eval_tile(t);
     }
+  }
+  if (record) {
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (valid[r] && zarg[r] >= 0) P.anchor_key[row0 + r * 32 + lane] = zarg[r];
   }
   const bool history = P.lse_prev && P.key_dmin;
   const float dmin = history ? ord_float(*P.key_dmin) : 0.0f;
@@ -242,14 +285,24 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
     const bool keep_s = sidx < S && (sidx == anchor / kSuper || sub_ub(sidx) >= thr);
     unsigned sbits = __ballot_sync(0xffffffffu, keep_s);
     unsigned word = 0u;
+    // Up to four kept super-tiles at a time: lane l loads tile l % 8 of the (l / 8)-th one
+    // (box and Hmax), so one round trip to L2 serves 32 tiles; the per-row tests below take
+    // them by shuffles.
     while (sbits) {
-      const int sl = __ffs(sbits) - 1;
-      sbits &= sbits - 1u;
-      const int tbase = (s0 + sl) * kSuper;
-      const int t = tbase + lane;
-      // lanes 0-7 load the run's tiles (box and Hmax) once; the per-row tests below take
-      // them by shuffles
-      const bool okl = lane < kSuper && t < T;
+      int sl[4];
+      int nsup = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        sl[q] = sbits ? __ffs(sbits) - 1 : -1;
+        if (sbits) {
+          sbits &= sbits - 1u;
+          ++nsup;
+        }
+      }
+      const int q = lane / kSuper;
+      const int myq_sl = q == 0 ? sl[0] : (q == 1 ? sl[1] : (q == 2 ? sl[2] : sl[3]));
+      const int t = myq_sl >= 0 ? (s0 + myq_sl) * kSuper + lane % kSuper : -1;
+      const bool okl = q < nsup && t >= 0 && t < T;
       float blo[D], bhi[D];
       float d2b = 0.0f;
 #pragma unroll
@@ -261,10 +314,13 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
       }
       const float thm = okl ? P.key_hmax[t] : -INFINITY;
       const bool keep_t = okl && (t == anchor || thm - P.kappa_f * d2b >= thr);
-      unsigned pat = __ballot_sync(0xffffffffu, keep_t) & 0xFFu;
-#pragma unroll
-      for (int tl = 0; tl < kSuper; ++tl) {
-        if (!((pat >> tl) & 1u) || tbase + tl == anchor) continue;
+      unsigned pat = __ballot_sync(0xffffffffu, keep_t);
+      unsigned test = pat;
+      while (test) {
+        const int tl = __ffs(test) - 1;
+        test &= test - 1u;
+        const int ttile = __shfl_sync(0xffffffffu, t, tl);
+        if (ttile == anchor) continue;
         u64 d2 = pk(0.0f, 0.0f);
 #pragma unroll
         for (int k = 0; k < D; ++k) {
@@ -282,7 +338,11 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
         const bool need = hm - P.kappa_f * e0 >= rthr[0] || hm - P.kappa_f * e1 >= rthr[1];
         if (!__any_sync(0xffffffffu, need)) pat &= ~(1u << tl);
       }
-      if (lane == sl / 4) word |= pat << ((sl % 4) * kSuper);
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        if (qq < nsup && lane == sl[qq] / 4)
+          word |= ((pat >> (qq * kSuper)) & 0xFFu) << ((sl[qq] % 4) * kSuper);
+      }
     }
     const int w = s0 / 4 + lane;
     if (lane < 8 && w < P.mask_words) {
