@@ -156,8 +156,12 @@ int num_sms_current() {
   return sms > 0 ? sms : 148;
 }
 
+// A stage of the copy ring: a key tile and, for D <= 3 (whose passes skip 16-point groups),
+// the tile's group records behind it.
 size_t pass_smem_bytes(int D, int tile_pairs, int stages = kStages, int np = 0) {
-  return static_cast<size_t>(stages) * tile_pairs * pair_floats(D, np) * 4;
+  const size_t stage = static_cast<size_t>(tile_pairs) * pair_floats(D, np) +
+                       (D <= 3 ? static_cast<size_t>(kTileGroupFloats) : 0u);
+  return static_cast<size_t>(stages) * stage * 4;
 }
 
 // Pass kernel selector: what the pass accumulates (PassMode) and, for transport products,
@@ -372,8 +376,9 @@ struct Layout {
       off_lse_x, off_lse_y;
   // queue mode: kept-tile masks, kept counts, unit starts and unit -> row block
   size_t off_kmask, off_kcount, off_ustart, off_unit_rb, off_unit_j;
-  // screening: each row's recorded anchor key (rows x, rows y)
-  size_t off_akey_x, off_akey_y;
+  // screening: each row's recorded anchor key (rows x, rows y); the 16-point group records of
+  // each cloud (D <= 3) and the rows' thresholds of the last screen
+  size_t off_akey_x, off_akey_y, off_gsum_x, off_gsum_y, off_rowthr;
   // general solve: deferred biases of x (symmetric schedule), potentials at the last check
   size_t off_defer, off_fprev, off_gprev;
   // transport products and the Hessian-vector product (layouts asked with acc_ch > 0):
@@ -511,6 +516,14 @@ Layout make_layout(int64_t n, int64_t m, int d, int sms, int acc_ch = 0, bool co
     o = align_up(o + static_cast<size_t>(n) * sizeof(float));
     L.off_lse_y = o;
     o = align_up(o + static_cast<size_t>(m) * sizeof(float));
+    if (L.D <= 3) {
+      L.off_gsum_x = o;
+      o = align_up(o + static_cast<size_t>(tiles_x) * kTileGroupFloats * sizeof(float));
+      L.off_gsum_y = o;
+      o = align_up(o + static_cast<size_t>(tiles_y) * kTileGroupFloats * sizeof(float));
+      L.off_rowthr = o;
+      o = align_up(o + static_cast<size_t>(std::max(n, m)) * sizeof(float));
+    }
     L.off_akey_x = o;
     o = align_up(o + static_cast<size_t>(n) * sizeof(int));
     L.off_akey_y = o;
@@ -923,10 +936,10 @@ void launch_bias_d(float* keys, int64_t count, const float* pot, const int* perm
 }
 
 template <int D>
-void launch_tile_box_d(const float* keys, int64_t count, int64_t tiles, float* box,
+void launch_tile_box_d(const float* keys, int64_t count, int64_t tiles, float* box, float* gsum,
                        cudaStream_t st) {
   // tile boxes, then super-tile boxes behind them (lower corners by min, upper by max)
-  tile_box_kernel<D><<<static_cast<unsigned>(tiles), 256, 0, st>>>(keys, count, box, tiles);
+  tile_box_kernel<D><<<static_cast<unsigned>(tiles), 256, 0, st>>>(keys, count, box, tiles, gsum);
   CK(cudaGetLastError());
   const int64_t supers = ceil_div(tiles, kSuper);
   super_reduce_kernel<<<static_cast<unsigned>(ceil_div(supers, 256)), 256, 0, st>>>(
@@ -936,9 +949,9 @@ void launch_tile_box_d(const float* keys, int64_t count, int64_t tiles, float* b
 }
 
 template <int D>
-void launch_tile_hmax_d(const float* keys, int64_t count, int64_t tiles, float* hmax,
+void launch_tile_hmax_d(const float* keys, int64_t count, int64_t tiles, float* hmax, float* gsum,
                         cudaStream_t st) {
-  tile_hmax_kernel<D><<<static_cast<unsigned>(tiles), 256, 0, st>>>(keys, count, hmax);
+  tile_hmax_kernel<D><<<static_cast<unsigned>(tiles), 256, 0, st>>>(keys, count, hmax, gsum);
   CK(cudaGetLastError());
   const int64_t supers = ceil_div(tiles, kSuper);
   super_reduce_kernel<<<static_cast<unsigned>(ceil_div(supers, 256)), 256, 0, st>>>(
@@ -1016,6 +1029,8 @@ struct Ctx {
   unsigned* kmask;
   int *kcount, *ustart, *unit_rb, *unit_j;
   int *akey_x, *akey_y;  // screening: each row's recorded anchor key
+  float *gsum_x, *gsum_y;  // 16-point group records (D <= 3), or NULL
+  float* rowthr;           // the rows' thresholds of the last screen (D <= 3), or NULL
   int anchor_records[2];  // screens that recorded anchor keys in this call (rows x, rows y)
   float *defer, *fprev, *gprev;
   float* paykeys; // transport passes: keys with payload channels
@@ -1096,6 +1111,11 @@ void carve(Ctx& c, void* ws) {
     c.lse_y = reinterpret_cast<float*>(c.ws + c.L.off_lse_y);
     c.kmask = reinterpret_cast<unsigned*>(c.ws + c.L.off_kmask);
     c.akey_x = reinterpret_cast<int*>(c.ws + c.L.off_akey_x);
+    if (c.L.off_gsum_x) {
+      c.gsum_x = reinterpret_cast<float*>(c.ws + c.L.off_gsum_x);
+      c.gsum_y = reinterpret_cast<float*>(c.ws + c.L.off_gsum_y);
+      c.rowthr = reinterpret_cast<float*>(c.ws + c.L.off_rowthr);
+    }
     c.akey_y = reinterpret_cast<int*>(c.ws + c.L.off_akey_y);
     c.kcount = reinterpret_cast<int*>(c.ws + c.L.off_kcount);
     c.ustart = reinterpret_cast<int*>(c.ws + c.L.off_ustart);
@@ -1252,8 +1272,8 @@ fs_status prepare(Ctx& c, const std::vector<std::pair<const float*, int64_t>>& p
   FS_DISPATCH_D(c.L.D, launch_pack_d, p->y, p->m, p->d, p->b, wu_y, c.perm_y, c.ky, c.lwy, c.L.py,
                 c.st);
   if (c.L.sorted) {
-    FS_DISPATCH_D(c.L.D, launch_tile_box_d, c.kx, p->n, c.L.px / kPairPad, c.box_x, c.st);
-    FS_DISPATCH_D(c.L.D, launch_tile_box_d, c.ky, p->m, c.L.py / kPairPad, c.box_y, c.st);
+    FS_DISPATCH_D(c.L.D, launch_tile_box_d, c.kx, p->n, c.L.px / kPairPad, c.box_x, c.gsum_x, c.st);
+    FS_DISPATCH_D(c.L.D, launch_tile_box_d, c.ky, p->m, c.L.py / kPairPad, c.box_y, c.gsum_y, c.st);
   }
   if (c.use_tc) {
     // Centre on the common mean (the cost is translation invariant) and scale by a power of
@@ -1343,7 +1363,8 @@ void set_bias(Ctx& c, bool cloud_x, const float* pot) {
   if (c.L.sorted) {
     // largest bias per tile, for the screening of the passes that take this cloud as keys
     FS_DISPATCH_D(c.L.D, launch_tile_hmax_d, cloud_x ? c.kx : c.ky, cloud_x ? c.p->n : c.p->m,
-                  (cloud_x ? c.L.px : c.L.py) / kPairPad, cloud_x ? c.hmax_x : c.hmax_y, c.st);
+                  (cloud_x ? c.L.px : c.L.py) / kPairPad, cloud_x ? c.hmax_x : c.hmax_y,
+                  cloud_x ? c.gsum_x : c.gsum_y, c.st);
   }
 }
 
@@ -1655,6 +1676,10 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
     // and record each row's best key; later ones evaluate only that key.
     const int dir = rows_x ? 0 : 1;
     P.anchor_key = rows_x ? c.akey_x : c.akey_y;
+    // the screen leaves each row's threshold; the pass then skips the 16-point groups of
+    // kept tiles that no row of its block needs
+    P.row_thr = c.rowthr;
+    P.gsum = rows_x ? c.gsum_y : c.gsum_x;
     P.anchor_mode = c.anchor_records[dir] >= kAnchorRecords ? 2 : 1;
     if (P.anchor_mode == 1) ++c.anchor_records[dir];
     int ti = c.timer->begin();
@@ -1687,7 +1712,8 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
   if (c.L.sorted && kind == kPot && !(rows_x && c.defer_x)) {
     // largest bias per tile of the cloud just updated: the next pass screens against it
     FS_DISPATCH_D(c.L.D, launch_tile_hmax_d, rows_x ? c.kx : c.ky, n_rows,
-                  (rows_x ? c.L.px : c.L.py) / kPairPad, rows_x ? c.hmax_x : c.hmax_y, c.st);
+                  (rows_x ? c.L.px : c.L.py) / kPairPad, rows_x ? c.hmax_x : c.hmax_y,
+                  rows_x ? c.gsum_x : c.gsum_y, c.st);
   }
 }
 
@@ -1763,7 +1789,7 @@ void apply_deferred_x(Ctx& c) {
   int* dmin = reinterpret_cast<int*>(c.scal + kDmin);  // slot 0: x
   CK(cudaMemsetAsync(dmin, 0x7F, sizeof(int), c.st));
   FS_DISPATCH_D(c.L.D, launch_apply_bias_d, c.kx, c.defer, n, dmin, c.st);
-  FS_DISPATCH_D(c.L.D, launch_tile_hmax_d, c.kx, n, c.L.px / kPairPad, c.hmax_x, c.st);
+  FS_DISPATCH_D(c.L.D, launch_tile_hmax_d, c.kx, n, c.L.px / kPairPad, c.hmax_x, c.gsum_x, c.st);
 }
 
 // max(|P1 - a|_inf, |P^T 1 - b|_inf) at (f, g): two marginal passes, one read-back.

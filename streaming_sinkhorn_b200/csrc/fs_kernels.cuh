@@ -124,6 +124,10 @@ struct PassParams {
   // it, 2 evaluates only the recorded key (0: anchor tiles, no record)
   int* anchor_key;
   int32_t anchor_mode;
+  // group skip (screened passes, D <= 3): the key cloud's 16-point group records and each
+  // query row's threshold (written by the screen, sorted order), or NULL
+  const float* gsum;
+  float* row_thr;
   const unsigned* key_codes; // Morton codes of the key cloud in sorted order (key_count)
   const unsigned* row_codes; // Morton codes of the query cloud in sorted order
   int64_t key_count;         // real keys
@@ -360,8 +364,14 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
 
   float* stages = reinterpret_cast<float*>(smem_raw);
   const int tid = threadIdx.x;
-  const uint32_t stage_floats = static_cast<uint32_t>(P.tile_pairs) * KP;
-  const uint32_t stage_bytes = stage_floats * 4u;
+  // A stage holds a key tile and, for the group skip (one-warp CTAs, D <= 3), the tile's
+  // 16-point group records behind it.
+  constexpr bool GT = NT == 32 && D <= 3;
+  static_assert(!GT || G * 2 == kGroupKeys, "a key-pair group of the pass is a record's group");
+  static_assert(!GT || R <= 2, "a lane tests its rows in the two halves of a packed register");
+  const uint32_t tile_floats = static_cast<uint32_t>(P.tile_pairs) * KP;
+  const uint32_t stage_floats = tile_floats + (GT ? kTileGroupFloats : 0u);
+  const uint32_t tile_bytes = tile_floats * 4u;
 
   // The work of this CTA: rows row0 .. row0 + RB and a list of key tiles. Split mode: the
   // tiles of column split blockIdx.y, in order. Queue mode (screened, sorted clouds): unit
@@ -446,14 +456,23 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     walk_bits = mrow[walk_w];
     for (int s = 0; s < s_walk[1]; ++s) walk_bits &= walk_bits - 1u;
   }
-  auto tile_src = [&](int e) -> const float* {
+  // Group skip: queue mode with the screen's row thresholds and the key cloud's records.
+  const bool gtest = GT && queue && P.row_thr && P.gsum;
+  const uint32_t copy_bytes = tile_bytes + (gtest ? kTileGroupFloats * 4u : 0u);
+  // Issues the copies of work item e (thread 0): the key tile, and its group records.
+  auto issue_tile = [&](int s, int e) {
     int tt = e;
     if (queue) {
       while (walk_bits == 0u && walk_w + 1 < P.mask_words) walk_bits = mrow[++walk_w];
       tt = walk_bits ? walk_w * 32 + __ffs(walk_bits) - 1 : 0;
       walk_bits &= walk_bits - 1u;
     }
-    return key_src + static_cast<int64_t>(tt) * stage_floats;
+    float* dst = stages + s * stage_floats;
+    mbar_expect_tx(&bars[s], copy_bytes);
+    bulk_g2s(dst, key_src + static_cast<int64_t>(tt) * tile_floats, tile_bytes, &bars[s]);
+    if (gtest)
+      bulk_g2s(dst + tile_floats, P.gsum + static_cast<int64_t>(tt) * kTileGroupFloats,
+               kTileGroupFloats * 4u, &bars[s]);
   };
 
   // Row state: coordinates duplicated into both lanes of a packed register; the running
@@ -478,6 +497,9 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
   u64 V[R][MODE == kModeDiff ? D : 1];  // kModeDiff: the row's vector v_i, in both lanes
   float q[R];        // CEN: kappa |x'|^2
   u64 cpk[D];        // CEN: the centre, in both lanes
+  u64 xb[GT ? D : 1];  // group skip: x' of the thread's two rows (one per lane)
+  u64 thr2 = pk(INFINITY, INFINITY);  // group skip: their thresholds
+  int groups_done = 0;  // group skip: 16-point groups this warp evaluated
   const u64 nkappa = pk(-P.kappa_f, -P.kappa_f);
   const u64 nhalf_ik = pk(-0.5f * P.inv_kappa_f, -0.5f * P.inv_kappa_f);  // X -> -x'
 #pragma unroll
@@ -525,6 +547,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       cpk[k] = pk(c, c);
     }
     const float k2 = 2.0f * P.kappa_f;
+    float xsv[R][D];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       float s2 = 0.0f;
@@ -534,11 +557,23 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
         upk(X[r][k], c0, c1);
         upk(cpk[k], cc, cd);
         const float xs = c0 - cc;
+        xsv[r][k] = xs;
         s2 = fmaf(xs, xs, s2);
         X[r][k] = pk(k2 * xs, k2 * xs);
       }
       q[r] = P.kappa_f * s2;
       mk[r] = pk(-q[r], -q[r]);
+    }
+    if constexpr (GT) {
+#pragma unroll
+      for (int k = 0; k < D; ++k) xb[k] = pk(xsv[0][k], xsv[R > 1 ? 1 : 0][k]);
+      if (gtest) {
+        float t0 = INFINITY, t1 = INFINITY;  // rows past the end need nothing
+        const int64_t i0 = row0 + tid, i1 = row0 + (R > 1 ? NT : 0) + tid;
+        if (i0 < P.n_rows) t0 = P.row_thr[i0];
+        if (R > 1 && i1 < P.n_rows) t1 = P.row_thr[i1];
+        thr2 = pk(t0, t1);
+      }
     }
   }
   // CEN: rewrite a tile in place to (y', H'); pairs are spread over the warp's lanes.
@@ -562,9 +597,37 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     }
   };
 
-  // Online max/sum of this thread's rows over one key tile in shared memory.
+  // Online max/sum of this thread's rows over one key tile in shared memory. With the group
+  // skip, a group of G key pairs is left out when for every row of the warp its upper bound
+  // Hmax_g - kappa dist(x_i, box_g)^2 is below the row's threshold (the screen's lower bound
+  // on the row's largest exponent minus the margin): each of its terms is then below
+  // 2^-margin of the row's largest, as for the tiles the screen drops, and all keys left out
+  // either way number at most M, so the omitted part of the row's sum stays below 2^-24 of it.
   auto process_tile = [&](const float* tile) {
     for (int pg = 0; pg < P.tile_pairs; pg += G) {
+      if constexpr (GT) {
+        if (gtest) {
+          const float* rec = tile + tile_floats + (pg / G) * kGroupRecFloats;
+          u64 d2 = pk(0.0f, 0.0f);
+#pragma unroll
+          for (int k = 0; k < D; ++k) {
+            float cc, cd, a0, a1, b0, b1;
+            upk(cpk[k], cc, cd);
+            const float lo = rec[k] - cc, hi = rec[3 + k] - cc;  // the box about the centre
+            upk(sub2(pk(lo, lo), xb[k]), a0, a1);
+            upk(sub2(xb[k], pk(hi, hi)), b0, b1);
+            const u64 gap = pk(max3(a0, b0, 0.0f), max3(a1, b1, 0.0f));
+            d2 = fma2(gap, gap, d2);
+          }
+          float e0, e1, h0, h1;
+          upk(d2, e0, e1);
+          upk(thr2, h0, h1);
+          const float hm = rec[6];
+          const bool need = hm - P.kappa_f * e0 >= h0 || hm - P.kappa_f * e1 >= h1;
+          if (!__any_sync(0xffffffffu, need)) continue;
+          ++groups_done;
+        }
+      }
       u64 tv[R][G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -657,10 +720,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     }  };
 
   if (tid == 0) {
-    for (int s = 0; s < kStages && s < n_work; ++s) {
-      mbar_expect_tx(&bars[s], stage_bytes);
-      bulk_g2s(stages + s * stage_floats, tile_src(s), stage_bytes, &bars[s]);
-    }
+    for (int s = 0; s < kStages && s < n_work; ++s) issue_tile(s, s);
   }
 
   // One CTA barrier per tile: after it every thread has finished the previous tile, so its
@@ -678,8 +738,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     if (tid == 0 && t >= 1 && t - 1 + kStages < n_work) {
       const int ps = (t - 1) % kStages;
       fence_proxy_async_smem();
-      mbar_expect_tx(&bars[ps], stage_bytes);
-      bulk_g2s(stages + ps * stage_floats, tile_src(t - 1 + kStages), stage_bytes, &bars[ps]);
+      issue_tile(ps, t - 1 + kStages);
     }
     if constexpr (CEN) centre_tile(stages + st * stage_floats);
     process_tile(stages + st * stage_floats);
@@ -687,7 +746,8 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     if constexpr (CEN) fence_proxy_async_smem();
   }
   if (queue && P.evaluated && tid == 0 && n_work > 0)
-    atomicAdd(P.evaluated, static_cast<unsigned long long>(n_work) * kScreenTile * RB);
+    atomicAdd(P.evaluated, gtest ? static_cast<unsigned long long>(groups_done) * kGroupKeys * RB
+                                 : static_cast<unsigned long long>(n_work) * kScreenTile * RB);
 
   if (aborted) {
     // Record the timeout, let this CTA's own copies still in flight land (bounded), leave.

@@ -268,6 +268,12 @@ __global__ void __launch_bounds__(32) screen_kernel(const PassParams P, unsigned
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mlb = fminf(mlb, __shfl_xor_sync(0xffffffffu, mlb, o));
   const float thr = mlb - P.skip_margin;
+  // each row's own threshold, for the pass's skip of 16-point groups inside kept tiles
+  if (P.row_thr) {
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (valid[r]) P.row_thr[row0 + r * 32 + lane] = rthr[r];
+  }
 
   // The mask, 32 super-tiles (8 mask words) per round; lane j < 8 assembles word j. A tile
   // is tested against the block's box and smallest bound, then each tile that passes row by

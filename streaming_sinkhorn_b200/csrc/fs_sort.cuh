@@ -153,13 +153,21 @@ __global__ void __launch_bounds__(256) perm_from_keys_kernel(const uint64_t* key
   codes[j] = static_cast<unsigned>(k >> 32);
 }
 
+// Group records of the screened passes (D <= 3): per 256-point tile, 16 groups of 16
+// consecutive points (8 key pairs, the pass's unit of work), each kGroupRecFloats floats
+// [lo_0 lo_1 lo_2 hi_0 hi_1 hi_2 Hmax pad], a tile's records contiguous (one bulk copy).
+constexpr int kGroupKeys = 16;
+constexpr int kGroupRecFloats = 8;
+constexpr int kTileGroupFloats = (256 / kGroupKeys) * kGroupRecFloats;  // 128 floats, 512 B
+
 // Bounding box (all D coordinates) of each 256-point tile of a packed cloud, stored by
 // component: box[k * T + t] = lo_k, box[(D + k) * T + t] = hi_k of tile t (T tiles), so that
 // a warp scanning consecutive tiles reads each component in one coalesced request. Only
-// real points count.
+// real points count. With gsum (D <= 3) the boxes of the tile's 16-point groups go to their
+// group records as well.
 template <int D>
 __global__ void __launch_bounds__(256) tile_box_kernel(const float* keys, int64_t count, float* box,
-                                                       int64_t T) {
+                                                       int64_t T, float* gsum) {
   constexpr int KP = ((2 * (D + 1) + 3) / 4) * 4;
   const int64_t t = blockIdx.x;
   const int64_t j = t * 256 + threadIdx.x;
@@ -172,10 +180,17 @@ __global__ void __launch_bounds__(256) tile_box_kernel(const float* keys, int64_
       v = u = keys[(j >> 1) * KP + 2 * k + (j & 1)];
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
+    for (int o = 8; o > 0; o >>= 1) {
       v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
       u = fmaxf(u, __shfl_xor_sync(0xffffffffu, u, o));
     }
+    if (D <= 3 && gsum && (lane & 15) == 0) {
+      float* rec = gsum + (t * (256 / kGroupKeys) + threadIdx.x / kGroupKeys) * kGroupRecFloats;
+      rec[k] = v;
+      rec[3 + k] = u;
+    }
+    v = fminf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+    u = fmaxf(u, __shfl_xor_sync(0xffffffffu, u, 16));
     if (lane == 0) {
       red[0][k][w] = v;
       red[1][k][w] = u;
@@ -194,10 +209,11 @@ __global__ void __launch_bounds__(256) tile_box_kernel(const float* keys, int64_
   }
 }
 
-// Largest key bias H of each 256-point tile of a packed cloud (kLogZero if none is real).
+// Largest key bias H of each 256-point tile of a packed cloud (kLogZero if none is real);
+// with gsum (D <= 3) also of each 16-point group, into its group record.
 template <int D>
 __global__ void __launch_bounds__(256) tile_hmax_kernel(const float* keys, int64_t count,
-                                                        float* hmax) {
+                                                        float* hmax, float* gsum) {
   constexpr int KP = ((2 * (D + 1) + 3) / 4) * 4;
   const int64_t T = blockIdx.x;
   const int64_t j = T * 256 + threadIdx.x;
@@ -205,7 +221,10 @@ __global__ void __launch_bounds__(256) tile_hmax_kernel(const float* keys, int64
   float h = kLogZero;
   if (j < count) h = keys[(j >> 1) * KP + 2 * D + (j & 1)];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) h = fmaxf(h, __shfl_xor_sync(0xffffffffu, h, o));
+  for (int o = 8; o > 0; o >>= 1) h = fmaxf(h, __shfl_xor_sync(0xffffffffu, h, o));
+  if (D <= 3 && gsum && (threadIdx.x & 15) == 0)
+    gsum[(T * (256 / kGroupKeys) + threadIdx.x / kGroupKeys) * kGroupRecFloats + 6] = h;
+  h = fmaxf(h, __shfl_xor_sync(0xffffffffu, h, 16));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = h;
   __syncthreads();
   if (threadIdx.x == 0) {

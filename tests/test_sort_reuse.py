@@ -21,8 +21,12 @@ def run(x, y, a, b, w, ws):
     return (f.cpu().numpy(), g.cpu().numpy(), gx.cpu().numpy()), fs.launch_count() - before
 
 
-def fresh(w):
-    return torch.empty(fs.workspace_bytes(w.n, w.m, w.d), dtype=torch.uint8, device="cuda")
+def fresh(*ws):
+    # fs_workspace_bytes is not monotone in the problem size (the column splits, and so the
+    # partial buffers, grow as the row count shrinks): a workspace shared by several problems
+    # takes the largest of their sizes
+    need = max(fs.workspace_bytes(w.n, w.m, w.d) for w in ws)
+    return torch.empty(need, dtype=torch.uint8, device="cuda")
 
 
 def test_same_clouds_reuse_the_order():
@@ -63,7 +67,7 @@ def test_other_problem_in_between():
     problem then sorts again and gets the same results."""
     w1 = workloads.clustered_cube(n=20000, seed=43, n_iters=5, eps=1e-3)
     w2 = workloads.clustered_cube(n=12000, seed=44, n_iters=5, eps=1e-3)
-    ws = fresh(w1)
+    ws = fresh(w1, w2)
     p1 = inputs(w1)
     p2 = inputs(w2)
     first, _ = run(*p1, w1, ws)
