@@ -156,12 +156,12 @@ int num_sms_current() {
   return sms > 0 ? sms : 148;
 }
 
-// A stage of the copy ring: a key tile and, for D <= 3 (whose passes skip 16-point groups),
-// the tile's group records behind it.
-size_t pass_smem_bytes(int D, int tile_pairs, int stages = kStages, int np = 0) {
-  const size_t stage = static_cast<size_t>(tile_pairs) * pair_floats(D, np) +
-                       (D <= 3 ? static_cast<size_t>(kTileGroupFloats) : 0u);
-  return static_cast<size_t>(stages) * stage * 4;
+// The copy ring of key tiles and, for the screened passes of D <= 3 (which skip 16-point
+// groups), one slot of group records behind it.
+size_t pass_smem_bytes(int D, int tile_pairs, int stages = kStages, int np = 0,
+                       bool group_recs = false) {
+  const size_t ring = static_cast<size_t>(stages) * tile_pairs * pair_floats(D, np);
+  return (ring + (group_recs && D <= 3 ? static_cast<size_t>(kTileGroupFloats) : 0u)) * 4;
 }
 
 // Pass kernel selector: what the pass accumulates (PassMode) and, for transport products,
@@ -169,7 +169,8 @@ size_t pass_smem_bytes(int D, int tile_pairs, int stages = kStages, int np = 0) 
 enum PassSel : int { kSelLse = 0, kSelGrad = 1, kSelPay1 = 2, kSelPay4 = 3, kSelPay16 = 4,
                      kSelDiff = 5 };
 
-int occupancy_for(int D, bool grad, int variant, size_t smem);  // defined after the kernels
+// defined after the kernels; queue: the screened launches' kernel
+int occupancy_for(int D, bool grad, int variant, size_t smem, bool queue = false);
 
 Plan make_plan(int64_t n_rows, int64_t key_pairs, int D, bool grad, int sms) {
   const int64_t fill = static_cast<int64_t>(sms) * (D > 16 ? 4 : 16);
@@ -264,7 +265,8 @@ QPlan make_qplan(const Plan& pl, int64_t key_pairs, int D, bool grad, int sms, b
   if (!q.on) return q;
   const int64_t slots = static_cast<int64_t>(sms) *
                         occupancy_for(D, grad, kQueueVariant,
-                                      pass_smem_bytes(D, kScreenTile / 2, kQueueStages));
+                                      pass_smem_bytes(D, kScreenTile / 2, kQueueStages, 0, true),
+                                      true);
   q.budget = std::max<int64_t>(1, std::min<int64_t>(kUnitWaves * slots, kUnitsPerBlock * q.rb));
   q.units_max = q.budget + q.rb;
   return q;
@@ -573,25 +575,35 @@ inline bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr)
 
 template <int D, int R, int NT, int MODE, int NP, int G, int MINB, int ST = kStages>
 struct PassKernel {
-  static constexpr auto fn = lse_pass_kernel<D, R, NT, G, MODE, NP, MINB, ST>;
+  // unscreened launches; screened ones (fnq) skip 16-point groups when D <= 3
+  static constexpr bool kGroups = D <= 3 && NT == 32;
+  static constexpr auto fn = lse_pass_kernel<D, R, NT, G, MODE, NP, MINB, ST, false>;
+  static constexpr auto fnq = lse_pass_kernel<D, R, NT, G, MODE, NP, MINB, ST, kGroups>;
   static void set_smem_attr() {
     static bool done = false;  // idempotent, so a race between threads is harmless
     if (!done) {
       CK(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(pass_smem_bytes(D, 128, ST, NP))));
+      CK(cudaFuncSetAttribute(fnq, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(pass_smem_bytes(D, 128, ST, NP, kGroups))));
       done = true;
     }
   }
-  static void launch(const PassParams& P, const Plan& pl, cudaStream_t st) {
+  static void launch(const PassParams& P0, const Plan& pl, cudaStream_t st) {
     set_smem_attr();
+    PassParams P = P0;
+    P.group_recs = 0;  // unscreened: stages hold key tiles only
     dim3 grid(static_cast<unsigned>(pl.row_blocks), static_cast<unsigned>(pl.n_splits));
     fn<<<grid, NT, pass_smem_bytes(D, pl.tile_pairs, ST, NP), st>>>(P);
     CK(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
-  static void launch_queue(const PassParams& P, int64_t units, cudaStream_t st) {
+  static void launch_queue(const PassParams& P0, int64_t units, cudaStream_t st) {
     set_smem_attr();
-    fn<<<static_cast<unsigned>(units), NT, pass_smem_bytes(D, kScreenTile / 2, ST, NP), st>>>(P);
+    PassParams P = P0;
+    P.group_recs = kGroups && P.row_thr && P.gsum ? 1 : 0;
+    fnq<<<static_cast<unsigned>(units), NT,
+          pass_smem_bytes(D, kScreenTile / 2, ST, NP, P.group_recs != 0), st>>>(P);
     CK(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
@@ -604,10 +616,12 @@ struct PassKernel {
       g_launches.fetch_add(1, std::memory_order_relaxed);
     }
   }
-  static int occupancy(size_t smem) {
+  static int occupancy(size_t smem, bool queue) {
     int n = 0;
     set_smem_attr();
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, NT, smem) != cudaSuccess || n < 1) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, queue ? fnq : fn, NT, smem) !=
+            cudaSuccess ||
+        n < 1) {
       cudaGetLastError();
       n = MINB;
     }
@@ -665,9 +679,10 @@ struct ScreenOp {
 
 struct OccupancyOp {
   size_t smem;
+  bool queue;
   int result = 1;
   template <typename K>
-  void run() { result = K::occupancy(smem); }
+  void run() { result = K::occupancy(smem, queue); }
 };
 
 template <int D>
@@ -869,8 +884,8 @@ void launch_image(const float* pts, int64_t count, int d, const TcCenter& ctr, f
   g_launches.fetch_add(1, std::memory_order_relaxed);
 }
 
-int occupancy_for(int D, bool grad, int variant, size_t smem) {
-  OccupancyOp op{smem};
+int occupancy_for(int D, bool grad, int variant, size_t smem, bool queue) {
+  OccupancyOp op{smem, queue};
   try {
     FS_DISPATCH_D(D, occupancy_d, grad, variant, &op);
   } catch (const CudaFail&) {

@@ -128,6 +128,9 @@ struct PassParams {
   // query row's threshold (written by the screen, sorted order), or NULL
   const float* gsum;
   float* row_thr;
+  // 1: the launch sized each stage of the copy ring for a key tile and its group records
+  // (set by the host for the screened launches of D <= 3 kernels only)
+  int32_t group_recs;
   const unsigned* key_codes; // Morton codes of the key cloud in sorted order (key_count)
   const unsigned* row_codes; // Morton codes of the query cloud in sorted order
   int64_t key_count;         // real keys
@@ -349,7 +352,9 @@ __device__ __forceinline__ void load_pair(const float* tile, int p, u64 (&comp)[
   }
 }
 
-template <int D, int R, int NT, int G, int MODE, int NP, int MINB, int ST>
+// GS: the instance of the screened launches of D <= 3, with the group skip; the unscreened
+// launches use the one without it (fewer registers in the hot loop).
+template <int D, int R, int NT, int G, int MODE, int NP, int MINB, int ST, bool GS>
 __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) {
   constexpr int kStages = ST;  // depth of the copy ring
   constexpr bool GRAD = MODE == kModeGrad;
@@ -360,18 +365,25 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
   constexpr int RB = R * NT;  // rows of one row block
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ uint64_t bars[kStages];
+  __shared__ uint64_t rbar;  // group skip: the record slot's copies
   __shared__ int s_walk[2];
 
   float* stages = reinterpret_cast<float*>(smem_raw);
   const int tid = threadIdx.x;
-  // A stage holds a key tile and, for the group skip (one-warp CTAs, D <= 3), the tile's
-  // 16-point group records behind it.
-  constexpr bool GT = NT == 32 && D <= 3;
+  // The copy ring holds kStages key tiles; with the group skip (one-warp CTAs, D <= 3,
+  // screened launches) one slot behind it holds the 16-point group records of the tile
+  // being processed. They are read only by the group tests at the start of the tile, after
+  // which the next tile's records are copied in, so one slot suffices and keeps the CTA's
+  // shared memory at the ring's size plus 512 B.
+  constexpr bool GT = GS && NT == 32 && D <= 3;
   static_assert(!GT || G * 2 == kGroupKeys, "a key-pair group of the pass is a record's group");
   static_assert(!GT || R <= 2, "a lane tests its rows in the two halves of a packed register");
+  static_assert(!GT || ST == 2, "the records of tile t + 1 follow the copy of tile t + 1");
   const uint32_t tile_floats = static_cast<uint32_t>(P.tile_pairs) * KP;
-  const uint32_t stage_floats = tile_floats + (GT ? kTileGroupFloats : 0u);
+  const bool recs = GT && P.group_recs != 0;
+  const uint32_t stage_floats = tile_floats;
   const uint32_t tile_bytes = tile_floats * 4u;
+  float* rslot = stages + kStages * stage_floats;
 
   // The work of this CTA: rows row0 .. row0 + RB and a list of key tiles. Split mode: the
   // tiles of column split blockIdx.y, in order. Queue mode (screened, sorted clouds): unit
@@ -441,6 +453,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+    if (recs) mbar_init(&rbar, 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -457,9 +470,9 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     for (int s = 0; s < s_walk[1]; ++s) walk_bits &= walk_bits - 1u;
   }
   // Group skip: queue mode with the screen's row thresholds and the key cloud's records.
-  const bool gtest = GT && queue && P.row_thr && P.gsum;
-  const uint32_t copy_bytes = tile_bytes + (gtest ? kTileGroupFloats * 4u : 0u);
-  // Issues the copies of work item e (thread 0): the key tile, and its group records.
+  const bool gtest = recs && queue && P.row_thr && P.gsum;
+  int rtt0 = 0, rtt1 = 0;  // thread 0: the key tiles of the work items in flight, by parity
+  // Issues the copy of work item e's key tile (thread 0).
   auto issue_tile = [&](int s, int e) {
     int tt = e;
     if (queue) {
@@ -467,12 +480,21 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       tt = walk_bits ? walk_w * 32 + __ffs(walk_bits) - 1 : 0;
       walk_bits &= walk_bits - 1u;
     }
+    if (e & 1)
+      rtt1 = tt;
+    else
+      rtt0 = tt;
     float* dst = stages + s * stage_floats;
-    mbar_expect_tx(&bars[s], copy_bytes);
+    mbar_expect_tx(&bars[s], tile_bytes);
     bulk_g2s(dst, key_src + static_cast<int64_t>(tt) * tile_floats, tile_bytes, &bars[s]);
-    if (gtest)
-      bulk_g2s(dst + tile_floats, P.gsum + static_cast<int64_t>(tt) * kTileGroupFloats,
-               kTileGroupFloats * 4u, &bars[s]);
+  };
+  // Issues the copy of work item e's group records into the slot (thread 0; its key tile
+  // has been issued).
+  auto issue_recs = [&](int e) {
+    const int tt = (e & 1) ? rtt1 : rtt0;
+    mbar_expect_tx(&rbar, kTileGroupFloats * 4u);
+    bulk_g2s(rslot, P.gsum + static_cast<int64_t>(tt) * kTileGroupFloats, kTileGroupFloats * 4u,
+             &rbar);
   };
 
   // Row state: coordinates duplicated into both lanes of a packed register; the running
@@ -497,8 +519,11 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
   u64 V[R][MODE == kModeDiff ? D : 1];  // kModeDiff: the row's vector v_i, in both lanes
   float q[R];        // CEN: kappa |x'|^2
   u64 cpk[D];        // CEN: the centre, in both lanes
-  u64 xb[GT ? D : 1];  // group skip: x' of the thread's two rows (one per lane)
+  u64 xb[GT ? D : 1];  // group skip: x of the thread's two rows (one per lane)
   u64 thr2 = pk(INFINITY, INFINITY);  // group skip: their thresholds
+  // group skip: the warp's row box (lo, hi per coordinate) and its smallest threshold, in
+  // shared memory (they are read once per tile)
+  __shared__ float s_wbox[2 * 3 + 1];
   int groups_done = 0;  // group skip: 16-point groups this warp evaluated
   const u64 nkappa = pk(-P.kappa_f, -P.kappa_f);
   const u64 nhalf_ik = pk(-0.5f * P.inv_kappa_f, -0.5f * P.inv_kappa_f);  // X -> -x'
@@ -545,9 +570,23 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       }
       const float c = lo <= hi ? 0.5f * (lo + hi) : 0.0f;
       cpk[k] = pk(c, c);
+      if constexpr (GT) {
+        if (tid == 0) {
+          s_wbox[k] = lo;
+          s_wbox[3 + k] = hi;
+        }
+      }
+    }
+    if constexpr (GT) {
+#pragma unroll
+      for (int k = 0; k < D; ++k) {
+        float c0, c1, d0, d1;
+        upk(X[0][k], c0, c1);
+        upk(X[R > 1 ? 1 : 0][k], d0, d1);
+        xb[k] = pk(c0, d0);
+      }
     }
     const float k2 = 2.0f * P.kappa_f;
-    float xsv[R][D];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       float s2 = 0.0f;
@@ -557,7 +596,6 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
         upk(X[r][k], c0, c1);
         upk(cpk[k], cc, cd);
         const float xs = c0 - cc;
-        xsv[r][k] = xs;
         s2 = fmaf(xs, xs, s2);
         X[r][k] = pk(k2 * xs, k2 * xs);
       }
@@ -565,21 +603,26 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       mk[r] = pk(-q[r], -q[r]);
     }
     if constexpr (GT) {
-#pragma unroll
-      for (int k = 0; k < D; ++k) xb[k] = pk(xsv[0][k], xsv[R > 1 ? 1 : 0][k]);
       if (gtest) {
         float t0 = INFINITY, t1 = INFINITY;  // rows past the end need nothing
         const int64_t i0 = row0 + tid, i1 = row0 + (R > 1 ? NT : 0) + tid;
         if (i0 < P.n_rows) t0 = P.row_thr[i0];
         if (R > 1 && i1 < P.n_rows) t1 = P.row_thr[i1];
         thr2 = pk(t0, t1);
+        float wthr = fminf(t0, t1);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) wthr = fminf(wthr, __shfl_xor_sync(0xffffffffu, wthr, o));
+        if (tid == 0) s_wbox[6] = wthr;
+        __syncwarp();
       }
     }
   }
   // CEN: rewrite a tile in place to (y', H'); pairs are spread over the warp's lanes.
-  auto centre_tile = [&](float* tile) {
+  // With the group skip, a run of 32 pairs (four groups) none of which is kept is left as it is.
+  auto centre_tile = [&](float* tile, unsigned gm) {
     if constexpr (CEN) {
       for (int p = tid; p < P.tile_pairs; p += 32) {
+        if (((gm >> ((p - tid) / G)) & 0xFu) == 0u) continue;
         u64 comp[KP / 2];
         load_pair<KP>(tile, p, comp);
         u64 s2 = pk(0.0f, 0.0f);
@@ -597,37 +640,68 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
     }
   };
 
+  // Group skip: bit g of the result is set when some row of the warp may need group g of the
+  // tile (records in the slot, coordinates uncentred, as the screen tests them). Lane g < 16
+  // first tests group g against the warp's row box and smallest threshold: a group that
+  // fails fails every row's own test, which then runs, two groups at a time, on the others.
+  auto group_mask = [&]() -> unsigned {
+    unsigned gm = 0u;
+    if constexpr (GT) {
+      bool cand = false;
+      if (tid < kTileGroupFloats / kGroupRecFloats) {
+        const float4* r4 = reinterpret_cast<const float4*>(rslot + tid * kGroupRecFloats);
+        const float4 ra = r4[0], rb = r4[1];  // lo0 lo1 lo2 hi0 | hi1 hi2 Hmax -
+        const float glo[3] = {ra.x, ra.y, ra.z}, ghi[3] = {ra.w, rb.x, rb.y};
+        float d2 = 0.0f;
+#pragma unroll
+        for (int k = 0; k < D; ++k) {
+          const float gap = max3(glo[k] - s_wbox[3 + k], s_wbox[k] - ghi[k], 0.0f);
+          d2 = fmaf(gap, gap, d2);
+        }
+        cand = rb.z - P.kappa_f * d2 >= s_wbox[6];
+      }
+      unsigned cm = __ballot_sync(0xffffffffu, cand);
+      float h0, h1;
+      upk(thr2, h0, h1);
+      auto row_test = [&](int gi) -> bool {
+        const float4* r4 = reinterpret_cast<const float4*>(rslot + gi * kGroupRecFloats);
+        const float4 ra = r4[0], rb = r4[1];
+        const float lo[3] = {ra.x, ra.y, ra.z}, hi[3] = {ra.w, rb.x, rb.y};
+        u64 d2 = pk(0.0f, 0.0f);
+#pragma unroll
+        for (int k = 0; k < D; ++k) {
+          float a0, a1, b0, b1;
+          upk(sub2(pk(lo[k], lo[k]), xb[k]), a0, a1);
+          upk(sub2(xb[k], pk(hi[k], hi[k])), b0, b1);
+          const u64 gap = pk(max3(a0, b0, 0.0f), max3(a1, b1, 0.0f));
+          d2 = fma2(gap, gap, d2);
+        }
+        float e0, e1;
+        upk(d2, e0, e1);
+        return rb.z - P.kappa_f * e0 >= h0 || rb.z - P.kappa_f * e1 >= h1;
+      };
+      while (cm) {
+        const int g0 = __ffs(cm) - 1;
+        cm &= cm - 1u;
+        const int g1 = cm ? __ffs(cm) - 1 : g0;
+        cm &= cm - 1u;
+        const bool n0 = row_test(g0), n1 = row_test(g1);
+        if (__any_sync(0xffffffffu, n0)) gm |= 1u << g0;
+        if (__any_sync(0xffffffffu, n1)) gm |= 1u << g1;
+      }
+    }
+    return gm;
+  };
+
   // Online max/sum of this thread's rows over one key tile in shared memory. With the group
   // skip, a group of G key pairs is left out when for every row of the warp its upper bound
   // Hmax_g - kappa dist(x_i, box_g)^2 is below the row's threshold (the screen's lower bound
   // on the row's largest exponent minus the margin): each of its terms is then below
   // 2^-margin of the row's largest, as for the tiles the screen drops, and all keys left out
   // either way number at most M, so the omitted part of the row's sum stays below 2^-24 of it.
-  auto process_tile = [&](const float* tile) {
+  auto process_tile = [&](const float* tile, unsigned gm) {
     for (int pg = 0; pg < P.tile_pairs; pg += G) {
-      if constexpr (GT) {
-        if (gtest) {
-          const float* rec = tile + tile_floats + (pg / G) * kGroupRecFloats;
-          u64 d2 = pk(0.0f, 0.0f);
-#pragma unroll
-          for (int k = 0; k < D; ++k) {
-            float cc, cd, a0, a1, b0, b1;
-            upk(cpk[k], cc, cd);
-            const float lo = rec[k] - cc, hi = rec[3 + k] - cc;  // the box about the centre
-            upk(sub2(pk(lo, lo), xb[k]), a0, a1);
-            upk(sub2(xb[k], pk(hi, hi)), b0, b1);
-            const u64 gap = pk(max3(a0, b0, 0.0f), max3(a1, b1, 0.0f));
-            d2 = fma2(gap, gap, d2);
-          }
-          float e0, e1, h0, h1;
-          upk(d2, e0, e1);
-          upk(thr2, h0, h1);
-          const float hm = rec[6];
-          const bool need = hm - P.kappa_f * e0 >= h0 || hm - P.kappa_f * e1 >= h1;
-          if (!__any_sync(0xffffffffu, need)) continue;
-          ++groups_done;
-        }
-      }
+      if ((gm >> (pg / G) & 1u) == 0u) continue;
       u64 tv[R][G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -721,6 +795,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
 
   if (tid == 0) {
     for (int s = 0; s < kStages && s < n_work; ++s) issue_tile(s, s);
+    if (gtest && n_work > 0) issue_recs(0);
   }
 
   // One CTA barrier per tile: after it every thread has finished the previous tile, so its
@@ -730,7 +805,8 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
   for (; t < n_work; ++t) {
     const int st = t % kStages;
     const uint32_t parity = static_cast<uint32_t>(t / kStages) & 1u;
-    const bool ok = mbar_wait_bounded(&bars[st], parity);
+    bool ok = mbar_wait_bounded(&bars[st], parity);
+    if (gtest) ok = mbar_wait_bounded(&rbar, static_cast<uint32_t>(t) & 1u) && ok;
     if (__syncthreads_or(!ok)) {
       aborted = true;
       break;
@@ -740,8 +816,22 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       fence_proxy_async_smem();
       issue_tile(ps, t - 1 + kStages);
     }
-    if constexpr (CEN) centre_tile(stages + st * stage_floats);
-    process_tile(stages + st * stage_floats);
+    unsigned gm = 0xffffffffu;
+    if constexpr (GT) {
+      if (gtest) {
+        gm = group_mask();
+        groups_done += __popc(gm);
+        // every lane's reads of the slot are done (the votes above): the next records may
+        // overwrite it; order those generic reads before the asynchronous copy
+        __syncwarp();
+        if (tid == 0 && t + 1 < n_work) {
+          fence_proxy_async_smem();
+          issue_recs(t + 1);
+        }
+      }
+    }
+    if constexpr (CEN) centre_tile(stages + st * stage_floats, gm);
+    process_tile(stages + st * stage_floats, gm);
     // the stage was written by this (generic) proxy: order that before its next copy
     if constexpr (CEN) fence_proxy_async_smem();
   }
@@ -757,6 +847,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       atomicOr(P.err, kErrTimeout);
       for (int u = t; u < n_work && u < t + kStages - 1; ++u)
         (void)mbar_wait_bounded(&bars[u % kStages], static_cast<uint32_t>(u / kStages) & 1u);
+      if (gtest) (void)mbar_wait_bounded(&rbar, static_cast<uint32_t>(t) & 1u);  // tile t's records
     }
     return;
   }
