@@ -48,7 +48,8 @@ def parse():
     ap.add_argument("--config", default="c5", choices=sorted(CONFIG_INDEX))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--n", type=int, default=None,
-                    help="clustered workload only: use n = m points (eps by the same spacing rule)")
+                    help="clustered (c5) or mixture (c4) workload: use n = m points (c5: eps by "
+                         "the same spacing rule; c4: the same eps), e.g. a small case to profile")
     ap.add_argument("--d", type=int, default=None,
                     help="50k-point mixture workload (c4) only: use d coordinates, eps = d / 64")
     ap.add_argument("--e2e-steps", type=int, default=None)
@@ -65,17 +66,20 @@ def parse():
 def workload(cfg: str, rank: int, n_override=None, d_override=None):
     from streaming_sinkhorn_b200 import workloads
     import dataclasses
+    if cfg == "c4" and (d_override is not None or n_override is not None):
+        # the same recipe at another width or size; eps grows with d so that kappa |x - y|^2
+        # keeps the scale it has at d = 64, eps = 1
+        d = 64 if d_override is None else d_override
+        n = 50000 if n_override is None else n_override
+        w = workloads.mixture_pair(n=n, d=d, k=10, mean_scale=2.0, std=1.0,
+                                   seed=3 + 1000 * rank, eps=d / 64.0, n_iters=100)
+        size = "50k" if n == 50000 else str(n)
+        return dataclasses.replace(w, name=f"mix_{size}_d{d}")
     if d_override is not None:
-        if cfg != "c4":
-            raise SystemExit("--d applies to the 50k-point mixture workload (c4) only")
-        # the same recipe at another width; eps grows with d so that kappa |x - y|^2 keeps the
-        # scale it has at d = 64, eps = 1
-        w = workloads.mixture_pair(n=50000, d=d_override, k=10, mean_scale=2.0, std=1.0,
-                                   seed=3 + 1000 * rank, eps=d_override / 64.0, n_iters=100)
-        return dataclasses.replace(w, name=f"mix_50k_d{d_override}")
+        raise SystemExit("--d applies to the 50k-point mixture workload (c4) only")
     if n_override is not None:
         if cfg != "c5":
-            raise SystemExit("--n applies to the clustered workload (c5) only")
+            raise SystemExit("--n applies to the clustered (c5) and mixture (c4) workloads only")
         w = workloads.clustered_cube(n=n_override, seed=4 + 1000 * rank, n_iters=20)
         return dataclasses.replace(w, name=f"clustered_cube_n{n_override}")
     # rank r > 0 runs an independently seeded replica of the same recipe
