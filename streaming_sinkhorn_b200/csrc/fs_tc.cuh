@@ -250,14 +250,20 @@ __device__ __forceinline__ void tc_lse_tile(TcRowLse& s, const float* v, const f
     tv[j] = add2(fma2(c2, pk(v[2 * j], v[2 * j + 1]), h.x), nmo);
     tv[j + 1] = add2(fma2(c2, pk(v[2 * j + 2], v[2 * j + 3]), h.y), nmo);
   }
-  float a0, a1;
+  // the tile's maximum and, below, its sum as two interleaved chains (even and odd column
+  // pairs): half the dependency depth for a thread that owns one row
+  float a0, a1, b0, b1;
   upk(tv[0], a0, a1);
-  float mx = fmaxf(a0, a1);
+  upk(tv[1], b0, b1);
+  float mxe = fmaxf(a0, a1), mxo = fmaxf(b0, b1);
 #pragma unroll
-  for (int j = 1; j < GP; ++j) {
+  for (int j = 2; j < GP; j += 2) {
     upk(tv[j], a0, a1);
-    mx = max3(mx, a0, a1);
+    mxe = max3(mxe, a0, a1);
+    upk(tv[j + 1], b0, b1);
+    mxo = max3(mxo, b0, b1);
   }
+  const float mx = fmaxf(mxe, mxo);
   const float mx_abs = mx + s.base;
   if (mx_abs > s.m + kLazyThr && mx > kEmptyCut) {
     const float sc = ex2(s.m - mx_abs);
@@ -271,16 +277,23 @@ __device__ __forceinline__ void tc_lse_tile(TcRowLse& s, const float* v, const f
   }
   // One column pair in kTcPolyEvery takes its exponentials on the FMA pipe (ex2_poly2), the
   // rest on the MUFU unit, which is this pass's bound while issue slots are free.
+  u64 se = pk(0.0f, 0.0f), so = pk(0.0f, 0.0f);
 #pragma unroll
   for (int j = 0; j < GP; ++j) {
+    u64 e;
     if (kTcPolyEvery > 0 && j % kTcPolyEvery == kTcPolyEvery - 1) {
-      s.L = add2(s.L, ex2_poly2(tv[j]));
+      e = ex2_poly2(tv[j]);
     } else {
       float t0, t1;
       upk(tv[j], t0, t1);
-      s.L = add2(s.L, pk(ex2(t0), ex2(t1)));
+      e = pk(ex2(t0), ex2(t1));
     }
+    if (j & 1)
+      so = add2(so, e);
+    else
+      se = add2(se, e);
   }
+  s.L = add2(s.L, add2(se, so));
 }
 
 // Merges the column groups' states of every row and completes the row: the pass kind's
