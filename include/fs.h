@@ -141,6 +141,11 @@ FS_API fs_status fs_workspace_invalidate(void* ws, size_t ws_bytes, fs_stream_t 
  * fails falls back to plain launches. Per-kernel timing (fs_timing_enable) turns it off,
  * and fs_potentials_noalloc never uses it (instantiating a graph may allocate). The call
  * returns once the replays have finished.
+ * Problems of at most 2^22 pairs with d <= 16 whose two clouds fit in 200 KB of shared
+ * memory (this call, and fs_solve with the alternating variant and FS_STOP_FIXED) run every
+ * iteration in one kernel launch on a thread-block cluster of 16 CTAs (8, 4, 2 or 1 where
+ * the device cannot co-schedule 16), the biases exchanged through distributed shared
+ * memory; the update is the same, in the direct-difference form.
  */
 FS_API fs_status fs_potentials(const fs_problem* p, int32_t n_iters, const float* g_init, float* f,
                         float* g, void* ws, size_t ws_bytes, fs_stream_t stream);
@@ -445,8 +450,9 @@ FS_API int64_t fs_launch_count(void);
 /*
  * Block screening, on by default (point clouds with d <= 16, which the library puts in a
  * spatial order). A pass skips a 256-point key tile when a bound shows that each of its
- * terms is below 2^-(24 + log2 M) times the largest term of every row it meets, so that
- * the omitted part of each row's sum is below 2^-24 of the sum (FlashSinkhorn 2 abstract,
+ * terms is below 2^-(24 + log2 M) times the largest term of every row it meets, and for
+ * d <= 3 a group of 16 consecutive keys of a tile it keeps by the same bound, so that the
+ * omitted part of each row's sum is below 2^-24 of the sum (FlashSinkhorn 2 abstract,
  * block-sparse screening, here with a provable bound). fs_screening_enable(0) makes every
  * later call evaluate all N x M pairs; the results agree to fp32 rounding either way.
  * Process-wide; takes effect at the next call.
