@@ -1958,6 +1958,7 @@ bool run_small_solve(Ctx& c, int32_t n_iters, const float* g_init, float* f, flo
   S.n_iters = n_iters;
   S.kappa = c.kappa;
   S.inv_kappa = 1.0 / c.kappa;
+  S.err = err_ptr(c.scal);
   const double pairs = 2.0 * static_cast<double>(p->n) * static_cast<double>(p->m) * n_iters;
   const int ti = c.timer->begin();
   bool ok = false;

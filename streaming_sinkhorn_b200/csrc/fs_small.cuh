@@ -6,14 +6,16 @@
 // streaming passes around it. Here one cluster of up to 16 CTAs runs every iteration in a
 // single kernel. Every CTA stages both clouds (coordinate-major) with their log2 weights in
 // shared memory once, and keeps the biases H_j = kappa pot_j + log2 w_j of both clouds there
-// too. Each half-iteration its warps take rows two at a time (the 32 lanes of a warp split
-// the keys, each key pair loaded once for both rows, two keys per packed fp32x2 operation),
-// merge their (max, sum) pairs by shuffles, write each row's new potential to global memory
-// and its new bias into the bias array of EVERY CTA of the cluster (distributed shared
-// memory stores), which the next half-iteration reads as its key biases. A hardware
-// cluster barrier (release / acquire at cluster scope) ends each half-iteration. It cannot
-// wait forever: every CTA of the cluster runs the same number of half-iterations and no CTA
-// leaves early.
+// too. Each half-iteration the rows go in groups of 32, one row per lane, the groups dealt to
+// the CTAs in turn; a CTA gives each of its groups 32 / WG warps (WG groups at a time), one
+// slice of the keys per warp, read by all its lanes at once (two keys per packed fp32x2
+// operation, the running max / sum of the lane's row kept lazily). The slices' (max, sum)
+// pairs meet in shared memory, the group's first warp merges them, writes each row's new
+// potential to global memory and its new bias into the bias array of EVERY CTA of the
+// cluster (distributed shared memory stores), which the next half-iteration reads as its
+// key biases. A hardware cluster barrier (release / acquire at cluster scope) ends each
+// half-iteration. It cannot wait forever: every CTA of the cluster runs the same number of
+// half-iterations and no CTA leaves early.
 //
 // The score is the direct difference z_ij = H_j - kappa |x_i - y_j|^2 in fp32 (the most
 // accurate form; the oracle's is the same in fp64), the log-sum-exp online in base 2.
@@ -31,7 +33,7 @@ constexpr size_t kSmallSmemBudget = 200u * 1024u;      // both staged clouds at 
 
 // Points per cloud as staged: padded to a multiple of 512 so that every lane takes whole
 // groups of kSmallGroup key pairs (padding keys carry log2(0) and add nothing).
-constexpr int kSmallGroup = 4;  // key pairs per lane per step and row (two rows: 16 exponentials)
+constexpr int kSmallGroup = 8;  // key pairs per step (16 independent exponentials per lane)
 __host__ __device__ constexpr int64_t small_pad(int64_t count) {
   return (count + 511) / 512 * 512;
 }
@@ -50,6 +52,7 @@ struct SmallParams {
   int32_t n_iters;
   double kappa;         // log2(e) / eps
   double inv_kappa;     // eps ln 2
+  unsigned* err;        // the workspace error word (a wait that timed out sets kErrTimeout)
 };
 
 __device__ __forceinline__ void cluster_barrier() {
@@ -79,18 +82,43 @@ __device__ __forceinline__ void merge_max_sum(float& mx, float& s, float mo, flo
 }
 
 // Shared memory of one CTA: both clouds coordinate-major (D coordinate arrays and the log2
-// weights, padded counts) and the biases of both clouds.
+// weights, padded counts), the biases of both clouds, and the warps' per-row partials.
 __host__ __device__ inline size_t small_smem_bytes(int64_t n, int64_t m, int D) {
   const int64_t np = small_pad(n), mp = small_pad(m);
-  return static_cast<size_t>((np + mp) * (D + 2)) * sizeof(float);
+  return static_cast<size_t>((np + mp) * (D + 2) + 2 * kSmallWarps * 32) * sizeof(float);
 }
 
-// Stores v at the address of `local` in the shared memory of CTA `rank` of the cluster.
-__device__ __forceinline__ void st_cluster(float* local, unsigned rank, float v) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)),
+// Stores v at the address of `local` in the shared memory of CTA `rank` of the cluster and
+// counts its 4 bytes on that CTA's mbarrier at the address of `bar` (asynchronous store).
+__device__ __forceinline__ void st_async_cluster(float* local, unsigned rank, float v,
+                                                 uint64_t* bar) {
+  uint32_t ra, rb;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)),
                "r"(rank));
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rb) : "r"(smem_u32(bar)),
+               "r"(rank));
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
+                   ra),
+               "r"(__float_as_uint(v)), "r"(rb)
+               : "memory");
+}
+
+// Bounded wait for a phase of an mbarrier that other CTAs of the cluster complete, with
+// acquire semantics at cluster scope (their stores are then visible here).
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
 }
 
 // The bias of a point from its (float) potential and log2 weight, in double, rounded once.
@@ -108,6 +136,10 @@ __global__ void __launch_bounds__(kSmallThreads) small_solve_kernel(const SmallP
   float* sy = sx + (D + 1) * np;        // y: [D][mp], then [mp] log2 b
   float* hx = sy + (D + 1) * mp;        // biases of x (the keys of the g-updates)
   float* hy = hx + np;                  // biases of y (the keys of the f-updates)
+  auto part = reinterpret_cast<float(*)[kSmallWarps][32]>(hy + mp);  // [max | sum][warp][lane]
+  // one per parity of the half-iteration: completes when every row's new bias of that
+  // half-iteration has landed in this CTA's shared memory
+  __shared__ uint64_t hbar[2];
   const unsigned crank = cluster_rank(), csize = cluster_size();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // both clouds once, with their log2 weights (kLogZero for a zero weight and for padding)
@@ -133,12 +165,18 @@ __global__ void __launch_bounds__(kSmallThreads) small_solve_kernel(const SmallP
     else
       hy[j] = j < count ? small_bias(S.kappa, S.g_init ? S.g_init[j] : 0.0f, lw) : kLogZero;
   }
-  // every CTA's arrays initialised before any CTA stores into them
+  if (tid == 0) {
+    mbar_init(&hbar[0], 1);
+    mbar_init(&hbar[1], 1);
+    fence_mbar_init();
+  }
+  // every CTA's arrays and mbarriers initialised before any CTA stores into them
   cluster_barrier();
   const u64 nkap = pk(-static_cast<float>(S.kappa), -static_cast<float>(S.kappa));
-  const int stride = static_cast<int>(csize) * kSmallWarps;  // warps of the cluster
   for (int h = 0; h < 2 * S.n_iters; ++h) {
     const bool rows_x = (h & 1) == 0;  // f-update first, then the g-update
+    uint64_t* bar = &hbar[h & 1];
+    if (tid == 0) mbar_expect_tx(bar, 4u * static_cast<uint32_t>(rows_x ? S.n : S.m));
     const float* R = rows_x ? sx : sy;
     const float* K = rows_x ? sy : sx;
     const int nr = rows_x ? S.n : S.m;
@@ -149,108 +187,99 @@ __global__ void __launch_bounds__(kSmallThreads) small_solve_kernel(const SmallP
 #pragma unroll
     for (int k = 0; k < D; ++k) kc[k] = reinterpret_cast<const u64*>(K + k * kpad);
     const u64* hv = reinterpret_cast<const u64*>(rows_x ? hy : hx);
-    // rows i and i + stride of this warp at once; a lane takes key pairs lane + 32 t,
-    // kSmallGroup at a time, and rescales a row's running sum only when a group's maximum
-    // exceeds its offset by more than kLazyThr
-    for (int i = static_cast<int>(crank) * kSmallWarps + warp; i < nr; i += 2 * stride) {
-      const int i2 = i + stride < nr ? i + stride : i;  // a lone last row is computed twice
-      u64 xa[D], xb[D];
+    // Rows in groups of 32 (lane l: row 32 g + l), groups dealt to the CTAs in turn; a CTA
+    // takes WG of its groups at a time and gives each S = 32 / WG warps, one slice of the
+    // keys each (kSmallGroup key pairs per step, read by all lanes at once). Each warp's
+    // (max, sum) per row goes to shared memory, and the group's first warp merges the S
+    // slices of its rows.
+    const int ngroups = (nr + 31) / 32;
+    const int gpc = (ngroups + static_cast<int>(csize) - 1) / static_cast<int>(csize);
+    int wg = 1;
+    while (wg < gpc && wg < kSmallWarps) wg *= 2;
+    const int slices = kSmallWarps / wg;
+    const int slot = warp / slices, slice = warp % slices;
+    const int per = kpad / 2 / slices;  // key pairs per slice (kpad / 2 is a multiple of 256)
+    const int q0 = slice * per;
+    for (int round = 0; round * wg < gpc; ++round) {
+      const int gl = round * wg + slot;
+      const int group = static_cast<int>(crank) + gl * static_cast<int>(csize);
+      const bool active = gl < gpc && group < ngroups;  // the same for the whole warp
+      const int i = group * 32 + lane;
+      float mr = -INFINITY;
+      u64 sr = pk(0.0f, 0.0f);
+      if (active) {
+        const int ic = i < nr ? i : nr - 1;  // lanes past the last row repeat it
+        u64 xi[D];
 #pragma unroll
-      for (int k = 0; k < D; ++k) {
-        const float ca = R[k * rpad + i], cb = R[k * rpad + i2];
-        xa[k] = pk(ca, ca);
-        xb[k] = pk(cb, cb);
-      }
-      float ma = -INFINITY, mb = -INFINITY;
-      u64 sa = pk(0.0f, 0.0f), sb = pk(0.0f, 0.0f);
-      for (int q0 = lane; q0 < kpad / 2; q0 += 32 * kSmallGroup) {
-        u64 za[kSmallGroup], zb[kSmallGroup];
-        float ga = -INFINITY, gb = -INFINITY;
-#pragma unroll
-        for (int t = 0; t < kSmallGroup; ++t) {
-          const int q = q0 + 32 * t;
-          u64 aa = pk(0.0f, 0.0f), ab = pk(0.0f, 0.0f);
-#pragma unroll
-          for (int k = 0; k < D; ++k) {
-            const u64 yk = kc[k][q];
-            const u64 da = sub2(xa[k], yk), db = sub2(xb[k], yk);
-            aa = fma2(da, da, aa);
-            ab = fma2(db, db, ab);
-          }
-          const u64 hq = hv[q];
-          za[t] = fma2(nkap, aa, hq);
-          zb[t] = fma2(nkap, ab, hq);
-          float z0, z1;
-          upk(za[t], z0, z1);
-          ga = max3(ga, z0, z1);
-          upk(zb[t], z0, z1);
-          gb = max3(gb, z0, z1);
+        for (int k = 0; k < D; ++k) {
+          const float c = R[k * rpad + ic];
+          xi[k] = pk(c, c);
         }
-        if (ga > ma + kLazyThr && ga > kEmptyCut) {
-          const float sc = ma == -INFINITY ? 0.0f : ex2(ma - ga);
-          sa = mul2(sa, pk(sc, sc));
-          ma = ga;
-        }
-        if (gb > mb + kLazyThr && gb > kEmptyCut) {
-          const float sc = mb == -INFINITY ? 0.0f : ex2(mb - gb);
-          sb = mul2(sb, pk(sc, sc));
-          mb = gb;
-        }
-        if (ma != -INFINITY) {
+        for (int q = q0; q < q0 + per; q += kSmallGroup) {
+          u64 z[kSmallGroup];
+          float gm = -INFINITY;
 #pragma unroll
           for (int t = 0; t < kSmallGroup; ++t) {
-            float z0, z1;
-            upk(za[t], z0, z1);
-            sa = add2(sa, pk(ex2(z0 - ma), ex2(z1 - ma)));
-          }
-        }
-        if (mb != -INFINITY) {
+            u64 acc = pk(0.0f, 0.0f);
 #pragma unroll
-          for (int t = 0; t < kSmallGroup; ++t) {
+            for (int k = 0; k < D; ++k) {
+              const u64 dk = sub2(xi[k], kc[k][q + t]);
+              acc = fma2(dk, dk, acc);
+            }
+            z[t] = fma2(nkap, acc, hv[q + t]);
             float z0, z1;
-            upk(zb[t], z0, z1);
-            sb = add2(sb, pk(ex2(z0 - mb), ex2(z1 - mb)));
+            upk(z[t], z0, z1);
+            gm = max3(gm, z0, z1);
+          }
+          if (gm > mr + kLazyThr && gm > kEmptyCut) {
+            const float sc = mr == -INFINITY ? 0.0f : ex2(mr - gm);
+            sr = mul2(sr, pk(sc, sc));
+            mr = gm;
+          }
+          if (mr != -INFINITY) {
+            const u64 nm = pk(-mr, -mr);
+#pragma unroll
+            for (int t = 0; t < kSmallGroup; ++t) {
+              float z0, z1;
+              upk(add2(z[t], nm), z0, z1);
+              sr = add2(sr, pk(ex2(z0), ex2(z1)));
+            }
           }
         }
       }
       float s0, s1;
-      upk(sa, s0, s1);
-      float suma = s0 + s1;
-      upk(sb, s0, s1);
-      float sumb = s0 + s1;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float mao = __shfl_xor_sync(0xffffffffu, ma, o);
-        const float sao = __shfl_xor_sync(0xffffffffu, suma, o);
-        const float mbo = __shfl_xor_sync(0xffffffffu, mb, o);
-        const float sbo = __shfl_xor_sync(0xffffffffu, sumb, o);
-        merge_max_sum(ma, suma, mao, sao);
-        merge_max_sum(mb, sumb, mbo, sbo);
+      upk(sr, s0, s1);
+      part[0][warp][lane] = mr;
+      part[1][warp][lane] = s0 + s1;
+      __syncthreads();
+      if (active && slice == 0) {
+        float m = -INFINITY, sum = 0.0f;
+        for (int j = 0; j < slices; ++j)
+          merge_max_sum(m, sum, part[0][warp + j][lane], part[1][warp + j][lane]);
+        if (i < nr) {
+          // log2 of the sum in fp32 (2^-23 relative on a value below ~25, ~3e-6 log2 units,
+          // far below the potentials' fp32 rounding); the rest in double as the other passes
+          const double lse2 = static_cast<double>(m) + static_cast<double>(log2f(sum));
+          const float pot = static_cast<float>(-lse2 * S.inv_kappa);
+          potr[i] = pot;
+          const float hnew = small_bias(S.kappa, pot, R[D * rpad + i]);
+          // the new bias into every CTA of the cluster
+          for (unsigned c = 0; c < csize; ++c) st_async_cluster(hr + i, c, hnew, bar);
+        }
       }
-      // lane 0: row i, lane 1: row i2 (log2 of the sum in fp32: 2^-23 relative on a value
-      // below ~25, ~3e-6 log2 units, far below the potentials' fp32 rounding; the rest in
-      // double as the other passes do)
-      const int row = lane == 0 ? i : i2;
-      float hnew = 0.0f;
-      if (lane < 2) {
-        const double lse2 = lane == 0 ? static_cast<double>(ma) + static_cast<double>(log2f(suma))
-                                      : static_cast<double>(mb) + static_cast<double>(log2f(sumb));
-        const float pot = static_cast<float>(-lse2 * S.inv_kappa);
-        if (lane == 0 || i2 != i) potr[row] = pot;
-        hnew = small_bias(S.kappa, pot, R[D * rpad + row]);
-      }
-      // the new biases into every CTA of the cluster: lane c < csize stores to CTA c
-      const float h0 = __shfl_sync(0xffffffffu, hnew, 0);
-      const float h1 = __shfl_sync(0xffffffffu, hnew, 1);
-      if (lane < static_cast<int>(csize)) {
-        st_cluster(hr + i, static_cast<unsigned>(lane), h0);
-        if (i2 != i) st_cluster(hr + i2, static_cast<unsigned>(lane), h1);
-      }
+      __syncthreads();  // the partials are read before the next round writes them
     }
-    // every row's potential and bias of this half-iteration written and visible to the
-    // whole cluster, and every CTA done reading the key biases it used
-    cluster_barrier();
+    // Every row's new bias of this half-iteration has reached this CTA: all CTAs have also
+    // finished reading the key biases of this half-iteration (each CTA's stores follow its
+    // last read of them), so the next one may overwrite them.
+    const bool ok = mbar_wait_cluster_bounded(bar, static_cast<uint32_t>(h >> 1) & 1u);
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) atomicOr(S.err, kErrTimeout);
+      break;
+    }
   }
+  // no CTA leaves while stores into its shared memory could still be in flight
+  cluster_barrier();
 }
 
 }  // namespace fs
