@@ -73,14 +73,6 @@ __device__ __forceinline__ unsigned cluster_size() {
   return r;
 }
 
-// Merges the (max, sum) pair of another lane into this one; an empty pair has max -inf.
-__device__ __forceinline__ void merge_max_sum(float& mx, float& s, float mo, float so) {
-  const float M = fmaxf(mx, mo);
-  if (M == -INFINITY) return;
-  s = (mx == -INFINITY ? 0.0f : s * ex2(mx - M)) + (mo == -INFINITY ? 0.0f : so * ex2(mo - M));
-  mx = M;
-}
-
 // Shared memory of one CTA: both clouds coordinate-major (D coordinate arrays and the log2
 // weights, padded counts), the biases of both clouds, and the warps' per-row partials.
 __host__ __device__ inline size_t small_smem_bytes(int64_t n, int64_t m, int D) {
@@ -111,10 +103,10 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(1000u)
         : "memory");
     if (done) return true;
     if (global_ns() - t0 > kWaitLimitNs) return false;
@@ -253,9 +245,16 @@ __global__ void __launch_bounds__(kSmallThreads) small_solve_kernel(const SmallP
       part[1][warp][lane] = s0 + s1;
       __syncthreads();
       if (active && slice == 0) {
+        // the slices' largest offset, then their sums scaled to it: independent terms
+        // instead of a chain of pairwise merges
         float m = -INFINITY, sum = 0.0f;
-        for (int j = 0; j < slices; ++j)
-          merge_max_sum(m, sum, part[0][warp + j][lane], part[1][warp + j][lane]);
+        for (int j = 0; j < slices; ++j) m = fmaxf(m, part[0][warp + j][lane]);
+        if (m != -INFINITY) {
+          for (int j = 0; j < slices; ++j) {
+            const float mj = part[0][warp + j][lane];
+            if (mj != -INFINITY) sum = fmaf(part[1][warp + j][lane], ex2(mj - m), sum);
+          }
+        }
         if (i < nr) {
           // log2 of the sum in fp32 (2^-23 relative on a value below ~25, ~3e-6 log2 units,
           // far below the potentials' fp32 rounding); the rest in double as the other passes
