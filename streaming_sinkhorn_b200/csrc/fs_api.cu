@@ -1056,7 +1056,12 @@ struct Ctx {
   float alpha;    // symmetric schedule: blend weight of the potential passes (0: plain)
   bool defer_x;   // the next x-row potential pass leaves its biases in `defer`
   bool no_screen;  // screening found to keep most tiles: the rest of the call runs unscreened
+  bool screen_on;  // fs_screening_enable's setting, read once at the start of the call
 };
+
+// Whether the passes of this call may still screen: sorted clouds, screening enabled when the
+// call began, and not switched off by the probe after the first iteration.
+inline bool screening_live(const Ctx& c) { return c.L.sorted && c.screen_on && !c.no_screen; }
 
 fs_status check_common(const fs_problem* p, void* ws, size_t ws_bytes, size_t* need_out,
                        int sms, int acc_ch = 0) {
@@ -1640,8 +1645,7 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
   P.err = err_ptr(c.scal);
   int* dmin_slots = reinterpret_cast<int*>(c.scal + kDmin);
   const int tk = grad ? kTGrad : (kind == kMarg ? kTMarg : kTLse);
-  const QPlan q = make_qplan(pl, key_pairs, c.L.D, grad, c.sms,
-                             c.L.sorted && !c.no_screen && g_screening.load());
+  const QPlan q = make_qplan(pl, key_pairs, c.L.D, grad, c.sms, screening_live(c));
   if (c.L.sorted) {
     P.perm = rows_x ? c.perm_x : c.perm_y;
     P.evaluated = reinterpret_cast<unsigned long long*>(c.scal + kEval + tk);
@@ -1724,8 +1728,9 @@ void run_pass(Ctx& c, bool rows_x, int kind, const float* pot_in, float* pot_out
       c.timer->end(ti, kTCombine, 0.0);
     }
   }
-  if (c.L.sorted && kind == kPot && !(rows_x && c.defer_x)) {
-    // largest bias per tile of the cloud just updated: the next pass screens against it
+  if (screening_live(c) && kind == kPot && !(rows_x && c.defer_x)) {
+    // largest bias per tile of the cloud just updated: the next pass screens against it (no
+    // later pass of this call screens once screening is off)
     FS_DISPATCH_D(c.L.D, launch_tile_hmax_d, rows_x ? c.kx : c.ky, n_rows,
                   (rows_x ? c.L.px : c.L.py) / kPairPad, rows_x ? c.hmax_x : c.hmax_y,
                   rows_x ? c.gsum_x : c.gsum_y, c.st);
@@ -1739,7 +1744,7 @@ void screening_probe(Ctx& c, bool rows_x) {
   const int64_t n_rows = rows_x ? c.p->n : c.p->m;
   const int64_t key_pairs = rows_x ? c.L.py : c.L.px;
   const Plan pl = make_plan(n_rows, key_pairs, c.L.D, false, c.sms);
-  const QPlan q = make_qplan(pl, key_pairs, c.L.D, false, c.sms, c.L.sorted && !c.no_screen);
+  const QPlan q = make_qplan(pl, key_pairs, c.L.D, false, c.sms, screening_live(c));
   if (!q.on) return;
   long long kept = 0;
   CK(cudaMemcpyAsync(&kept, c.scal + kKept, sizeof(kept), cudaMemcpyDeviceToHost, c.st));
@@ -1781,6 +1786,7 @@ fs_status guarded(cudaStream_t st, F&& body) {
 fs_status begin(Ctx& c, const fs_problem* p, void* ws, size_t ws_bytes, fs_stream_t stream,
                 int acc_ch = 0) {
   c.sms = num_sms_current();
+  c.screen_on = g_screening.load();
   size_t need = 0;
   const fs_status s = check_common(p, ws, ws_bytes, &need, c.sms, acc_ch);
   if (s != FS_OK) return s;
@@ -1804,7 +1810,8 @@ void apply_deferred_x(Ctx& c) {
   int* dmin = reinterpret_cast<int*>(c.scal + kDmin);  // slot 0: x
   CK(cudaMemsetAsync(dmin, 0x7F, sizeof(int), c.st));
   FS_DISPATCH_D(c.L.D, launch_apply_bias_d, c.kx, c.defer, n, dmin, c.st);
-  FS_DISPATCH_D(c.L.D, launch_tile_hmax_d, c.kx, n, c.L.px / kPairPad, c.hmax_x, c.gsum_x, c.st);
+  if (screening_live(c))
+    FS_DISPATCH_D(c.L.D, launch_tile_hmax_d, c.kx, n, c.L.px / kPairPad, c.hmax_x, c.gsum_x, c.st);
 }
 
 // max(|P1 - a|_inf, |P^T 1 - b|_inf) at (f, g): two marginal passes, one read-back.
