@@ -76,3 +76,16 @@ def test_reference_arm_runs_on_rank_zero_only():
                        env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_workload_overrides_keep_the_recipes():
+    """--n and --d build the named recipes at other sizes (small cases to profile): the
+    clustered cube keeps its spacing rule for eps, the mixture keeps eps = d / 64."""
+    w = bench.workload("c5", 0, 4096, None)
+    assert (w.n, w.m, w.d) == (4096, 4096, 3) and abs(w.eps - 4096.0 ** (-2.0 / 3.0)) < 1e-12
+    w0 = bench.workload("c4", 0, 16384, None)
+    assert (w0.n, w0.m, w0.d) == (16384, 16384, 64) and w0.eps == 1.0 and w0.n_iters == 100
+    w = bench.workload("c4", 0, None, 512)
+    assert (w.n, w.m, w.d) == (50000, 50000, 512) and w.eps == 8.0
+    r1 = bench.workload("c4", 1, 16384, None)  # rank 1: its own replica of the same recipe
+    assert r1.x.shape == w0.x.shape and not np.array_equal(r1.x, w0.x)
