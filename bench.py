@@ -320,6 +320,12 @@ def run_native(args, rank, world, local_rank):
                 "executed_ex2_per_launch": per_launch_pairs,
                 "nominal_pairs_per_launch": lse["pairs"] / max(lse["launches"], 1),
                 "screened_fraction": (1.0 - executed / lse["pairs"]) if lse["pairs"] else 0.0}
+    if lse["evaluated"] > 0 and roofline["screened_fraction"] > 0.5:
+        roofline["note"] = ("frac is the rate of the exponentials the screened pass issues: "
+                            "block screening and, for d <= 3, the 16-point group skip leave "
+                            "it only the pairs near each row's maximum, so each kept tile "
+                            "also carries its copy, centring and group tests; dense_pass "
+                            "gives the same kernel's rate on all N*M pairs")
 
     # The same pass with screening off, outside the timed region: one solve iteration (an
     # f pass and a g pass over all N x M pairs) on the same inputs, so the kernel's roofline
