@@ -381,9 +381,8 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
   static_assert(!GT || ST == 2, "the records of tile t + 1 follow the copy of tile t + 1");
   const uint32_t tile_floats = static_cast<uint32_t>(P.tile_pairs) * KP;
   const bool recs = GT && P.group_recs != 0;
-  const uint32_t stage_floats = tile_floats;
   const uint32_t tile_bytes = tile_floats * 4u;
-  float* rslot = stages + kStages * stage_floats;
+  float* rslot = stages + kStages * tile_floats;
 
   // The work of this CTA: rows row0 .. row0 + RB and a list of key tiles. Split mode: the
   // tiles of column split blockIdx.y, in order. Queue mode (screened, sorted clouds): unit
@@ -484,7 +483,7 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
       rtt1 = tt;
     else
       rtt0 = tt;
-    float* dst = stages + s * stage_floats;
+    float* dst = stages + s * tile_floats;
     mbar_expect_tx(&bars[s], tile_bytes);
     bulk_g2s(dst, key_src + static_cast<int64_t>(tt) * tile_floats, tile_bytes, &bars[s]);
   };
@@ -830,8 +829,8 @@ __global__ void __launch_bounds__(NT, MINB) lse_pass_kernel(const PassParams P) 
         }
       }
     }
-    if constexpr (CEN) centre_tile(stages + st * stage_floats, gm);
-    process_tile(stages + st * stage_floats, gm);
+    if constexpr (CEN) centre_tile(stages + st * tile_floats, gm);
+    process_tile(stages + st * tile_floats, gm);
     // the stage was written by this (generic) proxy: order that before its next copy
     if constexpr (CEN) fence_proxy_async_smem();
   }

@@ -29,10 +29,11 @@ constexpr int kSmallThreads = 1024;  // 8 warps per scheduler to hide shared-mem
 constexpr int kSmallWarps = kSmallThreads / 32;
 constexpr int kSmallMaxCluster = 16;                   // CTAs (SMs); a non-portable size
 constexpr int64_t kSmallMaxPairs = int64_t(1) << 22;   // n * m at most
-constexpr size_t kSmallSmemBudget = 200u * 1024u;      // both staged clouds at most
+constexpr size_t kSmallSmemBudget = 200u * 1024u;      // a CTA's shared memory at most
 
-// Points per cloud as staged: padded to a multiple of 512 so that every lane takes whole
-// groups of kSmallGroup key pairs (padding keys carry log2(0) and add nothing).
+// Points per cloud as staged: padded to a multiple of 512, so that each of up to 32 key
+// slices holds whole groups of kSmallGroup key pairs (padding keys carry log2(0) and add
+// nothing).
 constexpr int kSmallGroup = 8;  // key pairs per step (16 independent exponentials per lane)
 __host__ __device__ constexpr int64_t small_pad(int64_t count) {
   return (count + 511) / 512 * 512;
