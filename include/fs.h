@@ -107,7 +107,9 @@ FS_API const char* fs_last_cuda_error(void);
  * Bytes of scratch space every entry point below needs for `p` (pointer fields of
  * `p` are not read). Returns 0 when the shape (n, m, d) is invalid. The size depends
  * on the current device's SM count, so query it with the device current that the
- * calls will use.
+ * calls will use. It is not monotone in n and m (fewer rows get more column splits, and
+ * so more partial sums), so a workspace shared by several problems takes the largest of
+ * their sizes.
  */
 FS_API size_t fs_workspace_bytes(const fs_problem* p);
 
