@@ -154,3 +154,24 @@ def test_hvp_screened_equals_dense():
         out[screening] = (hv.cpu().numpy(), rep)
     assert out[True][1]["cg_rel_residual"] < 2e-3 and out[False][1]["cg_rel_residual"] < 2e-3
     close(out[True][0], out[False][0], 5e-3)
+
+
+@pytest.mark.parametrize("k", [3, 16])
+@pytest.mark.parametrize("transpose", [False, True])
+def test_transport_apply_screened_equals_dense(k, transpose):
+    """On a clustered problem the screened products (tile screening and the 16-point group
+    skip, 4- and 16-channel payload passes) agree with the unscreened ones: every term left
+    out is below 2^-(24 + log2 M) of its row's largest plan entry."""
+    w = workloads.clustered_cube(n=16384, seed=32, n_iters=6)
+    x, y, a, b = inputs(w)
+    f, g = fs.potentials(x, y, a, b, eps=w.eps, n_iters=6)
+    u = torch.from_numpy(np.random.default_rng(k).standard_normal((w.n, k)).astype(np.float32)).cuda()
+    out = {}
+    for screening in (False, True):
+        fs.screening_enable(screening)
+        try:
+            out[screening] = fs.transport_apply(x, y, f, g, u, a, b, eps=w.eps,
+                                                transpose=transpose).cpu().numpy()
+        finally:
+            fs.screening_enable(True)
+    close(out[True], out[False], 1e-4)
